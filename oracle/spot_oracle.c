@@ -1,0 +1,495 @@
+/*
+ * spot_oracle.c -- plain, slow, fp64 CPU oracle for the SpotAttention
+ * decode-time hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  The product path
+ * (the CUDA library under block_sparse_long_spot_b200/) never calls it and
+ * shares no code, header, table or helper with it.
+ *
+ * Source: "SpotAttention: Plug-In Block-Sparse Routing for Pretrained
+ * Long-Context Transformers" (arXiv HTML).  Each function names the section
+ * or equation it follows.  Everything is computed in fp64 with plain loops,
+ * in the order the definitions state; the only library primitives are exp(),
+ * log(), frexp()/ldexp() and qsort().
+ *
+ * Readings taken where the paper is silent (each also listed in the design doc):
+ *  - one selector key per (block, KV head); the index heads of a KV head are
+ *    the G query heads of its GQA group, mixing weight w[b,h] (NULL -> 1/G);
+ *  - the score of a block is s = (1/tau) * sum_h w_h * ReLU(q_h . k);
+ *  - "reaches p" means cumulative mass >= p; equal scores rank lower block
+ *    index first; p >= 1 takes the whole residual, p <= 0 an empty nucleus;
+ *  - the K_min floor is counted on |S| (reserved blocks included) and is
+ *    clamped to the number of blocks;
+ *  - a block that is not complete (seq_len not a multiple of the block size)
+ *    has no selector key and joins the recency set;
+ *  - attention scale sigma is an argument (1/sqrt(D) in every workload);
+ *    positions >= seq_len are not attended;
+ *  - INT4 keys: symmetric, scale = fp16_rne(amax/7) per group of 32,
+ *    code = clamp(rne(x/scale), -8, 7), two's complement nibbles, even
+ *    element in the low nibble; a scale above the fp16 range saturates to
+ *    65504;
+ *  - FP4 keys: OCP Microscaling v1.0 MXFP4 -- E2M1 elements, one E8M0 scale
+ *    per 32, X = floor(log2 amax) - 2 clamped to [-127, 127], elements
+ *    rounded to nearest even on the E2M1 grid with saturation at 6; the sign
+ *    bit is set only for x < 0; same nibble order as INT4.
+ *
+ * Parity status: every function here is pinned by tests/test_oracle_pins.py
+ * (hand-worked examples, brute force, closed forms, library special cases).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_FMT_BF16 = 0, ORC_FMT_INT4 = 1, ORC_FMT_MXFP4 = 2 };
+enum { ORC_MODE_TOPP = 0, ORC_MODE_TOPK = 1 };
+
+/* ------------------------------------------------------------------ */
+/* Exact decoders of the storage formats.                              */
+/* ------------------------------------------------------------------ */
+
+/* bf16 is the top half of an IEEE binary32. */
+static double bf16_to_f64(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits. */
+static double f16_to_f64(uint16_t bits) {
+    int sign = bits >> 15;
+    int e = (bits >> 10) & 0x1f;
+    int m = bits & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                 /* subnormal: m * 2^-24 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(m + 1024), e - 25);     /* (1 + m/1024) 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* fp64 -> binary16, round to nearest even, finite overflow saturates to
+ * the largest finite half (65504).  Only used for non-negative scales. */
+static uint16_t f64_to_f16_sat(double x) {
+    if (!(x > 0.0)) return 0;                      /* zero (and NaN -> 0) */
+    if (x >= 65504.0) return 0x7bff;
+    int ex;
+    (void)frexp(x, &ex);                           /* x = f 2^ex, f in [.5,1) */
+    int e = ex - 1;                                /* x in [2^e, 2^(e+1)) */
+    if (e < -14) e = -14;                          /* subnormal range: ulp 2^-24 */
+    double ulp = ldexp(1.0, e - 10);
+    double q = x / ulp;                            /* exact (power-of-2 divide) */
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double y = r * ulp;                            /* rounded value, exact */
+    if (y >= 65504.0) return 0x7bff;
+    /* Re-encode y exactly. */
+    if (y < ldexp(1.0, -14)) return (uint16_t)(y / ldexp(1.0, -24));
+    (void)frexp(y, &ex);
+    e = ex - 1;
+    int mant = (int)(y / ldexp(1.0, e - 10)) - 1024;
+    return (uint16_t)(((e + 15) << 10) | mant);
+}
+
+/* OCP MX v1.0 E2M1 element: sign, 2 exponent bits (bias 1), 1 mantissa bit.
+ * Magnitudes by code 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static double e2m1_to_f64(unsigned code) {
+    unsigned e = (code >> 1) & 3, m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, (int)e - 1);
+    return (code & 8) ? -mag : mag;
+}
+
+/* OCP MX v1.0 E8M0 scale: 2^(E-127); E = 255 is NaN. */
+static double e8m0_to_f64(uint8_t e) {
+    return e == 255 ? NAN : ldexp(1.0, (int)e - 127);
+}
+
+/* Dequantise `rows` selector keys of `ds` elements each into fp64.
+ * bf16:  data = uint16 [rows][ds], scales unused.
+ * INT4:  data = uint8 [rows][ds/2], scales = binary16 [rows][ds/32].
+ * MXFP4: data = uint8 [rows][ds/2], scales = E8M0 [rows][ds/32].
+ * Returns 0, or -1 for an unknown format. */
+int oracle_dequant_selector(int fmt, int64_t rows, int ds, const void* data,
+                            const void* scales, double* out) {
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int i = 0; i < ds; ++i) {
+            double v;
+            if (fmt == ORC_FMT_BF16) {
+                v = bf16_to_f64(((const uint16_t*)data)[r * ds + i]);
+            } else if (fmt == ORC_FMT_INT4 || fmt == ORC_FMT_MXFP4) {
+                uint8_t byte = ((const uint8_t*)data)[r * (ds / 2) + i / 2];
+                unsigned nib = (i % 2 == 0) ? (byte & 0xf) : (byte >> 4);
+                if (fmt == ORC_FMT_INT4) {
+                    int q = (nib >= 8) ? (int)nib - 16 : (int)nib;
+                    double s = f16_to_f64(((const uint16_t*)scales)[r * (ds / 32) + i / 32]);
+                    v = (double)q * s;
+                } else {
+                    double s = e8m0_to_f64(((const uint8_t*)scales)[r * (ds / 32) + i / 32]);
+                    v = e2m1_to_f64(nib) * s;
+                }
+            } else {
+                return -1;
+            }
+            out[r * ds + i] = v;
+        }
+    }
+    return 0;
+}
+
+/* Round |a| to the E2M1 grid, nearest, ties to the even code, saturating
+ * at 6.  Returns the 3-bit magnitude code. */
+static unsigned e2m1_rne_code(double a) {
+    static const double grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    if (a >= 6.0) return 7;
+    for (unsigned c = 0; c < 7; ++c) {
+        if (a <= grid[c + 1]) {
+            double mid = 0.5 * (grid[c] + grid[c + 1]);
+            if (a < mid) return c;
+            if (a > mid) return c + 1;
+            return (c % 2 == 0) ? c : c + 1;
+        }
+    }
+    return 7;
+}
+
+/* Quantise bf16 selector keys (the append step of the selector K-cache,
+ * SpotAttention §5.3 and App. G: group-32 INT4 / FP4 microscale).
+ * Layouts as in oracle_dequant_selector.  bf16 is a plain copy. */
+int oracle_quantize_selector(int fmt, int64_t rows, int ds, const uint16_t* keys,
+                             void* data, void* scales) {
+    if (ds % 32 != 0) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* row = keys + r * ds;
+        if (fmt == ORC_FMT_BF16) {
+            memcpy((uint16_t*)data + r * ds, row, (size_t)ds * sizeof(uint16_t));
+            continue;
+        }
+        uint8_t* out = (uint8_t*)data + r * (ds / 2);
+        memset(out, 0, (size_t)ds / 2);
+        for (int g = 0; g < ds / 32; ++g) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double x = fabs(bf16_to_f64(row[g * 32 + i]));
+                if (x > amax) amax = x;
+            }
+            if (fmt == ORC_FMT_INT4) {
+                uint16_t sbits = f64_to_f16_sat(amax / 7.0);
+                ((uint16_t*)scales)[r * (ds / 32) + g] = sbits;
+                double s = f16_to_f64(sbits);
+                for (int i = 0; i < 32; ++i) {
+                    double x = bf16_to_f64(row[g * 32 + i]);
+                    int q = 0;
+                    if (s > 0.0) {
+                        double t = nearbyint(x / s);       /* ties to even */
+                        if (t > 7.0) t = 7.0;
+                        if (t < -8.0) t = -8.0;
+                        q = (int)t;
+                    }
+                    unsigned nib = (unsigned)q & 0xf;
+                    int idx = g * 32 + i;
+                    out[idx / 2] |= (uint8_t)((idx % 2 == 0) ? nib : (nib << 4));
+                }
+            } else if (fmt == ORC_FMT_MXFP4) {
+                int X;
+                if (amax == 0.0) {
+                    X = -127;
+                } else {
+                    int ex;
+                    (void)frexp(amax, &ex);       /* amax = f 2^ex, f in [.5,1) */
+                    X = (ex - 1) - 2;             /* floor(log2 amax) - emax(E2M1) */
+                    if (X < -127) X = -127;
+                    if (X > 127) X = 127;
+                }
+                ((uint8_t*)scales)[r * (ds / 32) + g] = (uint8_t)(X + 127);
+                for (int i = 0; i < 32; ++i) {
+                    double x = bf16_to_f64(row[g * 32 + i]);
+                    double v = ldexp(x, -X);
+                    unsigned code = e2m1_rne_code(fabs(v)) | (x < 0.0 ? 8u : 0u);
+                    int idx = g * 32 + i;
+                    out[idx / 2] |= (uint8_t)((idx % 2 == 0) ? code : (code << 4));
+                }
+            } else {
+                return -1;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Shapes shared by the functions below.                               */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t batch, num_q_heads, num_kv_heads, head_dim, block_size, sel_dim;
+    int32_t sel_fmt, num_pages, max_blocks;
+} orc_shape_t;
+
+typedef struct {
+    int32_t mode;          /* ORC_MODE_TOPP (Eq. 8) or ORC_MODE_TOPK (Eq. 6) */
+    int32_t sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
+    double temperature;
+} orc_params_t;
+
+static int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+/* Selector score for every complete block of sequence b, KV head g
+ * (SpotAttention §2.1: s = sum_h w_h ReLU(q^I_h . k^I); block score = max
+ * over the block's keys, §2.3, which is the single key here; temperature
+ * from App. A Tab. 3).  keys_f64 = dequantised selector pool
+ * [num_pages][Hkv][ds].  Writes n_full scores into out. */
+static void unit_scores(const orc_shape_t* sh, const orc_params_t* pr, int b, int g,
+                        const uint16_t* q_sel, const float* w, const double* keys_f64,
+                        const int32_t* page_table, int64_t n_full, double* out) {
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    int ds = sh->sel_dim;
+    for (int64_t j = 0; j < n_full; ++j) {
+        int32_t page = page_table[(int64_t)b * sh->max_blocks + j];
+        const double* k = keys_f64 + ((int64_t)page * sh->num_kv_heads + g) * ds;
+        double s = 0.0;
+        for (int i = 0; i < G; ++i) {
+            int h = g * G + i;
+            const uint16_t* q = q_sel + ((int64_t)b * sh->num_q_heads + h) * ds;
+            double dot = 0.0;
+            for (int d = 0; d < ds; ++d) dot += bf16_to_f64(q[d]) * k[d];
+            double wh = w ? (double)w[(int64_t)b * sh->num_q_heads + h] : 1.0 / G;
+            s += wh * (dot > 0.0 ? dot : 0.0);
+        }
+        out[j] = s / pr->temperature;
+    }
+}
+
+/* Public form of unit_scores over all (b, g): scores[b][g][j] for
+ * j < floor(seq_len/bs); entries beyond are left untouched. */
+int oracle_block_scores(const orc_shape_t* sh, const orc_params_t* pr, const uint16_t* q_sel,
+                        const float* w, const void* sel_data, const void* sel_scales,
+                        const int32_t* page_table, const int32_t* seq_lens, double* scores) {
+    int64_t rows = (int64_t)sh->num_pages * sh->num_kv_heads;
+    double* keys = (double*)malloc((size_t)(rows * sh->sel_dim) * sizeof(double));
+    if (!keys) return -2;
+    if (oracle_dequant_selector(sh->sel_fmt, rows, sh->sel_dim, sel_data, sel_scales, keys)) {
+        free(keys);
+        return -1;
+    }
+    for (int b = 0; b < sh->batch; ++b)
+        for (int g = 0; g < sh->num_kv_heads; ++g)
+            unit_scores(sh, pr, b, g, q_sel, w, keys, page_table, seq_lens[b] / sh->block_size,
+                        scores + ((int64_t)b * sh->num_kv_heads + g) * sh->max_blocks);
+    free(keys);
+    return 0;
+}
+
+/* Ranking of residual blocks: score descending, lower block index first. */
+typedef struct { double s; int32_t j; } ranked_t;
+static int rank_cmp(const void* a, const void* b) {
+    const ranked_t* x = (const ranked_t*)a;
+    const ranked_t* y = (const ranked_t*)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->j < y->j) ? -1 : (x->j > y->j);
+}
+
+/* Block selection for one (sequence, KV head) from its block scores
+ * (SpotAttention §2.3).
+ *   nb       = number of blocks, n_full = blocks that have a score;
+ *   TOPP:    S = S_sink U S_rec U S_nuc, S_nuc the smallest prefix of the
+ *            residual blocks ranked by the residual softmax (Eq. 7) whose
+ *            cumulative mass reaches p; |S| >= K_min extends along the same
+ *            ranking (Eq. 8);
+ *   TOPK:    S = the topk_blocks best blocks (Eq. 6), still after the
+ *            reserved sink / recency blocks.
+ * Writes the selected block ids ascending into sel (capacity nb) and returns
+ * their count.  nuc_mass (may be NULL) receives the residual-softmax mass of
+ * the chosen residual blocks. */
+int oracle_select_from_scores(const double* scores, int32_t nb, int32_t n_full,
+                              const orc_params_t* pr, double p, int32_t* sel, double* nuc_mass) {
+    if (nb <= 0) { if (nuc_mass) *nuc_mass = 0.0; return 0; }
+    int32_t sink = pr->sink_blocks < nb ? pr->sink_blocks : nb;
+    if (sink < 0) sink = 0;
+    int32_t rec = pr->recency_blocks > 0 ? pr->recency_blocks : 0;
+    if (rec < nb - n_full) rec = nb - n_full;          /* incomplete block has no key */
+    if (rec > nb) rec = nb;
+    char* keep = (char*)calloc((size_t)nb, 1);
+    ranked_t* res = (ranked_t*)malloc((size_t)nb * sizeof(ranked_t));
+    int32_t n_res = 0, n_reserved = 0;
+    for (int32_t j = 0; j < nb; ++j) {
+        if (j < sink || j >= nb - rec) { keep[j] = 1; ++n_reserved; }
+        else { res[n_res].s = scores[j]; res[n_res].j = j; ++n_res; }
+    }
+    int32_t n_take = 0;
+    double taken_mass = 0.0;
+    if (n_res > 0) {
+        /* Residual softmax, Eq. 7. */
+        double m = res[0].s;
+        for (int32_t k = 1; k < n_res; ++k) if (res[k].s > m) m = res[k].s;
+        double Z = 0.0;
+        for (int32_t k = 0; k < n_res; ++k) Z += exp(res[k].s - m);
+        qsort(res, (size_t)n_res, sizeof(ranked_t), rank_cmp);
+        if (pr->mode == ORC_MODE_TOPK) {
+            n_take = pr->topk_blocks;
+        } else {
+            if (p >= 1.0) {
+                n_take = n_res;
+            } else if (p <= 0.0) {
+                n_take = 0;                           /* the empty prefix reaches p */
+            } else {
+                double cum = 0.0;
+                n_take = n_res;                       /* never reached: take all */
+                for (int32_t k = 0; k < n_res; ++k) {
+                    cum += exp(res[k].s - m) / Z;
+                    if (cum >= p) { n_take = k + 1; break; }
+                }
+            }
+            int32_t floor_res = pr->kmin_blocks - n_reserved;   /* |S| >= K_min */
+            if (n_take < floor_res) n_take = floor_res;
+        }
+        if (n_take > n_res) n_take = n_res;
+        if (n_take < 0) n_take = 0;
+        for (int32_t k = 0; k < n_take; ++k) {
+            keep[res[k].j] = 1;
+            taken_mass += exp(res[k].s - m) / Z;
+        }
+    }
+    int32_t cnt = 0;
+    for (int32_t j = 0; j < nb; ++j) if (keep[j]) sel[cnt++] = j;
+    if (nuc_mass) *nuc_mass = taken_mass;
+    free(keep);
+    free(res);
+    return cnt;
+}
+
+/* Exact softmax attention of the G query heads of KV head g over the tokens
+ * of the selected blocks (SpotAttention §2.3: the layer attends only to keys
+ * in the selected blocks; §3: decode only).  Token t of logical block j sits
+ * in pool page page_table[b][j], row t - j*bs.  Positions >= seq_len are not
+ * attended.  out[h][D] and lse[h] (natural log of the softmax denominator,
+ * -inf when no token is attended, out = 0 then). */
+static void unit_attention(const orc_shape_t* sh, int b, int g, const uint16_t* q,
+                           const uint16_t* k_pool, const uint16_t* v_pool,
+                           const int32_t* page_table, int32_t seq_len, const int32_t* sel,
+                           int32_t cnt, double sm_scale, double* out, double* lse) {
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    int D = sh->head_dim, bs = sh->block_size;
+    int64_t ntok_max = (int64_t)cnt * bs;
+    double* logit = (double*)malloc((size_t)(ntok_max > 0 ? ntok_max : 1) * sizeof(double));
+    int64_t* row = (int64_t*)malloc((size_t)(ntok_max > 0 ? ntok_max : 1) * sizeof(int64_t));
+    for (int i = 0; i < G; ++i) {
+        int h = g * G + i;
+        const uint16_t* qh = q + ((int64_t)b * sh->num_q_heads + h) * D;
+        int64_t n = 0;
+        for (int32_t c = 0; c < cnt; ++c) {
+            int32_t j = sel[c];
+            int32_t page = page_table[(int64_t)b * sh->max_blocks + j];
+            for (int t = 0; t < bs; ++t) {
+                int64_t pos = (int64_t)j * bs + t;
+                if (pos >= seq_len) break;
+                int64_t r = (((int64_t)page * sh->num_kv_heads + g) * bs + t) * D;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += bf16_to_f64(qh[d]) * bf16_to_f64(k_pool[r + d]);
+                logit[n] = sm_scale * dot;
+                row[n] = r;
+                ++n;
+            }
+        }
+        double* o = out + (int64_t)i * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (n == 0) { lse[i] = -INFINITY; continue; }
+        double m = logit[0];
+        for (int64_t k = 1; k < n; ++k) if (logit[k] > m) m = logit[k];
+        double z = 0.0;
+        for (int64_t k = 0; k < n; ++k) z += exp(logit[k] - m);
+        for (int64_t k = 0; k < n; ++k) {
+            double pk = exp(logit[k] - m) / z;
+            for (int d = 0; d < D; ++d) o[d] += pk * bf16_to_f64(v_pool[row[k] + d]);
+        }
+        lse[i] = m + log(z);
+    }
+    free(logit);
+    free(row);
+}
+
+/* Attention over given selections, for every (b, g):
+ * sel_idx[b][g][max_blocks], sel_cnt[b][g]; out[b][h][D], lse[b][h]. */
+int oracle_sparse_attention(const orc_shape_t* sh, const uint16_t* q, const uint16_t* k_pool,
+                            const uint16_t* v_pool, const int32_t* page_table,
+                            const int32_t* seq_lens, const int32_t* sel_idx,
+                            const int32_t* sel_cnt, double sm_scale, double* out, double* lse) {
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    int units = sh->batch * sh->num_kv_heads;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int u = 0; u < units; ++u) {
+        int b = u / sh->num_kv_heads, g = u % sh->num_kv_heads;
+        unit_attention(sh, b, g, q, k_pool, v_pool, page_table, seq_lens[b],
+                       sel_idx + (int64_t)u * sh->max_blocks, sel_cnt[u], sm_scale,
+                       out + ((int64_t)b * sh->num_q_heads + g * G) * sh->head_dim,
+                       lse + (int64_t)b * sh->num_q_heads + g * G);
+    }
+    return 0;
+}
+
+/* The whole decode step for a list of units (b, g) -- scoring, residual
+ * softmax, dual top-p (or static top-K), sparse attention -- as
+ * SpotAttention §2.1 and §2.3 define it.  units[n_units] holds b*Hkv+g;
+ * NULL means every unit.  Outputs are indexed as in the full problem:
+ * sel_idx[b][g][max_blocks], sel_cnt[b][g], nuc_mass[b][g] (may be NULL),
+ * out[b][h][D], lse[b][h].  Units run in parallel when built with OpenMP. */
+int oracle_decode_step(const orc_shape_t* sh, const orc_params_t* pr, const uint16_t* q_sel,
+                       const float* w, const void* sel_data, const void* sel_scales,
+                       const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                       const int32_t* page_table, const int32_t* seq_lens, const float* top_p,
+                       double sm_scale, const int32_t* units, int32_t n_units,
+                       int32_t* sel_idx, int32_t* sel_cnt, double* nuc_mass, double* out,
+                       double* lse) {
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    int64_t rows = (int64_t)sh->num_pages * sh->num_kv_heads;
+    double* keys = (double*)malloc((size_t)(rows * sh->sel_dim) * sizeof(double));
+    if (!keys) return -2;
+    if (oracle_dequant_selector(sh->sel_fmt, rows, sh->sel_dim, sel_data, sel_scales, keys)) {
+        free(keys);
+        return -1;
+    }
+    int total = units ? n_units : sh->batch * sh->num_kv_heads;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int k = 0; k < total; ++k) {
+        int u = units ? units[k] : k;
+        int b = u / sh->num_kv_heads, g = u % sh->num_kv_heads;
+        int32_t L = seq_lens[b];
+        int64_t nb = ceil_div64(L, sh->block_size), n_full = L / sh->block_size;
+        double* s = (double*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(double));
+        unit_scores(sh, pr, b, g, q_sel, w, keys, page_table, n_full, s);
+        int32_t* sel = sel_idx + (int64_t)u * sh->max_blocks;
+        double mass = 0.0;
+        int32_t cnt = oracle_select_from_scores(s, (int32_t)nb, (int32_t)n_full, pr,
+                                                (double)top_p[b], sel, &mass);
+        sel_cnt[u] = cnt;
+        if (nuc_mass) nuc_mass[u] = mass;
+        unit_attention(sh, b, g, q, k_pool, v_pool, page_table, L, sel, cnt, sm_scale,
+                       out + ((int64_t)b * sh->num_q_heads + g * G) * sh->head_dim,
+                       lse + (int64_t)b * sh->num_q_heads + g * G);
+        free(s);
+    }
+    free(keys);
+    return 0;
+}
+
+/* Threads the OpenMP runtime will use (1 without OpenMP). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

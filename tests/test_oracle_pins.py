@@ -1,0 +1,393 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each test ties one oracle function to something the SpotAttention paper or
+the mathematics fixes: hand-worked examples of Eq. 7-8 (tests/golden),
+brute-force subset enumeration, closed forms, hand-computed selector scores
+(§2.1), the published MX / binary16 formats, and the special cases in which
+sparse attention reduces to a library softmax attention (all blocks kept).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _bf16_bits(values):
+    t = torch.as_tensor(np.asarray(values, np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------- selection
+
+def test_topp_worked_example():
+    ex = _golden("topp_worked_example.json")
+    for case in ex["cases"]:
+        pr = oracle.make_params(sink_blocks=ex["sink_blocks"], recency_blocks=ex["recency_blocks"],
+                                kmin_blocks=case["kmin"])
+        sel, mass = oracle.select_from_scores(ex["scores"], params=pr, p=case["p"])
+        assert sel.tolist() == case["selected"], case
+        # The nucleus mass is the cumulative residual-softmax mass of the
+        # chosen residual blocks.
+        n_res = len(case["selected"]) - 2
+        expect = ex["cumulative_mass"][n_res - 1] if n_res > 0 else 0.0
+        assert abs(mass - expect) < 2e-6, (case, mass)
+    t = ex["tie_case"]
+    pr = oracle.make_params(sink_blocks=1, recency_blocks=1, kmin_blocks=t["kmin"])
+    sel, mass = oracle.select_from_scores(t["scores"], params=pr, p=t["p"])
+    assert sel.tolist() == t["selected"]
+    assert mass == 0.5
+
+
+def _brute_force_nucleus(scores, res, p):
+    """Smallest subsets of the residual blocks whose softmax mass reaches p,
+    found by enumerating every subset (no sorting, no prefix sums)."""
+    s = np.asarray([scores[j] for j in res], np.float64)
+    e = np.exp(s - s.max())
+    prob = e / e.sum()
+    if p <= 0:
+        return 0, [()]
+    for k in range(0, len(res) + 1):
+        hits = [c for c in itertools.combinations(range(len(res)), k)
+                if prob[list(c)].sum() >= p - 1e-12]
+        if hits:
+            return k, [tuple(res[i] for i in c) for c in hits]
+    return len(res), [tuple(res)]
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_select_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    nb = int(rng.integers(1, 15))
+    sink = int(rng.integers(0, 3))
+    rec = int(rng.integers(0, 3))
+    kmin = int(rng.integers(0, 8))
+    if seed % 2:
+        scores = rng.integers(-2, 3, size=nb).astype(np.float64)      # many ties
+    else:
+        scores = rng.normal(size=nb) * 2.0
+    p = float(rng.choice([0.3, 0.5, 0.7, 0.9, 0.95, 0.99, 1.0, 0.0]))
+    pr = oracle.make_params(sink_blocks=sink, recency_blocks=rec, kmin_blocks=kmin)
+    sel, _ = oracle.select_from_scores(scores, params=pr, p=p)
+    reserved = {j for j in range(nb) if j < sink or j >= nb - rec}
+    res = [j for j in range(nb) if j not in reserved]
+    sel_set = set(sel.tolist())
+    # Sorted, unique, reserved blocks always present.
+    assert sel.tolist() == sorted(sel_set)
+    assert reserved <= sel_set
+    nuc = sel_set - reserved
+    if res:
+        k_min_card, minimal = _brute_force_nucleus(scores, res, p)
+        expect_card = min(max(k_min_card, kmin - len(reserved)), len(res))
+        assert len(nuc) == expect_card
+        if expect_card == k_min_card:
+            assert tuple(sorted(nuc)) in [tuple(sorted(c)) for c in minimal]
+        # Ranked-prefix closure: nothing outside beats something inside,
+        # ties broken toward the lower block index.
+        for a in nuc:
+            for b in set(res) - nuc:
+                assert (scores[a] > scores[b]) or (scores[a] == scores[b] and a < b)
+    else:
+        assert nuc == set()
+    if nb:
+        assert len(sel) >= min(kmin, nb)
+
+
+def test_select_incomplete_last_block_is_reserved():
+    # 5 blocks, only 4 complete: block 4 has no score and must be kept.
+    pr = oracle.make_params(sink_blocks=0, recency_blocks=0, kmin_blocks=0)
+    sel, _ = oracle.select_from_scores([5.0, 0.0, 0.0, 0.0, float("nan")], nb=5, n_full=4,
+                                       params=pr, p=0.5)
+    assert sel.tolist() == [0, 4]
+
+
+def test_select_degenerate_sizes():
+    pr = oracle.make_params(sink_blocks=2, recency_blocks=4, kmin_blocks=8)
+    sel, _ = oracle.select_from_scores([1.0, 2.0, 3.0], params=pr, p=0.9)
+    assert sel.tolist() == [0, 1, 2]                       # reserved covers everything
+    sel, _ = oracle.select_from_scores(np.zeros(0), nb=0, params=pr, p=0.9)
+    assert sel.size == 0
+    pr = oracle.make_params(sink_blocks=0, recency_blocks=0, kmin_blocks=100)
+    sel, _ = oracle.select_from_scores(np.arange(10.0), params=pr, p=0.1)
+    assert sel.tolist() == list(range(10))                 # K_min clamps to nb
+
+
+def test_static_topk_mode():
+    pr = oracle.make_params(mode="topk", sink_blocks=0, recency_blocks=0, topk_blocks=3)
+    sel, _ = oracle.select_from_scores([0.5, 4.0, 1.0, 4.0, 3.0, -1.0], params=pr)
+    assert sel.tolist() == [1, 3, 4]
+    pr = oracle.make_params(mode="topk", sink_blocks=1, recency_blocks=1, topk_blocks=2)
+    sel, _ = oracle.select_from_scores([0.5, 2.0, 2.0, 2.0, 3.0, -1.0], params=pr)
+    assert sel.tolist() == [0, 1, 4, 5]
+
+
+# ---------------------------------------------------------------- scoring
+
+def _one_seq_shape(Hq, Hkv, num_pages, max_blocks, fmt="bf16"):
+    return oracle.make_shape(1, Hq, Hkv, 128, 64, 64, fmt, num_pages, max_blocks)
+
+
+def test_scores_hand_computed():
+    # Two query heads share one KV head (G = 2).  Selector dim 64.
+    q = np.zeros((1, 2, 64), np.float32)
+    q[0, 0, 0], q[0, 0, 1] = 1.0, 2.0          # head 0: e0 + 2 e1
+    q[0, 1, 0] = -1.0                           # head 1: -e0
+    keys = np.zeros((2, 1, 64), np.float32)     # two pages
+    keys[1, 0, 0], keys[1, 0, 1], keys[1, 0, 2] = 3.0, -1.0, 5.0   # page 1: dots 1, -3
+    keys[0, 0, 0], keys[0, 0, 1] = -1.0, 4.0                        # page 0: dots 7, 1
+    pt = np.array([[1, 0]], np.int32)           # logical block 0 -> page 1, block 1 -> page 0
+    lens = np.array([128], np.int32)
+    sh = _one_seq_shape(2, 1, 2, 2)
+    w = np.array([[0.25, 0.75]], np.float32)
+    s = oracle.block_scores(sh, oracle.make_params(), _bf16_bits(q), w, _bf16_bits(keys), None,
+                            pt, lens)
+    assert s[0, 0].tolist() == [0.25 * 1 + 0.75 * 0, 0.25 * 7 + 0.75 * 1]
+    s = oracle.block_scores(sh, oracle.make_params(), _bf16_bits(q), None, _bf16_bits(keys), None,
+                            pt, lens)
+    assert s[0, 0].tolist() == [0.5, 4.0]                   # w = 1/G
+    s = oracle.block_scores(sh, oracle.make_params(temperature=2.0), _bf16_bits(q), None,
+                            _bf16_bits(keys), None, pt, lens)
+    assert s[0, 0].tolist() == [0.25, 2.0]
+
+
+def test_scores_gqa_grouping_and_partial_block():
+    # Hq = 4, Hkv = 2: heads 2, 3 read KV head 1 only.
+    q = np.zeros((1, 4, 64), np.float32)
+    q[0, :, 0] = [1.0, 1.0, 2.0, 3.0]
+    keys = np.zeros((1, 2, 64), np.float32)
+    keys[0, 0, 0], keys[0, 1, 0] = 10.0, -1.0
+    sh = _one_seq_shape(4, 2, 1, 2)
+    s = oracle.block_scores(sh, oracle.make_params(), _bf16_bits(q), None, _bf16_bits(keys), None,
+                            np.array([[0, -1]], np.int32), np.array([100], np.int32))
+    assert s[0, 0, 0] == 10.0            # (1*10 + 1*10) / 2
+    assert s[0, 1, 0] == 0.0             # both dots negative: ReLU
+    assert np.isnan(s[0, 0, 1])          # block 1 is incomplete: no score
+
+
+# ---------------------------------------------------------------- key formats
+
+def test_decode_known_codes():
+    g = _golden("selector_codes.json")
+    for c in g["decode"]:
+        data = np.zeros(32, np.uint8)
+        data[0] = c["byte"]
+        if c["fmt"] == "int4":
+            scales = np.array([c["scale_bits"], 0x3C00], np.uint16)
+        else:
+            scales = np.array([c["scale"], 127], np.uint8)
+        vals = oracle.dequant_selector(c["fmt"], data, scales, 64)[0]
+        assert vals[:2].tolist() == c["values"], c["note"]
+
+
+def test_encode_known_codes():
+    g = _golden("selector_codes.json")
+    mx = g["encode_mxfp4"]
+    data, scales = oracle.quantize_selector("mxfp4", _bf16_bits(mx["inputs"] * 2)[None])
+    codes = [int(data[0, i // 2] >> (4 * (i % 2))) & 0xF for i in range(64)]
+    assert codes[:32] == mx["codes"] and codes[32:] == mx["codes"]
+    assert scales[0].tolist() == [mx["scale"], mx["scale"]]
+    i4 = g["encode_int4"]
+    data, scales = oracle.quantize_selector("int4", _bf16_bits(i4["inputs"] * 2)[None])
+    codes = [int(data[0, i // 2] >> (4 * (i % 2))) & 0xF for i in range(64)]
+    codes = [c - 16 if c >= 8 else c for c in codes]
+    assert codes[:32] == i4["codes"] and codes[32:] == i4["codes"]
+    assert scales[0].tolist() == [i4["scale_bits"], i4["scale_bits"]]
+
+
+def test_int4_scale_is_binary16_rne():
+    # The scale is amax/7 rounded to the nearest binary16 (numpy's IEEE
+    # conversion is the independent reference), saturating at 65504.
+    rng = np.random.default_rng(0)
+    amax = np.concatenate([np.exp(rng.uniform(-20, 12, size=400)), [1.0, 7.0, 0.1, 3e5, 1e-9]])
+    x = np.zeros((amax.size, 64), np.float32)
+    x[:, 3] = amax
+    x[:, 40] = -amax
+    bits = _bf16_bits(x)
+    _, scales = oracle.quantize_selector("int4", bits)
+    amax_bf16 = torch.as_tensor(amax.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    ref = np.minimum(amax_bf16 / 7.0, 65504.0).astype(np.float16).view(np.uint16)
+    assert (scales[:, 0] == ref).all() and (scales[:, 1] == ref).all()
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+def test_on_grid_values_round_trip_exactly(fmt):
+    rng = np.random.default_rng(1)
+    rows = 64
+    if fmt == "int4":
+        codes = rng.integers(-7, 8, size=(rows, 64)).astype(np.float64)
+        codes[:, 0], codes[:, 32] = 7, -7                 # amax = 7 * scale
+        scale = np.exp2(rng.integers(-6, 6, size=(rows, 1)))
+        x = codes * scale
+    else:
+        grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+        x = grid[rng.integers(0, 8, size=(rows, 64))] * rng.choice([-1, 1], size=(rows, 64))
+        x[:, 0], x[:, 32] = 6.0, -4.0                     # amax = 6 -> X = 0 before scaling
+        x = x * np.exp2(rng.integers(-10, 10, size=(rows, 1)))
+    bits = _bf16_bits(x)
+    data, scales = oracle.quantize_selector(fmt, bits)
+    back = oracle.dequant_selector(fmt, data, scales, 64)
+    assert np.array_equal(back, x)
+
+
+def test_quantisation_error_bounds():
+    rng = np.random.default_rng(2)
+    x = rng.normal(size=(256, 64)).astype(np.float32)
+    bits = _bf16_bits(x)
+    xb = torch.as_tensor(x).to(torch.bfloat16).double().numpy()
+    for fmt in ("int4", "mxfp4"):
+        data, scales = oracle.quantize_selector(fmt, bits)
+        back = oracle.dequant_selector(fmt, data, scales, 64).reshape(256, 2, 32)
+        xg = xb.reshape(256, 2, 32)
+        amax = np.abs(xg).max(-1, keepdims=True)
+        if fmt == "int4":
+            s = amax / 7.0
+            assert (np.abs(back - xg) <= 0.5 * s * (1 + 1e-3) + 1e-12).all()
+        else:
+            # Scale 2^X with X = floor(log2 amax) - 2 puts |x|/2^X below 8.
+            # Rounding on the E2M1 grid (steps 0.5 / 1 / 2) or saturation at 6
+            # moves an element by less than 2 * 2^X; below 2 * 2^X the grid
+            # step is 0.5, so the error there is at most 2^X / 4.
+            X = np.floor(np.log2(amax)) - 2
+            err = np.abs(back - xg)
+            assert (err < 2 * np.exp2(X)).all()
+            small = np.abs(xg) < 2 * np.exp2(X)
+            assert (err[small] <= (np.exp2(X) / 4 + 0 * xg)[small]).all()
+
+
+def test_footprint_closed_form():
+    # Selector K-cache bytes per element: bf16 16 bits, INT4 4 + 16/32 bits,
+    # MXFP4 4 + 8/32 bits.  The paper's GiB figures follow.
+    fp = _golden("selector_codes.json")["footprint"]
+    n = fp["layers"] * fp["tokens"] * fp["elements_per_token"]
+    for fmt, bits_per in (("bf16", 16.0), ("int4", 4.5), ("mxfp4", 4.25)):
+        x = np.zeros((1, 64), np.float32)
+        data, scales = oracle.quantize_selector(fmt, _bf16_bits(x))
+        stored = data.nbytes + (0 if scales is None else scales.nbytes)
+        assert stored * 8 / 64 == bits_per
+        assert round(n * bits_per / 8 / 2**30, 2) == fp["gib"][fmt]
+
+
+# ---------------------------------------------------------------- attention
+
+def _rand_kv(rng, num_pages, Hkv, Hq, B=1):
+    q = rng.normal(size=(B, Hq, 128)).astype(np.float32)
+    k = rng.normal(size=(num_pages, Hkv, 64, 128)).astype(np.float32)
+    v = rng.normal(size=(num_pages, Hkv, 64, 128)).astype(np.float32)
+    to64 = lambda a: torch.as_tensor(a).to(torch.bfloat16).double()
+    return (q, k, v), (to64(q), to64(k), to64(v))
+
+
+def _sdpa(q64, k64, v64, scale):
+    # torch's own scaled-dot-product attention in float64 (library routine).
+    o = torch.nn.functional.scaled_dot_product_attention(
+        q64[None, None, None], k64[None, None], v64[None, None], scale=scale)
+    return o[0, 0, 0]
+
+
+@pytest.mark.parametrize("L", [1, 64, 200, 256])
+def test_all_blocks_equals_dense_attention(L):
+    rng = np.random.default_rng(L)
+    Hq, Hkv, nb = 4, 2, (L + 63) // 64
+    (q, k, v), (q64, k64, v64) = _rand_kv(rng, nb + 1, Hkv, Hq)
+    pt = np.array([rng.permutation(nb + 1)[:nb]], np.int32)
+    sh = oracle.make_shape(1, Hq, Hkv, 128, 64, 64, "bf16", nb + 1, nb)
+    sel = np.tile(np.arange(nb, dtype=np.int32), (1, Hkv, 1))
+    cnt = np.full((1, Hkv), nb, np.int32)
+    scale = 1 / math.sqrt(128)
+    out, lse = oracle.sparse_attention(sh, _bf16_bits(q), _bf16_bits(k), _bf16_bits(v), pt,
+                                       np.array([L], np.int32), sel, cnt, scale)
+    for h in range(Hq):
+        g = h // 2
+        kk = k64[pt[0], g].reshape(-1, 128)[:L]
+        vv = v64[pt[0], g].reshape(-1, 128)[:L]
+        ref = _sdpa(q64[0, h], kk, vv, scale)
+        assert np.allclose(out[0, h], ref.numpy(), atol=1e-12, rtol=1e-10)
+        ref_lse = torch.logsumexp(scale * (kk @ q64[0, h]), 0).item()
+        assert abs(lse[0, h] - ref_lse) < 1e-10
+
+
+def test_subset_equals_attention_over_gathered_tokens():
+    rng = np.random.default_rng(7)
+    Hq, Hkv, nb = 8, 2, 6
+    (q, k, v), (q64, k64, v64) = _rand_kv(rng, nb, Hkv, Hq)
+    pt = np.array([rng.permutation(nb)], np.int32)
+    sh = oracle.make_shape(1, Hq, Hkv, 128, 64, 64, "bf16", nb, nb)
+    sel = np.full((1, Hkv, nb), -1, np.int32)
+    sel[0, 0, :3] = [0, 2, 5]
+    sel[0, 1, :2] = [1, 4]
+    cnt = np.array([[3, 2]], np.int32)
+    scale = 0.1
+    out, _ = oracle.sparse_attention(sh, _bf16_bits(q), _bf16_bits(k), _bf16_bits(v), pt,
+                                     np.array([nb * 64 - 10], np.int32), sel, cnt, scale)
+    for h in range(Hq):
+        g = h // 4
+        blocks = sel[0, g, :cnt[0, g]]
+        kk = torch.cat([k64[pt[0, j], g] for j in blocks])
+        vv = torch.cat([v64[pt[0, j], g] for j in blocks])
+        if blocks[-1] == nb - 1:
+            kk, vv = kk[:-10], vv[:-10]           # last block holds 54 valid tokens
+        ref = _sdpa(q64[0, h], kk, vv, scale)
+        assert np.allclose(out[0, h], ref.numpy(), atol=1e-12, rtol=1e-10)
+
+
+def test_single_token_and_empty_sequence():
+    rng = np.random.default_rng(3)
+    (q, k, v), (q64, k64, v64) = _rand_kv(rng, 1, 1, 1)
+    sh = oracle.make_shape(1, 1, 1, 128, 64, 64, "bf16", 1, 1)
+    out, lse = oracle.sparse_attention(sh, _bf16_bits(q), _bf16_bits(k), _bf16_bits(v),
+                                       np.array([[0]], np.int32), np.array([1], np.int32),
+                                       np.array([[[0]]], np.int32), np.array([[1]], np.int32), 0.3)
+    assert np.array_equal(out[0, 0], v64[0, 0, 0].numpy())            # o = v
+    assert lse[0, 0] == pytest.approx(0.3 * float(q64[0, 0] @ k64[0, 0, 0]), abs=1e-12)
+    out, lse = oracle.sparse_attention(sh, _bf16_bits(q), _bf16_bits(k), _bf16_bits(v),
+                                       np.array([[0]], np.int32), np.array([0], np.int32),
+                                       np.array([[[0]]], np.int32), np.array([[0]], np.int32), 0.3)
+    assert (out == 0).all() and lse[0, 0] == -np.inf
+
+
+def test_decode_step_composes_and_is_page_order_invariant():
+    import workloads
+    wl = workloads.make("tiny_4k", seed=3, seq_len=1024 + 64 * 3)
+    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, "bf16",
+                           wl.num_pages, wl.max_blocks)
+    pr = oracle.make_params(sink_blocks=1, recency_blocks=2, kmin_blocks=8)
+    args = dict(q_sel=workloads.bits(wl.q_sel), w=None, sel_data=workloads.bits(wl.sel_keys),
+                sel_scales=None, q=workloads.bits(wl.q), k_pool=workloads.bits(wl.k_pool),
+                v_pool=workloads.bits(wl.v_pool), page_table=wl.page_table.numpy(),
+                seq_lens=wl.seq_lens.numpy(), top_p=wl.top_p.numpy(), sm_scale=wl.sm_scale)
+    r = oracle.decode_step(sh, pr, **args)
+    s = oracle.block_scores(sh, pr, args["q_sel"], None, args["sel_data"], None,
+                            args["page_table"], args["seq_lens"])
+    for g in range(wl.num_kv_heads):
+        nb = (int(wl.seq_lens[0]) + 63) // 64
+        sel, _ = oracle.select_from_scores(s[0, g, :nb], params=pr, p=float(wl.top_p[0]))
+        assert sel.tolist() == r["sel_idx"][0, g, :r["sel_cnt"][0, g]].tolist()
+    out, lse = oracle.sparse_attention(sh, args["q"], args["k_pool"], args["v_pool"],
+                                       args["page_table"], args["seq_lens"], r["sel_idx"],
+                                       r["sel_cnt"], wl.sm_scale)
+    assert np.array_equal(out, r["out"]) and np.array_equal(lse, r["lse"])
+    # Planted hot blocks are selected.
+    for g in range(wl.num_kv_heads):
+        chosen = set(r["sel_idx"][0, g, :r["sel_cnt"][0, g]].tolist())
+        assert set(wl.hot_blocks[g]) <= chosen
+    # Moving the pages around (and the page table with them) changes nothing.
+    perm = np.random.default_rng(0).permutation(wl.num_pages)
+    inv = np.argsort(perm)
+    pt2 = np.where(args["page_table"] >= 0, inv[np.maximum(args["page_table"], 0)], -1)
+    args2 = dict(args, page_table=pt2.astype(np.int32), sel_data=args["sel_data"][perm],
+                 k_pool=args["k_pool"][perm], v_pool=args["v_pool"][perm])
+    r2 = oracle.decode_step(sh, pr, **args2)
+    assert np.array_equal(r2["sel_cnt"], r["sel_cnt"])
+    assert np.allclose(r2["out"], r["out"], atol=1e-13, rtol=0)
