@@ -1,0 +1,378 @@
+// api.cu -- the C ABI declared in include/spot.h: host-side validation,
+// workspace layout, tensor-map encoding and kernel launches.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "spot_internal.h"
+
+namespace spot {
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+spot_status_t check_desc(const spot_layer_desc_t* d) {
+    if (!d) return SPOT_ERR_INVALID_ARG;
+    if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_pages <= 0)
+        return SPOT_ERR_INVALID_ARG;
+    if (d->num_q_heads % d->num_kv_heads != 0) return SPOT_ERR_INVALID_ARG;
+    if (d->sel_fmt < SPOT_SEL_BF16 || d->sel_fmt > SPOT_SEL_MXFP4_G32_E8M0)
+        return SPOT_ERR_INVALID_ARG;
+    if (d->head_dim != kHeadDim || d->block_size != kBlock || d->sel_dim != kSelDim)
+        return SPOT_ERR_UNSUPPORTED;
+    if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return SPOT_ERR_UNSUPPORTED;
+    // TMA row coordinates are 32-bit.
+    if (static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock > INT32_MAX)
+        return SPOT_ERR_UNSUPPORTED;
+    return SPOT_OK;
+}
+
+spot_status_t check_batch(const spot_layer_desc_t* d, int batch, int max_blocks) {
+    if (batch < 0 || max_blocks <= 0) return SPOT_ERR_INVALID_ARG;
+    if (max_blocks > kMaxBlocks) return SPOT_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(batch) * d->num_kv_heads > kMaxUnits) return SPOT_ERR_UNSUPPORTED;
+    return SPOT_OK;
+}
+
+spot_status_t check_params(const spot_select_params_t* pr) {
+    if (!pr) return SPOT_ERR_INVALID_ARG;
+    if (pr->mode != SPOT_MODE_TOPP && pr->mode != SPOT_MODE_TOPK) return SPOT_ERR_INVALID_ARG;
+    if (pr->sink_blocks < 0 || pr->recency_blocks < 0 || pr->kmin_blocks < 0 ||
+        pr->topk_blocks < 0)
+        return SPOT_ERR_INVALID_ARG;
+    if (!(pr->temperature > 0.f) || !isfinite(pr->temperature)) return SPOT_ERR_INVALID_ARG;
+    return SPOT_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+bool make_pool_map(CUtensorMap* map, const void* pool, int num_pages, int num_kv_heads) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim),
+                                static_cast<cuuint64_t>(num_pages) * num_kv_heads * kBlock};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBlock)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Layout* out) {
+    const int U = batch * d->num_kv_heads;
+    const int G = d->num_q_heads / d->num_kv_heads;
+    const int grid = decode_grid(U);
+    if (grid <= 0) return false;
+    Layout L;
+    L.grid = grid;
+    size_t off = 0;
+    L.status = off;
+    off += kStatusBytes;
+    L.scores = off;
+    off = round_up(off + static_cast<size_t>(U) * max_blocks * sizeof(float), 256);
+    L.unit_off = off;
+    off = round_up(off + static_cast<size_t>(U + 1) * sizeof(int32_t), 256);
+    L.partials = off;
+    off = round_up(off + static_cast<size_t>(grid + U) * kDecodeConsumers * G *
+                             kPartialFloatsPerHead * sizeof(float),
+                   256);
+    L.total = off;
+    *out = L;
+    return true;
+}
+
+}  // namespace spot
+
+using namespace spot;
+
+namespace {
+
+spot_status_t do_select(const spot_layer_desc_t* d, const spot_select_params_t* pr,
+                        const uint16_t* q_sel, const float* w, const void* sel_data,
+                        const void* sel_scales, const int32_t* page_table, int32_t pt_stride,
+                        const int32_t* seq_lens, const float* top_p, int32_t batch,
+                        int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks, void* ws,
+                        size_t ws_bytes, const Layout& L, cudaStream_t s) {
+    (void)ws_bytes;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    ScoreParams sp;
+    sp.q_sel = q_sel;
+    sp.w = w;
+    sp.sel_data = sel_data;
+    sp.sel_scales = sel_scales;
+    sp.page_table = page_table;
+    sp.pt_stride = pt_stride;
+    sp.seq_lens = seq_lens;
+    sp.batch = batch;
+    sp.num_q_heads = d->num_q_heads;
+    sp.num_kv_heads = d->num_kv_heads;
+    sp.group = d->num_q_heads / d->num_kv_heads;
+    sp.num_pages = d->num_pages;
+    sp.max_blocks = max_blocks;
+    sp.inv_temp = 1.0f / pr->temperature;
+    sp.scores = reinterpret_cast<float*>(base + L.scores);
+    sp.status = reinterpret_cast<uint32_t*>(base + L.status);
+    if (launch_scores(sp, d->sel_fmt, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    SelectParams sl;
+    sl.scores = sp.scores;
+    sl.seq_lens = seq_lens;
+    sl.top_p = top_p;
+    sl.pt_stride = pt_stride;
+    sl.batch = batch;
+    sl.num_kv_heads = d->num_kv_heads;
+    sl.max_blocks = max_blocks;
+    sl.mode = pr->mode;
+    sl.sink_blocks = pr->sink_blocks;
+    sl.recency_blocks = pr->recency_blocks;
+    sl.kmin_blocks = pr->kmin_blocks;
+    sl.topk_blocks = pr->topk_blocks;
+    sl.sel_idx = sel_idx;
+    sl.sel_cnt = sel_cnt;
+    sl.status = sp.status;
+    if (launch_select(sl, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    return SPOT_OK;
+}
+
+spot_status_t do_decode(const spot_layer_desc_t* d, const uint16_t* q, const uint16_t* k_pool,
+                        const uint16_t* v_pool, const int32_t* page_table, int32_t pt_stride,
+                        const int32_t* seq_lens, const int32_t* sel_idx, const int32_t* sel_cnt,
+                        int32_t max_blocks, int32_t batch, float softmax_scale, float* out,
+                        float* lse, void* ws, const Layout& L, cudaStream_t s) {
+    CUtensorMap km, vm;
+    if (!make_pool_map(&km, k_pool, d->num_pages, d->num_kv_heads) ||
+        !make_pool_map(&vm, v_pool, d->num_pages, d->num_kv_heads))
+        return SPOT_ERR_CUDA;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    DecodeParams p;
+    p.q = q;
+    p.page_table = page_table;
+    p.pt_stride = pt_stride;
+    p.seq_lens = seq_lens;
+    p.sel_idx = sel_idx;
+    p.sel_cnt = sel_cnt;
+    p.max_blocks = max_blocks;
+    p.batch = batch;
+    p.num_q_heads = d->num_q_heads;
+    p.num_kv_heads = d->num_kv_heads;
+    p.group = d->num_q_heads / d->num_kv_heads;
+    p.num_pages = d->num_pages;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.unit_off = reinterpret_cast<int32_t*>(base + L.unit_off);
+    p.partials = reinterpret_cast<float*>(base + L.partials);
+    p.num_ctas = L.grid;
+    p.out = out;
+    p.lse = lse;
+    p.status = reinterpret_cast<uint32_t*>(base + L.status);
+    if (launch_sparse_decode(p, km, vm, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    return SPOT_OK;
+}
+
+spot_status_t check_select_args(const spot_layer_desc_t* d, const spot_select_params_t* pr,
+                                const uint16_t* q_sel, const float* w, const void* sel_data,
+                                const void* sel_scales, const int32_t* page_table,
+                                int32_t pt_stride, const int32_t* seq_lens, const float* top_p,
+                                int32_t* sel_idx, int32_t* sel_cnt) {
+    spot_status_t st = check_params(pr);
+    if (st != SPOT_OK) return st;
+    if (!q_sel || !sel_data || !page_table || !seq_lens || !sel_idx || !sel_cnt)
+        return SPOT_ERR_INVALID_ARG;
+    if (pr->mode == SPOT_MODE_TOPP && !top_p) return SPOT_ERR_INVALID_ARG;
+    if (d->sel_fmt != SPOT_SEL_BF16 && !sel_scales) return SPOT_ERR_INVALID_ARG;
+    if (pt_stride <= 0) return SPOT_ERR_INVALID_ARG;
+    if (!aligned(q_sel, 16) || !aligned(sel_data, 16) || !aligned(page_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(sel_idx, 4) || !aligned(sel_cnt, 4) ||
+        (w && !aligned(w, 4)) || (top_p && !aligned(top_p, 4)) ||
+        (sel_scales && !aligned(sel_scales, 4)))
+        return SPOT_ERR_INVALID_ARG;
+    return SPOT_OK;
+}
+
+spot_status_t check_decode_args(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                                const int32_t* page_table, int32_t pt_stride,
+                                const int32_t* seq_lens, const int32_t* sel_idx,
+                                const int32_t* sel_cnt, float softmax_scale, float* out,
+                                float* lse) {
+    if (!q || !k_pool || !v_pool || !page_table || !seq_lens || !sel_idx || !sel_cnt || !out)
+        return SPOT_ERR_INVALID_ARG;
+    if (pt_stride <= 0 || !isfinite(softmax_scale)) return SPOT_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_pool, 256) || !aligned(v_pool, 256) ||
+        !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(sel_idx, 4) ||
+        !aligned(sel_cnt, 4) || !aligned(out, 4) || (lse && !aligned(lse, 4)))
+        return SPOT_ERR_INVALID_ARG;
+    return SPOT_OK;
+}
+
+spot_status_t check_ws(void* ws, size_t ws_bytes, const Layout& L) {
+    if (!ws || !aligned(ws, 256)) return SPOT_ERR_INVALID_ARG;
+    if (ws_bytes < L.total) return SPOT_ERR_WORKSPACE;
+    return SPOT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t spot_workspace_size(const spot_layer_desc_t* desc, int32_t batch, int32_t max_blocks) {
+    if (check_desc(desc) != SPOT_OK || check_batch(desc, batch, max_blocks) != SPOT_OK) return 0;
+    Layout L;
+    if (!workspace_layout(desc, batch, max_blocks, &L)) return 0;
+    return L.total;
+}
+
+spot_status_t spot_append_selector_keys(const spot_layer_desc_t* desc, void* sel_data,
+                                        void* sel_scales, const int32_t* page_table,
+                                        int32_t num_seqs, int32_t pt_stride,
+                                        const int32_t* seq_ids, const int32_t* block_ids,
+                                        const uint16_t* keys, int32_t n, void* status_ws,
+                                        void* stream) {
+    spot_status_t st = check_desc(desc);
+    if (st != SPOT_OK) return st;
+    if (n < 0 || pt_stride <= 0 || num_seqs < 0) return SPOT_ERR_INVALID_ARG;
+    if (n == 0) return SPOT_OK;
+    if (!sel_data || !page_table || !seq_ids || !block_ids || !keys) return SPOT_ERR_INVALID_ARG;
+    if (desc->sel_fmt != SPOT_SEL_BF16 && !sel_scales) return SPOT_ERR_INVALID_ARG;
+    if (!aligned(sel_data, 4) || !aligned(keys, 4) || !aligned(page_table, 4) ||
+        !aligned(seq_ids, 4) || !aligned(block_ids, 4) || (sel_scales && !aligned(sel_scales, 2)))
+        return SPOT_ERR_INVALID_ARG;
+    if (status_ws && !aligned(status_ws, 256)) return SPOT_ERR_INVALID_ARG;
+    AppendParams p;
+    p.sel_data = sel_data;
+    p.sel_scales = sel_scales;
+    p.page_table = page_table;
+    p.num_seqs = num_seqs;
+    p.pt_stride = pt_stride;
+    p.seq_ids = seq_ids;
+    p.block_ids = block_ids;
+    p.keys = keys;
+    p.n = n;
+    p.num_kv_heads = desc->num_kv_heads;
+    p.num_pages = desc->num_pages;
+    p.fmt = desc->sel_fmt;
+    p.status = static_cast<uint32_t*>(status_ws);
+    return launch_append(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SPOT_OK
+                                                                             : SPOT_ERR_CUDA;
+}
+
+spot_status_t spot_select(const spot_layer_desc_t* desc, const spot_select_params_t* params,
+                          const uint16_t* q_sel, const float* w, const void* sel_data,
+                          const void* sel_scales, const int32_t* page_table, int32_t pt_stride,
+                          const int32_t* seq_lens, const float* top_p, int32_t batch,
+                          int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
+                          void* workspace, size_t ws_bytes, void* stream) {
+    spot_status_t st = check_desc(desc);
+    if (st == SPOT_OK) st = check_batch(desc, batch, max_blocks);
+    if (st != SPOT_OK) return st;
+    if (batch == 0) return SPOT_OK;
+    st = check_select_args(desc, params, q_sel, w, sel_data, sel_scales, page_table, pt_stride,
+                           seq_lens, top_p, sel_idx, sel_cnt);
+    if (st != SPOT_OK) return st;
+    Layout L;
+    if (!workspace_layout(desc, batch, max_blocks, &L)) return SPOT_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, L);
+    if (st != SPOT_OK) return st;
+    return do_select(desc, params, q_sel, w, sel_data, sel_scales, page_table, pt_stride,
+                     seq_lens, top_p, batch, sel_idx, sel_cnt, max_blocks, workspace, ws_bytes,
+                     L, static_cast<cudaStream_t>(stream));
+}
+
+spot_status_t spot_sparse_decode(const spot_layer_desc_t* desc, const uint16_t* q,
+                                 const uint16_t* k_pool, const uint16_t* v_pool,
+                                 const int32_t* page_table, int32_t pt_stride,
+                                 const int32_t* seq_lens, const int32_t* sel_idx,
+                                 const int32_t* sel_cnt, int32_t max_blocks, int32_t batch,
+                                 float softmax_scale, float* out, float* lse, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+    spot_status_t st = check_desc(desc);
+    if (st == SPOT_OK) st = check_batch(desc, batch, max_blocks);
+    if (st != SPOT_OK) return st;
+    if (batch == 0) return SPOT_OK;
+    st = check_decode_args(q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx, sel_cnt,
+                           softmax_scale, out, lse);
+    if (st != SPOT_OK) return st;
+    Layout L;
+    if (!workspace_layout(desc, batch, max_blocks, &L)) return SPOT_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, L);
+    if (st != SPOT_OK) return st;
+    return do_decode(desc, q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx, sel_cnt,
+                     max_blocks, batch, softmax_scale, out, lse, workspace, L,
+                     static_cast<cudaStream_t>(stream));
+}
+
+spot_status_t spot_decode_step(const spot_layer_desc_t* desc, const spot_select_params_t* params,
+                               const uint16_t* q_sel, const float* w, const void* sel_data,
+                               const void* sel_scales, const uint16_t* q, const uint16_t* k_pool,
+                               const uint16_t* v_pool, const int32_t* page_table,
+                               int32_t pt_stride, const int32_t* seq_lens, const float* top_p,
+                               int32_t batch, float softmax_scale, int32_t* sel_idx,
+                               int32_t* sel_cnt, int32_t max_blocks, float* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream) {
+    spot_status_t st = check_desc(desc);
+    if (st == SPOT_OK) st = check_batch(desc, batch, max_blocks);
+    if (st != SPOT_OK) return st;
+    if (batch == 0) return SPOT_OK;
+    st = check_select_args(desc, params, q_sel, w, sel_data, sel_scales, page_table, pt_stride,
+                           seq_lens, top_p, sel_idx, sel_cnt);
+    if (st == SPOT_OK)
+        st = check_decode_args(q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx,
+                               sel_cnt, softmax_scale, out, lse);
+    if (st != SPOT_OK) return st;
+    Layout L;
+    if (!workspace_layout(desc, batch, max_blocks, &L)) return SPOT_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, L);
+    if (st != SPOT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = do_select(desc, params, q_sel, w, sel_data, sel_scales, page_table, pt_stride, seq_lens,
+                   top_p, batch, sel_idx, sel_cnt, max_blocks, workspace, ws_bytes, L, s);
+    if (st != SPOT_OK) return st;
+    return do_decode(desc, q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx, sel_cnt,
+                     max_blocks, batch, softmax_scale, out, lse, workspace, L, s);
+}
+
+spot_status_t spot_read_device_status(void* workspace, void* stream) {
+    if (!workspace || !aligned(workspace, 256)) return SPOT_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SPOT_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPOT_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof word, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPOT_ERR_CUDA;
+    if (word & kStatusBounds) return SPOT_ERR_DEVICE_BOUNDS;
+    if (word & kStatusTimeout) return SPOT_ERR_DEVICE_TIMEOUT;
+    return SPOT_OK;
+}
+
+const char* spot_status_string(spot_status_t status) {
+    switch (status) {
+        case SPOT_OK: return "ok";
+        case SPOT_ERR_INVALID_ARG: return "invalid argument";
+        case SPOT_ERR_UNSUPPORTED: return "unsupported shape";
+        case SPOT_ERR_WORKSPACE: return "workspace too small";
+        case SPOT_ERR_CUDA: return "CUDA error";
+        case SPOT_ERR_DEVICE_BOUNDS: return "device: index out of range";
+        case SPOT_ERR_DEVICE_TIMEOUT: return "device: bounded wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

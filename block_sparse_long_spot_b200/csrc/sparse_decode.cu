@@ -1,0 +1,449 @@
+// sparse_decode.cu -- exact attention over the selected KV blocks
+// (SpotAttention §2.3: the layer attends only to keys in the selected
+// blocks; decode only), split across a persistent grid, then a combine.
+//
+// Work decomposition ("stream-K" over blocks): the selected blocks of all
+// (sequence, KV head) units, each unit's list in ascending block order, are
+// laid end to end; CTA i of the P-CTA grid takes the contiguous range
+// [floor(i N / P), floor((i+1) N / P)) of that list, so every CTA streams
+// the same number of 32 KiB (K + V) tiles whatever the per-unit budgets.
+// Where a range crosses a unit boundary the CTA emits one partial result per
+// unit it touched; the combine kernel merges a unit's partials with their
+// log-sum-exp weights.
+//
+// Inside a CTA one producer warp issues TMA tile loads of the gathered pages
+// (two 64 x 64 bf16 boxes each for K and V, 128-byte swizzled) into a ring
+// of stages guarded by mbarriers; NC consumer warps each take every NC-th
+// tile and keep their own online-softmax state for the G <= 8 query heads of
+// the unit's KV head:
+//   S^T[64 tok x 8 heads] = K[64 x 128] . Q^T        (mma m16n8k16, bf16)
+//   online softmax over tokens (exp2, scale folded into log2 domain)
+//   O^T[128 x 8] += V^T[128 x 64] . P^T[64 x 8]      (P^T via movmatrix)
+// Each warp writes its own partial (acc[G][128], m[G], l[G]).
+#include <math.h>
+#include <stdio.h>
+
+#include "spot_device.cuh"
+#include "spot_internal.h"
+
+namespace spot {
+namespace {
+
+constexpr int NC = kDecodeConsumers;
+constexpr int STAGES = kDecodeStages;
+constexpr int kThreads = (NC + 1) * 32;
+constexpr int kHalfTile = kBlock * 64 * 2;   // 8 KiB: 64 rows x 64 bf16
+
+struct Smem {
+    // stage s: [K lo | K hi | V lo | V hi], 8 KiB each, 1024-byte aligned
+    uint32_t stage_base;
+    uint64_t* full;
+    uint64_t* empty;
+    int* valid;          // [STAGES] valid tokens of the block in each stage
+    int* unit_off;       // [U + 1]
+    int* scan;           // [kThreads/32 + 1]
+};
+
+__device__ __forceinline__ int find_unit(const int* off, int U, int pos) {
+    // largest u in [0, U) with off[u] <= pos
+    int lo = 0, hi = U - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= pos) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ int range_begin(int64_t N, int64_t P, int64_t i) {
+    return static_cast<int>((N * i) / P);
+}
+
+__global__ void __launch_bounds__(kThreads)
+sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
+                     const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int U = p.batch * p.num_kv_heads;
+    const int G = p.group;
+
+    // ---- shared memory carve-up (stages first, 1024-aligned)
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    uint8_t* base = smem_raw + pad;
+    uint8_t* tail = base + STAGES * kStageBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(tail);
+    uint64_t* empty = full + STAGES;
+    int* valid = reinterpret_cast<int*>(empty + STAGES);
+    int* scan = valid + STAGES;
+    int* unit_off = scan + (kThreads / 32 + 1);
+    const uint32_t stage_base = smem_u32(base);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == NC && lane == 0) {
+        prefetch_tensormap(&k_map);
+        prefetch_tensormap(&v_map);
+    }
+
+    // ---- prefix sum of the per-unit counts (every CTA computes its own copy)
+    const int per = (U + kThreads - 1) / kThreads;
+    const int u_lo = min(U, static_cast<int>(threadIdx.x) * per);
+    const int u_hi = min(U, u_lo + per);
+    int local = 0;
+    for (int u = u_lo; u < u_hi; ++u) {
+        const int b = u / p.num_kv_heads;
+        const int L = max(p.seq_lens[b], 0);
+        const int nb = min((L + kBlock - 1) / kBlock, p.max_blocks);
+        int c = p.sel_cnt[u];
+        if (c < 0 || c > nb) {
+            if (blockIdx.x == 0) flag_status(p.status, kStatusBounds);
+            c = min(max(c, 0), nb);
+        }
+        unit_off[u] = c;          // temporarily the count
+        local += c;
+    }
+    int total;
+    int run = block_exclusive_scan<kThreads>(local, scan, &total);
+    for (int u = u_lo; u < u_hi; ++u) {
+        const int c = unit_off[u];
+        unit_off[u] = run;
+        run += c;
+    }
+    if (threadIdx.x == 0) unit_off[U] = total;
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int u = threadIdx.x; u <= U; u += kThreads) p.unit_off[u] = unit_off[u];
+    }
+
+    const int64_t N = total;
+    const int64_t P = p.num_ctas;
+    const int beg = range_begin(N, P, blockIdx.x);
+    const int end = range_begin(N, P, blockIdx.x + 1);
+    if (beg >= end) return;
+    const int n_it = end - beg;
+
+    if (warp == NC) {
+        // ================================================= producer warp
+        const uint64_t policy = l2_policy_evict_first();
+        bool alive = true;
+        int issued = 0;
+        for (int base_it = 0; base_it < n_it && alive; base_it += 32) {
+            const int it = base_it + lane;
+            int row = 0, nvalid = 0;
+            if (it < n_it) {
+                const int pos = beg + it;
+                const int u = find_unit(unit_off, U, pos);
+                const int i = pos - unit_off[u];
+                const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+                const int j = p.sel_idx[static_cast<int64_t>(u) * p.max_blocks + i];
+                const int L = max(p.seq_lens[b], 0);
+                const int nb = (L + kBlock - 1) / kBlock;
+                int page = -1;
+                if (j >= 0 && j < nb && j < p.pt_stride)
+                    page = p.page_table[static_cast<int64_t>(b) * p.pt_stride + j];
+                if (page < 0 || page >= p.num_pages) {
+                    flag_status(p.status, kStatusBounds);
+                    page = 0;
+                    nvalid = 0;                 // tile is loaded but not attended
+                } else {
+                    nvalid = min(kBlock, L - j * kBlock);
+                }
+                row = (page * p.num_kv_heads + g) * kBlock;
+            }
+            const int n_here = min(32, n_it - base_it);
+            for (int k = 0; k < n_here; ++k) {
+                const int r = __shfl_sync(0xffffffffu, row, k);
+                const int v = __shfl_sync(0xffffffffu, nvalid, k);
+                const int itk = base_it + k;
+                const int s = itk % STAGES;
+                const int round = itk / STAGES;
+                int ok = 1;
+                if (lane == 0) {
+                    if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
+                        flag_status(p.status, kStatusTimeout);
+                        ok = 0;
+                    } else {
+                        valid[s] = v;
+                        mbar_arrive_expect_tx(&full[s], kStageBytes);
+                        uint8_t* dst = base + s * kStageBytes;
+                        tma_load_2d(dst, &k_map, &full[s], 0, r, policy);
+                        tma_load_2d(dst + kHalfTile, &k_map, &full[s], 64, r, policy);
+                        tma_load_2d(dst + 2 * kHalfTile, &v_map, &full[s], 0, r, policy);
+                        tma_load_2d(dst + 3 * kHalfTile, &v_map, &full[s], 64, r, policy);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) { alive = false; break; }
+                ++issued;
+            }
+        }
+        if (!alive && lane == 0) {
+            // Let the copies already in flight land before the CTA can exit.
+            for (int itk = max(0, issued - STAGES); itk < issued; ++itk)
+                (void)mbar_wait_bounded(&full[itk % STAGES], (itk / STAGES) & 1);
+        }
+        return;
+    }
+
+    // ===================================================== consumer warps
+    const int c4 = lane & 3;         // column pair: heads 2*c4, 2*c4+1
+    const int r8 = lane >> 2;        // row within an 8-row group
+    int pos = beg;
+    while (pos < end) {
+        const int u = find_unit(unit_off, U, pos);
+        const int seg_end = min(end, unit_off[u + 1]);
+        const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+
+        // Q^T fragments (B operand, k = head dim, n = head): lane holds
+        // head r8, dims 16 ks + 2 c4 + {0,1} (b0) and + 8 (b1).
+        uint32_t qf[8][2];
+        {
+            const bool real = r8 < G;
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                p.q + (static_cast<int64_t>(b) * p.num_q_heads + g * G + (real ? r8 : 0)) *
+                          kHeadDim);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                qf[ks][0] = real ? __ldg(qrow + ks * 8 + c4) : 0u;
+                qf[ks][1] = real ? __ldg(qrow + ks * 8 + 4 + c4) : 0u;
+            }
+        }
+        float m0 = -INFINITY, m1 = -INFINITY;     // running max (log2 domain)
+        float l0 = 0.f, l1 = 0.f;                 // this lane's share of the sum
+        float acc[8][4];
+#pragma unroll
+        for (int md = 0; md < 8; ++md)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[md][e] = 0.f;
+
+        const int it0 = pos - beg, it1 = seg_end - beg;
+        const int first = it0 + ((warp - it0) % NC + NC) % NC;
+        bool alive = true;
+        for (int it = first; it < it1; it += NC) {
+            const int s = it % STAGES;
+            if (!mbar_wait_bounded(&full[s], (it / STAGES) & 1)) {
+                if (lane == 0) flag_status(p.status, kStatusTimeout);
+                alive = false;
+                break;
+            }
+            const int nvalid = valid[s];
+            const uint32_t kb = stage_base + s * kStageBytes;
+            const uint32_t vb = kb + 2 * kHalfTile;
+
+            // ---- S^T = K Q^T: 4 m-tiles of 16 tokens
+            float sc[4][4];
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t hb = kb + (ks >> 2) * kHalfTile;
+                const int chunk = ((ks & 3) << 1) + (lane >> 4);
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt) {
+                    const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(swz128(hb, row, chunk), a0, a1, a2, a3);
+                    mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                }
+            }
+            // ---- mask tokens past the end of the sequence
+            if (nvalid < kBlock) {
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt) {
+                    const int t0 = mt * 16 + r8, t1 = t0 + 8;
+                    if (t0 >= nvalid) { sc[mt][0] = -INFINITY; sc[mt][1] = -INFINITY; }
+                    if (t1 >= nvalid) { sc[mt][2] = -INFINITY; sc[mt][3] = -INFINITY; }
+                }
+            }
+            // ---- online softmax per head (columns 2 c4, 2 c4 + 1)
+            float x0 = fmaxf(fmaxf(sc[0][0], sc[0][2]), fmaxf(sc[1][0], sc[1][2]));
+            x0 = fmaxf(x0, fmaxf(fmaxf(sc[2][0], sc[2][2]), fmaxf(sc[3][0], sc[3][2])));
+            float x1 = fmaxf(fmaxf(sc[0][1], sc[0][3]), fmaxf(sc[1][1], sc[1][3]));
+            x1 = fmaxf(x1, fmaxf(fmaxf(sc[2][1], sc[2][3]), fmaxf(sc[3][1], sc[3][3])));
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, o));
+                x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, o));
+            }
+            const float n0 = fmaxf(m0, x0 * p.scale_log2);
+            const float n1 = fmaxf(m1, x1 * p.scale_log2);
+            // n == -inf only when nothing has been attended yet: keep 0 as
+            // the reference so exp2 stays finite (all p are 0 then).
+            const float r0 = (n0 == -INFINITY) ? 0.f : n0;
+            const float r1 = (n1 == -INFINITY) ? 0.f : n1;
+            const float al0 = exp2f(m0 - r0), al1 = exp2f(m1 - r1);
+            m0 = n0;
+            m1 = n1;
+            uint32_t pb[4][2];
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+                const float p0 = exp2f(fmaf(sc[mt][0], p.scale_log2, -r0));
+                const float p1 = exp2f(fmaf(sc[mt][1], p.scale_log2, -r1));
+                const float p2 = exp2f(fmaf(sc[mt][2], p.scale_log2, -r0));
+                const float p3 = exp2f(fmaf(sc[mt][3], p.scale_log2, -r1));
+                s0 += p0 + p2;
+                s1 += p1 + p3;
+                pb[mt][0] = movmatrix_trans(pack_bf16(p0, p1));
+                pb[mt][1] = movmatrix_trans(pack_bf16(p2, p3));
+            }
+            l0 = l0 * al0 + s0;
+            l1 = l1 * al1 + s1;
+#pragma unroll
+            for (int md = 0; md < 8; ++md) {
+                acc[md][0] *= al0;
+                acc[md][1] *= al1;
+                acc[md][2] *= al0;
+                acc[md][3] *= al1;
+            }
+            // ---- O^T += V^T P^T: 8 m-tiles of 16 dims x 4 k-tiles of 16 tokens
+#pragma unroll
+            for (int md = 0; md < 8; ++md) {
+                const uint32_t hb = vb + (md >> 2) * kHalfTile;
+                const int chunk = ((md & 3) << 1) + ((lane >> 3) & 1);
+#pragma unroll
+                for (int kt = 0; kt < 4; ++kt) {
+                    const int row = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_trans(swz128(hb, row, chunk), a0, a1, a2, a3);
+                    mma_bf16_16816(acc[md], a0, a1, a2, a3, pb[kt][0], pb[kt][1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        if (!alive) return;
+
+        // ---- this warp's partial for unit u
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        }
+        float* slot = p.partials + (static_cast<int64_t>(blockIdx.x + u) * NC + warp) *
+                                       (static_cast<int64_t>(G) * kPartialFloatsPerHead);
+        const int h0 = 2 * c4, h1 = 2 * c4 + 1;
+#pragma unroll
+        for (int md = 0; md < 8; ++md) {
+            const int d0 = md * 16 + r8, d1 = d0 + 8;
+            if (h0 < G) {
+                slot[h0 * kHeadDim + d0] = acc[md][0];
+                slot[h0 * kHeadDim + d1] = acc[md][2];
+            }
+            if (h1 < G) {
+                slot[h1 * kHeadDim + d0] = acc[md][1];
+                slot[h1 * kHeadDim + d1] = acc[md][3];
+            }
+        }
+        if (r8 == 0) {
+            if (h0 < G) {
+                slot[G * kHeadDim + h0] = m0;
+                slot[G * (kHeadDim + 1) + h0] = l0;
+            }
+            if (h1 < G) {
+                slot[G * kHeadDim + h1] = m1;
+                slot[G * (kHeadDim + 1) + h1] = l1;
+            }
+        }
+        pos = seg_end;
+    }
+}
+
+// CTA i of the persistent grid that owns flattened position pos.
+__device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
+    return static_cast<int>(((pos + 1) * P - 1) / N);
+}
+
+// One CTA per (sequence, KV head) unit, one thread per head dimension.
+__global__ void __launch_bounds__(kHeadDim) combine_kernel(const DecodeParams p) {
+    const int u = blockIdx.x;
+    const int U = p.batch * p.num_kv_heads;
+    const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+    const int G = p.group;
+    const int d = threadIdx.x;
+    const int lo = p.unit_off[u], hi = p.unit_off[u + 1];
+    const int64_t N = p.unit_off[U];
+    const int64_t P = p.num_ctas;
+    for (int n = 0; n < G; ++n) {
+        const int h = g * G + n;
+        float* o = p.out + (static_cast<int64_t>(b) * p.num_q_heads + h) * kHeadDim;
+        if (hi <= lo) {
+            o[d] = 0.f;
+            if (p.lse && d == 0) p.lse[static_cast<int64_t>(b) * p.num_q_heads + h] = -INFINITY;
+            continue;
+        }
+        const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
+        const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
+        float M = -INFINITY;
+        for (int i = i0; i <= i1; ++i) {
+            if (range_begin(N, P, i) == range_begin(N, P, i + 1)) continue;   // idle CTA
+            for (int w = 0; w < NC; ++w) {
+                const float* slot = p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
+                M = fmaxf(M, slot[G * kHeadDim + n]);
+            }
+        }
+        float L = 0.f, a = 0.f;
+        for (int i = i0; i <= i1; ++i) {
+            if (range_begin(N, P, i) == range_begin(N, P, i + 1)) continue;
+            for (int w = 0; w < NC; ++w) {
+                const float* slot = p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
+                const float m = slot[G * kHeadDim + n];
+                if (m == -INFINITY) continue;
+                const float f = exp2f(m - M);
+                L = fmaf(f, slot[G * (kHeadDim + 1) + n], L);
+                a = fmaf(f, slot[n * kHeadDim + d], a);
+            }
+        }
+        const bool empty = !(L > 0.f);      // only if every tile was rejected as out of range
+        o[d] = empty ? 0.f : a / L;
+        if (p.lse && d == 0)
+            p.lse[static_cast<int64_t>(b) * p.num_q_heads + h] =
+                empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+    }
+}
+
+}  // namespace
+
+size_t decode_smem_bytes(int units) {
+    return 1024 /* alignment slack */ + static_cast<size_t>(STAGES) * kStageBytes +
+           2 * STAGES * sizeof(uint64_t) + STAGES * sizeof(int) +
+           (kThreads / 32 + 1) * sizeof(int) + static_cast<size_t>(units + 1) * sizeof(int);
+}
+
+int decode_grid(int units) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    const size_t smem = decode_smem_bytes(units);
+    if (cudaFuncSetAttribute(sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_decode_kernel, kThreads,
+                                                      smem) != cudaSuccess)
+        return 0;
+    return sms * max(per_sm, 1);
+}
+
+cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
+                                 const CUtensorMap& v_map, cudaStream_t s) {
+    const int U = p.batch * p.num_kv_heads;
+    const size_t smem = decode_smem_bytes(U);
+    cudaError_t e = cudaFuncSetAttribute(
+        sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    sparse_decode_kernel<<<p.num_ctas, kThreads, smem, s>>>(k_map, v_map, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    combine_kernel<<<U, kHeadDim, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace spot

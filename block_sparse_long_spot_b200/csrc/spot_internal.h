@@ -1,0 +1,112 @@
+// spot_internal.h -- host-side declarations shared by the library's .cu
+// files: kernel parameter blocks, launchers and the workspace layout.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/spot.h"
+
+namespace spot {
+
+constexpr int kHeadDim = 128;
+constexpr int kBlock = 64;
+constexpr int kSelDim = 64;
+constexpr int kMaxGroup = 8;           // query heads per KV head (mma N = 8)
+constexpr int kMaxUnits = 4096;        // batch * num_kv_heads
+constexpr int kMaxBlocks = 16384;      // blocks per sequence
+constexpr int kStatusBytes = 256;      // workspace header
+
+// Status bits OR-ed into the workspace status word by kernels.
+constexpr uint32_t kStatusBounds = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+
+// Sparse-decode kernel configuration: consumer warps and pipeline stages
+// (one stage = the K and V tiles of one block of one KV head, 32 KiB).
+constexpr int kDecodeConsumers = 4;
+constexpr int kDecodeStages = 4;
+constexpr int kStageBytes = 2 * kBlock * kHeadDim * 2;   // 32768
+constexpr int kPartialFloatsPerHead = kHeadDim + 2;      // acc[128], m, l
+
+struct Layout {
+    size_t status, scores, unit_off, partials, total;
+    int grid;                           // persistent CTAs of the decode kernel
+};
+
+// Workspace layout for a shape on the current device.
+bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Layout* out);
+
+struct ScoreParams {
+    const uint16_t* q_sel;
+    const float* w;
+    const void* sel_data;
+    const void* sel_scales;
+    const int32_t* page_table;
+    int32_t pt_stride;
+    const int32_t* seq_lens;
+    int32_t batch, num_q_heads, num_kv_heads, group, num_pages, max_blocks;
+    float inv_temp;
+    float* scores;                      // [B][Hkv][max_blocks]
+    uint32_t* status;
+};
+
+struct SelectParams {
+    const float* scores;
+    const int32_t* seq_lens;
+    const float* top_p;
+    int32_t pt_stride;
+    int32_t batch, num_kv_heads, max_blocks;
+    int32_t mode, sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
+    int32_t* sel_idx;
+    int32_t* sel_cnt;
+    uint32_t* status;
+};
+
+struct DecodeParams {
+    const uint16_t* q;
+    const int32_t* page_table;
+    int32_t pt_stride;
+    const int32_t* seq_lens;
+    const int32_t* sel_idx;
+    const int32_t* sel_cnt;
+    int32_t max_blocks, batch, num_q_heads, num_kv_heads, group, num_pages;
+    float scale_log2;                   // softmax_scale * log2(e)
+    int32_t* unit_off;                  // [U + 1] written by CTA 0
+    float* partials;
+    int32_t num_ctas;
+    float* out;
+    float* lse;
+    uint32_t* status;
+};
+
+struct AppendParams {
+    void* sel_data;
+    void* sel_scales;
+    const int32_t* page_table;
+    int32_t num_seqs;
+    int32_t pt_stride;
+    const int32_t* seq_ids;
+    const int32_t* block_ids;
+    const uint16_t* keys;
+    int32_t n, num_kv_heads, num_pages, fmt;
+    uint32_t* status;
+};
+
+cudaError_t launch_scores(const ScoreParams& p, int fmt, cudaStream_t s);
+cudaError_t launch_select(const SelectParams& p, cudaStream_t s);
+cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
+                                 const CUtensorMap& v_map, cudaStream_t s);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+
+// Persistent grid of the decode kernel for U units on the current device.
+int decode_grid(int units);
+size_t decode_smem_bytes(int units);
+size_t select_smem_bytes(int max_blocks);
+
+// Tensor map over a KV pool viewed as [num_pages*Hkv*64 rows][128 bf16],
+// box 64 x 64, 128-byte swizzle.
+bool make_pool_map(CUtensorMap* map, const void* pool, int num_pages, int num_kv_heads);
+
+}  // namespace spot

@@ -1,0 +1,200 @@
+/*
+ * spot.h -- C ABI of the B200 (sm_100a) SpotAttention decode-path library.
+ *
+ * The operations follow "SpotAttention: Plug-In Block-Sparse Routing for
+ * Pretrained Long-Context Transformers" (arXiv HTML):
+ *   - selector score, §2.1:  s[q,t] = sum_h w_h ReLU(q^I_h . k^I_{h,t});
+ *   - block-wise scoring and selection modes, §2.3: block score = max over
+ *     the block's keys, static top-K (Eq. 6), residual softmax (Eq. 7) and
+ *     dual top-p with reserved sink / recency blocks and a K_min floor
+ *     (Eq. 8); softmax temperature 1.0 by default (App. A, Tab. 3);
+ *   - sparse attention: the layer attends only to the keys of the selected
+ *     blocks, at decode only (§2.3, §3 "Evaluation");
+ *   - selector K-cache stored in bf16, INT4 or FP4 group-32 microscale
+ *     (§5.3, App. G Tab. 9).
+ *
+ * Conventions for every call:
+ *   - All array arguments are DEVICE pointers of the current CUDA device,
+ *     owned by the caller; the library allocates no memory and keeps no
+ *     state between calls except a per-device cache of kernel attributes.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Return codes report argument errors detected on the
+ *     host and launch errors; errors detected by a kernel (an out-of-range
+ *     page id or block index, a wait that ran out of time) are OR-ed into a
+ *     status word inside the workspace and read with
+ *     spot_read_device_status().  Kernels never trap: a bad index is
+ *     recorded and the access is skipped.
+ *   - Shapes this build supports: head_dim 128, block_size 64 (one KV page
+ *     per block), sel_dim 64, 1 <= num_q_heads / num_kv_heads <= 8,
+ *     batch * num_kv_heads <= 4096, max_blocks <= 16384.  Other shapes
+ *     return SPOT_ERR_UNSUPPORTED.
+ *   - Alignment: bf16 arrays and the selector data plane 16 bytes, the KV
+ *     pools and the workspace 256 bytes, everything else 4 bytes.
+ *
+ * Layouts (row-major, innermost last):
+ *   q            bf16  [batch][num_q_heads][head_dim]
+ *   q_sel        bf16  [batch][num_q_heads][sel_dim]
+ *   w            fp32  [batch][num_q_heads]          (NULL: 1/G for all)
+ *   k_pool/v_pool bf16 [num_pages][num_kv_heads][block_size][head_dim]
+ *   sel_data     bf16  [num_pages][num_kv_heads][sel_dim]         (BF16)
+ *                u8    [num_pages][num_kv_heads][sel_dim/2]       (INT4, MXFP4)
+ *                      two elements per byte, even element in the low nibble
+ *   sel_scales   fp16  [num_pages][num_kv_heads][sel_dim/32]      (INT4)
+ *                u8    [num_pages][num_kv_heads][sel_dim/32]      (MXFP4, E8M0)
+ *                      unused (may be NULL) for BF16
+ *   page_table   int32 [batch][pt_stride]: logical block j of sequence b is
+ *                      pool page page_table[b*pt_stride + j] in the KV pools
+ *                      and in the selector pool alike
+ *   seq_lens     int32 [batch]: tokens in the cache, the current one included;
+ *                      nb(b) = ceil(seq_lens[b] / block_size) blocks
+ *   sel_idx      int32 [batch][num_kv_heads][max_blocks]: selected logical
+ *                      blocks, ascending, first sel_cnt entries valid
+ *   sel_cnt      int32 [batch][num_kv_heads]
+ *   out          fp32  [batch][num_q_heads][head_dim]
+ *   lse          fp32  [batch][num_q_heads]  natural-log softmax denominator
+ *                      of the scaled logits (NULL: not written)
+ *
+ * Query head h belongs to KV head h / G, G = num_q_heads / num_kv_heads.
+ * Selection is per (sequence, KV head): the G query heads of a group are the
+ * selector's index heads and share one selector key per block.
+ */
+#ifndef SPOT_H_
+#define SPOT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPOT_OK = 0,
+    SPOT_ERR_INVALID_ARG = 1,     /* null / misaligned pointer, bad size or parameter */
+    SPOT_ERR_UNSUPPORTED = 2,     /* shape outside what this build implements */
+    SPOT_ERR_WORKSPACE = 3,       /* workspace smaller than spot_workspace_size() */
+    SPOT_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+    SPOT_ERR_DEVICE_BOUNDS = 5,   /* a kernel met an out-of-range page id / block index */
+    SPOT_ERR_DEVICE_TIMEOUT = 6   /* a kernel's bounded wait ran out */
+} spot_status_t;
+
+/* Selector K-cache storage (§5.3, App. G). */
+typedef enum {
+    SPOT_SEL_BF16 = 0,            /* bf16 keys */
+    SPOT_SEL_INT4_G32_F16 = 1,    /* int4 codes, one fp16 scale per 32 (symmetric) */
+    SPOT_SEL_MXFP4_G32_E8M0 = 2   /* OCP MX v1.0 MXFP4: E2M1 codes, one E8M0 per 32 */
+} spot_sel_fmt_t;
+
+/* Selection rule (§2.3). */
+typedef enum {
+    SPOT_MODE_TOPP = 0,           /* dual top-p, Eq. 7-8 */
+    SPOT_MODE_TOPK = 1            /* static top-K, Eq. 6 (after the reserved blocks) */
+} spot_select_mode_t;
+
+typedef struct {
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;             /* 128 */
+    int32_t block_size;           /* 64 tokens per block and per KV page */
+    int32_t sel_dim;              /* 64 */
+    int32_t sel_fmt;              /* spot_sel_fmt_t */
+    int32_t num_pages;            /* pages in the KV and selector pools */
+} spot_layer_desc_t;
+
+typedef struct {
+    int32_t mode;                 /* spot_select_mode_t */
+    int32_t sink_blocks;          /* first blocks always kept (S_sink) */
+    int32_t recency_blocks;       /* last blocks always kept (S_rec); an incomplete
+                                     last block is always kept as well */
+    int32_t kmin_blocks;          /* |S| >= min(K_min, nb) in TOPP mode */
+    int32_t topk_blocks;          /* residual blocks kept in TOPK mode */
+    float temperature;            /* scores are divided by it; > 0 */
+} spot_select_params_t;
+
+/* Bytes of scratch the select / sparse-decode / decode-step calls need for
+ * this shape on the CURRENT device (it depends on the SM count).  The first
+ * 256 bytes hold the device status word: zero them once before first use
+ * (e.g. allocate the workspace zero-filled).  Returns 0 for a shape this
+ * build does not support. */
+size_t spot_workspace_size(const spot_layer_desc_t* desc, int32_t batch, int32_t max_blocks);
+
+/* Append (write, quantising if the format asks) one selector key per
+ * (entry, KV head) into the selector pool: entry i stores
+ * keys[i][g][0..sel_dim) for block block_ids[i] of sequence seq_ids[i] at
+ * page page_table[seq_ids[i]*pt_stride + block_ids[i]] (page_table has
+ * num_seqs rows).
+ *   keys bf16 [n][num_kv_heads][sel_dim]; seq_ids, block_ids int32 [n].
+ * INT4:  scale = fp16 round-to-nearest-even of amax/7 over each 32
+ *        elements (saturating at 65504), code = clamp(rne(x/scale), -8, 7).
+ * MXFP4: shared exponent X = floor(log2 amax) - 2 clamped to [-127, 127],
+ *        stored as X + 127; elements rounded to nearest even on the E2M1
+ *        grid, saturating at 6; sign bit set for x < 0.
+ * Cites §5.3 and App. G (group-32 INT4 / FP4 microscale selector K-cache).
+ * Entries whose sequence, block or page id is out of range are skipped and
+ * recorded in the status word of `status_ws` (a workspace, may be NULL: not
+ * recorded). */
+spot_status_t spot_append_selector_keys(const spot_layer_desc_t* desc, void* sel_data,
+                                        void* sel_scales, const int32_t* page_table,
+                                        int32_t num_seqs, int32_t pt_stride,
+                                        const int32_t* seq_ids, const int32_t* block_ids,
+                                        const uint16_t* keys, int32_t n, void* status_ws,
+                                        void* stream);
+
+/* Block selection for every (sequence, KV head) (§2.1 scoring, §2.3
+ * Eq. 6-8).  Scores every complete block of each sequence against the
+ * selector pool, then keeps the sink and recency blocks plus, in TOPP mode,
+ * the smallest prefix of the remaining blocks -- ranked by score, lower
+ * block index first on ties -- whose residual-softmax mass reaches
+ * top_p[b] (p >= 1: all of them, p <= 0: none), extended along the same
+ * ranking until |S| >= min(kmin_blocks, nb); in TOPK mode the prefix holds
+ * topk_blocks blocks.  Writes sel_idx (ascending) and sel_cnt.
+ * top_p: fp32 [batch] (may be NULL in TOPK mode).  Requires
+ * max_blocks >= nb(b) and pt_stride >= nb(b) for every b (checked on the
+ * device: violations are recorded and the sequence is truncated). */
+spot_status_t spot_select(const spot_layer_desc_t* desc, const spot_select_params_t* params,
+                          const uint16_t* q_sel, const float* w, const void* sel_data,
+                          const void* sel_scales, const int32_t* page_table, int32_t pt_stride,
+                          const int32_t* seq_lens, const float* top_p, int32_t batch,
+                          int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* Exact softmax attention of each query head over only the tokens of the
+ * selected blocks of its KV head (§2.3): for head h of KV head g,
+ *   out[b][h] = sum_t softmax_t(softmax_scale * q[b][h] . K_t) V_t
+ * over the positions t < seq_lens[b] of the blocks sel_idx[b][g][0..cnt).
+ * A (sequence, KV head) with no selected token gets out = 0, lse = -inf.
+ * Selected block ids must lie in [0, nb(b)) and be distinct; an
+ * out-of-range id or page is recorded in the status word and skipped. */
+spot_status_t spot_sparse_decode(const spot_layer_desc_t* desc, const uint16_t* q,
+                                 const uint16_t* k_pool, const uint16_t* v_pool,
+                                 const int32_t* page_table, int32_t pt_stride,
+                                 const int32_t* seq_lens, const int32_t* sel_idx,
+                                 const int32_t* sel_cnt, int32_t max_blocks, int32_t batch,
+                                 float softmax_scale, float* out, float* lse, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
+/* One decode step of a sparse layer: spot_select followed by
+ * spot_sparse_decode on the same stream and workspace; sel_idx / sel_cnt
+ * receive the selection. */
+spot_status_t spot_decode_step(const spot_layer_desc_t* desc, const spot_select_params_t* params,
+                               const uint16_t* q_sel, const float* w, const void* sel_data,
+                               const void* sel_scales, const uint16_t* q, const uint16_t* k_pool,
+                               const uint16_t* v_pool, const int32_t* page_table,
+                               int32_t pt_stride, const int32_t* seq_lens, const float* top_p,
+                               int32_t batch, float softmax_scale, int32_t* sel_idx,
+                               int32_t* sel_cnt, int32_t max_blocks, float* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, return the status recorded by kernels in
+ * `workspace` since the last read (SPOT_OK, SPOT_ERR_DEVICE_BOUNDS or
+ * SPOT_ERR_DEVICE_TIMEOUT; bounds wins if both), and clear it. */
+spot_status_t spot_read_device_status(void* workspace, void* stream);
+
+/* Static string for a status code. */
+const char* spot_status_string(spot_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPOT_H_ */

@@ -1,0 +1,223 @@
+"""Shared helpers of the GPU parity tests: run a workload through the CUDA
+library (C ABI via the Python binding) and through the fp64 oracle, and
+compare them under the parity rules.
+
+Parity rules (tolerances of the bf16-in / fp32-accumulate path):
+  * selection: on integer-valued inputs the selected sets must be identical;
+    on real-valued inputs every block whose oracle score lies more than 1e-6
+    (relative) from the cut -- the lowest score the oracle kept in the
+    nucleus -- must be treated identically, and any differing block must
+    leave the GPU's set valid in fp64: nucleus mass >= p - 1e-5 and the mass
+    without its lowest-ranked block < p + 1e-5;
+  * attention outputs: |gpu - oracle| <= 2e-3 + 1e-2 |oracle| element-wise,
+    for every (sequence, KV head) whose selection matches exactly.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import block_sparse_long_spot_b200 as spot
+import oracle
+import workloads
+
+ATOL, RTOL = 2e-3, 1e-2
+CUT_REL = 1e-6
+MASS_TOL = 1e-5
+
+
+def gpu_selector_pool(wl, fmt, device):
+    """Selector pool in `fmt`, written by the library's append kernel."""
+    data, scales = spot.selector_pool(fmt, wl.num_pages, wl.num_kv_heads, device=device)
+    pt = wl.page_table
+    lens = wl.seq_lens.cpu().numpy()
+    seq_ids, blk_ids, pages = [], [], []
+    ptn = pt.cpu().numpy()
+    for b in range(wl.batch):
+        nb = int(lens[b]) // 64               # complete blocks carry keys
+        seq_ids += [b] * nb
+        blk_ids += list(range(nb))
+        pages += ptn[b, :nb].tolist()
+    if seq_ids:
+        keys = wl.sel_keys[torch.as_tensor(pages, device=device).long()].contiguous()
+        desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, fmt)
+        spot.append_selector_keys(desc, data, scales, pt,
+                                  torch.as_tensor(seq_ids, dtype=torch.int32, device=device),
+                                  torch.as_tensor(blk_ids, dtype=torch.int32, device=device), keys)
+    return data, scales
+
+
+def oracle_selector_pool(wl, fmt):
+    return oracle.quantize_selector(fmt, workloads.bits(wl.sel_keys))
+
+
+def host_bytes(t):
+    if t is None:
+        return None
+    t = t.detach().contiguous().cpu()
+    if t.dtype in (torch.bfloat16, torch.float16):
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def run_gpu(wl, fmt="bf16", mode="topp", kmin=None, topk=0, sink=None, rec=None,
+            temperature=1.0, pool=None, max_blocks=None):
+    dev = wl.q.device
+    B, Hq, Hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
+    mb = wl.max_blocks if max_blocks is None else max_blocks
+    desc = spot.layer_desc(Hq, Hkv, wl.num_pages, fmt)
+    prm = spot.select_params(mode, wl.spec.sink_blocks if sink is None else sink,
+                             wl.spec.recency_blocks if rec is None else rec,
+                             wl.spec.kmin_blocks if kmin is None else kmin, topk, temperature)
+    data, scales = pool if pool is not None else gpu_selector_pool(wl, fmt, dev)
+    ws = spot.new_workspace(desc, B, mb, dev)
+    sel_idx = torch.full((B, Hkv, mb), -1, dtype=torch.int32, device=dev)
+    sel_cnt = torch.full((B, Hkv), -1, dtype=torch.int32, device=dev)
+    out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
+    spot.decode_step(desc, prm, wl.q_sel, wl.w, data, scales, wl.q, wl.k_pool, wl.v_pool,
+                     wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt, out, lse,
+                     ws)
+    torch.cuda.synchronize()
+    status = spot.read_device_status(ws)
+    return {"sel_idx": sel_idx.cpu().numpy(), "sel_cnt": sel_cnt.cpu().numpy(),
+            "out": out.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
+            "status": status, "pool": (data, scales)}
+
+
+def oracle_args(wl, fmt="bf16"):
+    data, scales = oracle_selector_pool(wl, fmt)
+    return dict(q_sel=workloads.bits(wl.q_sel), w=host_bytes(wl.w), sel_data=data,
+                sel_scales=scales, q=workloads.bits(wl.q), k_pool=workloads.bits(wl.k_pool),
+                v_pool=workloads.bits(wl.v_pool), page_table=wl.page_table.cpu().numpy(),
+                seq_lens=wl.seq_lens.cpu().numpy(), top_p=wl.top_p.cpu().numpy(),
+                sm_scale=wl.sm_scale)
+
+
+def oracle_shape_params(wl, fmt="bf16", mode="topp", kmin=None, topk=0, sink=None, rec=None,
+                        temperature=1.0, max_blocks=None):
+    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, fmt,
+                           wl.num_pages, wl.max_blocks if max_blocks is None else max_blocks)
+    pr = oracle.make_params(mode, wl.spec.sink_blocks if sink is None else sink,
+                            wl.spec.recency_blocks if rec is None else rec,
+                            wl.spec.kmin_blocks if kmin is None else kmin, topk, temperature)
+    return sh, pr
+
+
+def run_oracle(wl, fmt="bf16", units=None, args=None, **kw):
+    sh, pr = oracle_shape_params(wl, fmt, **kw)
+    a = args or oracle_args(wl, fmt)
+    if kw.get("max_blocks") is not None and kw["max_blocks"] != wl.max_blocks:
+        pt = np.full((wl.batch, kw["max_blocks"]), -1, np.int32)
+        pt[:, :wl.max_blocks] = a["page_table"]
+        a = dict(a, page_table=pt)
+    return oracle.decode_step(sh, pr, units=units, **a)
+
+
+def oracle_scores(wl, fmt="bf16", args=None, **kw):
+    sh, pr = oracle_shape_params(wl, fmt, **kw)
+    a = args or oracle_args(wl, fmt)
+    return oracle.block_scores(sh, pr, a["q_sel"], a["w"], a["sel_data"], a["sel_scales"],
+                               a["page_table"], a["seq_lens"])
+
+
+def unit_selection(res, b, g):
+    return res["sel_idx"][b, g, :res["sel_cnt"][b, g]].tolist()
+
+
+def check_selection_near_cut(gpu, ora, scores, wl, kmin=None, sink=None, rec=None):
+    """Apply the real-valued selection rule to every unit; return the number
+    of (sequence, KV head) units whose sets differ (all near the cut)."""
+    kmin = wl.spec.kmin_blocks if kmin is None else kmin
+    sink = wl.spec.sink_blocks if sink is None else sink
+    rec = wl.spec.recency_blocks if rec is None else rec
+    lens = wl.seq_lens.cpu().numpy()
+    p_all = wl.top_p.cpu().numpy()
+    n_diff = 0
+    for b in range(wl.batch):
+        L = int(lens[b])
+        nb, n_full = (L + 63) // 64, L // 64
+        r_eff = min(max(rec, nb - n_full), nb)
+        s_eff = min(sink, nb)
+        reserved = set(range(s_eff)) | set(range(nb - r_eff, nb))
+        res = [j for j in range(nb) if j not in reserved]
+        for g in range(wl.num_kv_heads):
+            sg, so = set(unit_selection(gpu, b, g)), set(unit_selection(ora, b, g))
+            assert reserved <= sg, (b, g)
+            if sg == so:
+                continue
+            n_diff += 1
+            s = scores[b, g]
+            nuc_o = so - reserved
+            assert nuc_o, (b, g)
+            cut = min(s[j] for j in nuc_o)
+            for j in sg ^ so:
+                assert j in res, (b, g, j)
+                assert abs(s[j] - cut) <= CUT_REL * abs(cut) + 1e-12, (b, g, j, s[j], cut)
+            # the GPU set is itself a valid nucleus in fp64
+            sr = np.array([s[j] for j in res])
+            e = np.exp(sr - sr.max())
+            e /= e.sum()
+            mass = {j: e[i] for i, j in enumerate(res)}
+            nuc_g = sorted(sg - reserved, key=lambda j: (-s[j], j))
+            if len(nuc_g) > max(kmin - len(reserved), 0):
+                m_g = sum(mass[j] for j in nuc_g)
+                p = float(p_all[b])
+                assert m_g >= p - MASS_TOL, (b, g, m_g, p)
+                assert m_g - mass[nuc_g[-1]] < p + MASS_TOL, (b, g, m_g, p)
+    return n_diff
+
+
+def check_outputs(gpu, ora, wl, units=None):
+    """Element-wise output check on units whose selections agree; returns
+    (max abs err, max rel err, units compared)."""
+    G = wl.num_q_heads // wl.num_kv_heads
+    if units is None:
+        units = [(b, g) for b in range(wl.batch) for g in range(wl.num_kv_heads)]
+    worst_a, worst_r, n = 0.0, 0.0, 0
+    for b, g in units:
+        if unit_selection(gpu, b, g) != unit_selection(ora, b, g):
+            continue
+        o_g = gpu["out"][b, g * G:(g + 1) * G]
+        o_r = ora["out"][b, g * G:(g + 1) * G]
+        err = np.abs(o_g - o_r)
+        bad = err > ATOL + RTOL * np.abs(o_r)
+        assert not bad.any(), (b, g, float(err.max()))
+        l_g = gpu["lse"][b, g * G:(g + 1) * G]
+        l_r = ora["lse"][b, g * G:(g + 1) * G]
+        fin = np.isfinite(l_r)
+        assert np.array_equal(fin, np.isfinite(l_g)), (b, g)
+        assert (np.abs(l_g[fin] - l_r[fin]) <= ATOL + RTOL * np.abs(l_r[fin])).all(), (b, g)
+        worst_a = max(worst_a, float(err.max()))
+        worst_r = max(worst_r, float((err / np.maximum(np.abs(o_r), 1e-3)).max()))
+        n += 1
+    return worst_a, worst_r, n
+
+
+def safe_top_p(wl, fmt="bf16", lo=0.5, hi=0.99, margin=2e-5, **kw):
+    """Per-sequence p values at least `margin` away from every cumulative
+    residual mass of every KV head of that sequence (from the oracle's own
+    scores), so the nucleus size is decided far from the fp boundary."""
+    scores = oracle_scores(wl, fmt, **kw)
+    lens = wl.seq_lens.cpu().numpy()
+    sink, rec = wl.spec.sink_blocks, wl.spec.recency_blocks
+    ps = []
+    for b in range(wl.batch):
+        nb, n_full = (int(lens[b]) + 63) // 64, int(lens[b]) // 64
+        r_eff = min(max(rec, nb - n_full), nb)
+        res = list(range(min(sink, nb), max(min(sink, nb), nb - r_eff)))
+        cums = [lo, hi]
+        for g in range(wl.num_kv_heads):
+            s = np.array([scores[b, g, j] for j in res])
+            if s.size == 0:
+                continue
+            order = sorted(range(len(res)), key=lambda i: (-s[i], res[i]))
+            e = np.exp(s - s.max())
+            e /= e.sum()
+            cums += np.cumsum(e[order]).tolist()
+        c = np.unique(np.clip(np.array(cums), lo, hi))
+        gaps = np.diff(c)
+        k = int(np.argmax(gaps))
+        assert gaps[k] > 2 * margin
+        ps.append(0.5 * (c[k] + c[k + 1]))
+    return torch.as_tensor(np.array(ps, np.float32), device=wl.top_p.device)
