@@ -1,0 +1,434 @@
+"""Benchmark of the SpotAttention decode hot path on B200.
+
+One step = one decode step of one sparse attention layer for the whole batch:
+selector scoring, residual softmax and dual top-p selection, then exact
+attention over the selected KV blocks (spot_select + spot_sparse_decode,
+i.e. spot_decode_step).  Steps rotate over several independent layer caches
+(each far larger than the 126 MB L2), so every step reads its KV from HBM.
+
+Default workload: the Qwen3-32B-shaped layer at L = 131072 (batch 4, 64 query
+/ 8 KV heads, head_dim 128, blocks of 64, bf16 selector keys, top-p 0.95).
+Reported: decode tokens/s for the whole model (per-layer time x 64 layers),
+us per layer, and the HBM roofline fraction of the sparse-attention kernels
+and of the whole step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spot|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch
+(data parallel over sequences, no collective on the data path); the time is
+the max over ranks and `value` counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+HBM_FALLBACK_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def unit_counts(wl):
+    lens = wl.seq_lens.cpu().numpy().astype(np.int64)
+    return (lens + 63) // 64, lens // 64
+
+
+def step_bytes(wl, sel_cnt: np.ndarray, fmt: str):
+    """Algorithmic HBM bytes of one decode step and of its sparse-attention
+    part, from the selection actually made."""
+    B, Hq, Hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
+    lens = wl.seq_lens.cpu().numpy().astype(np.int64)
+    nb, n_full = unit_counts(wl)
+    key_bytes = {"bf16": 128, "int4": 32 + 4, "mxfp4": 32 + 2}[fmt]
+    sel_cache = int(Hkv * n_full.sum() * key_bytes)
+    # tokens attended per (b, g): full blocks, the last one possibly partial
+    kv = 0
+    for b in range(B):
+        for g in range(Hkv):
+            c = int(sel_cnt[b, g])
+            kv += c * 64 * 128 * 2 * 2
+    part = (lens % 64 != 0)
+    # a partial last block is always selected: subtract its missing tokens
+    kv -= int((Hkv * (64 - lens[part] % 64) * 128 * 2 * 2).sum())
+    idx = int(sel_cnt.sum()) * 4 * 2          # selected list + page-table entry per block
+    q_io = B * Hq * (128 * 2 + 128 * 4 + 4) + B * Hkv * 4
+    sparse = kv + idx + q_io
+    select = sel_cache + B * Hq * 64 * 2 + int(n_full.sum()) * 4 + int(sel_cnt.sum()) * 4
+    return {"sparse": sparse, "select": select, "step": sparse + select, "kv": kv,
+            "selector": sel_cache}
+
+
+def run_spot(args, world, rank, local):
+    import block_sparse_long_spot_b200 as spot
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    fmt = args.sel_fmt
+    layers = []
+    for l in range(args.layers):
+        wl = workloads.make(args.workload, seed=1000 * rank + l, device=dev, sel_fmt=fmt)
+        desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, fmt)
+        if fmt == "bf16":
+            data, scales = wl.sel_keys, None
+        else:
+            data, scales = spot.selector_pool(fmt, wl.num_pages, wl.num_kv_heads, device=dev)
+            nb, n_full = unit_counts(wl)
+            seq = np.concatenate([np.full(n, b) for b, n in enumerate(n_full)]).astype(np.int32)
+            blk = np.concatenate([np.arange(n) for n in n_full]).astype(np.int32)
+            pages = wl.page_table.cpu().numpy()[seq, blk]
+            spot.append_selector_keys(desc, data, scales, wl.page_table,
+                                      torch.as_tensor(seq, device=dev),
+                                      torch.as_tensor(blk, device=dev),
+                                      wl.sel_keys[torch.as_tensor(pages, device=dev).long()])
+        layers.append((wl, desc, data, scales))
+    wl0, desc0 = layers[0][0], layers[0][1]
+    B, Hq, Hkv, mb = wl0.batch, wl0.num_q_heads, wl0.num_kv_heads, wl0.max_blocks
+    prm = spot.select_params("topp", wl0.spec.sink_blocks, wl0.spec.recency_blocks,
+                             wl0.spec.kmin_blocks)
+    ws = spot.new_workspace(desc0, B, mb, dev)
+    sel_idx = torch.empty(B, Hkv, mb, dtype=torch.int32, device=dev)
+    sel_cnt = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        wl, desc, data, scales = layers[i % len(layers)]
+        if ev is not None:
+            ev[0].record(stream)
+        spot.select(desc, prm, wl.q_sel, wl.w, data, scales, wl.page_table, wl.seq_lens,
+                    wl.top_p, sel_idx, sel_cnt, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        spot.sparse_decode(desc, wl.q, wl.k_pool, wl.v_pool, wl.page_table, wl.seq_lens, sel_idx,
+                           sel_cnt, wl.sm_scale, out, lse, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    # selection statistics and algorithmic bytes per layer
+    per_layer = []
+    for l in range(len(layers)):
+        step(l)
+        torch.cuda.synchronize()
+        cnt = sel_cnt.cpu().numpy().copy()
+        wl = layers[l][0]
+        nb, _ = unit_counts(wl)
+        per_layer.append((step_bytes(wl, cnt, fmt), cnt / np.maximum(nb[:, None], 1)))
+    status = spot.read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t0.record(stream)
+        for i in range(K):
+            step(i, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = t0.elapsed_time(t1)
+    ms_sel = [e[0].elapsed_time(e[1]) for e in evs]
+    ms_dec = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_step = max_over_ranks(ms_total / K, world)
+
+    # ---- end to end through the public call with host buffers
+    pin_q = [layers[l][0].q.cpu().pin_memory() for l in range(len(layers))]
+    pin_qs = [layers[l][0].q_sel.cpu().pin_memory() for l in range(len(layers))]
+    host_out = torch.empty(B, Hq, 128, dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(layers[0][0].q)
+    qs_dev = torch.empty_like(layers[0][0].q_sel)
+
+    def e2e_step(i):
+        wl, desc, data, scales = layers[i % len(layers)]
+        q_dev.copy_(pin_q[i % len(layers)], non_blocking=True)
+        qs_dev.copy_(pin_qs[i % len(layers)], non_blocking=True)
+        spot.decode_step(desc, prm, qs_dev, wl.w, data, scales, q_dev, wl.k_pool, wl.v_pool,
+                         wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt,
+                         out, lse, ws, stream)
+        host_out.copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K, world)
+    status = spot.read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after timing")
+
+    nl = len(layers)
+    b_sparse = np.mean([per_layer[i % nl][0]["sparse"] for i in range(K)])
+    b_step = np.mean([per_layer[i % nl][0]["step"] for i in range(K)])
+    frac_sel = np.concatenate([x[1].ravel() for x in per_layer])
+    dec_ms = float(np.mean(ms_dec))
+    sel_ms = float(np.mean(ms_sel))
+    peak, peak_kind = peaks()
+    layers_model = wl0.spec.layers_sparse
+    tokens_per_step = B * world
+    value = tokens_per_step / (ms_step / 1e3 * layers_model)
+    value_e2e = tokens_per_step / (ms_e2e / 1e3 * layers_model)
+    achieved = b_sparse / (dec_ms / 1e3) / 1e9
+    res = {
+        "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
+        "value": round(value, 3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "us_per_layer": round(ms_step * 1e3, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 with planted hot blocks)",
+        "config": {
+            "workload": args.workload, "batch_per_gpu": B, "q_heads": Hq, "kv_heads": Hkv,
+            "head_dim": 128, "context": int(wl0.seq_lens.max().item()), "block": 64,
+            "sel_fmt": fmt, "top_p": float(wl0.top_p[0].item()),
+            "sink_blocks": wl0.spec.sink_blocks, "recency_blocks": wl0.spec.recency_blocks,
+            "kmin_blocks": wl0.spec.kmin_blocks, "layers_in_model": layers_model,
+            "layer_caches_rotated": nl,
+            "l2": f"inputs larger than L2: {nl} layer caches of "
+                  f"{wl0.k_pool.numel() * 4 / 1e9:.2f} GB rotated per step",
+            "selected_fraction": {"mean": round(float(frac_sel.mean()), 4),
+                                  "min": round(float(frac_sel.min()), 4),
+                                  "max": round(float(frac_sel.max()), 4)},
+            "parallelism": f"dp{world} (sequences)",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "sparse decode (attention + combine)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": peak_kind,
+            "algorithmic_bytes_per_launch": int(b_sparse), "ms_per_launch": round(dec_ms, 5),
+        },
+        "step_roofline": {
+            "achieved": round(b_step / (ms_step / 1e3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(b_step / (ms_step / 1e3) / 1e9 / peak, 4),
+            "algorithmic_bytes_per_step": int(b_step),
+            "select_ms": round(sel_ms, 5),
+        },
+        "e2e": {"value": round(value_e2e, 3), "unit": "tokens/s",
+                "ms_per_step": round(ms_e2e, 5),
+                "h2d_bytes_per_step": int(layers[0][0].q.numel() * 2 + layers[0][0].q_sel.numel() * 2),
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": K * 4,
+        "clocks": clk.summary(),
+    }
+    return res, layers
+
+
+def oracle_sample(wl, fmt, seqs):
+    """Time the fp64 oracle on the sequences `seqs` of a layer (host cores)."""
+    import oracle
+    sub = workloads.gather_units(wl, seqs)
+    data, scales = oracle.quantize_selector(fmt, workloads.bits(sub.sel_keys))
+    sh = oracle.make_shape(sub.batch, sub.num_q_heads, sub.num_kv_heads, 128, 64, 64, fmt,
+                           sub.num_pages, sub.max_blocks)
+    pr = oracle.make_params(sink_blocks=sub.spec.sink_blocks,
+                            recency_blocks=sub.spec.recency_blocks,
+                            kmin_blocks=sub.spec.kmin_blocks)
+    args = dict(q_sel=workloads.bits(sub.q_sel), w=None, sel_data=data, sel_scales=scales,
+                q=workloads.bits(sub.q), k_pool=workloads.bits(sub.k_pool),
+                v_pool=workloads.bits(sub.v_pool), page_table=sub.page_table.cpu().numpy(),
+                seq_lens=sub.seq_lens.cpu().numpy(), top_p=sub.top_p.cpu().numpy(),
+                sm_scale=sub.sm_scale)
+    t = time.perf_counter()
+    oracle.decode_step(sh, pr, **args)
+    return time.perf_counter() - t, oracle.num_threads()
+
+
+def cpu_baseline(wl, fmt, n_seqs=1):
+    sec, cores = oracle_sample(wl, fmt, list(range(n_seqs)))
+    per_layer = sec * wl.batch / n_seqs
+    value = wl.batch / (per_layer * wl.spec.layers_sparse)
+    return {"value": round(value, 6), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle decode step of {n_seqs} of {wl.batch} sequences "
+                      f"(all {wl.num_kv_heads} KV heads) of one layer, {sec:.2f} s wall; "
+                      f"scaled x{wl.batch // n_seqs} to the layer and x{wl.spec.layers_sparse} "
+                      f"layers"}
+
+
+def run_reference(args, world, rank):
+    """The fp64 CPU oracle as the reference arm, on the same workload."""
+    if rank != 0:
+        return None
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = workloads.make(args.workload, seed=0, device=dev, sel_fmt=args.sel_fmt)
+    times = []
+    cores = 1
+    for i in range(args.warmup + args.steps):
+        sec, cores = oracle_sample(wl, args.sel_fmt, [i % wl.batch])
+        if i >= args.warmup:
+            times.append(sec * wl.batch)            # one layer = batch x one sequence
+    per_layer = float(np.mean(times))
+    value = wl.batch / (per_layer * wl.spec.layers_sparse)
+    return {
+        "impl": "reference",
+        "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
+        "value": round(value, 6), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_layer * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 with planted hot blocks)",
+        "config": {"workload": args.workload, "sel_fmt": args.sel_fmt,
+                   "sample": "each step times one sequence of the layer and scales by batch"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": "one sequence (all KV heads) of the layer per step, x batch"},
+        "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="spot", choices=["spot", "reference"])
+    ap.add_argument("--workload", default="qwen3_32b_128k")
+    ap.add_argument("--sel-fmt", default=None)
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.sel_fmt is None:
+        args.sel_fmt = workloads.SPECS[args.workload].sel_fmt
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            if world > 1:
+                torch.distributed.barrier()
+            res = run_reference(args, world, rank)
+            if res is not None:
+                print(json.dumps(res), flush=True)
+            return
+        res, layers = run_spot(args, world, rank, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(layers[0][0], args.sel_fmt)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

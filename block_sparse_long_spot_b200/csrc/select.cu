@@ -446,7 +446,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
         }
         kept += keep;
     }
-    int out_pos = block_exclusive_scan<NT>(kept, scan, &total);
+    int n_sel;
+    int out_pos = block_exclusive_scan<NT>(kept, scan, &n_sel);
     tie_rank = block_exclusive_scan<NT>(ties, scan, &total);
     int32_t* out = p.sel_idx + static_cast<int64_t>(u) * p.max_blocks;
     for (int j = lo; j < hi; ++j) {
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
         }
         if (keep) out[out_pos++] = j;
     }
-    if (threadIdx.x == 0) p.sel_cnt[u] = total;
+    if (threadIdx.x == 0) p.sel_cnt[u] = n_sel;
 }
 
 }  // namespace
