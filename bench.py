@@ -124,11 +124,23 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank timing over all ranks (the only cross-rank traffic)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def layer_seed(rank: int, layer: int) -> int:
+    """Seed of a rank's layer cache: every rank decodes its own sequences."""
+    return 1000 * rank + layer
+
+
+def shard_summary(batch_per_rank: int, world: int, ms_step_max: float, layers_model: int):
+    """Whole-job decode throughput: tokens of all ranks over the slowest rank."""
+    return batch_per_rank * world / (ms_step_max / 1e3 * layers_model)
 
 
 def unit_counts(wl):
@@ -168,7 +180,7 @@ def run_spot(args, world, rank, local):
     fmt = args.sel_fmt
     layers = []
     for l in range(args.layers):
-        wl = workloads.make(args.workload, seed=1000 * rank + l, device=dev, sel_fmt=fmt)
+        wl = workloads.make(args.workload, seed=layer_seed(rank, l), device=dev, sel_fmt=fmt)
         desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, fmt)
         if fmt == "bf16":
             data, scales = wl.sel_keys, None
@@ -280,9 +292,8 @@ def run_spot(args, world, rank, local):
     sel_ms = float(np.mean(ms_sel))
     peak, peak_kind = peaks()
     layers_model = wl0.spec.layers_sparse
-    tokens_per_step = B * world
-    value = tokens_per_step / (ms_step / 1e3 * layers_model)
-    value_e2e = tokens_per_step / (ms_e2e / 1e3 * layers_model)
+    value = shard_summary(B, world, ms_step, layers_model)
+    value_e2e = shard_summary(B, world, ms_e2e, layers_model)
     achieved = b_sparse / (dec_ms / 1e3) / 1e9
     res = {
         "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
