@@ -79,10 +79,13 @@ def lib():
                                          P]
         L.spot_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, P, P, i32, f32, P, P,
                                        i32, P, P, P, sz, P]
+        L.spot_sparse_decode_noalloc.argtypes = [P, P, P, P, P, i32, P, P, P, i32, i32, f32, P,
+                                                 P, P]
         L.spot_read_device_status.argtypes = [P, P]
         L.spot_status_string.restype = ctypes.c_char_p
         for name in ("spot_append_selector_keys", "spot_select", "spot_sparse_decode",
-                     "spot_decode_step", "spot_read_device_status"):
+                     "spot_decode_step", "spot_read_device_status",
+                     "spot_sparse_decode_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -164,6 +167,24 @@ def sparse_decode(desc: LayerDesc, q, k_pool, v_pool, page_table, seq_lens, sel_
         _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check(code, "sparse_decode")
+
+
+def sparse_decode_noalloc(desc: LayerDesc, q, k_pool, v_pool, page_table, seq_lens, sel_idx,
+                          sel_cnt, softmax_scale, out, lse, stream=None):
+    """sparse_decode without a workspace, for callers that cannot allocate
+    device memory: the scratch is an 8 MiB array inside the library, shared
+    by all calls (calls that overlap on the GPU race).  Shapes needing more
+    raise SpotError(3).  Make the first call on a device before any stream
+    capture."""
+    B, max_blocks = int(q.shape[0]), int(sel_idx.shape[-1])
+    code = lib().spot_sparse_decode_noalloc(
+        ctypes.byref(desc), _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
+        _ptr(v_pool, torch.bfloat16, "v_pool"), _ptr(page_table, torch.int32, "page_table"),
+        int(page_table.shape[-1]), _ptr(seq_lens, torch.int32, "seq_lens"),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"), max_blocks,
+        B, float(softmax_scale), _ptr(out, torch.float32, "out"), _ptr(lse, torch.float32, "lse"),
+        _stream(stream))
+    _check(code, "sparse_decode_noalloc")
 
 
 def decode_step(desc: LayerDesc, params: SelectParams, q_sel, w, sel_data, sel_scales, q, k_pool,

@@ -185,6 +185,35 @@ spot_status_t spot_decode_step(const spot_layer_desc_t* desc, const spot_select_
                                int32_t* sel_cnt, int32_t max_blocks, float* out, float* lse,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* spot_sparse_decode for callers that cannot allocate device memory.  The
+ * paper has no counterpart of this call: it exists for callers such as a
+ * serving engine that has reserved all free HBM for its paged KV pool and
+ * forbids further cudaMalloc calls, or a plugin host that passes the library
+ * the tensors of one call but no allocator, and so cannot provide the
+ * workspace spot_sparse_decode takes.
+ * Same arguments and results as spot_sparse_decode without the workspace.
+ * The scratch (status word, per-unit offsets, split partials) is a static
+ * device array of 8 MiB inside the library; every GPU that loads the library
+ * holds it until the process exits.  The call allocates nothing.
+ *   - The first call on a device looks up that array's device address with
+ *     the device current (cudaGetSymbolAddress) and remembers it; make that
+ *     first call before any stream capture.
+ *   - A shape whose scratch exceeds 8 MiB returns SPOT_ERR_WORKSPACE (about
+ *     (grid + U) * 4 * G * 520 bytes with U = batch * num_kv_heads and grid
+ *     = the SM count; e.g. 256 units of G = 4 need 3.4 MB).
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads) race
+ *     and must be serialised by the caller.
+ *   - Out-of-range page ids or block indices are skipped (not attended) as
+ *     in spot_sparse_decode, but this call cannot report them. */
+spot_status_t spot_sparse_decode_noalloc(const spot_layer_desc_t* desc, const uint16_t* q,
+                                         const uint16_t* k_pool, const uint16_t* v_pool,
+                                         const int32_t* page_table, int32_t pt_stride,
+                                         const int32_t* seq_lens, const int32_t* sel_idx,
+                                         const int32_t* sel_cnt, int32_t max_blocks,
+                                         int32_t batch, float softmax_scale, float* out,
+                                         float* lse, void* stream);
+
 /* Synchronise `stream`, return the status recorded by kernels in
  * `workspace` since the last read (SPOT_OK, SPOT_ERR_DEVICE_BOUNDS or
  * SPOT_ERR_DEVICE_TIMEOUT; bounds wins if both), and clear it. */
