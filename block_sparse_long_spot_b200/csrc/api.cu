@@ -217,7 +217,7 @@ spot_status_t check_decode_args(const uint16_t* q, const uint16_t* k_pool, const
     if (pt_stride <= 0 || !isfinite(softmax_scale)) return SPOT_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k_pool, 256) || !aligned(v_pool, 256) ||
         !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(sel_idx, 4) ||
-        !aligned(sel_cnt, 4) || !aligned(out, 4) || (lse && !aligned(lse, 4)))
+        !aligned(sel_cnt, 4) || !aligned(out, 16) || (lse && !aligned(lse, 4)))
         return SPOT_ERR_INVALID_ARG;
     return SPOT_OK;
 }

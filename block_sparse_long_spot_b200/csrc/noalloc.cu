@@ -71,7 +71,7 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
         return SPOT_ERR_INVALID_ARG;
     if (!is_aligned(q, 16) || !is_aligned(k_pool, 256) || !is_aligned(v_pool, 256) ||
         !is_aligned(page_table, 4) || !is_aligned(seq_lens, 4) || !is_aligned(sel_idx, 4) ||
-        !is_aligned(sel_cnt, 4) || !is_aligned(out, 4) || (lse && !is_aligned(lse, 4)))
+        !is_aligned(sel_cnt, 4) || !is_aligned(out, 16) || (lse && !is_aligned(lse, 4)))
         return SPOT_ERR_INVALID_ARG;
 
     // Scratch this shape needs: status word, unit offsets, split partials.

@@ -2,8 +2,9 @@
 // §2.3 Eq. 6-8).
 //
 // score_kernel: s[b,g,j] = (1/tau) sum_{h in group g} w[b,h] ReLU(q_sel[b,h] . k[page(b,j),g])
-//   for every complete block j.  One CTA per (sequence, 64 blocks); each warp
-//   takes tiles of 16 blocks of one KV head and computes the 16 x 8 dot
+//   for every complete block j.  One warp per (sequence, KV head, 16 blocks);
+//   the warps of a CTA cover adjacent KV heads of the same pages (adjacent in
+//   the selector pool).  Each warp computes the 16 x 8 dot
 //   products with bf16 mma.sync (keys as the M operand, the group's selector
 //   queries as N = 8).  INT4 / MXFP4 keys are widened to bf16 in registers
 //   (both code sets are exact in bf16) and the per-32 scales are applied to
@@ -28,8 +29,7 @@
 namespace spot {
 namespace {
 
-constexpr int kScoreWarps = 4;
-constexpr int kScoreBlocksPerCta = 64;
+constexpr int kScoreWarps = 8;
 constexpr int kSelectThreads = 512;
 constexpr int kFixShift = 40;
 
@@ -81,24 +81,23 @@ __device__ __forceinline__ float group_scale(const void* scales, int64_t row, in
 
 template <int FMT>
 __global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(const ScoreParams p) {
+    // One warp per (sequence, KV head, tile of 16 blocks): grid.x tiles,
+    // grid.y groups of kScoreWarps KV heads, grid.z sequences.
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int b = blockIdx.y;
+    const int b = blockIdx.z;
+    const int g = blockIdx.y * kScoreWarps + warp;
+    if (g >= p.num_kv_heads) return;
     const int L = max(p.seq_lens[b], 0);
     int n_full = L / kBlock;
     if (n_full > p.max_blocks || n_full > p.pt_stride) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) flag_status(p.status, kStatusBounds);
+        if (lane == 0 && blockIdx.x == 0 && g == 0) flag_status(p.status, kStatusBounds);
         n_full = min(n_full, min(p.max_blocks, p.pt_stride));
     }
-    const int j_cta = blockIdx.x * kScoreBlocksPerCta;
-    if (j_cta >= n_full) return;
+    const int j0 = blockIdx.x * 16;
+    if (j0 >= n_full) return;
     const int c4 = lane & 3, r8 = lane >> 2;
     const int G = p.group;
-    constexpr int kTiles = kScoreBlocksPerCta / 16;
-
-    for (int item = warp; item < p.num_kv_heads * kTiles; item += kScoreWarps) {
-        const int g = item / kTiles;
-        const int j0 = j_cta + (item % kTiles) * 16;
-        if (j0 >= n_full) continue;
+    {
         // ---- B operand: the group's selector queries (lane: head r8)
         const bool real = r8 < G;
         const int h = g * G + (real ? r8 : 0);
@@ -208,30 +207,39 @@ struct RadixOut {
     uint32_t above;        // elements strictly above the cut
 };
 
-// Radix search for the cut in descending key order over keys[0..n):
+// Search for the cut in descending score order over elements [0, n).
 //   by_mass: shortest prefix whose cumulative fixed-point mass is >= target;
 //   else:    prefix of exactly `target` elements (1 <= target < n).
-// Four passes of 8 key bits.  Called by every thread of the block.
-__device__ RadixOut radix_cut(const uint32_t* keys, const unsigned long long* mass, int n,
-                              unsigned long long target, bool by_mass,
-                              unsigned long long* h_mass, unsigned int* h_cnt,
+// Pass 0 buckets by the score's distance from the maximum (vbkt: 0 = the
+// top scores, monotone in the score, spreads the elements even when they
+// share their exponent bits); passes 1-4 refine the chosen bucket by the
+// 8-bit digits of the order-preserving key.  Called by every thread.
+__device__ RadixOut radix_cut(const uint32_t* keys, const uint8_t* vbkt,
+                              const unsigned long long* mass, int n, unsigned long long target,
+                              bool by_mass, unsigned long long* h_mass, unsigned int* h_cnt,
                               unsigned long long* sh) {
     uint32_t prefix = 0, pmask = 0;
+    int vsel = -1;
     unsigned long long above_mass = 0, above_cnt = 0;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int pass = 0; pass < 5; ++pass) {
+        const int shift = 32 - 8 * pass;          // key digit of passes 1..4
         for (int i = threadIdx.x; i < 256; i += blockDim.x) { h_mass[i] = 0; h_cnt[i] = 0; }
         __syncthreads();
         for (int j = threadIdx.x; j < n; j += blockDim.x) {
-            const uint32_t k = keys[j];
-            if ((k & pmask) == prefix) {
-                const uint32_t bkt = (k >> shift) & 255u;
-                if (by_mass) atomicAdd(&h_mass[bkt], mass[j]);
-                atomicAdd(&h_cnt[bkt], 1u);
+            uint32_t bkt;
+            if (pass == 0) {
+                bkt = 255u - vbkt[j];                 // larger index = larger score
+            } else {
+                const uint32_t k = keys[j];
+                if (vbkt[j] != vsel || (k & pmask) != prefix) continue;
+                bkt = (k >> shift) & 255u;
             }
+            if (by_mass) atomicAdd(&h_mass[bkt], mass[j]);
+            atomicAdd(&h_cnt[bkt], 1u);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
-            // lane l owns buckets 255 - 8l down to 248 - 8l (descending keys)
+            // lane l owns buckets 255 - 8l down to 248 - 8l (descending scores)
             const int lane = threadIdx.x;
             unsigned long long vm[8], vc[8], sm = 0, scn = 0;
 #pragma unroll
@@ -270,8 +278,12 @@ __device__ RadixOut radix_cut(const uint32_t* keys, const unsigned long long* ma
             }
         }
         __syncthreads();
-        prefix |= static_cast<uint32_t>(sh[0]) << shift;
-        pmask |= 255u << shift;
+        if (pass == 0) {
+            vsel = 255 - static_cast<int>(sh[0]);
+        } else {
+            prefix |= static_cast<uint32_t>(sh[0]) << shift;
+            pmask |= 255u << shift;
+        }
         above_mass += sh[1];
         above_cnt += sh[2];
         __syncthreads();
@@ -297,7 +309,8 @@ __device__ RadixOut radix_cut(const uint32_t* keys, const unsigned long long* ma
 }  // namespace
 
 size_t select_smem_bytes(int max_blocks) {
-    return static_cast<size_t>(max_blocks) * (sizeof(uint32_t) + sizeof(unsigned long long)) +
+    return static_cast<size_t>(max_blocks) *
+               (sizeof(uint32_t) + sizeof(unsigned long long) + sizeof(uint8_t)) +
            256 * (sizeof(unsigned long long) + sizeof(unsigned int)) +
            8 * sizeof(unsigned long long) + (kSelectThreads / 32 + 1) * sizeof(int) + 64;
 }
@@ -312,6 +325,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
     uint32_t* keys = reinterpret_cast<uint32_t*>(sh_state + 8);
     unsigned int* h_cnt = keys + p.max_blocks;
     int* scan = reinterpret_cast<int*>(h_cnt + 256);
+    uint8_t* vbkt = reinterpret_cast<uint8_t*>(scan + (kSelectThreads / 32 + 1));
     __shared__ float red_f[32];
 
     const int u = blockIdx.x;
@@ -352,7 +366,11 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
         if (threadIdx.x == 0) red_f[0] = v;
     }
     __syncthreads();
-    const double smax = static_cast<double>(red_f[0]);
+    const float smax_f = red_f[0];
+    const double smax = static_cast<double>(smax_f);
+    // distance-from-max buckets of 1/16, monotone in the score (pass 0 of the cut search)
+    for (int i = threadIdx.x; i < n_res; i += blockDim.x)
+        vbkt[i] = static_cast<uint8_t>(fminf((smax_f - s[r0 + i]) * 16.f, 255.f));
 
     // ---- fixed-point residual softmax numerators, total Z
     unsigned long long zloc = 0;
@@ -399,7 +417,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
     }
     RadixOut cut{0xFFFFFFFFu, 0u, 0u};
     if (by_mass_cut) {
-        cut = radix_cut(keys, mass, n_res, T, true, h_mass, h_cnt, sh_state);
+        cut = radix_cut(keys, vbkt, mass, n_res, T, true, h_mass, h_cnt, sh_state);
         n_take = static_cast<int>(cut.above) + static_cast<int>(cut.take_ties);
         const int floor_res = p.kmin_blocks - n_reserved;      // |S| >= K_min
         if (n_take < floor_res) {
@@ -419,8 +437,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
             cut.key = 0u;            // everything
             cut.take_ties = 0xFFFFFFFFu;
         } else {
-            cut = radix_cut(keys, mass, n_res, static_cast<unsigned long long>(n_take), false,
-                            h_mass, h_cnt, sh_state);
+            cut = radix_cut(keys, vbkt, mass, n_res, static_cast<unsigned long long>(n_take),
+                            false, h_mass, h_cnt, sh_state);
         }
     }
 
@@ -468,7 +486,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
 }  // namespace
 
 cudaError_t launch_scores(const ScoreParams& p, int fmt, cudaStream_t s) {
-    const dim3 grid((p.max_blocks + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta, p.batch);
+    const dim3 grid((p.max_blocks + 15) / 16, (p.num_kv_heads + kScoreWarps - 1) / kScoreWarps,
+                    p.batch);
     if (fmt == SPOT_SEL_BF16)
         score_kernel<SPOT_SEL_BF16><<<grid, kScoreWarps * 32, 0, s>>>(p);
     else if (fmt == SPOT_SEL_INT4_G32_F16)

@@ -23,6 +23,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "spot_device.cuh"
 #include "spot_internal.h"
 
@@ -362,52 +364,78 @@ __device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
     return static_cast<int>(((pos + 1) * P - 1) / N);
 }
 
-// One CTA per (sequence, KV head) unit, one thread per head dimension.
-__global__ void __launch_bounds__(kHeadDim) combine_kernel(const DecodeParams p) {
+// One CTA per (sequence, KV head) unit, one warp per query head of the
+// group; lane l owns head dimensions 4l..4l+3.  The partials of a unit are
+// the NC warp slots of every CTA whose range touched the unit; their loads
+// are independent, so the warp keeps many in flight.
+__global__ void __launch_bounds__(32 * kMaxGroup) combine_kernel(const DecodeParams p) {
     const int u = blockIdx.x;
     const int U = p.batch * p.num_kv_heads;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
     const int G = p.group;
-    const int d = threadIdx.x;
+    const int n = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (n >= G) return;
+    const int h = g * G + n;
+    float4* o = reinterpret_cast<float4*>(
+        p.out + (static_cast<int64_t>(b) * p.num_q_heads + h) * kHeadDim) + lane;
+    float* lse = p.lse ? p.lse + static_cast<int64_t>(b) * p.num_q_heads + h : nullptr;
     const int lo = p.unit_off[u], hi = p.unit_off[u + 1];
+    if (hi <= lo) {
+        *o = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lse && lane == 0) *lse = -INFINITY;
+        return;
+    }
     const int64_t N = p.unit_off[U];
     const int64_t P = p.num_ctas;
-    for (int n = 0; n < G; ++n) {
-        const int h = g * G + n;
-        float* o = p.out + (static_cast<int64_t>(b) * p.num_q_heads + h) * kHeadDim;
-        if (hi <= lo) {
-            o[d] = 0.f;
-            if (p.lse && d == 0) p.lse[static_cast<int64_t>(b) * p.num_q_heads + h] = -INFINITY;
-            continue;
-        }
-        const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
-        const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
-        float M = -INFINITY;
-        for (int i = i0; i <= i1; ++i) {
-            if (range_begin(N, P, i) == range_begin(N, P, i + 1)) continue;   // idle CTA
-            for (int w = 0; w < NC; ++w) {
-                const float* slot = p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
-                M = fmaxf(M, slot[G * kHeadDim + n]);
-            }
-        }
-        float L = 0.f, a = 0.f;
-        for (int i = i0; i <= i1; ++i) {
-            if (range_begin(N, P, i) == range_begin(N, P, i + 1)) continue;
-            for (int w = 0; w < NC; ++w) {
-                const float* slot = p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
-                const float m = slot[G * kHeadDim + n];
-                if (m == -INFINITY) continue;
-                const float f = exp2f(m - M);
-                L = fmaf(f, slot[G * (kHeadDim + 1) + n], L);
-                a = fmaf(f, slot[n * kHeadDim + d], a);
-            }
-        }
-        const bool empty = !(L > 0.f);      // only if every tile was rejected as out of range
-        o[d] = empty ? 0.f : a / L;
-        if (p.lse && d == 0)
-            p.lse[static_cast<int64_t>(b) * p.num_q_heads + h] =
-                empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+    const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
+    const int nslots = (i1 - i0 + 1) * NC;
+    const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
+    auto slot_of = [&](int s) -> const float* {
+        const int i = i0 + s / NC, w = s - (s / NC) * NC;
+        if (range_begin(N, P, i) == range_begin(N, P, i + 1)) return nullptr;   // idle CTA
+        return p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
+    };
+    float M = -INFINITY;
+    for (int s = lane; s < nslots; s += 32) {
+        const float* sl = slot_of(s);
+        if (sl) M = fmaxf(M, sl[G * kHeadDim + n]);
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int base = 0; base < nslots; base += 32) {
+        const int s = base + lane;
+        float wgt = 0.f;
+        if (s < nslots && M != -INFINITY) {
+            const float* sl = slot_of(s);
+            if (sl) {
+                const float m = sl[G * kHeadDim + n];
+                if (m != -INFINITY) {
+                    wgt = exp2f(m - M);
+                    L = fmaf(wgt, sl[G * (kHeadDim + 1) + n], L);
+                }
+            }
+        }
+        const int cnt = min(32, nslots - base);
+#pragma unroll 4
+        for (int k = 0; k < cnt; ++k) {
+            const float wk = __shfl_sync(0xffffffffu, wgt, k);
+            if (wk == 0.f) continue;                      // same value on every lane
+            const float4 v =
+                *(reinterpret_cast<const float4*>(slot_of(base + k) + n * kHeadDim) + lane);
+            a.x = fmaf(wk, v.x, a.x);
+            a.y = fmaf(wk, v.y, a.y);
+            a.z = fmaf(wk, v.z, a.z);
+            a.w = fmaf(wk, v.w, a.w);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    const bool empty = !(L > 0.f);        // only if every tile was rejected as out of range
+    const float inv = empty ? 0.f : 1.f / L;
+    *o = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+    if (lse && lane == 0) *lse = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
 }
 
 }  // namespace
@@ -418,31 +446,66 @@ size_t decode_smem_bytes(int units) {
            (kThreads / 32 + 1) * sizeof(int) + static_cast<size_t>(units + 1) * sizeof(int);
 }
 
+namespace {
+
+// Per-device memo of the kernel attributes the launches need: the dynamic
+// shared-memory limit already set on the kernel and the last grid size
+// computed (the grid depends on the device and, through shared memory, on U).
+struct DeviceMemo {
+    size_t smem_set = 0;
+    int units = -1;
+    int grid = 0;
+};
+constexpr int kMemoDevices = 64;
+DeviceMemo g_memo[kMemoDevices];
+std::mutex g_memo_mutex;
+
+cudaError_t ensure_smem(int dev, size_t smem) {
+    DeviceMemo& m = g_memo[dev];
+    if (m.smem_set >= smem) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(
+        sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess) m.smem_set = smem;
+    return e;
+}
+
+}  // namespace
+
 int decode_grid(int units) {
-    int dev = 0, sms = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMemoDevices) return 0;
+    std::lock_guard<std::mutex> lock(g_memo_mutex);
+    DeviceMemo& m = g_memo[dev];
+    if (m.units == units && m.grid > 0) return m.grid;
+    int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
     const size_t smem = decode_smem_bytes(units);
-    if (cudaFuncSetAttribute(sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return 0;
+    if (ensure_smem(dev, smem) != cudaSuccess) return 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_decode_kernel, kThreads,
                                                       smem) != cudaSuccess)
         return 0;
-    return sms * max(per_sm, 1);
+    m.units = units;
+    m.grid = sms * max(per_sm, 1);
+    return m.grid;
 }
 
 cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
                                  const CUtensorMap& v_map, cudaStream_t s) {
     const int U = p.batch * p.num_kv_heads;
     const size_t smem = decode_smem_bytes(U);
-    cudaError_t e = cudaFuncSetAttribute(
-        sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMemoDevices) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lock(g_memo_mutex);
+        e = ensure_smem(dev, smem);
+    }
     if (e != cudaSuccess) return e;
     sparse_decode_kernel<<<p.num_ctas, kThreads, smem, s>>>(k_map, v_map, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    combine_kernel<<<U, kHeadDim, 0, s>>>(p);
+    combine_kernel<<<U, 32 * p.group, 0, s>>>(p);
     return cudaGetLastError();
 }
 

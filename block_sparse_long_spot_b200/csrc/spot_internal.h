@@ -28,7 +28,9 @@ constexpr uint32_t kStatusTimeout = 2u;
 constexpr int kDecodeConsumers = 4;
 constexpr int kDecodeStages = 4;
 constexpr int kStageBytes = 2 * kBlock * kHeadDim * 2;   // 32768
-constexpr int kPartialFloatsPerHead = kHeadDim + 2;      // acc[128], m, l
+// Per-head share of a partial: acc[128], m, l, padded to 132 floats so
+// every slot (G x 132 floats) and every acc row starts 16-byte aligned.
+constexpr int kPartialFloatsPerHead = kHeadDim + 4;
 
 struct Layout {
     size_t status, scores, unit_off, partials, total;

@@ -28,8 +28,8 @@
  *     per block), sel_dim 64, 1 <= num_q_heads / num_kv_heads <= 8,
  *     batch * num_kv_heads <= 4096, max_blocks <= 16384.  Other shapes
  *     return SPOT_ERR_UNSUPPORTED.
- *   - Alignment: bf16 arrays and the selector data plane 16 bytes, the KV
- *     pools and the workspace 256 bytes, everything else 4 bytes.
+ *   - Alignment: bf16 arrays, the selector data plane and `out` 16 bytes,
+ *     the KV pools and the workspace 256 bytes, everything else 4 bytes.
  *
  * Layouts (row-major, innermost last):
  *   q            bf16  [batch][num_q_heads][head_dim]
@@ -199,7 +199,7 @@ spot_status_t spot_decode_step(const spot_layer_desc_t* desc, const spot_select_
  *     the device current (cudaGetSymbolAddress) and remembers it; make that
  *     first call before any stream capture.
  *   - A shape whose scratch exceeds 8 MiB returns SPOT_ERR_WORKSPACE (about
- *     (grid + U) * 4 * G * 520 bytes with U = batch * num_kv_heads and grid
+ *     (grid + U) * 4 * G * 528 bytes with U = batch * num_kv_heads and grid
  *     = the SM count; e.g. 256 units of G = 4 need 3.4 MB).
  *   - All calls share the one array and it keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other host threads) race
