@@ -90,8 +90,8 @@ bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Lay
     off += kStatusBytes;
     L.scores = off;
     off = round_up(off + static_cast<size_t>(U) * max_blocks * sizeof(float), 256);
-    L.unit_off = off;
-    off = round_up(off + static_cast<size_t>(U + 1) * sizeof(int32_t), 256);
+    L.unit_done = off;
+    off = round_up(off + static_cast<size_t>(U) * sizeof(uint32_t), 256);
     L.partials = off;
     off = round_up(off + static_cast<size_t>(grid + U) * kDecodeConsumers * G *
                              kPartialFloatsPerHead * sizeof(float),
@@ -177,7 +177,7 @@ spot_status_t do_decode(const spot_layer_desc_t* d, const uint16_t* q, const uin
     p.group = d->num_q_heads / d->num_kv_heads;
     p.num_pages = d->num_pages;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    p.unit_off = reinterpret_cast<int32_t*>(base + L.unit_off);
+    p.unit_done = reinterpret_cast<uint32_t*>(base + L.unit_done);
     p.partials = reinterpret_cast<float*>(base + L.partials);
     p.num_ctas = L.grid;
     p.out = out;

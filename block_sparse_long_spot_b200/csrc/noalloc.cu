@@ -6,7 +6,7 @@
 // device allocation, or a plugin host that hands the library the tensors of
 // one call and no allocator at all.  Such a caller cannot provide the
 // workspace that spot_sparse_decode needs.  This entry point runs the same
-// kernels with their scratch (status word, per-unit offsets, split partials)
+// kernels with their scratch (status word, per-unit counters, split partials)
 // in a fixed array that lives in the library itself, `g_noalloc_scratch`
 // below, of kNoAllocScratchBytes bytes.  Every GPU that loads the library
 // holds that array until the process exits.
@@ -74,13 +74,13 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
         !is_aligned(sel_cnt, 4) || !is_aligned(out, 16) || (lse && !is_aligned(lse, 4)))
         return SPOT_ERR_INVALID_ARG;
 
-    // Scratch this shape needs: status word, unit offsets, split partials.
+    // Scratch this shape needs: status word, per-unit counters, split partials.
     const int U = batch * d->num_kv_heads;
     const int G = d->num_q_heads / d->num_kv_heads;
     const int grid = decode_grid(U);
     if (grid <= 0) return SPOT_ERR_CUDA;
     const size_t off_units = kStatusBytes;
-    const size_t off_partials = round256(off_units + static_cast<size_t>(U + 1) * sizeof(int32_t));
+    const size_t off_partials = round256(off_units + static_cast<size_t>(U) * sizeof(uint32_t));
     const size_t need = off_partials + static_cast<size_t>(grid + U) * kDecodeConsumers * G *
                                            kPartialFloatsPerHead * sizeof(float);
     if (need > kNoAllocScratchBytes) return SPOT_ERR_WORKSPACE;
@@ -96,9 +96,9 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
         return SPOT_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* base = static_cast<uint8_t*>(scratch);
-    // The status word must start at zero; the other regions are fully
-    // written by the kernels before they are read.
-    if (cudaMemsetAsync(base, 0, kStatusBytes, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    // The status word and the per-unit arrival counters must start at zero;
+    // the partials are written by the kernel before they are read.
+    if (cudaMemsetAsync(base, 0, off_partials, s) != cudaSuccess) return SPOT_ERR_CUDA;
 
     DecodeParams p;
     p.q = q;
@@ -114,7 +114,7 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
     p.group = G;
     p.num_pages = d->num_pages;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    p.unit_off = reinterpret_cast<int32_t*>(base + off_units);
+    p.unit_done = reinterpret_cast<uint32_t*>(base + off_units);
     p.partials = reinterpret_cast<float*>(base + off_partials);
     p.num_ctas = grid;
     p.out = out;

@@ -30,7 +30,7 @@ namespace spot {
 namespace {
 
 constexpr int kScoreWarps = 8;
-constexpr int kSelectThreads = 512;
+constexpr int kSelectThreads = 256;
 constexpr int kFixShift = 40;
 
 // --------------------------------------------------------------- scoring
@@ -83,6 +83,7 @@ template <int FMT>
 __global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(const ScoreParams p) {
     // One warp per (sequence, KV head, tile of 16 blocks): grid.x tiles,
     // grid.y groups of kScoreWarps KV heads, grid.z sequences.
+    pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = blockIdx.z;
     const int g = blockIdx.y * kScoreWarps + warp;
@@ -201,132 +202,257 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-struct RadixOut {
-    uint32_t key;          // exact key of the cut
-    uint32_t take_ties;    // elements equal to the cut that are kept (lowest index first)
-    uint32_t above;        // elements strictly above the cut
+constexpr int kNB = 1024;              // value buckets of the first pass
+constexpr float kBucketScale = 32.f;    // buckets per unit of score below the maximum
+constexpr int NT = kSelectThreads;
+constexpr int NW = NT / 32;
+
+struct SelSmem {
+    uint32_t* keys;               // [max_blocks] order-preserving keys of the residual scores
+    unsigned long long* mass;     // [max_blocks] fixed-point exp(s - max)
+    uint16_t* vb;                 // [max_blocks] value bucket (0 = the top scores)
+    uint8_t* keep;                // [max_blocks] 1 keep, 2 tie at the cut, 0 drop
+    float* hmass;                 // [kNB] approximate (fp32) mass per bucket
+    uint32_t* hcnt;               // [kNB] exact count per bucket
+    uint32_t* ckey;               // [NT] candidates of the cut bucket: key
+    int* cidx;                    //      element index
+    unsigned long long* cval;     //      mass (or 1) stored at the candidate's rank
+    unsigned long long* red;      // [3 * NW] reduction scratch
+    int* misc;                    // [8]
+    int* scan;                    // [NW + 1]
+    float* fscan;                 // [NW + 1]
 };
 
-// Search for the cut in descending score order over elements [0, n).
-//   by_mass: shortest prefix whose cumulative fixed-point mass is >= target;
-//   else:    prefix of exactly `target` elements (1 <= target < n).
-// Pass 0 buckets by the score's distance from the maximum (vbkt: 0 = the
-// top scores, monotone in the score, spreads the elements even when they
-// share their exponent bits); passes 1-4 refine the chosen bucket by the
-// 8-bit digits of the order-preserving key.  Called by every thread.
-__device__ RadixOut radix_cut(const uint32_t* keys, const uint8_t* vbkt,
-                              const unsigned long long* mass, int n, unsigned long long target,
-                              bool by_mass, unsigned long long* h_mass, unsigned int* h_cnt,
-                              unsigned long long* sh) {
-    uint32_t prefix = 0, pmask = 0;
-    int vsel = -1;
-    unsigned long long above_mass = 0, above_cnt = 0;
-    for (int pass = 0; pass < 5; ++pass) {
-        const int shift = 32 - 8 * pass;          // key digit of passes 1..4
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) { h_mass[i] = 0; h_cnt[i] = 0; }
-        __syncthreads();
-        for (int j = threadIdx.x; j < n; j += blockDim.x) {
-            uint32_t bkt;
-            if (pass == 0) {
-                bkt = 255u - vbkt[j];                 // larger index = larger score
-            } else {
-                const uint32_t k = keys[j];
-                if (vbkt[j] != vsel || (k & pmask) != prefix) continue;
-                bkt = (k >> shift) & 255u;
-            }
-            if (by_mass) atomicAdd(&h_mass[bkt], mass[j]);
-            atomicAdd(&h_cnt[bkt], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            // lane l owns buckets 255 - 8l down to 248 - 8l (descending scores)
-            const int lane = threadIdx.x;
-            unsigned long long vm[8], vc[8], sm = 0, scn = 0;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int bkt = 255 - 8 * lane - k;
-                vm[k] = h_mass[bkt];
-                vc[k] = h_cnt[bkt];
-                sm += vm[k];
-                scn += vc[k];
-            }
-            unsigned long long im = sm, ic = scn;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned long long a = __shfl_up_sync(0xffffffffu, im, o);
-                const unsigned long long c = __shfl_up_sync(0xffffffffu, ic, o);
-                if (lane >= o) { im += a; ic += c; }
-            }
-            const unsigned long long em = im - sm, ec = ic - scn;
-            const unsigned long long base = by_mass ? above_mass : above_cnt;
-            const unsigned long long incl = by_mass ? im : ic, excl = by_mass ? em : ec;
-            const bool hit = (base + excl < target) && (base + incl >= target);
-            const unsigned ballot = __ballot_sync(0xffffffffu, hit);
-            if (ballot && lane == __ffs(ballot) - 1) {
-                unsigned long long dm = em, dc = ec;   // mass / count above this lane
-                int bsel = 255 - 8 * lane - 7;
-                for (int k = 0; k < 8; ++k) {
-                    const unsigned long long v = by_mass ? vm[k] : vc[k];
-                    const unsigned long long run = base + (by_mass ? dm : dc);
-                    if (run + v >= target) { bsel = 255 - 8 * lane - k; break; }
-                    dm += vm[k];
-                    dc += vc[k];
-                }
-                sh[0] = static_cast<unsigned long long>(bsel);
-                sh[1] = dm;
-                sh[2] = dc;
-            }
-        }
-        __syncthreads();
-        if (pass == 0) {
-            vsel = 255 - static_cast<int>(sh[0]);
-        } else {
-            prefix |= static_cast<uint32_t>(sh[0]) << shift;
-            pmask |= 255u << shift;
-        }
-        above_mass += sh[1];
-        above_cnt += sh[2];
-        __syncthreads();
-    }
-    RadixOut r;
-    r.key = prefix;
-    r.above = static_cast<uint32_t>(above_cnt);
-    if (by_mass) {
-        // every element equal to the cut has the same mass e* > 0
-        for (int j = threadIdx.x; j < n; j += blockDim.x)
-            if (keys[j] == prefix) sh[3] = mass[j];
-        __syncthreads();
-        const unsigned long long e_star = sh[3];
-        const unsigned long long need = target - above_mass;
-        r.take_ties = e_star ? static_cast<uint32_t>((need + e_star - 1) / e_star) : 0u;
-    } else {
-        r.take_ties = static_cast<uint32_t>(target - above_cnt);
+// Sums of three values over the block (two barriers).
+__device__ __forceinline__ void block_sum3(const SelSmem& sm, unsigned long long& a,
+                                           unsigned long long& b, unsigned long long& c) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    a = warp_sum(a);
+    b = warp_sum(b);
+    c = warp_sum(c);
+    if (lane == 0) {
+        sm.red[warp] = a;
+        sm.red[NW + warp] = b;
+        sm.red[2 * NW + warp] = c;
     }
     __syncthreads();
-    return r;
+    a = b = c = 0;
+    for (int w = 0; w < NW; ++w) {
+        a += sm.red[w];
+        b += sm.red[NW + w];
+        c += sm.red[2 * NW + w];
+    }
+    __syncthreads();
+}
+
+// Exclusive prefix over the block of a float (two barriers); *total = sum.
+__device__ __forceinline__ float block_exclusive_scan_f(const SelSmem& sm, float v, float* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) sm.fscan[warp] = incl;
+    __syncthreads();
+    float base = 0.f, tot = 0.f;
+    for (int w = 0; w < NW; ++w) {
+        if (w < warp) base += sm.fscan[w];
+        tot += sm.fscan[w];
+    }
+    *total = tot;
+    __syncthreads();
+    return base + incl - v;
+}
+
+// Bucket of the cut, found on the bucket histograms: the first bucket (from
+// the top) where the cumulative value reaches `target`.  by_mass uses the
+// approximate fp32 masses (the caller corrects the result exactly), else the
+// exact counts.  Returns the bucket; *before receives the exact count of
+// elements in the buckets above it (count mode only).
+__device__ int cut_bucket(const SelSmem& sm, double target, bool by_mass, int* before) {
+    constexpr int PER = kNB / NT;
+    float loc = 0.f;
+    int cnt = 0, last = -1;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int bkt = threadIdx.x * PER + k;
+        loc += by_mass ? sm.hmass[bkt] : static_cast<float>(sm.hcnt[bkt]);
+        cnt += sm.hcnt[bkt];
+        if (sm.hcnt[bkt]) last = bkt;
+    }
+    if (threadIdx.x == 0) { sm.misc[0] = -1; sm.misc[1] = -1; }
+    int ctot;
+    const int cbase = block_exclusive_scan<NT>(cnt, sm.scan, &ctot);
+    float ftot;
+    const float fbase = block_exclusive_scan_f(sm, loc, &ftot);
+    // the thread whose buckets hold the crossing point records it
+    float run = fbase;
+    int crun = cbase;
+    for (int k = 0; k < PER; ++k) {
+        const int bkt = threadIdx.x * PER + k;
+        const float v = by_mass ? sm.hmass[bkt] : static_cast<float>(sm.hcnt[bkt]);
+        const bool hit = by_mass ? (run < target && run + v >= target)
+                                 : (crun < target && crun + static_cast<int>(sm.hcnt[bkt]) >= target);
+        if (hit && sm.hcnt[bkt]) {
+            sm.misc[0] = bkt;
+            sm.misc[2] = crun;
+        }
+        run += v;
+        crun += sm.hcnt[bkt];
+    }
+    if (last >= 0) atomicMax(&sm.misc[1], last);
+    __syncthreads();
+    int b = sm.misc[0];
+    int bef = sm.misc[2];
+    if (b < 0) {            // fp32 rounding kept the total below the target
+        b = sm.misc[1];
+        bef = ctot - static_cast<int>(sm.hcnt[b]);
+    }
+    *before = bef;
+    __syncthreads();
+    return b;
+}
+
+struct Cut {
+    int bucket;            // elements in buckets above it are kept, below it dropped
+    int kept_above;        // elements kept from the buckets above
+    int kept_in_bucket;    // elements kept from the bucket itself
+};
+
+// Exact resolution inside bucket b: keeps the shortest prefix (ranked by
+// score, lower block index first) whose cumulative mass (or count) added to
+// `above` reaches `target`; writes the keep flags of the bucket's elements.
+__device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long long above,
+                              unsigned long long target, bool by_mass) {
+    const int c = static_cast<int>(sm.hcnt[b]);
+    if (threadIdx.x == 0) { sm.misc[3] = 0; sm.misc[4] = c - 1; }
+    __syncthreads();
+    if (c <= NT) {
+        for (int i = threadIdx.x; i < n; i += NT) {
+            if (sm.vb[i] == b) {
+                const int slot = atomicAdd(&sm.misc[3], 1);
+                sm.ckey[slot] = sm.keys[i];
+                sm.cidx[slot] = i;
+            }
+        }
+        __syncthreads();
+        int rank = 0;
+        if (threadIdx.x < c) {
+            const uint32_t k = sm.ckey[threadIdx.x];
+            const int j = sm.cidx[threadIdx.x];
+            for (int d = 0; d < c; ++d) {
+                const uint32_t kd = sm.ckey[d];
+                rank += (kd > k) || (kd == k && sm.cidx[d] < j);
+            }
+            sm.cval[rank] = by_mass ? sm.mass[j] : 1ull;
+        }
+        __syncthreads();
+        // cumulative value in rank order: thread t holds rank t
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        unsigned long long v = threadIdx.x < c ? sm.cval[threadIdx.x] : 0ull, incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long x = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += x;
+        }
+        if (lane == 31) sm.red[warp] = incl;
+        __syncthreads();
+        unsigned long long base = above;
+        for (int w = 0; w < warp; ++w) base += sm.red[w];
+        if (threadIdx.x < c && base + incl - v < target && base + incl >= target)
+            sm.misc[4] = threadIdx.x;                 // the rank that reaches the target
+        __syncthreads();
+        const int r_cut = sm.misc[4];
+        if (threadIdx.x < c) sm.keep[sm.cidx[threadIdx.x]] = rank <= r_cut ? 1 : 0;
+        __syncthreads();
+        return r_cut + 1;
+    }
+    // Many elements share the bucket (heavy ties): exact threshold search on
+    // the keys of the bucket by bisection, each probe an exact block sum.
+    uint32_t lo = 0u, hi = 0xFFFFFFFFu;      // the cut key lies in [lo, hi]
+    unsigned long long m_hi = 0, c_hi = 0;   // mass / count of keys > hi within the bucket
+    while (lo < hi) {
+        const uint32_t mid = lo + (hi - lo) / 2 + 1;       // test "keys >= mid"
+        unsigned long long m = 0, cn = 0, dummy = 0;
+        for (int i = threadIdx.x; i < n; i += NT)
+            if (sm.vb[i] == b && sm.keys[i] >= mid) { m += sm.mass[i]; ++cn; }
+        block_sum3(sm, m, cn, dummy);
+        const unsigned long long val = by_mass ? m : cn;
+        if (above + val >= target) {
+            lo = mid;                          // the cut is at or above mid
+        } else {
+            hi = mid - 1;
+            m_hi = m;
+            c_hi = cn;
+        }
+    }
+    // keys > lo are kept; ties at lo by block index
+    unsigned long long m_eq = 0, c_eq = 0, dummy = 0;
+    for (int i = threadIdx.x; i < n; i += NT)
+        if (sm.vb[i] == b && sm.keys[i] == lo) { m_eq += sm.mass[i]; ++c_eq; }
+    block_sum3(sm, m_eq, c_eq, dummy);
+    unsigned long long take;
+    if (by_mass) {
+        const unsigned long long e = c_eq ? m_eq / c_eq : 0ull;
+        const unsigned long long need = target - above - m_hi;
+        take = e ? (need + e - 1) / e : 0ull;
+    } else {
+        take = target - above - c_hi;
+    }
+    for (int i = threadIdx.x; i < n; i += NT)
+        if (sm.vb[i] == b) sm.keep[i] = sm.keys[i] > lo ? 1 : (sm.keys[i] == lo ? 2 : 0);
+    if (threadIdx.x == 0) sm.misc[5] = static_cast<int>(take);
+    __syncthreads();
+    return static_cast<int>(c_hi + take);
 }
 
 }  // namespace
 
 size_t select_smem_bytes(int max_blocks) {
     return static_cast<size_t>(max_blocks) *
-               (sizeof(uint32_t) + sizeof(unsigned long long) + sizeof(uint8_t)) +
-           256 * (sizeof(unsigned long long) + sizeof(unsigned int)) +
-           8 * sizeof(unsigned long long) + (kSelectThreads / 32 + 1) * sizeof(int) + 64;
+               (sizeof(uint32_t) + sizeof(unsigned long long) + sizeof(uint16_t) + 1) +
+           kNB * (sizeof(float) + sizeof(uint32_t)) +
+           NT * (sizeof(uint32_t) + sizeof(int) + sizeof(unsigned long long)) +
+           3 * NW * sizeof(unsigned long long) + 8 * sizeof(int) +
+           2 * (NW + 1) * sizeof(int) + 128;
 }
 
 namespace {
 
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
-    unsigned long long* mass = reinterpret_cast<unsigned long long*>(smem);
-    unsigned long long* h_mass = mass + p.max_blocks;
-    unsigned long long* sh_state = h_mass + 256;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(sh_state + 8);
-    unsigned int* h_cnt = keys + p.max_blocks;
-    int* scan = reinterpret_cast<int*>(h_cnt + 256);
-    uint8_t* vbkt = reinterpret_cast<uint8_t*>(scan + (kSelectThreads / 32 + 1));
-    __shared__ float red_f[32];
+    SelSmem sm;
+    {
+        uint8_t* q = smem;
+        sm.mass = reinterpret_cast<unsigned long long*>(q);
+        q += sizeof(unsigned long long) * p.max_blocks;
+        sm.cval = reinterpret_cast<unsigned long long*>(q);
+        q += sizeof(unsigned long long) * NT;
+        sm.red = reinterpret_cast<unsigned long long*>(q);
+        q += sizeof(unsigned long long) * 3 * NW;
+        sm.keys = reinterpret_cast<uint32_t*>(q);
+        q += sizeof(uint32_t) * p.max_blocks;
+        sm.hmass = reinterpret_cast<float*>(q);
+        q += sizeof(float) * kNB;
+        sm.hcnt = reinterpret_cast<uint32_t*>(q);
+        q += sizeof(uint32_t) * kNB;
+        sm.ckey = reinterpret_cast<uint32_t*>(q);
+        q += sizeof(uint32_t) * NT;
+        sm.cidx = reinterpret_cast<int*>(q);
+        q += sizeof(int) * NT;
+        sm.misc = reinterpret_cast<int*>(q);
+        q += sizeof(int) * 8;
+        sm.scan = reinterpret_cast<int*>(q);
+        q += sizeof(int) * (NW + 1);
+        sm.fscan = reinterpret_cast<float*>(q);
+        q += sizeof(float) * (NW + 1);
+        sm.vb = reinterpret_cast<uint16_t*>(q);
+        q += sizeof(uint16_t) * p.max_blocks;
+        sm.keep = q;
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
     const int u = blockIdx.x;
     const int b = u / p.num_kv_heads;
@@ -344,146 +470,144 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
     rec = max(rec, nb - n_full);
     rec = min(rec, nb);
     const int r0 = sink, r1 = max(sink, nb - rec);    // residual blocks [r0, r1)
-    const int n_res = r1 - r0;
-    const int n_reserved = nb - n_res;
+    const int n = r1 - r0;
+    const int n_reserved = nb - n;
     const float* s = p.scores + static_cast<int64_t>(u) * p.max_blocks;
+    for (int i = threadIdx.x; i < kNB; i += NT) { sm.hmass[i] = 0.f; sm.hcnt[i] = 0u; }
+    if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
+    pdl_trigger();
+    pdl_wait();                                       // scores of the scoring kernel
 
-    // ---- residual scores -> keys, max
+    // ---- residual scores -> keys, maximum
     float mloc = -INFINITY;
-    for (int i = threadIdx.x; i < n_res; i += blockDim.x) {
+    for (int i = threadIdx.x; i < n; i += NT) {
         const float v = s[r0 + i];
-        keys[i] = score_key(v);
+        sm.keys[i] = score_key(v);
         mloc = fmaxf(mloc, v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
-    if ((threadIdx.x & 31) == 0) red_f[threadIdx.x >> 5] = mloc;
+    if (lane == 0) sm.fscan[warp] = mloc;
     __syncthreads();
-    if (threadIdx.x < 32) {
-        float v = (threadIdx.x < blockDim.x / 32) ? red_f[threadIdx.x] : -INFINITY;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (threadIdx.x == 0) red_f[0] = v;
-    }
-    __syncthreads();
-    const float smax_f = red_f[0];
+    float smax_f = -INFINITY;
+    for (int w = 0; w < NW; ++w) smax_f = fmaxf(smax_f, sm.fscan[w]);
     const double smax = static_cast<double>(smax_f);
-    // distance-from-max buckets of 1/16, monotone in the score (pass 0 of the cut search)
-    for (int i = threadIdx.x; i < n_res; i += blockDim.x)
-        vbkt[i] = static_cast<uint8_t>(fminf((smax_f - s[r0 + i]) * 16.f, 255.f));
 
-    // ---- fixed-point residual softmax numerators, total Z
+    // ---- exact fixed-point numerators exp(s - max), their total Z, value
+    // buckets (monotone in the score) with exact counts and fp32 masses
     unsigned long long zloc = 0;
-    for (int i = threadIdx.x; i < n_res; i += blockDim.x) {
-        const double e = exp(static_cast<double>(s[r0 + i]) - smax);
+    for (int i = threadIdx.x; i < n; i += NT) {
+        const float v = s[r0 + i];
+        const double e = exp(static_cast<double>(v) - smax);
         const unsigned long long f = __double2ull_rn(ldexp(e, kFixShift));
-        mass[i] = f;
+        sm.mass[i] = f;
+        const int bkt = static_cast<int>(fminf((smax_f - v) * kBucketScale, kNB - 1.f));
+        sm.vb[i] = static_cast<uint16_t>(bkt);
+        atomicAdd(&sm.hcnt[bkt], 1u);
+        atomicAdd(&sm.hmass[bkt], static_cast<float>(e));
         zloc += f;
     }
-    zloc = warp_sum(zloc);
-    if ((threadIdx.x & 31) == 0) h_mass[threadIdx.x >> 5] = zloc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned long long z = 0;
-        for (int w = 0; w < static_cast<int>(blockDim.x / 32); ++w) z += h_mass[w];
-        sh_state[6] = z;
-    }
-    __syncthreads();
-    const unsigned long long Z = sh_state[6];
-    __syncthreads();
+    unsigned long long Z = zloc, d1 = 0, d2 = 0;
+    block_sum3(sm, Z, d1, d2);
 
-    // ---- how many residual blocks to keep
-    int n_take;
-    bool by_mass_cut = false;
-    unsigned long long T = 0;
-    if (n_res == 0) {
-        n_take = 0;
-    } else if (p.mode == SPOT_MODE_TOPK) {
-        n_take = min(max(p.topk_blocks, 0), n_res);
-    } else {
-        const float pb = p.top_p ? p.top_p[b] : 1.f;
-        if (pb >= 1.f) {
-            n_take = n_res;
-        } else if (pb <= 0.f) {
-            n_take = 0;
+    // ---- how many residual blocks to keep, and which
+    int n_take = 0;        // -1: decided by the mass cut below
+    if (n > 0) {
+        if (p.mode == SPOT_MODE_TOPK) {
+            n_take = min(max(p.topk_blocks, 0), n);
         } else {
-            T = static_cast<unsigned long long>(ceil(static_cast<double>(pb) *
-                                                     static_cast<double>(Z)));
-            if (T == 0) T = 1;
-            if (T > Z) T = Z;
-            by_mass_cut = true;
-            n_take = -1;       // resolved below
+            const float pb = p.top_p ? p.top_p[b] : 1.f;
+            n_take = pb >= 1.f ? n : (pb <= 0.f ? 0 : -1);
         }
     }
-    RadixOut cut{0xFFFFFFFFu, 0u, 0u};
-    if (by_mass_cut) {
-        cut = radix_cut(keys, vbkt, mass, n_res, T, true, h_mass, h_cnt, sh_state);
-        n_take = static_cast<int>(cut.above) + static_cast<int>(cut.take_ties);
+    bool done = false;
+    if (n_take < 0) {
+        unsigned long long T = static_cast<unsigned long long>(
+            ceil(static_cast<double>(p.top_p[b]) * static_cast<double>(Z)));
+        T = T < 1ull ? 1ull : (T > Z ? Z : T);
+        int before;
+        int bk = cut_bucket(sm, ldexp(static_cast<double>(T), -kFixShift), true, &before);
+        // exact check of the bucket on the fixed-point masses; step to the
+        // neighbouring non-empty bucket while the fp32 estimate was off
+        unsigned long long A, Bm, Ac;
+        for (int guard = 0; guard < kNB; ++guard) {
+            A = 0; Bm = 0; Ac = 0;
+            for (int i = threadIdx.x; i < n; i += NT) {
+                const int v = sm.vb[i];
+                if (v < bk) { A += sm.mass[i]; ++Ac; }
+                else if (v == bk) Bm += sm.mass[i];
+            }
+            block_sum3(sm, A, Bm, Ac);
+            int step = 0;
+            if (A >= T) step = -1;
+            else if (A + Bm < T) step = 1;
+            if (step == 0) break;
+            int nbk = bk + step;
+            while (nbk >= 0 && nbk < kNB && sm.hcnt[nbk] == 0) nbk += step;
+            if (nbk < 0 || nbk >= kNB) break;
+            bk = nbk;
+        }
+        for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
+        __syncthreads();
+        n_take = static_cast<int>(Ac) + resolve_bucket(sm, n, bk, A, T, true);
+        done = true;
         const int floor_res = p.kmin_blocks - n_reserved;      // |S| >= K_min
         if (n_take < floor_res) {
-            n_take = min(floor_res, n_res);
-            by_mass_cut = false;
+            n_take = min(floor_res, n);
+            done = false;
         }
+    } else if (p.mode == SPOT_MODE_TOPP && n > 0) {
+        const int floor_res = p.kmin_blocks - n_reserved;
+        if (n_take < floor_res) n_take = min(floor_res, n);
     }
-    if (!by_mass_cut) {
-        if (p.mode == SPOT_MODE_TOPP) {
-            const int floor_res = p.kmin_blocks - n_reserved;
-            n_take = min(max(n_take, floor_res), n_res);
-        }
-        if (n_take <= 0) {
-            cut.key = 0xFFFFFFFFu;   // nothing from the residual
-            cut.take_ties = 0;
-        } else if (n_take >= n_res) {
-            cut.key = 0u;            // everything
-            cut.take_ties = 0xFFFFFFFFu;
+    if (!done) {
+        if (threadIdx.x == 0) sm.misc[5] = 0;
+        if (n_take <= 0 || n_take >= n) {
+            for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = n_take > 0 ? 1 : 0;
+            __syncthreads();
         } else {
-            cut = radix_cut(keys, vbkt, mass, n_res, static_cast<unsigned long long>(n_take),
-                            false, h_mass, h_cnt, sh_state);
+            int before;
+            const int bk = cut_bucket(sm, static_cast<double>(n_take), false, &before);
+            for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
+            __syncthreads();
+            resolve_bucket(sm, n, bk, static_cast<unsigned long long>(before),
+                           static_cast<unsigned long long>(n_take), false);
         }
     }
+    const uint32_t take = static_cast<uint32_t>(sm.misc[5]);
 
-    // ---- compaction: each thread owns a contiguous run of block ids
-    constexpr int NT = kSelectThreads;
+    // ---- compaction: each thread owns a contiguous run of block ids; one
+    // block scan of (ties at a key cut << 16 | other kept blocks)
     const int per = (nb + NT - 1) / NT;
     const int lo = min(nb, static_cast<int>(threadIdx.x) * per), hi = min(nb, lo + per);
-    int ties = 0;
-    for (int j = lo; j < hi; ++j)
-        if (j >= r0 && j < r1 && keys[j - r0] == cut.key) ++ties;
-    int total;
-    int tie_rank = block_exclusive_scan<NT>(ties, scan, &total);
-    int kept = 0;
+    int ties = 0, kept = 0;
     for (int j = lo; j < hi; ++j) {
-        bool keep;
-        if (j < r0 || j >= r1) {
-            keep = true;
-        } else {
-            const uint32_t k = keys[j - r0];
-            if (k > cut.key) keep = true;
-            else if (k == cut.key) keep = static_cast<uint32_t>(tie_rank++) < cut.take_ties;
-            else keep = false;
-        }
-        kept += keep;
+        if (j < r0 || j >= r1) { ++kept; continue; }
+        const int f = sm.keep[j - r0];
+        kept += f == 1;
+        ties += f == 2;
     }
-    int n_sel;
-    int out_pos = block_exclusive_scan<NT>(kept, scan, &n_sel);
-    tie_rank = block_exclusive_scan<NT>(ties, scan, &total);
+    int total;
+    const int before = block_exclusive_scan<NT>((ties << 16) | kept, sm.scan, &total);
+    uint32_t tie_rank = static_cast<uint32_t>(before >> 16);
+    int out_pos = (before & 0xFFFF) + static_cast<int>(min(tie_rank, take));
     int32_t* out = p.sel_idx + static_cast<int64_t>(u) * p.max_blocks;
     for (int j = lo; j < hi; ++j) {
         bool keep;
         if (j < r0 || j >= r1) {
             keep = true;
         } else {
-            const uint32_t k = keys[j - r0];
-            if (k > cut.key) keep = true;
-            else if (k == cut.key) keep = static_cast<uint32_t>(tie_rank++) < cut.take_ties;
-            else keep = false;
+            const int f = sm.keep[j - r0];
+            keep = f == 1 || (f == 2 && tie_rank++ < take);
         }
         if (keep) out[out_pos++] = j;
     }
-    if (threadIdx.x == 0) p.sel_cnt[u] = n_sel;
+    if (threadIdx.x == 0)
+        p.sel_cnt[u] = (total & 0xFFFF) + static_cast<int>(min(static_cast<uint32_t>(total >> 16), take));
 }
 
 }  // namespace
+
 
 cudaError_t launch_scores(const ScoreParams& p, int fmt, cudaStream_t s) {
     const dim3 grid((p.max_blocks + 15) / 16, (p.num_kv_heads + kScoreWarps - 1) / kScoreWarps,
@@ -502,8 +626,8 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    select_kernel<<<p.batch * p.num_kv_heads, kSelectThreads, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(select_kernel, dim3(p.batch * p.num_kv_heads), dim3(kSelectThreads), smem, s,
+                      p);
 }
 
 }  // namespace spot

@@ -1,6 +1,6 @@
 // sparse_decode.cu -- exact attention over the selected KV blocks
 // (SpotAttention §2.3: the layer attends only to keys in the selected
-// blocks; decode only), split across a persistent grid, then a combine.
+// blocks; decode only), split across a persistent grid and merged in place.
 //
 // Work decomposition ("stream-K" over blocks): the selected blocks of all
 // (sequence, KV head) units, each unit's list in ascending block order, are
@@ -8,8 +8,10 @@
 // [floor(i N / P), floor((i+1) N / P)) of that list, so every CTA streams
 // the same number of 32 KiB (K + V) tiles whatever the per-unit budgets.
 // Where a range crosses a unit boundary the CTA emits one partial result per
-// unit it touched; the combine kernel merges a unit's partials with their
-// log-sum-exp weights.
+// unit it touched.  The CTA whose partial completes a unit (a per-unit
+// arrival counter in the workspace reaches the unit's block count) merges the
+// unit's partials with their log-sum-exp weights and writes the output; the
+// counter is reset to zero by that CTA, so it is zero again for the next call.
 //
 // Inside a CTA one producer warp issues TMA tile loads of the gathered pages
 // (two 64 x 64 bf16 boxes each for K and V, 128-byte swizzled) into a ring
@@ -60,6 +62,79 @@ __device__ __forceinline__ int range_begin(int64_t N, int64_t P, int64_t i) {
     return static_cast<int>((N * i) / P);
 }
 
+// Barrier of the NC consumer warps only (the producer runs ahead).
+__device__ __forceinline__ void consumer_barrier() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
+}
+
+// CTA i of the persistent grid that owns flattened position pos.
+__device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
+    return static_cast<int>(((pos + 1) * P - 1) / N);
+}
+
+// Merge the partials of query head n of unit u (blocks [lo, hi) of the
+// flattened list) and write out / lse.  One warp; lane l owns head
+// dimensions 4l..4l+3.  The partials are those of the NC warps of every CTA
+// whose range touched the unit; other CTAs of this launch wrote them, so they
+// are read through L2 (ld.global.cg).
+__device__ void merge_unit_head(const DecodeParams& p, int u, int n, int lo, int hi, int64_t N,
+                                int64_t P, int lane) {
+    const int G = p.group;
+    const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+    const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
+    const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
+    const int nslots = (i1 - i0 + 1) * NC;
+    const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
+    const bool some_idle = N < P;          // only then can a CTA own no blocks
+    auto slot_of = [&](int sidx) -> const float* {
+        const int i = i0 + sidx / NC, w = sidx % NC;
+        if (some_idle && range_begin(N, P, i) == range_begin(N, P, i + 1)) return nullptr;
+        return p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
+    };
+    float M = -INFINITY;
+    for (int sidx = lane; sidx < nslots; sidx += 32) {
+        const float* sl = slot_of(sidx);
+        if (sl) M = fmaxf(M, __ldcg(sl + G * kHeadDim + n));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int base = 0; base < nslots; base += 32) {
+        const int sidx = base + lane;
+        float wgt = 0.f;
+        if (sidx < nslots && M != -INFINITY) {
+            const float* sl = slot_of(sidx);
+            if (sl) {
+                const float m = __ldcg(sl + G * kHeadDim + n);
+                if (m != -INFINITY) {
+                    wgt = exp2f(m - M);
+                    L = fmaf(wgt, __ldcg(sl + G * (kHeadDim + 1) + n), L);
+                }
+            }
+        }
+        const int cnt = min(32, nslots - base);
+#pragma unroll 4
+        for (int k = 0; k < cnt; ++k) {
+            const float wk = __shfl_sync(0xffffffffu, wgt, k);
+            if (wk == 0.f) continue;                      // same value on every lane
+            const float4 v =
+                __ldcg(reinterpret_cast<const float4*>(slot_of(base + k) + n * kHeadDim) + lane);
+            a.x = fmaf(wk, v.x, a.x);
+            a.y = fmaf(wk, v.y, a.y);
+            a.z = fmaf(wk, v.z, a.z);
+            a.w = fmaf(wk, v.w, a.w);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    const bool empty = !(L > 0.f);        // only if every tile was rejected as out of range
+    const float inv = empty ? 0.f : 1.f / L;
+    reinterpret_cast<float4*>(p.out + h * kHeadDim)[lane] =
+        make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+    if (p.lse && lane == 0) p.lse[h] = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+}
+
 __global__ void __launch_bounds__(kThreads)
 sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
@@ -78,7 +153,8 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
     uint64_t* empty = full + STAGES;
     int* valid = reinterpret_cast<int*>(empty + STAGES);
     int* scan = valid + STAGES;
-    int* unit_off = scan + (kThreads / 32 + 1);
+    volatile int* flags = scan + (kThreads / 32 + 1);   // [0] abort, [1] unit complete
+    int* unit_off = scan + (kThreads / 32 + 1) + 2;
     const uint32_t stage_base = smem_u32(base);
 
     if (threadIdx.x == 0) {
@@ -87,11 +163,15 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
             mbar_init(&empty[s], 1);
         }
         fence_mbar_init();
+        flags[0] = 0;
+        flags[1] = 0;
     }
     if (warp == NC && lane == 0) {
         prefetch_tensormap(&k_map);
         prefetch_tensormap(&v_map);
     }
+    pdl_wait();                                       // selection of the previous kernel
+    pdl_trigger();
 
     // ---- prefix sum of the per-unit counts (every CTA computes its own copy)
     const int per = (U + kThreads - 1) / kThreads;
@@ -120,7 +200,17 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
     if (threadIdx.x == 0) unit_off[U] = total;
     __syncthreads();
     if (blockIdx.x == 0) {
-        for (int u = threadIdx.x; u <= U; u += kThreads) p.unit_off[u] = unit_off[u];
+        // (sequence, KV head) units with nothing selected: out = 0, lse = -inf
+        for (int t = threadIdx.x; t < U * G * (kHeadDim / 4); t += kThreads) {
+            const int u = t / (G * (kHeadDim / 4));
+            if (unit_off[u + 1] != unit_off[u]) continue;
+            const int r = t - u * G * (kHeadDim / 4);
+            const int n = r / (kHeadDim / 4), d4 = r - n * (kHeadDim / 4);
+            const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+            const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
+            reinterpret_cast<float4*>(p.out + h * kHeadDim)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p.lse && d4 == 0) p.lse[h] = -INFINITY;
+        }
     }
 
     const int64_t N = total;
@@ -167,8 +257,10 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                 const int round = itk / STAGES;
                 int ok = 1;
                 if (lane == 0) {
-                    if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
+                    if (flags[0] ||
+                        (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1))) {
                         flag_status(p.status, kStatusTimeout);
+                        flags[0] = 1;
                         ok = 0;
                     } else {
                         valid[s] = v;
@@ -226,12 +318,17 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
 
         const int it0 = pos - beg, it1 = seg_end - beg;
         const int first = it0 + ((warp - it0) % NC + NC) % NC;
-        bool alive = true;
         for (int it = first; it < it1; it += NC) {
             const int s = it % STAGES;
-            if (!mbar_wait_bounded(&full[s], (it / STAGES) & 1)) {
-                if (lane == 0) flag_status(p.status, kStatusTimeout);
-                alive = false;
+            // After a timeout anywhere in the CTA the warps stop waiting but
+            // keep their place in the named barriers below.
+            int ok = __shfl_sync(0xffffffffu, flags[0], 0) == 0;
+            if (ok) ok = mbar_wait_bounded(&full[s], (it / STAGES) & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) {
+                    flag_status(p.status, kStatusTimeout);
+                    flags[0] = 1;
+                }
                 break;
             }
             const int nvalid = valid[s];
@@ -322,7 +419,6 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        if (!alive) return;
 
         // ---- this warp's partial for unit u
 #pragma unroll
@@ -355,87 +451,24 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                 slot[G * (kHeadDim + 1) + h1] = l1;
             }
         }
+        __threadfence();                 // the partial is visible GPU-wide ...
+        consumer_barrier();
+        if (warp == 0 && lane == 0) {    // ... before this CTA's arrival is counted
+            const unsigned seg_len = static_cast<unsigned>(seg_end - pos);
+            const unsigned cnt_u = static_cast<unsigned>(unit_off[u + 1] - unit_off[u]);
+            const unsigned old = atomicAdd(&p.unit_done[u], seg_len);
+            const int last = (old + seg_len == cnt_u);
+            if (last) p.unit_done[u] = 0u;          // every arrival is in: ready for the next call
+            flags[1] = last;
+        }
+        consumer_barrier();
+        if (flags[1]) {
+            __threadfence();
+            for (int n = warp; n < G; n += NC)
+                merge_unit_head(p, u, n, unit_off[u], unit_off[u + 1], N, P, lane);
+        }
         pos = seg_end;
     }
-}
-
-// CTA i of the persistent grid that owns flattened position pos.
-__device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
-    return static_cast<int>(((pos + 1) * P - 1) / N);
-}
-
-// One CTA per (sequence, KV head) unit, one warp per query head of the
-// group; lane l owns head dimensions 4l..4l+3.  The partials of a unit are
-// the NC warp slots of every CTA whose range touched the unit; their loads
-// are independent, so the warp keeps many in flight.
-__global__ void __launch_bounds__(32 * kMaxGroup) combine_kernel(const DecodeParams p) {
-    const int u = blockIdx.x;
-    const int U = p.batch * p.num_kv_heads;
-    const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
-    const int G = p.group;
-    const int n = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (n >= G) return;
-    const int h = g * G + n;
-    float4* o = reinterpret_cast<float4*>(
-        p.out + (static_cast<int64_t>(b) * p.num_q_heads + h) * kHeadDim) + lane;
-    float* lse = p.lse ? p.lse + static_cast<int64_t>(b) * p.num_q_heads + h : nullptr;
-    const int lo = p.unit_off[u], hi = p.unit_off[u + 1];
-    if (hi <= lo) {
-        *o = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lse && lane == 0) *lse = -INFINITY;
-        return;
-    }
-    const int64_t N = p.unit_off[U];
-    const int64_t P = p.num_ctas;
-    const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
-    const int nslots = (i1 - i0 + 1) * NC;
-    const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
-    auto slot_of = [&](int s) -> const float* {
-        const int i = i0 + s / NC, w = s - (s / NC) * NC;
-        if (range_begin(N, P, i) == range_begin(N, P, i + 1)) return nullptr;   // idle CTA
-        return p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
-    };
-    float M = -INFINITY;
-    for (int s = lane; s < nslots; s += 32) {
-        const float* sl = slot_of(s);
-        if (sl) M = fmaxf(M, sl[G * kHeadDim + n]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int base = 0; base < nslots; base += 32) {
-        const int s = base + lane;
-        float wgt = 0.f;
-        if (s < nslots && M != -INFINITY) {
-            const float* sl = slot_of(s);
-            if (sl) {
-                const float m = sl[G * kHeadDim + n];
-                if (m != -INFINITY) {
-                    wgt = exp2f(m - M);
-                    L = fmaf(wgt, sl[G * (kHeadDim + 1) + n], L);
-                }
-            }
-        }
-        const int cnt = min(32, nslots - base);
-#pragma unroll 4
-        for (int k = 0; k < cnt; ++k) {
-            const float wk = __shfl_sync(0xffffffffu, wgt, k);
-            if (wk == 0.f) continue;                      // same value on every lane
-            const float4 v =
-                *(reinterpret_cast<const float4*>(slot_of(base + k) + n * kHeadDim) + lane);
-            a.x = fmaf(wk, v.x, a.x);
-            a.y = fmaf(wk, v.y, a.y);
-            a.z = fmaf(wk, v.z, a.z);
-            a.w = fmaf(wk, v.w, a.w);
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    const bool empty = !(L > 0.f);        // only if every tile was rejected as out of range
-    const float inv = empty ? 0.f : 1.f / L;
-    *o = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
-    if (lse && lane == 0) *lse = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
 }
 
 }  // namespace
@@ -443,7 +476,7 @@ __global__ void __launch_bounds__(32 * kMaxGroup) combine_kernel(const DecodePar
 size_t decode_smem_bytes(int units) {
     return 1024 /* alignment slack */ + static_cast<size_t>(STAGES) * kStageBytes +
            2 * STAGES * sizeof(uint64_t) + STAGES * sizeof(int) +
-           (kThreads / 32 + 1) * sizeof(int) + static_cast<size_t>(units + 1) * sizeof(int);
+           (kThreads / 32 + 1 + 2) * sizeof(int) + static_cast<size_t>(units + 1) * sizeof(int);
 }
 
 namespace {
@@ -502,11 +535,8 @@ cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map
         e = ensure_smem(dev, smem);
     }
     if (e != cudaSuccess) return e;
-    sparse_decode_kernel<<<p.num_ctas, kThreads, smem, s>>>(k_map, v_map, p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    combine_kernel<<<U, 32 * p.group, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(sparse_decode_kernel, dim3(p.num_ctas), dim3(kThreads), smem, s, k_map,
+                      v_map, p);
 }
 
 }  // namespace spot

@@ -29,6 +29,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------------- PDL
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor on the stream is still
+// running; pdl_wait() blocks until the predecessor has completed and its
+// writes are visible (a no-op for kernels launched the ordinary way), and
+// pdl_trigger() lets the successor start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

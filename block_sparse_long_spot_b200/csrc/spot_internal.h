@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/spot.h"
 
 namespace spot {
@@ -16,7 +18,7 @@ constexpr int kBlock = 64;
 constexpr int kSelDim = 64;
 constexpr int kMaxGroup = 8;           // query heads per KV head (mma N = 8)
 constexpr int kMaxUnits = 4096;        // batch * num_kv_heads
-constexpr int kMaxBlocks = 16384;      // blocks per sequence
+constexpr int kMaxBlocks = 8192;       // blocks per sequence (512K tokens)
 constexpr int kStatusBytes = 256;      // workspace header
 
 // Status bits OR-ed into the workspace status word by kernels.
@@ -33,7 +35,7 @@ constexpr int kStageBytes = 2 * kBlock * kHeadDim * 2;   // 32768
 constexpr int kPartialFloatsPerHead = kHeadDim + 4;
 
 struct Layout {
-    size_t status, scores, unit_off, partials, total;
+    size_t status, scores, unit_done, partials, total;
     int grid;                           // persistent CTAs of the decode kernel
 };
 
@@ -75,7 +77,7 @@ struct DecodeParams {
     const int32_t* sel_cnt;
     int32_t max_blocks, batch, num_q_heads, num_kv_heads, group, num_pages;
     float scale_log2;                   // softmax_scale * log2(e)
-    int32_t* unit_off;                  // [U + 1] written by CTA 0
+    uint32_t* unit_done;                // [U] arrival counters, zero between calls
     float* partials;
     int32_t num_ctas;
     float* out;
@@ -95,6 +97,24 @@ struct AppendParams {
     int32_t n, num_kv_heads, num_pages, fmt;
     uint32_t* status;
 };
+
+// Launch with programmatic stream serialisation (the kernel must call
+// pdl_wait() before touching anything its predecessor writes).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 cudaError_t launch_scores(const ScoreParams& p, int fmt, cudaStream_t s);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t s);

@@ -26,7 +26,7 @@
  *     recorded and the access is skipped.
  *   - Shapes this build supports: head_dim 128, block_size 64 (one KV page
  *     per block), sel_dim 64, 1 <= num_q_heads / num_kv_heads <= 8,
- *     batch * num_kv_heads <= 4096, max_blocks <= 16384.  Other shapes
+ *     batch * num_kv_heads <= 4096, max_blocks <= 8192 (512K tokens).  Other shapes
  *     return SPOT_ERR_UNSUPPORTED.
  *   - Alignment: bf16 arrays, the selector data plane and `out` 16 bytes,
  *     the KV pools and the workspace 256 bytes, everything else 4 bytes.

@@ -247,6 +247,26 @@ def test_p_one_is_dense_attention_and_p_zero_keeps_reserved():
     assert (gpu["sel_cnt"] == 1 + 4).all()
 
 
+def test_heavy_ties_in_the_cut():
+    # All scores equal (q_sel = 0): one tie group of 507 residual blocks; the
+    # cut takes the lowest block indices.  Then four score levels from one
+    # selector-query dimension: tie groups of ~70-300 blocks at the cut.
+    wl = workloads.make("qwen3_4b_32k", seed=9, device=DEV, integer=True, batch=2)
+    wl.q_sel.zero_()
+    for p in (0.3, 0.5, 0.77):
+        wl.top_p = torch.full((2,), p, device=DEV)
+        gpu = run_gpu(wl, kmin=0)
+        ora = run_oracle(wl, kmin=0)
+        _assert_same_selection(gpu, ora, wl)
+    wl.q_sel[:, :, 0] = 1.0
+    wl.top_p = safe_top_p(wl)
+    for kw in (dict(kmin=0), dict(kmin=300), dict(mode="topk", topk=200)):
+        gpu = run_gpu(wl, **kw)
+        ora = run_oracle(wl, **kw)
+        _assert_same_selection(gpu, ora, wl)
+        check_outputs(gpu, ora, wl)
+
+
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (12, 4), (16, 2), (8, 8)])
 def test_group_sizes(hq, hkv):
     wl = workloads.make("qwen3_4b_32k", seed=7, device=DEV, seq_len=2048 + 64 * 3, batch=3,
