@@ -93,8 +93,7 @@ bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Lay
     L.unit_done = off;
     off = round_up(off + static_cast<size_t>(U) * sizeof(uint32_t), 256);
     L.partials = off;
-    off = round_up(off + static_cast<size_t>(grid + U) * kDecodeConsumers * G *
-                             kPartialFloatsPerHead * sizeof(float),
+    off = round_up(off + static_cast<size_t>(grid + U) * G * kPartialFloatsPerHead * sizeof(float),
                    256);
     L.total = off;
     *out = L;

@@ -81,8 +81,8 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
     if (grid <= 0) return SPOT_ERR_CUDA;
     const size_t off_units = kStatusBytes;
     const size_t off_partials = round256(off_units + static_cast<size_t>(U) * sizeof(uint32_t));
-    const size_t need = off_partials + static_cast<size_t>(grid + U) * kDecodeConsumers * G *
-                                           kPartialFloatsPerHead * sizeof(float);
+    const size_t need =
+        off_partials + static_cast<size_t>(grid + U) * G * kPartialFloatsPerHead * sizeof(float);
     if (need > kNoAllocScratchBytes) return SPOT_ERR_WORKSPACE;
 
     int dev = 0;

@@ -21,7 +21,8 @@
 //   S^T[64 tok x 8 heads] = K[64 x 128] . Q^T        (mma m16n8k16, bf16)
 //   online softmax over tokens (exp2, scale folded into log2 domain)
 //   O^T[128 x 8] += V^T[128 x 64] . P^T[64 x 8]      (P^T via movmatrix)
-// Each warp writes its own partial (acc[G][128], m[G], l[G]).
+// At the end of a unit's segment the NC warps merge their states in shared
+// memory and the CTA writes one partial (acc[G][128], m[G], l[G]).
 #include <math.h>
 #include <stdio.h>
 
@@ -74,60 +75,66 @@ __device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
 
 // Merge the partials of query head n of unit u (blocks [lo, hi) of the
 // flattened list) and write out / lse.  One warp; lane l owns head
-// dimensions 4l..4l+3.  The partials are those of the NC warps of every CTA
-// whose range touched the unit; other CTAs of this launch wrote them, so they
-// are read through L2 (ld.global.cg).
+// dimensions 4l..4l+3.  The partials are one per CTA whose range touched the
+// unit; other CTAs of this launch wrote them, so they are read through L2
+// (ld.global.cg).  Slots are taken 32 at a time with an online rescale, and
+// the accumulator loads of 8 slots are issued together.
 __device__ void merge_unit_head(const DecodeParams& p, int u, int n, int lo, int hi, int64_t N,
                                 int64_t P, int lane) {
     const int G = p.group;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
     const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
     const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
-    const int nslots = (i1 - i0 + 1) * NC;
+    const int nslots = i1 - i0 + 1;
     const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
     const bool some_idle = N < P;          // only then can a CTA own no blocks
-    auto slot_of = [&](int sidx) -> const float* {
-        const int i = i0 + sidx / NC, w = sidx % NC;
-        if (some_idle && range_begin(N, P, i) == range_begin(N, P, i + 1)) return nullptr;
-        return p.partials + (static_cast<int64_t>(i + u) * NC + w) * stride;
-    };
-    float M = -INFINITY;
-    for (int sidx = lane; sidx < nslots; sidx += 32) {
-        const float* sl = slot_of(sidx);
-        if (sl) M = fmaxf(M, __ldcg(sl + G * kHeadDim + n));
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
+    float M = -INFINITY, L = 0.f;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int base = 0; base < nslots; base += 32) {
-        const int sidx = base + lane;
-        float wgt = 0.f;
-        if (sidx < nslots && M != -INFINITY) {
-            const float* sl = slot_of(sidx);
-            if (sl) {
-                const float m = __ldcg(sl + G * kHeadDim + n);
-                if (m != -INFINITY) {
-                    wgt = exp2f(m - M);
-                    L = fmaf(wgt, __ldcg(sl + G * (kHeadDim + 1) + n), L);
-                }
+        const int i = i0 + base + lane;
+        float m = -INFINITY, l = 0.f;
+        if (base + lane < nslots &&
+            !(some_idle && range_begin(N, P, i) == range_begin(N, P, i + 1))) {
+            const float* sl = p.partials + static_cast<int64_t>(i + u) * stride;
+            m = __ldcg(sl + G * kHeadDim + n);
+            l = __ldcg(sl + G * (kHeadDim + 1) + n);
+        }
+        float cm = m;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+        const float nm = fmaxf(M, cm);
+        if (nm == -INFINITY) continue;
+        const float sc = (M == -INFINITY) ? 0.f : exp2f(M - nm);
+        L *= sc;
+        a.x *= sc; a.y *= sc; a.z *= sc; a.w *= sc;
+        M = nm;
+        const float wgt = (m == -INFINITY) ? 0.f : exp2f(m - M);
+        float wl = wgt * l;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, off);
+        L += wl;
+        const int cnt = min(32, nslots - base);
+        for (int k0 = 0; k0 < cnt; k0 += 8) {
+            float wk[8];
+            float4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                wk[k] = __shfl_sync(0xffffffffu, wgt, (k0 + k) & 31);
+                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (k0 + k < cnt && wk[k] != 0.f)
+                    v[k] = __ldcg(reinterpret_cast<const float4*>(
+                                      p.partials + static_cast<int64_t>(i0 + base + k0 + k + u) *
+                                                       stride + n * kHeadDim) + lane);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                a.x = fmaf(wk[k], v[k].x, a.x);
+                a.y = fmaf(wk[k], v[k].y, a.y);
+                a.z = fmaf(wk[k], v[k].z, a.z);
+                a.w = fmaf(wk[k], v[k].w, a.w);
             }
         }
-        const int cnt = min(32, nslots - base);
-#pragma unroll 4
-        for (int k = 0; k < cnt; ++k) {
-            const float wk = __shfl_sync(0xffffffffu, wgt, k);
-            if (wk == 0.f) continue;                      // same value on every lane
-            const float4 v =
-                __ldcg(reinterpret_cast<const float4*>(slot_of(base + k) + n * kHeadDim) + lane);
-            a.x = fmaf(wk, v.x, a.x);
-            a.y = fmaf(wk, v.y, a.y);
-            a.z = fmaf(wk, v.z, a.z);
-            a.w = fmaf(wk, v.w, a.w);
-        }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
     const bool empty = !(L > 0.f);        // only if every tile was rejected as out of range
     const float inv = empty ? 0.f : 1.f / L;
     reinterpret_cast<float4*>(p.out + h * kHeadDim)[lane] =
@@ -148,7 +155,9 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* base = smem_raw + pad;
-    uint8_t* tail = base + STAGES * kStageBytes;
+    float* red_acc = reinterpret_cast<float*>(base + STAGES * kStageBytes);   // [NC][8][132]
+    float* red_ml = red_acc + NC * kMaxGroup * kPartialFloatsPerHead;          // [NC][8][2]
+    uint8_t* tail = reinterpret_cast<uint8_t*>(red_ml + NC * kMaxGroup * 2);
     uint64_t* full = reinterpret_cast<uint64_t*>(tail);
     uint64_t* empty = full + STAGES;
     int* valid = reinterpret_cast<int*>(empty + STAGES);
@@ -420,35 +429,61 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
             if (lane == 0) mbar_arrive(&empty[s]);
         }
 
-        // ---- this warp's partial for unit u
+        // ---- merge the NC warps' states for unit u inside the CTA, then
+        // write the CTA's partial (one slot per CTA and unit)
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             l0 += __shfl_xor_sync(0xffffffffu, l0, o);
             l1 += __shfl_xor_sync(0xffffffffu, l1, o);
         }
-        float* slot = p.partials + (static_cast<int64_t>(blockIdx.x + u) * NC + warp) *
-                                       (static_cast<int64_t>(G) * kPartialFloatsPerHead);
-        const int h0 = 2 * c4, h1 = 2 * c4 + 1;
+        {
+            float* ra = red_acc + warp * kMaxGroup * kPartialFloatsPerHead;
+            const int h0 = 2 * c4, h1 = 2 * c4 + 1;
 #pragma unroll
-        for (int md = 0; md < 8; ++md) {
-            const int d0 = md * 16 + r8, d1 = d0 + 8;
-            if (h0 < G) {
-                slot[h0 * kHeadDim + d0] = acc[md][0];
-                slot[h0 * kHeadDim + d1] = acc[md][2];
+            for (int md = 0; md < 8; ++md) {
+                const int d0 = md * 16 + r8, d1 = d0 + 8;
+                if (h0 < G) {
+                    ra[h0 * kPartialFloatsPerHead + d0] = acc[md][0];
+                    ra[h0 * kPartialFloatsPerHead + d1] = acc[md][2];
+                }
+                if (h1 < G) {
+                    ra[h1 * kPartialFloatsPerHead + d0] = acc[md][1];
+                    ra[h1 * kPartialFloatsPerHead + d1] = acc[md][3];
+                }
             }
-            if (h1 < G) {
-                slot[h1 * kHeadDim + d0] = acc[md][1];
-                slot[h1 * kHeadDim + d1] = acc[md][3];
+            if (r8 == 0) {
+                float* ml = red_ml + warp * kMaxGroup * 2;
+                if (h0 < G) { ml[2 * h0] = m0; ml[2 * h0 + 1] = l0; }
+                if (h1 < G) { ml[2 * h1] = m1; ml[2 * h1 + 1] = l1; }
             }
         }
-        if (r8 == 0) {
-            if (h0 < G) {
-                slot[G * kHeadDim + h0] = m0;
-                slot[G * (kHeadDim + 1) + h0] = l0;
-            }
-            if (h1 < G) {
-                slot[G * kHeadDim + h1] = m1;
-                slot[G * (kHeadDim + 1) + h1] = l1;
+        consumer_barrier();
+        {
+            float* slot = p.partials + static_cast<int64_t>(blockIdx.x + u) *
+                                           (static_cast<int64_t>(G) * kPartialFloatsPerHead);
+            for (int n = warp; n < G; n += NC) {
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NC; ++w) M = fmaxf(M, red_ml[(w * kMaxGroup + n) * 2]);
+                float L = 0.f;
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int w = 0; w < NC; ++w) {
+                    const float m = red_ml[(w * kMaxGroup + n) * 2];
+                    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+                    L = fmaf(f, red_ml[(w * kMaxGroup + n) * 2 + 1], L);
+                    const float4 v = reinterpret_cast<const float4*>(
+                        red_acc + (w * kMaxGroup + n) * kPartialFloatsPerHead)[lane];
+                    a.x = fmaf(f, v.x, a.x);
+                    a.y = fmaf(f, v.y, a.y);
+                    a.z = fmaf(f, v.z, a.z);
+                    a.w = fmaf(f, v.w, a.w);
+                }
+                reinterpret_cast<float4*>(slot + n * kHeadDim)[lane] = a;
+                if (lane == 0) {
+                    slot[G * kHeadDim + n] = M;
+                    slot[G * (kHeadDim + 1) + n] = L;
+                }
             }
         }
         __threadfence();                 // the partial is visible GPU-wide ...
@@ -475,6 +510,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
 
 size_t decode_smem_bytes(int units) {
     return 1024 /* alignment slack */ + static_cast<size_t>(STAGES) * kStageBytes +
+           NC * kMaxGroup * (kPartialFloatsPerHead + 2) * sizeof(float) +
            2 * STAGES * sizeof(uint64_t) + STAGES * sizeof(int) +
            (kThreads / 32 + 1 + 2) * sizeof(int) + static_cast<size_t>(units + 1) * sizeof(int);
 }

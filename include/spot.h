@@ -199,8 +199,8 @@ spot_status_t spot_decode_step(const spot_layer_desc_t* desc, const spot_select_
  *     the device current (cudaGetSymbolAddress) and remembers it; make that
  *     first call before any stream capture.
  *   - A shape whose scratch exceeds 8 MiB returns SPOT_ERR_WORKSPACE (about
- *     (grid + U) * 4 * G * 528 bytes with U = batch * num_kv_heads and grid
- *     = the SM count; e.g. 256 units of G = 4 need 3.4 MB).
+ *     (grid + U) * G * 528 bytes with U = batch * num_kv_heads and grid =
+ *     the SM count; e.g. 256 units of G = 4 need 0.9 MB).
  *   - All calls share the one array and it keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other host threads) race
  *     and must be serialised by the caller.
