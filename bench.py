@@ -39,6 +39,24 @@ import workloads  # noqa: E402
 
 HBM_FALLBACK_GBS = 6650.0
 
+# DRAM bytes (read + write) of one sparse-decode launch from an ncu capture of
+# the same workload (profiles/sparse_decode_kernel_qwen3_32b_128k.md), valid
+# only for the kernel source it was taken on (sha256 prefix of the .cu file).
+NCU_TRAFFIC = {
+    "qwen3_32b_128k": {"bytes": 728988416 + 3467264, "kernel_sha256": "80f7ea5c959e94c5"},
+}
+
+
+def measured_traffic(workload: str):
+    import hashlib
+    rec = NCU_TRAFFIC.get(workload)
+    if rec is None:
+        return None
+    src = os.path.join(ROOT, "block_sparse_long_spot_b200", "csrc", "sparse_decode.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    return rec["bytes"] if sha == rec["kernel_sha256"] else None
+
 
 def peaks():
     try:
@@ -326,7 +344,7 @@ def run_spot(args, world, rank, local):
         "roofline": {
             "bound": "hbm", "kernel": "sparse decode (attention + combine)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.workload),
             "peak_source": peak_kind,
             "algorithmic_bytes_per_launch": int(b_sparse), "ms_per_launch": round(dec_ms, 5),
         },
@@ -340,7 +358,7 @@ def run_spot(args, world, rank, local):
                 "ms_per_step": round(ms_e2e, 5),
                 "h2d_bytes_per_step": int(layers[0][0].q.numel() * 2 + layers[0][0].q_sel.numel() * 2),
                 "d2h_bytes_per_step": int(out.numel() * 4)},
-        "gpu_launches": K * 4,
+        "gpu_launches": K * 3,          # score, select, sparse decode per step
         "clocks": clk.summary(),
     }
     return res, layers

@@ -204,6 +204,8 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 
 constexpr int kNB = 1024;              // value buckets of the first pass
 constexpr float kBucketScale = 32.f;    // buckets per unit of score below the maximum
+constexpr int kApproxShift = 18;        // bucket masses for the search: 2^-18 fixed point
+                                        // (<= 8192 elements of mass <= 1 fit in 32 bits)
 constexpr int NT = kSelectThreads;
 constexpr int NW = NT / 32;
 
@@ -212,7 +214,7 @@ struct SelSmem {
     unsigned long long* mass;     // [max_blocks] fixed-point exp(s - max)
     uint16_t* vb;                 // [max_blocks] value bucket (0 = the top scores)
     uint8_t* keep;                // [max_blocks] 1 keep, 2 tie at the cut, 0 drop
-    float* hmass;                 // [kNB] approximate (fp32) mass per bucket
+    uint32_t* hmass;              // [kNB] approximate mass per bucket, 2^-18 fixed point
     uint32_t* hcnt;               // [kNB] exact count per bucket
     uint32_t* ckey;               // [NT] candidates of the cut bucket: key
     int* cidx;                    //      element index
@@ -278,7 +280,7 @@ __device__ int cut_bucket(const SelSmem& sm, double target, bool by_mass, int* b
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
         const int bkt = threadIdx.x * PER + k;
-        loc += by_mass ? sm.hmass[bkt] : static_cast<float>(sm.hcnt[bkt]);
+        loc += static_cast<float>(by_mass ? sm.hmass[bkt] : sm.hcnt[bkt]);
         cnt += sm.hcnt[bkt];
         if (sm.hcnt[bkt]) last = bkt;
     }
@@ -292,7 +294,7 @@ __device__ int cut_bucket(const SelSmem& sm, double target, bool by_mass, int* b
     int crun = cbase;
     for (int k = 0; k < PER; ++k) {
         const int bkt = threadIdx.x * PER + k;
-        const float v = by_mass ? sm.hmass[bkt] : static_cast<float>(sm.hcnt[bkt]);
+        const float v = static_cast<float>(by_mass ? sm.hmass[bkt] : sm.hcnt[bkt]);
         const bool hit = by_mass ? (run < target && run + v >= target)
                                  : (crun < target && crun + static_cast<int>(sm.hcnt[bkt]) >= target);
         if (hit && sm.hcnt[bkt]) {
@@ -327,8 +329,46 @@ struct Cut {
 __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long long above,
                               unsigned long long target, bool by_mass) {
     const int c = static_cast<int>(sm.hcnt[b]);
-    if (threadIdx.x == 0) { sm.misc[3] = 0; sm.misc[4] = c - 1; }
-    __syncthreads();
+    // (the caller has set sm.misc[3] = 0 before its last barrier)
+    if (c <= 32) {
+        for (int i = threadIdx.x; i < n; i += NT) {
+            if (sm.vb[i] == b) {
+                const int slot = atomicAdd(&sm.misc[3], 1);
+                sm.ckey[slot] = sm.keys[i];
+                sm.cidx[slot] = i;
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {                       // one warp ranks the few candidates
+            const int lane = threadIdx.x;
+            int rank = 0, j = -1;
+            if (lane < c) {
+                const uint32_t k = sm.ckey[lane];
+                j = sm.cidx[lane];
+                for (int d = 0; d < c; ++d) {
+                    const uint32_t kd = sm.ckey[d];
+                    rank += (kd > k) || (kd == k && sm.cidx[d] < j);
+                }
+                sm.cval[rank] = by_mass ? sm.mass[j] : 1ull;
+            }
+            __syncwarp();
+            const unsigned long long v = lane < c ? sm.cval[lane] : 0ull;
+            unsigned long long incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long x = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += x;
+            }
+            const bool hit = lane < c && above + incl - v < target && above + incl >= target;
+            const unsigned hm = __ballot_sync(0xffffffffu, hit);
+            const int r_cut = hm ? __ffs(hm) - 1 : c - 1;
+            if (lane < c) sm.keep[j] = rank <= r_cut ? 1 : 0;
+            if (lane == 0) sm.misc[4] = r_cut;
+        }
+        __syncthreads();
+        return sm.misc[4] + 1;
+    }
+    if (threadIdx.x == 0) sm.misc[4] = c - 1;
     if (c <= NT) {
         for (int i = threadIdx.x; i < n; i += NT) {
             if (sm.vb[i] == b) {
@@ -413,7 +453,7 @@ __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long lon
 size_t select_smem_bytes(int max_blocks) {
     return static_cast<size_t>(max_blocks) *
                (sizeof(uint32_t) + sizeof(unsigned long long) + sizeof(uint16_t) + 1) +
-           kNB * (sizeof(float) + sizeof(uint32_t)) +
+           kNB * (sizeof(uint32_t) + sizeof(uint32_t)) +
            NT * (sizeof(uint32_t) + sizeof(int) + sizeof(unsigned long long)) +
            3 * NW * sizeof(unsigned long long) + 8 * sizeof(int) +
            2 * (NW + 1) * sizeof(int) + 128;
@@ -434,8 +474,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
         q += sizeof(unsigned long long) * 3 * NW;
         sm.keys = reinterpret_cast<uint32_t*>(q);
         q += sizeof(uint32_t) * p.max_blocks;
-        sm.hmass = reinterpret_cast<float*>(q);
-        q += sizeof(float) * kNB;
+        sm.hmass = reinterpret_cast<uint32_t*>(q);
+        q += sizeof(uint32_t) * kNB;
         sm.hcnt = reinterpret_cast<uint32_t*>(q);
         q += sizeof(uint32_t) * kNB;
         sm.ckey = reinterpret_cast<uint32_t*>(q);
@@ -473,7 +513,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
     const int n = r1 - r0;
     const int n_reserved = nb - n;
     const float* s = p.scores + static_cast<int64_t>(u) * p.max_blocks;
-    for (int i = threadIdx.x; i < kNB; i += NT) { sm.hmass[i] = 0.f; sm.hcnt[i] = 0u; }
+    for (int i = threadIdx.x; i < kNB; i += NT) { sm.hmass[i] = 0u; sm.hcnt[i] = 0u; }
     if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
     pdl_trigger();
     pdl_wait();                                       // scores of the scoring kernel
@@ -504,7 +544,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
         const int bkt = static_cast<int>(fminf((smax_f - v) * kBucketScale, kNB - 1.f));
         sm.vb[i] = static_cast<uint16_t>(bkt);
         atomicAdd(&sm.hcnt[bkt], 1u);
-        atomicAdd(&sm.hmass[bkt], static_cast<float>(e));
+        atomicAdd(&sm.hmass[bkt], static_cast<uint32_t>(ldexp(e, kApproxShift) + 0.5));
         zloc += f;
     }
     unsigned long long Z = zloc, d1 = 0, d2 = 0;
@@ -526,7 +566,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
             ceil(static_cast<double>(p.top_p[b]) * static_cast<double>(Z)));
         T = T < 1ull ? 1ull : (T > Z ? Z : T);
         int before;
-        int bk = cut_bucket(sm, ldexp(static_cast<double>(T), -kFixShift), true, &before);
+        int bk = cut_bucket(sm, ldexp(static_cast<double>(T), kApproxShift - kFixShift), true,
+                            &before);
         // exact check of the bucket on the fixed-point masses; step to the
         // neighbouring non-empty bucket while the fp32 estimate was off
         unsigned long long A, Bm, Ac;
@@ -547,6 +588,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
             if (nbk < 0 || nbk >= kNB) break;
             bk = nbk;
         }
+        if (threadIdx.x == 0) sm.misc[3] = 0;
         for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
         __syncthreads();
         n_take = static_cast<int>(Ac) + resolve_bucket(sm, n, bk, A, T, true);
@@ -568,6 +610,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
         } else {
             int before;
             const int bk = cut_bucket(sm, static_cast<double>(n_take), false, &before);
+            if (threadIdx.x == 0) sm.misc[3] = 0;
             for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
             __syncthreads();
             resolve_bucket(sm, n, bk, static_cast<unsigned long long>(before),
