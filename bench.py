@@ -198,7 +198,9 @@ def run_spot(args, world, rank, local):
     fmt = args.sel_fmt
     layers = []
     for l in range(args.layers):
-        wl = workloads.make(args.workload, seed=layer_seed(rank, l), device=dev, sel_fmt=fmt)
+        # layers of one model share sequence lengths and page tables
+        wl = workloads.make(args.workload, seed=layer_seed(rank, l), device=dev, sel_fmt=fmt,
+                            structure_from=layers[0][0] if layers else None)
         desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, fmt)
         if fmt == "bf16":
             data, scales = wl.sel_keys, None

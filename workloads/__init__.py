@@ -121,10 +121,13 @@ def _int_bf16(shape, gen, device, lo=-3, hi=3):
 
 
 def make(name: str, seed: int = 0, device="cpu", *, seq_len=None, batch=None, sel_fmt=None,
-         integer: bool = False, top_p=None, max_blocks=None, **spec_overrides) -> Workload:
+         integer: bool = False, top_p=None, max_blocks=None, structure_from=None,
+         **spec_overrides) -> Workload:
     """Build a seeded workload.  Overrides shrink a spec for oracle-sized
     runs (seq_len, batch) or switch its selector format; integer=True draws
-    selector queries and keys from {-3..3} (exact scores in any precision)."""
+    selector queries and keys from {-3..3} (exact scores in any precision).
+    structure_from=<Workload> reuses that workload's sequence lengths, page
+    table and top-p (another layer of the same model) and draws new data."""
     spec = dataclasses.replace(SPECS[name], **spec_overrides)
     if seq_len is not None:
         spec = dataclasses.replace(spec, seq_len=seq_len)
@@ -140,7 +143,9 @@ def make(name: str, seed: int = 0, device="cpu", *, seq_len=None, batch=None, se
     gen.manual_seed(seed)
 
     B, Hq, Hkv = spec.batch, spec.num_q_heads, spec.num_kv_heads
-    if spec.seq_len is None:
+    if structure_from is not None:
+        lens = structure_from.seq_lens.cpu().numpy().astype(np.int64)
+    elif spec.seq_len is None:
         lo, hi = spec.ragged_range
         lens = rng.integers(lo // BLOCK, hi // BLOCK + 1, size=B) * BLOCK
     else:
@@ -154,8 +159,13 @@ def make(name: str, seed: int = 0, device="cpu", *, seq_len=None, batch=None, se
     for b in range(B):
         pt[b, :nbs[b]] = pages[off:off + nbs[b]]
         off += nbs[b]
+    if structure_from is not None:
+        pt = structure_from.page_table.cpu().numpy()
+        num_pages = structure_from.num_pages
 
-    if spec.top_p_choices:
+    if structure_from is not None:
+        p = structure_from.top_p.cpu().numpy()
+    elif spec.top_p_choices:
         p = rng.choice(np.asarray(spec.top_p_choices, np.float32), size=B)
     else:
         p = np.full(B, spec.top_p, np.float32)
