@@ -82,6 +82,8 @@ def lib():
         L.spot_sparse_decode_noalloc.argtypes = [P, P, P, P, P, i32, P, P, P, i32, i32, f32, P,
                                                  P, P]
         L.spot_read_device_status.argtypes = [P, P]
+        L.spot_check_wait_timeout.argtypes = [P, P]
+        L.spot_check_wait_timeout.restype = ctypes.c_int
         L.spot_status_string.restype = ctypes.c_char_p
         for name in ("spot_append_selector_keys", "spot_select", "spot_sparse_decode",
                      "spot_decode_step", "spot_read_device_status",
@@ -204,6 +206,13 @@ def decode_step(desc: LayerDesc, params: SelectParams, q_sel, w, sel_data, sel_s
         _ptr(lse, torch.float32, "lse"), _ptr(workspace, name="workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "decode_step")
+
+
+def check_wait_timeout(workspace, stream=None):
+    """Run the failure-path check kernel (a wait nothing satisfies); the
+    timeout is then visible through read_device_status."""
+    _check(lib().spot_check_wait_timeout(_ptr(workspace, name="workspace"), _stream(stream)),
+           "check_wait_timeout")
 
 
 def read_device_status(workspace, stream=None) -> int:

@@ -219,6 +219,14 @@ spot_status_t spot_sparse_decode_noalloc(const spot_layer_desc_t* desc, const ui
  * SPOT_ERR_DEVICE_TIMEOUT; bounds wins if both), and clear it. */
 spot_status_t spot_read_device_status(void* workspace, void* stream);
 
+/* Failure-path check: launches one kernel whose bounded wait on an mbarrier
+ * can never complete (nothing arrives on it).  After the wait limit (about
+ * one second of the GPU's global timer) the kernel records
+ * SPOT_ERR_DEVICE_TIMEOUT in the status word of `status_ws` (a workspace)
+ * and returns; spot_read_device_status then reports it and the context stays
+ * usable.  The library's pipelines use the same bounded wait everywhere. */
+spot_status_t spot_check_wait_timeout(void* status_ws, void* stream);
+
 /* Static string for a status code. */
 const char* spot_status_string(spot_status_t status);
 

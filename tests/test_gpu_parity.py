@@ -2,6 +2,7 @@
 oracle, on the seeded workloads of the SpotAttention decode configurations
 and on edge cases.  Rules and tolerances: tests/harness.py."""
 import math
+import time
 
 import numpy as np
 import pytest
@@ -303,6 +304,19 @@ def test_bad_page_id_is_reported_not_faulted():
     # the context is still usable
     wl2 = workloads.make("tiny_4k", seed=0, device=DEV)
     assert run_gpu(wl2)["status"] == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    # A wait that nothing satisfies gives up after about a second, records
+    # SPOT_ERR_DEVICE_TIMEOUT (6) and the context keeps working.
+    ws = torch.zeros(4096, dtype=torch.uint8, device=DEV)
+    t0 = time.time()
+    spot.check_wait_timeout(ws)
+    assert spot.read_device_status(ws) == 6
+    assert 0.5 < time.time() - t0 < 30
+    assert spot.read_device_status(ws) == 0          # read clears it
+    wl = workloads.make("tiny_4k", seed=0, device=DEV)
+    assert run_gpu(wl)["status"] == 0
 
 
 def test_workspace_too_small_and_bad_arguments():
