@@ -88,8 +88,6 @@ bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Lay
     size_t off = 0;
     L.status = off;
     off += kStatusBytes;
-    L.scores = off;
-    off = round_up(off + static_cast<size_t>(U) * max_blocks * sizeof(float), 256);
     L.unit_done = off;
     off = round_up(off + static_cast<size_t>(U) * sizeof(uint32_t), 256);
     L.partials = off;
@@ -114,32 +112,22 @@ spot_status_t do_select(const spot_layer_desc_t* d, const spot_select_params_t* 
                         size_t ws_bytes, const Layout& L, cudaStream_t s) {
     (void)ws_bytes;
     uint8_t* base = static_cast<uint8_t*>(ws);
-    ScoreParams sp;
-    sp.q_sel = q_sel;
-    sp.w = w;
-    sp.sel_data = sel_data;
-    sp.sel_scales = sel_scales;
-    sp.page_table = page_table;
-    sp.pt_stride = pt_stride;
-    sp.seq_lens = seq_lens;
-    sp.batch = batch;
-    sp.num_q_heads = d->num_q_heads;
-    sp.num_kv_heads = d->num_kv_heads;
-    sp.group = d->num_q_heads / d->num_kv_heads;
-    sp.num_pages = d->num_pages;
-    sp.max_blocks = max_blocks;
-    sp.inv_temp = 1.0f / pr->temperature;
-    sp.scores = reinterpret_cast<float*>(base + L.scores);
-    sp.status = reinterpret_cast<uint32_t*>(base + L.status);
-    if (launch_scores(sp, d->sel_fmt, s) != cudaSuccess) return SPOT_ERR_CUDA;
     SelectParams sl;
-    sl.scores = sp.scores;
+    sl.q_sel = q_sel;
+    sl.w = w;
+    sl.sel_data = sel_data;
+    sl.sel_scales = sel_scales;
+    sl.page_table = page_table;
+    sl.pt_stride = pt_stride;
     sl.seq_lens = seq_lens;
     sl.top_p = top_p;
-    sl.pt_stride = pt_stride;
     sl.batch = batch;
+    sl.num_q_heads = d->num_q_heads;
     sl.num_kv_heads = d->num_kv_heads;
+    sl.group = d->num_q_heads / d->num_kv_heads;
+    sl.num_pages = d->num_pages;
     sl.max_blocks = max_blocks;
+    sl.inv_temp = 1.0f / pr->temperature;
     sl.mode = pr->mode;
     sl.sink_blocks = pr->sink_blocks;
     sl.recency_blocks = pr->recency_blocks;
@@ -147,8 +135,8 @@ spot_status_t do_select(const spot_layer_desc_t* d, const spot_select_params_t* 
     sl.topk_blocks = pr->topk_blocks;
     sl.sel_idx = sel_idx;
     sl.sel_cnt = sel_cnt;
-    sl.status = sp.status;
-    if (launch_select(sl, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    sl.status = reinterpret_cast<uint32_t*>(base + L.status);
+    if (launch_select(sl, d->sel_fmt, s) != cudaSuccess) return SPOT_ERR_CUDA;
     return SPOT_OK;
 }
 

@@ -1,26 +1,27 @@
 // select.cu -- selector scoring and block selection (SpotAttention §2.1,
-// §2.3 Eq. 6-8).
+// §2.3 Eq. 6-8), one fused kernel with one CTA per (sequence, KV head).
 //
-// score_kernel: s[b,g,j] = (1/tau) sum_{h in group g} w[b,h] ReLU(q_sel[b,h] . k[page(b,j),g])
-//   for every complete block j.  One warp per (sequence, KV head, 16 blocks);
-//   the warps of a CTA cover adjacent KV heads of the same pages (adjacent in
-//   the selector pool).  Each warp computes the 16 x 8 dot
-//   products with bf16 mma.sync (keys as the M operand, the group's selector
-//   queries as N = 8).  INT4 / MXFP4 keys are widened to bf16 in registers
-//   (both code sets are exact in bf16) and the per-32 scales are applied to
-//   the two half-accumulators afterwards, so dequantisation is exact.  The
-//   head dimension is consumed in a permuted order, identical for the keys
-//   and the queries, that lets every lane load 16 contiguous bytes.
+// Scoring: s[j] = (1/tau) sum_{h in group} w[b,h] ReLU(q_sel[b,h] . k[page(b,j),g])
+//   for every complete block j.  Each warp scores tiles of 16 blocks with
+//   bf16 mma.sync (keys as the M operand, the group's selector queries as
+//   N = 8), four tiles at a time so their gathered loads are in flight
+//   together.  INT4 / MXFP4 keys are widened to bf16 in registers (both code
+//   sets are exact in bf16) and the per-32 scales are applied to the two
+//   half-accumulators afterwards, so dequantisation is exact.  The head
+//   dimension is consumed in a permuted order, identical for the keys and the
+//   queries, that lets every lane load 16 contiguous bytes.  Scores stay in
+//   shared memory.
 //
-// select_kernel: one CTA per (sequence, KV head).  Residual softmax masses
-//   exp(s - max) are computed in fp64 and accumulated as 2^-40 fixed-point
-//   integers (exact, order-independent sums).  The nucleus cut is found by a
-//   4-pass radix search over the order-preserving 32-bit keys of the scores:
-//   each pass histograms mass and count of the candidates by the next 8 key
-//   bits and descends into the bucket where the cumulative mass (from the
-//   top) reaches p * Z.  Ties at the cut are taken lowest block index first.
-//   The K_min floor / static top-K use the same radix search on counts.  A
-//   block-wide scan compacts the kept blocks in ascending order.
+// Selection: residual softmax numerators exp(s - max) are computed in fp64
+//   and held as 2^-40 fixed-point integers (exact, order-independent sums).
+//   The nucleus cut is a bucketed threshold search: the residual blocks are
+//   histogrammed into 1024 buckets of the score's distance from the maximum
+//   (monotone in the score; exact counts, 2^-18 fixed-point masses), the
+//   bucket where the cumulative mass from the top reaches p * Z is found by a
+//   block scan and confirmed on the exact fixed-point masses, and the few
+//   blocks inside that bucket are ranked exactly (score descending, lower
+//   block index first).  The K_min floor and static top-K use the same search
+//   on counts.  A block scan compacts the kept blocks in ascending order.
 #include <math.h>
 
 #include "spot_device.cuh"
@@ -29,9 +30,9 @@
 namespace spot {
 namespace {
 
-constexpr int kScoreWarps = 8;
-constexpr int kSelectThreads = 256;
+constexpr int kSelectThreads = 512;
 constexpr int kFixShift = 40;
+constexpr int kTileBatch = 4;           // 16-block tiles a warp scores with loads in flight
 
 // --------------------------------------------------------------- scoring
 
@@ -79,117 +80,134 @@ __device__ __forceinline__ float group_scale(const void* scales, int64_t row, in
     }
 }
 
-template <int FMT>
-__global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(const ScoreParams p) {
-    // One warp per (sequence, KV head, tile of 16 blocks): grid.x tiles,
-    // grid.y groups of kScoreWarps KV heads, grid.z sequences.
-    pdl_trigger();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int b = blockIdx.z;
-    const int g = blockIdx.y * kScoreWarps + warp;
-    if (g >= p.num_kv_heads) return;
-    const int L = max(p.seq_lens[b], 0);
-    int n_full = L / kBlock;
-    if (n_full > p.max_blocks || n_full > p.pt_stride) {
-        if (lane == 0 && blockIdx.x == 0 && g == 0) flag_status(p.status, kStatusBounds);
-        n_full = min(n_full, min(p.max_blocks, p.pt_stride));
-    }
-    const int j0 = blockIdx.x * 16;
-    if (j0 >= n_full) return;
-    const int c4 = lane & 3, r8 = lane >> 2;
-    const int G = p.group;
-    {
-        // ---- B operand: the group's selector queries (lane: head r8)
-        const bool real = r8 < G;
-        const int h = g * G + (real ? r8 : 0);
-        const uint4* qrow = reinterpret_cast<const uint4*>(
-            p.q_sel + (static_cast<int64_t>(b) * p.num_q_heads + h) * kSelDim);
-        uint32_t qw[8];
-        {
-            // bf16 keys: lane c4 owns dims [16 c4, 16 c4 + 16);
-            // 4-bit keys: dims [8 c4, 8 c4 + 8) and [32 + 8 c4, 32 + 8 c4 + 8).
-            uint4 x0, x1;
-            if (FMT == SPOT_SEL_BF16) {
-                x0 = real ? __ldg(qrow + 2 * c4) : make_uint4(0, 0, 0, 0);
-                x1 = real ? __ldg(qrow + 2 * c4 + 1) : make_uint4(0, 0, 0, 0);
-            } else {
-                x0 = real ? __ldg(qrow + c4) : make_uint4(0, 0, 0, 0);
-                x1 = real ? __ldg(qrow + 4 + c4) : make_uint4(0, 0, 0, 0);
-            }
-            qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
-            qw[4] = x1.x; qw[5] = x1.y; qw[6] = x1.z; qw[7] = x1.w;
-        }
-        const float wh0 = (2 * c4 < G)
-            ? (p.w ? p.w[static_cast<int64_t>(b) * p.num_q_heads + g * G + 2 * c4] : 1.f / G) : 0.f;
-        const float wh1 = (2 * c4 + 1 < G)
-            ? (p.w ? p.w[static_cast<int64_t>(b) * p.num_q_heads + g * G + 2 * c4 + 1] : 1.f / G)
-            : 0.f;
 
-        // ---- A operand: keys of blocks j0 + r8 and j0 + r8 + 8
-        const int ja = j0 + r8, jb = j0 + r8 + 8;
+// Scores of tiles t0, t0 + stride, ... (kTileBatch of them) of 16 blocks
+// each, for KV head g of sequence b, into scores[j] (j < n_full).  qw: the
+// group's selector queries as mma B fragments (lane: head r8); wh0 / wh1:
+// weights of heads 2 c4, 2 c4 + 1 (0 for padding heads).
+template <int FMT>
+__device__ __forceinline__ void score_tiles(const SelectParams& p, int b, int g,
+                                            const uint32_t (&qw)[8], float wh0, float wh1,
+                                            int t0, int stride, int n_full, float* scores,
+                                            int lane) {
+    const int c4 = lane & 3, r8 = lane >> 2;
+    int64_t rowa[kTileBatch], rowb[kTileBatch];
+#pragma unroll
+    for (int k = 0; k < kTileBatch; ++k) {
+        const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
         int pa = (ja < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + ja] : 0;
         int pb = (jb < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + jb] : 0;
         if (pa < 0 || pa >= p.num_pages) { flag_status(p.status, kStatusBounds); pa = 0; }
         if (pb < 0 || pb >= p.num_pages) { flag_status(p.status, kStatusBounds); pb = 0; }
-        const int64_t rowa = static_cast<int64_t>(pa) * p.num_kv_heads + g;
-        const int64_t rowb = static_cast<int64_t>(pb) * p.num_kv_heads + g;
-
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f};
-        float acc1[4] = {0.f, 0.f, 0.f, 0.f};
-        if (FMT == SPOT_SEL_BF16) {
-            const uint4* ka = reinterpret_cast<const uint4*>(p.sel_data) + rowa * 8 + 2 * c4;
-            const uint4* kb = reinterpret_cast<const uint4*>(p.sel_data) + rowb * 8 + 2 * c4;
-            const uint4 a0 = __ldg(ka), a1 = __ldg(ka + 1), b0 = __ldg(kb), b1 = __ldg(kb + 1);
-            const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        rowa[k] = static_cast<int64_t>(pa) * p.num_kv_heads + g;
+        rowb[k] = static_cast<int64_t>(pb) * p.num_kv_heads + g;
+    }
+    float acc[kTileBatch][4];
+    if (FMT == SPOT_SEL_BF16) {
+        uint4 a0[kTileBatch], a1[kTileBatch], b0[kTileBatch], b1[kTileBatch];
+#pragma unroll
+        for (int k = 0; k < kTileBatch; ++k) {
+            const uint4* ka = reinterpret_cast<const uint4*>(p.sel_data) + rowa[k] * 8 + 2 * c4;
+            const uint4* kb = reinterpret_cast<const uint4*>(p.sel_data) + rowb[k] * 8 + 2 * c4;
+            a0[k] = __ldg(ka);
+            a1[k] = __ldg(ka + 1);
+            b0[k] = __ldg(kb);
+            b1[k] = __ldg(kb + 1);
+        }
+#pragma unroll
+        for (int k = 0; k < kTileBatch; ++k) {
+            const uint32_t wa[8] = {a0[k].x, a0[k].y, a0[k].z, a0[k].w,
+                                    a1[k].x, a1[k].y, a1[k].z, a1[k].w};
+            const uint32_t wb[8] = {b0[k].x, b0[k].y, b0[k].z, b0[k].w,
+                                    b1[k].x, b1[k].y, b1[k].z, b1[k].w};
+            acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16_16816(acc0, wa[2 * s], wb[2 * s], wa[2 * s + 1], wb[2 * s + 1],
+                mma_bf16_16816(acc[k], wa[2 * s], wb[2 * s], wa[2 * s + 1], wb[2 * s + 1],
                                qw[2 * s], qw[2 * s + 1]);
-        } else {
-            const uint32_t* da = reinterpret_cast<const uint32_t*>(p.sel_data) + rowa * 8;
-            const uint32_t* db = reinterpret_cast<const uint32_t*>(p.sel_data) + rowb * 8;
-            const uint32_t ga0 = __ldg(da + c4), ga1 = __ldg(da + 4 + c4);
-            const uint32_t gb0 = __ldg(db + c4), gb1 = __ldg(db + 4 + c4);
-            // group 0 -> acc0 (k-steps 0, 1), group 1 -> acc1 (k-steps 2, 3)
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const uint32_t a_lo = byte_to_bf16x2<FMT>((ga0 >> (16 * s)) & 0xFFu);
-                const uint32_t a_hi = byte_to_bf16x2<FMT>((ga0 >> (16 * s + 8)) & 0xFFu);
-                const uint32_t b_lo = byte_to_bf16x2<FMT>((gb0 >> (16 * s)) & 0xFFu);
-                const uint32_t b_hi = byte_to_bf16x2<FMT>((gb0 >> (16 * s + 8)) & 0xFFu);
-                mma_bf16_16816(acc0, a_lo, b_lo, a_hi, b_hi, qw[2 * s], qw[2 * s + 1]);
-            }
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const uint32_t a_lo = byte_to_bf16x2<FMT>((ga1 >> (16 * s)) & 0xFFu);
-                const uint32_t a_hi = byte_to_bf16x2<FMT>((ga1 >> (16 * s + 8)) & 0xFFu);
-                const uint32_t b_lo = byte_to_bf16x2<FMT>((gb1 >> (16 * s)) & 0xFFu);
-                const uint32_t b_hi = byte_to_bf16x2<FMT>((gb1 >> (16 * s + 8)) & 0xFFu);
-                mma_bf16_16816(acc1, a_lo, b_lo, a_hi, b_hi, qw[4 + 2 * s], qw[4 + 2 * s + 1]);
-            }
-            const float sa0 = group_scale<FMT>(p.sel_scales, rowa, 0);
-            const float sa1 = group_scale<FMT>(p.sel_scales, rowa, 1);
-            const float sb0 = group_scale<FMT>(p.sel_scales, rowb, 0);
-            const float sb1 = group_scale<FMT>(p.sel_scales, rowb, 1);
-            acc0[0] = acc0[0] * sa0 + acc1[0] * sa1;
-            acc0[1] = acc0[1] * sa0 + acc1[1] * sa1;
-            acc0[2] = acc0[2] * sb0 + acc1[2] * sb1;
-            acc0[3] = acc0[3] * sb0 + acc1[3] * sb1;
         }
-        // ---- epilogue: weighted ReLU sum over the group's heads
-        float sa = wh0 * fmaxf(acc0[0], 0.f) + wh1 * fmaxf(acc0[1], 0.f);
-        float sb = wh0 * fmaxf(acc0[2], 0.f) + wh1 * fmaxf(acc0[3], 0.f);
+    } else {
+        uint32_t ga0[kTileBatch], ga1[kTileBatch], gb0[kTileBatch], gb1[kTileBatch];
+        float sa0[kTileBatch], sa1[kTileBatch], sb0[kTileBatch], sb1[kTileBatch];
+#pragma unroll
+        for (int k = 0; k < kTileBatch; ++k) {
+            const uint32_t* da = reinterpret_cast<const uint32_t*>(p.sel_data) + rowa[k] * 8;
+            const uint32_t* db = reinterpret_cast<const uint32_t*>(p.sel_data) + rowb[k] * 8;
+            ga0[k] = __ldg(da + c4);
+            ga1[k] = __ldg(da + 4 + c4);
+            gb0[k] = __ldg(db + c4);
+            gb1[k] = __ldg(db + 4 + c4);
+            sa0[k] = group_scale<FMT>(p.sel_scales, rowa[k], 0);
+            sa1[k] = group_scale<FMT>(p.sel_scales, rowa[k], 1);
+            sb0[k] = group_scale<FMT>(p.sel_scales, rowb[k], 0);
+            sb1[k] = group_scale<FMT>(p.sel_scales, rowb[k], 1);
+        }
+#pragma unroll
+        for (int k = 0; k < kTileBatch; ++k) {
+            // group 0 -> acc0 (k-steps 0, 1), group 1 -> acc1 (k-steps 2, 3)
+            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                mma_bf16_16816(acc0, byte_to_bf16x2<FMT>((ga0[k] >> (16 * s)) & 0xFFu),
+                               byte_to_bf16x2<FMT>((gb0[k] >> (16 * s)) & 0xFFu),
+                               byte_to_bf16x2<FMT>((ga0[k] >> (16 * s + 8)) & 0xFFu),
+                               byte_to_bf16x2<FMT>((gb0[k] >> (16 * s + 8)) & 0xFFu),
+                               qw[2 * s], qw[2 * s + 1]);
+                mma_bf16_16816(acc1, byte_to_bf16x2<FMT>((ga1[k] >> (16 * s)) & 0xFFu),
+                               byte_to_bf16x2<FMT>((gb1[k] >> (16 * s)) & 0xFFu),
+                               byte_to_bf16x2<FMT>((ga1[k] >> (16 * s + 8)) & 0xFFu),
+                               byte_to_bf16x2<FMT>((gb1[k] >> (16 * s + 8)) & 0xFFu),
+                               qw[4 + 2 * s], qw[4 + 2 * s + 1]);
+            }
+            acc[k][0] = acc0[0] * sa0[k] + acc1[0] * sa1[k];
+            acc[k][1] = acc0[1] * sa0[k] + acc1[1] * sa1[k];
+            acc[k][2] = acc0[2] * sb0[k] + acc1[2] * sb1[k];
+            acc[k][3] = acc0[3] * sb0[k] + acc1[3] * sb1[k];
+        }
+    }
+    // epilogue: weighted ReLU sum over the group's heads (columns 2 c4, 2 c4 + 1)
+#pragma unroll
+    for (int k = 0; k < kTileBatch; ++k) {
+        float sa = wh0 * fmaxf(acc[k][0], 0.f) + wh1 * fmaxf(acc[k][1], 0.f);
+        float sb = wh0 * fmaxf(acc[k][2], 0.f) + wh1 * fmaxf(acc[k][3], 0.f);
         sa += __shfl_xor_sync(0xffffffffu, sa, 1);
         sa += __shfl_xor_sync(0xffffffffu, sa, 2);
         sb += __shfl_xor_sync(0xffffffffu, sb, 1);
         sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+        const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
         if (c4 == 0) {
-            float* out = p.scores + (static_cast<int64_t>(b) * p.num_kv_heads + g) * p.max_blocks;
-            if (ja < n_full) out[ja] = sa * p.inv_temp;
-            if (jb < n_full) out[jb] = sb * p.inv_temp;
+            if (ja < n_full) scores[ja] = sa * p.inv_temp;
+            if (jb < n_full) scores[jb] = sb * p.inv_temp;
         }
     }
+}
+
+// Selector queries of head group g as mma B fragments (lane: head r8) and
+// the weights of heads 2 c4, 2 c4 + 1.
+template <int FMT>
+__device__ __forceinline__ void load_queries(const SelectParams& p, int b, int g, int lane,
+                                             uint32_t (&qw)[8], float& wh0, float& wh1) {
+    const int c4 = lane & 3, r8 = lane >> 2;
+    const int G = p.group;
+    const bool real = r8 < G;
+    const int h = g * G + (real ? r8 : 0);
+    const uint4* qrow = reinterpret_cast<const uint4*>(
+        p.q_sel + (static_cast<int64_t>(b) * p.num_q_heads + h) * kSelDim);
+    // bf16 keys: lane c4 owns dims [16 c4, 16 c4 + 16);
+    // 4-bit keys: dims [8 c4, 8 c4 + 8) and [32 + 8 c4, 32 + 8 c4 + 8).
+    uint4 x0, x1;
+    if (FMT == SPOT_SEL_BF16) {
+        x0 = real ? __ldg(qrow + 2 * c4) : make_uint4(0, 0, 0, 0);
+        x1 = real ? __ldg(qrow + 2 * c4 + 1) : make_uint4(0, 0, 0, 0);
+    } else {
+        x0 = real ? __ldg(qrow + c4) : make_uint4(0, 0, 0, 0);
+        x1 = real ? __ldg(qrow + 4 + c4) : make_uint4(0, 0, 0, 0);
+    }
+    qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
+    qw[4] = x1.x; qw[5] = x1.y; qw[6] = x1.z; qw[7] = x1.w;
+    const int64_t wrow = static_cast<int64_t>(b) * p.num_q_heads + g * G;
+    wh0 = (2 * c4 < G) ? (p.w ? p.w[wrow + 2 * c4] : 1.f / G) : 0.f;
+    wh1 = (2 * c4 + 1 < G) ? (p.w ? p.w[wrow + 2 * c4 + 1] : 1.f / G) : 0.f;
 }
 
 // --------------------------------------------------------------- selection
@@ -210,6 +228,7 @@ constexpr int NT = kSelectThreads;
 constexpr int NW = NT / 32;
 
 struct SelSmem {
+    float* score;                 // [max_blocks] selector scores of the complete blocks
     uint32_t* keys;               // [max_blocks] order-preserving keys of the residual scores
     unsigned long long* mass;     // [max_blocks] fixed-point exp(s - max)
     uint16_t* vb;                 // [max_blocks] value bucket (0 = the top scores)
@@ -452,7 +471,8 @@ __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long lon
 
 size_t select_smem_bytes(int max_blocks) {
     return static_cast<size_t>(max_blocks) *
-               (sizeof(uint32_t) + sizeof(unsigned long long) + sizeof(uint16_t) + 1) +
+               (sizeof(float) + sizeof(uint32_t) + sizeof(unsigned long long) +
+                sizeof(uint16_t) + 1) +
            kNB * (sizeof(uint32_t) + sizeof(uint32_t)) +
            NT * (sizeof(uint32_t) + sizeof(int) + sizeof(unsigned long long)) +
            3 * NW * sizeof(unsigned long long) + 8 * sizeof(int) +
@@ -461,17 +481,23 @@ size_t select_smem_bytes(int max_blocks) {
 
 namespace {
 
-__global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectParams p) {
+
+template <int FMT>
+__global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
     SelSmem sm;
     {
         uint8_t* q = smem;
+        // 8-byte arrays first, then 4-, 2- and 1-byte ones: every array stays
+        // aligned whatever max_blocks is
         sm.mass = reinterpret_cast<unsigned long long*>(q);
         q += sizeof(unsigned long long) * p.max_blocks;
         sm.cval = reinterpret_cast<unsigned long long*>(q);
         q += sizeof(unsigned long long) * NT;
         sm.red = reinterpret_cast<unsigned long long*>(q);
         q += sizeof(unsigned long long) * 3 * NW;
+        sm.score = reinterpret_cast<float*>(q);
+        q += sizeof(float) * p.max_blocks;
         sm.keys = reinterpret_cast<uint32_t*>(q);
         q += sizeof(uint32_t) * p.max_blocks;
         sm.hmass = reinterpret_cast<uint32_t*>(q);
@@ -512,11 +538,22 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
     const int r0 = sink, r1 = max(sink, nb - rec);    // residual blocks [r0, r1)
     const int n = r1 - r0;
     const int n_reserved = nb - n;
-    const float* s = p.scores + static_cast<int64_t>(u) * p.max_blocks;
+    const float* s = sm.score;
     for (int i = threadIdx.x; i < kNB; i += NT) { sm.hmass[i] = 0u; sm.hcnt[i] = 0u; }
     if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
-    pdl_trigger();
-    pdl_wait();                                       // scores of the scoring kernel
+    pdl_trigger();                                    // the decode kernel may start its prologue
+
+    // ---- selector scores of the complete blocks (§2.1), into shared memory
+    {
+        const int g = u - b * p.num_kv_heads;
+        uint32_t qw[8];
+        float wh0, wh1;
+        load_queries<FMT>(p, b, g, lane, qw, wh0, wh1);
+        const int tiles = (n_full + 15) / 16;
+        for (int t0 = warp; t0 < tiles; t0 += NW * kTileBatch)
+            score_tiles<FMT>(p, b, g, qw, wh0, wh1, t0, NW, n_full, sm.score, lane);
+    }
+    __syncthreads();
 
     // ---- residual scores -> keys, maximum
     float mloc = -INFINITY;
@@ -651,26 +688,25 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
 
 }  // namespace
 
-
-cudaError_t launch_scores(const ScoreParams& p, int fmt, cudaStream_t s) {
-    const dim3 grid((p.max_blocks + 15) / 16, (p.num_kv_heads + kScoreWarps - 1) / kScoreWarps,
-                    p.batch);
-    if (fmt == SPOT_SEL_BF16)
-        score_kernel<SPOT_SEL_BF16><<<grid, kScoreWarps * 32, 0, s>>>(p);
-    else if (fmt == SPOT_SEL_INT4_G32_F16)
-        score_kernel<SPOT_SEL_INT4_G32_F16><<<grid, kScoreWarps * 32, 0, s>>>(p);
-    else
-        score_kernel<SPOT_SEL_MXFP4_G32_E8M0><<<grid, kScoreWarps * 32, 0, s>>>(p);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
+cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s) {
     const size_t smem = select_smem_bytes(p.max_blocks);
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    const dim3 grid(p.batch * p.num_kv_heads), block(kSelectThreads);
+    cudaError_t e;
+    if (fmt == SPOT_SEL_BF16) {
+        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_BF16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess) select_kernel<SPOT_SEL_BF16><<<grid, block, smem, s>>>(p);
+    } else if (fmt == SPOT_SEL_INT4_G32_F16) {
+        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_INT4_G32_F16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess) select_kernel<SPOT_SEL_INT4_G32_F16><<<grid, block, smem, s>>>(p);
+    } else {
+        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_MXFP4_G32_E8M0>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess) select_kernel<SPOT_SEL_MXFP4_G32_E8M0><<<grid, block, smem, s>>>(p);
+    }
     if (e != cudaSuccess) return e;
-    return launch_pdl(select_kernel, dim3(p.batch * p.num_kv_heads), dim3(kSelectThreads), smem, s,
-                      p);
+    return cudaGetLastError();
 }
 
 }  // namespace spot

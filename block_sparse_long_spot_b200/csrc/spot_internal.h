@@ -35,14 +35,15 @@ constexpr int kStageBytes = 2 * kBlock * kHeadDim * 2;   // 32768
 constexpr int kPartialFloatsPerHead = kHeadDim + 4;
 
 struct Layout {
-    size_t status, scores, unit_done, partials, total;
+    size_t status, unit_done, partials, total;
     int grid;                           // persistent CTAs of the decode kernel
 };
 
 // Workspace layout for a shape on the current device.
 bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Layout* out);
 
-struct ScoreParams {
+// Parameters of the fused scoring + selection kernel.
+struct SelectParams {
     const uint16_t* q_sel;
     const float* w;
     const void* sel_data;
@@ -50,18 +51,9 @@ struct ScoreParams {
     const int32_t* page_table;
     int32_t pt_stride;
     const int32_t* seq_lens;
+    const float* top_p;
     int32_t batch, num_q_heads, num_kv_heads, group, num_pages, max_blocks;
     float inv_temp;
-    float* scores;                      // [B][Hkv][max_blocks]
-    uint32_t* status;
-};
-
-struct SelectParams {
-    const float* scores;
-    const int32_t* seq_lens;
-    const float* top_p;
-    int32_t pt_stride;
-    int32_t batch, num_kv_heads, max_blocks;
     int32_t mode, sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
     int32_t* sel_idx;
     int32_t* sel_cnt;
@@ -116,8 +108,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-cudaError_t launch_scores(const ScoreParams& p, int fmt, cudaStream_t s);
-cudaError_t launch_select(const SelectParams& p, cudaStream_t s);
+cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s);
 cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
                                  const CUtensorMap& v_map, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);

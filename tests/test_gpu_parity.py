@@ -286,8 +286,10 @@ def test_weights_temperature_and_padding():
     wl.w = (wl.w * 8).round() / 8                       # exact in fp32 and fp64
     for temp in (1.0, 2.0, 0.5):
         wl.top_p = safe_top_p(wl, temperature=temp)
-        gpu = run_gpu(wl, temperature=temp, max_blocks=wl.max_blocks + 37)
-        ora = run_oracle(wl, temperature=temp, max_blocks=wl.max_blocks + 37)
+        # an odd max_blocks (47 + 38 = 85) also checks the alignment of the
+        # kernels' shared-memory layouts
+        gpu = run_gpu(wl, temperature=temp, max_blocks=wl.max_blocks + 38)
+        ora = run_oracle(wl, temperature=temp, max_blocks=wl.max_blocks + 38)
         _assert_same_selection(gpu, ora, wl)
         check_outputs(gpu, ora, wl)
 
