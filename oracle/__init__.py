@@ -27,8 +27,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "spot_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
-FMT = {"bf16": 0, "int4": 1, "mxfp4": 2}
+FMT = {"bf16": 0, "int4": 1, "mxfp4": 2, "fp8": 3, "int8": 4}
 MODE = {"topp": 0, "topk": 1}
+_FMT_NAME = {v: k for k, v in FMT.items()}
 
 _lib = None
 
@@ -102,12 +103,28 @@ def make_params(mode="topp", sink_blocks=1, recency_blocks=4, kmin_blocks=8, top
                   kmin_blocks, topk_blocks, float(temperature))
 
 
+def _data_dtype(fmt):
+    return {"bf16": np.uint16, "int8": np.int8}.get(fmt, np.uint8)
+
+
+def _scale_dtype(fmt):
+    return np.uint16 if fmt in ("int4", "int8") else np.uint8
+
+
+def _row_elems(fmt, ds):
+    return {"bf16": ds, "fp8": ds, "int8": ds}.get(fmt, ds // 2)
+
+
+def _scales_per_row(fmt, ds):
+    return {"int4": ds // 32, "mxfp4": ds // 32, "int8": 1}.get(fmt, 0)
+
+
 def dequant_selector(fmt: str, data: np.ndarray, scales, ds: int) -> np.ndarray:
     """Exact fp64 values of selector keys stored as `fmt` ([rows, ds])."""
-    rows = data.size // (ds if fmt == "bf16" else ds // 2)
-    data = _c(data, np.uint16 if fmt == "bf16" else np.uint8)
+    rows = data.size // _row_elems(fmt, ds)
+    data = _c(data, _data_dtype(fmt))
     if scales is not None:
-        scales = _c(scales, np.uint16 if fmt == "int4" else np.uint8)
+        scales = _c(scales, _scale_dtype(fmt))
     out = np.empty((rows, ds), np.float64)
     rc = _load().oracle_dequant_selector(FMT[fmt], rows, ds, _ptr(data), _ptr(scales), _ptr(out))
     assert rc == 0
@@ -120,11 +137,9 @@ def quantize_selector(fmt: str, keys_bits: np.ndarray):
     lead = keys_bits.shape[:-1]
     rows = int(np.prod(lead)) if lead else 1
     keys = _c(keys_bits, np.uint16)
-    if fmt == "bf16":
-        data, scales = np.empty(lead + (ds,), np.uint16), None
-    else:
-        data = np.empty(lead + (ds // 2,), np.uint8)
-        scales = np.empty(lead + (ds // 32,), np.uint16 if fmt == "int4" else np.uint8)
+    data = np.empty(lead + (_row_elems(fmt, ds),), _data_dtype(fmt))
+    nsc = _scales_per_row(fmt, ds)
+    scales = np.empty(lead + (nsc,), _scale_dtype(fmt)) if nsc else None
     rc = _load().oracle_quantize_selector(FMT[fmt], rows, ds, _ptr(keys), _ptr(data),
                                           _ptr(scales))
     assert rc == 0
@@ -151,8 +166,8 @@ def block_scores(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, p
     fmt = shape.sel_fmt
     rc = _load().oracle_block_scores(
         ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_sel, np.uint16)),
-        _ptr(_c(w, np.float32)), _ptr(_c(sel_data, np.uint16 if fmt == 0 else np.uint8)),
-        _ptr(_c(sel_scales, np.uint16 if fmt == 1 else np.uint8)),
+        _ptr(_c(w, np.float32)), _ptr(_c(sel_data, _data_dtype(_FMT_NAME[fmt]))),
+        _ptr(_c(sel_scales, _scale_dtype(_FMT_NAME[fmt]))),
         _ptr(_c(page_table, np.int32)), _ptr(_c(seq_lens, np.int32)), _ptr(scores))
     assert rc == 0
     return scores
@@ -185,8 +200,8 @@ def decode_step(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, q,
     u = None if units is None else _c(units, np.int32)
     _load().oracle_decode_step(
         ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_sel, np.uint16)),
-        _ptr(_c(w, np.float32)), _ptr(_c(sel_data, np.uint16 if fmt == 0 else np.uint8)),
-        _ptr(_c(sel_scales, np.uint16 if fmt == 1 else np.uint8)), _ptr(_c(q, np.uint16)),
+        _ptr(_c(w, np.float32)), _ptr(_c(sel_data, _data_dtype(_FMT_NAME[fmt]))),
+        _ptr(_c(sel_scales, _scale_dtype(_FMT_NAME[fmt]))), _ptr(_c(q, np.uint16)),
         _ptr(_c(k_pool, np.uint16)), _ptr(_c(v_pool, np.uint16)), _ptr(_c(page_table, np.int32)),
         _ptr(_c(seq_lens, np.int32)), _ptr(_c(top_p, np.float32)), float(sm_scale), _ptr(u),
         0 if u is None else len(u), _ptr(sel_idx), _ptr(sel_cnt), _ptr(mass), _ptr(out),

@@ -32,7 +32,12 @@
  *  - FP4 keys: OCP Microscaling v1.0 MXFP4 -- E2M1 elements, one E8M0 scale
  *    per 32, X = floor(log2 amax) - 2 clamped to [-127, 127], elements
  *    rounded to nearest even on the E2M1 grid with saturation at 6; the sign
- *    bit is set only for x < 0; same nibble order as INT4.
+ *    bit is set only for x < 0; same nibble order as INT4;
+ *  - FP8 keys: OCP FP8 E4M3 (bias 7, no infinities, S.1111.111 is NaN), one
+ *    byte per element and no scale (8 bits = 0.5x bf16, App. G Tab. 9),
+ *    round to nearest even, saturating at +-448;
+ *  - INT8 keys: symmetric, one binary16 scale per key = fp16_rne(amax/127)
+ *    (saturating at 65504), code = clamp(rne(x/scale), -128, 127).
  *
  * Parity status: every function here is pinned by tests/test_oracle_pins.py
  * (hand-worked examples, brute force, closed forms, library special cases).
@@ -46,7 +51,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_FMT_BF16 = 0, ORC_FMT_INT4 = 1, ORC_FMT_MXFP4 = 2 };
+enum { ORC_FMT_BF16 = 0, ORC_FMT_INT4 = 1, ORC_FMT_MXFP4 = 2, ORC_FMT_FP8 = 3, ORC_FMT_INT8 = 4 };
 enum { ORC_MODE_TOPP = 0, ORC_MODE_TOPK = 1 };
 
 /* ------------------------------------------------------------------ */
@@ -113,10 +118,47 @@ static double e8m0_to_f64(uint8_t e) {
     return e == 255 ? NAN : ldexp(1.0, (int)e - 127);
 }
 
+/* OCP FP8 E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent
+ * 0 is subnormal (m 2^-9); S.1111.111 is NaN (no infinities). */
+static double e4m3_to_f64(uint8_t code) {
+    int e = (code >> 3) & 15, m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m, -9);
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+    return (code & 0x80) ? -mag : mag;
+}
+
+/* fp64 -> E4M3, round to nearest even, magnitudes beyond 448 saturate to
+ * 448 (the largest finite E4M3). */
+static uint8_t f64_to_e4m3_sat(double x) {
+    uint8_t sign = (x < 0.0) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0) return sign | 0x7E;
+    int ex;
+    (void)frexp(a, &ex);                   /* a = f 2^ex, f in [.5, 1) */
+    int e = ex - 1;                        /* a in [2^e, 2^(e+1)) */
+    if (a == 0.0 || e < -6) e = -6;        /* subnormal range: ulp 2^-9 */
+    double ulp = ldexp(1.0, e - 3);
+    double q = a / ulp;                    /* exact */
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double y = r * ulp;                    /* rounded magnitude, exact */
+    if (y >= 448.0) return sign | 0x7E;
+    if (y < ldexp(1.0, -6)) return sign | (uint8_t)(y / ldexp(1.0, -9));
+    (void)frexp(y, &ex);
+    e = ex - 1;
+    int mant = (int)(y / ldexp(1.0, e - 3)) - 8;
+    return sign | (uint8_t)(((e + 7) << 3) | mant);
+}
+
 /* Dequantise `rows` selector keys of `ds` elements each into fp64.
  * bf16:  data = uint16 [rows][ds], scales unused.
  * INT4:  data = uint8 [rows][ds/2], scales = binary16 [rows][ds/32].
  * MXFP4: data = uint8 [rows][ds/2], scales = E8M0 [rows][ds/32].
+ * FP8:   data = uint8 E4M3 [rows][ds], scales unused.
+ * INT8:  data = int8 [rows][ds], scales = binary16 [rows][1].
  * Returns 0, or -1 for an unknown format. */
 int oracle_dequant_selector(int fmt, int64_t rows, int ds, const void* data,
                             const void* scales, double* out) {
@@ -125,6 +167,10 @@ int oracle_dequant_selector(int fmt, int64_t rows, int ds, const void* data,
             double v;
             if (fmt == ORC_FMT_BF16) {
                 v = bf16_to_f64(((const uint16_t*)data)[r * ds + i]);
+            } else if (fmt == ORC_FMT_FP8) {
+                v = e4m3_to_f64(((const uint8_t*)data)[r * ds + i]);
+            } else if (fmt == ORC_FMT_INT8) {
+                v = (double)((const int8_t*)data)[r * ds + i] * f16_to_f64(((const uint16_t*)scales)[r]);
             } else if (fmt == ORC_FMT_INT4 || fmt == ORC_FMT_MXFP4) {
                 uint8_t byte = ((const uint8_t*)data)[r * (ds / 2) + i / 2];
                 unsigned nib = (i % 2 == 0) ? (byte & 0xf) : (byte >> 4);
@@ -162,7 +208,7 @@ static unsigned e2m1_rne_code(double a) {
 }
 
 /* Quantise bf16 selector keys (the append step of the selector K-cache,
- * SpotAttention §5.3 and App. G: group-32 INT4 / FP4 microscale).
+ * SpotAttention §5.3 and App. G: group-32 INT4 / FP4 microscale, INT8, FP8).
  * Layouts as in oracle_dequant_selector.  bf16 is a plain copy. */
 int oracle_quantize_selector(int fmt, int64_t rows, int ds, const uint16_t* keys,
                              void* data, void* scales) {
@@ -171,6 +217,32 @@ int oracle_quantize_selector(int fmt, int64_t rows, int ds, const uint16_t* keys
         const uint16_t* row = keys + r * ds;
         if (fmt == ORC_FMT_BF16) {
             memcpy((uint16_t*)data + r * ds, row, (size_t)ds * sizeof(uint16_t));
+            continue;
+        }
+        if (fmt == ORC_FMT_FP8) {
+            for (int i = 0; i < ds; ++i)
+                ((uint8_t*)data)[r * ds + i] = f64_to_e4m3_sat(bf16_to_f64(row[i]));
+            continue;
+        }
+        if (fmt == ORC_FMT_INT8) {
+            double amax = 0.0;
+            for (int i = 0; i < ds; ++i) {
+                double x = fabs(bf16_to_f64(row[i]));
+                if (x > amax) amax = x;
+            }
+            uint16_t sbits = f64_to_f16_sat(amax / 127.0);
+            ((uint16_t*)scales)[r] = sbits;
+            double sc = f16_to_f64(sbits);
+            for (int i = 0; i < ds; ++i) {
+                int q = 0;
+                if (sc > 0.0) {
+                    double t = nearbyint(bf16_to_f64(row[i]) / sc);    /* ties to even */
+                    if (t > 127.0) t = 127.0;
+                    if (t < -128.0) t = -128.0;
+                    q = (int)t;
+                }
+                ((int8_t*)data)[r * ds + i] = (int8_t)q;
+            }
             continue;
         }
         uint8_t* out = (uint8_t*)data + r * (ds / 2);

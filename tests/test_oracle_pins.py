@@ -267,16 +267,75 @@ def test_quantisation_error_bounds():
 
 
 def test_footprint_closed_form():
-    # Selector K-cache bytes per element: bf16 16 bits, INT4 4 + 16/32 bits,
-    # MXFP4 4 + 8/32 bits.  The paper's GiB figures follow.
+    # Selector K-cache bits per element: bf16 16, INT4 4 + 16/32, MXFP4
+    # 4 + 8/32, FP8 8, INT8 8 + 16/64.  The paper's GiB figures for BF16,
+    # INT4 and FP4 (§5.3) follow; FP8 is its 0.500x (App. G Tab. 9), INT8
+    # carries a per-key scale on top.
     fp = _golden("selector_codes.json")["footprint"]
     n = fp["layers"] * fp["tokens"] * fp["elements_per_token"]
-    for fmt, bits_per in (("bf16", 16.0), ("int4", 4.5), ("mxfp4", 4.25)):
+    for fmt, bits_per in fp["bits"].items():
         x = np.zeros((1, 64), np.float32)
         data, scales = oracle.quantize_selector(fmt, _bf16_bits(x))
         stored = data.nbytes + (0 if scales is None else scales.nbytes)
         assert stored * 8 / 64 == bits_per
         assert round(n * bits_per / 8 / 2**30, 2) == fp["gib"][fmt]
+    assert fp["bits"]["fp8"] / fp["bits"]["bf16"] == 0.5
+
+
+def test_fp8_known_codes():
+    g = _golden("selector_codes.json")
+    enc = g["encode_fp8"]
+    data, scales = oracle.quantize_selector("fp8", _bf16_bits(enc["inputs"] * 4)[None])
+    assert scales is None
+    assert data[0].tolist() == enc["codes"] * 4
+    dec = g["decode_fp8"]
+    vals = oracle.dequant_selector("fp8", np.array(dec["codes"] + [0] * 57, np.uint8), None, 64)[0]
+    for v, e in zip(vals, dec["values"]):
+        assert (np.isnan(v) if e == "nan" else v == e)
+
+
+def test_fp8_rounding_matches_torch_float8():
+    # torch's float8_e4m3fn cast (round to nearest even) is an independent
+    # implementation of the same format for magnitudes up to 448.
+    rng = np.random.default_rng(4)
+    x = np.concatenate([rng.normal(size=4000) * 10.0 ** rng.uniform(-3, 2.6, size=4000),
+                        np.linspace(-448, 448, 1793)])
+    x = torch.as_tensor(x.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    x = x[np.abs(x) <= 448][: 64 * 80]
+    bits = _bf16_bits(x.reshape(-1, 64))
+    data, _ = oracle.quantize_selector("fp8", bits)
+    ref = torch.as_tensor(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = data.reshape(-1)
+    zero = x == 0
+    assert np.array_equal(ours[~zero], ref[~zero])
+    assert (ours[zero] == 0).all()
+    back = oracle.dequant_selector("fp8", data, None, 64).reshape(-1)
+    ref_back = torch.as_tensor(x).to(torch.float8_e4m3fn).float().numpy()
+    assert np.array_equal(back, ref_back)
+
+
+def test_int8_known_codes_and_scale():
+    g = _golden("selector_codes.json")["encode_int8"]
+    row = g["inputs"] + [0.0] * (64 - len(g["inputs"]))
+    data, scales = oracle.quantize_selector("int8", _bf16_bits(row)[None])
+    assert data[0, :len(g["codes"])].tolist() == g["codes"]
+    assert scales[0].tolist() == [g["scale_bits"]]
+    rng = np.random.default_rng(5)
+    x = (rng.normal(size=(300, 64)) * 10.0 ** rng.uniform(-4, 4, size=(300, 1))).astype(np.float32)
+    bits = _bf16_bits(x)
+    data, scales = oracle.quantize_selector("int8", bits)
+    xb = torch.as_tensor(x).to(torch.bfloat16).double().numpy()
+    amax = np.abs(xb).max(1)
+    ref = np.minimum(amax / 127.0, 65504.0).astype(np.float16).view(np.uint16)
+    assert (scales[:, 0] == ref).all()
+    back = oracle.dequant_selector("int8", data, scales, 64)
+    s = scales[:, 0].view(np.float16).astype(np.float64)[:, None]
+    assert (np.abs(back - xb) <= 0.5 * s * (1 + 1e-9) + 1e-300).all()
+    e = np.exp2(rng.integers(-8, 8, size=(8, 1)))
+    on_grid = rng.integers(-127, 128, size=(8, 64)) * e
+    on_grid[:, 0] = 127 * e[:, 0]                      # amax = 127 * scale
+    d2, s2 = oracle.quantize_selector("int8", _bf16_bits(on_grid))
+    assert np.array_equal(oracle.dequant_selector("int8", d2, s2, 64), on_grid)
 
 
 # ---------------------------------------------------------------- attention
