@@ -172,7 +172,7 @@ def step_bytes(wl, sel_cnt: np.ndarray, fmt: str):
     B, Hq, Hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
     lens = wl.seq_lens.cpu().numpy().astype(np.int64)
     nb, n_full = unit_counts(wl)
-    key_bytes = {"bf16": 128, "int4": 32 + 4, "mxfp4": 32 + 2}[fmt]
+    key_bytes = {"bf16": 128, "int4": 32 + 4, "mxfp4": 32 + 2, "fp8": 64, "int8": 64 + 2}[fmt]
     sel_cache = int(Hkv * n_full.sum() * key_bytes)
     # tokens attended per (b, g): full blocks, the last one possibly partial
     kv = 0

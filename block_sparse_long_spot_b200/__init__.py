@@ -22,7 +22,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libspot_b200.so")
 
-SEL_FMT = {"bf16": 0, "int4": 1, "mxfp4": 2}
+SEL_FMT = {"bf16": 0, "int4": 1, "mxfp4": 2, "fp8": 3, "int8": 4}
 MODE = {"topp": 0, "topk": 1}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace too small",
           4: "CUDA error", 5: "device: index out of range", 6: "device: bounded wait timed out"}
@@ -227,6 +227,12 @@ def selector_pool(fmt: str, num_pages: int, num_kv_heads: int, sel_dim: int = 64
     if fmt == "bf16":
         return (torch.zeros(num_pages, num_kv_heads, sel_dim, dtype=torch.bfloat16, device=device),
                 None)
+    if fmt == "fp8":
+        return (torch.zeros(num_pages, num_kv_heads, sel_dim, dtype=torch.uint8, device=device),
+                None)
+    if fmt == "int8":
+        return (torch.zeros(num_pages, num_kv_heads, sel_dim, dtype=torch.int8, device=device),
+                torch.zeros(num_pages, num_kv_heads, 1, dtype=torch.float16, device=device))
     data = torch.zeros(num_pages, num_kv_heads, sel_dim // 2, dtype=torch.uint8, device=device)
     sdt = torch.float16 if fmt == "int4" else torch.uint8
     return data, torch.zeros(num_pages, num_kv_heads, sel_dim // 32, dtype=sdt, device=device)
@@ -234,4 +240,5 @@ def selector_pool(fmt: str, num_pages: int, num_kv_heads: int, sel_dim: int = 64
 
 def selector_bytes_per_element(fmt: str) -> float:
     """Stored bits / 8 per selector-key element, scales included."""
-    return {"bf16": 2.0, "int4": (4 + 16 / 32) / 8, "mxfp4": (4 + 8 / 32) / 8}[fmt]
+    return {"bf16": 2.0, "int4": (4 + 16 / 32) / 8, "mxfp4": (4 + 8 / 32) / 8, "fp8": 1.0,
+            "int8": (8 + 16 / 64) / 8}[fmt]

@@ -15,12 +15,17 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+bool needs_scales(int fmt) {
+    return fmt == SPOT_SEL_INT4_G32_F16 || fmt == SPOT_SEL_MXFP4_G32_E8M0 ||
+           fmt == SPOT_SEL_INT8_F16;
+}
+
 spot_status_t check_desc(const spot_layer_desc_t* d) {
     if (!d) return SPOT_ERR_INVALID_ARG;
     if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_pages <= 0)
         return SPOT_ERR_INVALID_ARG;
     if (d->num_q_heads % d->num_kv_heads != 0) return SPOT_ERR_INVALID_ARG;
-    if (d->sel_fmt < SPOT_SEL_BF16 || d->sel_fmt > SPOT_SEL_MXFP4_G32_E8M0)
+    if (d->sel_fmt < SPOT_SEL_BF16 || d->sel_fmt > SPOT_SEL_INT8_F16)
         return SPOT_ERR_INVALID_ARG;
     if (d->head_dim != kHeadDim || d->block_size != kBlock || d->sel_dim != kSelDim)
         return SPOT_ERR_UNSUPPORTED;
@@ -184,7 +189,7 @@ spot_status_t check_select_args(const spot_layer_desc_t* d, const spot_select_pa
     if (!q_sel || !sel_data || !page_table || !seq_lens || !sel_idx || !sel_cnt)
         return SPOT_ERR_INVALID_ARG;
     if (pr->mode == SPOT_MODE_TOPP && !top_p) return SPOT_ERR_INVALID_ARG;
-    if (d->sel_fmt != SPOT_SEL_BF16 && !sel_scales) return SPOT_ERR_INVALID_ARG;
+    if (needs_scales(d->sel_fmt) && !sel_scales) return SPOT_ERR_INVALID_ARG;
     if (pt_stride <= 0) return SPOT_ERR_INVALID_ARG;
     if (!aligned(q_sel, 16) || !aligned(sel_data, 16) || !aligned(page_table, 4) ||
         !aligned(seq_lens, 4) || !aligned(sel_idx, 4) || !aligned(sel_cnt, 4) ||
@@ -237,7 +242,7 @@ spot_status_t spot_append_selector_keys(const spot_layer_desc_t* desc, void* sel
     if (n < 0 || pt_stride <= 0 || num_seqs < 0) return SPOT_ERR_INVALID_ARG;
     if (n == 0) return SPOT_OK;
     if (!sel_data || !page_table || !seq_ids || !block_ids || !keys) return SPOT_ERR_INVALID_ARG;
-    if (desc->sel_fmt != SPOT_SEL_BF16 && !sel_scales) return SPOT_ERR_INVALID_ARG;
+    if (needs_scales(desc->sel_fmt) && !sel_scales) return SPOT_ERR_INVALID_ARG;
     if (!aligned(sel_data, 4) || !aligned(keys, 4) || !aligned(page_table, 4) ||
         !aligned(seq_ids, 4) || !aligned(block_ids, 4) || (sel_scales && !aligned(sel_scales, 2)))
         return SPOT_ERR_INVALID_ARG;

@@ -9,7 +9,14 @@
 //          code = clamp(rne(x / scale), -8, 7) (0 when the scale is 0);
 //   MXFP4: X = floor(log2 amax) - 2 in [-127, 127] (-127 for amax = 0),
 //          E8M0 = X + 127, code = E2M1 round-to-nearest-even of x / 2^X with
-//          saturation at 6 and the sign bit set for x < 0.
+//          saturation at 6 and the sign bit set for x < 0;
+//   FP8:   E4M3 round-to-nearest-even with saturation at +-448 (CUDA's
+//          satfinite conversion); zero is stored as +0;
+//   INT8:  scale = binary16 RNE of amax/127 over the whole key (saturating at
+//          65504), code = clamp(rne(x / scale), -128, 127).
+// For the 8-bit formats lane l writes bytes 2 l and 2 l + 1 of the 64-byte
+// code row.
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include "spot_device.cuh"
@@ -59,6 +66,32 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
         return;
     }
     const float x0 = bf16_bits_to_float(two & 0xFFFFu), x1 = bf16_bits_to_float(two >> 16);
+    if (p.fmt == SPOT_SEL_FP8_E4M3) {
+        uint32_t c0 = x0 == 0.f ? 0u : __nv_cvt_float_to_fp8(x0, __NV_SATFINITE, __NV_E4M3);
+        uint32_t c1 = x1 == 0.f ? 0u : __nv_cvt_float_to_fp8(x1, __NV_SATFINITE, __NV_E4M3);
+        reinterpret_cast<uint16_t*>(p.sel_data)[row * (kSelDim / 2) + lane] =
+            static_cast<uint16_t>(c0 | (c1 << 8));
+        return;
+    }
+    if (p.fmt == SPOT_SEL_INT8_F16) {
+        float km = fmaxf(fabsf(x0), fabsf(x1));
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o));
+        const double t = static_cast<double>(km) / 127.0;
+        const uint16_t sbits = (t >= 65504.0) ? static_cast<uint16_t>(0x7BFFu)
+                                              : __half_as_ushort(__double2half(t));
+        const double sc = static_cast<double>(__half2float(__ushort_as_half(sbits)));
+        int q0 = 0, q1 = 0;
+        if (sc > 0.0) {
+            q0 = static_cast<int>(fmin(127.0, fmax(-128.0, rint(static_cast<double>(x0) / sc))));
+            q1 = static_cast<int>(fmin(127.0, fmax(-128.0, rint(static_cast<double>(x1) / sc))));
+        }
+        reinterpret_cast<uint16_t*>(p.sel_data)[row * (kSelDim / 2) + lane] =
+            static_cast<uint16_t>((static_cast<uint32_t>(q0) & 0xFFu) |
+                                  ((static_cast<uint32_t>(q1) & 0xFFu) << 8));
+        if (lane == 0) reinterpret_cast<uint16_t*>(p.sel_scales)[row] = sbits;
+        return;
+    }
     float amax = fmaxf(fabsf(x0), fabsf(x1));
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));

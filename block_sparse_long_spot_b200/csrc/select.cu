@@ -5,9 +5,10 @@
 //   for every complete block j.  Each warp scores tiles of 16 blocks with
 //   bf16 mma.sync (keys as the M operand, the group's selector queries as
 //   N = 8), four tiles at a time so their gathered loads are in flight
-//   together.  INT4 / MXFP4 keys are widened to bf16 in registers (both code
-//   sets are exact in bf16) and the per-32 scales are applied to the two
-//   half-accumulators afterwards, so dequantisation is exact.  The head
+//   together.  INT4 / MXFP4 / INT8 / FP8 E4M3 keys are widened to bf16 in
+//   registers (all these code sets are exact in bf16) and the scales (per 32
+//   for INT4 / MXFP4, per key for INT8) are applied to the accumulators
+//   afterwards, so dequantisation is exact.  The head
 //   dimension is consumed in a permuted order, identical for the keys and the
 //   queries, that lets every lane load 16 contiguous bytes.  Scores stay in
 //   shared memory.
@@ -22,6 +23,7 @@
 //   blocks inside that bucket are ranked exactly (score descending, lower
 //   block index first).  The K_min floor and static top-K use the same search
 //   on counts.  A block scan compacts the kept blocks in ascending order.
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include "spot_device.cuh"
@@ -65,6 +67,20 @@ __device__ __forceinline__ uint32_t byte_to_bf16x2(uint32_t byte) {
     const uint32_t lo = byte & 0xFu, hi = (byte >> 4) & 0xFu;
     if (FMT == SPOT_SEL_INT4_G32_F16) return int4_bf16_bits(lo) | (int4_bf16_bits(hi) << 16);
     return e2m1_bf16_bits(lo) | (e2m1_bf16_bits(hi) << 16);
+}
+
+// Two 8-bit codes (the even element in the low byte) -> packed bf16x2 with
+// the even element in the low half; INT8 and E4M3 values are exact in bf16.
+template <int FMT>
+__device__ __forceinline__ uint32_t pair8_to_bf16x2(uint32_t two) {
+    if (FMT == SPOT_SEL_INT8_F16) {
+        const int lo = static_cast<int8_t>(two & 0xFFu), hi = static_cast<int8_t>((two >> 8) & 0xFFu);
+        return pack_bf16(static_cast<float>(lo), static_cast<float>(hi));
+    }
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu),
+                                                     __NV_E4M3);
+    const float2 f = __half22float2(__half2(hr));
+    return pack_bf16(f.x, f.y);
 }
 
 template <int FMT>
@@ -125,6 +141,36 @@ __device__ __forceinline__ void score_tiles(const SelectParams& p, int b, int g,
             for (int s = 0; s < 4; ++s)
                 mma_bf16_16816(acc[k], wa[2 * s], wb[2 * s], wa[2 * s + 1], wb[2 * s + 1],
                                qw[2 * s], qw[2 * s + 1]);
+        }
+    } else if (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
+        // 64-byte rows: lane c4 owns bytes (= dims) [16 c4, 16 c4 + 16)
+        uint4 ra[kTileBatch], rb[kTileBatch];
+        float sca[kTileBatch], scb[kTileBatch];
+#pragma unroll
+        for (int k = 0; k < kTileBatch; ++k) {
+            ra[k] = __ldg(reinterpret_cast<const uint4*>(p.sel_data) + rowa[k] * 4 + c4);
+            rb[k] = __ldg(reinterpret_cast<const uint4*>(p.sel_data) + rowb[k] * 4 + c4);
+            if (FMT == SPOT_SEL_INT8_F16) {
+                sca[k] = __half2float(reinterpret_cast<const __half*>(p.sel_scales)[rowa[k]]);
+                scb[k] = __half2float(reinterpret_cast<const __half*>(p.sel_scales)[rowb[k]]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kTileBatch; ++k) {
+            const uint32_t wa[4] = {ra[k].x, ra[k].y, ra[k].z, ra[k].w};
+            const uint32_t wb[4] = {rb[k].x, rb[k].y, rb[k].z, rb[k].w};
+            acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16_16816(acc[k], pair8_to_bf16x2<FMT>(wa[s]), pair8_to_bf16x2<FMT>(wb[s]),
+                               pair8_to_bf16x2<FMT>(wa[s] >> 16), pair8_to_bf16x2<FMT>(wb[s] >> 16),
+                               qw[2 * s], qw[2 * s + 1]);
+            if (FMT == SPOT_SEL_INT8_F16) {
+                acc[k][0] *= sca[k];
+                acc[k][1] *= sca[k];
+                acc[k][2] *= scb[k];
+                acc[k][3] *= scb[k];
+            }
         }
     } else {
         uint32_t ga0[kTileBatch], ga1[kTileBatch], gb0[kTileBatch], gb1[kTileBatch];
@@ -193,10 +239,10 @@ __device__ __forceinline__ void load_queries(const SelectParams& p, int b, int g
     const int h = g * G + (real ? r8 : 0);
     const uint4* qrow = reinterpret_cast<const uint4*>(
         p.q_sel + (static_cast<int64_t>(b) * p.num_q_heads + h) * kSelDim);
-    // bf16 keys: lane c4 owns dims [16 c4, 16 c4 + 16);
+    // bf16 / 8-bit keys: lane c4 owns dims [16 c4, 16 c4 + 16);
     // 4-bit keys: dims [8 c4, 8 c4 + 8) and [32 + 8 c4, 32 + 8 c4 + 8).
     uint4 x0, x1;
-    if (FMT == SPOT_SEL_BF16) {
+    if (FMT == SPOT_SEL_BF16 || FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
         x0 = real ? __ldg(qrow + 2 * c4) : make_uint4(0, 0, 0, 0);
         x1 = real ? __ldg(qrow + 2 * c4 + 1) : make_uint4(0, 0, 0, 0);
     } else {
@@ -700,10 +746,18 @@ cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s) {
         e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_INT4_G32_F16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e == cudaSuccess) select_kernel<SPOT_SEL_INT4_G32_F16><<<grid, block, smem, s>>>(p);
-    } else {
+    } else if (fmt == SPOT_SEL_MXFP4_G32_E8M0) {
         e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_MXFP4_G32_E8M0>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e == cudaSuccess) select_kernel<SPOT_SEL_MXFP4_G32_E8M0><<<grid, block, smem, s>>>(p);
+    } else if (fmt == SPOT_SEL_FP8_E4M3) {
+        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_FP8_E4M3>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess) select_kernel<SPOT_SEL_FP8_E4M3><<<grid, block, smem, s>>>(p);
+    } else {
+        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_INT8_F16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess) select_kernel<SPOT_SEL_INT8_F16><<<grid, block, smem, s>>>(p);
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -10,8 +10,8 @@
  *     (Eq. 8); softmax temperature 1.0 by default (App. A, Tab. 3);
  *   - sparse attention: the layer attends only to the keys of the selected
  *     blocks, at decode only (§2.3, §3 "Evaluation");
- *   - selector K-cache stored in bf16, INT4 or FP4 group-32 microscale
- *     (§5.3, App. G Tab. 9).
+ *   - selector K-cache stored in bf16, INT8, FP8 or INT4 / FP4 group-32
+ *     microscale (§5.3, App. G Tab. 9).
  *
  * Conventions for every call:
  *   - All array arguments are DEVICE pointers of the current CUDA device,
@@ -39,9 +39,11 @@
  *   sel_data     bf16  [num_pages][num_kv_heads][sel_dim]         (BF16)
  *                u8    [num_pages][num_kv_heads][sel_dim/2]       (INT4, MXFP4)
  *                      two elements per byte, even element in the low nibble
+ *                u8    [num_pages][num_kv_heads][sel_dim]         (FP8 E4M3, INT8)
  *   sel_scales   fp16  [num_pages][num_kv_heads][sel_dim/32]      (INT4)
  *                u8    [num_pages][num_kv_heads][sel_dim/32]      (MXFP4, E8M0)
- *                      unused (may be NULL) for BF16
+ *                fp16  [num_pages][num_kv_heads][1]               (INT8)
+ *                      unused (may be NULL) for BF16 and FP8
  *   page_table   int32 [batch][pt_stride]: logical block j of sequence b is
  *                      pool page page_table[b*pt_stride + j] in the KV pools
  *                      and in the selector pool alike
@@ -82,7 +84,9 @@ typedef enum {
 typedef enum {
     SPOT_SEL_BF16 = 0,            /* bf16 keys */
     SPOT_SEL_INT4_G32_F16 = 1,    /* int4 codes, one fp16 scale per 32 (symmetric) */
-    SPOT_SEL_MXFP4_G32_E8M0 = 2   /* OCP MX v1.0 MXFP4: E2M1 codes, one E8M0 per 32 */
+    SPOT_SEL_MXFP4_G32_E8M0 = 2,  /* OCP MX v1.0 MXFP4: E2M1 codes, one E8M0 per 32 */
+    SPOT_SEL_FP8_E4M3 = 3,        /* OCP FP8 E4M3 codes, no scale (0.5x bf16) */
+    SPOT_SEL_INT8_F16 = 4         /* int8 codes, one fp16 scale per key (symmetric) */
 } spot_sel_fmt_t;
 
 /* Selection rule (§2.3). */
@@ -129,7 +133,12 @@ size_t spot_workspace_size(const spot_layer_desc_t* desc, int32_t batch, int32_t
  * MXFP4: shared exponent X = floor(log2 amax) - 2 clamped to [-127, 127],
  *        stored as X + 127; elements rounded to nearest even on the E2M1
  *        grid, saturating at 6; sign bit set for x < 0.
- * Cites §5.3 and App. G (group-32 INT4 / FP4 microscale selector K-cache).
+ * FP8:   each element rounded to nearest even on the E4M3 grid, saturating
+ *        at +-448; sign bit set for x < 0.
+ * INT8:  scale = fp16 round-to-nearest-even of amax/127 over the key
+ *        (saturating at 65504), code = clamp(rne(x/scale), -128, 127).
+ * Cites §5.3 and App. G Tab. 9 (INT8, FP8 and group-32 INT4 / FP4
+ * microscale selector K-cache).
  * Entries whose sequence, block or page id is out of range are skipped and
  * recorded in the status word of `status_ws` (a workspace, may be NULL: not
  * recorded). */

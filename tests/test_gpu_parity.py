@@ -54,6 +54,7 @@ INTEGER_CASES = [
     ("qwen3_4b_32k", dict(seq_len=8192), "bf16"),
     ("qwen3_32b_128k", dict(seq_len=16384, batch=2), "bf16"),
     ("quant_128k", dict(seq_len=8192, batch=4), "mxfp4"),
+    ("quant_128k", dict(seq_len=8192, batch=4), "fp8"),
     ("ragged_hybrid", dict(batch=8, ragged_range=(512, 8192)), "bf16"),
 ]
 
@@ -61,7 +62,7 @@ INTEGER_CASES = [
 @pytest.mark.parametrize("name,kw,fmt", INTEGER_CASES)
 def test_integer_inputs_select_bit_exact(name, kw, fmt):
     # Selector queries and keys in {-3..3}: every score is exact in fp32 and
-    # fp64 (MXFP4 stores these values losslessly), so the selected sets must
+    # fp64 (MXFP4 and FP8 E4M3 store these values losslessly), so the selected sets must
     # be identical; p is placed away from every cumulative mass.
     wl = workloads.make(name, seed=11, device=DEV, integer=True, **kw)
     wl.top_p = safe_top_p(wl, fmt)
@@ -82,7 +83,7 @@ def test_integer_inputs_topk_and_kmin_modes():
         check_outputs(gpu, ora, wl)
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["bf16", "int4", "mxfp4", "fp8", "int8"])
 def test_append_matches_oracle_quantiser(fmt):
     wl = workloads.make("qwen3_4b_32k", seed=3, device=DEV, seq_len=4096 + 64 * 7)
     data, scales = gpu_selector_pool(wl, fmt, DEV)
@@ -90,10 +91,12 @@ def test_append_matches_oracle_quantiser(fmt):
     g_data = data.cpu().view(torch.int16).numpy().view(np.uint16) if fmt == "bf16" \
         else data.cpu().numpy()
     assert np.array_equal(g_data, o_data)
-    if fmt != "bf16":
-        g_scales = scales.cpu().view(torch.int16).numpy().view(np.uint16) if fmt == "int4" \
-            else scales.cpu().numpy()
+    if o_scales is not None:
+        g_scales = scales.cpu().view(torch.int16).numpy().view(np.uint16) \
+            if fmt in ("int4", "int8") else scales.cpu().numpy()
         assert np.array_equal(g_scales, o_scales)
+    else:
+        assert scales is None
 
 
 def test_append_extreme_values_match_oracle():
@@ -106,17 +109,19 @@ def test_append_extreme_values_match_oracle():
     x[3] = -x[3].abs()
     keys = x.to(torch.bfloat16).to(DEV)
     pt = torch.arange(rows, dtype=torch.int32, device=DEV).view(1, rows)
-    for fmt in ("int4", "mxfp4"):
+    for fmt in ("int4", "mxfp4", "fp8", "int8"):
         desc = spot.layer_desc(1, 1, rows, fmt)
         data, scales = spot.selector_pool(fmt, rows, 1, device=DEV)
         spot.append_selector_keys(desc, data, scales, pt,
                                   torch.zeros(rows, dtype=torch.int32, device=DEV),
                                   torch.arange(rows, dtype=torch.int32, device=DEV), keys)
         o_data, o_scales = oracle.quantize_selector(fmt, workloads.bits(keys))
-        assert np.array_equal(data.cpu().numpy(), o_data)
-        sc = scales.cpu()
-        sc = sc.view(torch.int16).numpy().view(np.uint16) if fmt == "int4" else sc.numpy()
-        assert np.array_equal(sc, o_scales)
+        assert np.array_equal(data.cpu().numpy(), o_data), fmt
+        if o_scales is not None:
+            sc = scales.cpu()
+            sc = sc.view(torch.int16).numpy().view(np.uint16) if fmt in ("int4", "int8") \
+                else sc.numpy()
+            assert np.array_equal(sc, o_scales), fmt
 
 
 def test_sparse_decode_on_oracle_selection():
@@ -147,6 +152,8 @@ FULL = [
     ("qwen3_32b_128k", "bf16", [0, 3]),
     ("quant_128k", "int4", [1, 14]),
     ("quant_128k", "mxfp4", [0, 9]),
+    ("quant_128k", "fp8", [3, 12]),
+    ("quant_128k", "int8", [2, 11]),
     ("ragged_hybrid", "mxfp4", [0, 7, 31]),
 ]
 
