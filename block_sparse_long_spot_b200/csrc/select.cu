@@ -98,21 +98,34 @@ __device__ __forceinline__ float group_scale(const void* scales, int64_t row, in
 
 
 // Scores of tiles t0, t0 + stride, ... (kTileBatch of them) of 16 blocks
-// each, for KV head g of sequence b, into scores[j] (j < n_full).  qw: the
-// group's selector queries as mma B fragments (lane: head r8); wh0 / wh1:
-// weights of heads 2 c4, 2 c4 + 1 (0 for padding heads).
+// each, for KV head g, into scores[j] (j < n_full), given the blocks' page
+// ids (load_pages).  qw: the group's selector queries as mma B fragments
+// (lane: head r8); wh0 / wh1: weights of heads 2 c4, 2 c4 + 1 (0 for
+// padding heads).
+// Page ids of the blocks of tiles t0, t0 + stride, ... (rows r8 and r8 + 8).
+__device__ __forceinline__ void load_pages(const SelectParams& p, int b, int t0, int stride,
+                                           int n_full, int lane, int (&pa)[kTileBatch],
+                                           int (&pb)[kTileBatch]) {
+    const int r8 = lane >> 2;
+#pragma unroll
+    for (int k = 0; k < kTileBatch; ++k) {
+        const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
+        pa[k] = (ja < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + ja] : 0;
+        pb[k] = (jb < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + jb] : 0;
+    }
+}
+
 template <int FMT>
-__device__ __forceinline__ void score_tiles(const SelectParams& p, int b, int g,
+__device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
                                             const uint32_t (&qw)[8], float wh0, float wh1,
                                             int t0, int stride, int n_full, float* scores,
-                                            int lane) {
+                                            int lane, const int (&pga)[kTileBatch],
+                                            const int (&pgb)[kTileBatch]) {
     const int c4 = lane & 3, r8 = lane >> 2;
     int64_t rowa[kTileBatch], rowb[kTileBatch];
 #pragma unroll
     for (int k = 0; k < kTileBatch; ++k) {
-        const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
-        int pa = (ja < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + ja] : 0;
-        int pb = (jb < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + jb] : 0;
+        int pa = pga[k], pb = pgb[k];
         if (pa < 0 || pa >= p.num_pages) { flag_status(p.status, kStatusBounds); pa = 0; }
         if (pb < 0 || pb >= p.num_pages) { flag_status(p.status, kStatusBounds); pb = 0; }
         rowa[k] = static_cast<int64_t>(pa) * p.num_kv_heads + g;
@@ -392,18 +405,21 @@ struct Cut {
 // score, lower block index first) whose cumulative mass (or count) added to
 // `above` reaches `target`; writes the keep flags of the bucket's elements.
 __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long long above,
-                              unsigned long long target, bool by_mass) {
+                              unsigned long long target, bool by_mass, bool gathered = false) {
     const int c = static_cast<int>(sm.hcnt[b]);
-    // (the caller has set sm.misc[3] = 0 before its last barrier)
+    // (the caller has set sm.misc[3] = 0 before its last barrier, or, with
+    // `gathered`, already collected the bucket's candidates behind a barrier)
     if (c <= 32) {
-        for (int i = threadIdx.x; i < n; i += NT) {
-            if (sm.vb[i] == b) {
-                const int slot = atomicAdd(&sm.misc[3], 1);
-                sm.ckey[slot] = sm.keys[i];
-                sm.cidx[slot] = i;
+        if (!gathered) {
+            for (int i = threadIdx.x; i < n; i += NT) {
+                if (sm.vb[i] == b) {
+                    const int slot = atomicAdd(&sm.misc[3], 1);
+                    sm.ckey[slot] = sm.keys[i];
+                    sm.cidx[slot] = i;
+                }
             }
+            __syncthreads();
         }
-        __syncthreads();
         if (threadIdx.x < 32) {                       // one warp ranks the few candidates
             const int lane = threadIdx.x;
             int rank = 0, j = -1;
@@ -596,8 +612,17 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
         float wh0, wh1;
         load_queries<FMT>(p, b, g, lane, qw, wh0, wh1);
         const int tiles = (n_full + 15) / 16;
-        for (int t0 = warp; t0 < tiles; t0 += NW * kTileBatch)
-            score_tiles<FMT>(p, b, g, qw, wh0, wh1, t0, NW, n_full, sm.score, lane);
+        const int step = NW * kTileBatch;
+        int pa[kTileBatch], pb[kTileBatch];
+        if (warp < tiles) load_pages(p, b, warp, NW, n_full, lane, pa, pb);
+        for (int t0 = warp; t0 < tiles; t0 += step) {
+            // the next batch's page ids load while this batch's keys do
+            int na[kTileBatch], nb2[kTileBatch];
+            if (t0 + step < tiles) load_pages(p, b, t0 + step, NW, n_full, lane, na, nb2);
+            score_tiles<FMT>(p, g, qw, wh0, wh1, t0, NW, n_full, sm.score, lane, pa, pb);
+#pragma unroll
+            for (int k = 0; k < kTileBatch; ++k) { pa[k] = na[k]; pb[k] = nb2[k]; }
+        }
     }
     __syncthreads();
 
@@ -649,19 +674,37 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
             ceil(static_cast<double>(p.top_p[b]) * static_cast<double>(Z)));
         T = T < 1ull ? 1ull : (T > Z ? Z : T);
         int before;
+        if (threadIdx.x == 0) sm.misc[3] = 0;
         int bk = cut_bucket(sm, ldexp(static_cast<double>(T), kApproxShift - kFixShift), true,
                             &before);
-        // exact check of the bucket on the fixed-point masses; step to the
-        // neighbouring non-empty bucket while the fp32 estimate was off
+        // Exact check of the bucket on the fixed-point masses.  The first
+        // pass also writes the keep flags and gathers the bucket's candidates
+        // (sm.misc[3] was zeroed before cut_bucket's barriers); if the
+        // approximate bucket was off, step to the neighbouring non-empty
+        // bucket and redo the flags and the gather.
         unsigned long long A, Bm, Ac;
-        for (int guard = 0; guard < kNB; ++guard) {
+        const bool small = sm.hcnt[bk] <= 32u;
+        {
             A = 0; Bm = 0; Ac = 0;
             for (int i = threadIdx.x; i < n; i += NT) {
                 const int v = sm.vb[i];
-                if (v < bk) { A += sm.mass[i]; ++Ac; }
-                else if (v == bk) Bm += sm.mass[i];
+                sm.keep[i] = v < bk ? 1 : 0;
+                if (v < bk) {
+                    A += sm.mass[i];
+                    ++Ac;
+                } else if (v == bk) {
+                    Bm += sm.mass[i];
+                    if (small) {
+                        const int slot = atomicAdd(&sm.misc[3], 1);
+                        sm.ckey[slot] = sm.keys[i];
+                        sm.cidx[slot] = i;
+                    }
+                }
             }
             block_sum3(sm, A, Bm, Ac);
+        }
+        bool gathered = small;
+        for (int guard = 0; guard < kNB; ++guard) {
             int step = 0;
             if (A >= T) step = -1;
             else if (A + Bm < T) step = 1;
@@ -670,11 +713,21 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
             while (nbk >= 0 && nbk < kNB && sm.hcnt[nbk] == 0) nbk += step;
             if (nbk < 0 || nbk >= kNB) break;
             bk = nbk;
+            gathered = false;
+            A = 0; Bm = 0; Ac = 0;
+            for (int i = threadIdx.x; i < n; i += NT) {
+                const int v = sm.vb[i];
+                if (v < bk) { A += sm.mass[i]; ++Ac; }
+                else if (v == bk) Bm += sm.mass[i];
+            }
+            block_sum3(sm, A, Bm, Ac);
         }
-        if (threadIdx.x == 0) sm.misc[3] = 0;
-        for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
-        __syncthreads();
-        n_take = static_cast<int>(Ac) + resolve_bucket(sm, n, bk, A, T, true);
+        if (!gathered) {
+            if (threadIdx.x == 0) sm.misc[3] = 0;
+            for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
+            __syncthreads();
+        }
+        n_take = static_cast<int>(Ac) + resolve_bucket(sm, n, bk, A, T, true, gathered);
         done = true;
         const int floor_res = p.kmin_blocks - n_reserved;      // |S| >= K_min
         if (n_take < floor_res) {
