@@ -44,7 +44,8 @@ class LayerDesc(ctypes.Structure):
 class SelectParams(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("sink_blocks", ctypes.c_int32),
                 ("recency_blocks", ctypes.c_int32), ("kmin_blocks", ctypes.c_int32),
-                ("topk_blocks", ctypes.c_int32), ("temperature", ctypes.c_float)]
+                ("topk_blocks", ctypes.c_int32), ("temperature", ctypes.c_float),
+                ("quantize_queries", ctypes.c_int32)]
 
 
 def layer_desc(num_q_heads, num_kv_heads, num_pages, sel_fmt="bf16", head_dim=128,
@@ -54,9 +55,10 @@ def layer_desc(num_q_heads, num_kv_heads, num_pages, sel_fmt="bf16", head_dim=12
 
 
 def select_params(mode="topp", sink_blocks=1, recency_blocks=4, kmin_blocks=8, topk_blocks=0,
-                  temperature=1.0) -> SelectParams:
+                  temperature=1.0, quantize_queries=False) -> SelectParams:
     return SelectParams(MODE[mode] if isinstance(mode, str) else int(mode), sink_blocks,
-                        recency_blocks, kmin_blocks, topk_blocks, float(temperature))
+                        recency_blocks, kmin_blocks, topk_blocks, float(temperature),
+                        1 if quantize_queries else 0)
 
 
 _lib = None

@@ -50,6 +50,7 @@ spot_status_t check_params(const spot_select_params_t* pr) {
         pr->topk_blocks < 0)
         return SPOT_ERR_INVALID_ARG;
     if (!(pr->temperature > 0.f) || !isfinite(pr->temperature)) return SPOT_ERR_INVALID_ARG;
+    if (pr->quantize_queries != 0 && pr->quantize_queries != 1) return SPOT_ERR_INVALID_ARG;
     return SPOT_OK;
 }
 
@@ -138,6 +139,7 @@ spot_status_t do_select(const spot_layer_desc_t* d, const spot_select_params_t* 
     sl.recency_blocks = pr->recency_blocks;
     sl.kmin_blocks = pr->kmin_blocks;
     sl.topk_blocks = pr->topk_blocks;
+    sl.quantize_queries = pr->quantize_queries;
     sl.sel_idx = sel_idx;
     sl.sel_cnt = sel_cnt;
     sl.status = reinterpret_cast<uint32_t*>(base + L.status);

@@ -8,7 +8,9 @@
 //   together.  INT4 / MXFP4 / INT8 / FP8 E4M3 keys are widened to bf16 in
 //   registers (all these code sets are exact in bf16) and the scales (per 32
 //   for INT4 / MXFP4, per key for INT8) are applied to the accumulators
-//   afterwards, so dequantisation is exact.  The head
+//   afterwards, so dequantisation is exact.  With quantize_queries the
+//   group's selector queries are first quantised with the key format's rule
+//   (quant.cuh) and their scales join the keys' after the mma.  The head
 //   dimension is consumed in a permuted order, identical for the keys and the
 //   queries, that lets every lane load 16 contiguous bytes.  Scores stay in
 //   shared memory.
@@ -26,6 +28,7 @@
 #include <cuda_fp8.h>
 #include <math.h>
 
+#include "quant.cuh"
 #include "spot_device.cuh"
 #include "spot_internal.h"
 
@@ -117,8 +120,8 @@ __device__ __forceinline__ void load_pages(const SelectParams& p, int b, int t0,
 
 template <int FMT>
 __device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
-                                            const uint32_t (&qw)[8], float wh0, float wh1,
-                                            int t0, int stride, int n_full, float* scores,
+                                            const uint32_t (&qw)[8], const float (&qsc)[2][2],
+                                            float wh0, float wh1, int t0, int stride, int n_full, float* scores,
                                             int lane, const int (&pga)[kTileBatch],
                                             const int (&pgb)[kTileBatch]) {
     const int c4 = lane & 3, r8 = lane >> 2;
@@ -179,10 +182,10 @@ __device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
                                pair8_to_bf16x2<FMT>(wa[s] >> 16), pair8_to_bf16x2<FMT>(wb[s] >> 16),
                                qw[2 * s], qw[2 * s + 1]);
             if (FMT == SPOT_SEL_INT8_F16) {
-                acc[k][0] *= sca[k];
-                acc[k][1] *= sca[k];
-                acc[k][2] *= scb[k];
-                acc[k][3] *= scb[k];
+                acc[k][0] = acc[k][0] * sca[k] * qsc[0][0];
+                acc[k][1] = acc[k][1] * sca[k] * qsc[0][1];
+                acc[k][2] = acc[k][2] * scb[k] * qsc[0][0];
+                acc[k][3] = acc[k][3] * scb[k] * qsc[0][1];
             }
         }
     } else {
@@ -218,10 +221,10 @@ __device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
                                byte_to_bf16x2<FMT>((gb1[k] >> (16 * s + 8)) & 0xFFu),
                                qw[4 + 2 * s], qw[4 + 2 * s + 1]);
             }
-            acc[k][0] = acc0[0] * sa0[k] + acc1[0] * sa1[k];
-            acc[k][1] = acc0[1] * sa0[k] + acc1[1] * sa1[k];
-            acc[k][2] = acc0[2] * sb0[k] + acc1[2] * sb1[k];
-            acc[k][3] = acc0[3] * sb0[k] + acc1[3] * sb1[k];
+            acc[k][0] = acc0[0] * sa0[k] * qsc[0][0] + acc1[0] * sa1[k] * qsc[1][0];
+            acc[k][1] = acc0[1] * sa0[k] * qsc[0][1] + acc1[1] * sa1[k] * qsc[1][1];
+            acc[k][2] = acc0[2] * sb0[k] * qsc[0][0] + acc1[2] * sb1[k] * qsc[1][0];
+            acc[k][3] = acc0[3] * sb0[k] * qsc[0][1] + acc1[3] * sb1[k] * qsc[1][1];
         }
     }
     // epilogue: weighted ReLU sum over the group's heads (columns 2 c4, 2 c4 + 1)
@@ -241,11 +244,54 @@ __device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
     }
 }
 
-// Selector queries of head group g as mma B fragments (lane: head r8) and
-// the weights of heads 2 c4, 2 c4 + 1.
+// Quantises this lane's 16 query elements f (two halves of 8, see
+// load_queries) with the key format's rule and replaces them by their codes'
+// values (exact in bf16).  qs[h]: the scale of half h, the query head's
+// group scale for the 4-bit formats (half 0 lies in dims 0-31, half 1 in
+// dims 32-63) and its per-head scale for INT8; 1 for FP8.  The four lanes of
+// a quad (same r8) hold one query head between them.
+template <int FMT>
+__device__ __forceinline__ void quantize_query(float (&f)[16], float (&qs)[2]) {
+    if (FMT == SPOT_SEL_FP8_E4M3) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) f[i] = fp8_value(fp8_code(f[i]));
+        qs[0] = qs[1] = 1.f;
+        return;
+    }
+    float am[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) am[i >> 3] = fmaxf(am[i >> 3], fabsf(f[i]));
+    if (FMT == SPOT_SEL_INT8_F16) am[0] = am[1] = fmaxf(am[0], am[1]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        am[h] = fmaxf(am[h], __shfl_xor_sync(0xffffffffu, am[h], 1));
+        am[h] = fmaxf(am[h], __shfl_xor_sync(0xffffffffu, am[h], 2));
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (FMT == SPOT_SEL_MXFP4_G32_E8M0) {
+            const int X = mx_exponent(am[h]);
+#pragma unroll
+            for (int i = 8 * h; i < 8 * h + 8; ++i) f[i] = e2m1_value(mx_code(f[i], X));
+            qs[h] = ldexpf(1.f, X);
+        } else {
+            const bool i8 = FMT == SPOT_SEL_INT8_F16;
+            const float sc = f16_bits_value(f16_scale_bits(am[h], i8 ? 127.0 : 7.0));
+#pragma unroll
+            for (int i = 8 * h; i < 8 * h + 8; ++i)
+                f[i] = static_cast<float>(int_code(f[i], sc, i8 ? -128 : -8, i8 ? 127 : 7));
+            qs[h] = sc;
+        }
+    }
+}
+
+// Selector queries of head group g as mma B fragments (lane: head r8), the
+// weights of heads 2 c4, 2 c4 + 1, and the query scales of those two heads
+// qsc[half][column] (all 1 unless the queries are quantised).
 template <int FMT>
 __device__ __forceinline__ void load_queries(const SelectParams& p, int b, int g, int lane,
-                                             uint32_t (&qw)[8], float& wh0, float& wh1) {
+                                             uint32_t (&qw)[8], float (&qsc)[2][2], float& wh0,
+                                             float& wh1) {
     const int c4 = lane & 3, r8 = lane >> 2;
     const int G = p.group;
     const bool real = r8 < G;
@@ -264,6 +310,26 @@ __device__ __forceinline__ void load_queries(const SelectParams& p, int b, int g
     }
     qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
     qw[4] = x1.x; qw[5] = x1.y; qw[6] = x1.z; qw[7] = x1.w;
+    qsc[0][0] = qsc[0][1] = qsc[1][0] = qsc[1][1] = 1.f;
+    if (FMT != SPOT_SEL_BF16 && p.quantize_queries) {
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[2 * i] = __uint_as_float(qw[i] << 16);
+            f[2 * i + 1] = __uint_as_float(qw[i] & 0xFFFF0000u);
+        }
+        float qs[2];
+        quantize_query<FMT>(f, qs);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qw[i] = pack_bf16(f[2 * i], f[2 * i + 1]);
+        // column 0 / 1 of this lane's accumulators = heads 2 c4 / 2 c4 + 1,
+        // whose scales sit in lanes 4 * (2 c4) and 4 * (2 c4 + 1)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            qsc[hf][0] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4);
+            qsc[hf][1] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4 + 4);
+        }
+    }
     const int64_t wrow = static_cast<int64_t>(b) * p.num_q_heads + g * G;
     wh0 = (2 * c4 < G) ? (p.w ? p.w[wrow + 2 * c4] : 1.f / G) : 0.f;
     wh1 = (2 * c4 + 1 < G) ? (p.w ? p.w[wrow + 2 * c4 + 1] : 1.f / G) : 0.f;
@@ -609,8 +675,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     {
         const int g = u - b * p.num_kv_heads;
         uint32_t qw[8];
-        float wh0, wh1;
-        load_queries<FMT>(p, b, g, lane, qw, wh0, wh1);
+        float qsc[2][2], wh0, wh1;
+        load_queries<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
         const int tiles = (n_full + 15) / 16;
         const int step = NW * kTileBatch;
         int pa[kTileBatch], pb[kTileBatch];
@@ -619,7 +685,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
             // the next batch's page ids load while this batch's keys do
             int na[kTileBatch], nb2[kTileBatch];
             if (t0 + step < tiles) load_pages(p, b, t0 + step, NW, n_full, lane, na, nb2);
-            score_tiles<FMT>(p, g, qw, wh0, wh1, t0, NW, n_full, sm.score, lane, pa, pb);
+            score_tiles<FMT>(p, g, qw, qsc, wh0, wh1, t0, NW, n_full, sm.score, lane, pa, pb);
 #pragma unroll
             for (int k = 0; k < kTileBatch; ++k) { pa[k] = na[k]; pb[k] = nb2[k]; }
         }

@@ -55,6 +55,7 @@ struct SelectParams {
     int32_t batch, num_q_heads, num_kv_heads, group, num_pages, max_blocks;
     float inv_temp;
     int32_t mode, sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
+    int32_t quantize_queries;           // quantise q_sel with the key format's rule
     int32_t* sel_idx;
     int32_t* sel_cnt;
     uint32_t* status;

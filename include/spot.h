@@ -113,6 +113,11 @@ typedef struct {
     int32_t kmin_blocks;          /* |S| >= min(K_min, nb) in TOPP mode */
     int32_t topk_blocks;          /* residual blocks kept in TOPK mode */
     float temperature;            /* scores are divided by it; > 0 */
+    int32_t quantize_queries;     /* 0: bf16 selector queries; 1: each query head is
+                                     first quantised with the key format's own rule
+                                     (group-32 INT4 / MXFP4, per-head INT8, FP8 E4M3;
+                                     §5.3 and App. G Tab. 9 quantise queries and
+                                     keys together); no effect for bf16 keys */
 } spot_select_params_t;
 
 /* Bytes of scratch the select / sparse-decode / decode-step calls need for

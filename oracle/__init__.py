@@ -57,7 +57,8 @@ class Shape(ctypes.Structure):
 class Params(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("sink_blocks", ctypes.c_int32),
                 ("recency_blocks", ctypes.c_int32), ("kmin_blocks", ctypes.c_int32),
-                ("topk_blocks", ctypes.c_int32), ("temperature", ctypes.c_double)]
+                ("topk_blocks", ctypes.c_int32), ("temperature", ctypes.c_double),
+                ("quantize_queries", ctypes.c_int32)]
 
 
 def _load():
@@ -98,9 +99,9 @@ def make_shape(batch, num_q_heads, num_kv_heads, head_dim, block_size, sel_dim, 
 
 
 def make_params(mode="topp", sink_blocks=1, recency_blocks=4, kmin_blocks=8, topk_blocks=0,
-                temperature=1.0) -> Params:
+                temperature=1.0, quantize_queries=False) -> Params:
     return Params(MODE[mode] if isinstance(mode, str) else mode, sink_blocks, recency_blocks,
-                  kmin_blocks, topk_blocks, float(temperature))
+                  kmin_blocks, topk_blocks, float(temperature), 1 if quantize_queries else 0)
 
 
 def _data_dtype(fmt):
@@ -198,7 +199,7 @@ def decode_step(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, q,
     lse = np.zeros((B, Hq))
     fmt = shape.sel_fmt
     u = None if units is None else _c(units, np.int32)
-    _load().oracle_decode_step(
+    rc = _load().oracle_decode_step(
         ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_sel, np.uint16)),
         _ptr(_c(w, np.float32)), _ptr(_c(sel_data, _data_dtype(_FMT_NAME[fmt]))),
         _ptr(_c(sel_scales, _scale_dtype(_FMT_NAME[fmt]))), _ptr(_c(q, np.uint16)),
@@ -206,4 +207,5 @@ def decode_step(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, q,
         _ptr(_c(seq_lens, np.int32)), _ptr(_c(top_p, np.float32)), float(sm_scale), _ptr(u),
         0 if u is None else len(u), _ptr(sel_idx), _ptr(sel_cnt), _ptr(mass), _ptr(out),
         _ptr(lse))
+    assert rc == 0
     return {"sel_idx": sel_idx, "sel_cnt": sel_cnt, "nuc_mass": mass, "out": out, "lse": lse}

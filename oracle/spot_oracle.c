@@ -310,17 +310,45 @@ typedef struct {
     int32_t mode;          /* ORC_MODE_TOPP (Eq. 8) or ORC_MODE_TOPK (Eq. 6) */
     int32_t sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
     double temperature;
+    int32_t quantize_queries;  /* 1: selector queries quantised like the keys */
 } orc_params_t;
 
 static int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+/* Selector queries of KV head g's G query heads for sequence b, as fp64
+ * [G][ds].  With quantize_queries (SpotAttention §5.3 and App. G Tab. 9: the
+ * selector's queries and key cache are quantised together, at inference)
+ * each query row goes through the same quantiser as a key row of the
+ * selector format and is read back exactly; otherwise the bf16 values are
+ * widened.  Returns 0, or -1 for an unknown format. */
+static int unit_queries(const orc_shape_t* sh, const orc_params_t* pr, int b, int g,
+                        const uint16_t* q_sel, double* qv) {
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    int ds = sh->sel_dim;
+    const uint16_t* q0 = q_sel + ((int64_t)b * sh->num_q_heads + (int64_t)g * G) * ds;
+    if (!pr->quantize_queries || sh->sel_fmt == ORC_FMT_BF16) {
+        for (int64_t i = 0; i < (int64_t)G * ds; ++i) qv[i] = bf16_to_f64(q0[i]);
+        return 0;
+    }
+    /* room for the largest row of codes (ds bytes) and scales (ds/32 x 2 bytes) */
+    uint8_t* codes = (uint8_t*)malloc((size_t)G * ds);
+    uint16_t* scales = (uint16_t*)malloc((size_t)G * (ds / 32 + 1) * sizeof(uint16_t));
+    int rc = (codes && scales) ? 0 : -2;
+    if (rc == 0) rc = oracle_quantize_selector(sh->sel_fmt, G, ds, q0, codes, scales);
+    if (rc == 0) rc = oracle_dequant_selector(sh->sel_fmt, G, ds, codes, scales, qv);
+    free(codes);
+    free(scales);
+    return rc;
+}
+
 /* Selector score for every complete block of sequence b, KV head g
  * (SpotAttention §2.1: s = sum_h w_h ReLU(q^I_h . k^I); block score = max
  * over the block's keys, §2.3, which is the single key here; temperature
- * from App. A Tab. 3).  keys_f64 = dequantised selector pool
- * [num_pages][Hkv][ds].  Writes n_full scores into out. */
+ * from App. A Tab. 3).  qv = the unit's queries from unit_queries;
+ * keys_f64 = dequantised selector pool [num_pages][Hkv][ds].  Writes n_full
+ * scores into out. */
 static void unit_scores(const orc_shape_t* sh, const orc_params_t* pr, int b, int g,
-                        const uint16_t* q_sel, const float* w, const double* keys_f64,
+                        const double* qv, const float* w, const double* keys_f64,
                         const int32_t* page_table, int64_t n_full, double* out) {
     int G = sh->num_q_heads / sh->num_kv_heads;
     int ds = sh->sel_dim;
@@ -330,9 +358,9 @@ static void unit_scores(const orc_shape_t* sh, const orc_params_t* pr, int b, in
         double s = 0.0;
         for (int i = 0; i < G; ++i) {
             int h = g * G + i;
-            const uint16_t* q = q_sel + ((int64_t)b * sh->num_q_heads + h) * ds;
+            const double* q = qv + (int64_t)i * ds;
             double dot = 0.0;
-            for (int d = 0; d < ds; ++d) dot += bf16_to_f64(q[d]) * k[d];
+            for (int d = 0; d < ds; ++d) dot += q[d] * k[d];
             double wh = w ? (double)w[(int64_t)b * sh->num_q_heads + h] : 1.0 / G;
             s += wh * (dot > 0.0 ? dot : 0.0);
         }
@@ -352,12 +380,19 @@ int oracle_block_scores(const orc_shape_t* sh, const orc_params_t* pr, const uin
         free(keys);
         return -1;
     }
-    for (int b = 0; b < sh->batch; ++b)
-        for (int g = 0; g < sh->num_kv_heads; ++g)
-            unit_scores(sh, pr, b, g, q_sel, w, keys, page_table, seq_lens[b] / sh->block_size,
-                        scores + ((int64_t)b * sh->num_kv_heads + g) * sh->max_blocks);
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    double* qv = (double*)malloc((size_t)G * sh->sel_dim * sizeof(double));
+    int rc = qv ? 0 : -2;
+    for (int b = 0; b < sh->batch && rc == 0; ++b)
+        for (int g = 0; g < sh->num_kv_heads && rc == 0; ++g) {
+            rc = unit_queries(sh, pr, b, g, q_sel, qv);
+            if (rc == 0)
+                unit_scores(sh, pr, b, g, qv, w, keys, page_table, seq_lens[b] / sh->block_size,
+                            scores + ((int64_t)b * sh->num_kv_heads + g) * sh->max_blocks);
+        }
+    free(qv);
     free(keys);
-    return 0;
+    return rc;
 }
 
 /* Ranking of residual blocks: score descending, lower block index first. */
@@ -532,6 +567,7 @@ int oracle_decode_step(const orc_shape_t* sh, const orc_params_t* pr, const uint
         return -1;
     }
     int total = units ? n_units : sh->batch * sh->num_kv_heads;
+    int err = 0;
 #ifdef _OPENMP
 #pragma omp parallel for schedule(dynamic, 1)
 #endif
@@ -541,7 +577,18 @@ int oracle_decode_step(const orc_shape_t* sh, const orc_params_t* pr, const uint
         int32_t L = seq_lens[b];
         int64_t nb = ceil_div64(L, sh->block_size), n_full = L / sh->block_size;
         double* s = (double*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(double));
-        unit_scores(sh, pr, b, g, q_sel, w, keys, page_table, n_full, s);
+        double* qv = (double*)malloc((size_t)G * sh->sel_dim * sizeof(double));
+        if (!s || !qv || unit_queries(sh, pr, b, g, q_sel, qv) != 0) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = -2;
+            free(s);
+            free(qv);
+            continue;
+        }
+        unit_scores(sh, pr, b, g, qv, w, keys, page_table, n_full, s);
+        free(qv);
         int32_t* sel = sel_idx + (int64_t)u * sh->max_blocks;
         double mass = 0.0;
         int32_t cnt = oracle_select_from_scores(s, (int32_t)nb, (int32_t)n_full, pr,
@@ -554,7 +601,7 @@ int oracle_decode_step(const orc_shape_t* sh, const orc_params_t* pr, const uint
         free(s);
     }
     free(keys);
-    return 0;
+    return err;
 }
 
 /* Threads the OpenMP runtime will use (1 without OpenMP). */

@@ -61,14 +61,15 @@ def host_bytes(t):
 
 
 def run_gpu(wl, fmt="bf16", mode="topp", kmin=None, topk=0, sink=None, rec=None,
-            temperature=1.0, pool=None, max_blocks=None):
+            temperature=1.0, pool=None, max_blocks=None, quantize_queries=False):
     dev = wl.q.device
     B, Hq, Hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
     mb = wl.max_blocks if max_blocks is None else max_blocks
     desc = spot.layer_desc(Hq, Hkv, wl.num_pages, fmt)
     prm = spot.select_params(mode, wl.spec.sink_blocks if sink is None else sink,
                              wl.spec.recency_blocks if rec is None else rec,
-                             wl.spec.kmin_blocks if kmin is None else kmin, topk, temperature)
+                             wl.spec.kmin_blocks if kmin is None else kmin, topk, temperature,
+                             quantize_queries)
     data, scales = pool if pool is not None else gpu_selector_pool(wl, fmt, dev)
     ws = spot.new_workspace(desc, B, mb, dev)
     sel_idx = torch.full((B, Hkv, mb), -1, dtype=torch.int32, device=dev)
@@ -95,12 +96,13 @@ def oracle_args(wl, fmt="bf16"):
 
 
 def oracle_shape_params(wl, fmt="bf16", mode="topp", kmin=None, topk=0, sink=None, rec=None,
-                        temperature=1.0, max_blocks=None):
+                        temperature=1.0, max_blocks=None, quantize_queries=False):
     sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, fmt,
                            wl.num_pages, wl.max_blocks if max_blocks is None else max_blocks)
     pr = oracle.make_params(mode, wl.spec.sink_blocks if sink is None else sink,
                             wl.spec.recency_blocks if rec is None else rec,
-                            wl.spec.kmin_blocks if kmin is None else kmin, topk, temperature)
+                            wl.spec.kmin_blocks if kmin is None else kmin, topk, temperature,
+                            quantize_queries)
     return sh, pr
 
 

@@ -73,6 +73,33 @@ def test_integer_inputs_select_bit_exact(name, kw, fmt):
     check_outputs(gpu, ora, wl)
 
 
+@pytest.mark.parametrize("fmt", ["mxfp4", "fp8"])
+def test_integer_inputs_quantised_queries_select_bit_exact(fmt):
+    # Queries in {-3..3} are stored losslessly by MXFP4 (power-of-two group
+    # scales) and E4M3, so quantising them keeps every score exact on both
+    # sides and the selections must be identical.
+    wl = workloads.make("quant_128k", seed=12, device=DEV, integer=True, seq_len=8192, batch=4)
+    wl.top_p = safe_top_p(wl, fmt, quantize_queries=True)
+    gpu = run_gpu(wl, fmt, quantize_queries=True)
+    assert gpu["status"] == 0
+    ora = run_oracle(wl, fmt, quantize_queries=True)
+    _assert_same_selection(gpu, ora, wl)
+    check_outputs(gpu, ora, wl)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "fp8", "int8"])
+def test_quantised_queries_tiny(fmt):
+    wl = workloads.make("tiny_4k", seed=3, device=DEV, sel_fmt=fmt)
+    gpu = run_gpu(wl, fmt, quantize_queries=True)
+    assert gpu["status"] == 0
+    scores = oracle_scores(wl, fmt, quantize_queries=True)
+    assert not np.allclose(scores, oracle_scores(wl, fmt), equal_nan=True)
+    ora = run_oracle(wl, fmt, quantize_queries=True)
+    assert check_selection_near_cut(gpu, ora, scores, wl) <= 1
+    _, _, n = check_outputs(gpu, ora, wl)
+    assert n >= wl.batch * wl.num_kv_heads - 1
+
+
 def test_integer_inputs_topk_and_kmin_modes():
     wl = workloads.make("qwen3_4b_32k", seed=5, device=DEV, integer=True, seq_len=4096)
     for kw in (dict(mode="topk", topk=17), dict(mode="topk", topk=0), dict(kmin=40),
@@ -148,23 +175,28 @@ def test_sparse_decode_on_oracle_selection():
 # ------------------------------------------------------------ full size
 
 FULL = [
-    ("qwen3_4b_32k", "bf16", None),
-    ("qwen3_32b_128k", "bf16", [0, 3]),
-    ("quant_128k", "int4", [1, 14]),
-    ("quant_128k", "mxfp4", [0, 9]),
-    ("quant_128k", "fp8", [3, 12]),
-    ("quant_128k", "int8", [2, 11]),
-    ("ragged_hybrid", "mxfp4", [0, 7, 31]),
+    ("qwen3_4b_32k", "bf16", None, False),
+    ("qwen3_32b_128k", "bf16", [0, 3], False),
+    ("quant_128k", "int4", [1, 14], False),
+    ("quant_128k", "mxfp4", [0, 9], False),
+    ("quant_128k", "fp8", [3, 12], False),
+    ("quant_128k", "int8", [2, 11], False),
+    ("quant_128k", "int4", [4], True),
+    ("quant_128k", "mxfp4", [6], True),
+    ("quant_128k", "fp8", [8], True),
+    ("quant_128k", "int8", [10], True),
+    ("ragged_hybrid", "mxfp4", [0, 7, 31], False),
 ]
 
 
-@pytest.mark.parametrize("name,fmt,sample", FULL)
-def test_full_size_config(name, fmt, sample):
+@pytest.mark.parametrize("name,fmt,sample,qq", FULL)
+def test_full_size_config(name, fmt, sample, qq):
     """Full-size workload in the benchmark's launch configuration: selection
     of every (sequence, KV head) checked against the oracle's scores; the
-    attention output of the sampled sequences against the oracle."""
+    attention output of the sampled sequences against the oracle.  qq: the
+    selector queries are quantised like the keys."""
     wl = workloads.make(name, seed=1, device=DEV, sel_fmt=fmt)
-    gpu = run_gpu(wl, fmt)
+    gpu = run_gpu(wl, fmt, quantize_queries=qq)
     assert gpu["status"] == 0
     pool = gpu.pop("pool")
     del pool
@@ -173,7 +205,7 @@ def test_full_size_config(name, fmt, sample):
                                wl.num_pages, wl.max_blocks), None
     o_data, o_scales = oracle_selector_pool(wl, fmt)
     pr = oracle.make_params(sink_blocks=wl.spec.sink_blocks, recency_blocks=wl.spec.recency_blocks,
-                            kmin_blocks=wl.spec.kmin_blocks)
+                            kmin_blocks=wl.spec.kmin_blocks, quantize_queries=qq)
     scores = oracle.block_scores(sh, pr, workloads.bits(wl.q_sel), None, o_data, o_scales,
                                  wl.page_table.cpu().numpy(), wl.seq_lens.cpu().numpy())
     lens = wl.seq_lens.cpu().numpy()
@@ -194,7 +226,7 @@ def test_full_size_config(name, fmt, sample):
     # attention, sampled sequences
     seqs = list(range(wl.batch)) if sample is None else sample
     sub = workloads.gather_units(wl, seqs)
-    ora = run_oracle(sub, fmt)
+    ora = run_oracle(sub, fmt, quantize_queries=qq)
     g_sub = {k: gpu[k][seqs] for k in ("sel_idx", "sel_cnt", "out", "lse")}
     _assert_same_selection_or_near(g_sub, ora, sub)
     _, _, n = check_outputs(g_sub, ora, sub)

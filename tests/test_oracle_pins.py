@@ -338,6 +338,93 @@ def test_int8_known_codes_and_scale():
     assert np.array_equal(oracle.dequant_selector("int8", d2, s2, 64), on_grid)
 
 
+# ------------------------------------------------ quantised selector queries
+# SpotAttention §5.3 / App. G Tab. 9 quantise the selector's queries along
+# with its key cache; a query row goes through the key format's quantiser.
+
+# One hand-worked case per format: (query elements {index: value}, key row
+# as codes + scales, score with quantised queries, score with bf16 queries).
+_QQ_CASES = {
+    # E4M3 at [1, 2) has step 1/8: 1.0625 is a tie -> 1.0 (even mantissa);
+    # at [2, 4) step 1/4: 3.375 is a tie -> 3.5.  Key = (1, 2).
+    "fp8": ({0: 1.0625, 1: 3.375},
+            (np.array([0x38, 0x40] + [0] * 62, np.uint8), None), 8.0, 7.8125),
+    # group 0 amax 7 -> scale 1: codes 7, 4 (3.5 ties to even), -1;
+    # group 1 amax 14 -> scale 2: code 7.  Key = 1 at dims 0, 1, 2, 32.
+    "int4": ({0: 7.0, 1: 3.5, 2: -1.2, 32: 14.0},
+             (np.array([0x11, 0x01] + [0] * 14 + [0x01] + [0] * 15, np.uint8),
+              np.array([0x3C00, 0x3C00], np.uint16)), 24.0, 7 + 3.5 - 1.203125 + 14),
+    # amax 127 -> scale 1: codes 127, 2 (2.5 ties to even), -4 (-3.5 ties to
+    # even), 0.  Key = 1 at dims 0-3.
+    "int8": ({0: 127.0, 1: 2.5, 2: -3.5, 3: 0.4},
+             (np.array([1, 1, 1, 1] + [0] * 60, np.int8), np.array([0x3C00], np.uint16)),
+             125.0, 127 + 2.5 - 3.5 + 0.400390625),
+    # group 0 amax 6 -> X = 2 - 2 = 0: 6 -> 6, 2.5 -> 2 (tie between codes 4
+    # and 5, even code), 0.2 -> 0.  Key = 1.0 (code 2, E8M0 127) at dims 0-2.
+    "mxfp4": ({0: 6.0, 1: 2.5, 2: 0.2},
+              (np.array([0x22, 0x02] + [0] * 30, np.uint8), np.array([127, 127], np.uint8)),
+              8.0, 6 + 2.5 + 0.2001953125),
+}
+
+
+@pytest.mark.parametrize("fmt", sorted(_QQ_CASES))
+def test_quantised_query_scores_hand_worked(fmt):
+    qvals, (data, scales), want_q, want_plain = _QQ_CASES[fmt]
+    q = np.zeros((1, 1, 64), np.float32)
+    for i, v in qvals.items():
+        q[0, 0, i] = v
+    sh = _one_seq_shape(1, 1, 1, 1, fmt)
+    args = (_bf16_bits(q), None, data, scales, np.array([[0]], np.int32),
+            np.array([64], np.int32))
+    s_q = oracle.block_scores(sh, oracle.make_params(quantize_queries=True), *args)
+    s_p = oracle.block_scores(sh, oracle.make_params(), *args)
+    assert s_q[0, 0, 0] == want_q
+    assert s_p[0, 0, 0] == want_plain
+
+
+def test_quantised_queries_have_no_effect_on_bf16_keys():
+    rng = np.random.default_rng(7)
+    sh = oracle.make_shape(2, 8, 2, 128, 64, 64, "bf16", 6, 3)
+    q = _bf16_bits(rng.normal(size=(2, 8, 64)))
+    keys = _bf16_bits(rng.normal(size=(6, 2, 64)))
+    pt = np.array([[0, 1, 2], [3, 4, 5]], np.int32)
+    lens = np.array([192, 150], np.int32)
+    a = oracle.block_scores(sh, oracle.make_params(quantize_queries=True), q, None, keys, None,
+                            pt, lens)
+    b = oracle.block_scores(sh, oracle.make_params(), q, None, keys, None, pt, lens)
+    assert np.array_equal(a, b, equal_nan=True)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "fp8", "int8"])
+def test_quantised_queries_follow_the_key_quantiser(fmt):
+    # Every query head's row is quantised on its own, with the pinned key
+    # quantiser, and read back exactly; the score is then the plain weighted
+    # ReLU sum (numpy matmul here).
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, P, MB = 2, 8, 2, 8, 4
+    q = _bf16_bits(rng.normal(size=(B, Hq, 64)) * 10.0 ** rng.uniform(-2, 2, size=(B, Hq, 1)))
+    kb = _bf16_bits(rng.normal(size=(P, Hkv, 64)))
+    kdata, kscales = oracle.quantize_selector(fmt, kb)
+    w = rng.uniform(0.1, 1.0, size=(B, Hq)).astype(np.float32)
+    pt = rng.permutation(P).astype(np.int32).reshape(B, MB)
+    lens = np.array([256, 200], np.int32)
+    sh = oracle.make_shape(B, Hq, Hkv, 128, 64, 64, fmt, P, MB)
+    got = oracle.block_scores(sh, oracle.make_params(quantize_queries=True), q, w, kdata, kscales,
+                              pt, lens)
+    qd_, qs_ = oracle.quantize_selector(fmt, q)
+    qd = oracle.dequant_selector(fmt, qd_, qs_, 64).reshape(B, Hq, 64)
+    kd = oracle.dequant_selector(fmt, kdata, kscales, 64).reshape(P, Hkv, 64)
+    G = Hq // Hkv
+    for b in range(B):
+        for g in range(Hkv):
+            for j in range(lens[b] // 64):
+                dots = qd[b, g * G:(g + 1) * G] @ kd[pt[b, j], g]
+                want = float((w[b, g * G:(g + 1) * G] * np.maximum(dots, 0.0)).sum())
+                assert abs(got[b, g, j] - want) <= 1e-12 * max(1.0, abs(want)), (b, g, j)
+    plain = oracle.block_scores(sh, oracle.make_params(), q, w, kdata, kscales, pt, lens)
+    assert not np.allclose(got, plain, equal_nan=True)       # the queries really changed
+
+
 # ---------------------------------------------------------------- attention
 
 def _rand_kv(rng, num_pages, Hkv, Hq, B=1):
