@@ -61,6 +61,12 @@ class Params(ctypes.Structure):
                 ("quantize_queries", ctypes.c_int32)]
 
 
+class TokShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "num_q_heads", "num_kv_heads", "head_dim", "page_size", "idx_heads", "idx_dim",
+        "sel_block", "num_pages", "max_pages", "max_blocks")]
+
+
 def _load():
     global _lib
     if _lib is None:
@@ -75,6 +81,9 @@ def _load():
         lib.oracle_sparse_attention.argtypes = [P, P, P, P, P, P, P, P, dbl, P, P]
         lib.oracle_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
                                            P, P, P, P, P]
+        lib.oracle_tok_block_scores.argtypes = [P, P, P, P, P, P, P, P]
+        lib.oracle_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
+                                               P, P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -206,6 +215,52 @@ def decode_step(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, q,
         _ptr(_c(k_pool, np.uint16)), _ptr(_c(v_pool, np.uint16)), _ptr(_c(page_table, np.int32)),
         _ptr(_c(seq_lens, np.int32)), _ptr(_c(top_p, np.float32)), float(sm_scale), _ptr(u),
         0 if u is None else len(u), _ptr(sel_idx), _ptr(sel_cnt), _ptr(mass), _ptr(out),
+        _ptr(lse))
+    assert rc == 0
+    return {"sel_idx": sel_idx, "sel_cnt": sel_cnt, "nuc_mass": mass, "out": out, "lse": lse}
+
+
+# ---------------------------------------------------------------------------
+# Token-level, layer-shared selector (§2.1 / §2.3 / App. A Tab. 3 as written)
+
+def make_tok_shape(batch, num_q_heads, num_kv_heads, num_pages, max_pages, head_dim=128,
+                   page_size=64, idx_heads=4, idx_dim=128, sel_block=16,
+                   max_blocks=None) -> TokShape:
+    mb = max_pages * (page_size // sel_block) if max_blocks is None else max_blocks
+    return TokShape(batch, num_q_heads, num_kv_heads, head_dim, page_size, idx_heads, idx_dim,
+                    sel_block, num_pages, max_pages, mb)
+
+
+def tok_block_scores(shape: TokShape, params: Params, q_idx, w, sel_tok, page_table,
+                     seq_lens) -> np.ndarray:
+    """Block scores [B, max_blocks] of the token-level selector (max over
+    each block's token scores; NaN where no complete block)."""
+    scores = np.full((shape.batch, shape.max_blocks), np.nan)
+    rc = _load().oracle_tok_block_scores(
+        ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_idx, np.uint16)),
+        _ptr(_c(w, np.float32)), _ptr(_c(sel_tok, np.uint16)), _ptr(_c(page_table, np.int32)),
+        _ptr(_c(seq_lens, np.int32)), _ptr(scores))
+    assert rc == 0
+    return scores
+
+
+def tok_decode_step(shape: TokShape, params: Params, q_idx, w, sel_tok, q, k_pool, v_pool,
+                    page_table, seq_lens, top_p, sm_scale, seqs=None):
+    """Decode step of the token-level selector for sequences `seqs` (default
+    all): one selection per sequence shared by every head."""
+    B, Hq = shape.batch, shape.num_q_heads
+    sel_idx = np.full((B, max(shape.max_blocks, 1)), -1, np.int32)
+    sel_cnt = np.zeros(B, np.int32)
+    mass = np.zeros(B)
+    out = np.zeros((B, Hq, shape.head_dim))
+    lse = np.zeros((B, Hq))
+    sq = None if seqs is None else _c(seqs, np.int32)
+    rc = _load().oracle_tok_decode_step(
+        ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_idx, np.uint16)),
+        _ptr(_c(w, np.float32)), _ptr(_c(sel_tok, np.uint16)), _ptr(_c(q, np.uint16)),
+        _ptr(_c(k_pool, np.uint16)), _ptr(_c(v_pool, np.uint16)), _ptr(_c(page_table, np.int32)),
+        _ptr(_c(seq_lens, np.int32)), _ptr(_c(top_p, np.float32)), float(sm_scale), _ptr(sq),
+        0 if sq is None else len(sq), _ptr(sel_idx), _ptr(sel_cnt), _ptr(mass), _ptr(out),
         _ptr(lse))
     assert rc == 0
     return {"sel_idx": sel_idx, "sel_cnt": sel_cnt, "nuc_mass": mass, "out": out, "lse": lse}

@@ -13,7 +13,7 @@
  * in the order the definitions state; the only library primitives are exp(),
  * log(), frexp()/ldexp() and qsort().
  *
- * Readings taken where the paper is silent (each also listed in the design doc):
+ * Readings taken where the paper is silent:
  *  - one selector key per (block, KV head); the index heads of a KV head are
  *    the G query heads of its GQA group, mixing weight w[b,h] (NULL -> 1/G);
  *  - the score of a block is s = (1/tau) * sum_h w_h * ReLU(q_h . k);
@@ -476,30 +476,32 @@ int oracle_select_from_scores(const double* scores, int32_t nb, int32_t n_full,
 
 /* Exact softmax attention of the G query heads of KV head g over the tokens
  * of the selected blocks (SpotAttention §2.3: the layer attends only to keys
- * in the selected blocks; §3: decode only).  Token t of logical block j sits
- * in pool page page_table[b][j], row t - j*bs.  Positions >= seq_len are not
- * attended.  out[h][D] and lse[h] (natural log of the softmax denominator,
- * -inf when no token is attended, out = 0 then). */
-static void unit_attention(const orc_shape_t* sh, int b, int g, const uint16_t* q,
-                           const uint16_t* k_pool, const uint16_t* v_pool,
-                           const int32_t* page_table, int32_t seq_len, const int32_t* sel,
-                           int32_t cnt, double sm_scale, double* out, double* lse) {
-    int G = sh->num_q_heads / sh->num_kv_heads;
-    int D = sh->head_dim, bs = sh->block_size;
-    int64_t ntok_max = (int64_t)cnt * bs;
+ * in the selected blocks; §3: decode only).  Selected block j covers
+ * positions [j*sb, (j+1)*sb); position t sits in pool page
+ * page_table[b][t / ps] (row stride pt_stride), row t % ps of that page
+ * (pool layout [pages][Hkv][ps][D]).  Positions >= seq_len are not attended.
+ * out[h][D] and lse[h] (natural log of the softmax denominator, -inf when no
+ * token is attended, out = 0 then). */
+static void attend_blocks(int Hq, int Hkv, int D, int ps, int64_t pt_stride, int sb, int b,
+                          int g, const uint16_t* q, const uint16_t* k_pool,
+                          const uint16_t* v_pool, const int32_t* page_table, int32_t seq_len,
+                          const int32_t* sel, int32_t cnt, double sm_scale, double* out,
+                          double* lse) {
+    int G = Hq / Hkv;
+    int64_t ntok_max = (int64_t)cnt * sb;
     double* logit = (double*)malloc((size_t)(ntok_max > 0 ? ntok_max : 1) * sizeof(double));
     int64_t* row = (int64_t*)malloc((size_t)(ntok_max > 0 ? ntok_max : 1) * sizeof(int64_t));
     for (int i = 0; i < G; ++i) {
         int h = g * G + i;
-        const uint16_t* qh = q + ((int64_t)b * sh->num_q_heads + h) * D;
+        const uint16_t* qh = q + ((int64_t)b * Hq + h) * D;
         int64_t n = 0;
         for (int32_t c = 0; c < cnt; ++c) {
             int32_t j = sel[c];
-            int32_t page = page_table[(int64_t)b * sh->max_blocks + j];
-            for (int t = 0; t < bs; ++t) {
-                int64_t pos = (int64_t)j * bs + t;
+            for (int t = 0; t < sb; ++t) {
+                int64_t pos = (int64_t)j * sb + t;
                 if (pos >= seq_len) break;
-                int64_t r = (((int64_t)page * sh->num_kv_heads + g) * bs + t) * D;
+                int32_t page = page_table[(int64_t)b * pt_stride + pos / ps];
+                int64_t r = (((int64_t)page * Hkv + g) * ps + pos % ps) * D;
                 double dot = 0.0;
                 for (int d = 0; d < D; ++d) dot += bf16_to_f64(qh[d]) * bf16_to_f64(k_pool[r + d]);
                 logit[n] = sm_scale * dot;
@@ -522,6 +524,17 @@ static void unit_attention(const orc_shape_t* sh, int b, int g, const uint16_t* 
     }
     free(logit);
     free(row);
+}
+
+/* The per-(block, KV head) selector's attention: selection blocks are the
+ * pool pages (sb = ps = block_size), page table row stride max_blocks. */
+static void unit_attention(const orc_shape_t* sh, int b, int g, const uint16_t* q,
+                           const uint16_t* k_pool, const uint16_t* v_pool,
+                           const int32_t* page_table, int32_t seq_len, const int32_t* sel,
+                           int32_t cnt, double sm_scale, double* out, double* lse) {
+    attend_blocks(sh->num_q_heads, sh->num_kv_heads, sh->head_dim, sh->block_size,
+                  sh->max_blocks, sh->block_size, b, g, q, k_pool, v_pool, page_table, seq_len,
+                  sel, cnt, sm_scale, out, lse);
 }
 
 /* Attention over given selections, for every (b, g):
@@ -601,6 +614,123 @@ int oracle_decode_step(const orc_shape_t* sh, const orc_params_t* pr, const uint
         free(s);
     }
     free(keys);
+    return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* Token-level, layer-shared selector (SpotAttention §2.1, §2.3 and    */
+/* App. A Tab. 3 as written).                                          */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t batch, num_q_heads, num_kv_heads, head_dim;
+    int32_t page_size;       /* tokens per pool page (KV and selector pools) */
+    int32_t idx_heads;       /* H_idx */
+    int32_t idx_dim;         /* d_idx */
+    int32_t sel_block;       /* tokens per selection block; divides page_size */
+    int32_t num_pages;
+    int32_t max_pages;       /* page-table row stride */
+    int32_t max_blocks;      /* selection row stride (sel_idx, scores) */
+} orc_tok_shape_t;
+
+/* Score of every complete selection block of sequence b (§2.1 and §2.3):
+ * the token score s[t] = (1/tau) sum_h w_h ReLU(q^I_h . k^I_{h,t}) with one
+ * key per index head and token, and the block score is the maximum of its
+ * tokens' scores.  Token t's keys sit in sel_tok[page][t % ps][h][d_idx]
+ * with page = page_table[b][t / ps].  w (NULL -> 1/H_idx) is [B][H_idx].
+ * Writes n_full = floor(seq_len / sel_block) scores into out. */
+static void tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, int b,
+                            const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
+                            const int32_t* page_table, int32_t seq_len, double* out) {
+    int Hi = sh->idx_heads, di = sh->idx_dim, sb = sh->sel_block, ps = sh->page_size;
+    int64_t n_full = seq_len / sb;
+    for (int64_t j = 0; j < n_full; ++j) {
+        double best = -INFINITY;
+        for (int64_t t = j * sb; t < (j + 1) * sb; ++t) {
+            int32_t page = page_table[(int64_t)b * sh->max_pages + t / ps];
+            double s = 0.0;
+            for (int h = 0; h < Hi; ++h) {
+                const uint16_t* q = q_idx + ((int64_t)b * Hi + h) * di;
+                const uint16_t* k = sel_tok + (((int64_t)page * ps + t % ps) * Hi + h) * di;
+                double dot = 0.0;
+                for (int d = 0; d < di; ++d) dot += bf16_to_f64(q[d]) * bf16_to_f64(k[d]);
+                double wh = w ? (double)w[(int64_t)b * Hi + h] : 1.0 / Hi;
+                s += wh * (dot > 0.0 ? dot : 0.0);
+            }
+            s /= pr->temperature;
+            if (s > best) best = s;
+        }
+        out[j] = best;
+    }
+}
+
+/* Block scores [B][max_blocks] of the token-level selector; entries past
+ * each sequence's complete blocks are left untouched. */
+int oracle_tok_block_scores(const orc_tok_shape_t* sh, const orc_params_t* pr,
+                            const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
+                            const int32_t* page_table, const int32_t* seq_lens, double* scores) {
+    if (sh->sel_block <= 0 || sh->page_size % sh->sel_block != 0) return -1;
+    for (int b = 0; b < sh->batch; ++b)
+        tok_unit_scores(sh, pr, b, q_idx, w, sel_tok, page_table, seq_lens[b],
+                        scores + (int64_t)b * sh->max_blocks);
+    return 0;
+}
+
+/* The decode step of the token-level selector for sequences seqs[n_seqs]
+ * (NULL: all): block scores, one selection per sequence shared by every
+ * head (§2.3, Eq. 6-8, blocks of sel_block tokens), and exact attention of
+ * every query head over the selected blocks' tokens.  Outputs indexed as
+ * in the full problem: sel_idx[b][max_blocks], sel_cnt[b], nuc_mass[b] (may
+ * be NULL), out[b][h][D], lse[b][h]. */
+int oracle_tok_decode_step(const orc_tok_shape_t* sh, const orc_params_t* pr,
+                           const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
+                           const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                           const int32_t* page_table, const int32_t* seq_lens,
+                           const float* top_p, double sm_scale, const int32_t* seqs,
+                           int32_t n_seqs, int32_t* sel_idx, int32_t* sel_cnt, double* nuc_mass,
+                           double* out, double* lse) {
+    if (sh->sel_block <= 0 || sh->page_size % sh->sel_block != 0) return -1;
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    int total = seqs ? n_seqs : sh->batch;
+    int err = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int k = 0; k < total; ++k) {
+        int b = seqs ? seqs[k] : k;
+        int32_t L = seq_lens[b];
+        int64_t nb = ceil_div64(L, sh->sel_block), n_full = L / sh->sel_block;
+        double* s = (double*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(double));
+        if (!s) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = -2;
+            continue;
+        }
+        tok_unit_scores(sh, pr, b, q_idx, w, sel_tok, page_table, L, s);
+        int32_t* sel = sel_idx + (int64_t)b * sh->max_blocks;
+        double mass = 0.0;
+        int32_t cnt = oracle_select_from_scores(s, (int32_t)nb, (int32_t)n_full, pr,
+                                                (double)top_p[b], sel, &mass);
+        sel_cnt[b] = cnt;
+        if (nuc_mass) nuc_mass[b] = mass;
+        free(s);
+    }
+    /* attention of every (sequence, KV head) over the shared selection */
+    int units = total * sh->num_kv_heads;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int u = 0; u < units; ++u) {
+        int k = u / sh->num_kv_heads, g = u % sh->num_kv_heads;
+        int b = seqs ? seqs[k] : k;
+        attend_blocks(sh->num_q_heads, sh->num_kv_heads, sh->head_dim, sh->page_size,
+                      sh->max_pages, sh->sel_block, b, g, q, k_pool, v_pool, page_table,
+                      seq_lens[b], sel_idx + (int64_t)b * sh->max_blocks, sel_cnt[b], sm_scale,
+                      out + ((int64_t)b * sh->num_q_heads + g * G) * sh->head_dim,
+                      lse + (int64_t)b * sh->num_q_heads + g * G);
+    }
     return err;
 }
 

@@ -537,3 +537,133 @@ def test_decode_step_composes_and_is_page_order_invariant():
     r2 = oracle.decode_step(sh, pr, **args2)
     assert np.array_equal(r2["sel_cnt"], r["sel_cnt"])
     assert np.allclose(r2["out"], r["out"], atol=1e-13, rtol=0)
+
+
+# ------------------------------------------- token-level, layer-shared selector
+# §2.1 / §2.3 / App. A Tab. 3 as written: per-token keys for each index head,
+# a block's score is the maximum of its tokens' scores, one selection per
+# sequence shared by every head, blocks of 16 tokens inside 64-token pages.
+
+def _tok_shape(B, Hq, Hkv, num_pages, max_pages, idx_heads=2):
+    return oracle.make_tok_shape(B, Hq, Hkv, num_pages, max_pages, idx_heads=idx_heads)
+
+
+def test_tok_scores_hand_computed():
+    q = np.zeros((1, 2, 128), np.float32)
+    q[0, 0, 0] = 1.0                         # head 0: e0
+    q[0, 1, 1] = 2.0                         # head 1: 2 e1
+    keys = np.zeros((1, 64, 2, 128), np.float32)
+    keys[0, 3, 0, 0], keys[0, 3, 1, 1] = 5.0, -1.0     # token 3: dots 5, -2
+    keys[0, 7, 0, 0], keys[0, 7, 1, 1] = 1.0, 1.5      # token 7: dots 1, 3
+    keys[0, 20, 0, 0], keys[0, 20, 1, 1] = -3.0, 2.0   # token 20: dots -3, 4
+    sh = _tok_shape(1, 4, 2, 1, 1)
+    args = (_bf16_bits(q), None, _bf16_bits(keys), np.array([[0]], np.int32),
+            np.array([40], np.int32))
+    w = np.array([[0.5, 0.25]], np.float32)
+    s = oracle.tok_block_scores(sh, oracle.make_params(), args[0], w, *args[2:])
+    # block 0: max(0.5*5, 0.5*1 + 0.25*3) = 2.5 (the max, not the sum 3.75);
+    # block 1: 0.25*4 = 1; block 2 (tokens 32..39) is incomplete: no score
+    assert s[0, :2].tolist() == [2.5, 1.0]
+    assert np.isnan(s[0, 2:]).all()
+    s = oracle.tok_block_scores(sh, oracle.make_params(), *args)           # w = 1/H_idx
+    assert s[0, :2].tolist() == [2.5, 2.0]
+    s = oracle.tok_block_scores(sh, oracle.make_params(temperature=2.0), *args)
+    assert s[0, :2].tolist() == [1.25, 1.0]
+
+
+def test_tok_page_indirection_and_invariance():
+    rng = np.random.default_rng(3)
+    q = _bf16_bits(rng.normal(size=(1, 2, 128)))
+    keys = rng.normal(size=(3, 64, 2, 128)).astype(np.float32) * 0.1
+    keys[2, 17, 0] = 10.0 * np.asarray(q[0, 0].view(np.uint16).astype(np.uint32) << 16,
+                                       np.uint32).view(np.float32)    # a hot token
+    sh = _tok_shape(1, 4, 2, 3, 3)
+    pt = np.array([[1, 2, 0]], np.int32)     # logical page 1 -> physical page 2
+    lens = np.array([192], np.int32)
+    s = oracle.tok_block_scores(sh, oracle.make_params(), q, None, _bf16_bits(keys), pt, lens)
+    assert int(np.argmax(s[0, :12])) == 4 + 17 // 16          # logical block 5
+    perm = np.array([2, 0, 1])               # physical page i moves to perm[i]
+    moved = np.empty_like(keys)
+    moved[perm] = keys
+    s2 = oracle.tok_block_scores(sh, oracle.make_params(), q, None, _bf16_bits(moved),
+                                 perm[pt].astype(np.int32), lens)
+    assert np.array_equal(s, s2, equal_nan=True)
+
+
+def _tok_problem(rng, B=1, Hq=4, Hkv=2, L=160, idx_heads=2):
+    npg = (L + 63) // 64
+    q_idx = _bf16_bits(rng.normal(size=(B, idx_heads, 128)) * 0.3)
+    sel_tok = _bf16_bits(rng.normal(size=(B * npg, 64, idx_heads, 128)))
+    (q, k, v), (q64, k64, v64) = _rand_kv(rng, B * npg, Hkv, Hq, B)
+    pt = rng.permutation(B * npg).astype(np.int32).reshape(B, npg)
+    sh = _tok_shape(B, Hq, Hkv, B * npg, npg, idx_heads)
+    return sh, q_idx, sel_tok, (q, k, v), (q64, k64, v64), pt
+
+
+def _tok_tokens(k64, v64, pt, b, g, positions):
+    rows_k = torch.stack([k64[pt[b, t // 64], g, t % 64] for t in positions])
+    rows_v = torch.stack([v64[pt[b, t // 64], g, t % 64] for t in positions])
+    return rows_k, rows_v
+
+
+def test_tok_all_blocks_is_dense_attention_for_every_head():
+    rng = np.random.default_rng(8)
+    L = 150
+    sh, q_idx, sel_tok, (q, k, v), (q64, k64, v64), pt = _tok_problem(rng, L=L)
+    pr = oracle.make_params(sink_blocks=1, recency_blocks=1, kmin_blocks=0)
+    r = oracle.tok_decode_step(sh, pr, q_idx, None, sel_tok, _bf16_bits(q), _bf16_bits(k),
+                               _bf16_bits(v), pt, np.array([L], np.int32),
+                               np.array([1.0], np.float32), 1 / math.sqrt(128))
+    nb = (L + 15) // 16
+    assert r["sel_idx"][0, :r["sel_cnt"][0]].tolist() == list(range(nb))
+    G = 2
+    for h in range(4):
+        kk, vv = _tok_tokens(k64, v64, pt, 0, h // G, range(L))
+        ref = _sdpa(q64[0, h], kk, vv, 1 / math.sqrt(128))
+        assert np.allclose(r["out"][0, h], ref.numpy(), atol=1e-12, rtol=1e-10)
+
+
+def test_tok_topk_selection_feeds_attention_of_every_head():
+    # Static top-K with no reserved blocks keeps exactly the planted blocks;
+    # every head then attends exactly their tokens (16-token granularity
+    # inside 64-token pages).
+    rng = np.random.default_rng(9)
+    L = 256
+    sh, q_idx, sel_tok, (q, k, v), (q64, k64, v64), pt = _tok_problem(rng, L=L)
+    tok = sel_tok.copy()
+    hot = [2, 5, 13]
+    qv = torch.as_tensor(q_idx.view(np.int16)).view(torch.bfloat16).double().numpy()[0]
+    keys = torch.as_tensor(tok.view(np.int16)).view(torch.bfloat16).float().numpy()
+    for j in hot:
+        for t in range(16 * j, 16 * j + 16):
+            keys[pt[0, t // 64], t % 64] += 20.0 * qv / np.linalg.norm(qv, axis=1, keepdims=True)
+    tok = _bf16_bits(keys)
+    pr = oracle.make_params(mode="topk", sink_blocks=0, recency_blocks=0, topk_blocks=3)
+    r = oracle.tok_decode_step(sh, pr, q_idx, None, tok, _bf16_bits(q), _bf16_bits(k),
+                               _bf16_bits(v), pt, np.array([L], np.int32),
+                               np.array([0.9], np.float32), 0.1)
+    assert r["sel_idx"][0, :r["sel_cnt"][0]].tolist() == hot
+    pos = [t for j in hot for t in range(16 * j, 16 * j + 16)]
+    for h in range(4):
+        kk, vv = _tok_tokens(k64, v64, pt, 0, h // 2, pos)
+        ref = _sdpa(q64[0, h], kk, vv, 0.1)
+        assert np.allclose(r["out"][0, h], ref.numpy(), atol=1e-12, rtol=1e-10)
+
+
+def test_tok_reserved_blocks_and_incomplete_last_block():
+    rng = np.random.default_rng(10)
+    L = 16 * 10 + 5                           # 11 blocks, the last one incomplete
+    sh, q_idx, sel_tok, (q, k, v), _, pt = _tok_problem(rng, L=L)
+    pr = oracle.make_params(sink_blocks=2, recency_blocks=2, kmin_blocks=0)
+    r = oracle.tok_decode_step(sh, pr, q_idx, None, sel_tok, _bf16_bits(q), _bf16_bits(k),
+                               _bf16_bits(v), pt, np.array([L], np.int32),
+                               np.array([0.0], np.float32), 0.1)
+    # p = 0: empty nucleus; the incomplete block 10 joins the recency blocks
+    assert r["sel_idx"][0, :r["sel_cnt"][0]].tolist() == [0, 1, 9, 10]
+    pr = oracle.make_params(sink_blocks=2, recency_blocks=2, kmin_blocks=6)
+    r2 = oracle.tok_decode_step(sh, pr, q_idx, None, sel_tok, _bf16_bits(q), _bf16_bits(k),
+                                _bf16_bits(v), pt, np.array([L], np.int32),
+                                np.array([0.0], np.float32), 0.1)
+    s = oracle.tok_block_scores(sh, pr, q_idx, None, sel_tok, pt, np.array([L], np.int32))[0]
+    best = sorted(range(2, 9), key=lambda j: (-s[j], j))[:2]           # K_min floor of 6
+    assert r2["sel_idx"][0, :r2["sel_cnt"][0]].tolist() == sorted([0, 1, 9, 10] + best)

@@ -267,3 +267,180 @@ def gather_units(wl: Workload, seqs) -> Workload:
                     wl.v_pool[idx].contiguous(), wl.top_p[seqs].contiguous(),
                     [wl.hot_blocks[b * wl.num_kv_heads + g] for b in seqs
                      for g in range(wl.num_kv_heads)])
+
+
+# --------------------------------------------------------------------------
+# Token-level, layer-shared selector (SpotAttention §2.1 and App. A Tab. 3 as
+# written: H_idx = 4 index heads of width d_idx = 128 with per-token keys,
+# blocks of 16 tokens scored by their maximum token score, one selection per
+# query shared by every head of the layer).
+
+TOK_PAGE = 64          # tokens per KV / selector page (the paged-cache page)
+
+
+@dataclasses.dataclass
+class TokSpec:
+    name: str
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    seq_len: Optional[int]              # None -> ragged draw
+    idx_heads: int = 4
+    idx_dim: int = 128
+    sel_block: int = 16
+    top_p: float = 0.9
+    sink_blocks: int = 8                # 128 tokens (Tab. 3)
+    recency_blocks: int = 16            # 256 tokens
+    kmin_blocks: int = 32               # 512 tokens
+    q_scale: float = 0.3                # selector query scale: ~40% of blocks at p = 0.9, 128K
+    hot_count: int = 64                 # hot 16-token blocks per sequence
+    page_order: str = "permuted"
+    ragged_range: tuple = (8192, 131072)
+    layers_total: int = 1
+    layers_sparse: int = 1
+
+
+TOK_SPECS = {
+    "tok_tiny_2k": TokSpec("tok_tiny_2k", 1, 8, 2, 2048, hot_count=6, page_order="contiguous"),
+    "qwen3_8b_128k_tok": TokSpec("qwen3_8b_128k_tok", 1, 32, 8, 131072, layers_total=36,
+                                 layers_sparse=36),
+}
+
+
+@dataclasses.dataclass
+class TokWorkload:
+    spec: TokSpec
+    seed: int
+    seq_lens: torch.Tensor              # int32 [B]
+    page_table: torch.Tensor            # int32 [B, max_pages], -1 past each sequence
+    num_pages: int
+    q: torch.Tensor                     # bf16 [B, Hq, D]
+    q_idx: torch.Tensor                 # bf16 [B, H_idx, d_idx]
+    w_idx: Optional[torch.Tensor]       # fp32 [B, H_idx] or None (uniform 1/H_idx)
+    sel_tok: torch.Tensor               # bf16 [num_pages, TOK_PAGE, H_idx, d_idx]
+    k_pool: torch.Tensor                # bf16 [num_pages, Hkv, TOK_PAGE, D]
+    v_pool: torch.Tensor                # bf16 [num_pages, Hkv, TOK_PAGE, D]
+    top_p: torch.Tensor                 # fp32 [B]
+    hot_blocks: list                    # per b: logical ids of planted 16-token blocks
+
+    @property
+    def batch(self):
+        return self.spec.batch
+
+    @property
+    def num_q_heads(self):
+        return self.spec.num_q_heads
+
+    @property
+    def num_kv_heads(self):
+        return self.spec.num_kv_heads
+
+    @property
+    def max_pages(self):
+        return int(self.page_table.shape[1])
+
+    @property
+    def max_blocks(self):
+        return self.max_pages * (TOK_PAGE // self.spec.sel_block)
+
+    @property
+    def sm_scale(self):
+        return 1.0 / math.sqrt(HEAD_DIM)
+
+
+def make_tok(name: str, seed: int = 0, device="cpu", *, seq_len=None, batch=None,
+             integer: bool = False, top_p=None, uniform_w: bool = False,
+             **spec_overrides) -> TokWorkload:
+    """Seeded token-selector workload.  integer=True draws selector queries
+    and keys from {-3..3} and uses uniform weights (exact scores in any
+    precision)."""
+    spec = dataclasses.replace(TOK_SPECS[name], **spec_overrides)
+    if seq_len is not None:
+        spec = dataclasses.replace(spec, seq_len=seq_len)
+    if batch is not None:
+        spec = dataclasses.replace(spec, batch=batch)
+    if top_p is not None:
+        spec = dataclasses.replace(spec, top_p=top_p)
+    device = torch.device(device)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    B, Hq, Hkv, Hi, di = spec.batch, spec.num_q_heads, spec.num_kv_heads, spec.idx_heads, spec.idx_dim
+    if spec.seq_len is None:
+        lo, hi = spec.ragged_range
+        lens = rng.integers(lo // spec.sel_block, hi // spec.sel_block + 1, size=B) * spec.sel_block
+    else:
+        lens = np.full(B, spec.seq_len, np.int64)
+    npg = (lens + TOK_PAGE - 1) // TOK_PAGE
+    mp = int(max(npg.max() if B else 0, 1))
+    num_pages = int(max(npg.sum(), 1))
+    pages = np.arange(num_pages) if spec.page_order == "contiguous" else rng.permutation(num_pages)
+    pt = np.full((B, mp), -1, np.int32)
+    off = 0
+    for b in range(B):
+        pt[b, :npg[b]] = pages[off:off + npg[b]]
+        off += npg[b]
+    p = np.full(B, spec.top_p, np.float32)
+
+    q = _normal_bf16((B, Hq, HEAD_DIM), gen, device)
+    if integer:
+        q_idx = _int_bf16((B, Hi, di), gen, device)
+        sel_tok = _int_bf16((num_pages, TOK_PAGE, Hi, di), gen, device)
+        w_idx = None
+    else:
+        q_idx = (torch.randn((B, Hi, di), generator=gen, device=device) * spec.q_scale).to(
+            torch.bfloat16)
+        sel_tok = _normal_bf16((num_pages, TOK_PAGE, Hi, di), gen, device)
+        w_idx = None if uniform_w else torch.as_tensor(
+            rng.uniform(0.5, 1.5, size=(B, Hi)) / Hi, dtype=torch.float32, device=device)
+    k_pool = _normal_bf16((num_pages, Hkv, TOK_PAGE, HEAD_DIM), gen, device)
+    v_pool = _normal_bf16((num_pages, Hkv, TOK_PAGE, HEAD_DIM), gen, device)
+    wl = TokWorkload(spec, seed, torch.as_tensor(lens, dtype=torch.int32, device=device),
+                     torch.as_tensor(pt, device=device), num_pages, q, q_idx, w_idx, sel_tok,
+                     k_pool, v_pool, torch.as_tensor(p, device=device), [])
+    _plant_hot_tok(wl, rng, integer)
+    return wl
+
+
+def _plant_hot_tok(wl: TokWorkload, rng, integer: bool):
+    """Per sequence, some 16-token blocks (outside the sink / recency blocks)
+    get every token's selector key shifted along each index head's query
+    direction by o / |q_h| (o ~ U[2, 4]: each head's dot rises by o, so the
+    weighted token score rises by about o * sum_h w_h), and their backbone
+    keys shifted along each KV group's summed query direction (the group's
+    mean scaled logit rises by o).  Integer workloads set the hot tokens'
+    selector keys to 3 * sign(q_h) instead."""
+    spec = wl.spec
+    B, Hkv, sb = spec.batch, spec.num_kv_heads, spec.sel_block
+    G = spec.num_q_heads // Hkv
+    per_page = TOK_PAGE // sb
+    qk = wl.q.float().view(B, Hkv, G, HEAD_DIM).sum(2)
+    pt = wl.page_table.cpu().numpy()
+    lens = wl.seq_lens.cpu().numpy()
+    dev = wl.q.device
+    for b in range(B):
+        nb = int((lens[b] + sb - 1) // sb)
+        cand = np.arange(max(spec.sink_blocks, 0), max(nb - spec.recency_blocks, 0))
+        n_hot = min(spec.hot_count, cand.size)
+        hot = np.sort(rng.choice(cand, size=n_hot, replace=False)) if n_hot else cand[:0]
+        wl.hot_blocks.append(hot.tolist())
+        if n_hot == 0:
+            continue
+        o = torch.as_tensor(rng.uniform(2.0, 4.0, size=n_hot), dtype=torch.float32, device=dev)
+        pages = torch.as_tensor(pt[b, hot // per_page].astype(np.int64), device=dev)
+        slot0 = torch.as_tensor((hot % per_page) * sb, device=dev)
+        slots = slot0[:, None] + torch.arange(sb, device=dev)[None, :]        # [n_hot, sb]
+        pg = pages[:, None].expand(-1, sb)
+        qi = wl.q_idx[b].float()                                              # [Hi, di]
+        if integer:
+            new = (3.0 * torch.sign(qi))[None, None].expand(n_hot, sb, -1, -1)
+        else:
+            u = qi / qi.norm(dim=1, keepdim=True)
+            c = o[:, None] / qi.norm(dim=1)[None, :]                          # [n_hot, Hi]
+            new = wl.sel_tok[pg, slots].float() + c[:, None, :, None] * u[None, None]
+        wl.sel_tok[pg, slots] = new.to(torch.bfloat16)
+        for g in range(Hkv):
+            nkv = qk[b, g].norm()
+            ck = o * G * math.sqrt(HEAD_DIM) / nkv
+            kk = wl.k_pool[pg, g, slots].float() + ck[:, None, None] * (qk[b, g] / nkv)
+            wl.k_pool[pg, g, slots] = kk.to(torch.bfloat16)
