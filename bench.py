@@ -366,6 +366,218 @@ def run_spot(args, world, rank, local):
     return res, layers
 
 
+def tok_step_bytes(wl, sel_cnt: np.ndarray):
+    """Algorithmic HBM bytes of one token-selector decode step: the
+    per-token selector keys of every complete 16-token block, the K and V
+    rows of the selected tokens for every KV head, indices and queries."""
+    B, Hq, Hkv, sb = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.spec.sel_block
+    lens = wl.seq_lens.cpu().numpy().astype(np.int64)
+    n_full = lens // sb
+    sel_cache = int(n_full.sum()) * sb * wl.spec.idx_heads * wl.spec.idx_dim * 2
+    kv = int(sel_cnt.sum()) * sb * Hkv * 128 * 2 * 2
+    part = lens % sb != 0                     # the partial last block is always selected
+    kv -= int((Hkv * (sb - lens[part] % sb) * 128 * 2 * 2).sum())
+    idx = int(sel_cnt.sum()) * 4 * 2 * Hkv    # each KV head reads the list and the page id
+    q_io = B * Hq * (128 * 2 + 128 * 4 + 4)
+    select = (sel_cache + B * wl.spec.idx_heads * (wl.spec.idx_dim * 2 + 4) +
+              int(n_full.sum()) * 4 + int(sel_cnt.sum()) * 4)
+    sparse = kv + idx + q_io
+    return {"sparse": sparse, "select": select, "step": sparse + select, "kv": kv,
+            "selector": sel_cache}
+
+
+def run_spot_tok(args, world, rank, local):
+    """The token-level, layer-shared selector path (tok_select, then
+    tok_sparse_decode), timed like run_spot."""
+    import block_sparse_long_spot_b200 as spot
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    layers = []
+    for l in range(args.layers):
+        wl = workloads.make_tok(args.workload, seed=layer_seed(rank, l), device=dev)
+        layers.append((wl, spot.tok_layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages)))
+    wl0, desc0 = layers[0]
+    B, Hq, mb = wl0.batch, wl0.num_q_heads, wl0.max_blocks
+    sp = wl0.spec
+    prm = spot.select_params("topp", sp.sink_blocks, sp.recency_blocks, sp.kmin_blocks)
+    # one workspace per layer cache: the layers differ in their page counts
+    wss = [spot.new_tok_workspace(d, B, mb, dev) for _, d in layers]
+    sel_idx = torch.empty(B, mb, dtype=torch.int32, device=dev)
+    sel_cnt = torch.empty(B, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        wl, desc = layers[i % len(layers)]
+        ws = wss[i % len(layers)]
+        if ev is not None:
+            ev[0].record(stream)
+        spot.tok_select(desc, prm, wl.q_idx, wl.w_idx, wl.sel_tok, wl.page_table, wl.seq_lens,
+                        wl.top_p, sel_idx, sel_cnt, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        spot.tok_sparse_decode(desc, wl.q, wl.k_pool, wl.v_pool, wl.page_table, wl.seq_lens,
+                               sel_idx, sel_cnt, wl.sm_scale, out, lse, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    per_layer = []
+    for l in range(len(layers)):
+        step(l)
+        torch.cuda.synchronize()
+        cnt = sel_cnt.cpu().numpy().copy()
+        wl = layers[l][0]
+        nb = (wl.seq_lens.cpu().numpy() + sp.sel_block - 1) // sp.sel_block
+        per_layer.append((tok_step_bytes(wl, cnt), cnt / np.maximum(nb, 1)))
+    for ws in wss:
+        status = spot.read_device_status(ws)
+        if status != 0:
+            raise RuntimeError(f"device status {status} after warm-up")
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t0.record(stream)
+        for i in range(K):
+            step(i, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / K, world)
+    sel_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    dec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+
+    pin_q = [wl.q.cpu().pin_memory() for wl, _ in layers]
+    pin_qi = [wl.q_idx.cpu().pin_memory() for wl, _ in layers]
+    host_out = torch.empty(B, Hq, 128, dtype=torch.float32).pin_memory()
+    q_dev, qi_dev = torch.empty_like(wl0.q), torch.empty_like(wl0.q_idx)
+
+    def e2e_step(i):
+        wl, desc = layers[i % len(layers)]
+        q_dev.copy_(pin_q[i % len(layers)], non_blocking=True)
+        qi_dev.copy_(pin_qi[i % len(layers)], non_blocking=True)
+        spot.tok_decode_step(desc, prm, qi_dev, wl.w_idx, wl.sel_tok, q_dev, wl.k_pool,
+                             wl.v_pool, wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale,
+                             sel_idx, sel_cnt, out, lse, wss[i % len(layers)], stream)
+        host_out.copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K, world)
+    for ws in wss:
+        status = spot.read_device_status(ws)
+        if status != 0:
+            raise RuntimeError(f"device status {status} after timing")
+
+    nl = len(layers)
+    b_sparse = float(np.mean([per_layer[i % nl][0]["sparse"] for i in range(K)]))
+    b_select = float(np.mean([per_layer[i % nl][0]["select"] for i in range(K)]))
+    b_step = b_sparse + b_select
+    frac_sel = np.concatenate([x[1].ravel() for x in per_layer])
+    peak, peak_kind = peaks()
+    layers_model = sp.layers_sparse
+    value = shard_summary(B, world, ms_step, layers_model)
+    value_e2e = shard_summary(B, world, ms_e2e, layers_model)
+    dom_sparse = b_sparse >= b_select
+    kb, kms = (b_sparse, dec_ms) if dom_sparse else (b_select, sel_ms)
+    achieved = kb / (kms / 1e3) / 1e9
+    return {
+        "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
+        "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "us_per_layer": round(ms_step * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 with planted hot 16-token blocks)",
+        "config": {
+            "workload": args.workload, "selector": "token-level, layer-shared",
+            "batch_per_gpu": B, "q_heads": Hq, "kv_heads": wl0.num_kv_heads, "head_dim": 128,
+            "idx_heads": sp.idx_heads, "idx_dim": sp.idx_dim, "sel_block": sp.sel_block,
+            "context": int(wl0.seq_lens.max().item()), "sel_fmt": "bf16",
+            "top_p": float(wl0.top_p[0].item()), "sink_blocks": sp.sink_blocks,
+            "recency_blocks": sp.recency_blocks, "kmin_blocks": sp.kmin_blocks,
+            "layers_in_model": layers_model, "layer_caches_rotated": nl,
+            "l2": f"inputs larger than L2: {nl} layer caches of "
+                  f"{(wl0.k_pool.numel() * 4 + wl0.sel_tok.numel() * 2) / 1e9:.2f} GB rotated",
+            "selected_fraction": {"mean": round(float(frac_sel.mean()), 4),
+                                  "min": round(float(frac_sel.min()), 4),
+                                  "max": round(float(frac_sel.max()), 4)},
+            "parallelism": f"dp{world} (sequences)",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "sparse decode (attention + combine)" if dom_sparse else
+                      "token selector (scoring + selection)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_kind,
+            "algorithmic_bytes_per_launch": int(kb), "ms_per_launch": round(kms, 5),
+        },
+        "select_roofline": {
+            "achieved": round(b_select / (sel_ms / 1e3) / 1e9, 1), "peak": peak,
+            "frac": round(b_select / (sel_ms / 1e3) / 1e9 / peak, 4),
+            "algorithmic_bytes": int(b_select), "ms": round(sel_ms, 5)},
+        "sparse_roofline": {
+            "achieved": round(b_sparse / (dec_ms / 1e3) / 1e9, 1), "peak": peak,
+            "frac": round(b_sparse / (dec_ms / 1e3) / 1e9 / peak, 4),
+            "algorithmic_bytes": int(b_sparse), "ms": round(dec_ms, 5)},
+        "step_roofline": {
+            "achieved": round(b_step / (ms_step / 1e3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(b_step / (ms_step / 1e3) / 1e9 / peak, 4),
+            "algorithmic_bytes_per_step": int(b_step)},
+        "e2e": {"value": round(value_e2e, 3), "unit": "tokens/s",
+                "ms_per_step": round(ms_e2e, 5),
+                "h2d_bytes_per_step": int(wl0.q.numel() * 2 + wl0.q_idx.numel() * 2),
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": K * 3,          # token scoring, selection, sparse decode per step
+        "clocks": clk.summary(),
+    }, layers
+
+
+def cpu_baseline_tok(wl, min_s=10.0, max_s=30.0):
+    """The fp64 oracle's token-selector decode step on the host cores, one
+    sequence at a time, until about 10 s of work; scaled to the model."""
+    import oracle
+    sp = wl.spec
+    sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
+                               wl.max_pages)
+    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
+                            kmin_blocks=sp.kmin_blocks)
+    a = dict(q_idx=workloads.bits(wl.q_idx),
+             w=None if wl.w_idx is None else wl.w_idx.cpu().numpy(),
+             sel_tok=workloads.bits(wl.sel_tok), q=workloads.bits(wl.q),
+             k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
+             page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
+             top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
+    total, n = 0.0, 0
+    while total < min_s and n < 64:
+        t = time.perf_counter()
+        oracle.tok_decode_step(sh, pr, seqs=[n % wl.batch], **a)
+        total += time.perf_counter() - t
+        n += 1
+        if total > max_s:
+            break
+    per_seq = total / n
+    value = 1.0 / (per_seq * sp.layers_sparse)
+    return {"value": round(value, 6), "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 oracle token-selector decode step of one sequence (all heads), "
+                      f"{n} runs, {total:.1f} s; x{sp.layers_sparse} layers"}
+
+
 def prepare_oracle(wl, fmt, seqs):
     """Host copies of sequences `seqs` of a layer, ready for the fp64 oracle."""
     import oracle
@@ -451,6 +663,49 @@ def run_reference(args, world, rank):
     }
 
 
+def run_reference_tok(args, world, rank):
+    """Reference arm for the token-selector workloads: each step times the
+    fp64 oracle's decode step of one sequence (all heads) on the host cores."""
+    if rank != 0:
+        return None
+    import oracle
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = workloads.make_tok(args.workload, seed=0, device=dev)
+    times = []
+    sp = wl.spec
+    sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
+                               wl.max_pages)
+    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
+                            kmin_blocks=sp.kmin_blocks)
+    a = dict(q_idx=workloads.bits(wl.q_idx),
+             w=None if wl.w_idx is None else wl.w_idx.cpu().numpy(),
+             sel_tok=workloads.bits(wl.sel_tok), q=workloads.bits(wl.q),
+             k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
+             page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
+             top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        oracle.tok_decode_step(sh, pr, seqs=[i % wl.batch], **a)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    per_layer = float(np.mean(times)) * wl.batch
+    value = wl.batch / (per_layer * sp.layers_sparse)
+    sample = f"one sequence (all heads) per step; x{wl.batch} sequences x{sp.layers_sparse} layers"
+    return {
+        "impl": "reference",
+        "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
+        "value": round(value, 6), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_layer * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 with planted hot 16-token blocks)",
+        "config": {"workload": args.workload, "sel_fmt": "bf16", "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s",
+                         "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -462,22 +717,27 @@ def main():
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    tok = args.workload in workloads.TOK_SPECS
     if args.sel_fmt is None:
-        args.sel_fmt = workloads.SPECS[args.workload].sel_fmt
+        args.sel_fmt = "bf16" if tok else workloads.SPECS[args.workload].sel_fmt
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
             if world > 1:
                 torch.distributed.barrier()
-            res = run_reference(args, world, rank)
+            res = (run_reference_tok if tok else run_reference)(args, world, rank)
             if res is not None:
                 print(json.dumps(res), flush=True)
             return
-        res, layers = run_spot(args, world, rank, local)
+        if tok:
+            res, layers = run_spot_tok(args, world, rank, local)
+        else:
+            res, layers = run_spot(args, world, rank, local)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = cpu_baseline(layers[0][0], args.sel_fmt)
+                res["cpu_baseline"] = (cpu_baseline_tok(layers[0][0]) if tok else
+                                       cpu_baseline(layers[0][0], args.sel_fmt))
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

@@ -48,6 +48,18 @@ class SelectParams(ctypes.Structure):
                 ("quantize_queries", ctypes.c_int32)]
 
 
+class TokLayerDesc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_q_heads", "num_kv_heads", "head_dim", "page_size", "idx_heads", "idx_dim",
+        "sel_block", "num_pages")]
+
+
+def tok_layer_desc(num_q_heads, num_kv_heads, num_pages, head_dim=128, page_size=64,
+                   idx_heads=4, idx_dim=128, sel_block=16) -> TokLayerDesc:
+    return TokLayerDesc(num_q_heads, num_kv_heads, head_dim, page_size, idx_heads, idx_dim,
+                        sel_block, num_pages)
+
+
 def layer_desc(num_q_heads, num_kv_heads, num_pages, sel_fmt="bf16", head_dim=128,
                block_size=64, sel_dim=64) -> LayerDesc:
     return LayerDesc(num_q_heads, num_kv_heads, head_dim, block_size, sel_dim,
@@ -83,13 +95,22 @@ def lib():
                                        i32, P, P, P, sz, P]
         L.spot_sparse_decode_noalloc.argtypes = [P, P, P, P, P, i32, P, P, P, i32, i32, f32, P,
                                                  P, P]
+        L.spot_tok_workspace_size.argtypes = [P, i32, i32]
+        L.spot_tok_workspace_size.restype = sz
+        L.spot_tok_append_selector_keys.argtypes = [P, P, P, i32, i32, P, P, P, i32, P, P]
+        L.spot_tok_select.argtypes = [P, P, P, P, P, P, i32, P, P, i32, P, P, i32, P, sz, P]
+        L.spot_tok_sparse_decode.argtypes = [P, P, P, P, P, i32, P, P, P, i32, i32, f32, P, P,
+                                             P, sz, P]
+        L.spot_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, P, i32, f32, P, P,
+                                           i32, P, P, P, sz, P]
         L.spot_read_device_status.argtypes = [P, P]
         L.spot_check_wait_timeout.argtypes = [P, P]
         L.spot_check_wait_timeout.restype = ctypes.c_int
         L.spot_status_string.restype = ctypes.c_char_p
         for name in ("spot_append_selector_keys", "spot_select", "spot_sparse_decode",
                      "spot_decode_step", "spot_read_device_status",
-                     "spot_sparse_decode_noalloc"):
+                     "spot_sparse_decode_noalloc", "spot_tok_append_selector_keys",
+                     "spot_tok_select", "spot_tok_sparse_decode", "spot_tok_decode_step"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -208,6 +229,89 @@ def decode_step(desc: LayerDesc, params: SelectParams, q_sel, w, sel_data, sel_s
         _ptr(lse, torch.float32, "lse"), _ptr(workspace, name="workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "decode_step")
+
+
+# ---------------------------------------------- token-level, layer-shared selector
+
+def tok_workspace_size(desc: TokLayerDesc, batch: int, max_blocks: int) -> int:
+    n = lib().spot_tok_workspace_size(ctypes.byref(desc), batch, max_blocks)
+    if n == 0:
+        raise SpotError(2, "tok_workspace_size")
+    return int(n)
+
+
+def new_tok_workspace(desc: TokLayerDesc, batch: int, max_blocks: int, device=None):
+    """Zero-filled workspace for the token selector's calls."""
+    n = tok_workspace_size(desc, batch, max_blocks)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def tok_selector_pool(num_pages: int, page_size=64, idx_heads=4, idx_dim=128, device="cuda"):
+    """Empty per-token selector pool bf16 [pages, page_size, idx_heads, idx_dim]."""
+    return torch.zeros(num_pages, page_size, idx_heads, idx_dim, dtype=torch.bfloat16,
+                       device=device)
+
+
+def tok_append_selector_keys(desc: TokLayerDesc, sel_tok, page_table, seq_ids, positions, keys,
+                             status_ws=None, stream=None):
+    """Write per-token selector keys bf16 [n, idx_heads, idx_dim] by position."""
+    pt = page_table
+    code = lib().spot_tok_append_selector_keys(
+        ctypes.byref(desc), _ptr(sel_tok, torch.bfloat16, "sel_tok"),
+        _ptr(pt, torch.int32, "page_table"), int(pt.shape[0]), int(pt.shape[-1]),
+        _ptr(seq_ids, torch.int32, "seq_ids"), _ptr(positions, torch.int32, "positions"),
+        _ptr(keys, torch.bfloat16, "keys"), int(keys.shape[0]),
+        _ptr(status_ws, name="status_ws"), _stream(stream))
+    _check(code, "tok_append_selector_keys")
+
+
+def tok_select(desc: TokLayerDesc, params: SelectParams, q_idx, w_idx, sel_tok, page_table,
+               seq_lens, top_p, sel_idx, sel_cnt, workspace, stream=None):
+    """One selection per sequence into sel_idx int32 [B, max_blocks], sel_cnt int32 [B]."""
+    B, max_blocks = int(q_idx.shape[0]), int(sel_idx.shape[-1])
+    code = lib().spot_tok_select(
+        ctypes.byref(desc), ctypes.byref(params), _ptr(q_idx, torch.bfloat16, "q_idx"),
+        _ptr(w_idx, torch.float32, "w_idx"), _ptr(sel_tok, torch.bfloat16, "sel_tok"),
+        _ptr(page_table, torch.int32, "page_table"), int(page_table.shape[-1]),
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(top_p, torch.float32, "top_p"), B,
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        max_blocks, _ptr(workspace, name="workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "tok_select")
+
+
+def tok_sparse_decode(desc: TokLayerDesc, q, k_pool, v_pool, page_table, seq_lens, sel_idx,
+                      sel_cnt, softmax_scale, out, lse, workspace, stream=None):
+    """Attention of every head over its sequence's selected 16-token blocks."""
+    B, max_blocks = int(q.shape[0]), int(sel_idx.shape[-1])
+    code = lib().spot_tok_sparse_decode(
+        ctypes.byref(desc), _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
+        _ptr(v_pool, torch.bfloat16, "v_pool"), _ptr(page_table, torch.int32, "page_table"),
+        int(page_table.shape[-1]), _ptr(seq_lens, torch.int32, "seq_lens"),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"), max_blocks,
+        B, float(softmax_scale), _ptr(out, torch.float32, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(code, "tok_sparse_decode")
+
+
+def tok_decode_step(desc: TokLayerDesc, params: SelectParams, q_idx, w_idx, sel_tok, q, k_pool,
+                    v_pool, page_table, seq_lens, top_p, softmax_scale, sel_idx, sel_cnt, out,
+                    lse, workspace, stream=None):
+    """tok_select followed by tok_sparse_decode on one stream."""
+    B, max_blocks = int(q.shape[0]), int(sel_idx.shape[-1])
+    code = lib().spot_tok_decode_step(
+        ctypes.byref(desc), ctypes.byref(params), _ptr(q_idx, torch.bfloat16, "q_idx"),
+        _ptr(w_idx, torch.float32, "w_idx"), _ptr(sel_tok, torch.bfloat16, "sel_tok"),
+        _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
+        _ptr(v_pool, torch.bfloat16, "v_pool"), _ptr(page_table, torch.int32, "page_table"),
+        int(page_table.shape[-1]), _ptr(seq_lens, torch.int32, "seq_lens"),
+        _ptr(top_p, torch.float32, "top_p"), B, float(softmax_scale),
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"), max_blocks,
+        _ptr(out, torch.float32, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(code, "tok_decode_step")
 
 
 def check_wait_timeout(workspace, stream=None):

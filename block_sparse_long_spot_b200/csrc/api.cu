@@ -71,14 +71,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 bool make_pool_map(CUtensorMap* map, const void* pool, int num_pages, int num_kv_heads) {
+    return make_rows_map(map, pool, static_cast<int64_t>(num_pages) * num_kv_heads * kBlock,
+                         kBlock);
+}
+
+bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim),
-                                static_cast<cuuint64_t>(num_pages) * num_kv_heads * kBlock};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBlock)};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims,
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -100,6 +104,21 @@ bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Lay
     off = round_up(off + static_cast<size_t>(grid + U) * G * kPartialFloatsPerHead * sizeof(float),
                    256);
     L.total = off;
+    L.tok_scores = 0;
+    *out = L;
+    return true;
+}
+
+// Token selector: the decode layout of (batch x num_kv_heads) units plus the
+// block scores [batch][max_blocks] fp32.
+bool tok_workspace_layout(const spot_tok_layer_desc_t* d, int batch, int max_blocks,
+                          Layout* out) {
+    spot_layer_desc_t bd = {d->num_q_heads, d->num_kv_heads, kHeadDim, kBlock, kSelDim,
+                            SPOT_SEL_BF16, d->num_pages};
+    Layout L;
+    if (!workspace_layout(&bd, batch, max_blocks, &L)) return false;
+    L.tok_scores = L.total;
+    L.total = round_up(L.total + static_cast<size_t>(batch) * max_blocks * sizeof(float), 256);
     *out = L;
     return true;
 }
@@ -140,6 +159,8 @@ spot_status_t do_select(const spot_layer_desc_t* d, const spot_select_params_t* 
     sl.kmin_blocks = pr->kmin_blocks;
     sl.topk_blocks = pr->topk_blocks;
     sl.quantize_queries = pr->quantize_queries;
+    sl.blocks_per_page = 1;
+    sl.scores_in = nullptr;
     sl.sel_idx = sel_idx;
     sl.sel_cnt = sel_cnt;
     sl.status = reinterpret_cast<uint32_t*>(base + L.status);
@@ -177,7 +198,7 @@ spot_status_t do_decode(const spot_layer_desc_t* d, const uint16_t* q, const uin
     p.out = out;
     p.lse = lse;
     p.status = reinterpret_cast<uint32_t*>(base + L.status);
-    if (launch_sparse_decode(p, km, vm, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    if (launch_sparse_decode(p, km, vm, false, s) != cudaSuccess) return SPOT_ERR_CUDA;
     return SPOT_OK;
 }
 
@@ -367,6 +388,265 @@ const char* spot_status_string(spot_status_t status) {
         case SPOT_ERR_DEVICE_TIMEOUT: return "device: bounded wait timed out";
     }
     return "unknown status";
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ token selector
+
+namespace {
+
+spot_status_t check_tok_desc(const spot_tok_layer_desc_t* d) {
+    if (!d) return SPOT_ERR_INVALID_ARG;
+    if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_pages <= 0)
+        return SPOT_ERR_INVALID_ARG;
+    if (d->num_q_heads % d->num_kv_heads != 0) return SPOT_ERR_INVALID_ARG;
+    if (d->head_dim != kHeadDim || d->page_size != kBlock || d->idx_heads != kIdxHeads ||
+        d->idx_dim != kIdxDim || d->sel_block != kTokBlock)
+        return SPOT_ERR_UNSUPPORTED;
+    if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return SPOT_ERR_UNSUPPORTED;
+    // TMA row coordinates are 32-bit (KV rows and selector rows).
+    if (static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock > INT32_MAX ||
+        static_cast<int64_t>(d->num_pages) * kBlock * kIdxHeads > INT32_MAX)
+        return SPOT_ERR_UNSUPPORTED;
+    return SPOT_OK;
+}
+
+spot_status_t check_tok_batch(const spot_tok_layer_desc_t* d, int batch, int max_blocks) {
+    if (batch < 0 || max_blocks <= 0) return SPOT_ERR_INVALID_ARG;
+    if (max_blocks > kMaxBlocks) return SPOT_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(batch) * d->num_kv_heads > kMaxUnits) return SPOT_ERR_UNSUPPORTED;
+    return SPOT_OK;
+}
+
+spot_status_t check_tok_select_args(const spot_select_params_t* pr, const uint16_t* q_idx,
+                                    const float* w, const uint16_t* sel_tok,
+                                    const int32_t* page_table, int32_t pt_stride,
+                                    const int32_t* seq_lens, const float* top_p,
+                                    int32_t* sel_idx, int32_t* sel_cnt) {
+    spot_status_t st = check_params(pr);
+    if (st != SPOT_OK) return st;
+    if (pr->quantize_queries) return SPOT_ERR_UNSUPPORTED;
+    if (!q_idx || !sel_tok || !page_table || !seq_lens || !sel_idx || !sel_cnt)
+        return SPOT_ERR_INVALID_ARG;
+    if (pr->mode == SPOT_MODE_TOPP && !top_p) return SPOT_ERR_INVALID_ARG;
+    if (pt_stride <= 0) return SPOT_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(sel_tok, 256) || !aligned(page_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(sel_idx, 4) || !aligned(sel_cnt, 4) ||
+        (w && !aligned(w, 4)) || (top_p && !aligned(top_p, 4)))
+        return SPOT_ERR_INVALID_ARG;
+    return SPOT_OK;
+}
+
+spot_status_t do_tok_select(const spot_tok_layer_desc_t* d, const spot_select_params_t* pr,
+                            const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
+                            const int32_t* page_table, int32_t pt_stride,
+                            const int32_t* seq_lens, const float* top_p, int32_t batch,
+                            int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks, void* ws,
+                            const Layout& L, cudaStream_t s) {
+    CUtensorMap sm;
+    if (!make_rows_map(&sm, sel_tok, static_cast<int64_t>(d->num_pages) * kBlock * kIdxHeads,
+                       kTokBlock * kIdxHeads))
+        return SPOT_ERR_CUDA;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* scores = reinterpret_cast<float*>(base + L.tok_scores);
+    uint32_t* status = reinterpret_cast<uint32_t*>(base + L.status);
+    TokScoreParams tp;
+    tp.q_idx = q_idx;
+    tp.w = w;
+    tp.page_table = page_table;
+    tp.pt_stride = pt_stride;
+    tp.seq_lens = seq_lens;
+    tp.batch = batch;
+    tp.max_blocks = max_blocks;
+    tp.num_pages = d->num_pages;
+    tp.inv_temp = 1.0f / pr->temperature;
+    tp.scores = scores;
+    tp.num_ctas = tok_score_grid(batch);
+    tp.status = status;
+    if (tp.num_ctas <= 0) return SPOT_ERR_CUDA;
+    if (launch_tok_score(tp, sm, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    SelectParams sl = {};
+    sl.page_table = page_table;
+    sl.pt_stride = pt_stride;
+    sl.seq_lens = seq_lens;
+    sl.top_p = top_p;
+    sl.batch = batch;
+    sl.num_q_heads = 1;
+    sl.num_kv_heads = 1;                 // one selection unit per sequence
+    sl.group = 1;
+    sl.num_pages = d->num_pages;
+    sl.max_blocks = max_blocks;
+    sl.inv_temp = 1.0f;
+    sl.mode = pr->mode;
+    sl.sink_blocks = pr->sink_blocks;
+    sl.recency_blocks = pr->recency_blocks;
+    sl.kmin_blocks = pr->kmin_blocks;
+    sl.topk_blocks = pr->topk_blocks;
+    sl.quantize_queries = 0;
+    sl.blocks_per_page = kTokBlocksPerPage;
+    sl.scores_in = scores;
+    sl.sel_idx = sel_idx;
+    sl.sel_cnt = sel_cnt;
+    sl.status = status;
+    if (launch_select(sl, kSelectFromScores, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    return SPOT_OK;
+}
+
+spot_status_t do_tok_decode(const spot_tok_layer_desc_t* d, const uint16_t* q,
+                            const uint16_t* k_pool, const uint16_t* v_pool,
+                            const int32_t* page_table, int32_t pt_stride,
+                            const int32_t* seq_lens, const int32_t* sel_idx,
+                            const int32_t* sel_cnt, int32_t max_blocks, int32_t batch,
+                            float softmax_scale, float* out, float* lse, void* ws,
+                            const Layout& L, cudaStream_t s) {
+    CUtensorMap km, vm;
+    const int64_t rows = static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock;
+    if (!make_rows_map(&km, k_pool, rows, kTokBlock) || !make_rows_map(&vm, v_pool, rows, kTokBlock))
+        return SPOT_ERR_CUDA;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    DecodeParams p;
+    p.q = q;
+    p.page_table = page_table;
+    p.pt_stride = pt_stride;
+    p.seq_lens = seq_lens;
+    p.sel_idx = sel_idx;
+    p.sel_cnt = sel_cnt;
+    p.max_blocks = max_blocks;
+    p.batch = batch;
+    p.num_q_heads = d->num_q_heads;
+    p.num_kv_heads = d->num_kv_heads;
+    p.group = d->num_q_heads / d->num_kv_heads;
+    p.num_pages = d->num_pages;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.unit_done = reinterpret_cast<uint32_t*>(base + L.unit_done);
+    p.partials = reinterpret_cast<float*>(base + L.partials);
+    p.num_ctas = L.grid;
+    p.out = out;
+    p.lse = lse;
+    p.status = reinterpret_cast<uint32_t*>(base + L.status);
+    if (launch_sparse_decode(p, km, vm, true, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    return SPOT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t spot_tok_workspace_size(const spot_tok_layer_desc_t* desc, int32_t batch,
+                               int32_t max_blocks) {
+    if (check_tok_desc(desc) != SPOT_OK || check_tok_batch(desc, batch, max_blocks) != SPOT_OK)
+        return 0;
+    Layout L;
+    if (!tok_workspace_layout(desc, batch, max_blocks, &L)) return 0;
+    return L.total;
+}
+
+spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, uint16_t* sel_tok,
+                                            const int32_t* page_table, int32_t num_seqs,
+                                            int32_t pt_stride, const int32_t* seq_ids,
+                                            const int32_t* positions, const uint16_t* keys,
+                                            int32_t n, void* status_ws, void* stream) {
+    spot_status_t st = check_tok_desc(desc);
+    if (st != SPOT_OK) return st;
+    if (n < 0 || pt_stride <= 0 || num_seqs < 0) return SPOT_ERR_INVALID_ARG;
+    if (n == 0) return SPOT_OK;
+    if (!sel_tok || !page_table || !seq_ids || !positions || !keys) return SPOT_ERR_INVALID_ARG;
+    if (!aligned(sel_tok, 16) || !aligned(keys, 16) || !aligned(page_table, 4) ||
+        !aligned(seq_ids, 4) || !aligned(positions, 4))
+        return SPOT_ERR_INVALID_ARG;
+    if (status_ws && !aligned(status_ws, 256)) return SPOT_ERR_INVALID_ARG;
+    TokAppendParams p;
+    p.sel_tok = sel_tok;
+    p.page_table = page_table;
+    p.num_seqs = num_seqs;
+    p.pt_stride = pt_stride;
+    p.seq_ids = seq_ids;
+    p.positions = positions;
+    p.keys = keys;
+    p.n = n;
+    p.num_pages = desc->num_pages;
+    p.status = static_cast<uint32_t*>(status_ws);
+    return launch_tok_append(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SPOT_OK
+                                                                                 : SPOT_ERR_CUDA;
+}
+
+spot_status_t spot_tok_select(const spot_tok_layer_desc_t* desc,
+                              const spot_select_params_t* params, const uint16_t* q_idx,
+                              const float* w_idx, const uint16_t* sel_tok,
+                              const int32_t* page_table, int32_t pt_stride,
+                              const int32_t* seq_lens, const float* top_p, int32_t batch,
+                              int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    spot_status_t st = check_tok_desc(desc);
+    if (st == SPOT_OK) st = check_tok_batch(desc, batch, max_blocks);
+    if (st != SPOT_OK) return st;
+    if (batch == 0) return SPOT_OK;
+    st = check_tok_select_args(params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+                               top_p, sel_idx, sel_cnt);
+    if (st != SPOT_OK) return st;
+    Layout L;
+    if (!tok_workspace_layout(desc, batch, max_blocks, &L)) return SPOT_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, L);
+    if (st != SPOT_OK) return st;
+    return do_tok_select(desc, params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+                         top_p, batch, sel_idx, sel_cnt, max_blocks, workspace, L,
+                         static_cast<cudaStream_t>(stream));
+}
+
+spot_status_t spot_tok_sparse_decode(const spot_tok_layer_desc_t* desc, const uint16_t* q,
+                                     const uint16_t* k_pool, const uint16_t* v_pool,
+                                     const int32_t* page_table, int32_t pt_stride,
+                                     const int32_t* seq_lens, const int32_t* sel_idx,
+                                     const int32_t* sel_cnt, int32_t max_blocks, int32_t batch,
+                                     float softmax_scale, float* out, float* lse,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+    spot_status_t st = check_tok_desc(desc);
+    if (st == SPOT_OK) st = check_tok_batch(desc, batch, max_blocks);
+    if (st != SPOT_OK) return st;
+    if (batch == 0) return SPOT_OK;
+    st = check_decode_args(q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx, sel_cnt,
+                           softmax_scale, out, lse);
+    if (st != SPOT_OK) return st;
+    Layout L;
+    if (!tok_workspace_layout(desc, batch, max_blocks, &L)) return SPOT_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, L);
+    if (st != SPOT_OK) return st;
+    return do_tok_decode(desc, q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx,
+                         sel_cnt, max_blocks, batch, softmax_scale, out, lse, workspace, L,
+                         static_cast<cudaStream_t>(stream));
+}
+
+spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
+                                   const spot_select_params_t* params, const uint16_t* q_idx,
+                                   const float* w_idx, const uint16_t* sel_tok,
+                                   const uint16_t* q, const uint16_t* k_pool,
+                                   const uint16_t* v_pool, const int32_t* page_table,
+                                   int32_t pt_stride, const int32_t* seq_lens,
+                                   const float* top_p, int32_t batch, float softmax_scale,
+                                   int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
+                                   float* out, float* lse, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+    spot_status_t st = check_tok_desc(desc);
+    if (st == SPOT_OK) st = check_tok_batch(desc, batch, max_blocks);
+    if (st != SPOT_OK) return st;
+    if (batch == 0) return SPOT_OK;
+    st = check_tok_select_args(params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+                               top_p, sel_idx, sel_cnt);
+    if (st == SPOT_OK)
+        st = check_decode_args(q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx,
+                               sel_cnt, softmax_scale, out, lse);
+    if (st != SPOT_OK) return st;
+    Layout L;
+    if (!tok_workspace_layout(desc, batch, max_blocks, &L)) return SPOT_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, L);
+    if (st != SPOT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = do_tok_select(desc, params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+                       top_p, batch, sel_idx, sel_cnt, max_blocks, workspace, L, s);
+    if (st != SPOT_OK) return st;
+    return do_tok_decode(desc, q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx,
+                         sel_cnt, max_blocks, batch, softmax_scale, out, lse, workspace, L, s);
 }
 
 }  // extern "C"

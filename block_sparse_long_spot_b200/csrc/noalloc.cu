@@ -120,5 +120,5 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
     p.out = out;
     p.lse = lse;
     p.status = reinterpret_cast<uint32_t*>(base);
-    return launch_sparse_decode(p, km, vm, s) == cudaSuccess ? SPOT_OK : SPOT_ERR_CUDA;
+    return launch_sparse_decode(p, km, vm, false, s) == cudaSuccess ? SPOT_OK : SPOT_ERR_CUDA;
 }

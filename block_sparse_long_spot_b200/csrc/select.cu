@@ -25,6 +25,9 @@
 //   blocks inside that bucket are ranked exactly (score descending, lower
 //   block index first).  The K_min floor and static top-K use the same search
 //   on counts.  A block scan compacts the kept blocks in ascending order.
+//
+// The token-level selector reuses the selection with its block scores
+// computed by tok_select.cu (one CTA per sequence, blocks of 16 tokens).
 #include <cuda_fp8.h>
 #include <math.h>
 
@@ -651,9 +654,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     const int u = blockIdx.x;
     const int b = u / p.num_kv_heads;
     const int L = max(p.seq_lens[b], 0);
-    int nb = (L + kBlock - 1) / kBlock;
-    int n_full = L / kBlock;
-    const int cap = min(p.max_blocks, p.pt_stride);
+    const int bsz = kBlock / p.blocks_per_page;        // tokens per selection block
+    int nb = (L + bsz - 1) / bsz;
+    int n_full = L / bsz;
+    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
     if (nb > cap) {
         if (threadIdx.x == 0) flag_status(p.status, kStatusBounds);
         nb = cap;
@@ -672,7 +676,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     pdl_trigger();                                    // the decode kernel may start its prologue
 
     // ---- selector scores of the complete blocks (§2.1), into shared memory
-    {
+    if constexpr (FMT == kSelectFromScores) {
+        pdl_wait();                                   // block scores of the scoring kernel
+        const float* src = p.scores_in + static_cast<int64_t>(u) * p.max_blocks;
+        for (int j = threadIdx.x; j < n_full; j += NT) sm.score[j] = src[j];
+    } else {
         const int g = u - b * p.num_kv_heads;
         uint32_t qw[8];
         float qsc[2][2], wh0, wh1;
@@ -857,7 +865,12 @@ cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s) {
     const size_t smem = select_smem_bytes(p.max_blocks);
     const dim3 grid(p.batch * p.num_kv_heads), block(kSelectThreads);
     cudaError_t e;
-    if (fmt == SPOT_SEL_BF16) {
+    if (fmt == kSelectFromScores) {
+        e = cudaFuncSetAttribute(select_kernel<kSelectFromScores>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess)
+            e = launch_pdl(select_kernel<kSelectFromScores>, grid, block, smem, s, p);
+    } else if (fmt == SPOT_SEL_BF16) {
         e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_BF16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e == cudaSuccess) select_kernel<SPOT_SEL_BF16><<<grid, block, smem, s>>>(p);

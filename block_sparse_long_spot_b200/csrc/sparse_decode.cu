@@ -23,6 +23,13 @@
 //   O^T[128 x 8] += V^T[128 x 64] . P^T[64 x 8]      (P^T via movmatrix)
 // At the end of a unit's segment the NC warps merge their states in shared
 // memory and the CTA writes one partial (acc[G][128], m[G], l[G]).
+//
+// The same kernel serves the token-level selector (S16): there one
+// selection per sequence, in blocks of 16 tokens, is shared by every KV head
+// of the sequence, and a stage gathers four selected 16-token blocks (four
+// 16-row boxes each for K and V, into the four 16-row slices of the tile), so
+// the consumers' 64-token tile computation is unchanged; each slice carries
+// its own count of valid tokens.
 #include <math.h>
 #include <stdio.h>
 
@@ -44,7 +51,7 @@ struct Smem {
     uint32_t stage_base;
     uint64_t* full;
     uint64_t* empty;
-    int* valid;          // [STAGES] valid tokens of the block in each stage
+    int* valid;          // [STAGES] valid tokens of each 16-row slice, 4 packed bytes
     int* unit_off;       // [U + 1]
     int* scan;           // [kThreads/32 + 1]
 };
@@ -142,6 +149,16 @@ __device__ void merge_unit_head(const DecodeParams& p, int u, int n, int lo, int
     if (p.lse && lane == 0) p.lse[h] = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
 }
 
+// Valid tokens of the four 16-row slices of a 64-row tile, one byte each.
+__device__ __forceinline__ uint32_t pack_valid64(int nvalid) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        v |= static_cast<uint32_t>(min(max(nvalid - 16 * k, 0), 16)) << (8 * k);
+    return v;
+}
+
+template <bool S16>
 __global__ void __launch_bounds__(kThreads)
 sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
@@ -190,12 +207,14 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
     for (int u = u_lo; u < u_hi; ++u) {
         const int b = u / p.num_kv_heads;
         const int L = max(p.seq_lens[b], 0);
-        const int nb = min((L + kBlock - 1) / kBlock, p.max_blocks);
-        int c = p.sel_cnt[u];
+        const int bsz = S16 ? kTokBlock : kBlock;
+        const int nb = min((L + bsz - 1) / bsz, p.max_blocks);
+        int c = p.sel_cnt[S16 ? b : u];
         if (c < 0 || c > nb) {
             if (blockIdx.x == 0) flag_status(p.status, kStatusBounds);
             c = min(max(c, 0), nb);
         }
+        if (S16) c = (c + 3) / 4;  // four selected blocks per 64-row tile
         unit_off[u] = c;          // temporarily the count
         local += c;
     }
@@ -236,31 +255,71 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
         int issued = 0;
         for (int base_it = 0; base_it < n_it && alive; base_it += 32) {
             const int it = base_it + lane;
-            int row = 0, nvalid = 0;
+            int row[S16 ? 4 : 1] = {};
+            uint32_t vpack = 0;
             if (it < n_it) {
                 const int pos = beg + it;
                 const int u = find_unit(unit_off, U, pos);
                 const int i = pos - unit_off[u];
                 const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
-                const int j = p.sel_idx[static_cast<int64_t>(u) * p.max_blocks + i];
                 const int L = max(p.seq_lens[b], 0);
-                const int nb = (L + kBlock - 1) / kBlock;
-                int page = -1;
-                if (j >= 0 && j < nb && j < p.pt_stride)
-                    page = p.page_table[static_cast<int64_t>(b) * p.pt_stride + j];
-                if (page < 0 || page >= p.num_pages) {
-                    flag_status(p.status, kStatusBounds);
-                    page = 0;
-                    nvalid = 0;                 // tile is loaded but not attended
+                if (S16) {
+                    // selected 16-token blocks 4 i .. 4 i + 3 of sequence b; a
+                    // missing or bad one re-reads a valid slice with 0 tokens
+                    const int nb = (L + kTokBlock - 1) / kTokBlock;
+                    const int cnt = min(max(p.sel_cnt[b], 0), min(nb, p.max_blocks));
+                    const int32_t* sl = p.sel_idx + static_cast<int64_t>(b) * p.max_blocks;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        int r = -1, nv = 0;
+                        if (4 * i + k < cnt) {
+                            const int j = sl[4 * i + k];
+                            int page = -1;
+                            if (j >= 0 && j < nb && j / kTokBlocksPerPage < p.pt_stride)
+                                page = p.page_table[static_cast<int64_t>(b) * p.pt_stride +
+                                                    j / kTokBlocksPerPage];
+                            if (page < 0 || page >= p.num_pages) {
+                                flag_status(p.status, kStatusBounds);
+                            } else {
+                                r = (page * p.num_kv_heads + g) * kBlock +
+                                    (j % kTokBlocksPerPage) * kTokBlock;
+                                nv = min(kTokBlock, L - j * kTokBlock);
+                            }
+                        }
+                        row[k] = r;
+                        vpack |= static_cast<uint32_t>(nv) << (8 * k);
+                    }
+                    int fallback = 0;
+#pragma unroll
+                    for (int k = 3; k >= 0; --k)
+                        if (row[k] >= 0) fallback = row[k];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (row[k] < 0) row[k] = fallback;
                 } else {
-                    nvalid = min(kBlock, L - j * kBlock);
+                    const int j = p.sel_idx[static_cast<int64_t>(u) * p.max_blocks + i];
+                    const int nb = (L + kBlock - 1) / kBlock;
+                    int page = -1;
+                    int nvalid;
+                    if (j >= 0 && j < nb && j < p.pt_stride)
+                        page = p.page_table[static_cast<int64_t>(b) * p.pt_stride + j];
+                    if (page < 0 || page >= p.num_pages) {
+                        flag_status(p.status, kStatusBounds);
+                        page = 0;
+                        nvalid = 0;                 // tile is loaded but not attended
+                    } else {
+                        nvalid = min(kBlock, L - j * kBlock);
+                    }
+                    row[0] = (page * p.num_kv_heads + g) * kBlock;
+                    vpack = pack_valid64(nvalid);
                 }
-                row = (page * p.num_kv_heads + g) * kBlock;
             }
             const int n_here = min(32, n_it - base_it);
             for (int k = 0; k < n_here; ++k) {
-                const int r = __shfl_sync(0xffffffffu, row, k);
-                const int v = __shfl_sync(0xffffffffu, nvalid, k);
+                int r[S16 ? 4 : 1];
+#pragma unroll
+                for (int e = 0; e < (S16 ? 4 : 1); ++e) r[e] = __shfl_sync(0xffffffffu, row[e], k);
+                const uint32_t v = __shfl_sync(0xffffffffu, vpack, k);
                 const int itk = base_it + k;
                 const int s = itk % STAGES;
                 const int round = itk / STAGES;
@@ -272,13 +331,18 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                         flags[0] = 1;
                         ok = 0;
                     } else {
-                        valid[s] = v;
+                        valid[s] = static_cast<int>(v);
                         mbar_arrive_expect_tx(&full[s], kStageBytes);
                         uint8_t* dst = base + s * kStageBytes;
-                        tma_load_2d(dst, &k_map, &full[s], 0, r, policy);
-                        tma_load_2d(dst + kHalfTile, &k_map, &full[s], 64, r, policy);
-                        tma_load_2d(dst + 2 * kHalfTile, &v_map, &full[s], 0, r, policy);
-                        tma_load_2d(dst + 3 * kHalfTile, &v_map, &full[s], 64, r, policy);
+#pragma unroll
+                        for (int e = 0; e < (S16 ? 4 : 1); ++e) {
+                            // S16: slice e = rows [16 e, 16 e + 16) of each half
+                            uint8_t* d = dst + e * (kHalfTile / 4);
+                            tma_load_2d(d, &k_map, &full[s], 0, r[e], policy);
+                            tma_load_2d(d + kHalfTile, &k_map, &full[s], 64, r[e], policy);
+                            tma_load_2d(d + 2 * kHalfTile, &v_map, &full[s], 0, r[e], policy);
+                            tma_load_2d(d + 3 * kHalfTile, &v_map, &full[s], 64, r[e], policy);
+                        }
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -340,7 +404,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                 }
                 break;
             }
-            const int nvalid = valid[s];
+            const uint32_t vpack = static_cast<uint32_t>(valid[s]);
             const uint32_t kb = stage_base + s * kStageBytes;
             const uint32_t vb = kb + 2 * kHalfTile;
 
@@ -362,13 +426,14 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                     mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
                 }
             }
-            // ---- mask tokens past the end of the sequence
-            if (nvalid < kBlock) {
+            // ---- mask rows past each slice's valid tokens (sequence end,
+            // missing or rejected blocks); m-tile mt is slice mt
+            if (vpack != 0x10101010u) {
 #pragma unroll
                 for (int mt = 0; mt < 4; ++mt) {
-                    const int t0 = mt * 16 + r8, t1 = t0 + 8;
-                    if (t0 >= nvalid) { sc[mt][0] = -INFINITY; sc[mt][1] = -INFINITY; }
-                    if (t1 >= nvalid) { sc[mt][2] = -INFINITY; sc[mt][3] = -INFINITY; }
+                    const int nv = static_cast<int>((vpack >> (8 * mt)) & 0xFFu);
+                    if (r8 >= nv) { sc[mt][0] = -INFINITY; sc[mt][1] = -INFINITY; }
+                    if (r8 + 8 >= nv) { sc[mt][2] = -INFINITY; sc[mt][3] = -INFINITY; }
                 }
             }
             // ---- online softmax per head (columns 2 c4, 2 c4 + 1)
@@ -521,7 +586,7 @@ namespace {
 // shared-memory limit already set on the kernel and the last grid size
 // computed (the grid depends on the device and, through shared memory, on U).
 struct DeviceMemo {
-    size_t smem_set = 0;
+    size_t smem_set[2] = {0, 0};       // per kernel instance (64-token, shared 16-token)
     int units = -1;
     int grid = 0;
 };
@@ -529,12 +594,16 @@ constexpr int kMemoDevices = 64;
 DeviceMemo g_memo[kMemoDevices];
 std::mutex g_memo_mutex;
 
-cudaError_t ensure_smem(int dev, size_t smem) {
+cudaError_t ensure_smem(int dev, size_t smem, bool s16) {
     DeviceMemo& m = g_memo[dev];
-    if (m.smem_set >= smem) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(
-        sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e == cudaSuccess) m.smem_set = smem;
+    if (m.smem_set[s16] >= smem) return cudaSuccess;
+    cudaError_t e = s16 ? cudaFuncSetAttribute(sparse_decode_kernel<true>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem))
+                        : cudaFuncSetAttribute(sparse_decode_kernel<false>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e == cudaSuccess) m.smem_set[s16] = smem;
     return e;
 }
 
@@ -549,9 +618,10 @@ int decode_grid(int units) {
     int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
     const size_t smem = decode_smem_bytes(units);
-    if (ensure_smem(dev, smem) != cudaSuccess) return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_decode_kernel, kThreads,
-                                                      smem) != cudaSuccess)
+    if (ensure_smem(dev, smem, false) != cudaSuccess) return 0;
+    // both instances use the same threads and shared memory
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_decode_kernel<false>,
+                                                      kThreads, smem) != cudaSuccess)
         return 0;
     m.units = units;
     m.grid = sms * max(per_sm, 1);
@@ -559,7 +629,7 @@ int decode_grid(int units) {
 }
 
 cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
-                                 const CUtensorMap& v_map, cudaStream_t s) {
+                                 const CUtensorMap& v_map, bool shared16, cudaStream_t s) {
     const int U = p.batch * p.num_kv_heads;
     const size_t smem = decode_smem_bytes(U);
     int dev = 0;
@@ -568,11 +638,14 @@ cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map
     if (dev < 0 || dev >= kMemoDevices) return cudaErrorInvalidDevice;
     {
         std::lock_guard<std::mutex> lock(g_memo_mutex);
-        e = ensure_smem(dev, smem);
+        e = ensure_smem(dev, smem, shared16);
     }
     if (e != cudaSuccess) return e;
-    return launch_pdl(sparse_decode_kernel, dim3(p.num_ctas), dim3(kThreads), smem, s, k_map,
-                      v_map, p);
+    if (shared16)
+        return launch_pdl(sparse_decode_kernel<true>, dim3(p.num_ctas), dim3(kThreads), smem, s,
+                          k_map, v_map, p);
+    return launch_pdl(sparse_decode_kernel<false>, dim3(p.num_ctas), dim3(kThreads), smem, s,
+                      k_map, v_map, p);
 }
 
 }  // namespace spot

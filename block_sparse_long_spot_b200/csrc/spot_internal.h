@@ -34,8 +34,17 @@ constexpr int kStageBytes = 2 * kBlock * kHeadDim * 2;   // 32768
 // every slot (G x 132 floats) and every acc row starts 16-byte aligned.
 constexpr int kPartialFloatsPerHead = kHeadDim + 4;
 
+// Token-level, layer-shared selector (per-token keys of kIdxHeads index
+// heads x kIdxDim, selection blocks of kTokBlock tokens inside the pages).
+constexpr int kIdxHeads = 4;
+constexpr int kIdxDim = 128;
+constexpr int kTokBlock = 16;
+constexpr int kTokBlocksPerPage = kBlock / kTokBlock;     // 4
+constexpr int kSelectFromScores = -1;  // launch_select "format": scores precomputed
+
 struct Layout {
     size_t status, unit_done, partials, total;
+    size_t tok_scores;                  // token selector: block scores [B][max_blocks]
     int grid;                           // persistent CTAs of the decode kernel
 };
 
@@ -56,6 +65,8 @@ struct SelectParams {
     float inv_temp;
     int32_t mode, sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
     int32_t quantize_queries;           // quantise q_sel with the key format's rule
+    int32_t blocks_per_page;            // selection blocks per page-table entry (1 or 4)
+    const float* scores_in;             // kSelectFromScores: block scores [units][max_blocks]
     int32_t* sel_idx;
     int32_t* sel_cnt;
     uint32_t* status;
@@ -91,6 +102,32 @@ struct AppendParams {
     uint32_t* status;
 };
 
+// Block scores of the token-level selector.
+struct TokScoreParams {
+    const uint16_t* q_idx;              // [B][kIdxHeads][kIdxDim]
+    const float* w;                     // [B][kIdxHeads] or null (1 / kIdxHeads)
+    const int32_t* page_table;
+    int32_t pt_stride;
+    const int32_t* seq_lens;
+    int32_t batch, max_blocks, num_pages;
+    float inv_temp;
+    float* scores;                      // [B][max_blocks]
+    int32_t num_ctas;
+    uint32_t* status;
+};
+
+// Append of per-token selector keys.
+struct TokAppendParams {
+    uint16_t* sel_tok;                  // [num_pages][kBlock][kIdxHeads][kIdxDim]
+    const int32_t* page_table;
+    int32_t num_seqs, pt_stride;
+    const int32_t* seq_ids;
+    const int32_t* positions;
+    const uint16_t* keys;               // [n][kIdxHeads][kIdxDim]
+    int32_t n, num_pages;
+    uint32_t* status;
+};
+
 // Launch with programmatic stream serialisation (the kernel must call
 // pdl_wait() before touching anything its predecessor writes).
 template <typename... KArgs, typename... Args>
@@ -110,8 +147,13 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s);
+// shared16: the token selector's layout (one selection per sequence shared
+// by its KV heads, blocks of kTokBlock tokens; maps with 16-row boxes).
 cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
-                                 const CUtensorMap& v_map, cudaStream_t s);
+                                 const CUtensorMap& v_map, bool shared16, cudaStream_t s);
+cudaError_t launch_tok_score(const TokScoreParams& p, const CUtensorMap& sel_map, cudaStream_t s);
+cudaError_t launch_tok_append(const TokAppendParams& p, cudaStream_t s);
+int tok_score_grid(int batch);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
 // Persistent grid of the decode kernel for U units on the current device.
@@ -122,5 +164,8 @@ size_t select_smem_bytes(int max_blocks);
 // Tensor map over a KV pool viewed as [num_pages*Hkv*64 rows][128 bf16],
 // box 64 x 64, 128-byte swizzle.
 bool make_pool_map(CUtensorMap* map, const void* pool, int num_pages, int num_kv_heads);
+// Tensor map over `rows` rows of 128 bf16 (256 B), box 64 columns x
+// box_rows rows, 128-byte swizzle.
+bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 
 }  // namespace spot

@@ -228,6 +228,86 @@ spot_status_t spot_sparse_decode_noalloc(const spot_layer_desc_t* desc, const ui
                                          int32_t batch, float softmax_scale, float* out,
                                          float* lse, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Token-level, layer-shared selector (§2.1, §2.3 and App. A Tab. 3 as the
+ * paper writes them): every token carries one selector key per index head,
+ * the token score is s[t] = (1/tau) sum_h w_h ReLU(q^I_h . k^I_{h,t}), a
+ * block of sel_block tokens scores the maximum of its tokens' scores, and
+ * ONE selection per sequence (dual top-p / static top-K over those blocks,
+ * Eq. 6-8) is shared by every head of the layer.  Supported: idx_heads 4,
+ * idx_dim 128, sel_block 16, page_size 64, head_dim 128, bf16 keys,
+ * 1 <= G <= 8, batch * num_kv_heads <= 4096, max_blocks <= 8192 (128K tokens).
+ *
+ * Layouts (in addition to the ones above; pages are shared with the KV pools):
+ *   q_idx      bf16  [batch][idx_heads][idx_dim]
+ *   w_idx      fp32  [batch][idx_heads]          (NULL: 1/idx_heads)
+ *   sel_tok    bf16  [num_pages][page_size][idx_heads][idx_dim]: token t of
+ *                    sequence b at page page_table[b*pt_stride + t/page_size],
+ *                    row t % page_size
+ *   sel_idx    int32 [batch][max_blocks]: selected blocks of sel_block tokens,
+ *                    ascending, first sel_cnt entries valid
+ *   sel_cnt    int32 [batch]
+ * The selection parameters count blocks of sel_block tokens (the paper's
+ * sink 128 / recency 256 / K_min 512 tokens are 8 / 16 / 32 blocks);
+ * quantize_queries must be 0.  nb(b) = ceil(seq_lens[b] / sel_block); an
+ * incomplete last block has no score and is always kept.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;             /* 128 */
+    int32_t page_size;            /* 64 tokens per KV / selector page */
+    int32_t idx_heads;            /* H_idx = 4 */
+    int32_t idx_dim;              /* d_idx = 128 */
+    int32_t sel_block;            /* 16 tokens per selection block */
+    int32_t num_pages;
+} spot_tok_layer_desc_t;
+
+/* Scratch bytes for the token selector's calls (same rules as
+ * spot_workspace_size: zero the first 256 bytes once).  0 if unsupported. */
+size_t spot_tok_workspace_size(const spot_tok_layer_desc_t* desc, int32_t batch,
+                               int32_t max_blocks);
+
+/* Write n tokens' selector keys keys[i] (bf16 [n][idx_heads][idx_dim]) for
+ * token positions[i] of sequence seq_ids[i] into sel_tok.  Bad ids or pages
+ * are skipped and recorded in status_ws (may be NULL). */
+spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, uint16_t* sel_tok,
+                                            const int32_t* page_table, int32_t num_seqs,
+                                            int32_t pt_stride, const int32_t* seq_ids,
+                                            const int32_t* positions, const uint16_t* keys,
+                                            int32_t n, void* status_ws, void* stream);
+
+/* Block scores and one selection per sequence: writes sel_idx / sel_cnt. */
+spot_status_t spot_tok_select(const spot_tok_layer_desc_t* desc,
+                              const spot_select_params_t* params, const uint16_t* q_idx,
+                              const float* w_idx, const uint16_t* sel_tok,
+                              const int32_t* page_table, int32_t pt_stride,
+                              const int32_t* seq_lens, const float* top_p, int32_t batch,
+                              int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* Exact attention of every query head over the tokens of its sequence's
+ * selected blocks (the selection is shared by all KV heads). */
+spot_status_t spot_tok_sparse_decode(const spot_tok_layer_desc_t* desc, const uint16_t* q,
+                                     const uint16_t* k_pool, const uint16_t* v_pool,
+                                     const int32_t* page_table, int32_t pt_stride,
+                                     const int32_t* seq_lens, const int32_t* sel_idx,
+                                     const int32_t* sel_cnt, int32_t max_blocks, int32_t batch,
+                                     float softmax_scale, float* out, float* lse,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+/* spot_tok_select followed by spot_tok_sparse_decode (three kernels). */
+spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
+                                   const spot_select_params_t* params, const uint16_t* q_idx,
+                                   const float* w_idx, const uint16_t* sel_tok,
+                                   const uint16_t* q, const uint16_t* k_pool,
+                                   const uint16_t* v_pool, const int32_t* page_table,
+                                   int32_t pt_stride, const int32_t* seq_lens,
+                                   const float* top_p, int32_t batch, float softmax_scale,
+                                   int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
+                                   float* out, float* lse, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
 /* Synchronise `stream`, return the status recorded by kernels in
  * `workspace` since the last read (SPOT_OK, SPOT_ERR_DEVICE_BOUNDS or
  * SPOT_ERR_DEVICE_TIMEOUT; bounds wins if both), and clear it. */

@@ -127,6 +127,41 @@ def unit_selection(res, b, g):
     return res["sel_idx"][b, g, :res["sel_cnt"][b, g]].tolist()
 
 
+def _reserved_residual(L, bsz, sink, rec):
+    """Reserved (sink / recency, incomplete last block) and residual block
+    ids of a sequence of L tokens in blocks of bsz."""
+    nb, n_full = (L + bsz - 1) // bsz, L // bsz
+    r_eff = min(max(rec, nb - n_full), nb)
+    s_eff = min(sink, nb)
+    reserved = set(range(s_eff)) | set(range(nb - r_eff, nb))
+    return reserved, [j for j in range(nb) if j not in reserved]
+
+
+def _unit_near_cut(sg, so, s, reserved, res, p, kmin, where):
+    """Check one unit's GPU set sg against the oracle's so under the
+    real-valued rule; returns 1 if they differ (all near the cut), else 0."""
+    assert reserved <= sg, where
+    if sg == so:
+        return 0
+    nuc_o = so - reserved
+    assert nuc_o, where
+    cut = min(s[j] for j in nuc_o)
+    for j in sg ^ so:
+        assert j in res, (where, j)
+        assert abs(s[j] - cut) <= CUT_REL * abs(cut) + 1e-12, (where, j, s[j], cut)
+    # the GPU set is itself a valid nucleus in fp64
+    sr = np.array([s[j] for j in res])
+    e = np.exp(sr - sr.max())
+    e /= e.sum()
+    mass = {j: e[i] for i, j in enumerate(res)}
+    nuc_g = sorted(sg - reserved, key=lambda j: (-s[j], j))
+    if len(nuc_g) > max(kmin - len(reserved), 0):
+        m_g = sum(mass[j] for j in nuc_g)
+        assert m_g >= p - MASS_TOL, (where, m_g, p)
+        assert m_g - mass[nuc_g[-1]] < p + MASS_TOL, (where, m_g, p)
+    return 1
+
+
 def check_selection_near_cut(gpu, ora, scores, wl, kmin=None, sink=None, rec=None):
     """Apply the real-valued selection rule to every unit; return the number
     of (sequence, KV head) units whose sets differ (all near the cut)."""
@@ -137,36 +172,10 @@ def check_selection_near_cut(gpu, ora, scores, wl, kmin=None, sink=None, rec=Non
     p_all = wl.top_p.cpu().numpy()
     n_diff = 0
     for b in range(wl.batch):
-        L = int(lens[b])
-        nb, n_full = (L + 63) // 64, L // 64
-        r_eff = min(max(rec, nb - n_full), nb)
-        s_eff = min(sink, nb)
-        reserved = set(range(s_eff)) | set(range(nb - r_eff, nb))
-        res = [j for j in range(nb) if j not in reserved]
+        reserved, res = _reserved_residual(int(lens[b]), 64, sink, rec)
         for g in range(wl.num_kv_heads):
-            sg, so = set(unit_selection(gpu, b, g)), set(unit_selection(ora, b, g))
-            assert reserved <= sg, (b, g)
-            if sg == so:
-                continue
-            n_diff += 1
-            s = scores[b, g]
-            nuc_o = so - reserved
-            assert nuc_o, (b, g)
-            cut = min(s[j] for j in nuc_o)
-            for j in sg ^ so:
-                assert j in res, (b, g, j)
-                assert abs(s[j] - cut) <= CUT_REL * abs(cut) + 1e-12, (b, g, j, s[j], cut)
-            # the GPU set is itself a valid nucleus in fp64
-            sr = np.array([s[j] for j in res])
-            e = np.exp(sr - sr.max())
-            e /= e.sum()
-            mass = {j: e[i] for i, j in enumerate(res)}
-            nuc_g = sorted(sg - reserved, key=lambda j: (-s[j], j))
-            if len(nuc_g) > max(kmin - len(reserved), 0):
-                m_g = sum(mass[j] for j in nuc_g)
-                p = float(p_all[b])
-                assert m_g >= p - MASS_TOL, (b, g, m_g, p)
-                assert m_g - mass[nuc_g[-1]] < p + MASS_TOL, (b, g, m_g, p)
+            n_diff += _unit_near_cut(set(unit_selection(gpu, b, g)), set(unit_selection(ora, b, g)),
+                                     scores[b, g], reserved, res, float(p_all[b]), kmin, (b, g))
     return n_diff
 
 
@@ -213,6 +222,128 @@ def safe_top_p(wl, fmt="bf16", lo=0.5, hi=0.99, margin=2e-5, **kw):
             s = np.array([scores[b, g, j] for j in res])
             if s.size == 0:
                 continue
+            order = sorted(range(len(res)), key=lambda i: (-s[i], res[i]))
+            e = np.exp(s - s.max())
+            e /= e.sum()
+            cums += np.cumsum(e[order]).tolist()
+        c = np.unique(np.clip(np.array(cums), lo, hi))
+        gaps = np.diff(c)
+        k = int(np.argmax(gaps))
+        assert gaps[k] > 2 * margin
+        ps.append(0.5 * (c[k] + c[k + 1]))
+    return torch.as_tensor(np.array(ps, np.float32), device=wl.top_p.device)
+
+
+# ------------------------------------------------ token-level, layer-shared selector
+
+def _tok_sel(spec, kmin, sink, rec):
+    return (spec.kmin_blocks if kmin is None else kmin, spec.sink_blocks if sink is None else sink,
+            spec.recency_blocks if rec is None else rec)
+
+
+def run_gpu_tok(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None, temperature=1.0,
+                max_blocks=None, pool=None):
+    dev = wl.q.device
+    B, Hq, Hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
+    mb = wl.max_blocks if max_blocks is None else max_blocks
+    kmin, sink, rec = _tok_sel(wl.spec, kmin, sink, rec)
+    desc = spot.tok_layer_desc(Hq, Hkv, wl.num_pages)
+    prm = spot.select_params(mode, sink, rec, kmin, topk, temperature)
+    ws = spot.new_tok_workspace(desc, B, mb, dev)
+    sel_idx = torch.full((B, mb), -1, dtype=torch.int32, device=dev)
+    sel_cnt = torch.full((B,), -1, dtype=torch.int32, device=dev)
+    out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
+    spot.tok_decode_step(desc, prm, wl.q_idx, wl.w_idx, wl.sel_tok if pool is None else pool,
+                         wl.q, wl.k_pool, wl.v_pool, wl.page_table, wl.seq_lens, wl.top_p,
+                         wl.sm_scale, sel_idx, sel_cnt, out, lse, ws)
+    torch.cuda.synchronize()
+    status = spot.read_device_status(ws)
+    return {"sel_idx": sel_idx.cpu().numpy(), "sel_cnt": sel_cnt.cpu().numpy(),
+            "out": out.cpu().double().numpy(), "lse": lse.cpu().double().numpy(),
+            "status": status}
+
+
+def tok_oracle_args(wl):
+    return dict(q_idx=workloads.bits(wl.q_idx), w=host_bytes(wl.w_idx),
+                sel_tok=workloads.bits(wl.sel_tok), q=workloads.bits(wl.q),
+                k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
+                page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
+                top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
+
+
+def tok_oracle_shape_params(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None,
+                            temperature=1.0, max_blocks=None):
+    kmin, sink, rec = _tok_sel(wl.spec, kmin, sink, rec)
+    sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
+                               wl.max_pages, max_blocks=wl.max_blocks if max_blocks is None
+                               else max_blocks)
+    pr = oracle.make_params(mode, sink, rec, kmin, topk, temperature)
+    return sh, pr
+
+
+def run_oracle_tok(wl, seqs=None, args=None, **kw):
+    sh, pr = tok_oracle_shape_params(wl, **kw)
+    a = args or tok_oracle_args(wl)
+    return oracle.tok_decode_step(sh, pr, seqs=seqs, **a)
+
+
+def oracle_tok_scores(wl, args=None, **kw):
+    sh, pr = tok_oracle_shape_params(wl, **kw)
+    a = args or tok_oracle_args(wl)
+    return oracle.tok_block_scores(sh, pr, a["q_idx"], a["w"], a["sel_tok"], a["page_table"],
+                                   a["seq_lens"])
+
+
+def tok_selection(res, b):
+    return res["sel_idx"][b, :res["sel_cnt"][b]].tolist()
+
+
+def check_tok_selection_near_cut(gpu, ora, scores, wl, seqs=None, kmin=None, sink=None,
+                                 rec=None):
+    """The real-valued selection rule per sequence; returns how many
+    sequences' shared selections differ (all near the cut)."""
+    kmin, sink, rec = _tok_sel(wl.spec, kmin, sink, rec)
+    lens = wl.seq_lens.cpu().numpy()
+    p_all = wl.top_p.cpu().numpy()
+    n_diff = 0
+    for b in (range(wl.batch) if seqs is None else seqs):
+        reserved, res = _reserved_residual(int(lens[b]), wl.spec.sel_block, sink, rec)
+        n_diff += _unit_near_cut(set(tok_selection(gpu, b)), set(tok_selection(ora, b)),
+                                 scores[b], reserved, res, float(p_all[b]), kmin, b)
+    return n_diff
+
+
+def check_tok_outputs(gpu, ora, wl, seqs=None):
+    """Element-wise output check of every head of the sequences whose
+    selections agree; returns (max abs err, sequences compared)."""
+    worst, n = 0.0, 0
+    for b in (range(wl.batch) if seqs is None else seqs):
+        if tok_selection(gpu, b) != tok_selection(ora, b):
+            continue
+        err = np.abs(gpu["out"][b] - ora["out"][b])
+        bad = err > ATOL + RTOL * np.abs(ora["out"][b])
+        assert not bad.any(), (b, float(err.max()))
+        fin = np.isfinite(ora["lse"][b])
+        assert np.array_equal(fin, np.isfinite(gpu["lse"][b])), b
+        assert (np.abs(gpu["lse"][b][fin] - ora["lse"][b][fin]) <=
+                ATOL + RTOL * np.abs(ora["lse"][b][fin])).all(), b
+        worst = max(worst, float(err.max()))
+        n += 1
+    return worst, n
+
+
+def safe_top_p_tok(wl, lo=0.5, hi=0.99, margin=2e-5, **kw):
+    """Per-sequence p at least `margin` from every cumulative residual mass."""
+    scores = oracle_tok_scores(wl, **kw)
+    kmin, sink, rec = _tok_sel(wl.spec, kw.get("kmin"), kw.get("sink"), kw.get("rec"))
+    lens = wl.seq_lens.cpu().numpy()
+    ps = []
+    for b in range(wl.batch):
+        _, res = _reserved_residual(int(lens[b]), wl.spec.sel_block, sink, rec)
+        cums = [lo, hi]
+        if res:
+            s = np.array([scores[b, j] for j in res])
             order = sorted(range(len(res)), key=lambda i: (-s[i], res[i]))
             e = np.exp(s - s.max())
             e /= e.sum()

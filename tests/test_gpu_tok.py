@@ -1,0 +1,164 @@
+"""GPU parity of the token-level, layer-shared selector path (per-token keys
+of 4 index heads x 128, blocks of 16 tokens scored by their maximum token
+score, one selection per sequence shared by every head) through the C ABI,
+against the fp64 oracle.  Rules and tolerances: tests/harness.py."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_spot_b200 as spot
+import workloads
+from harness import (check_tok_outputs, check_tok_selection_near_cut, oracle_tok_scores,
+                     run_gpu_tok, run_oracle_tok, safe_top_p_tok, tok_oracle_args,
+                     tok_selection)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _same(gpu, ora, wl):
+    assert np.array_equal(gpu["sel_cnt"], ora["sel_cnt"]), (gpu["sel_cnt"], ora["sel_cnt"])
+    for b in range(wl.batch):
+        assert tok_selection(gpu, b) == tok_selection(ora, b), b
+
+
+@pytest.mark.parametrize("kmin", [32, 0])
+def test_tok_tiny_decode_step(kmin):
+    wl = workloads.make_tok("tok_tiny_2k", seed=0, device=DEV)
+    gpu = run_gpu_tok(wl, kmin=kmin)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl)
+    ora = run_oracle_tok(wl, args=args, kmin=kmin)
+    scores = oracle_tok_scores(wl, args=args)
+    assert check_tok_selection_near_cut(gpu, ora, scores, wl, kmin=kmin) == 0
+    _, n = check_tok_outputs(gpu, ora, wl)
+    assert n == wl.batch
+
+
+INTEGER = [
+    ("tok_tiny_2k", dict()),
+    ("tok_tiny_2k", dict(batch=5, seq_len=None, ragged_range=(16, 4096))),
+    ("qwen3_8b_128k_tok", dict(seq_len=16384, batch=3)),
+]
+
+
+@pytest.mark.parametrize("name,kw", INTEGER)
+def test_tok_integer_inputs_select_bit_exact(name, kw):
+    # Selector queries and keys in {-3..3}, uniform weights: every token and
+    # block score is exact in fp32 and fp64, so the selections must match.
+    wl = workloads.make_tok(name, seed=5, device=DEV, integer=True, **kw)
+    wl.top_p = safe_top_p_tok(wl)
+    gpu = run_gpu_tok(wl)
+    assert gpu["status"] == 0
+    ora = run_oracle_tok(wl)
+    _same(gpu, ora, wl)
+    check_tok_outputs(gpu, ora, wl)
+
+
+def test_tok_topk_and_reserved_modes():
+    wl = workloads.make_tok("tok_tiny_2k", seed=6, device=DEV, integer=True, batch=3,
+                            seq_len=None, ragged_range=(64, 2048))
+    for kw in (dict(mode="topk", topk=10), dict(mode="topk", topk=0, sink=0, rec=1),
+               dict(kmin=200), dict(sink=300, rec=0)):
+        gpu = run_gpu_tok(wl, **kw)
+        assert gpu["status"] == 0
+        ora = run_oracle_tok(wl, **kw)
+        _same(gpu, ora, wl)
+        check_tok_outputs(gpu, ora, wl)
+
+
+def test_tok_ragged_partial_blocks_and_empty_sequences():
+    wl = workloads.make_tok("tok_tiny_2k", seed=7, device=DEV, batch=7, seq_len=None,
+                            ragged_range=(2048, 2048))
+    lens = torch.tensor([0, 1, 15, 16, 17, 16 * 37 + 9, 2048], dtype=torch.int32)
+    wl.seq_lens = lens.to(DEV)
+    gpu = run_gpu_tok(wl)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl)
+    ora = run_oracle_tok(wl, args=args)
+    scores = oracle_tok_scores(wl, args=args)
+    assert check_tok_selection_near_cut(gpu, ora, scores, wl) <= 1
+    check_tok_outputs(gpu, ora, wl)
+    assert gpu["sel_cnt"][0] == 0 and np.all(gpu["out"][0] == 0)
+    assert np.all(np.isneginf(gpu["lse"][0]))
+
+
+@pytest.mark.parametrize("batch,seq_len", [(1, 131072), (2, None)])
+def test_tok_full_size(batch, seq_len):
+    """Qwen3-8B layer at 128K (and two ragged sequences): the selection of
+    every sequence checked on the oracle's scores, every head's attention
+    output against the oracle."""
+    kw = dict(batch=batch)
+    if seq_len is None:
+        kw.update(seq_len=None, ragged_range=(60000, 131072))
+    wl = workloads.make_tok("qwen3_8b_128k_tok", seed=1, device=DEV, **kw)
+    gpu = run_gpu_tok(wl)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl)
+    ora = run_oracle_tok(wl, args=args)
+    scores = oracle_tok_scores(wl, args=args)
+    n_diff = check_tok_selection_near_cut(gpu, ora, scores, wl)
+    assert n_diff <= 1
+    frac = gpu["sel_cnt"] / np.maximum(1, (wl.seq_lens.cpu().numpy() + 15) // 16)
+    print(f"|S|/nb {frac.tolist()}, near-cut differences {n_diff}")
+    _, n = check_tok_outputs(gpu, ora, wl)
+    assert n >= wl.batch - n_diff
+
+
+def test_tok_append_writes_the_pool():
+    wl = workloads.make_tok("tok_tiny_2k", seed=8, device=DEV, batch=3, seq_len=None,
+                            ragged_range=(100, 2048))
+    desc = spot.tok_layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages)
+    pool = spot.tok_selector_pool(wl.num_pages, device=DEV)
+    lens = wl.seq_lens.cpu().numpy()
+    pt = wl.page_table.cpu().numpy()
+    seq_ids = np.concatenate([np.full(lens[b], b) for b in range(wl.batch)]).astype(np.int32)
+    pos = np.concatenate([np.arange(lens[b]) for b in range(wl.batch)]).astype(np.int32)
+    perm = np.random.default_rng(0).permutation(seq_ids.size)
+    seq_ids, pos = seq_ids[perm], pos[perm]
+    pages = pt[seq_ids, pos // 64]
+    keys = wl.sel_tok[torch.as_tensor(pages).long().to(DEV), torch.as_tensor(pos % 64).long().to(DEV)]
+    ws = spot.new_tok_workspace(desc, wl.batch, wl.max_blocks, DEV)
+    spot.tok_append_selector_keys(desc, pool, wl.page_table, torch.as_tensor(seq_ids).to(DEV),
+                                  torch.as_tensor(pos).to(DEV), keys.contiguous(), ws)
+    torch.cuda.synchronize()
+    assert spot.read_device_status(ws) == 0
+    written = torch.zeros(wl.num_pages, 64, dtype=torch.bool)
+    written[torch.as_tensor(pages).long(), torch.as_tensor(pos % 64).long()] = True
+    a = pool.cpu().view(torch.int16)
+    b = wl.sel_tok.cpu().view(torch.int16)
+    assert torch.equal(a[written], b[written])
+    assert (a[~written] == 0).all()
+    # a bad position / sequence is skipped and reported
+    bad = torch.tensor([wl.batch, 0], dtype=torch.int32, device=DEV)
+    badpos = torch.tensor([0, 64 * wl.max_pages], dtype=torch.int32, device=DEV)
+    spot.tok_append_selector_keys(desc, pool, wl.page_table, bad, badpos, keys[:2].contiguous(),
+                                  ws)
+    torch.cuda.synchronize()
+    assert spot.read_device_status(ws) == 5              # SPOT_ERR_DEVICE_BOUNDS
+    assert torch.equal(pool.cpu().view(torch.int16)[written], b[written])
+
+
+def test_tok_bad_selection_is_reported_not_faulted():
+    wl = workloads.make_tok("tok_tiny_2k", seed=9, device=DEV)
+    desc = spot.tok_layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages)
+    ws = spot.new_tok_workspace(desc, 1, wl.max_blocks, DEV)
+    sel_idx = torch.tensor([[0, 5, 10_000, 7] + [-1] * (wl.max_blocks - 4)], dtype=torch.int32,
+                           device=DEV)
+    sel_cnt = torch.tensor([4], dtype=torch.int32, device=DEV)
+    out = torch.empty(1, wl.num_q_heads, 128, dtype=torch.float32, device=DEV)
+    spot.tok_sparse_decode(desc, wl.q, wl.k_pool, wl.v_pool, wl.page_table, wl.seq_lens,
+                           sel_idx, sel_cnt, wl.sm_scale, out, None, ws)
+    torch.cuda.synchronize()
+    assert spot.read_device_status(ws) == 5
+    assert torch.isfinite(out).all()
