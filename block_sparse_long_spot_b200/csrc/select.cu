@@ -18,8 +18,9 @@
 // Selection: residual softmax numerators exp(s - max) are computed in fp64
 //   and held as 2^-40 fixed-point integers (exact, order-independent sums).
 //   The nucleus cut is a bucketed threshold search: the residual blocks are
-//   histogrammed into 1024 buckets of the score's distance from the maximum
-//   (monotone in the score; exact counts, 2^-18 fixed-point masses), the
+//   histogrammed into 4096 buckets of the score's distance from the maximum,
+//   scaled so the residual range spans them all (monotone in the score;
+//   exact counts, 2^-18 fixed-point masses), the
 //   bucket where the cumulative mass from the top reaches p * Z is found by a
 //   block scan and confirmed on the exact fixed-point masses, and the few
 //   blocks inside that bucket are ranked exactly (score descending, lower
@@ -348,8 +349,9 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-constexpr int kNB = 1024;              // value buckets of the first pass
-constexpr float kBucketScale = 32.f;    // buckets per unit of score below the maximum
+constexpr int kNB = 4096;              // most value buckets of the first pass (1024 up to
+                                        // 2048 residual blocks, 2048 up to 4096, then 4096),
+                                        // spread over the residual scores' range
 constexpr int kApproxShift = 18;        // bucket masses for the search: 2^-18 fixed point
                                         // (<= 8192 elements of mass <= 1 fit in 32 bits)
 constexpr int NT = kSelectThreads;
@@ -420,11 +422,11 @@ __device__ __forceinline__ float block_exclusive_scan_f(const SelSmem& sm, float
 // approximate fp32 masses (the caller corrects the result exactly), else the
 // exact counts.  Returns the bucket; *before receives the exact count of
 // elements in the buckets above it (count mode only).
-__device__ int cut_bucket(const SelSmem& sm, double target, bool by_mass, int* before) {
-    constexpr int PER = kNB / NT;
+__device__ int cut_bucket(const SelSmem& sm, double target, bool by_mass, int* before,
+                          int nbk) {
+    const int PER = nbk / NT;
     float loc = 0.f;
     int cnt = 0, last = -1;
-#pragma unroll
     for (int k = 0; k < PER; ++k) {
         const int bkt = threadIdx.x * PER + k;
         loc += static_cast<float>(by_mass ? sm.hmass[bkt] : sm.hcnt[bkt]);
@@ -470,6 +472,33 @@ struct Cut {
     int kept_in_bucket;    // elements kept from the bucket itself
 };
 
+// Appends element i (when `hit`) to the candidate list (sm.ckey / sm.cidx,
+// length sm.misc[3]) with one shared atomic per warp.  Every lane of the
+// warp must call it.
+__device__ __forceinline__ void push_candidate(const SelSmem& sm, bool hit, int i) {
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (m == 0u) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(&sm.misc[3], __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (hit) {
+        const int slot = base + __popc(m & ((1u << lane) - 1u));
+        sm.ckey[slot] = sm.keys[i];
+        sm.cidx[slot] = i;
+    }
+}
+
+// Collects the elements of bucket b as candidates (warp-uniform loop).
+__device__ __forceinline__ void gather_bucket(const SelSmem& sm, int n, int b) {
+    const int lane = threadIdx.x & 31;
+    for (int i0 = threadIdx.x - lane; i0 < n; i0 += NT) {
+        const int i = i0 + lane;
+        push_candidate(sm, i < n && sm.vb[i] == b, i);
+    }
+}
+
 // Exact resolution inside bucket b: keeps the shortest prefix (ranked by
 // score, lower block index first) whose cumulative mass (or count) added to
 // `above` reaches `target`; writes the keep flags of the bucket's elements.
@@ -480,13 +509,7 @@ __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long lon
     // `gathered`, already collected the bucket's candidates behind a barrier)
     if (c <= 32) {
         if (!gathered) {
-            for (int i = threadIdx.x; i < n; i += NT) {
-                if (sm.vb[i] == b) {
-                    const int slot = atomicAdd(&sm.misc[3], 1);
-                    sm.ckey[slot] = sm.keys[i];
-                    sm.cidx[slot] = i;
-                }
-            }
+            gather_bucket(sm, n, b);
             __syncthreads();
         }
         if (threadIdx.x < 32) {                       // one warp ranks the few candidates
@@ -520,13 +543,7 @@ __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long lon
     }
     if (threadIdx.x == 0) sm.misc[4] = c - 1;
     if (c <= NT) {
-        for (int i = threadIdx.x; i < n; i += NT) {
-            if (sm.vb[i] == b) {
-                const int slot = atomicAdd(&sm.misc[3], 1);
-                sm.ckey[slot] = sm.keys[i];
-                sm.cidx[slot] = i;
-            }
-        }
+        gather_bucket(sm, n, b);
         __syncthreads();
         int rank = 0;
         if (threadIdx.x < c) {
@@ -671,7 +688,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     const int n = r1 - r0;
     const int n_reserved = nb - n;
     const float* s = sm.score;
-    for (int i = threadIdx.x; i < kNB; i += NT) { sm.hmass[i] = 0u; sm.hcnt[i] = 0u; }
+    const int nbk = n > 4096 ? 4096 : (n > 2048 ? 2048 : 1024);     // value buckets
+    for (int i = threadIdx.x; i < nbk; i += NT) { sm.hmass[i] = 0u; sm.hcnt[i] = 0u; }
     if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
     pdl_trigger();                                    // the decode kernel may start its prologue
 
@@ -679,7 +697,18 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     if constexpr (FMT == kSelectFromScores) {
         pdl_wait();                                   // block scores of the scoring kernel
         const float* src = p.scores_in + static_cast<int64_t>(u) * p.max_blocks;
-        for (int j = threadIdx.x; j < n_full; j += NT) sm.score[j] = src[j];
+        constexpr int kBatch = 8;                     // loads in flight per thread
+        for (int j0 = threadIdx.x; j0 < n_full; j0 += NT * kBatch) {
+            float v[kBatch];
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const int j = j0 + k * NT;
+                v[k] = j < n_full ? __ldcg(src + j) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k)
+                if (j0 + k * NT < n_full) sm.score[j0 + k * NT] = v[k];
+        }
     } else {
         const int g = u - b * p.num_kv_heads;
         uint32_t qw[8];
@@ -700,34 +729,63 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     }
     __syncthreads();
 
-    // ---- residual scores -> keys, maximum
-    float mloc = -INFINITY;
+    // ---- residual scores -> keys, maximum and minimum
+    float mloc = -INFINITY, nloc = INFINITY;
     for (int i = threadIdx.x; i < n; i += NT) {
         const float v = s[r0 + i];
         sm.keys[i] = score_key(v);
         mloc = fmaxf(mloc, v);
+        nloc = fminf(nloc, v);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
-    if (lane == 0) sm.fscan[warp] = mloc;
+    for (int o = 16; o > 0; o >>= 1) {
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+        nloc = fminf(nloc, __shfl_xor_sync(0xffffffffu, nloc, o));
+    }
+    float* wmin = reinterpret_cast<float*>(sm.scan);  // next written after two barriers
+    if (lane == 0) {
+        sm.fscan[warp] = mloc;
+        wmin[warp] = nloc;
+    }
     __syncthreads();
-    float smax_f = -INFINITY;
-    for (int w = 0; w < NW; ++w) smax_f = fmaxf(smax_f, sm.fscan[w]);
+    float smax_f = -INFINITY, smin_f = INFINITY;
+    for (int w = 0; w < NW; ++w) {
+        smax_f = fmaxf(smax_f, sm.fscan[w]);
+        smin_f = fminf(smin_f, wmin[w]);
+    }
     const double smax = static_cast<double>(smax_f);
+    // buckets per unit of score: the residual range spans all nbk buckets,
+    // up to 40 below the maximum (exp(-40) is below the fixed point's 2^-40;
+    // anything lower shares the last bucket)
+    const float range = fminf(smax_f - smin_f, 40.f);
+    const float bscale = range > 1e-30f ? static_cast<float>(nbk - 1) / range : 1.f;
 
     // ---- exact fixed-point numerators exp(s - max), their total Z, value
     // buckets (monotone in the score) with exact counts and fp32 masses
     unsigned long long zloc = 0;
-    for (int i = threadIdx.x; i < n; i += NT) {
-        const float v = s[r0 + i];
-        const double e = exp(static_cast<double>(v) - smax);
-        const unsigned long long f = __double2ull_rn(ldexp(e, kFixShift));
-        sm.mass[i] = f;
-        const int bkt = static_cast<int>(fminf((smax_f - v) * kBucketScale, kNB - 1.f));
-        sm.vb[i] = static_cast<uint16_t>(bkt);
-        atomicAdd(&sm.hcnt[bkt], 1u);
-        atomicAdd(&sm.hmass[bkt], static_cast<uint32_t>(ldexp(e, kApproxShift) + 0.5));
-        zloc += f;
+    constexpr int kUnroll = 4;                        // independent exps in flight
+    for (int i0 = threadIdx.x; i0 < n; i0 += kUnroll * NT) {
+        float v[kUnroll];
+        double e[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const int i = i0 + k * NT;
+            v[k] = i < n ? s[r0 + i] : smax_f;
+        }
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) e[k] = exp(static_cast<double>(v[k]) - smax);
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const int i = i0 + k * NT;
+            if (i >= n) break;
+            const unsigned long long f = __double2ull_rn(ldexp(e[k], kFixShift));
+            sm.mass[i] = f;
+            const int bkt = static_cast<int>(fminf((smax_f - v[k]) * bscale, nbk - 1.f));
+            sm.vb[i] = static_cast<uint16_t>(bkt);
+            atomicAdd(&sm.hcnt[bkt], 1u);
+            atomicAdd(&sm.hmass[bkt], static_cast<uint32_t>(ldexp(e[k], kApproxShift) + 0.5));
+            zloc += f;
+        }
     }
     unsigned long long Z = zloc, d1 = 0, d2 = 0;
     block_sum3(sm, Z, d1, d2);
@@ -750,7 +808,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
         int before;
         if (threadIdx.x == 0) sm.misc[3] = 0;
         int bk = cut_bucket(sm, ldexp(static_cast<double>(T), kApproxShift - kFixShift), true,
-                            &before);
+                            &before, nbk);
         // Exact check of the bucket on the fixed-point masses.  The first
         // pass also writes the keep flags and gathers the bucket's candidates
         // (sm.misc[3] was zeroed before cut_bucket's barriers); if the
@@ -760,33 +818,30 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
         const bool small = sm.hcnt[bk] <= 32u;
         {
             A = 0; Bm = 0; Ac = 0;
-            for (int i = threadIdx.x; i < n; i += NT) {
-                const int v = sm.vb[i];
-                sm.keep[i] = v < bk ? 1 : 0;
-                if (v < bk) {
+            for (int i0 = threadIdx.x - lane; i0 < n; i0 += NT) {   // warp-uniform
+                const int i = i0 + lane;
+                const int v = i < n ? sm.vb[i] : -1;
+                if (i < n) sm.keep[i] = v < bk ? 1 : 0;
+                if (i < n && v < bk) {
                     A += sm.mass[i];
                     ++Ac;
                 } else if (v == bk) {
                     Bm += sm.mass[i];
-                    if (small) {
-                        const int slot = atomicAdd(&sm.misc[3], 1);
-                        sm.ckey[slot] = sm.keys[i];
-                        sm.cidx[slot] = i;
-                    }
                 }
+                if (small) push_candidate(sm, v == bk, i);
             }
             block_sum3(sm, A, Bm, Ac);
         }
         bool gathered = small;
-        for (int guard = 0; guard < kNB; ++guard) {
+        for (int guard = 0; guard < nbk; ++guard) {
             int step = 0;
             if (A >= T) step = -1;
             else if (A + Bm < T) step = 1;
             if (step == 0) break;
-            int nbk = bk + step;
-            while (nbk >= 0 && nbk < kNB && sm.hcnt[nbk] == 0) nbk += step;
-            if (nbk < 0 || nbk >= kNB) break;
-            bk = nbk;
+            int nbk_ = bk + step;
+            while (nbk_ >= 0 && nbk_ < nbk && sm.hcnt[nbk_] == 0) nbk_ += step;
+            if (nbk_ < 0 || nbk_ >= nbk) break;
+            bk = nbk_;
             gathered = false;
             A = 0; Bm = 0; Ac = 0;
             for (int i = threadIdx.x; i < n; i += NT) {
@@ -819,7 +874,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
             __syncthreads();
         } else {
             int before;
-            const int bk = cut_bucket(sm, static_cast<double>(n_take), false, &before);
+            const int bk = cut_bucket(sm, static_cast<double>(n_take), false, &before, nbk);
             if (threadIdx.x == 0) sm.misc[3] = 0;
             for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
             __syncthreads();
@@ -829,34 +884,50 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     }
     const uint32_t take = static_cast<uint32_t>(sm.misc[5]);
 
-    // ---- compaction: each thread owns a contiguous run of block ids; one
-    // block scan of (ties at a key cut << 16 | other kept blocks)
-    const int per = (nb + NT - 1) / NT;
-    const int lo = min(nb, static_cast<int>(threadIdx.x) * per), hi = min(nb, lo + per);
-    int ties = 0, kept = 0;
-    for (int j = lo; j < hi; ++j) {
-        if (j < r0 || j >= r1) { ++kept; continue; }
-        const int f = sm.keep[j - r0];
-        kept += f == 1;
-        ties += f == 2;
+    // ---- compaction: warp w owns a contiguous run of block ids and takes 32
+    // consecutive ids per step; ballots count and place the kept ones
+    // (reserved blocks, flag 1, and the first `take` ties at a key cut, flag
+    // 2, in block order).  The list is assembled in shared memory (over the
+    // keys, no longer needed) and written out with coalesced stores.
+    const int per_w = ((nb + NW - 1) / NW + 31) & ~31;
+    const int wlo = min(nb, warp * per_w), whi = min(nb, wlo + per_w);
+    const unsigned lt = (1u << lane) - 1u;
+    int wk = 0, wt = 0;
+    for (int j0 = wlo; j0 < whi; j0 += 32) {
+        const int j = j0 + lane;
+        const int f = j >= whi ? 0 : ((j < r0 || j >= r1) ? 1 : sm.keep[j - r0]);
+        wk += __popc(__ballot_sync(0xffffffffu, f == 1));
+        wt += __popc(__ballot_sync(0xffffffffu, f == 2));
     }
-    int total;
-    const int before = block_exclusive_scan<NT>((ties << 16) | kept, sm.scan, &total);
-    uint32_t tie_rank = static_cast<uint32_t>(before >> 16);
-    int out_pos = (before & 0xFFFF) + static_cast<int>(min(tie_rank, take));
+    if (lane == 0) {
+        sm.scan[warp] = wk;
+        reinterpret_cast<int*>(sm.red)[warp] = wt;
+    }
+    __syncthreads();
+    int kb = 0, tb = 0, ktot = 0, ttot = 0;
+    for (int w = 0; w < NW; ++w) {
+        const int a = sm.scan[w], t = reinterpret_cast<int*>(sm.red)[w];
+        if (w < warp) { kb += a; tb += t; }
+        ktot += a;
+        ttot += t;
+    }
+    int* list = reinterpret_cast<int*>(sm.keys);
+    int pos = kb + min(tb, static_cast<int>(take)), tr = tb;
+    for (int j0 = wlo; j0 < whi; j0 += 32) {
+        const int j = j0 + lane;
+        const int f = j >= whi ? 0 : ((j < r0 || j >= r1) ? 1 : sm.keep[j - r0]);
+        const unsigned tbal = __ballot_sync(0xffffffffu, f == 2);
+        const bool keep = f == 1 || (f == 2 && static_cast<uint32_t>(tr + __popc(tbal & lt)) < take);
+        const unsigned kbal = __ballot_sync(0xffffffffu, keep);
+        if (keep) list[pos + __popc(kbal & lt)] = j;
+        pos += __popc(kbal);
+        tr += __popc(tbal);
+    }
+    const int cnt = ktot + min(ttot, static_cast<int>(take));
+    __syncthreads();
     int32_t* out = p.sel_idx + static_cast<int64_t>(u) * p.max_blocks;
-    for (int j = lo; j < hi; ++j) {
-        bool keep;
-        if (j < r0 || j >= r1) {
-            keep = true;
-        } else {
-            const int f = sm.keep[j - r0];
-            keep = f == 1 || (f == 2 && tie_rank++ < take);
-        }
-        if (keep) out[out_pos++] = j;
-    }
-    if (threadIdx.x == 0)
-        p.sel_cnt[u] = (total & 0xFFFF) + static_cast<int>(min(static_cast<uint32_t>(total >> 16), take));
+    for (int i = threadIdx.x; i < cnt; i += NT) out[i] = list[i];
+    if (threadIdx.x == 0) p.sel_cnt[u] = cnt;
 }
 
 }  // namespace

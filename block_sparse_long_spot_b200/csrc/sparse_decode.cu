@@ -43,6 +43,10 @@ namespace {
 
 constexpr int NC = kDecodeConsumers;
 constexpr int STAGES = kDecodeStages;
+// Each stage must always be consumed by the same warp: a warp waiting on a
+// stage's full barrier can then only be one round ahead of it, which is all
+// a parity wait can tell apart.
+static_assert(STAGES % NC == 0, "stage count must be a multiple of the consumer count");
 constexpr int kThreads = (NC + 1) * 32;
 constexpr int kHalfTile = kBlock * 64 * 2;   // 8 KiB: 64 rows x 64 bf16
 
@@ -80,73 +84,76 @@ __device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
     return static_cast<int>(((pos + 1) * P - 1) / N);
 }
 
-// Merge the partials of query head n of unit u (blocks [lo, hi) of the
-// flattened list) and write out / lse.  One warp; lane l owns head
-// dimensions 4l..4l+3.  The partials are one per CTA whose range touched the
-// unit; other CTAs of this launch wrote them, so they are read through L2
-// (ld.global.cg).  Slots are taken 32 at a time with an online rescale, and
-// the accumulator loads of 8 slots are issued together.
-__device__ void merge_unit_head(const DecodeParams& p, int u, int n, int lo, int hi, int64_t N,
-                                int64_t P, int lane) {
+// Merge the partials of unit u (blocks [lo, hi) of the flattened list) and
+// write out / lse of its G heads, with all NC consumer warps (tid < NC*32).
+// The partials are one per CTA whose range touched the unit; other CTAs of
+// this launch wrote them, so they are read through L2 (ld.global.cg).  First
+// the (m, l) of every slot and head go to shared memory (ml, at least
+// nslots * G * 2 floats: every load in flight at once), then each thread
+// takes (head, 4 dims) items and combines the slots' accumulators with their
+// log-sum-exp weights, kMergeBatch slots' loads in flight per step.
+constexpr int kMergeBatch = 8;           // slot loads in flight per thread and step
+
+__device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t N, int64_t P,
+                           float* ml, int tid) {
+    constexpr int T = NC * 32;
     const int G = p.group;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
-    const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
     const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
     const int nslots = i1 - i0 + 1;
     const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
     const bool some_idle = N < P;          // only then can a CTA own no blocks
-    float M = -INFINITY, L = 0.f;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int base = 0; base < nslots; base += 32) {
-        const int i = i0 + base + lane;
+    for (int t = tid; t < nslots * G; t += T) {
+        const int k = t / G, n = t - k * G;
+        const int i = i0 + k;
         float m = -INFINITY, l = 0.f;
-        if (base + lane < nslots &&
-            !(some_idle && range_begin(N, P, i) == range_begin(N, P, i + 1))) {
+        if (!(some_idle && range_begin(N, P, i) == range_begin(N, P, i + 1))) {
             const float* sl = p.partials + static_cast<int64_t>(i + u) * stride;
             m = __ldcg(sl + G * kHeadDim + n);
             l = __ldcg(sl + G * (kHeadDim + 1) + n);
         }
-        float cm = m;
+        ml[2 * t] = m;
+        ml[2 * t + 1] = l;
+    }
+    consumer_barrier();
+    for (int item = tid; item < G * (kHeadDim / 4); item += T) {
+        const int n = item / (kHeadDim / 4), d4 = item - n * (kHeadDim / 4);
+        float M = -INFINITY;
+        for (int k = 0; k < nslots; ++k) M = fmaxf(M, ml[2 * (k * G + n)]);
+        float L = 0.f;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY) {
+            for (int k0 = 0; k0 < nslots; k0 += kMergeBatch) {
+                float wk[kMergeBatch];
+                float4 v[kMergeBatch];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
-        const float nm = fmaxf(M, cm);
-        if (nm == -INFINITY) continue;
-        const float sc = (M == -INFINITY) ? 0.f : exp2f(M - nm);
-        L *= sc;
-        a.x *= sc; a.y *= sc; a.z *= sc; a.w *= sc;
-        M = nm;
-        const float wgt = (m == -INFINITY) ? 0.f : exp2f(m - M);
-        float wl = wgt * l;
+                for (int k = 0; k < kMergeBatch; ++k) {
+                    const float m = k0 + k < nslots ? ml[2 * ((k0 + k) * G + n)] : -INFINITY;
+                    wk[k] = (m == -INFINITY) ? 0.f : exp2f(m - M);
+                    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (wk[k] != 0.f)
+                        v[k] = __ldcg(reinterpret_cast<const float4*>(
+                                          p.partials + static_cast<int64_t>(i0 + k0 + k + u) *
+                                                           stride + n * kHeadDim) + d4);
+                }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, off);
-        L += wl;
-        const int cnt = min(32, nslots - base);
-        for (int k0 = 0; k0 < cnt; k0 += 8) {
-            float wk[8];
-            float4 v[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                wk[k] = __shfl_sync(0xffffffffu, wgt, (k0 + k) & 31);
-                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (k0 + k < cnt && wk[k] != 0.f)
-                    v[k] = __ldcg(reinterpret_cast<const float4*>(
-                                      p.partials + static_cast<int64_t>(i0 + base + k0 + k + u) *
-                                                       stride + n * kHeadDim) + lane);
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                a.x = fmaf(wk[k], v[k].x, a.x);
-                a.y = fmaf(wk[k], v[k].y, a.y);
-                a.z = fmaf(wk[k], v[k].z, a.z);
-                a.w = fmaf(wk[k], v[k].w, a.w);
+                for (int k = 0; k < kMergeBatch; ++k) {
+                    if (wk[k] != 0.f) L = fmaf(wk[k], ml[2 * ((k0 + k) * G + n) + 1], L);
+                    a.x = fmaf(wk[k], v[k].x, a.x);
+                    a.y = fmaf(wk[k], v[k].y, a.y);
+                    a.z = fmaf(wk[k], v[k].z, a.z);
+                    a.w = fmaf(wk[k], v[k].w, a.w);
+                }
             }
         }
+        const bool empty = !(L > 0.f);    // only if every tile was rejected as out of range
+        const float inv = empty ? 0.f : 1.f / L;
+        const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
+        reinterpret_cast<float4*>(p.out + h * kHeadDim)[d4] =
+            make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+        if (p.lse && d4 == 0) p.lse[h] = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
     }
-    const bool empty = !(L > 0.f);        // only if every tile was rejected as out of range
-    const float inv = empty ? 0.f : 1.f / L;
-    reinterpret_cast<float4*>(p.out + h * kHeadDim)[lane] =
-        make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
-    if (p.lse && lane == 0) p.lse[h] = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+    consumer_barrier();                   // ml (shared scratch) is free again
 }
 
 // Valid tokens of the four 16-row slices of a 64-row tile, one byte each.
@@ -564,8 +571,8 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
         consumer_barrier();
         if (flags[1]) {
             __threadfence();
-            for (int n = warp; n < G; n += NC)
-                merge_unit_head(p, u, n, unit_off[u], unit_off[u + 1], N, P, lane);
+            // red_acc is free again: the CTA's partial has been written
+            merge_unit(p, u, unit_off[u], unit_off[u + 1], N, P, red_acc, threadIdx.x);
         }
         pos = seg_end;
     }
@@ -624,7 +631,9 @@ int decode_grid(int units) {
                                                       kThreads, smem) != cudaSuccess)
         return 0;
     m.units = units;
-    m.grid = sms * max(per_sm, 1);
+    // the merge keeps (m, l) of up to `grid` slots x 8 heads in red_acc
+    constexpr int kMaxGrid = NC * kMaxGroup * kPartialFloatsPerHead / (2 * kMaxGroup);
+    m.grid = min(sms * max(per_sm, 1), kMaxGrid);
     return m.grid;
 }
 
