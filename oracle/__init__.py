@@ -84,6 +84,11 @@ def _load():
         lib.oracle_tok_block_scores.argtypes = [P, P, P, P, P, P, P, P]
         lib.oracle_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
                                                P, P, P, P, P]
+        lib.oracle_prefill_num_tiles.argtypes = [P, P, P]
+        lib.oracle_prefill_num_tiles.restype = i64
+        lib.oracle_prefill_scores.argtypes = [P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_prefill_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
+                                            P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -264,3 +269,64 @@ def tok_decode_step(shape: TokShape, params: Params, q_idx, w, sel_tok, q, k_poo
         _ptr(lse))
     assert rc == 0
     return {"sel_idx": sel_idx, "sel_cnt": sel_cnt, "nuc_mass": mass, "out": out, "lse": lse}
+
+
+# ---------------------------------------------------------------------------
+# Sparse prefill (§2.3 applied to a chunk of queries; tiles of one KV block)
+
+def prefill_tiles(seq_lens, q_lens, block_size=64):
+    """(b, first position, last position, first row) of every query tile."""
+    out, row = [], 0
+    for b, (L, T) in enumerate(zip(np.asarray(seq_lens).tolist(), np.asarray(q_lens).tolist())):
+        if T <= 0:
+            continue
+        q0 = L - T
+        for m in range(q0 // block_size, (L - 1) // block_size + 1):
+            lo, hi = max(q0, m * block_size), min(L - 1, m * block_size + block_size - 1)
+            out.append((b, lo, hi, row + lo - q0))
+        row += T
+    return out
+
+
+def prefill_scores(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, page_table,
+                   seq_lens, q_lens) -> np.ndarray:
+    """Block scores [tiles, Hkv, max_blocks] of every query tile (max over
+    the tile's queries; NaN where no complete block)."""
+    lens, ql = _c(seq_lens, np.int32), _c(q_lens, np.int32)
+    nt = int(_load().oracle_prefill_num_tiles(ctypes.byref(shape), _ptr(lens), _ptr(ql)))
+    scores = np.full((max(nt, 1), shape.num_kv_heads, shape.max_blocks), np.nan)
+    fmt = shape.sel_fmt
+    rc = _load().oracle_prefill_scores(
+        ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_sel, np.uint16)),
+        _ptr(_c(w, np.float32)), _ptr(_c(sel_data, _data_dtype(_FMT_NAME[fmt]))),
+        _ptr(_c(sel_scales, _scale_dtype(_FMT_NAME[fmt]))), _ptr(_c(page_table, np.int32)),
+        _ptr(lens), _ptr(ql), _ptr(scores))
+    assert rc == 0
+    return scores[:nt]
+
+
+def prefill_step(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, q, k_pool, v_pool,
+                 page_table, seq_lens, q_lens, top_p, sm_scale, tiles=None):
+    """Sparse prefill of the chunks' query rows (packed [rows, Hq, ...]):
+    selection per (tile, KV head) and causal attention over it.  `tiles`
+    restricts the work to some tiles (their rows of out / lse are filled)."""
+    lens, ql = _c(seq_lens, np.int32), _c(q_lens, np.int32)
+    nt = int(_load().oracle_prefill_num_tiles(ctypes.byref(shape), _ptr(lens), _ptr(ql)))
+    rows = int(np.maximum(ql, 0).sum())
+    Hkv, Hq = shape.num_kv_heads, shape.num_q_heads
+    sel_idx = np.full((max(nt, 1), Hkv, max(shape.max_blocks, 1)), -1, np.int32)
+    sel_cnt = np.zeros((max(nt, 1), Hkv), np.int32)
+    out = np.zeros((max(rows, 1), Hq, shape.head_dim))
+    lse = np.zeros((max(rows, 1), Hq))
+    fmt = shape.sel_fmt
+    tl = None if tiles is None else _c(tiles, np.int32)
+    rc = _load().oracle_prefill_step(
+        ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_sel, np.uint16)),
+        _ptr(_c(w, np.float32)), _ptr(_c(sel_data, _data_dtype(_FMT_NAME[fmt]))),
+        _ptr(_c(sel_scales, _scale_dtype(_FMT_NAME[fmt]))), _ptr(_c(q, np.uint16)),
+        _ptr(_c(k_pool, np.uint16)), _ptr(_c(v_pool, np.uint16)), _ptr(_c(page_table, np.int32)),
+        _ptr(lens), _ptr(ql), _ptr(_c(top_p, np.float32)), float(sm_scale), _ptr(tl),
+        0 if tl is None else len(tl), _ptr(sel_idx), _ptr(sel_cnt), _ptr(out), _ptr(lse))
+    assert rc == 0
+    return {"sel_idx": sel_idx[:nt], "sel_cnt": sel_cnt[:nt], "out": out[:rows], "lse": lse[:rows],
+            "tiles": prefill_tiles(lens, ql, shape.block_size)}

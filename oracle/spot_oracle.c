@@ -618,6 +618,198 @@ int oracle_decode_step(const orc_shape_t* sh, const orc_params_t* pr, const uint
 }
 
 /* ------------------------------------------------------------------ */
+/* Sparse prefill (§2.3 applied to a chunk of queries).                */
+/* ------------------------------------------------------------------ */
+
+/* Sequence b holds seq_lens[b] tokens in the cache; its last q_lens[b] are
+ * the chunk's queries, packed as rows q_off(b) .. q_off(b) + q_lens[b] - 1
+ * of q / q_sel / w / out / lse (q_off = running sum of q_lens).  A query
+ * tile is the set of chunk queries whose positions fall in one KV block m;
+ * tiles are numbered sequence by sequence, m ascending.  Tile (b, m) selects
+ * for each KV head exactly as a decode query at L_eff = 1 + the tile's last
+ * position would (Eq. 6-8, sink / recency / K_min, the incomplete block
+ * kept), from the block scores s[j] = max over the tile's queries of the
+ * query's score (1/tau) sum_h w_h ReLU(q^I_h . k_j) -- the paper's
+ * per-block maximum taken over the query block as well (§2.1: one score per
+ * query-block x key-block tile).  Every query then attends, causally (key
+ * positions <= its own), to the tokens of its tile's selected blocks. */
+
+static int64_t prefill_tiles_of(int32_t seq_len, int32_t q_len, int bs) {
+    if (q_len <= 0) return 0;
+    int32_t q_start = seq_len - q_len;
+    return (int64_t)((seq_len - 1) / bs) - (q_start / bs) + 1;
+}
+
+/* Number of query tiles of the whole batch (the rows of sel_idx / sel_cnt). */
+int64_t oracle_prefill_num_tiles(const orc_shape_t* sh, const int32_t* seq_lens,
+                                 const int32_t* q_lens) {
+    int64_t t = 0;
+    for (int b = 0; b < sh->batch; ++b) t += prefill_tiles_of(seq_lens[b], q_lens[b], sh->block_size);
+    return t;
+}
+
+/* Locate tile `tile`: sequence, first / last query position, first row. */
+static void prefill_tile(const orc_shape_t* sh, const int32_t* seq_lens, const int32_t* q_lens,
+                         int64_t tile, int* b_out, int32_t* p_lo, int32_t* p_hi, int64_t* row0) {
+    int bs = sh->block_size;
+    int64_t t = tile, off = 0;
+    for (int b = 0; b < sh->batch; ++b) {
+        int64_t n = prefill_tiles_of(seq_lens[b], q_lens[b], bs);
+        if (t < n) {
+            int32_t q_start = seq_lens[b] - q_lens[b];
+            int32_t m = q_start / bs + (int32_t)t;
+            *b_out = b;
+            *p_lo = m * bs > q_start ? m * bs : q_start;
+            *p_hi = m * bs + bs - 1 < seq_lens[b] - 1 ? m * bs + bs - 1 : seq_lens[b] - 1;
+            *row0 = off + (*p_lo - q_start);
+            return;
+        }
+        t -= n;
+        off += q_lens[b] > 0 ? q_lens[b] : 0;
+    }
+    *b_out = -1;
+}
+
+/* Scores of tile `tile` for KV head g: s[j], j < floor(L_eff / bs). */
+static int prefill_tile_scores(const orc_shape_t* sh, const orc_params_t* pr,
+                               const uint16_t* q_sel, const float* w, const double* keys_f64,
+                               const int32_t* page_table, int b, int32_t p_lo, int32_t p_hi,
+                               int64_t row0, int g, double* s) {
+    int G = sh->num_q_heads / sh->num_kv_heads, ds = sh->sel_dim;
+    int64_t n_full = (int64_t)(p_hi + 1) / sh->block_size;
+    double* qv = (double*)malloc((size_t)G * ds * sizeof(double));
+    double* tmp = (double*)malloc((size_t)(n_full > 0 ? n_full : 1) * sizeof(double));
+    if (!qv || !tmp) { free(qv); free(tmp); return -2; }
+    for (int64_t j = 0; j < n_full; ++j) s[j] = -INFINITY;
+    /* the query rows are laid out like a batch of rows: row r plays "b = r" */
+    orc_shape_t rs = *sh;
+    rs.max_blocks = sh->max_blocks;
+    for (int32_t pos = p_lo; pos <= p_hi; ++pos) {
+        int64_t r = row0 + (pos - p_lo);
+        if (unit_queries(&rs, pr, (int)r, g, q_sel, qv)) { free(qv); free(tmp); return -1; }
+        for (int64_t j = 0; j < n_full; ++j) {
+            int32_t page = page_table[(int64_t)b * sh->max_blocks + j];
+            const double* k = keys_f64 + ((int64_t)page * sh->num_kv_heads + g) * ds;
+            double sc = 0.0;
+            for (int i = 0; i < G; ++i) {
+                int h = g * G + i;
+                const double* qq = qv + (int64_t)i * ds;
+                double dot = 0.0;
+                for (int d = 0; d < ds; ++d) dot += qq[d] * k[d];
+                double wh = w ? (double)w[r * sh->num_q_heads + h] : 1.0 / G;
+                sc += wh * (dot > 0.0 ? dot : 0.0);
+            }
+            sc /= pr->temperature;
+            if (sc > s[j]) s[j] = sc;
+        }
+    }
+    free(qv);
+    free(tmp);
+    return 0;
+}
+
+/* Block scores of every tile: scores[tile][g][max_blocks] (entries past a
+ * tile's complete blocks untouched). */
+int oracle_prefill_scores(const orc_shape_t* sh, const orc_params_t* pr, const uint16_t* q_sel,
+                          const float* w, const void* sel_data, const void* sel_scales,
+                          const int32_t* page_table, const int32_t* seq_lens,
+                          const int32_t* q_lens, double* scores) {
+    int64_t rows = (int64_t)sh->num_pages * sh->num_kv_heads;
+    double* keys = (double*)malloc((size_t)(rows * sh->sel_dim) * sizeof(double));
+    if (!keys) return -2;
+    if (oracle_dequant_selector(sh->sel_fmt, rows, sh->sel_dim, sel_data, sel_scales, keys)) {
+        free(keys);
+        return -1;
+    }
+    int64_t nt = oracle_prefill_num_tiles(sh, seq_lens, q_lens);
+    int err = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t k = 0; k < nt * sh->num_kv_heads; ++k) {
+        int64_t t = k / sh->num_kv_heads;
+        int g = (int)(k % sh->num_kv_heads);
+        int b;
+        int32_t p_lo, p_hi;
+        int64_t row0;
+        prefill_tile(sh, seq_lens, q_lens, t, &b, &p_lo, &p_hi, &row0);
+        if (prefill_tile_scores(sh, pr, q_sel, w, keys, page_table, b, p_lo, p_hi, row0, g,
+                                scores + (t * sh->num_kv_heads + g) * sh->max_blocks)) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = -2;
+        }
+    }
+    free(keys);
+    return err;
+}
+
+/* The whole sparse-prefill step for tiles `tiles[n_tiles]` (NULL: all):
+ * selection per (tile, KV head) into sel_idx[tile][g][max_blocks] /
+ * sel_cnt[tile][g], and out[row][h][D] / lse[row][h] of the tiles' query
+ * rows (rows of other tiles untouched). */
+int oracle_prefill_step(const orc_shape_t* sh, const orc_params_t* pr, const uint16_t* q_sel,
+                        const float* w, const void* sel_data, const void* sel_scales,
+                        const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                        const int32_t* page_table, const int32_t* seq_lens,
+                        const int32_t* q_lens, const float* top_p, double sm_scale,
+                        const int32_t* tiles, int32_t n_tiles, int32_t* sel_idx,
+                        int32_t* sel_cnt, double* out, double* lse) {
+    int G = sh->num_q_heads / sh->num_kv_heads;
+    int64_t rows = (int64_t)sh->num_pages * sh->num_kv_heads;
+    double* keys = (double*)malloc((size_t)(rows * sh->sel_dim) * sizeof(double));
+    if (!keys) return -2;
+    if (oracle_dequant_selector(sh->sel_fmt, rows, sh->sel_dim, sel_data, sel_scales, keys)) {
+        free(keys);
+        return -1;
+    }
+    int64_t total = tiles ? n_tiles : oracle_prefill_num_tiles(sh, seq_lens, q_lens);
+    int err = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t k = 0; k < total * sh->num_kv_heads; ++k) {
+        int64_t t = tiles ? tiles[k / sh->num_kv_heads] : k / sh->num_kv_heads;
+        int g = (int)(k % sh->num_kv_heads);
+        int b;
+        int32_t p_lo, p_hi;
+        int64_t row0;
+        prefill_tile(sh, seq_lens, q_lens, t, &b, &p_lo, &p_hi, &row0);
+        int32_t L_eff = p_hi + 1;
+        int64_t nb = ceil_div64(L_eff, sh->block_size), n_full = L_eff / sh->block_size;
+        double* s = (double*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(double));
+        if (!s || prefill_tile_scores(sh, pr, q_sel, w, keys, page_table, b, p_lo, p_hi, row0,
+                                      g, s)) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = -2;
+            free(s);
+            continue;
+        }
+        int32_t* sel = sel_idx + (t * sh->num_kv_heads + g) * sh->max_blocks;
+        double mass = 0.0;
+        int32_t cnt = oracle_select_from_scores(s, (int32_t)nb, (int32_t)n_full, pr,
+                                                (double)top_p[b], sel, &mass);
+        sel_cnt[t * sh->num_kv_heads + g] = cnt;
+        for (int32_t pos = p_lo; pos <= p_hi; ++pos) {
+            int64_t r = row0 + (pos - p_lo);
+            attend_blocks(sh->num_q_heads, sh->num_kv_heads, sh->head_dim, sh->block_size,
+                          sh->max_blocks, sh->block_size, 0, g,
+                          q + r * sh->num_q_heads * sh->head_dim, k_pool, v_pool,
+                          page_table + (int64_t)b * sh->max_blocks, pos + 1, sel, cnt, sm_scale,
+                          out + (r * sh->num_q_heads + g * G) * sh->head_dim,
+                          lse + r * sh->num_q_heads + g * G);
+        }
+        (void)n_full;
+        free(s);
+    }
+    free(keys);
+    return err;
+}
+
+/* ------------------------------------------------------------------ */
 /* Token-level, layer-shared selector (SpotAttention §2.1, §2.3 and    */
 /* App. A Tab. 3 as written).                                          */
 /* ------------------------------------------------------------------ */

@@ -667,3 +667,118 @@ def test_tok_reserved_blocks_and_incomplete_last_block():
     s = oracle.tok_block_scores(sh, pr, q_idx, None, sel_tok, pt, np.array([L], np.int32))[0]
     best = sorted(range(2, 9), key=lambda j: (-s[j], j))[:2]           # K_min floor of 6
     assert r2["sel_idx"][0, :r2["sel_cnt"][0]].tolist() == sorted([0, 1, 9, 10] + best)
+
+
+# ------------------------------------------------------------ sparse prefill
+# A chunk's queries are grouped into tiles (queries whose positions share a
+# KV block); each tile selects like a decode query at the tile's last
+# position, from block scores maxed over its queries, and every query
+# attends causally over its tile's selection.
+
+def _prefill_problem(rng, lens, qlens, Hq=4, Hkv=2, fmt="bf16"):
+    B = len(lens)
+    nbs = [(L + 63) // 64 for L in lens]
+    mb = max(nbs)
+    P = sum(nbs)
+    rows = sum(qlens)
+    q_sel = rng.normal(size=(rows, Hq, 64)).astype(np.float32)
+    keys = rng.normal(size=(P, Hkv, 64)).astype(np.float32)
+    (q, k, v), (q64, k64, v64) = _rand_kv(rng, P, Hkv, Hq, rows)
+    perm = rng.permutation(P).astype(np.int32)
+    pt = np.full((B, mb), -1, np.int32)
+    off = 0
+    for b, n in enumerate(nbs):
+        pt[b, :n] = perm[off:off + n]
+        off += n
+    sh = oracle.make_shape(B, Hq, Hkv, 128, 64, 64, fmt, P, mb)
+    return sh, q_sel, keys, (q, k, v), (q64, k64, v64), pt
+
+
+def _prefill(sh, pr, q_sel, keys, qkv, pt, lens, qlens, p, scale=0.1):
+    q, k, v = qkv
+    return oracle.prefill_step(sh, pr, _bf16_bits(q_sel), None, _bf16_bits(keys), None,
+                               _bf16_bits(q), _bf16_bits(k), _bf16_bits(v), pt,
+                               np.array(lens, np.int32), np.array(qlens, np.int32),
+                               np.full(len(lens), p, np.float32), scale)
+
+
+def test_prefill_single_query_chunk_equals_decode():
+    rng = np.random.default_rng(20)
+    lens, qlens = [300, 64, 1000], [1, 1, 1]
+    sh, q_sel, keys, qkv, _, pt = _prefill_problem(rng, lens, qlens)
+    pr = oracle.make_params(sink_blocks=1, recency_blocks=2, kmin_blocks=4)
+    pf = _prefill(sh, pr, q_sel, keys, qkv, pt, lens, qlens, 0.8)
+    q, k, v = qkv
+    dec = oracle.decode_step(sh, pr, _bf16_bits(q_sel), None, _bf16_bits(keys), None,
+                             _bf16_bits(q), _bf16_bits(k), _bf16_bits(v), pt,
+                             np.array(lens, np.int32), np.full(3, 0.8, np.float32), 0.1)
+    assert len(pf["tiles"]) == 3
+    for t in range(3):
+        for g in range(2):
+            a = pf["sel_idx"][t, g, :pf["sel_cnt"][t, g]].tolist()
+            assert a == dec["sel_idx"][t, g, :dec["sel_cnt"][t, g]].tolist()
+    assert np.array_equal(pf["out"], dec["out"])
+    assert np.array_equal(pf["lse"], dec["lse"])
+
+
+def test_prefill_keep_all_is_causal_dense_attention():
+    rng = np.random.default_rng(21)
+    lens, qlens = [200, 130], [150, 67]       # chunks start mid-block
+    sh, q_sel, keys, qkv, (q64, k64, v64), pt = _prefill_problem(rng, lens, qlens)
+    pr = oracle.make_params(sink_blocks=1, recency_blocks=1, kmin_blocks=0)
+    pf = _prefill(sh, pr, q_sel, keys, qkv, pt, lens, qlens, 1.0)
+    row = 0
+    for b, (L, T) in enumerate(zip(lens, qlens)):
+        for i in range(T):
+            pos = L - T + i
+            for h in range(4):
+                kk = torch.stack([k64[pt[b, t // 64], h // 2, t % 64] for t in range(pos + 1)])
+                vv = torch.stack([v64[pt[b, t // 64], h // 2, t % 64] for t in range(pos + 1)])
+                ref = _sdpa(q64[row, h], kk, vv, 0.1)
+                assert np.allclose(pf["out"][row, h], ref.numpy(), atol=1e-12, rtol=1e-10), (b, i, h)
+            row += 1
+
+
+def test_prefill_tile_score_is_the_max_over_its_queries():
+    rng = np.random.default_rng(22)
+    lens, qlens = [260], [100]               # tiles: [160, 191], [192, 255], [256, 259]
+    sh, q_sel, keys, qkv, _, pt = _prefill_problem(rng, lens, qlens)
+    pr = oracle.make_params()
+    sc = oracle.prefill_scores(sh, pr, _bf16_bits(q_sel), None, _bf16_bits(keys), None, pt,
+                               np.array(lens, np.int32), np.array(qlens, np.int32))
+    tiles = oracle.prefill_tiles(lens, qlens)
+    assert [(lo, hi) for _, lo, hi, _ in tiles] == [(160, 191), (192, 255), (256, 259)]
+    # each query scored alone (as a decode query) against its tile's blocks:
+    # the complete blocks below the tile's last position + 1
+    rows = 100
+    dsh = oracle.make_shape(rows, 4, 2, 128, 64, 64, "bf16", sh.num_pages, sh.max_blocks)
+    tile_end = np.concatenate([np.full(hi - lo + 1, hi + 1) for _, lo, hi, _ in tiles])
+    per_q = oracle.block_scores(dsh, pr, _bf16_bits(q_sel), None, _bf16_bits(keys), None,
+                                np.repeat(pt, rows, axis=0), tile_end.astype(np.int32))
+    for t, (_, lo, hi, r0) in enumerate(tiles):
+        nf = (hi + 1) // 64
+        want = np.max(per_q[r0:r0 + hi - lo + 1, :, :nf], axis=0)
+        assert np.array_equal(sc[t, :, :nf], want), t
+        assert np.isnan(sc[t, :, nf:]).all()
+
+
+def test_prefill_causal_mask_and_tile_recency():
+    rng = np.random.default_rng(23)
+    lens, qlens = [512], [130]
+    sh, q_sel, keys, (q, k, v), _, pt = _prefill_problem(rng, lens, qlens)
+    pr = oracle.make_params(sink_blocks=1, recency_blocks=2, kmin_blocks=0)
+    base = _prefill(sh, pr, q_sel, keys, (q, k, v), pt, lens, qlens, 0.5)
+    # tiles [382, 383], [384, 447], [448, 511]: each keeps block 0 and its last two blocks
+    for t, (_, lo, hi, _) in enumerate(base["tiles"]):
+        nb = (hi + 1 + 63) // 64
+        s = set(base["sel_idx"][t, 0, :base["sel_cnt"][t, 0]].tolist())
+        assert {0, nb - 2, nb - 1} <= s and max(s) == nb - 1
+    # keys / values after position 400 change: rows of queries at <= 400 do not
+    k2, v2 = k.copy(), v.copy()
+    for t in range(401, 512):
+        k2[pt[0, t // 64], :, t % 64] += 5.0
+        v2[pt[0, t // 64], :, t % 64] -= 7.0
+    pert = _prefill(sh, pr, q_sel, keys, (q, k2, v2), pt, lens, qlens, 0.5)
+    r400 = 400 - 382
+    assert np.array_equal(base["out"][:r400 + 1], pert["out"][:r400 + 1])
+    assert not np.allclose(base["out"][r400 + 1:], pert["out"][r400 + 1:])

@@ -444,3 +444,141 @@ def _plant_hot_tok(wl: TokWorkload, rng, integer: bool):
             ck = o * G * math.sqrt(HEAD_DIM) / nkv
             kk = wl.k_pool[pg, g, slots].float() + ck[:, None, None] * (qk[b, g] / nkv)
             wl.k_pool[pg, g, slots] = kk.to(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------
+# Sparse prefill: a chunk of new queries per sequence (the last q_len of its
+# seq_len cached tokens), selector keys per (block, KV head) as in decode.
+
+@dataclasses.dataclass
+class PrefillSpec:
+    name: str
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    seq_len: int
+    q_len: int
+    top_p: float = 0.9
+    sink_blocks: int = 1
+    recency_blocks: int = 4
+    kmin_blocks: int = 8
+    hot_count: int = 16
+    page_order: str = "permuted"
+
+
+PREFILL_SPECS = {
+    "prefill_tiny": PrefillSpec("prefill_tiny", 2, 8, 2, 1000, 300, hot_count=3,
+                                page_order="contiguous"),
+    "qwen3_8b_prefill_32k": PrefillSpec("qwen3_8b_prefill_32k", 1, 32, 8, 32768, 32768),
+}
+
+
+@dataclasses.dataclass
+class PrefillWorkload:
+    spec: PrefillSpec
+    seed: int
+    seq_lens: torch.Tensor              # int32 [B]
+    q_lens: torch.Tensor                # int32 [B]
+    page_table: torch.Tensor            # int32 [B, max_blocks]
+    num_pages: int
+    q: torch.Tensor                     # bf16 [rows, Hq, D]   (rows = sum of q_lens)
+    q_sel: torch.Tensor                 # bf16 [rows, Hq, ds]
+    w: Optional[torch.Tensor]           # fp32 [rows, Hq] or None (1/G)
+    sel_keys: torch.Tensor              # bf16 [num_pages, Hkv, ds]
+    k_pool: torch.Tensor
+    v_pool: torch.Tensor
+    top_p: torch.Tensor                 # fp32 [B]
+
+    @property
+    def batch(self):
+        return self.spec.batch
+
+    @property
+    def num_q_heads(self):
+        return self.spec.num_q_heads
+
+    @property
+    def num_kv_heads(self):
+        return self.spec.num_kv_heads
+
+    @property
+    def max_blocks(self):
+        return int(self.page_table.shape[1])
+
+    @property
+    def sm_scale(self):
+        return 1.0 / math.sqrt(HEAD_DIM)
+
+
+def make_prefill(name: str, seed: int = 0, device="cpu", *, seq_lens=None, q_lens=None,
+                 batch=None, integer: bool = False, top_p=None, **spec_overrides):
+    """Seeded prefill workload.  seq_lens / q_lens (lists) override the
+    spec's uniform ones; integer=True draws selector queries and keys from
+    {-3..3}."""
+    spec = dataclasses.replace(PREFILL_SPECS[name], **spec_overrides)
+    if batch is not None:
+        spec = dataclasses.replace(spec, batch=batch)
+    if top_p is not None:
+        spec = dataclasses.replace(spec, top_p=top_p)
+    device = torch.device(device)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    B, Hq, Hkv = spec.batch, spec.num_q_heads, spec.num_kv_heads
+    lens = np.array(seq_lens if seq_lens is not None else [spec.seq_len] * B, np.int64)
+    qls = np.array(q_lens if q_lens is not None else [spec.q_len] * B, np.int64)
+    B = len(lens)
+    spec = dataclasses.replace(spec, batch=B)
+    nbs = (lens + BLOCK - 1) // BLOCK
+    mb = int(max(nbs.max() if B else 0, 1))
+    num_pages = int(max(nbs.sum(), 1))
+    pages = np.arange(num_pages) if spec.page_order == "contiguous" else rng.permutation(num_pages)
+    pt = np.full((B, mb), -1, np.int32)
+    off = 0
+    for b in range(B):
+        pt[b, :nbs[b]] = pages[off:off + nbs[b]]
+        off += nbs[b]
+    rows = int(qls.sum())
+    q = _normal_bf16((rows, Hq, HEAD_DIM), gen, device)
+    if integer:
+        q_sel = _int_bf16((rows, Hq, SEL_DIM), gen, device)
+        sel_keys = _int_bf16((num_pages, Hkv, SEL_DIM), gen, device)
+    else:
+        q_sel = _normal_bf16((rows, Hq, SEL_DIM), gen, device)
+        sel_keys = _normal_bf16((num_pages, Hkv, SEL_DIM), gen, device)
+    k_pool = _normal_bf16((num_pages, Hkv, BLOCK, HEAD_DIM), gen, device)
+    v_pool = _normal_bf16((num_pages, Hkv, BLOCK, HEAD_DIM), gen, device)
+    wl = PrefillWorkload(spec, seed, torch.as_tensor(lens, dtype=torch.int32, device=device),
+                         torch.as_tensor(qls, dtype=torch.int32, device=device),
+                         torch.as_tensor(pt, device=device), num_pages, q, q_sel, None, sel_keys,
+                         k_pool, v_pool,
+                         torch.full((B,), spec.top_p, dtype=torch.float32, device=device))
+    # hot blocks per (sequence, KV head) along the chunk's mean query direction
+    G = Hq // Hkv
+    row = 0
+    for b in range(B):
+        nb = int(nbs[b])
+        cand = np.arange(spec.sink_blocks, max(nb - spec.recency_blocks, spec.sink_blocks))
+        rows_b = slice(row, row + int(qls[b]))
+        row += int(qls[b])
+        if cand.size == 0 or qls[b] == 0:
+            continue
+        qs = q_sel[rows_b].float().view(-1, Hkv, G, SEL_DIM).sum((0, 2))
+        qk = q[rows_b].float().view(-1, Hkv, G, HEAD_DIM).sum((0, 2))
+        for g in range(Hkv):
+            n_hot = min(spec.hot_count, cand.size)
+            hot = np.sort(rng.choice(cand, size=n_hot, replace=False))
+            o = torch.as_tensor(rng.uniform(2.0, 4.0, size=n_hot), dtype=torch.float32,
+                                device=device)
+            pg = torch.as_tensor(pt[b, hot].astype(np.int64), device=device)
+            us, uk = qs[g] / qs[g].norm(), qk[g] / qk[g].norm()
+            if integer:
+                wl.sel_keys[pg, g] = (3.0 * torch.sign(qs[g])).expand(n_hot, SEL_DIM).to(
+                    torch.bfloat16)
+            else:
+                wl.sel_keys[pg, g] = (wl.sel_keys[pg, g].float() +
+                                      (o * 8.0)[:, None] * us).to(torch.bfloat16)
+            wl.k_pool[pg, g] = (wl.k_pool[pg, g].float() +
+                                (o * math.sqrt(HEAD_DIM) / 4.0)[:, None, None] * uk).to(
+                                    torch.bfloat16)
+    return wl
