@@ -103,6 +103,13 @@ def lib():
                                              P, sz, P]
         L.spot_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, P, i32, f32, P, P,
                                            i32, P, P, P, sz, P]
+        L.spot_prefill_num_tiles.argtypes = [P, P, i32]
+        L.spot_prefill_num_tiles.restype = ctypes.c_int64
+        L.spot_prefill_workspace_size.argtypes = [P, i32, i32, i32]
+        L.spot_prefill_workspace_size.restype = sz
+        L.spot_prefill.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, P, P, i32, i32, f32, P, P,
+                                   i32, P, P, P, sz, P]
+        L.spot_prefill.restype = ctypes.c_int
         L.spot_read_device_status.argtypes = [P, P]
         L.spot_check_wait_timeout.argtypes = [P, P]
         L.spot_check_wait_timeout.restype = ctypes.c_int
@@ -312,6 +319,55 @@ def tok_decode_step(desc: TokLayerDesc, params: SelectParams, q_idx, w_idx, sel_
         _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check(code, "tok_decode_step")
+
+
+# ---------------------------------------------------------------- sparse prefill
+
+def prefill_num_tiles(seq_lens, q_lens) -> int:
+    """Query tiles of a batch (host lists / arrays of seq_lens and q_lens)."""
+    import numpy as _np
+    a = _np.ascontiguousarray(_np.asarray(seq_lens, dtype=_np.int32))
+    b = _np.ascontiguousarray(_np.asarray(q_lens, dtype=_np.int32))
+    n = lib().spot_prefill_num_tiles(a.ctypes.data_as(ctypes.c_void_p),
+                                     b.ctypes.data_as(ctypes.c_void_p), int(a.size))
+    if n < 0:
+        raise SpotError(1, "prefill_num_tiles")
+    return int(n)
+
+
+def prefill_workspace_size(desc: LayerDesc, batch: int, max_tiles: int, max_blocks: int) -> int:
+    n = lib().spot_prefill_workspace_size(ctypes.byref(desc), batch, max_tiles, max_blocks)
+    if n == 0:
+        raise SpotError(2, "prefill_workspace_size")
+    return int(n)
+
+
+def new_prefill_workspace(desc: LayerDesc, batch: int, max_tiles: int, max_blocks: int,
+                          device=None) -> torch.Tensor:
+    n = prefill_workspace_size(desc, batch, max_tiles, max_blocks)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def prefill(desc: LayerDesc, params: SelectParams, q_sel, w, sel_data, q, k_pool, v_pool,
+            page_table, seq_lens, q_lens, top_p, softmax_scale, sel_idx, sel_cnt, out, lse,
+            workspace, stream=None):
+    """Sparse prefill of packed chunk queries: per (tile, KV head) selection
+    into sel_idx int32 [max_tiles, Hkv, max_blocks] / sel_cnt [max_tiles, Hkv],
+    causal attention into out fp32 [rows, Hq, D] (+ lse [rows, Hq])."""
+    B = int(seq_lens.shape[0])
+    max_tiles, max_blocks = int(sel_idx.shape[0]), int(sel_idx.shape[-1])
+    code = lib().spot_prefill(
+        ctypes.byref(desc), ctypes.byref(params), _ptr(q_sel, torch.bfloat16, "q_sel"),
+        _ptr(w, torch.float32, "w"), _ptr(sel_data, torch.bfloat16, "sel_data"),
+        _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
+        _ptr(v_pool, torch.bfloat16, "v_pool"), _ptr(page_table, torch.int32, "page_table"),
+        int(page_table.shape[-1]), _ptr(seq_lens, torch.int32, "seq_lens"),
+        _ptr(q_lens, torch.int32, "q_lens"), _ptr(top_p, torch.float32, "top_p"), B, max_tiles,
+        float(softmax_scale), _ptr(sel_idx, torch.int32, "sel_idx"),
+        _ptr(sel_cnt, torch.int32, "sel_cnt"), max_blocks, _ptr(out, torch.float32, "out"),
+        _ptr(lse, torch.float32, "lse"), _ptr(workspace, name="workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "prefill")
 
 
 def check_wait_timeout(workspace, stream=None):

@@ -650,3 +650,143 @@ spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ sparse prefill
+
+namespace {
+
+struct PrefillLayout {
+    size_t status, tile_info, tile_len, tile_p, scores, total;
+};
+
+bool prefill_layout(const spot_layer_desc_t* d, int max_tiles, int max_blocks, PrefillLayout* out) {
+    PrefillLayout L;
+    size_t off = 0;
+    L.status = off;
+    off += kStatusBytes;
+    L.tile_info = off;
+    off = round_up(off + static_cast<size_t>(max_tiles) * sizeof(int4), 256);
+    L.tile_len = off;
+    off = round_up(off + static_cast<size_t>(max_tiles) * sizeof(int32_t), 256);
+    L.tile_p = off;
+    off = round_up(off + static_cast<size_t>(max_tiles) * sizeof(float), 256);
+    L.scores = off;
+    off = round_up(off + static_cast<size_t>(max_tiles) * d->num_kv_heads * max_blocks *
+                             sizeof(float), 256);
+    L.total = off;
+    *out = L;
+    return true;
+}
+
+spot_status_t check_prefill_shape(const spot_layer_desc_t* d, int batch, int max_tiles,
+                                  int max_blocks) {
+    spot_status_t st = check_desc(d);
+    if (st != SPOT_OK) return st;
+    if (d->sel_fmt != SPOT_SEL_BF16) return SPOT_ERR_UNSUPPORTED;
+    if (batch < 0 || max_tiles < 0 || max_blocks <= 0) return SPOT_ERR_INVALID_ARG;
+    if (max_blocks > kMaxBlocks || batch > kMaxUnits) return SPOT_ERR_UNSUPPORTED;
+    // selection grid and unit indices
+    if (static_cast<int64_t>(max_tiles) * d->num_kv_heads * prefill_row_groups(
+            d->num_q_heads / d->num_kv_heads) > INT32_MAX / 2)
+        return SPOT_ERR_UNSUPPORTED;
+    return SPOT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t spot_prefill_num_tiles(const int32_t* seq_lens_host, const int32_t* q_lens_host,
+                               int32_t batch) {
+    if (!seq_lens_host || !q_lens_host || batch < 0) return -1;
+    int64_t t = 0;
+    for (int b = 0; b < batch; ++b) {
+        const int32_t L = seq_lens_host[b], T = q_lens_host[b];
+        if (L < 0 || T < 0 || T > L) return -1;
+        if (T > 0) t += (L - 1) / kBlock - (L - T) / kBlock + 1;
+    }
+    return t;
+}
+
+size_t spot_prefill_workspace_size(const spot_layer_desc_t* desc, int32_t batch,
+                                   int32_t max_tiles, int32_t max_blocks) {
+    if (check_prefill_shape(desc, batch, max_tiles, max_blocks) != SPOT_OK) return 0;
+    PrefillLayout L;
+    if (!prefill_layout(desc, max_tiles, max_blocks, &L)) return 0;
+    return L.total;
+}
+
+spot_status_t spot_prefill(const spot_layer_desc_t* desc, const spot_select_params_t* params,
+                           const uint16_t* q_sel, const float* w, const void* sel_data,
+                           const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                           const int32_t* page_table, int32_t pt_stride,
+                           const int32_t* seq_lens, const int32_t* q_lens, const float* top_p,
+                           int32_t batch, int32_t max_tiles, float softmax_scale,
+                           int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks, float* out,
+                           float* lse, void* workspace, size_t ws_bytes, void* stream) {
+    spot_status_t st = check_prefill_shape(desc, batch, max_tiles, max_blocks);
+    if (st != SPOT_OK) return st;
+    if (batch == 0 || max_tiles == 0) return SPOT_OK;
+    st = check_params(params);
+    if (st != SPOT_OK) return st;
+    if (params->quantize_queries) return SPOT_ERR_UNSUPPORTED;
+    if (!q_sel || !sel_data || !q || !k_pool || !v_pool || !page_table || !seq_lens || !q_lens ||
+        !sel_idx || !sel_cnt || !out)
+        return SPOT_ERR_INVALID_ARG;
+    if (params->mode == SPOT_MODE_TOPP && !top_p) return SPOT_ERR_INVALID_ARG;
+    if (pt_stride <= 0 || !isfinite(softmax_scale)) return SPOT_ERR_INVALID_ARG;
+    if (!aligned(q_sel, 16) || !aligned(sel_data, 16) || !aligned(q, 16) ||
+        !aligned(k_pool, 256) || !aligned(v_pool, 256) || !aligned(page_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(q_lens, 4) || !aligned(sel_idx, 4) ||
+        !aligned(sel_cnt, 4) || !aligned(out, 8) || (w && !aligned(w, 4)) ||
+        (top_p && !aligned(top_p, 4)) || (lse && !aligned(lse, 4)))
+        return SPOT_ERR_INVALID_ARG;
+    PrefillLayout L;
+    if (!prefill_layout(desc, max_tiles, max_blocks, &L)) return SPOT_ERR_CUDA;
+    if (!workspace || !aligned(workspace, 256)) return SPOT_ERR_INVALID_ARG;
+    if (ws_bytes < L.total) return SPOT_ERR_WORKSPACE;
+    CUtensorMap km, vm;
+    if (!make_pool_map(&km, k_pool, desc->num_pages, desc->num_kv_heads) ||
+        !make_pool_map(&vm, v_pool, desc->num_pages, desc->num_kv_heads))
+        return SPOT_ERR_CUDA;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    PrefillParams p;
+    p.seq_lens = seq_lens;
+    p.q_lens = q_lens;
+    p.top_p = top_p;
+    p.batch = batch;
+    p.max_tiles = max_tiles;
+    p.tile_info = reinterpret_cast<int4*>(base + L.tile_info);
+    p.tile_len = reinterpret_cast<int32_t*>(base + L.tile_len);
+    p.tile_p = reinterpret_cast<float*>(base + L.tile_p);
+    p.page_table = page_table;
+    p.pt_stride = pt_stride;
+    p.num_pages = desc->num_pages;
+    p.num_q_heads = desc->num_q_heads;
+    p.num_kv_heads = desc->num_kv_heads;
+    p.group = desc->num_q_heads / desc->num_kv_heads;
+    p.max_blocks = max_blocks;
+    p.sel_data = sel_data;
+    p.q_sel = q_sel;
+    p.w = w;
+    p.inv_temp = 1.0f / params->temperature;
+    p.scores = reinterpret_cast<float*>(base + L.scores);
+    p.mode = params->mode;
+    p.sink_blocks = params->sink_blocks;
+    p.recency_blocks = params->recency_blocks;
+    p.kmin_blocks = params->kmin_blocks;
+    p.topk_blocks = params->topk_blocks;
+    p.sel_idx = sel_idx;
+    p.sel_cnt = sel_cnt;
+    p.q = q;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.row_groups = prefill_row_groups(p.group);
+    p.out = out;
+    p.lse = lse;
+    p.status = reinterpret_cast<uint32_t*>(base + L.status);
+    return launch_prefill(p, km, vm, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SPOT_OK
+               : SPOT_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -667,6 +667,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
         sm.keep = q;
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // precomputed scores: the lengths and p may come from a preceding kernel too
+    if constexpr (FMT == kSelectFromScores) pdl_wait();
 
     const int u = blockIdx.x;
     const int b = u / p.num_kv_heads;
@@ -695,7 +697,6 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
 
     // ---- selector scores of the complete blocks (§2.1), into shared memory
     if constexpr (FMT == kSelectFromScores) {
-        pdl_wait();                                   // block scores of the scoring kernel
         const float* src = p.scores_in + static_cast<int64_t>(u) * p.max_blocks;
         constexpr int kBatch = 8;                     // loads in flight per thread
         for (int j0 = threadIdx.x; j0 < n_full; j0 += NT * kBatch) {

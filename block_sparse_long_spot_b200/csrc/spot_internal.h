@@ -128,6 +128,33 @@ struct TokAppendParams {
     uint32_t* status;
 };
 
+// Sparse prefill: all four kernels share one parameter block.
+struct PrefillParams {
+    const int32_t* seq_lens;            // [B] cached tokens, the chunk included
+    const int32_t* q_lens;              // [B] chunk queries (the last q_lens of seq_lens)
+    const float* top_p;                 // [B]
+    int32_t batch, max_tiles;
+    int4* tile_info;                    // [max_tiles] (b, first pos, last pos, first row)
+    int32_t* tile_len;                  // [max_tiles] last pos + 1 (0: no tile)
+    float* tile_p;                      // [max_tiles]
+    const int32_t* page_table;
+    int32_t pt_stride, num_pages, num_q_heads, num_kv_heads, group, max_blocks;
+    const void* sel_data;               // bf16 selector keys [num_pages][Hkv][64]
+    const uint16_t* q_sel;              // [rows][Hq][64]
+    const float* w;                     // [rows][Hq] or null
+    float inv_temp;
+    float* scores;                      // [max_tiles * Hkv][max_blocks]
+    int32_t mode, sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
+    int32_t* sel_idx;                   // [max_tiles * Hkv][max_blocks]
+    int32_t* sel_cnt;                   // [max_tiles * Hkv]
+    const uint16_t* q;                  // [rows][Hq][128]
+    float scale_log2;
+    int32_t row_groups;                 // CTAs per (tile, KV head) in the attention kernel
+    float* out;                         // [rows][Hq][128]
+    float* lse;                         // [rows][Hq] or null
+    uint32_t* status;
+};
+
 // Launch with programmatic stream serialisation (the kernel must call
 // pdl_wait() before touching anything its predecessor writes).
 template <typename... KArgs, typename... Args>
@@ -153,6 +180,9 @@ cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map
                                  const CUtensorMap& v_map, bool shared16, cudaStream_t s);
 cudaError_t launch_tok_score(const TokScoreParams& p, const CUtensorMap& sel_map, cudaStream_t s);
 cudaError_t launch_tok_append(const TokAppendParams& p, cudaStream_t s);
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& k_map,
+                           const CUtensorMap& v_map, cudaStream_t s);
+int prefill_row_groups(int group);
 int tok_score_grid(int batch);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 

@@ -308,6 +308,50 @@ spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
                                    float* out, float* lse, void* workspace, size_t ws_bytes,
                                    void* stream);
 
+/* ------------------------------------------------------------------------
+ * Sparse prefill (§2.1 / §2.3 applied to a chunk of queries; the selector
+ * scores query-block x key-block tiles).  Sequence b has seq_lens[b] tokens
+ * in the cache (KV and selector keys of the chunk already appended); its
+ * chunk is the last q_lens[b] of them, stored as rows
+ * q_off(b) .. q_off(b) + q_lens[b] - 1 of the packed query arrays, q_off(b)
+ * = sum of q_lens[b'] over b' < b.  The chunk's queries are grouped into
+ * tiles -- the queries whose positions share one KV block -- numbered
+ * sequence by sequence, block ascending (spot_prefill_num_tiles counts
+ * them).  Tile (b, m), KV head g, keeps the blocks a decode query at the
+ * tile's last position would keep (same parameters, Eq. 6-8), scored by the
+ * maximum over the tile's queries of (1/tau) sum_h w_h ReLU(q_sel_h . k);
+ * every query attends to the keys of its tile's selection at positions up
+ * to its own.  bf16 selector keys; quantize_queries must be 0.
+ *
+ * Layouts:
+ *   q_sel   bf16 [rows][num_q_heads][sel_dim]     w fp32 [rows][num_q_heads] or NULL
+ *   q       bf16 [rows][num_q_heads][head_dim]
+ *   sel_idx int32 [max_tiles][num_kv_heads][max_blocks]  (ascending, sel_cnt valid)
+ *   sel_cnt int32 [max_tiles][num_kv_heads]
+ *   out     fp32 [rows][num_q_heads][head_dim]   lse fp32 [rows][num_q_heads] or NULL
+ * max_tiles bounds the tile count (tiles past it are not computed and
+ * SPOT_ERR_DEVICE_BOUNDS is recorded); max_blocks <= 8192 bounds
+ * ceil(seq_len / 64) and is the page-table width used for the selection.
+ * ------------------------------------------------------------------------ */
+
+/* Tiles of a batch, from host copies of seq_lens and q_lens. */
+int64_t spot_prefill_num_tiles(const int32_t* seq_lens_host, const int32_t* q_lens_host,
+                               int32_t batch);
+
+/* Scratch bytes for spot_prefill (zero the first 256 bytes once); 0 if
+ * unsupported. */
+size_t spot_prefill_workspace_size(const spot_layer_desc_t* desc, int32_t batch,
+                                   int32_t max_tiles, int32_t max_blocks);
+
+spot_status_t spot_prefill(const spot_layer_desc_t* desc, const spot_select_params_t* params,
+                           const uint16_t* q_sel, const float* w, const void* sel_data,
+                           const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                           const int32_t* page_table, int32_t pt_stride,
+                           const int32_t* seq_lens, const int32_t* q_lens, const float* top_p,
+                           int32_t batch, int32_t max_tiles, float softmax_scale,
+                           int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks, float* out,
+                           float* lse, void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, return the status recorded by kernels in
  * `workspace` since the last read (SPOT_OK, SPOT_ERR_DEVICE_BOUNDS or
  * SPOT_ERR_DEVICE_TIMEOUT; bounds wins if both), and clear it. */

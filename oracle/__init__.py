@@ -86,7 +86,7 @@ def _load():
                                                P, P, P, P, P]
         lib.oracle_prefill_num_tiles.argtypes = [P, P, P]
         lib.oracle_prefill_num_tiles.restype = i64
-        lib.oracle_prefill_scores.argtypes = [P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_prefill_scores.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, P]
         lib.oracle_prefill_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
                                             P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -289,18 +289,19 @@ def prefill_tiles(seq_lens, q_lens, block_size=64):
 
 
 def prefill_scores(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, page_table,
-                   seq_lens, q_lens) -> np.ndarray:
-    """Block scores [tiles, Hkv, max_blocks] of every query tile (max over
-    the tile's queries; NaN where no complete block)."""
+                   seq_lens, q_lens, tiles=None) -> np.ndarray:
+    """Block scores [tiles, Hkv, max_blocks] of the query tiles (max over
+    the tile's queries; NaN where no complete block or tile not listed)."""
     lens, ql = _c(seq_lens, np.int32), _c(q_lens, np.int32)
     nt = int(_load().oracle_prefill_num_tiles(ctypes.byref(shape), _ptr(lens), _ptr(ql)))
     scores = np.full((max(nt, 1), shape.num_kv_heads, shape.max_blocks), np.nan)
     fmt = shape.sel_fmt
+    tl = None if tiles is None else _c(tiles, np.int32)
     rc = _load().oracle_prefill_scores(
         ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_sel, np.uint16)),
         _ptr(_c(w, np.float32)), _ptr(_c(sel_data, _data_dtype(_FMT_NAME[fmt]))),
         _ptr(_c(sel_scales, _scale_dtype(_FMT_NAME[fmt]))), _ptr(_c(page_table, np.int32)),
-        _ptr(lens), _ptr(ql), _ptr(scores))
+        _ptr(lens), _ptr(ql), _ptr(tl), 0 if tl is None else len(tl), _ptr(scores))
     assert rc == 0
     return scores[:nt]
 

@@ -708,12 +708,14 @@ static int prefill_tile_scores(const orc_shape_t* sh, const orc_params_t* pr,
     return 0;
 }
 
-/* Block scores of every tile: scores[tile][g][max_blocks] (entries past a
- * tile's complete blocks untouched). */
+/* Block scores of the tiles `tiles[n_tiles]` (NULL: all):
+ * scores[tile][g][max_blocks] (entries past a tile's complete blocks
+ * untouched). */
 int oracle_prefill_scores(const orc_shape_t* sh, const orc_params_t* pr, const uint16_t* q_sel,
                           const float* w, const void* sel_data, const void* sel_scales,
                           const int32_t* page_table, const int32_t* seq_lens,
-                          const int32_t* q_lens, double* scores) {
+                          const int32_t* q_lens, const int32_t* tiles, int32_t n_tiles,
+                          double* scores) {
     int64_t rows = (int64_t)sh->num_pages * sh->num_kv_heads;
     double* keys = (double*)malloc((size_t)(rows * sh->sel_dim) * sizeof(double));
     if (!keys) return -2;
@@ -721,13 +723,13 @@ int oracle_prefill_scores(const orc_shape_t* sh, const orc_params_t* pr, const u
         free(keys);
         return -1;
     }
-    int64_t nt = oracle_prefill_num_tiles(sh, seq_lens, q_lens);
+    int64_t nt = tiles ? n_tiles : oracle_prefill_num_tiles(sh, seq_lens, q_lens);
     int err = 0;
 #ifdef _OPENMP
 #pragma omp parallel for schedule(dynamic, 1)
 #endif
     for (int64_t k = 0; k < nt * sh->num_kv_heads; ++k) {
-        int64_t t = k / sh->num_kv_heads;
+        int64_t t = tiles ? tiles[k / sh->num_kv_heads] : k / sh->num_kv_heads;
         int g = (int)(k % sh->num_kv_heads);
         int b;
         int32_t p_lo, p_hi;

@@ -354,3 +354,143 @@ def safe_top_p_tok(wl, lo=0.5, hi=0.99, margin=2e-5, **kw):
         assert gaps[k] > 2 * margin
         ps.append(0.5 * (c[k] + c[k + 1]))
     return torch.as_tensor(np.array(ps, np.float32), device=wl.top_p.device)
+
+
+# ------------------------------------------------------------------ sparse prefill
+
+def _pf_sel(spec, kmin, sink, rec):
+    return (spec.kmin_blocks if kmin is None else kmin, spec.sink_blocks if sink is None else sink,
+            spec.recency_blocks if rec is None else rec)
+
+
+def run_gpu_prefill(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None, temperature=1.0,
+                    max_tiles=None):
+    dev = wl.q.device
+    Hq, Hkv, mb = wl.num_q_heads, wl.num_kv_heads, wl.max_blocks
+    kmin, sink, rec = _pf_sel(wl.spec, kmin, sink, rec)
+    nt = spot.prefill_num_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    mt = max(nt, 1) if max_tiles is None else max_tiles
+    desc = spot.layer_desc(Hq, Hkv, wl.num_pages, "bf16")
+    prm = spot.select_params(mode, sink, rec, kmin, topk, temperature)
+    ws = spot.new_prefill_workspace(desc, wl.batch, mt, mb, dev)
+    rows = int(wl.q.shape[0])
+    sel_idx = torch.full((mt, Hkv, mb), -1, dtype=torch.int32, device=dev)
+    sel_cnt = torch.full((mt, Hkv), -1, dtype=torch.int32, device=dev)
+    out = torch.full((max(rows, 1), Hq, 128), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.full((max(rows, 1), Hq), float("nan"), dtype=torch.float32, device=dev)
+    spot.prefill(desc, prm, wl.q_sel, wl.w, wl.sel_keys, wl.q, wl.k_pool, wl.v_pool,
+                 wl.page_table, wl.seq_lens, wl.q_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt,
+                 out, lse, ws)
+    torch.cuda.synchronize()
+    status = spot.read_device_status(ws)
+    return {"sel_idx": sel_idx.cpu().numpy()[:nt], "sel_cnt": sel_cnt.cpu().numpy()[:nt],
+            "out": out.cpu().double().numpy()[:rows], "lse": lse.cpu().double().numpy()[:rows],
+            "status": status, "num_tiles": nt}
+
+
+def prefill_oracle_args(wl):
+    return dict(q_sel=workloads.bits(wl.q_sel), w=host_bytes(wl.w),
+                sel_data=workloads.bits(wl.sel_keys), sel_scales=None, q=workloads.bits(wl.q),
+                k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
+                page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
+                q_lens=wl.q_lens.cpu().numpy(), top_p=wl.top_p.cpu().numpy(),
+                sm_scale=wl.sm_scale)
+
+
+def prefill_shape_params(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None,
+                         temperature=1.0):
+    kmin, sink, rec = _pf_sel(wl.spec, kmin, sink, rec)
+    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, "bf16",
+                           wl.num_pages, wl.max_blocks)
+    return sh, oracle.make_params(mode, sink, rec, kmin, topk, temperature)
+
+
+def run_oracle_prefill(wl, tiles=None, args=None, **kw):
+    sh, pr = prefill_shape_params(wl, **kw)
+    return oracle.prefill_step(sh, pr, tiles=tiles, **(args or prefill_oracle_args(wl)))
+
+
+def oracle_prefill_scores(wl, tiles=None, args=None, **kw):
+    sh, pr = prefill_shape_params(wl, **kw)
+    a = args or prefill_oracle_args(wl)
+    return oracle.prefill_scores(sh, pr, a["q_sel"], a["w"], a["sel_data"], None,
+                                 a["page_table"], a["seq_lens"], a["q_lens"], tiles=tiles)
+
+
+def tile_selection(res, t, g):
+    return res["sel_idx"][t, g, :res["sel_cnt"][t, g]].tolist()
+
+
+def check_prefill_selection_near_cut(gpu, ora, scores, wl, tiles=None, kmin=None, sink=None,
+                                     rec=None):
+    """The real-valued rule per (tile, KV head); returns how many differ."""
+    kmin, sink, rec = _pf_sel(wl.spec, kmin, sink, rec)
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    p_all = wl.top_p.cpu().numpy()
+    n_diff = 0
+    for t in (range(len(info)) if tiles is None else tiles):
+        b, lo, hi, _ = info[t]
+        reserved, res = _reserved_residual(hi + 1, 64, sink, rec)
+        for g in range(wl.num_kv_heads):
+            n_diff += _unit_near_cut(set(tile_selection(gpu, t, g)), set(tile_selection(ora, t, g)),
+                                     scores[t, g], reserved, res, float(p_all[b]), kmin, (t, g))
+    return n_diff
+
+
+def check_prefill_outputs(gpu, ora, wl, tiles=None):
+    """Element-wise check of the query rows of every (tile, KV head) whose
+    selections agree; returns (max abs err, units compared).
+
+    Tolerance: the kernel rounds the softmax weights p to bf16 (relative
+    2^-9) before the P.V product, an output error of at most
+    2^-9 * sum_i p_i |v_i| / l <= 2^-9 * max |v|.  Decode rows average
+    hundreds of tokens and stay far inside ATOL; a prefill row near its
+    chunk's start may see a handful, so the bound itself is added."""
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    G = wl.num_q_heads // wl.num_kv_heads
+    atol = ATOL + 2.0 ** -9 * float(wl.v_pool.abs().max().item())
+    worst, n = 0.0, 0
+    for t in (range(len(info)) if tiles is None else tiles):
+        _, lo, hi, r0 = info[t]
+        rows = slice(r0, r0 + hi - lo + 1)
+        for g in range(wl.num_kv_heads):
+            if tile_selection(gpu, t, g) != tile_selection(ora, t, g):
+                continue
+            hs = slice(g * G, (g + 1) * G)
+            o_g, o_r = gpu["out"][rows, hs], ora["out"][rows, hs]
+            err = np.abs(o_g - o_r)
+            assert not (err > atol + RTOL * np.abs(o_r)).any(), (t, g, float(err.max()))
+            l_g, l_r = gpu["lse"][rows, hs], ora["lse"][rows, hs]
+            fin = np.isfinite(l_r)
+            assert np.array_equal(fin, np.isfinite(l_g)), (t, g)
+            assert (np.abs(l_g[fin] - l_r[fin]) <= ATOL + RTOL * np.abs(l_r[fin])).all(), (t, g)
+            worst = max(worst, float(err.max()) if err.size else 0.0)
+            n += 1
+    return worst, n
+
+
+def safe_top_p_prefill(wl, lo=0.5, hi=0.99, margin=2e-5, **kw):
+    """Per-sequence p at least `margin` from every cumulative residual mass
+    of every (tile, KV head) of that sequence."""
+    kmin, sink, rec = _pf_sel(wl.spec, kw.get("kmin"), kw.get("sink"), kw.get("rec"))
+    scores = oracle_prefill_scores(wl, **kw)
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    cums = {b: [lo, hi] for b in range(wl.batch)}
+    for t, (b, _, hi_pos, _) in enumerate(info):
+        _, res = _reserved_residual(hi_pos + 1, 64, sink, rec)
+        for g in range(wl.num_kv_heads):
+            if not res:
+                continue
+            s = np.array([scores[t, g, j] for j in res])
+            order = sorted(range(len(res)), key=lambda i: (-s[i], res[i]))
+            e = np.exp(s - s.max())
+            e /= e.sum()
+            cums[b] += np.cumsum(e[order]).tolist()
+    ps = []
+    for b in range(wl.batch):
+        c = np.unique(np.clip(np.array(cums[b]), lo, hi))
+        gaps = np.diff(c)
+        k = int(np.argmax(gaps))
+        assert gaps[k] > 2 * margin
+        ps.append(0.5 * (c[k] + c[k + 1]))
+    return torch.as_tensor(np.array(ps, np.float32), device=wl.top_p.device)

@@ -1,0 +1,122 @@
+"""GPU parity of the sparse-prefill path (query tiles of one KV block select
+like a decode query at the tile's end from block scores maxed over the
+tile's queries; causal attention over the selection) through the C ABI,
+against the fp64 oracle.  Rules and tolerances: tests/harness.py."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_spot_b200 as spot
+import oracle
+import workloads
+from harness import (check_prefill_outputs, check_prefill_selection_near_cut,
+                     oracle_prefill_scores, prefill_oracle_args, run_gpu_prefill,
+                     run_oracle_prefill, safe_top_p_prefill, tile_selection)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _same(gpu, ora, wl):
+    assert gpu["num_tiles"] == len(ora["tiles"])
+    assert np.array_equal(gpu["sel_cnt"], ora["sel_cnt"]), (gpu["sel_cnt"], ora["sel_cnt"])
+    for t in range(gpu["num_tiles"]):
+        for g in range(wl.num_kv_heads):
+            assert tile_selection(gpu, t, g) == tile_selection(ora, t, g), (t, g)
+
+
+def test_prefill_tiny():
+    wl = workloads.make_prefill("prefill_tiny", seed=0, device=DEV)
+    gpu = run_gpu_prefill(wl)
+    assert gpu["status"] == 0
+    args = prefill_oracle_args(wl)
+    ora = run_oracle_prefill(wl, args=args)
+    scores = oracle_prefill_scores(wl, args=args)
+    assert check_prefill_selection_near_cut(gpu, ora, scores, wl) <= 1
+    _, n = check_prefill_outputs(gpu, ora, wl)
+    assert n >= gpu["num_tiles"] * wl.num_kv_heads - 1
+
+
+@pytest.mark.parametrize("lens,qlens", [
+    ([1000, 1000], [300, 300]),
+    ([777, 64, 129, 2048, 5], [777, 1, 70, 200, 5]),
+])
+def test_prefill_integer_inputs_select_bit_exact(lens, qlens):
+    wl = workloads.make_prefill("prefill_tiny", seed=3, device=DEV, integer=True, seq_lens=lens,
+                                q_lens=qlens)
+    wl.top_p = safe_top_p_prefill(wl)
+    gpu = run_gpu_prefill(wl)
+    assert gpu["status"] == 0
+    ora = run_oracle_prefill(wl)
+    _same(gpu, ora, wl)
+    check_prefill_outputs(gpu, ora, wl)
+
+
+def test_prefill_keep_all_and_modes():
+    wl = workloads.make_prefill("prefill_tiny", seed=4, device=DEV, integer=True,
+                                seq_lens=[900, 300], q_lens=[250, 300])
+    for kw in (dict(mode="topk", topk=3), dict(kmin=12), dict(sink=100, rec=0),
+               dict(mode="topk", topk=0, sink=0, rec=1)):
+        gpu = run_gpu_prefill(wl, **kw)
+        assert gpu["status"] == 0
+        ora = run_oracle_prefill(wl, **kw)
+        _same(gpu, ora, wl)
+        check_prefill_outputs(gpu, ora, wl)
+    wl.top_p = torch.ones_like(wl.top_p)          # p = 1: dense causal attention
+    gpu = run_gpu_prefill(wl)
+    ora = run_oracle_prefill(wl)
+    _same(gpu, ora, wl)
+    check_prefill_outputs(gpu, ora, wl)
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 2), (12, 4)])
+def test_prefill_group_sizes(hq, hkv):
+    wl = workloads.make_prefill("prefill_tiny", seed=5, device=DEV, num_q_heads=hq,
+                                num_kv_heads=hkv, seq_lens=[600], q_lens=[200])
+    gpu = run_gpu_prefill(wl)
+    assert gpu["status"] == 0
+    args = prefill_oracle_args(wl)
+    ora = run_oracle_prefill(wl, args=args)
+    scores = oracle_prefill_scores(wl, args=args)
+    assert check_prefill_selection_near_cut(gpu, ora, scores, wl) <= 1
+    check_prefill_outputs(gpu, ora, wl)
+
+
+def test_prefill_full_size_sampled_tiles():
+    """Qwen3-8B layer, 32K-token prefill in the benchmark's launch
+    configuration; selection and outputs of sampled tiles against the oracle."""
+    wl = workloads.make_prefill("qwen3_8b_prefill_32k", seed=1, device=DEV)
+    gpu = run_gpu_prefill(wl)
+    assert gpu["status"] == 0
+    nt = gpu["num_tiles"]
+    tiles = [0, 3, nt // 2, nt - 2, nt - 1]
+    args = prefill_oracle_args(wl)
+    ora = run_oracle_prefill(wl, tiles=tiles, args=args)
+    scores = oracle_prefill_scores(wl, tiles=tiles, args=args)
+    n_diff = check_prefill_selection_near_cut(gpu, ora, scores, wl, tiles=tiles)
+    assert n_diff <= 1
+    frac = [gpu["sel_cnt"][t].mean() / (t + 1) for t in tiles]
+    print("selected fraction of sampled tiles", np.round(frac, 3).tolist())
+    _, n = check_prefill_outputs(gpu, ora, wl, tiles=tiles)
+    assert n >= len(tiles) * wl.num_kv_heads - n_diff
+
+
+def test_prefill_bad_page_id_and_small_max_tiles_are_reported():
+    wl = workloads.make_prefill("prefill_tiny", seed=6, device=DEV)
+    wl.page_table[0, 3] = wl.num_pages + 7
+    gpu = run_gpu_prefill(wl)
+    assert gpu["status"] == 5
+    assert np.isfinite(gpu["out"]).all()
+    wl = workloads.make_prefill("prefill_tiny", seed=6, device=DEV)
+    gpu = run_gpu_prefill(wl, max_tiles=2)
+    assert gpu["status"] == 5

@@ -464,6 +464,8 @@ class PrefillSpec:
     kmin_blocks: int = 8
     hot_count: int = 16
     page_order: str = "permuted"
+    q_scale: float = 0.12               # selector query scale: ~45% of a late tile's blocks
+                                        # at p = 0.9 (the tile score is a max over 64 queries)
 
 
 PREFILL_SPECS = {
@@ -544,7 +546,8 @@ def make_prefill(name: str, seed: int = 0, device="cpu", *, seq_lens=None, q_len
         q_sel = _int_bf16((rows, Hq, SEL_DIM), gen, device)
         sel_keys = _int_bf16((num_pages, Hkv, SEL_DIM), gen, device)
     else:
-        q_sel = _normal_bf16((rows, Hq, SEL_DIM), gen, device)
+        q_sel = (torch.randn((rows, Hq, SEL_DIM), generator=gen, device=device) *
+                 spec.q_scale).to(torch.bfloat16)
         sel_keys = _normal_bf16((num_pages, Hkv, SEL_DIM), gen, device)
     k_pool = _normal_bf16((num_pages, Hkv, BLOCK, HEAD_DIM), gen, device)
     v_pool = _normal_bf16((num_pages, Hkv, BLOCK, HEAD_DIM), gen, device)
