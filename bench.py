@@ -43,7 +43,8 @@ HBM_FALLBACK_GBS = 6650.0
 # the same workload (profiles/sparse_decode_kernel_qwen3_32b_128k.md), valid
 # only for the kernel source it was taken on (sha256 prefix of the .cu file).
 NCU_TRAFFIC = {
-    "qwen3_32b_128k": {"bytes": 728988416 + 3467264, "kernel_sha256": "80f7ea5c959e94c5"},
+    "qwen3_32b_128k": {"bytes": 728982528 + 3904768, "kernel_sha256": "82c100300b60004f"},
+    "qwen3_8b_128k_tok": {"bytes": 246840064 + 4134144, "kernel_sha256": "82c100300b60004f"},
 }
 
 
@@ -523,7 +524,9 @@ def run_spot_tok(args, world, rank, local):
             "kernel": "sparse decode (attention + combine)" if dom_sparse else
                       "token selector (scoring + selection)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_kind,
+            "frac": round(achieved / peak, 4),
+            "traffic": measured_traffic(args.workload) if dom_sparse else None,
+            "peak_source": peak_kind,
             "algorithmic_bytes_per_launch": int(kb), "ms_per_launch": round(kms, 5),
         },
         "select_roofline": {
@@ -576,6 +579,206 @@ def cpu_baseline_tok(wl, min_s=10.0, max_s=30.0):
             "kind": "oracle",
             "sample": f"fp64 oracle token-selector decode step of one sequence (all heads), "
                       f"{n} runs, {total:.1f} s; x{sp.layers_sparse} layers"}
+
+
+def prefill_flops(wl, sel_idx: np.ndarray, sel_cnt: np.ndarray):
+    """Algorithmic FLOPs of one sparse-prefill layer from the selection made:
+    attention 4 * 128 per (query, head, attended key) -- QK^T and PV -- and
+    tile scoring 2 * 64 per (query, head, scored block)."""
+    import oracle
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    G = wl.num_q_heads // wl.num_kv_heads
+    attn = 0
+    score = 0
+    for t, (_, lo, hi, _) in enumerate(info):
+        m = lo // 64
+        nq = hi - lo + 1
+        pos = np.arange(lo, hi + 1)
+        n_full = (hi + 1) // 64
+        for g in range(wl.num_kv_heads):
+            sel = sel_idx[t, g, :sel_cnt[t, g]]
+            before = int((sel < m).sum()) * 64
+            keys = before * nq + ((pos - m * 64 + 1).sum() if (sel == m).any() else 0)
+            attn += int(keys) * G * 4 * 128
+            score += nq * G * n_full * 64 * 2
+    return attn, score
+
+
+def run_spot_prefill(args, world, rank, local):
+    """One sparse-prefill layer (plan, tile scoring, selection, attention)
+    per step over the whole chunk."""
+    import block_sparse_long_spot_b200 as spot
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    layers = [workloads.make_prefill(args.workload, seed=layer_seed(rank, l), device=dev)
+              for l in range(args.layers)]
+    wl0 = layers[0]
+    sp = wl0.spec
+    Hq, Hkv, mb = wl0.num_q_heads, wl0.num_kv_heads, wl0.max_blocks
+    nt = spot.prefill_num_tiles(wl0.seq_lens.cpu().numpy(), wl0.q_lens.cpu().numpy())
+    descs = [spot.layer_desc(Hq, Hkv, w.num_pages, "bf16") for w in layers]
+    prm = spot.select_params("topp", sp.sink_blocks, sp.recency_blocks, sp.kmin_blocks)
+    wss = [spot.new_prefill_workspace(d, wl0.batch, nt, mb, dev) for d in descs]
+    rows = int(wl0.q.shape[0])
+    sel_idx = torch.empty(nt, Hkv, mb, dtype=torch.int32, device=dev)
+    sel_cnt = torch.empty(nt, Hkv, dtype=torch.int32, device=dev)
+    out = torch.empty(rows, Hq, 128, dtype=torch.float32, device=dev)
+    lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, q=None, q_sel=None):
+        w = layers[i % len(layers)]
+        spot.prefill(descs[i % len(layers)], prm, w.q_sel if q_sel is None else q_sel, w.w,
+                     w.sel_keys, w.q if q is None else q, w.k_pool, w.v_pool, w.page_table,
+                     w.seq_lens, w.q_lens, w.top_p, w.sm_scale, sel_idx, sel_cnt, out, lse,
+                     wss[i % len(layers)], stream)
+
+    flops = []
+    sel0 = None
+    for l in range(len(layers)):
+        step(l)
+        torch.cuda.synchronize()
+        if l == 0:
+            sel0 = (sel_idx.cpu().numpy(), sel_cnt.cpu().numpy())
+        flops.append(prefill_flops(layers[l], sel_idx.cpu().numpy(), sel_cnt.cpu().numpy()))
+        frac = (sel_cnt.cpu().numpy().astype(np.float64) /
+                (np.arange(nt)[:, None] + 1)).mean()
+    for ws in wss:
+        if spot.read_device_status(ws) != 0:
+            raise RuntimeError("device status after warm-up")
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t0.record(stream)
+        for i in range(K):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / K, world)
+    # end to end: the step's queries (q, q_sel) copied from pinned host memory
+    pin = [(w.q.cpu().pin_memory(), w.q_sel.cpu().pin_memory()) for w in layers]
+    host_out = torch.empty(rows, Hq, 128, dtype=torch.float32).pin_memory()
+    q_dev, qs_dev = torch.empty_like(wl0.q), torch.empty_like(wl0.q_sel)
+
+    def e2e_step(i):
+        hq, hqs = pin[i % len(layers)]
+        q_dev.copy_(hq, non_blocking=True)
+        qs_dev.copy_(hqs, non_blocking=True)
+        step(i, q_dev, qs_dev)
+        host_out.copy_(out, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K, world)
+    for ws in wss:
+        if spot.read_device_status(ws) != 0:
+            raise RuntimeError("device status after timing")
+    nl = len(layers)
+    f_attn = float(np.mean([flops[i % nl][0] for i in range(K)]))
+    f_score = float(np.mean([flops[i % nl][1] for i in range(K)]))
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, peak_kind = float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        peak, peak_kind = 1400.0, "fallback (sustained)"
+    tokens = int(wl0.q_lens.sum().item())
+    value = tokens * world / (ms_step / 1e3 * sp_layers(args))
+    achieved = (f_attn + f_score) / (ms_step / 1e3) / 1e12
+    return {
+        "metric": "prefill tokens/s at L=32K (whole model = per-layer time x layers)",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 with planted hot blocks)",
+        "config": {"workload": args.workload, "batch_per_gpu": wl0.batch, "q_heads": Hq,
+                   "kv_heads": Hkv, "head_dim": 128, "context": int(wl0.seq_lens.max().item()),
+                   "chunk": int(wl0.q_lens.max().item()), "tiles": nt, "block": 64,
+                   "top_p": sp.top_p, "sink_blocks": sp.sink_blocks,
+                   "recency_blocks": sp.recency_blocks, "kmin_blocks": sp.kmin_blocks,
+                   "layers_in_model": sp_layers(args), "layer_caches_rotated": nl,
+                   "selected_fraction_mean": round(float(frac), 4),
+                   "l2": "compute-bound; KV of a layer re-read from L2 by its tiles",
+                   "parallelism": f"dp{world} (sequences)"},
+        "roofline": {"bound": "tensor", "kernel": "sparse prefill (all four kernels)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_flops_per_step": int(f_attn + f_score),
+                     "attention_flops": int(f_attn), "scoring_flops": int(f_score)},
+        "e2e": {"value": round(tokens * world / (ms_e2e / 1e3 * sp_layers(args)), 1),
+                "unit": "tokens/s", "ms_per_step": round(ms_e2e, 4),
+                "h2d_bytes_per_step": int(wl0.q.numel() * 2 + wl0.q_sel.numel() * 2),
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": K * 4,          # plan, tile scores, selection, attention per step
+        "clocks": clk.summary(),
+    }, (layers, sel0[0], sel0[1])
+
+
+def cpu_baseline_prefill(wl, sel_idx, sel_cnt, layers_model):
+    """The fp64 oracle's sparse prefill on the host cores for two tiles (the
+    last and a middle one, all KV heads), scaled to the layer by the share of
+    the layer's attention FLOPs those tiles hold, then to the model."""
+    import oracle
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    nt = len(info)
+    tiles = [nt - 1, nt // 2]
+    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, "bf16",
+                           wl.num_pages, wl.max_blocks)
+    sp = wl.spec
+    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
+                            kmin_blocks=sp.kmin_blocks)
+    args = dict(q_sel=workloads.bits(wl.q_sel), w=None, sel_data=workloads.bits(wl.sel_keys),
+                sel_scales=None, q=workloads.bits(wl.q), k_pool=workloads.bits(wl.k_pool),
+                v_pool=workloads.bits(wl.v_pool), page_table=wl.page_table.cpu().numpy(),
+                seq_lens=wl.seq_lens.cpu().numpy(), q_lens=wl.q_lens.cpu().numpy(),
+                top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
+    t = time.perf_counter()
+    oracle.prefill_step(sh, pr, tiles=tiles, **args)
+    sec = time.perf_counter() - t
+    mask = np.zeros(nt, bool)
+    mask[tiles] = True
+    part = prefill_flops_tiles(wl, sel_idx, sel_cnt, mask)
+    total = prefill_flops_tiles(wl, sel_idx, sel_cnt, np.ones(nt, bool))
+    layer_s = sec * total / max(part, 1)
+    tokens = int(wl.q_lens.sum().item())
+    return {"value": round(tokens / (layer_s * layers_model), 3), "unit": "tokens/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle sparse prefill of tiles {tiles} (all KV heads), {sec:.1f} s, "
+                      f"scaled by attention FLOPs to the {nt} tiles of the layer, "
+                      f"x{layers_model} layers"}
+
+
+def prefill_flops_tiles(wl, sel_idx, sel_cnt, mask):
+    import oracle
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    G = wl.num_q_heads // wl.num_kv_heads
+    total = 0
+    for t, (_, lo, hi, _) in enumerate(info):
+        if not mask[t]:
+            continue
+        m, nq = lo // 64, hi - lo + 1
+        pos = np.arange(lo, hi + 1)
+        for g in range(wl.num_kv_heads):
+            sel = sel_idx[t, g, :sel_cnt[t, g]]
+            keys = int((sel < m).sum()) * 64 * nq + (int((pos - m * 64 + 1).sum())
+                                                     if (sel == m).any() else 0)
+            total += keys * G * 4 * 128
+    return total
+
+
+def sp_layers(args):
+    return 36 if "qwen3_8b" in args.workload else 1
 
 
 def prepare_oracle(wl, fmt, seqs):
@@ -718,8 +921,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     tok = args.workload in workloads.TOK_SPECS
+    pf = args.workload in workloads.PREFILL_SPECS
     if args.sel_fmt is None:
-        args.sel_fmt = "bf16" if tok else workloads.SPECS[args.workload].sel_fmt
+        args.sel_fmt = "bf16" if (tok or pf) else workloads.SPECS[args.workload].sel_fmt
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args.gpus)
     try:
@@ -730,14 +934,20 @@ def main():
             if res is not None:
                 print(json.dumps(res), flush=True)
             return
-        if tok:
+        if pf:
+            res, layers = run_spot_prefill(args, world, rank, local)
+        elif tok:
             res, layers = run_spot_tok(args, world, rank, local)
         else:
             res, layers = run_spot(args, world, rank, local)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = (cpu_baseline_tok(layers[0][0]) if tok else
-                                       cpu_baseline(layers[0][0], args.sel_fmt))
+                if pf:
+                    res["cpu_baseline"] = cpu_baseline_prefill(layers[0][0], layers[1], layers[2],
+                                                               sp_layers(args))
+                else:
+                    res["cpu_baseline"] = (cpu_baseline_tok(layers[0][0]) if tok else
+                                           cpu_baseline(layers[0][0], args.sel_fmt))
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:
