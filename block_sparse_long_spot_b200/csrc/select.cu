@@ -18,7 +18,7 @@
 // Selection: residual softmax numerators exp(s - max) are computed in fp64
 //   and held as 2^-40 fixed-point integers (exact, order-independent sums).
 //   The nucleus cut is a bucketed threshold search: the residual blocks are
-//   histogrammed into 4096 buckets of the score's distance from the maximum,
+//   histogrammed into 1024 or 2048 buckets of the score's distance from the maximum,
 //   scaled so the residual range spans them all (monotone in the score;
 //   exact counts, 2^-18 fixed-point masses), the
 //   bucket where the cumulative mass from the top reaches p * Z is found by a
@@ -349,9 +349,9 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-constexpr int kNB = 4096;              // most value buckets of the first pass (1024 up to
-                                        // 2048 residual blocks, 2048 up to 4096, then 4096),
-                                        // spread over the residual scores' range
+constexpr int kNB = 2048;              // most value buckets of the first pass (1024 up to
+                                        // 2048 residual blocks, then 2048), spread over the
+                                        // residual scores' range
 constexpr int kApproxShift = 18;        // bucket masses for the search: 2^-18 fixed point
                                         // (<= 8192 elements of mass <= 1 fit in 32 bits)
 constexpr int NT = kSelectThreads;
@@ -690,7 +690,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     const int n = r1 - r0;
     const int n_reserved = nb - n;
     const float* s = sm.score;
-    const int nbk = n > 4096 ? 4096 : (n > 2048 ? 2048 : 1024);     // value buckets
+    const int nbk = n > 2048 ? 2048 : 1024;          // value buckets
     for (int i = threadIdx.x; i < nbk; i += NT) { sm.hmass[i] = 0u; sm.hcnt[i] = 0u; }
     if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
     pdl_trigger();                                    // the decode kernel may start its prologue

@@ -29,7 +29,7 @@ namespace spot {
 namespace {
 
 constexpr int NCS = 4;                                          // consumer warps
-constexpr int SST = 8;                                          // pipeline stages
+constexpr int SST = 12;                                         // pipeline stages
 constexpr int kSThreads = (NCS + 1) * 32;
 static_assert(SST % NCS == 0, "each stage must always be consumed by the same warp");
 constexpr int kTokStageBytes = kTokBlock * kIdxHeads * kIdxDim * 2;   // 16 KiB
