@@ -227,18 +227,19 @@ def run_spot(args, world, rank, local):
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(i, ev=None):
+    def step(i, ev=None, st=None):
+        st = stream if st is None else st
         wl, desc, data, scales = layers[i % len(layers)]
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(st)
         spot.select(desc, prm, wl.q_sel, wl.w, data, scales, wl.page_table, wl.seq_lens,
-                    wl.top_p, sel_idx, sel_cnt, ws, stream)
+                    wl.top_p, sel_idx, sel_cnt, ws, st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
         spot.sparse_decode(desc, wl.q, wl.k_pool, wl.v_pool, wl.page_table, wl.seq_lens, sel_idx,
-                           sel_cnt, wl.sm_scale, out, lse, ws, stream)
+                           sel_cnt, wl.sm_scale, out, lse, ws, st)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(st)
 
     # selection statistics and algorithmic bytes per layer
     per_layer = []
@@ -257,21 +258,47 @@ def run_spot(args, world, rank, local):
         step(i)
     torch.cuda.synchronize()
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         t0.record(stream)
         for i in range(K):
-            step(i, evs[i])
+            step(i)
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     ms_total = t0.elapsed_time(t1)
+    ms_step = max_over_ranks(ms_total / K, world)
+    # per-kernel durations in a second pass (events between the two calls keep
+    # them from overlapping, so this pass is not the step time)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(K):
+        step(i, evs[i])
+    torch.cuda.synchronize()
     ms_sel = [e[0].elapsed_time(e[1]) for e in evs]
     ms_dec = [e[1].elapsed_time(e[2]) for e in evs]
-    ms_step = max_over_ranks(ms_total / K, world)
+
+    # ---- the same steps replayed from CUDA graphs (one per layer cache):
+    # the host's per-launch work leaves the timed region
+    cap = torch.cuda.Stream(dev)
+    graphs = []
+    for l in range(len(layers)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            step(l, st=cap)
+        graphs.append(g)
+    for i in range(args.warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for i in range(K):
+        graphs[i % len(graphs)].replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    ms_graph = max_over_ranks(g0.elapsed_time(g1) / K, world)
+    del graphs
 
     # ---- end to end through the public call with host buffers
     pin_q = [layers[l][0].q.cpu().pin_memory() for l in range(len(layers))]
@@ -361,7 +388,10 @@ def run_spot(args, world, rank, local):
                 "ms_per_step": round(ms_e2e, 5),
                 "h2d_bytes_per_step": int(layers[0][0].q.numel() * 2 + layers[0][0].q_sel.numel() * 2),
                 "d2h_bytes_per_step": int(out.numel() * 4)},
-        "gpu_launches": K * 3,          # score, select, sparse decode per step
+        "graph": {"ms_per_step": round(ms_graph, 5),
+                  "value": round(shard_summary(B, world, ms_graph, layers_model), 3),
+                  "note": "the same steps replayed from captured CUDA graphs"},
+        "gpu_launches": K * 2,          # selection (scoring fused), sparse decode per step
         "clocks": clk.summary(),
     }
     return res, layers
@@ -439,18 +469,22 @@ def run_spot_tok(args, world, rank, local):
         step(i)
     torch.cuda.synchronize()
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         t0.record(stream)
         for i in range(K):
-            step(i, evs[i])
+            step(i)
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     ms_step = max_over_ranks(t0.elapsed_time(t1) / K, world)
+    # per-kernel durations in a second pass (not the step time)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(K):
+        step(i, evs[i])
+    torch.cuda.synchronize()
     sel_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     dec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
 

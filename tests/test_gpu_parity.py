@@ -382,3 +382,46 @@ def test_workspace_too_small_and_bad_arguments():
         spot.select(bad, prm, wl.q_sel, None, wl.sel_keys, None, wl.page_table, wl.seq_lens,
                     wl.top_p, sel_idx, sel_cnt, ws)
     assert e.value.code == 1
+
+
+def test_decode_step_captured_in_a_cuda_graph():
+    """spot_decode_step is capture-safe: one capture, replayed on new
+    queries copied into the captured buffers, matches the oracle."""
+    wl = workloads.make("tiny_4k", seed=21, device=DEV)
+    desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, "bf16")
+    prm = spot.select_params("topp", wl.spec.sink_blocks, wl.spec.recency_blocks,
+                             wl.spec.kmin_blocks)
+    B, Hq, Hkv, mb = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.max_blocks
+    ws = spot.new_workspace(desc, B, mb, DEV)
+    q, q_sel = wl.q.clone(), wl.q_sel.clone()
+    sel_idx = torch.full((B, Hkv, mb), -1, dtype=torch.int32, device=DEV)
+    sel_cnt = torch.zeros((B, Hkv), dtype=torch.int32, device=DEV)
+    out = torch.zeros((B, Hq, 128), dtype=torch.float32, device=DEV)
+    lse = torch.zeros((B, Hq), dtype=torch.float32, device=DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        spot.decode_step(desc, prm, q_sel, wl.w, wl.sel_keys, None, q, wl.k_pool, wl.v_pool,
+                         wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt,
+                         out, lse, ws, s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        spot.decode_step(desc, prm, q_sel, wl.w, wl.sel_keys, None, q, wl.k_pool, wl.v_pool,
+                         wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt,
+                         out, lse, ws, s)
+    for seed in (22, 23):
+        other = workloads.make("tiny_4k", seed=seed, device=DEV)
+        wl2 = workloads.make("tiny_4k", seed=21, device=DEV)
+        wl2.q, wl2.q_sel = other.q, other.q_sel
+        q.copy_(other.q)
+        q_sel.copy_(other.q_sel)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert spot.read_device_status(ws) == 0
+        gpu = {"sel_idx": sel_idx.cpu().numpy(), "sel_cnt": sel_cnt.cpu().numpy(),
+               "out": out.cpu().double().numpy(), "lse": lse.cpu().double().numpy()}
+        ora = run_oracle(wl2)
+        assert check_selection_near_cut(gpu, ora, oracle_scores(wl2), wl2) == 0
+        _, _, n = check_outputs(gpu, ora, wl2)
+        assert n == B * Hkv
+    del graph
