@@ -64,7 +64,7 @@ class Params(ctypes.Structure):
 class TokShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "num_q_heads", "num_kv_heads", "head_dim", "page_size", "idx_heads", "idx_dim",
-        "sel_block", "num_pages", "max_pages", "max_blocks")]
+        "sel_block", "num_pages", "max_pages", "max_blocks", "sel_fmt")]
 
 
 def _load():
@@ -81,8 +81,8 @@ def _load():
         lib.oracle_sparse_attention.argtypes = [P, P, P, P, P, P, P, P, dbl, P, P]
         lib.oracle_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
                                            P, P, P, P, P]
-        lib.oracle_tok_block_scores.argtypes = [P, P, P, P, P, P, P, P]
-        lib.oracle_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
+        lib.oracle_tok_block_scores.argtypes = [P, P, P, P, P, P, P, P, P]
+        lib.oracle_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
                                                P, P, P, P, P]
         lib.oracle_prefill_num_tiles.argtypes = [P, P, P]
         lib.oracle_prefill_num_tiles.restype = i64
@@ -230,27 +230,36 @@ def decode_step(shape: Shape, params: Params, q_sel, w, sel_data, sel_scales, q,
 
 def make_tok_shape(batch, num_q_heads, num_kv_heads, num_pages, max_pages, head_dim=128,
                    page_size=64, idx_heads=4, idx_dim=128, sel_block=16,
-                   max_blocks=None) -> TokShape:
+                   max_blocks=None, sel_fmt="bf16") -> TokShape:
     mb = max_pages * (page_size // sel_block) if max_blocks is None else max_blocks
     return TokShape(batch, num_q_heads, num_kv_heads, head_dim, page_size, idx_heads, idx_dim,
-                    sel_block, num_pages, max_pages, mb)
+                    sel_block, num_pages, max_pages, mb,
+                    FMT[sel_fmt] if isinstance(sel_fmt, str) else sel_fmt)
+
+
+def _tok_pool(shape, sel_tok, sel_scales):
+    fmt = _FMT_NAME[shape.sel_fmt]
+    return (_c(sel_tok, _data_dtype(fmt)),
+            None if sel_scales is None else _c(sel_scales, _scale_dtype(fmt)))
 
 
 def tok_block_scores(shape: TokShape, params: Params, q_idx, w, sel_tok, page_table,
-                     seq_lens) -> np.ndarray:
+                     seq_lens, sel_scales=None) -> np.ndarray:
     """Block scores [B, max_blocks] of the token-level selector (max over
-    each block's token scores; NaN where no complete block)."""
+    each block's token scores; NaN where no complete block).  sel_tok /
+    sel_scales: the per-token key pool in the shape's format."""
     scores = np.full((shape.batch, shape.max_blocks), np.nan)
+    data, scales = _tok_pool(shape, sel_tok, sel_scales)
     rc = _load().oracle_tok_block_scores(
         ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_idx, np.uint16)),
-        _ptr(_c(w, np.float32)), _ptr(_c(sel_tok, np.uint16)), _ptr(_c(page_table, np.int32)),
+        _ptr(_c(w, np.float32)), _ptr(data), _ptr(scales), _ptr(_c(page_table, np.int32)),
         _ptr(_c(seq_lens, np.int32)), _ptr(scores))
     assert rc == 0
     return scores
 
 
 def tok_decode_step(shape: TokShape, params: Params, q_idx, w, sel_tok, q, k_pool, v_pool,
-                    page_table, seq_lens, top_p, sm_scale, seqs=None):
+                    page_table, seq_lens, top_p, sm_scale, seqs=None, sel_scales=None):
     """Decode step of the token-level selector for sequences `seqs` (default
     all): one selection per sequence shared by every head."""
     B, Hq = shape.batch, shape.num_q_heads
@@ -260,9 +269,10 @@ def tok_decode_step(shape: TokShape, params: Params, q_idx, w, sel_tok, q, k_poo
     out = np.zeros((B, Hq, shape.head_dim))
     lse = np.zeros((B, Hq))
     sq = None if seqs is None else _c(seqs, np.int32)
+    data, scales = _tok_pool(shape, sel_tok, sel_scales)
     rc = _load().oracle_tok_decode_step(
         ctypes.byref(shape), ctypes.byref(params), _ptr(_c(q_idx, np.uint16)),
-        _ptr(_c(w, np.float32)), _ptr(_c(sel_tok, np.uint16)), _ptr(_c(q, np.uint16)),
+        _ptr(_c(w, np.float32)), _ptr(data), _ptr(scales), _ptr(_c(q, np.uint16)),
         _ptr(_c(k_pool, np.uint16)), _ptr(_c(v_pool, np.uint16)), _ptr(_c(page_table, np.int32)),
         _ptr(_c(seq_lens, np.int32)), _ptr(_c(top_p, np.float32)), float(sm_scale), _ptr(sq),
         0 if sq is None else len(sq), _ptr(sel_idx), _ptr(sel_cnt), _ptr(mass), _ptr(out),

@@ -825,7 +825,36 @@ typedef struct {
     int32_t num_pages;
     int32_t max_pages;       /* page-table row stride */
     int32_t max_blocks;      /* selection row stride (sel_idx, scores) */
+    int32_t sel_fmt;         /* ORC_FMT_*: each (token, head) key row of d_idx elements is
+                                stored like a selector key row (oracle_dequant_selector) */
 } orc_tok_shape_t;
+
+/* Exact values of key row `row` (= (page * page_size + slot) * H_idx + h) of
+ * a per-token selector pool stored in sh->sel_fmt. */
+static int tok_key_row(const orc_tok_shape_t* sh, const void* data, const void* scales,
+                       int64_t row, double* out) {
+    int di = sh->idx_dim;
+    switch (sh->sel_fmt) {
+        case ORC_FMT_BF16:
+            return oracle_dequant_selector(ORC_FMT_BF16, 1, di,
+                                           (const uint16_t*)data + row * di, NULL, out);
+        case ORC_FMT_FP8:
+            return oracle_dequant_selector(ORC_FMT_FP8, 1, di,
+                                           (const uint8_t*)data + row * di, NULL, out);
+        case ORC_FMT_INT8:
+            return oracle_dequant_selector(ORC_FMT_INT8, 1, di, (const int8_t*)data + row * di,
+                                           (const uint16_t*)scales + row, out);
+        case ORC_FMT_INT4:
+            return oracle_dequant_selector(ORC_FMT_INT4, 1, di,
+                                           (const uint8_t*)data + row * (di / 2),
+                                           (const uint16_t*)scales + row * (di / 32), out);
+        case ORC_FMT_MXFP4:
+            return oracle_dequant_selector(ORC_FMT_MXFP4, 1, di,
+                                           (const uint8_t*)data + row * (di / 2),
+                                           (const uint8_t*)scales + row * (di / 32), out);
+    }
+    return -1;
+}
 
 /* Score of every complete selection block of sequence b (§2.1 and §2.3):
  * the token score s[t] = (1/tau) sum_h w_h ReLU(q^I_h . k^I_{h,t}) with one
@@ -833,11 +862,14 @@ typedef struct {
  * tokens' scores.  Token t's keys sit in sel_tok[page][t % ps][h][d_idx]
  * with page = page_table[b][t / ps].  w (NULL -> 1/H_idx) is [B][H_idx].
  * Writes n_full = floor(seq_len / sel_block) scores into out. */
-static void tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, int b,
-                            const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
-                            const int32_t* page_table, int32_t seq_len, double* out) {
+static int tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, int b,
+                           const uint16_t* q_idx, const float* w, const void* sel_tok,
+                           const void* sel_scales, const int32_t* page_table, int32_t seq_len,
+                           double* out) {
     int Hi = sh->idx_heads, di = sh->idx_dim, sb = sh->sel_block, ps = sh->page_size;
     int64_t n_full = seq_len / sb;
+    double* k = (double*)malloc((size_t)di * sizeof(double));
+    if (!k) return -2;
     for (int64_t j = 0; j < n_full; ++j) {
         double best = -INFINITY;
         for (int64_t t = j * sb; t < (j + 1) * sb; ++t) {
@@ -845,9 +877,13 @@ static void tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, i
             double s = 0.0;
             for (int h = 0; h < Hi; ++h) {
                 const uint16_t* q = q_idx + ((int64_t)b * Hi + h) * di;
-                const uint16_t* k = sel_tok + (((int64_t)page * ps + t % ps) * Hi + h) * di;
+                if (tok_key_row(sh, sel_tok, sel_scales,
+                                ((int64_t)page * ps + t % ps) * Hi + h, k)) {
+                    free(k);
+                    return -1;
+                }
                 double dot = 0.0;
-                for (int d = 0; d < di; ++d) dot += bf16_to_f64(q[d]) * bf16_to_f64(k[d]);
+                for (int d = 0; d < di; ++d) dot += bf16_to_f64(q[d]) * k[d];
                 double wh = w ? (double)w[(int64_t)b * Hi + h] : 1.0 / Hi;
                 s += wh * (dot > 0.0 ? dot : 0.0);
             }
@@ -856,17 +892,21 @@ static void tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, i
         }
         out[j] = best;
     }
+    free(k);
+    return 0;
 }
 
 /* Block scores [B][max_blocks] of the token-level selector; entries past
  * each sequence's complete blocks are left untouched. */
 int oracle_tok_block_scores(const orc_tok_shape_t* sh, const orc_params_t* pr,
-                            const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
-                            const int32_t* page_table, const int32_t* seq_lens, double* scores) {
+                            const uint16_t* q_idx, const float* w, const void* sel_tok,
+                            const void* sel_scales, const int32_t* page_table,
+                            const int32_t* seq_lens, double* scores) {
     if (sh->sel_block <= 0 || sh->page_size % sh->sel_block != 0) return -1;
     for (int b = 0; b < sh->batch; ++b)
-        tok_unit_scores(sh, pr, b, q_idx, w, sel_tok, page_table, seq_lens[b],
-                        scores + (int64_t)b * sh->max_blocks);
+        if (tok_unit_scores(sh, pr, b, q_idx, w, sel_tok, sel_scales, page_table, seq_lens[b],
+                            scores + (int64_t)b * sh->max_blocks))
+            return -1;
     return 0;
 }
 
@@ -877,8 +917,8 @@ int oracle_tok_block_scores(const orc_tok_shape_t* sh, const orc_params_t* pr,
  * in the full problem: sel_idx[b][max_blocks], sel_cnt[b], nuc_mass[b] (may
  * be NULL), out[b][h][D], lse[b][h]. */
 int oracle_tok_decode_step(const orc_tok_shape_t* sh, const orc_params_t* pr,
-                           const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
-                           const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                           const uint16_t* q_idx, const float* w, const void* sel_tok,
+                           const void* sel_scales, const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
                            const int32_t* page_table, const int32_t* seq_lens,
                            const float* top_p, double sm_scale, const int32_t* seqs,
                            int32_t n_seqs, int32_t* sel_idx, int32_t* sel_cnt, double* nuc_mass,
@@ -902,7 +942,14 @@ int oracle_tok_decode_step(const orc_tok_shape_t* sh, const orc_params_t* pr,
             err = -2;
             continue;
         }
-        tok_unit_scores(sh, pr, b, q_idx, w, sel_tok, page_table, L, s);
+        if (tok_unit_scores(sh, pr, b, q_idx, w, sel_tok, sel_scales, page_table, L, s)) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = -1;
+            free(s);
+            continue;
+        }
         int32_t* sel = sel_idx + (int64_t)b * sh->max_blocks;
         double mass = 0.0;
         int32_t cnt = oracle_select_from_scores(s, (int32_t)nb, (int32_t)n_full, pr,

@@ -782,3 +782,31 @@ def test_prefill_causal_mask_and_tile_recency():
     r400 = 400 - 382
     assert np.array_equal(base["out"][:r400 + 1], pert["out"][:r400 + 1])
     assert not np.allclose(base["out"][r400 + 1:], pert["out"][r400 + 1:])
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "fp8", "int8"])
+def test_tok_quantised_keys_follow_the_key_quantiser(fmt):
+    # Each (token, head) key row of 128 elements is stored like a selector
+    # key row of that format (pinned quantiser above); the scores are the
+    # plain token scores of the read-back rows, maxed over 16-token blocks.
+    rng = np.random.default_rng(30)
+    P, Hi, L = 3, 2, 150
+    keys = _bf16_bits(rng.normal(size=(P, 64, Hi, 128)))
+    data, scales = oracle.quantize_selector(fmt, keys)
+    q = _bf16_bits(rng.normal(size=(1, Hi, 128)) * 0.3)
+    w = np.array([[0.7, 0.4]], np.float32)
+    pt = np.array([[2, 0, 1]], np.int32)
+    sh = oracle.make_tok_shape(1, 4, 2, P, 3, idx_heads=Hi, sel_fmt=fmt)
+    got = oracle.tok_block_scores(sh, oracle.make_params(), q, w, data, pt,
+                                  np.array([L], np.int32), sel_scales=scales)
+    kd = oracle.dequant_selector(fmt, data.reshape(-1, data.shape[-1]),
+                                 None if scales is None else scales.reshape(-1, scales.shape[-1]),
+                                 128).reshape(P, 64, Hi, 128)
+    qd = torch.as_tensor(q.view(np.int16)).view(torch.bfloat16).double().numpy()[0]
+    for j in range(L // 16):
+        tok = []
+        for t in range(16 * j, 16 * j + 16):
+            dots = np.einsum("hd,hd->h", qd, kd[pt[0, t // 64], t % 64])
+            tok.append(float((w[0] * np.maximum(dots, 0.0)).sum()))
+        assert abs(got[0, j] - max(tok)) <= 1e-12 * max(1.0, abs(max(tok))), j
+    assert np.isnan(got[0, L // 16:]).all()
