@@ -397,14 +397,22 @@ def run_spot(args, world, rank, local):
     return res, layers
 
 
-def tok_step_bytes(wl, sel_cnt: np.ndarray):
+def tok_row_bytes(fmt: str, idx_dim: int = 128) -> int:
+    """Bytes of one stored per-token selector key row (codes + scales)."""
+    return {"bf16": 2 * idx_dim, "fp8": idx_dim, "int8": idx_dim + 2,
+            "int4": idx_dim // 2 + 2 * (idx_dim // 32),
+            "mxfp4": idx_dim // 2 + idx_dim // 32}[fmt]
+
+
+def tok_step_bytes(wl, sel_cnt: np.ndarray, fmt: str = "bf16"):
     """Algorithmic HBM bytes of one token-selector decode step: the
-    per-token selector keys of every complete 16-token block, the K and V
-    rows of the selected tokens for every KV head, indices and queries."""
+    per-token selector keys of every complete 16-token block (codes and
+    scales of the stored format), the K and V rows of the selected tokens
+    for every KV head, indices and queries."""
     B, Hq, Hkv, sb = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.spec.sel_block
     lens = wl.seq_lens.cpu().numpy().astype(np.int64)
     n_full = lens // sb
-    sel_cache = int(n_full.sum()) * sb * wl.spec.idx_heads * wl.spec.idx_dim * 2
+    sel_cache = int(n_full.sum()) * sb * wl.spec.idx_heads * tok_row_bytes(fmt, wl.spec.idx_dim)
     kv = int(sel_cnt.sum()) * sb * Hkv * 128 * 2 * 2
     part = lens % sb != 0                     # the partial last block is always selected
     kv -= int((Hkv * (sb - lens[part] % sb) * 128 * 2 * 2).sum())
@@ -417,16 +425,44 @@ def tok_step_bytes(wl, sel_cnt: np.ndarray):
             "selector": sel_cache}
 
 
+def sel_pool_bytes(pool) -> int:
+    return sum(t.numel() * t.element_size() for t in pool if t is not None)
+
+
+def tok_pool(spot, wl, desc, fmt):
+    """The layer's per-token selector pool in `fmt`: the workload's bf16
+    keys as they are, or written through the library's quantising append
+    (every cached token, by sequence and position)."""
+    if fmt == "bf16":
+        return wl.sel_tok, None
+    dev = wl.q.device
+    data, scales = spot.tok_selector_pool(wl.num_pages, fmt, device=dev)
+    lens = wl.seq_lens.cpu().numpy()
+    pt = wl.page_table.cpu().numpy()
+    seq = np.concatenate([np.full(int(L), b) for b, L in enumerate(lens)]).astype(np.int32)
+    pos = np.concatenate([np.arange(int(L)) for L in lens]).astype(np.int32)
+    page = torch.as_tensor(pt[seq, pos // 64].astype(np.int64), device=dev)
+    keys = wl.sel_tok[page, torch.as_tensor(pos % 64, device=dev).long()].contiguous()
+    spot.tok_append_selector_keys(desc, data, scales, wl.page_table,
+                                  torch.as_tensor(seq, device=dev),
+                                  torch.as_tensor(pos, device=dev), keys)
+    torch.cuda.synchronize()
+    return data, scales
+
+
 def run_spot_tok(args, world, rank, local):
     """The token-level, layer-shared selector path (tok_select, then
     tok_sparse_decode), timed like run_spot."""
     import block_sparse_long_spot_b200 as spot
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
-    layers = []
+    fmt = args.sel_fmt
+    layers, pools = [], []
     for l in range(args.layers):
         wl = workloads.make_tok(args.workload, seed=layer_seed(rank, l), device=dev)
-        layers.append((wl, spot.tok_layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages)))
+        desc = spot.tok_layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, sel_fmt=fmt)
+        layers.append((wl, desc))
+        pools.append(tok_pool(spot, wl, desc, fmt))
     wl0, desc0 = layers[0]
     B, Hq, mb = wl0.batch, wl0.num_q_heads, wl0.max_blocks
     sp = wl0.spec
@@ -442,9 +478,10 @@ def run_spot_tok(args, world, rank, local):
     def step(i, ev=None):
         wl, desc = layers[i % len(layers)]
         ws = wss[i % len(layers)]
+        sd, ss = pools[i % len(layers)]
         if ev is not None:
             ev[0].record(stream)
-        spot.tok_select(desc, prm, wl.q_idx, wl.w_idx, wl.sel_tok, wl.page_table, wl.seq_lens,
+        spot.tok_select(desc, prm, wl.q_idx, wl.w_idx, sd, ss, wl.page_table, wl.seq_lens,
                         wl.top_p, sel_idx, sel_cnt, ws, stream)
         if ev is not None:
             ev[1].record(stream)
@@ -460,7 +497,7 @@ def run_spot_tok(args, world, rank, local):
         cnt = sel_cnt.cpu().numpy().copy()
         wl = layers[l][0]
         nb = (wl.seq_lens.cpu().numpy() + sp.sel_block - 1) // sp.sel_block
-        per_layer.append((tok_step_bytes(wl, cnt), cnt / np.maximum(nb, 1)))
+        per_layer.append((tok_step_bytes(wl, cnt, fmt), cnt / np.maximum(nb, 1)))
     for ws in wss:
         status = spot.read_device_status(ws)
         if status != 0:
@@ -495,9 +532,10 @@ def run_spot_tok(args, world, rank, local):
 
     def e2e_step(i):
         wl, desc = layers[i % len(layers)]
+        sd, ss = pools[i % len(layers)]
         q_dev.copy_(pin_q[i % len(layers)], non_blocking=True)
         qi_dev.copy_(pin_qi[i % len(layers)], non_blocking=True)
-        spot.tok_decode_step(desc, prm, qi_dev, wl.w_idx, wl.sel_tok, q_dev, wl.k_pool,
+        spot.tok_decode_step(desc, prm, qi_dev, wl.w_idx, sd, ss, q_dev, wl.k_pool,
                              wl.v_pool, wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale,
                              sel_idx, sel_cnt, out, lse, wss[i % len(layers)], stream)
         host_out.copy_(out, non_blocking=True)
@@ -542,12 +580,12 @@ def run_spot_tok(args, world, rank, local):
             "workload": args.workload, "selector": "token-level, layer-shared",
             "batch_per_gpu": B, "q_heads": Hq, "kv_heads": wl0.num_kv_heads, "head_dim": 128,
             "idx_heads": sp.idx_heads, "idx_dim": sp.idx_dim, "sel_block": sp.sel_block,
-            "context": int(wl0.seq_lens.max().item()), "sel_fmt": "bf16",
+            "context": int(wl0.seq_lens.max().item()), "sel_fmt": fmt,
             "top_p": float(wl0.top_p[0].item()), "sink_blocks": sp.sink_blocks,
             "recency_blocks": sp.recency_blocks, "kmin_blocks": sp.kmin_blocks,
             "layers_in_model": layers_model, "layer_caches_rotated": nl,
             "l2": f"inputs larger than L2: {nl} layer caches of "
-                  f"{(wl0.k_pool.numel() * 4 + wl0.sel_tok.numel() * 2) / 1e9:.2f} GB rotated",
+                  f"{(wl0.k_pool.numel() * 4 + sel_pool_bytes(pools[0])) / 1e9:.2f} GB rotated",
             "selected_fraction": {"mean": round(float(frac_sel.mean()), 4),
                                   "min": round(float(frac_sel.min()), 4),
                                   "max": round(float(frac_sel.max()), 4)},
@@ -584,21 +622,32 @@ def run_spot_tok(args, world, rank, local):
     }, layers
 
 
-def cpu_baseline_tok(wl, min_s=10.0, max_s=30.0):
+def tok_oracle_inputs(wl, fmt="bf16"):
+    """(shape, params, arguments) of the oracle's token-selector decode step
+    for a workload, the selector keys quantised by the oracle to `fmt`."""
+    import oracle
+    sp = wl.spec
+    sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
+                               wl.max_pages, sel_fmt=fmt)
+    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
+                            kmin_blocks=sp.kmin_blocks)
+    bits = workloads.bits(wl.sel_tok)
+    data, scales = (bits, None) if fmt == "bf16" else oracle.quantize_selector(fmt, bits)
+    a = dict(q_idx=workloads.bits(wl.q_idx),
+             w=None if wl.w_idx is None else wl.w_idx.cpu().numpy(),
+             sel_tok=data, sel_scales=scales, q=workloads.bits(wl.q),
+             k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
+             page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
+             top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
+    return sh, pr, a
+
+
+def cpu_baseline_tok(wl, fmt="bf16", min_s=10.0, max_s=30.0):
     """The fp64 oracle's token-selector decode step on the host cores, one
     sequence at a time, until about 10 s of work; scaled to the model."""
     import oracle
     sp = wl.spec
-    sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
-                               wl.max_pages)
-    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
-                            kmin_blocks=sp.kmin_blocks)
-    a = dict(q_idx=workloads.bits(wl.q_idx),
-             w=None if wl.w_idx is None else wl.w_idx.cpu().numpy(),
-             sel_tok=workloads.bits(wl.sel_tok), q=workloads.bits(wl.q),
-             k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
-             page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
-             top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
+    sh, pr, a = tok_oracle_inputs(wl, fmt)
     total, n = 0.0, 0
     while total < min_s and n < 64:
         t = time.perf_counter()
@@ -910,16 +959,7 @@ def run_reference_tok(args, world, rank):
     wl = workloads.make_tok(args.workload, seed=0, device=dev)
     times = []
     sp = wl.spec
-    sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
-                               wl.max_pages)
-    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
-                            kmin_blocks=sp.kmin_blocks)
-    a = dict(q_idx=workloads.bits(wl.q_idx),
-             w=None if wl.w_idx is None else wl.w_idx.cpu().numpy(),
-             sel_tok=workloads.bits(wl.sel_tok), q=workloads.bits(wl.q),
-             k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
-             page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
-             top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
+    sh, pr, a = tok_oracle_inputs(wl, args.sel_fmt)
     for i in range(args.warmup + args.steps):
         t = time.perf_counter()
         oracle.tok_decode_step(sh, pr, seqs=[i % wl.batch], **a)
@@ -935,7 +975,7 @@ def run_reference_tok(args, world, rank):
         "warmup": args.warmup, "ms_per_step": round(per_layer * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 with planted hot 16-token blocks)",
-        "config": {"workload": args.workload, "sel_fmt": "bf16", "sample": sample},
+        "config": {"workload": args.workload, "sel_fmt": args.sel_fmt, "sample": sample},
         "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s",
                          "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -980,7 +1020,7 @@ def main():
                     res["cpu_baseline"] = cpu_baseline_prefill(layers[0][0], layers[1], layers[2],
                                                                sp_layers(args))
                 else:
-                    res["cpu_baseline"] = (cpu_baseline_tok(layers[0][0]) if tok else
+                    res["cpu_baseline"] = (cpu_baseline_tok(layers[0][0], args.sel_fmt) if tok else
                                            cpu_baseline(layers[0][0], args.sel_fmt))
             print(json.dumps(res), flush=True)
     finally:

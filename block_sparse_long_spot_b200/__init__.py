@@ -51,13 +51,14 @@ class SelectParams(ctypes.Structure):
 class TokLayerDesc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_q_heads", "num_kv_heads", "head_dim", "page_size", "idx_heads", "idx_dim",
-        "sel_block", "num_pages")]
+        "sel_block", "num_pages", "sel_fmt")]
 
 
 def tok_layer_desc(num_q_heads, num_kv_heads, num_pages, head_dim=128, page_size=64,
-                   idx_heads=4, idx_dim=128, sel_block=16) -> TokLayerDesc:
+                   idx_heads=4, idx_dim=128, sel_block=16, sel_fmt="bf16") -> TokLayerDesc:
     return TokLayerDesc(num_q_heads, num_kv_heads, head_dim, page_size, idx_heads, idx_dim,
-                        sel_block, num_pages)
+                        sel_block, num_pages,
+                        SEL_FMT[sel_fmt] if isinstance(sel_fmt, str) else int(sel_fmt))
 
 
 def layer_desc(num_q_heads, num_kv_heads, num_pages, sel_fmt="bf16", head_dim=128,
@@ -97,12 +98,12 @@ def lib():
                                                  P, P]
         L.spot_tok_workspace_size.argtypes = [P, i32, i32]
         L.spot_tok_workspace_size.restype = sz
-        L.spot_tok_append_selector_keys.argtypes = [P, P, P, i32, i32, P, P, P, i32, P, P]
-        L.spot_tok_select.argtypes = [P, P, P, P, P, P, i32, P, P, i32, P, P, i32, P, sz, P]
+        L.spot_tok_append_selector_keys.argtypes = [P, P, P, P, i32, i32, P, P, P, i32, P, P]
+        L.spot_tok_select.argtypes = [P, P, P, P, P, P, P, i32, P, P, i32, P, P, i32, P, sz, P]
         L.spot_tok_sparse_decode.argtypes = [P, P, P, P, P, i32, P, P, P, i32, i32, f32, P, P,
                                              P, sz, P]
-        L.spot_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, P, i32, f32, P, P,
-                                           i32, P, P, P, sz, P]
+        L.spot_tok_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, P, P, i32, f32, P,
+                                           P, i32, P, P, P, sz, P]
         L.spot_prefill_num_tiles.argtypes = [P, P, i32]
         L.spot_prefill_num_tiles.restype = ctypes.c_int64
         L.spot_prefill_workspace_size.argtypes = [P, i32, i32, i32]
@@ -253,18 +254,31 @@ def new_tok_workspace(desc: TokLayerDesc, batch: int, max_blocks: int, device=No
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def tok_selector_pool(num_pages: int, page_size=64, idx_heads=4, idx_dim=128, device="cuda"):
-    """Empty per-token selector pool bf16 [pages, page_size, idx_heads, idx_dim]."""
-    return torch.zeros(num_pages, page_size, idx_heads, idx_dim, dtype=torch.bfloat16,
-                       device=device)
+def tok_selector_pool(num_pages: int, fmt: str = "bf16", page_size=64, idx_heads=4, idx_dim=128,
+                      device="cuda"):
+    """Empty per-token selector pool (data, scales) for a format: key rows
+    [pages, page_size, idx_heads, row] and their scales (None for bf16 /
+    FP8)."""
+    lead = (num_pages, page_size, idx_heads)
+    if fmt == "bf16":
+        return torch.zeros(*lead, idx_dim, dtype=torch.bfloat16, device=device), None
+    if fmt == "fp8":
+        return torch.zeros(*lead, idx_dim, dtype=torch.uint8, device=device), None
+    if fmt == "int8":
+        return (torch.zeros(*lead, idx_dim, dtype=torch.int8, device=device),
+                torch.zeros(*lead, 1, dtype=torch.float16, device=device))
+    data = torch.zeros(*lead, idx_dim // 2, dtype=torch.uint8, device=device)
+    sdt = torch.float16 if fmt == "int4" else torch.uint8
+    return data, torch.zeros(*lead, idx_dim // 32, dtype=sdt, device=device)
 
 
-def tok_append_selector_keys(desc: TokLayerDesc, sel_tok, page_table, seq_ids, positions, keys,
-                             status_ws=None, stream=None):
-    """Write per-token selector keys bf16 [n, idx_heads, idx_dim] by position."""
+def tok_append_selector_keys(desc: TokLayerDesc, sel_data, sel_scales, page_table, seq_ids,
+                             positions, keys, status_ws=None, stream=None):
+    """Write (quantising to the pool's format) per-token selector keys bf16
+    [n, idx_heads, idx_dim] by position."""
     pt = page_table
     code = lib().spot_tok_append_selector_keys(
-        ctypes.byref(desc), _ptr(sel_tok, torch.bfloat16, "sel_tok"),
+        ctypes.byref(desc), _ptr(sel_data, name="sel_data"), _ptr(sel_scales, name="sel_scales"),
         _ptr(pt, torch.int32, "page_table"), int(pt.shape[0]), int(pt.shape[-1]),
         _ptr(seq_ids, torch.int32, "seq_ids"), _ptr(positions, torch.int32, "positions"),
         _ptr(keys, torch.bfloat16, "keys"), int(keys.shape[0]),
@@ -272,13 +286,14 @@ def tok_append_selector_keys(desc: TokLayerDesc, sel_tok, page_table, seq_ids, p
     _check(code, "tok_append_selector_keys")
 
 
-def tok_select(desc: TokLayerDesc, params: SelectParams, q_idx, w_idx, sel_tok, page_table,
-               seq_lens, top_p, sel_idx, sel_cnt, workspace, stream=None):
+def tok_select(desc: TokLayerDesc, params: SelectParams, q_idx, w_idx, sel_data, sel_scales,
+               page_table, seq_lens, top_p, sel_idx, sel_cnt, workspace, stream=None):
     """One selection per sequence into sel_idx int32 [B, max_blocks], sel_cnt int32 [B]."""
     B, max_blocks = int(q_idx.shape[0]), int(sel_idx.shape[-1])
     code = lib().spot_tok_select(
         ctypes.byref(desc), ctypes.byref(params), _ptr(q_idx, torch.bfloat16, "q_idx"),
-        _ptr(w_idx, torch.float32, "w_idx"), _ptr(sel_tok, torch.bfloat16, "sel_tok"),
+        _ptr(w_idx, torch.float32, "w_idx"), _ptr(sel_data, name="sel_data"),
+        _ptr(sel_scales, name="sel_scales"),
         _ptr(page_table, torch.int32, "page_table"), int(page_table.shape[-1]),
         _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(top_p, torch.float32, "top_p"), B,
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
@@ -302,14 +317,15 @@ def tok_sparse_decode(desc: TokLayerDesc, q, k_pool, v_pool, page_table, seq_len
     _check(code, "tok_sparse_decode")
 
 
-def tok_decode_step(desc: TokLayerDesc, params: SelectParams, q_idx, w_idx, sel_tok, q, k_pool,
-                    v_pool, page_table, seq_lens, top_p, softmax_scale, sel_idx, sel_cnt, out,
-                    lse, workspace, stream=None):
+def tok_decode_step(desc: TokLayerDesc, params: SelectParams, q_idx, w_idx, sel_data,
+                    sel_scales, q, k_pool, v_pool, page_table, seq_lens, top_p, softmax_scale,
+                    sel_idx, sel_cnt, out, lse, workspace, stream=None):
     """tok_select followed by tok_sparse_decode on one stream."""
     B, max_blocks = int(q.shape[0]), int(sel_idx.shape[-1])
     code = lib().spot_tok_decode_step(
         ctypes.byref(desc), ctypes.byref(params), _ptr(q_idx, torch.bfloat16, "q_idx"),
-        _ptr(w_idx, torch.float32, "w_idx"), _ptr(sel_tok, torch.bfloat16, "sel_tok"),
+        _ptr(w_idx, torch.float32, "w_idx"), _ptr(sel_data, name="sel_data"),
+        _ptr(sel_scales, name="sel_scales"),
         _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
         _ptr(v_pool, torch.bfloat16, "v_pool"), _ptr(page_table, torch.int32, "page_table"),
         int(page_table.shape[-1]), _ptr(seq_lens, torch.int32, "seq_lens"),

@@ -88,6 +88,19 @@ bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_row
     return r == CUDA_SUCCESS;
 }
 
+bool make_bytes_map(CUtensorMap* map, const void* base, int64_t lines, int box_lines) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(lines)};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_lines)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Layout* out) {
     const int U = batch * d->num_kv_heads;
     const int G = d->num_q_heads / d->num_kv_heads;
@@ -404,6 +417,7 @@ spot_status_t check_tok_desc(const spot_tok_layer_desc_t* d) {
     if (d->head_dim != kHeadDim || d->page_size != kBlock || d->idx_heads != kIdxHeads ||
         d->idx_dim != kIdxDim || d->sel_block != kTokBlock)
         return SPOT_ERR_UNSUPPORTED;
+    if (d->sel_fmt < SPOT_SEL_BF16 || d->sel_fmt > SPOT_SEL_INT8_F16) return SPOT_ERR_INVALID_ARG;
     if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return SPOT_ERR_UNSUPPORTED;
     // TMA row coordinates are 32-bit (KV rows and selector rows).
     if (static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock > INT32_MAX ||
@@ -419,19 +433,22 @@ spot_status_t check_tok_batch(const spot_tok_layer_desc_t* d, int batch, int max
     return SPOT_OK;
 }
 
-spot_status_t check_tok_select_args(const spot_select_params_t* pr, const uint16_t* q_idx,
-                                    const float* w, const uint16_t* sel_tok,
+spot_status_t check_tok_select_args(const spot_tok_layer_desc_t* d,
+                                    const spot_select_params_t* pr, const uint16_t* q_idx,
+                                    const float* w, const void* sel_data, const void* sel_scales,
                                     const int32_t* page_table, int32_t pt_stride,
                                     const int32_t* seq_lens, const float* top_p,
                                     int32_t* sel_idx, int32_t* sel_cnt) {
     spot_status_t st = check_params(pr);
     if (st != SPOT_OK) return st;
     if (pr->quantize_queries) return SPOT_ERR_UNSUPPORTED;
-    if (!q_idx || !sel_tok || !page_table || !seq_lens || !sel_idx || !sel_cnt)
+    if (!q_idx || !sel_data || !page_table || !seq_lens || !sel_idx || !sel_cnt)
+        return SPOT_ERR_INVALID_ARG;
+    if (needs_scales(d->sel_fmt) && (!sel_scales || !aligned(sel_scales, 16)))
         return SPOT_ERR_INVALID_ARG;
     if (pr->mode == SPOT_MODE_TOPP && !top_p) return SPOT_ERR_INVALID_ARG;
     if (pt_stride <= 0) return SPOT_ERR_INVALID_ARG;
-    if (!aligned(q_idx, 16) || !aligned(sel_tok, 256) || !aligned(page_table, 4) ||
+    if (!aligned(q_idx, 16) || !aligned(sel_data, 256) || !aligned(page_table, 4) ||
         !aligned(seq_lens, 4) || !aligned(sel_idx, 4) || !aligned(sel_cnt, 4) ||
         (w && !aligned(w, 4)) || (top_p && !aligned(top_p, 4)))
         return SPOT_ERR_INVALID_ARG;
@@ -439,15 +456,21 @@ spot_status_t check_tok_select_args(const spot_select_params_t* pr, const uint16
 }
 
 spot_status_t do_tok_select(const spot_tok_layer_desc_t* d, const spot_select_params_t* pr,
-                            const uint16_t* q_idx, const float* w, const uint16_t* sel_tok,
+                            const uint16_t* q_idx, const float* w, const void* sel_data,
+                            const void* sel_scales,
                             const int32_t* page_table, int32_t pt_stride,
                             const int32_t* seq_lens, const float* top_p, int32_t batch,
                             int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks, void* ws,
                             const Layout& L, cudaStream_t s) {
     CUtensorMap sm;
-    if (!make_rows_map(&sm, sel_tok, static_cast<int64_t>(d->num_pages) * kBlock * kIdxHeads,
-                       kTokBlock * kIdxHeads))
-        return SPOT_ERR_CUDA;
+    const int64_t rows = static_cast<int64_t>(d->num_pages) * kBlock * kIdxHeads;
+    const int rb = tok_row_bytes_host(d->sel_fmt);
+    const bool ok_map =
+        d->sel_fmt == SPOT_SEL_BF16
+            ? make_rows_map(&sm, sel_data, rows, kTokBlock * kIdxHeads)
+            // code rows viewed as 128-byte lines (4-bit: two rows per line)
+            : make_bytes_map(&sm, sel_data, rows * rb / 128, (kTokBlock * kIdxHeads * rb) / 128);
+    if (!ok_map) return SPOT_ERR_CUDA;
     uint8_t* base = static_cast<uint8_t*>(ws);
     float* scores = reinterpret_cast<float*>(base + L.tok_scores);
     uint32_t* status = reinterpret_cast<uint32_t*>(base + L.status);
@@ -462,7 +485,9 @@ spot_status_t do_tok_select(const spot_tok_layer_desc_t* d, const spot_select_pa
     tp.num_pages = d->num_pages;
     tp.inv_temp = 1.0f / pr->temperature;
     tp.scores = scores;
-    tp.num_ctas = tok_score_grid(batch);
+    tp.num_ctas = tok_score_grid(d->sel_fmt, batch);
+    tp.fmt = d->sel_fmt;
+    tp.sel_scales = sel_scales;
     tp.status = status;
     if (tp.num_ctas <= 0) return SPOT_ERR_CUDA;
     if (launch_tok_score(tp, sm, s) != cudaSuccess) return SPOT_ERR_CUDA;
@@ -542,7 +567,8 @@ size_t spot_tok_workspace_size(const spot_tok_layer_desc_t* desc, int32_t batch,
     return L.total;
 }
 
-spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, uint16_t* sel_tok,
+spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, void* sel_data,
+                                            void* sel_scales,
                                             const int32_t* page_table, int32_t num_seqs,
                                             int32_t pt_stride, const int32_t* seq_ids,
                                             const int32_t* positions, const uint16_t* keys,
@@ -551,13 +577,17 @@ spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, u
     if (st != SPOT_OK) return st;
     if (n < 0 || pt_stride <= 0 || num_seqs < 0) return SPOT_ERR_INVALID_ARG;
     if (n == 0) return SPOT_OK;
-    if (!sel_tok || !page_table || !seq_ids || !positions || !keys) return SPOT_ERR_INVALID_ARG;
-    if (!aligned(sel_tok, 16) || !aligned(keys, 16) || !aligned(page_table, 4) ||
+    if (!sel_data || !page_table || !seq_ids || !positions || !keys) return SPOT_ERR_INVALID_ARG;
+    if (needs_scales(desc->sel_fmt) && (!sel_scales || !aligned(sel_scales, 16)))
+        return SPOT_ERR_INVALID_ARG;
+    if (!aligned(sel_data, 16) || !aligned(keys, 16) || !aligned(page_table, 4) ||
         !aligned(seq_ids, 4) || !aligned(positions, 4))
         return SPOT_ERR_INVALID_ARG;
     if (status_ws && !aligned(status_ws, 256)) return SPOT_ERR_INVALID_ARG;
     TokAppendParams p;
-    p.sel_tok = sel_tok;
+    p.sel_data = sel_data;
+    p.sel_scales = sel_scales;
+    p.fmt = desc->sel_fmt;
     p.page_table = page_table;
     p.num_seqs = num_seqs;
     p.pt_stride = pt_stride;
@@ -573,7 +603,7 @@ spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, u
 
 spot_status_t spot_tok_select(const spot_tok_layer_desc_t* desc,
                               const spot_select_params_t* params, const uint16_t* q_idx,
-                              const float* w_idx, const uint16_t* sel_tok,
+                              const float* w_idx, const void* sel_data, const void* sel_scales,
                               const int32_t* page_table, int32_t pt_stride,
                               const int32_t* seq_lens, const float* top_p, int32_t batch,
                               int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
@@ -582,14 +612,16 @@ spot_status_t spot_tok_select(const spot_tok_layer_desc_t* desc,
     if (st == SPOT_OK) st = check_tok_batch(desc, batch, max_blocks);
     if (st != SPOT_OK) return st;
     if (batch == 0) return SPOT_OK;
-    st = check_tok_select_args(params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+    st = check_tok_select_args(desc, params, q_idx, w_idx, sel_data, sel_scales, page_table,
+                               pt_stride, seq_lens,
                                top_p, sel_idx, sel_cnt);
     if (st != SPOT_OK) return st;
     Layout L;
     if (!tok_workspace_layout(desc, batch, max_blocks, &L)) return SPOT_ERR_CUDA;
     st = check_ws(workspace, ws_bytes, L);
     if (st != SPOT_OK) return st;
-    return do_tok_select(desc, params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+    return do_tok_select(desc, params, q_idx, w_idx, sel_data, sel_scales, page_table, pt_stride,
+                         seq_lens,
                          top_p, batch, sel_idx, sel_cnt, max_blocks, workspace, L,
                          static_cast<cudaStream_t>(stream));
 }
@@ -619,8 +651,9 @@ spot_status_t spot_tok_sparse_decode(const spot_tok_layer_desc_t* desc, const ui
 
 spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
                                    const spot_select_params_t* params, const uint16_t* q_idx,
-                                   const float* w_idx, const uint16_t* sel_tok,
-                                   const uint16_t* q, const uint16_t* k_pool,
+                                   const float* w_idx, const void* sel_data,
+                                   const void* sel_scales, const uint16_t* q,
+                                   const uint16_t* k_pool,
                                    const uint16_t* v_pool, const int32_t* page_table,
                                    int32_t pt_stride, const int32_t* seq_lens,
                                    const float* top_p, int32_t batch, float softmax_scale,
@@ -631,7 +664,8 @@ spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
     if (st == SPOT_OK) st = check_tok_batch(desc, batch, max_blocks);
     if (st != SPOT_OK) return st;
     if (batch == 0) return SPOT_OK;
-    st = check_tok_select_args(params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+    st = check_tok_select_args(desc, params, q_idx, w_idx, sel_data, sel_scales, page_table,
+                               pt_stride, seq_lens,
                                top_p, sel_idx, sel_cnt);
     if (st == SPOT_OK)
         st = check_decode_args(q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx,
@@ -642,7 +676,8 @@ spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
     st = check_ws(workspace, ws_bytes, L);
     if (st != SPOT_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = do_tok_select(desc, params, q_idx, w_idx, sel_tok, page_table, pt_stride, seq_lens,
+    st = do_tok_select(desc, params, q_idx, w_idx, sel_data, sel_scales, page_table, pt_stride,
+                       seq_lens,
                        top_p, batch, sel_idx, sel_cnt, max_blocks, workspace, L, s);
     if (st != SPOT_OK) return st;
     return do_tok_decode(desc, q, k_pool, v_pool, page_table, pt_stride, seq_lens, sel_idx,

@@ -11,10 +11,14 @@
 //          clamp(rne(x / scale), -128, 127).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <math.h>
 #include <stdint.h>
+
+#include "../../include/spot.h"
+#include "spot_device.cuh"
 
 namespace spot {
 
@@ -75,6 +79,62 @@ __device__ __forceinline__ uint32_t fp8_code(float x) {
 __device__ __forceinline__ float fp8_value(uint32_t code) {
     const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
     return __half2float(__half(h));
+}
+
+// ---- code -> bf16 widening for the tensor-core scoring paths (every INT4,
+// E2M1, INT8 and E4M3 value is exact in bf16; scales are applied after the
+// mma)
+
+// E2M1 code (bit 3 = sign) -> bf16 bit pattern of its value.
+__device__ __forceinline__ uint32_t e2m1_bf16_bits(uint32_t code) {
+    // magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 as bf16: 0x0000 0x3F00 0x3F80 0x3FC0
+    // 0x4000 0x4040 0x4080 0x40C0
+    const uint32_t mag = code & 7u;
+    uint32_t bits;
+    if (mag == 0) bits = 0;
+    else if (mag == 1) bits = 0x3F00u;
+    else {
+        const uint32_t e = (mag >> 1);            // 1..3: value = (1 + m/2) 2^(e-1)
+        const uint32_t m = mag & 1u;
+        bits = ((126u + e) << 7) | (m << 6);
+    }
+    return bits | ((code & 8u) << 12);
+}
+
+__device__ __forceinline__ uint32_t int4_bf16_bits(uint32_t nib) {
+    const int q = (nib & 8u) ? static_cast<int>(nib) - 16 : static_cast<int>(nib);
+    const __nv_bfloat16 v = __int2bfloat16_rn(q);
+    return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&v));
+}
+
+// One byte of 4-bit codes (two elements, even element in the low nibble)
+// -> packed bf16x2 with the even element in the low half.
+template <int FMT>
+__device__ __forceinline__ uint32_t byte_to_bf16x2(uint32_t byte) {
+    const uint32_t lo = byte & 0xFu, hi = (byte >> 4) & 0xFu;
+    if (FMT == SPOT_SEL_INT4_G32_F16) return int4_bf16_bits(lo) | (int4_bf16_bits(hi) << 16);
+    return e2m1_bf16_bits(lo) | (e2m1_bf16_bits(hi) << 16);
+}
+
+// Two 8-bit codes (the even element in the low byte) -> packed bf16x2 with
+// the even element in the low half; INT8 and E4M3 values are exact in bf16.
+template <int FMT>
+__device__ __forceinline__ uint32_t pair8_to_bf16x2(uint32_t two) {
+    if (FMT == SPOT_SEL_INT8_F16) {
+        const int lo = static_cast<int8_t>(two & 0xFFu), hi = static_cast<int8_t>((two >> 8) & 0xFFu);
+        return pack_bf16(static_cast<float>(lo), static_cast<float>(hi));
+    }
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu),
+                                                     __NV_E4M3);
+    const float2 f = __half22float2(__half2(hr));
+    return pack_bf16(f.x, f.y);
+}
+
+// E8M0 scale byte -> its value 2^(e - 127) (255 is NaN).
+__device__ __forceinline__ float e8m0_value(uint32_t e) {
+    if (e == 255u) return __int_as_float(0x7fc00000);
+    if (e == 0u) return __int_as_float(0x00400000);            // 2^-127
+    return __int_as_float(static_cast<int>(e << 23));
 }
 
 }  // namespace spot

@@ -45,51 +45,6 @@ constexpr int kTileBatch = 4;           // 16-block tiles a warp scores with loa
 
 // --------------------------------------------------------------- scoring
 
-// E2M1 code (bit 3 = sign) -> bf16 bit pattern of its value.
-__device__ __forceinline__ uint32_t e2m1_bf16_bits(uint32_t code) {
-    // magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 as bf16: 0x0000 0x3F00 0x3F80 0x3FC0
-    // 0x4000 0x4040 0x4080 0x40C0
-    const uint32_t mag = code & 7u;
-    uint32_t bits;
-    if (mag == 0) bits = 0;
-    else if (mag == 1) bits = 0x3F00u;
-    else {
-        const uint32_t e = (mag >> 1);            // 1..3: value = (1 + m/2) 2^(e-1)
-        const uint32_t m = mag & 1u;
-        bits = ((126u + e) << 7) | (m << 6);
-    }
-    return bits | ((code & 8u) << 12);
-}
-
-__device__ __forceinline__ uint32_t int4_bf16_bits(uint32_t nib) {
-    const int q = (nib & 8u) ? static_cast<int>(nib) - 16 : static_cast<int>(nib);
-    const __nv_bfloat16 v = __int2bfloat16_rn(q);
-    return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&v));
-}
-
-// One byte of 4-bit codes (two elements, even element in the low nibble)
-// -> packed bf16x2 with the even element in the low half.
-template <int FMT>
-__device__ __forceinline__ uint32_t byte_to_bf16x2(uint32_t byte) {
-    const uint32_t lo = byte & 0xFu, hi = (byte >> 4) & 0xFu;
-    if (FMT == SPOT_SEL_INT4_G32_F16) return int4_bf16_bits(lo) | (int4_bf16_bits(hi) << 16);
-    return e2m1_bf16_bits(lo) | (e2m1_bf16_bits(hi) << 16);
-}
-
-// Two 8-bit codes (the even element in the low byte) -> packed bf16x2 with
-// the even element in the low half; INT8 and E4M3 values are exact in bf16.
-template <int FMT>
-__device__ __forceinline__ uint32_t pair8_to_bf16x2(uint32_t two) {
-    if (FMT == SPOT_SEL_INT8_F16) {
-        const int lo = static_cast<int8_t>(two & 0xFFu), hi = static_cast<int8_t>((two >> 8) & 0xFFu);
-        return pack_bf16(static_cast<float>(lo), static_cast<float>(hi));
-    }
-    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu),
-                                                     __NV_E4M3);
-    const float2 f = __half22float2(__half2(hr));
-    return pack_bf16(f.x, f.y);
-}
-
 template <int FMT>
 __device__ __forceinline__ float group_scale(const void* scales, int64_t row, int grp) {
     if (FMT == SPOT_SEL_INT4_G32_F16) {

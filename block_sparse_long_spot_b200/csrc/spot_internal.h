@@ -113,12 +113,16 @@ struct TokScoreParams {
     float inv_temp;
     float* scores;                      // [B][max_blocks]
     int32_t num_ctas;
+    int32_t fmt;                        // spot_sel_fmt_t of the per-token key rows
+    const void* sel_scales;             // their scales (INT4 / MXFP4 / INT8), else null
     uint32_t* status;
 };
 
 // Append of per-token selector keys.
 struct TokAppendParams {
-    uint16_t* sel_tok;                  // [num_pages][kBlock][kIdxHeads][kIdxDim]
+    void* sel_data;                     // rows [num_pages][kBlock][kIdxHeads] in `fmt`
+    void* sel_scales;
+    int32_t fmt;
     const int32_t* page_table;
     int32_t num_seqs, pt_stride;
     const int32_t* seq_ids;
@@ -183,7 +187,9 @@ cudaError_t launch_tok_append(const TokAppendParams& p, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& k_map,
                            const CUtensorMap& v_map, cudaStream_t s);
 int prefill_row_groups(int group);
-int tok_score_grid(int batch);
+int tok_score_grid(int fmt, int batch);
+int tok_row_bytes_host(int fmt);         // bytes of one (token, head) key row
+int tok_scale_bytes_host(int fmt);       // bytes of its scales
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
 // Persistent grid of the decode kernel for U units on the current device.
@@ -197,5 +203,8 @@ bool make_pool_map(CUtensorMap* map, const void* pool, int num_pages, int num_kv
 // Tensor map over `rows` rows of 128 bf16 (256 B), box 64 columns x
 // box_rows rows, 128-byte swizzle.
 bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
+// Tensor map over `lines` lines of 128 bytes, box 128 bytes x box_lines,
+// 128-byte swizzle.
+bool make_bytes_map(CUtensorMap* map, const void* base, int64_t lines, int box_lines);
 
 }  // namespace spot

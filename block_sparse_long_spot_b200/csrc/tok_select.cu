@@ -22,6 +22,7 @@
 
 #include <mutex>
 
+#include "quant.cuh"
 #include "spot_device.cuh"
 #include "spot_internal.h"
 
@@ -32,8 +33,23 @@ constexpr int NCS = 4;                                          // consumer warp
 constexpr int SST = 12;                                         // pipeline stages
 constexpr int kSThreads = (NCS + 1) * 32;
 static_assert(SST % NCS == 0, "each stage must always be consumed by the same warp");
-constexpr int kTokStageBytes = kTokBlock * kIdxHeads * kIdxDim * 2;   // 16 KiB
-constexpr int kTokHalf = kTokStageBytes / 2;                    // 64 rows x 64 bf16
+constexpr int kRowsPerBlock = kTokBlock * kIdxHeads;            // 64 (token, head) rows
+
+// Bytes of one (token, head) key row and of its scales, per format.
+__host__ __device__ constexpr int tok_row_bytes(int fmt) {
+    return fmt == SPOT_SEL_BF16 ? 2 * kIdxDim
+           : (fmt == SPOT_SEL_FP8_E4M3 || fmt == SPOT_SEL_INT8_F16) ? kIdxDim : kIdxDim / 2;
+}
+__host__ __device__ constexpr int tok_scale_bytes(int fmt) {
+    return fmt == SPOT_SEL_INT4_G32_F16 ? 2 * (kIdxDim / 32)
+           : fmt == SPOT_SEL_MXFP4_G32_E8M0 ? kIdxDim / 32
+           : fmt == SPOT_SEL_INT8_F16 ? 2 : 0;
+}
+// One stage = one 16-token block: its code rows, then its scales.
+__host__ __device__ constexpr int tok_code_bytes(int fmt) { return kRowsPerBlock * tok_row_bytes(fmt); }
+__host__ __device__ constexpr int tok_stage_bytes(int fmt) {
+    return (tok_code_bytes(fmt) + kRowsPerBlock * tok_scale_bytes(fmt) + 1023) / 1024 * 1024;
+}
 
 __device__ __forceinline__ int find_seq(const int* off, int B, int pos) {
     // largest b in [0, B) with off[b] <= pos
@@ -49,8 +65,134 @@ __device__ __forceinline__ int range_begin(int64_t N, int64_t P, int64_t i) {
     return static_cast<int>((N * i) / P);
 }
 
+// The scores of the 64 (token, head) rows of m-tile group `mt` (rows
+// 16 mt + r8 and + 8 of the stage) against Q^T: per row, the dot with the
+// query of every index head (column h), scales applied.  The head dimension
+// is consumed in a format-dependent order, the same for keys and queries
+// (qf holds the query fragments in that order).
+//   bf16:  the stage holds two 64 x 64 bf16 halves (128-byte swizzle);
+//   8-bit: 64 rows of 128 code bytes (128-byte swizzle); 16-byte chunk c is
+//          dims 16 c .. 16 c + 15;
+//   4-bit: 32 double rows of 128 bytes (128-byte swizzle): row r is half
+//          r & 1 of double row r / 2; chunk c of a row is dims 32 c .. + 31,
+//          the scale group c.
+template <int FMT>
+__device__ __forceinline__ void tile_dots(uint32_t kb, const uint8_t* sc_smem, int mt, int lane,
+                                          const uint32_t (&qf)[8][2], float (&acc)[4]) {
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+    const int r8 = lane >> 2;
+    const int rowA = mt * 16 + r8, rowB = rowA + 8;       // this lane's two rows
+    if constexpr (FMT == SPOT_SEL_BF16) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t hb = kb + (ks >> 2) * (tok_code_bytes(FMT) / 2);
+            const int chunk = ((ks & 3) << 1) + (lane >> 4);
+            const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(swz128(hb, row, chunk), a0, a1, a2, a3);
+            mma_bf16_16816(acc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        }
+    } else if constexpr (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
+        const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+        for (int cp = 0; cp < 4; ++cp) {
+            uint32_t r0, r1, r2, r3;                       // chunks 2 cp, 2 cp + 1
+            ldsm_x4(swz128(kb, row, 2 * cp + (lane >> 4)), r0, r1, r2, r3);
+            mma_bf16_16816(acc, pair8_to_bf16x2<FMT>(r0), pair8_to_bf16x2<FMT>(r1),
+                           pair8_to_bf16x2<FMT>(r0 >> 16), pair8_to_bf16x2<FMT>(r1 >> 16),
+                           qf[2 * cp][0], qf[2 * cp][1]);
+            mma_bf16_16816(acc, pair8_to_bf16x2<FMT>(r2), pair8_to_bf16x2<FMT>(r3),
+                           pair8_to_bf16x2<FMT>(r2 >> 16), pair8_to_bf16x2<FMT>(r3 >> 16),
+                           qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+        }
+        if constexpr (FMT == SPOT_SEL_INT8_F16) {
+            const __half* s = reinterpret_cast<const __half*>(sc_smem);
+            const float sa = __half2float(s[rowA]), sb = __half2float(s[rowB]);
+            acc[0] *= sa;
+            acc[1] *= sa;
+            acc[2] *= sb;
+            acc[3] *= sb;
+        }
+    } else {
+        const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        float g[4][4];
+#pragma unroll
+        for (int cp = 0; cp < 2; ++cp) {
+            const int c = 2 * cp + (lane >> 4);            // this lane's address: chunk c
+            uint32_t r0, r1, r2, r3;                       // chunks 2 cp, 2 cp + 1
+            ldsm_x4(swz128(kb, row >> 1, ((row & 1) << 2) + c), r0, r1, r2, r3);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t ra = h ? r2 : r0, rb = h ? r3 : r1;
+                float (&a)[4] = g[2 * cp + h];
+                a[0] = a[1] = a[2] = a[3] = 0.f;
+                mma_bf16_16816(a, byte_to_bf16x2<FMT>(ra & 0xFFu), byte_to_bf16x2<FMT>(rb & 0xFFu),
+                               byte_to_bf16x2<FMT>((ra >> 8) & 0xFFu),
+                               byte_to_bf16x2<FMT>((rb >> 8) & 0xFFu), qf[2 * (2 * cp + h)][0],
+                               qf[2 * (2 * cp + h)][1]);
+                mma_bf16_16816(a, byte_to_bf16x2<FMT>((ra >> 16) & 0xFFu),
+                               byte_to_bf16x2<FMT>((rb >> 16) & 0xFFu), byte_to_bf16x2<FMT>(ra >> 24),
+                               byte_to_bf16x2<FMT>(rb >> 24), qf[2 * (2 * cp + h) + 1][0],
+                               qf[2 * (2 * cp + h) + 1][1]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float sa, sb;
+            if constexpr (FMT == SPOT_SEL_INT4_G32_F16) {
+                const __half* s = reinterpret_cast<const __half*>(sc_smem);
+                sa = __half2float(s[rowA * 4 + c]);
+                sb = __half2float(s[rowB * 4 + c]);
+            } else {
+                sa = e8m0_value(sc_smem[rowA * 4 + c]);
+                sb = e8m0_value(sc_smem[rowB * 4 + c]);
+            }
+            acc[0] = fmaf(g[c][0], sa, acc[0]);
+            acc[1] = fmaf(g[c][1], sa, acc[1]);
+            acc[2] = fmaf(g[c][2], sb, acc[2]);
+            acc[3] = fmaf(g[c][3], sb, acc[3]);
+        }
+    }
+}
+
+// Query fragments (B operand, n = index head r8, heads 4..7 zero) in the
+// order tile_dots consumes the head dimension: k-step ks, pair (2 c4, +1)
+// and (2 c4 + 8, +9) of the fragment map to dims
+//   bf16:  16 ks + 2 c4 + {0,1} and + 8     (u32 8 ks + c4, 8 ks + 4 + c4)
+//   8-bit: 16 ks + 4 c4 + {0,1} and {2,3}  (u32 8 ks + 2 c4, + 1)
+//   4-bit: step ks = 2 c + t: 32 c + 8 c4 + 4 t + {0,1} and {2,3}
+//          (u32 16 c + 4 c4 + 2 t, + 1)
+template <int FMT>
+__device__ __forceinline__ void load_tok_queries(const uint16_t* q_idx, int b, int lane,
+                                                 uint32_t (&qf)[8][2]) {
+    const int c4 = lane & 3, r8 = lane >> 2;
+    const bool real = r8 < kIdxHeads;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        q_idx + (static_cast<int64_t>(b) * kIdxHeads + (real ? r8 : 0)) * kIdxDim);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        int i0, i1;
+        if constexpr (FMT == SPOT_SEL_BF16) {
+            i0 = 8 * ks + c4;
+            i1 = 8 * ks + 4 + c4;
+        } else if constexpr (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
+            i0 = 8 * ks + 2 * c4;
+            i1 = i0 + 1;
+        } else {
+            i0 = 16 * (ks >> 1) + 4 * c4 + 2 * (ks & 1);
+            i1 = i0 + 1;
+        }
+        qf[ks][0] = real ? __ldg(qrow + i0) : 0u;
+        qf[ks][1] = real ? __ldg(qrow + i1) : 0u;
+    }
+}
+
+template <int FMT>
 __global__ void __launch_bounds__(kSThreads)
 tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScoreParams p) {
+    constexpr int kStage = tok_stage_bytes(FMT);
+    constexpr int kCode = tok_code_bytes(FMT);
+    constexpr int kScale = kRowsPerBlock * tok_scale_bytes(FMT);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -59,7 +201,7 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* base = smem_raw + pad;
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + SST * kTokStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + SST * kStage);
     uint64_t* empty = full + SST;
     int* scan = reinterpret_cast<int*>(empty + SST);            // [kSThreads / 32 + 1]
     volatile int* flags = scan + (kSThreads / 32 + 1);          // [0] abort
@@ -115,7 +257,7 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
         int issued = 0;
         for (int base_it = 0; base_it < n_it && alive; base_it += 32) {
             const int it = base_it + lane;
-            int row = 0;
+            int row = 0;                                // first (token, head) row of the block
             if (it < n_it) {
                 const int pos = beg + it;
                 const int b = find_seq(seq_off, B, pos);
@@ -142,10 +284,21 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
                         flags[0] = 1;
                         ok = 0;
                     } else {
-                        mbar_arrive_expect_tx(&full[s], kTokStageBytes);
-                        uint8_t* dst = base + s * kTokStageBytes;
-                        tma_load_2d(dst, &sel_map, &full[s], 0, r, policy);
-                        tma_load_2d(dst + kTokHalf, &sel_map, &full[s], 64, r, policy);
+                        mbar_arrive_expect_tx(&full[s], kCode + kScale);
+                        uint8_t* dst = base + s * kStage;
+                        if constexpr (FMT == SPOT_SEL_BF16) {
+                            tma_load_2d(dst, &sel_map, &full[s], 0, r, policy);
+                            tma_load_2d(dst + kCode / 2, &sel_map, &full[s], 64, r, policy);
+                        } else if constexpr (tok_row_bytes(FMT) == kIdxDim) {
+                            tma_load_2d(dst, &sel_map, &full[s], 0, r, policy);
+                        } else {
+                            tma_load_2d(dst, &sel_map, &full[s], 0, r / 2, policy);
+                        }
+                        if constexpr (kScale > 0)
+                            bulk_load(dst + kCode,
+                                      static_cast<const uint8_t*>(p.sel_scales) +
+                                          static_cast<int64_t>(r) * tok_scale_bytes(FMT),
+                                      kScale, &full[s], policy);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -174,16 +327,7 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
         const int b = find_seq(seq_off, B, pos);
         const int j = pos - seq_off[b];
         if (b != cur_b) {
-            // Q^T fragments (B operand, k = dim, n = index head r8; heads
-            // 4..7 are zero padding)
-            const bool real = r8 < kIdxHeads;
-            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-                p.q_idx + (static_cast<int64_t>(b) * kIdxHeads + (real ? r8 : 0)) * kIdxDim);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                qf[ks][0] = real ? __ldg(qrow + ks * 8 + c4) : 0u;
-                qf[ks][1] = real ? __ldg(qrow + ks * 8 + 4 + c4) : 0u;
-            }
+            load_tok_queries<FMT>(p.q_idx, b, lane, qf);
             wh = p.w ? p.w[static_cast<int64_t>(b) * kIdxHeads + head] : 1.f / kIdxHeads;
             cur_b = b;
         }
@@ -197,33 +341,17 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
             }
             break;
         }
-        const uint32_t kb = stage_base + s * kTokStageBytes;
-        float sc[4][4];
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t hb = kb + (ks >> 2) * kTokHalf;
-            const int chunk = ((ks & 3) << 1) + (lane >> 4);
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-                const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(swz128(hb, row, chunk), a0, a1, a2, a3);
-                mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        // rows 16 mt + r8 and 16 mt + r8 + 8 are (token 4 mt + r8/4, head)
-        // and (token 4 mt + 2 + r8/4, head); a half-warp sums its 4 heads
+        const uint32_t kb = stage_base + s * kStage;
+        const uint8_t* scl = base + s * kStage + kCode;
+        // rows 16 mt + r8 and + 8 are (token 4 mt + r8/4, head) and
+        // (token 4 mt + 2 + r8/4, head); a half-warp sums its 4 heads
         float best = -INFINITY;
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
-            float top = odd ? sc[mt][1] : sc[mt][0];
-            float bot = odd ? sc[mt][3] : sc[mt][2];
+            float acc[4];
+            tile_dots<FMT>(kb, scl, mt, lane, qf, acc);
+            float top = odd ? acc[1] : acc[0];
+            float bot = odd ? acc[3] : acc[2];
             top = owner ? wh * fmaxf(top, 0.f) : 0.f;
             bot = owner ? wh * fmaxf(bot, 0.f) : 0.f;
 #pragma unroll
@@ -233,17 +361,26 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
             }
             best = fmaxf(best, fmaxf(top, bot));
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
         best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 16));
         if (lane == 0) p.scores[static_cast<int64_t>(b) * p.max_blocks + j] = best * p.inv_temp;
     }
 }
 
-size_t tok_score_smem_bytes(int batch) {
-    return 1024 + static_cast<size_t>(SST) * kTokStageBytes + 2 * SST * sizeof(uint64_t) +
+size_t tok_score_smem_bytes(int fmt, int batch) {
+    const int stage = fmt == SPOT_SEL_BF16 ? tok_stage_bytes(SPOT_SEL_BF16)
+                      : fmt == SPOT_SEL_INT4_G32_F16 ? tok_stage_bytes(SPOT_SEL_INT4_G32_F16)
+                      : fmt == SPOT_SEL_MXFP4_G32_E8M0 ? tok_stage_bytes(SPOT_SEL_MXFP4_G32_E8M0)
+                      : fmt == SPOT_SEL_FP8_E4M3 ? tok_stage_bytes(SPOT_SEL_FP8_E4M3)
+                                                 : tok_stage_bytes(SPOT_SEL_INT8_F16);
+    return 1024 + static_cast<size_t>(SST) * stage + 2 * SST * sizeof(uint64_t) +
            (kSThreads / 32 + 1 + 1) * sizeof(int) + static_cast<size_t>(batch + 1) * sizeof(int);
 }
 
-// One warp per appended token: 4 x 128 bf16 = 1 KiB, 32 bytes per lane.
+// One warp per appended token: 4 heads x 128 dims; lane l takes head l / 8,
+// dims 16 (l % 8) .. + 15 and quantises them with the format's rule
+// (quant.cuh) over groups of 32 (two lanes) or the whole row (INT8, 8 lanes).
 __global__ void __launch_bounds__(128) tok_append_kernel(const TokAppendParams p) {
     const int lane = threadIdx.x & 31;
     const int64_t i = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
@@ -258,53 +395,131 @@ __global__ void __launch_bounds__(128) tok_append_kernel(const TokAppendParams p
         if (lane == 0) flag_status(p.status, kStatusBounds);
         return;
     }
-    const uint4* src = reinterpret_cast<const uint4*>(p.keys + i * kIdxHeads * kIdxDim);
-    uint4* dst = reinterpret_cast<uint4*>(
-        p.sel_tok + (static_cast<int64_t>(page) * kBlock + pos % kBlock) * kIdxHeads * kIdxDim);
-    const uint4 x0 = __ldg(src + 2 * lane), x1 = __ldg(src + 2 * lane + 1);
-    dst[2 * lane] = x0;
-    dst[2 * lane + 1] = x1;
+    const int h = lane >> 3, seg = lane & 7;
+    const int64_t row = (static_cast<int64_t>(page) * kBlock + pos % kBlock) * kIdxHeads + h;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        p.keys + (i * kIdxHeads + h) * kIdxDim + seg * 16);
+    const uint4 x0 = __ldg(src), x1 = __ldg(src + 1);
+    if (p.fmt == SPOT_SEL_BF16) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.sel_data) + row * kIdxDim +
+                                              seg * 16);
+        dst[0] = x0;
+        dst[1] = x1;
+        return;
+    }
+    float f[16];
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        f[2 * k] = __uint_as_float(w[k] << 16);
+        f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+    float am = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) am = fmaxf(am, fabsf(f[k]));
+    uint8_t* codes = static_cast<uint8_t*>(p.sel_data);
+    if (p.fmt == SPOT_SEL_FP8_E4M3 || p.fmt == SPOT_SEL_INT8_F16) {
+        uint32_t out[4] = {0u, 0u, 0u, 0u};
+        if (p.fmt == SPOT_SEL_FP8_E4M3) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) out[k >> 2] |= fp8_code(f[k]) << (8 * (k & 3));
+        } else {
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+            const uint16_t sbits = f16_scale_bits(am, 127.0);
+            const float sc = f16_bits_value(sbits);
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                out[k >> 2] |= (static_cast<uint32_t>(int_code(f[k], sc, -128, 127)) & 0xFFu)
+                               << (8 * (k & 3));
+            if (seg == 0) static_cast<uint16_t*>(p.sel_scales)[row] = sbits;
+        }
+        *reinterpret_cast<uint4*>(codes + row * kIdxDim + seg * 16) =
+            make_uint4(out[0], out[1], out[2], out[3]);
+        return;
+    }
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));      // groups of 32 dims = 2 lanes
+    const int grp = seg >> 1;
+    uint32_t out[2] = {0u, 0u};
+    if (p.fmt == SPOT_SEL_INT4_G32_F16) {
+        const uint16_t sbits = f16_scale_bits(am, 7.0);
+        const float sc = f16_bits_value(sbits);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            out[k >> 3] |= (static_cast<uint32_t>(int_code(f[k], sc, -8, 7)) & 0xFu) << (4 * (k & 7));
+        if ((seg & 1) == 0) static_cast<uint16_t*>(p.sel_scales)[row * 4 + grp] = sbits;
+    } else {
+        const int X = mx_exponent(am);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) out[k >> 3] |= mx_code(f[k], X) << (4 * (k & 7));
+        if ((seg & 1) == 0)
+            static_cast<uint8_t*>(p.sel_scales)[row * 4 + grp] = static_cast<uint8_t>(X + 127);
+    }
+    *reinterpret_cast<uint2*>(codes + row * (kIdxDim / 2) + seg * 8) = make_uint2(out[0], out[1]);
 }
 
 struct ScoreMemo {
-    size_t smem_set = 0;
-    int batch = -1;
+    size_t smem_set[5] = {0, 0, 0, 0, 0};       // per format instance
+    int key = -1;                              // batch * 8 + fmt of the cached grid
     int grid = 0;
 };
 constexpr int kMemoDevices = 64;
 ScoreMemo g_score_memo[kMemoDevices];
 std::mutex g_score_mutex;
 
+template <int FMT>
 cudaError_t ensure_score_smem(ScoreMemo& m, size_t smem) {
-    if (m.smem_set >= smem) return cudaSuccess;
+    if (m.smem_set[FMT] >= smem) return cudaSuccess;
     const cudaError_t e = cudaFuncSetAttribute(
-        tok_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e == cudaSuccess) m.smem_set = smem;
+        tok_score_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess) m.smem_set[FMT] = smem;
     return e;
 }
 
+template <int FMT>
 int score_grid_locked(int dev, int batch) {
     ScoreMemo& m = g_score_memo[dev];
-    if (m.batch == batch && m.grid > 0) return m.grid;
+    if (m.key == batch * 8 + FMT && m.grid > 0) return m.grid;
     int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    const size_t smem = tok_score_smem_bytes(batch);
-    if (ensure_score_smem(m, smem) != cudaSuccess) return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tok_score_kernel, kSThreads,
+    const size_t smem = tok_score_smem_bytes(FMT, batch);
+    if (ensure_score_smem<FMT>(m, smem) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tok_score_kernel<FMT>, kSThreads,
                                                       smem) != cudaSuccess)
         return 0;
-    m.batch = batch;
+    m.key = batch * 8 + FMT;
     m.grid = sms * max(per_sm, 1);
     return m.grid;
 }
 
+template <int FMT>
+cudaError_t launch_score_fmt(const TokScoreParams& p, const CUtensorMap& sel_map, cudaStream_t s,
+                             int dev) {
+    const size_t smem = tok_score_smem_bytes(FMT, p.batch);
+    cudaError_t e;
+    {
+        std::lock_guard<std::mutex> lock(g_score_mutex);
+        e = ensure_score_smem<FMT>(g_score_memo[dev], smem);
+    }
+    if (e != cudaSuccess) return e;
+    tok_score_kernel<FMT><<<p.num_ctas, kSThreads, smem, s>>>(sel_map, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
-int tok_score_grid(int batch) {
+int tok_score_grid(int fmt, int batch) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMemoDevices) return 0;
     std::lock_guard<std::mutex> lock(g_score_mutex);
-    return score_grid_locked(dev, batch);
+    switch (fmt) {
+        case SPOT_SEL_BF16: return score_grid_locked<SPOT_SEL_BF16>(dev, batch);
+        case SPOT_SEL_INT4_G32_F16: return score_grid_locked<SPOT_SEL_INT4_G32_F16>(dev, batch);
+        case SPOT_SEL_MXFP4_G32_E8M0: return score_grid_locked<SPOT_SEL_MXFP4_G32_E8M0>(dev, batch);
+        case SPOT_SEL_FP8_E4M3: return score_grid_locked<SPOT_SEL_FP8_E4M3>(dev, batch);
+        default: return score_grid_locked<SPOT_SEL_INT8_F16>(dev, batch);
+    }
 }
 
 cudaError_t launch_tok_score(const TokScoreParams& p, const CUtensorMap& sel_map, cudaStream_t s) {
@@ -312,14 +527,14 @@ cudaError_t launch_tok_score(const TokScoreParams& p, const CUtensorMap& sel_map
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMemoDevices) return cudaErrorInvalidDevice;
-    const size_t smem = tok_score_smem_bytes(p.batch);
-    {
-        std::lock_guard<std::mutex> lock(g_score_mutex);
-        e = ensure_score_smem(g_score_memo[dev], smem);
+    switch (p.fmt) {
+        case SPOT_SEL_BF16: return launch_score_fmt<SPOT_SEL_BF16>(p, sel_map, s, dev);
+        case SPOT_SEL_INT4_G32_F16: return launch_score_fmt<SPOT_SEL_INT4_G32_F16>(p, sel_map, s, dev);
+        case SPOT_SEL_MXFP4_G32_E8M0:
+            return launch_score_fmt<SPOT_SEL_MXFP4_G32_E8M0>(p, sel_map, s, dev);
+        case SPOT_SEL_FP8_E4M3: return launch_score_fmt<SPOT_SEL_FP8_E4M3>(p, sel_map, s, dev);
+        default: return launch_score_fmt<SPOT_SEL_INT8_F16>(p, sel_map, s, dev);
     }
-    if (e != cudaSuccess) return e;
-    tok_score_kernel<<<p.num_ctas, kSThreads, smem, s>>>(sel_map, p);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_tok_append(const TokAppendParams& p, cudaStream_t s) {
@@ -327,5 +542,8 @@ cudaError_t launch_tok_append(const TokAppendParams& p, cudaStream_t s) {
     tok_append_kernel<<<static_cast<unsigned>(blocks), 128, 0, s>>>(p);
     return cudaGetLastError();
 }
+
+int tok_row_bytes_host(int fmt) { return tok_row_bytes(fmt); }
+int tok_scale_bytes_host(int fmt) { return tok_scale_bytes(fmt); }
 
 }  // namespace spot

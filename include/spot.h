@@ -235,15 +235,24 @@ spot_status_t spot_sparse_decode_noalloc(const spot_layer_desc_t* desc, const ui
  * block of sel_block tokens scores the maximum of its tokens' scores, and
  * ONE selection per sequence (dual top-p / static top-K over those blocks,
  * Eq. 6-8) is shared by every head of the layer.  Supported: idx_heads 4,
- * idx_dim 128, sel_block 16, page_size 64, head_dim 128, bf16 keys,
+ * idx_dim 128, sel_block 16, page_size 64, head_dim 128,
  * 1 <= G <= 8, batch * num_kv_heads <= 4096, max_blocks <= 8192 (128K tokens).
+ * The key rows (one per token and index head, idx_dim elements) are stored
+ * in sel_fmt like the selector keys above: bf16, FP8 E4M3, INT8 with one
+ * fp16 scale per row, INT4 (fp16) or MXFP4 (E8M0) with one scale per 32
+ * elements (§5.3, App. G Tab. 9).
  *
  * Layouts (in addition to the ones above; pages are shared with the KV pools):
  *   q_idx      bf16  [batch][idx_heads][idx_dim]
  *   w_idx      fp32  [batch][idx_heads]          (NULL: 1/idx_heads)
- *   sel_tok    bf16  [num_pages][page_size][idx_heads][idx_dim]: token t of
+ *   sel_data   [num_pages][page_size][idx_heads] key rows of idx_dim elements:
+ *                    bf16 (256 B), FP8 / INT8 (128 B) or INT4 / MXFP4
+ *                    (64 B, even element in the low nibble); token t of
  *                    sequence b at page page_table[b*pt_stride + t/page_size],
  *                    row t % page_size
+ *   sel_scales [num_pages][page_size][idx_heads][n]: n = 4 fp16 (INT4),
+ *                    4 E8M0 (MXFP4), 1 fp16 (INT8); NULL for bf16 / FP8;
+ *                    16-byte aligned
  *   sel_idx    int32 [batch][max_blocks]: selected blocks of sel_block tokens,
  *                    ascending, first sel_cnt entries valid
  *   sel_cnt    int32 [batch]
@@ -261,6 +270,7 @@ typedef struct {
     int32_t idx_dim;              /* d_idx = 128 */
     int32_t sel_block;            /* 16 tokens per selection block */
     int32_t num_pages;
+    int32_t sel_fmt;              /* spot_sel_fmt_t of the per-token key rows */
 } spot_tok_layer_desc_t;
 
 /* Scratch bytes for the token selector's calls (same rules as
@@ -269,9 +279,11 @@ size_t spot_tok_workspace_size(const spot_tok_layer_desc_t* desc, int32_t batch,
                                int32_t max_blocks);
 
 /* Write n tokens' selector keys keys[i] (bf16 [n][idx_heads][idx_dim]) for
- * token positions[i] of sequence seq_ids[i] into sel_tok.  Bad ids or pages
- * are skipped and recorded in status_ws (may be NULL). */
-spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, uint16_t* sel_tok,
+ * token positions[i] of sequence seq_ids[i] into the pool, quantising each
+ * row to sel_fmt.  Bad ids or pages are skipped and recorded in status_ws
+ * (may be NULL). */
+spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, void* sel_data,
+                                            void* sel_scales,
                                             const int32_t* page_table, int32_t num_seqs,
                                             int32_t pt_stride, const int32_t* seq_ids,
                                             const int32_t* positions, const uint16_t* keys,
@@ -280,7 +292,7 @@ spot_status_t spot_tok_append_selector_keys(const spot_tok_layer_desc_t* desc, u
 /* Block scores and one selection per sequence: writes sel_idx / sel_cnt. */
 spot_status_t spot_tok_select(const spot_tok_layer_desc_t* desc,
                               const spot_select_params_t* params, const uint16_t* q_idx,
-                              const float* w_idx, const uint16_t* sel_tok,
+                              const float* w_idx, const void* sel_data, const void* sel_scales,
                               const int32_t* page_table, int32_t pt_stride,
                               const int32_t* seq_lens, const float* top_p, int32_t batch,
                               int32_t* sel_idx, int32_t* sel_cnt, int32_t max_blocks,
@@ -299,7 +311,8 @@ spot_status_t spot_tok_sparse_decode(const spot_tok_layer_desc_t* desc, const ui
 /* spot_tok_select followed by spot_tok_sparse_decode (three kernels). */
 spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
                                    const spot_select_params_t* params, const uint16_t* q_idx,
-                                   const float* w_idx, const uint16_t* sel_tok,
+                                   const float* w_idx, const void* sel_data,
+                                   const void* sel_scales,
                                    const uint16_t* q, const uint16_t* k_pool,
                                    const uint16_t* v_pool, const int32_t* page_table,
                                    int32_t pt_stride, const int32_t* seq_lens,

@@ -241,22 +241,45 @@ def _tok_sel(spec, kmin, sink, rec):
             spec.recency_blocks if rec is None else rec)
 
 
+def gpu_tok_pool(wl, fmt, desc):
+    """Per-token selector pool in `fmt`, written by the library's append
+    kernel from the workload's bf16 keys (every cached token)."""
+    dev = wl.q.device
+    if fmt == "bf16":
+        return wl.sel_tok, None
+    data, scales = spot.tok_selector_pool(wl.num_pages, fmt, device=dev)
+    lens = wl.seq_lens.cpu().numpy()
+    pt = wl.page_table.cpu().numpy()
+    seq = np.concatenate([np.full(int(L), b) for b, L in enumerate(lens)]).astype(np.int32)
+    pos = np.concatenate([np.arange(int(L)) for L in lens]).astype(np.int32)
+    if seq.size == 0:
+        return data, scales
+    pages = torch.as_tensor(pt[seq, pos // 64].astype(np.int64), device=dev)
+    keys = wl.sel_tok[pages, torch.as_tensor(pos % 64, device=dev).long()].contiguous()
+    spot.tok_append_selector_keys(desc, data, scales, wl.page_table,
+                                  torch.as_tensor(seq, device=dev), torch.as_tensor(pos, device=dev),
+                                  keys)
+    torch.cuda.synchronize()
+    return data, scales
+
+
 def run_gpu_tok(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None, temperature=1.0,
-                max_blocks=None, pool=None):
+                max_blocks=None, pool=None, fmt="bf16"):
     dev = wl.q.device
     B, Hq, Hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
     mb = wl.max_blocks if max_blocks is None else max_blocks
     kmin, sink, rec = _tok_sel(wl.spec, kmin, sink, rec)
-    desc = spot.tok_layer_desc(Hq, Hkv, wl.num_pages)
+    desc = spot.tok_layer_desc(Hq, Hkv, wl.num_pages, sel_fmt=fmt)
+    data, scales = gpu_tok_pool(wl, fmt, desc) if pool is None else pool
     prm = spot.select_params(mode, sink, rec, kmin, topk, temperature)
     ws = spot.new_tok_workspace(desc, B, mb, dev)
     sel_idx = torch.full((B, mb), -1, dtype=torch.int32, device=dev)
     sel_cnt = torch.full((B,), -1, dtype=torch.int32, device=dev)
     out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
     lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
-    spot.tok_decode_step(desc, prm, wl.q_idx, wl.w_idx, wl.sel_tok if pool is None else pool,
-                         wl.q, wl.k_pool, wl.v_pool, wl.page_table, wl.seq_lens, wl.top_p,
-                         wl.sm_scale, sel_idx, sel_cnt, out, lse, ws)
+    spot.tok_decode_step(desc, prm, wl.q_idx, wl.w_idx, data, scales, wl.q, wl.k_pool, wl.v_pool,
+                         wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt, out,
+                         lse, ws)
     torch.cuda.synchronize()
     status = spot.read_device_status(ws)
     return {"sel_idx": sel_idx.cpu().numpy(), "sel_cnt": sel_cnt.cpu().numpy(),
@@ -264,35 +287,40 @@ def run_gpu_tok(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None, tempera
             "status": status}
 
 
-def tok_oracle_args(wl):
+def tok_oracle_args(wl, fmt="bf16"):
+    bits = workloads.bits(wl.sel_tok)
+    if fmt == "bf16":
+        data, scales = bits, None
+    else:
+        data, scales = oracle.quantize_selector(fmt, bits)
     return dict(q_idx=workloads.bits(wl.q_idx), w=host_bytes(wl.w_idx),
-                sel_tok=workloads.bits(wl.sel_tok), q=workloads.bits(wl.q),
+                sel_tok=data, sel_scales=scales, q=workloads.bits(wl.q),
                 k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
                 page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
                 top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
 
 
 def tok_oracle_shape_params(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None,
-                            temperature=1.0, max_blocks=None):
+                            temperature=1.0, max_blocks=None, fmt="bf16"):
     kmin, sink, rec = _tok_sel(wl.spec, kmin, sink, rec)
     sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
                                wl.max_pages, max_blocks=wl.max_blocks if max_blocks is None
-                               else max_blocks)
+                               else max_blocks, sel_fmt=fmt)
     pr = oracle.make_params(mode, sink, rec, kmin, topk, temperature)
     return sh, pr
 
 
 def run_oracle_tok(wl, seqs=None, args=None, **kw):
     sh, pr = tok_oracle_shape_params(wl, **kw)
-    a = args or tok_oracle_args(wl)
+    a = args or tok_oracle_args(wl, kw.get("fmt", "bf16"))
     return oracle.tok_decode_step(sh, pr, seqs=seqs, **a)
 
 
 def oracle_tok_scores(wl, args=None, **kw):
     sh, pr = tok_oracle_shape_params(wl, **kw)
-    a = args or tok_oracle_args(wl)
+    a = args or tok_oracle_args(wl, kw.get("fmt", "bf16"))
     return oracle.tok_block_scores(sh, pr, a["q_idx"], a["w"], a["sel_tok"], a["page_table"],
-                                   a["seq_lens"])
+                                   a["seq_lens"], sel_scales=a["sel_scales"])
 
 
 def tok_selection(res, b):

@@ -7,10 +7,11 @@ import pytest
 import torch
 
 import block_sparse_long_spot_b200 as spot
+import oracle
 import workloads
-from harness import (check_tok_outputs, check_tok_selection_near_cut, oracle_tok_scores,
-                     run_gpu_tok, run_oracle_tok, safe_top_p_tok, tok_oracle_args,
-                     tok_selection)
+from harness import (check_tok_outputs, check_tok_selection_near_cut, gpu_tok_pool,
+                     oracle_tok_scores, run_gpu_tok, run_oracle_tok, safe_top_p_tok,
+                     tok_oracle_args, tok_selection)
 
 pytestmark = pytest.mark.gpu
 
@@ -119,7 +120,7 @@ def test_tok_append_writes_the_pool():
     wl = workloads.make_tok("tok_tiny_2k", seed=8, device=DEV, batch=3, seq_len=None,
                             ragged_range=(100, 2048))
     desc = spot.tok_layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages)
-    pool = spot.tok_selector_pool(wl.num_pages, device=DEV)
+    pool, _ = spot.tok_selector_pool(wl.num_pages, device=DEV)
     lens = wl.seq_lens.cpu().numpy()
     pt = wl.page_table.cpu().numpy()
     seq_ids = np.concatenate([np.full(lens[b], b) for b in range(wl.batch)]).astype(np.int32)
@@ -129,7 +130,8 @@ def test_tok_append_writes_the_pool():
     pages = pt[seq_ids, pos // 64]
     keys = wl.sel_tok[torch.as_tensor(pages).long().to(DEV), torch.as_tensor(pos % 64).long().to(DEV)]
     ws = spot.new_tok_workspace(desc, wl.batch, wl.max_blocks, DEV)
-    spot.tok_append_selector_keys(desc, pool, wl.page_table, torch.as_tensor(seq_ids).to(DEV),
+    spot.tok_append_selector_keys(desc, pool, None, wl.page_table,
+                                  torch.as_tensor(seq_ids).to(DEV),
                                   torch.as_tensor(pos).to(DEV), keys.contiguous(), ws)
     torch.cuda.synchronize()
     assert spot.read_device_status(ws) == 0
@@ -142,7 +144,8 @@ def test_tok_append_writes_the_pool():
     # a bad position / sequence is skipped and reported
     bad = torch.tensor([wl.batch, 0], dtype=torch.int32, device=DEV)
     badpos = torch.tensor([0, 64 * wl.max_pages], dtype=torch.int32, device=DEV)
-    spot.tok_append_selector_keys(desc, pool, wl.page_table, bad, badpos, keys[:2].contiguous(),
+    spot.tok_append_selector_keys(desc, pool, None, wl.page_table, bad, badpos,
+                                  keys[:2].contiguous(),
                                   ws)
     torch.cuda.synchronize()
     assert spot.read_device_status(ws) == 5              # SPOT_ERR_DEVICE_BOUNDS
@@ -162,3 +165,69 @@ def test_tok_bad_selection_is_reported_not_faulted():
     torch.cuda.synchronize()
     assert spot.read_device_status(ws) == 5
     assert torch.isfinite(out).all()
+
+
+# ------------------------------------------------ quantised per-token keys
+
+QFMTS = ["int4", "mxfp4", "fp8", "int8"]
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_tok_append_quantises_like_the_oracle(fmt):
+    wl = workloads.make_tok("tok_tiny_2k", seed=12, device=DEV, batch=2, seq_len=None,
+                            ragged_range=(700, 2048))
+    desc = spot.tok_layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, sel_fmt=fmt)
+    data, scales = gpu_tok_pool(wl, fmt, desc)
+    ref_d, ref_s = oracle.quantize_selector(fmt, workloads.bits(wl.sel_tok))
+    lens = wl.seq_lens.cpu().numpy()
+    pt = wl.page_table.cpu().numpy()
+    rows = np.zeros(wl.num_pages * 64, bool)          # (page, slot) rows that were appended
+    for b, L in enumerate(lens):
+        for t in range(int(L)):
+            rows[pt[b, t // 64] * 64 + t % 64] = True
+    gd = data.cpu().view(torch.uint8).numpy().reshape(wl.num_pages * 64, -1)
+    assert np.array_equal(gd[rows], ref_d.view(np.uint8).reshape(wl.num_pages * 64, -1)[rows])
+    if ref_s is not None:
+        gs = scales.cpu()
+        gs = (gs.view(torch.int16).numpy().view(np.uint16) if gs.dtype == torch.float16
+              else gs.numpy()).reshape(wl.num_pages * 64, -1)
+        assert np.array_equal(gs[rows], ref_s.reshape(wl.num_pages * 64, -1)[rows])
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_tok_quantised_keys_tiny(fmt):
+    wl = workloads.make_tok("tok_tiny_2k", seed=13, device=DEV)
+    gpu = run_gpu_tok(wl, fmt=fmt)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl, fmt)
+    ora = run_oracle_tok(wl, args=args, fmt=fmt)
+    scores = oracle_tok_scores(wl, args=args, fmt=fmt)
+    assert check_tok_selection_near_cut(gpu, ora, scores, wl) <= 1
+    _, n = check_tok_outputs(gpu, ora, wl)
+    assert n >= wl.batch - 1
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "fp8"])
+def test_tok_quantised_integer_keys_select_bit_exact(fmt):
+    # keys in {-3..3} are stored losslessly by MXFP4 (power-of-two group
+    # scales) and E4M3: every score stays exact on both sides
+    wl = workloads.make_tok("tok_tiny_2k", seed=14, device=DEV, integer=True, batch=3,
+                            seq_len=None, ragged_range=(64, 4096))
+    wl.top_p = safe_top_p_tok(wl, fmt=fmt)
+    gpu = run_gpu_tok(wl, fmt=fmt)
+    assert gpu["status"] == 0
+    ora = run_oracle_tok(wl, fmt=fmt)
+    _same(gpu, ora, wl)
+    check_tok_outputs(gpu, ora, wl)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+def test_tok_quantised_keys_full_size(fmt):
+    wl = workloads.make_tok("qwen3_8b_128k_tok", seed=2, device=DEV)
+    gpu = run_gpu_tok(wl, fmt=fmt)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl, fmt)
+    ora = run_oracle_tok(wl, args=args, fmt=fmt)
+    scores = oracle_tok_scores(wl, args=args, fmt=fmt)
+    assert check_tok_selection_near_cut(gpu, ora, scores, wl) <= 1
+    check_tok_outputs(gpu, ora, wl)
