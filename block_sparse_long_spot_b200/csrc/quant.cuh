@@ -13,6 +13,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <math.h>
 #include <stdint.h>
@@ -128,6 +129,57 @@ __device__ __forceinline__ uint32_t pair8_to_bf16x2(uint32_t two) {
                                                      __NV_E4M3);
     const float2 f = __half22float2(__half2(hr));
     return pack_bf16(f.x, f.y);
+}
+
+// ---- code -> f16 widening for the per-token scorer.  Every INT4, E2M1,
+// INT8 and E4M3 value is an f16 number, so the widening is exact.
+
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+    const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a),
+                              *reinterpret_cast<const __half2*>(&b));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// 4 E4M3 codes (byte j = element j) -> f16x2 lo = (0, 1), hi = (2, 3).
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const __half2_raw a =
+        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+    const __half2_raw b =
+        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+    lo = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    hi = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
+}
+
+// 4 INT8 codes (byte j = element j) -> f16x2 lo = (0, 1), hi = (2, 3).  A
+// code v with its sign bit flipped is the byte v + 128; placed under the
+// high byte 0x64 it forms the f16 number 1024 + v + 128, and subtracting
+// 1152 (0x6480) leaves v.
+__device__ __forceinline__ void int8x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    lo = hsub2_bits(prmt(u, 0x64646464u, 0x4140u), 0x64806480u);
+    hi = hsub2_bits(prmt(u, 0x64646464u, 0x4342u), 0x64806480u);
+}
+
+// 8 INT4 codes (nibble j = element j) -> f16x2 out[j] = (j, j + 4), j < 4.
+// Same construction with nibbles: 1024 + v + 8 (mantissa bits 0..3) minus
+// 1032 (0x6408).
+__device__ __forceinline__ void int4x8_to_f16x2(uint32_t w, uint32_t (&out)[4]) {
+    const uint32_t u = w ^ 0x88888888u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        out[j] = hsub2_bits(((u >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0x64086408u);
+}
+
+// 8 E2M1 codes (nibble j = element j) -> f16x2 out[j] = (j, j + 4), j < 4,
+// each f16 equal to the code's value times 2^-14: the magnitude bits (e1 e0
+// m) moved to f16 bits 11..9 read as 2^(e - 15) (1 + m / 2) for e > 0 and as
+// the subnormal m 2^-15 for e = 0; the sign bit moves to bit 15.
+__device__ __forceinline__ void e2m1x8_to_f16x2_scaled(uint32_t w, uint32_t (&out)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t x = w >> (4 * j);
+        out[j] = ((x << 9) & 0x0E000E00u) | ((x << 12) & 0x80008000u);
+    }
 }
 
 // E8M0 scale byte -> its value 2^(e - 127) (255 is NaN).

@@ -67,9 +67,12 @@ __device__ __forceinline__ int range_begin(int64_t N, int64_t P, int64_t i) {
 
 // The scores of the 64 (token, head) rows of m-tile group `mt` (rows
 // 16 mt + r8 and + 8 of the stage) against Q^T: per row, the dot with the
-// query of every index head (column h), scales applied.  The head dimension
-// is consumed in a format-dependent order, the same for keys and queries
-// (qf holds the query fragments in that order).
+// query of every index head (column h), scales applied.  bf16 keys meet the
+// bf16 queries; codes of the other formats are widened exactly to f16 and
+// meet f16 queries that carry a power-of-two factor per index head (undone
+// by the caller).  The head dimension is consumed in a format-dependent
+// order, the same for keys and queries (qf holds the query fragments in that
+// order):
 //   bf16:  the stage holds two 64 x 64 bf16 halves (128-byte swizzle);
 //   8-bit: 64 rows of 128 code bytes (128-byte swizzle); 16-byte chunk c is
 //          dims 16 c .. 16 c + 15;
@@ -82,28 +85,30 @@ __device__ __forceinline__ void tile_dots(uint32_t kb, const uint8_t* sc_smem, i
     acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
     const int r8 = lane >> 2;
     const int rowA = mt * 16 + r8, rowB = rowA + 8;       // this lane's two rows
+    const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);   // ldmatrix address row
     if constexpr (FMT == SPOT_SEL_BF16) {
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint32_t hb = kb + (ks >> 2) * (tok_code_bytes(FMT) / 2);
             const int chunk = ((ks & 3) << 1) + (lane >> 4);
-            const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
             uint32_t a0, a1, a2, a3;
             ldsm_x4(swz128(hb, row, chunk), a0, a1, a2, a3);
             mma_bf16_16816(acc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
         }
     } else if constexpr (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
-        const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        // word j of a chunk row: dims 4 j .. 4 j + 3 -> (0, 1) and (2, 3)
 #pragma unroll
         for (int cp = 0; cp < 4; ++cp) {
-            uint32_t r0, r1, r2, r3;                       // chunks 2 cp, 2 cp + 1
-            ldsm_x4(swz128(kb, row, 2 * cp + (lane >> 4)), r0, r1, r2, r3);
-            mma_bf16_16816(acc, pair8_to_bf16x2<FMT>(r0), pair8_to_bf16x2<FMT>(r1),
-                           pair8_to_bf16x2<FMT>(r0 >> 16), pair8_to_bf16x2<FMT>(r1 >> 16),
-                           qf[2 * cp][0], qf[2 * cp][1]);
-            mma_bf16_16816(acc, pair8_to_bf16x2<FMT>(r2), pair8_to_bf16x2<FMT>(r3),
-                           pair8_to_bf16x2<FMT>(r2 >> 16), pair8_to_bf16x2<FMT>(r3 >> 16),
-                           qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+            uint32_t r[4];                                 // rows A / B of chunks 2 cp, 2 cp + 1
+            ldsm_x4(swz128(kb, row, 2 * cp + (lane >> 4)), r[0], r[1], r[2], r[3]);
+            uint32_t lo[4], hi[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if constexpr (FMT == SPOT_SEL_FP8_E4M3) e4m3x4_to_f16x2(r[i], lo[i], hi[i]);
+                else int8x4_to_f16x2(r[i], lo[i], hi[i]);
+            }
+            mma_f16_16816(acc, lo[0], lo[1], hi[0], hi[1], qf[2 * cp][0], qf[2 * cp][1]);
+            mma_f16_16816(acc, lo[2], lo[3], hi[2], hi[3], qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
         }
         if constexpr (FMT == SPOT_SEL_INT8_F16) {
             const __half* s = reinterpret_cast<const __half*>(sc_smem);
@@ -114,26 +119,29 @@ __device__ __forceinline__ void tile_dots(uint32_t kb, const uint8_t* sc_smem, i
             acc[3] *= sb;
         }
     } else {
-        const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        // word of a chunk row: dims 8 j .. 8 j + 7 -> four f16x2 a[i] holding
+        // dims (i, i + 4); k-step t takes a[2t], a[2t + 1]
         float g[4][4];
 #pragma unroll
         for (int cp = 0; cp < 2; ++cp) {
-            const int c = 2 * cp + (lane >> 4);            // this lane's address: chunk c
-            uint32_t r0, r1, r2, r3;                       // chunks 2 cp, 2 cp + 1
-            ldsm_x4(swz128(kb, row >> 1, ((row & 1) << 2) + c), r0, r1, r2, r3);
+            uint32_t r[4];                                 // rows A / B of chunks 2 cp, 2 cp + 1
+            ldsm_x4(swz128(kb, row >> 1, ((row & 1) << 2) + 2 * cp + (lane >> 4)), r[0], r[1],
+                    r[2], r[3]);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const uint32_t ra = h ? r2 : r0, rb = h ? r3 : r1;
-                float (&a)[4] = g[2 * cp + h];
-                a[0] = a[1] = a[2] = a[3] = 0.f;
-                mma_bf16_16816(a, byte_to_bf16x2<FMT>(ra & 0xFFu), byte_to_bf16x2<FMT>(rb & 0xFFu),
-                               byte_to_bf16x2<FMT>((ra >> 8) & 0xFFu),
-                               byte_to_bf16x2<FMT>((rb >> 8) & 0xFFu), qf[2 * (2 * cp + h)][0],
-                               qf[2 * (2 * cp + h)][1]);
-                mma_bf16_16816(a, byte_to_bf16x2<FMT>((ra >> 16) & 0xFFu),
-                               byte_to_bf16x2<FMT>((rb >> 16) & 0xFFu), byte_to_bf16x2<FMT>(ra >> 24),
-                               byte_to_bf16x2<FMT>(rb >> 24), qf[2 * (2 * cp + h) + 1][0],
-                               qf[2 * (2 * cp + h) + 1][1]);
+                const int c = 2 * cp + h;                  // scale group
+                uint32_t a[4], b[4];
+                if constexpr (FMT == SPOT_SEL_INT4_G32_F16) {
+                    int4x8_to_f16x2(r[2 * h], a);
+                    int4x8_to_f16x2(r[2 * h + 1], b);
+                } else {                                   // values x 2^-14
+                    e2m1x8_to_f16x2_scaled(r[2 * h], a);
+                    e2m1x8_to_f16x2_scaled(r[2 * h + 1], b);
+                }
+                float (&gc)[4] = g[c];
+                gc[0] = gc[1] = gc[2] = gc[3] = 0.f;
+                mma_f16_16816(gc, a[0], b[0], a[1], b[1], qf[2 * c][0], qf[2 * c][1]);
+                mma_f16_16816(gc, a[2], b[2], a[3], b[3], qf[2 * c + 1][0], qf[2 * c + 1][1]);
             }
         }
 #pragma unroll
@@ -155,35 +163,69 @@ __device__ __forceinline__ void tile_dots(uint32_t kb, const uint8_t* sc_smem, i
     }
 }
 
-// Query fragments (B operand, n = index head r8, heads 4..7 zero) in the
-// order tile_dots consumes the head dimension: k-step ks, pair (2 c4, +1)
-// and (2 c4 + 8, +9) of the fragment map to dims
-//   bf16:  16 ks + 2 c4 + {0,1} and + 8     (u32 8 ks + c4, 8 ks + 4 + c4)
-//   8-bit: 16 ks + 4 c4 + {0,1} and {2,3}  (u32 8 ks + 2 c4, + 1)
-//   4-bit: step ks = 2 c + t: 32 c + 8 c4 + 4 t + {0,1} and {2,3}
-//          (u32 16 c + 4 c4 + 2 t, + 1)
+// Head dimension of element e (0 = low, 1 = high half) of B-fragment
+// register j (0, 1) at k-step ks for lane quad position c4, in the order
+// tile_dots consumes the dimension:
+//   bf16:  16 ks + 2 c4 + e + 8 j
+//   8-bit: 16 ks + 4 c4 + 2 j + e
+//   4-bit: 32 c + 8 c4 + 2 t + j + 4 e     (ks = 2 c + t)
 template <int FMT>
-__device__ __forceinline__ void load_tok_queries(const uint16_t* q_idx, int b, int lane,
-                                                 uint32_t (&qf)[8][2]) {
+__device__ __forceinline__ int query_dim(int ks, int j, int e, int c4) {
+    if constexpr (FMT == SPOT_SEL_BF16) return 16 * ks + 2 * c4 + e + 8 * j;
+    else if constexpr (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16)
+        return 16 * ks + 4 * c4 + 2 * j + e;
+    else return 32 * (ks >> 1) + 8 * c4 + 2 * (ks & 1) + j + 4 * e;
+}
+
+// Query fragments (B operand, n = index head r8, heads 4..7 zero).  bf16
+// keys: the bf16 queries as they are (returns 1).  Other formats: f16
+// copies of q * 2^s with s chosen per index head so that the head's largest
+// |q| lands in [2^14, 2^15) -- no overflow, and only elements below 2^-29 of
+// that maximum round -- returning 2^-s for the head of this lane's column
+// (index head (lane >> 2) & 3), times 2^14 for MXFP4 (whose widened keys
+// carry 2^-14).
+template <int FMT>
+__device__ __forceinline__ float load_tok_queries(const uint16_t* q_idx, int b, int lane,
+                                                  uint32_t (&qf)[8][2]) {
     const int c4 = lane & 3, r8 = lane >> 2;
     const bool real = r8 < kIdxHeads;
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-        q_idx + (static_cast<int64_t>(b) * kIdxHeads + (real ? r8 : 0)) * kIdxDim);
+    const uint16_t* qrow = q_idx + (static_cast<int64_t>(b) * kIdxHeads + (real ? r8 : 0)) * kIdxDim;
+    if constexpr (FMT == SPOT_SEL_BF16) {
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-        int i0, i1;
-        if constexpr (FMT == SPOT_SEL_BF16) {
-            i0 = 8 * ks + c4;
-            i1 = 8 * ks + 4 + c4;
-        } else if constexpr (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
-            i0 = 8 * ks + 2 * c4;
-            i1 = i0 + 1;
-        } else {
-            i0 = 16 * (ks >> 1) + 4 * c4 + 2 * (ks & 1);
-            i1 = i0 + 1;
-        }
-        qf[ks][0] = real ? __ldg(qrow + i0) : 0u;
-        qf[ks][1] = real ? __ldg(qrow + i1) : 0u;
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int d = query_dim<FMT>(ks, j, 0, c4);          // even: a bf16 pair
+                qf[ks][j] = real ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d)) : 0u;
+            }
+        return 1.f;
+    } else {
+        float v[8][2][2];
+        float am = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const uint16_t bits = real ? __ldg(qrow + query_dim<FMT>(ks, j, e, c4)) : 0;
+                    v[ks][j][e] = __uint_as_float(static_cast<uint32_t>(bits) << 16);
+                    am = fmaxf(am, fabsf(v[ks][j][e]));
+                }
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));   // the quad holds one head
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+        const int sh = am > 0.f ? min(120, max(-113, 14 - ilogbf(am))) : 0;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const __half2 h = __floats2half2_rn(ldexpf(v[ks][j][0], sh), ldexpf(v[ks][j][1], sh));
+                qf[ks][j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+        // 2^-sh of index head (lane >> 2) & 3, held by quad lanes 4 * head
+        const int sh_col = __shfl_sync(0xffffffffu, sh, 4 * ((lane >> 2) & 3));
+        const int e = (FMT == SPOT_SEL_MXFP4_G32_E8M0 ? 14 : 0) - sh_col;
+        return __int_as_float((127 + e) << 23);
     }
 }
 
@@ -321,13 +363,13 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
     const bool odd = head & 1;
     int cur_b = -1;
     uint32_t qf[8][2];
-    float wh = 0.f;
+    float wh = 0.f, unscale = 1.f;
     for (int it = warp; it < n_it; it += NCS) {
         const int pos = beg + it;
         const int b = find_seq(seq_off, B, pos);
         const int j = pos - seq_off[b];
         if (b != cur_b) {
-            load_tok_queries<FMT>(p.q_idx, b, lane, qf);
+            unscale = load_tok_queries<FMT>(p.q_idx, b, lane, qf);
             wh = p.w ? p.w[static_cast<int64_t>(b) * kIdxHeads + head] : 1.f / kIdxHeads;
             cur_b = b;
         }
@@ -350,8 +392,8 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
         for (int mt = 0; mt < 4; ++mt) {
             float acc[4];
             tile_dots<FMT>(kb, scl, mt, lane, qf, acc);
-            float top = odd ? acc[1] : acc[0];
-            float bot = odd ? acc[3] : acc[2];
+            float top = (odd ? acc[1] : acc[0]) * unscale;
+            float bot = (odd ? acc[3] : acc[2]) * unscale;
             top = owner ? wh * fmaxf(top, 0.f) : 0.f;
             bot = owner ? wh * fmaxf(bot, 0.f) : 0.f;
 #pragma unroll

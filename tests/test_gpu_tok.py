@@ -231,3 +231,27 @@ def test_tok_quantised_keys_full_size(fmt):
     scores = oracle_tok_scores(wl, args=args, fmt=fmt)
     assert check_tok_selection_near_cut(gpu, ora, scores, wl) <= 1
     check_tok_outputs(gpu, ora, wl)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "fp8"])
+def test_tok_every_e2m1_magnitude_bit_exact(fmt):
+    # Keys over {0, +-1/4, +-1/2, +-3/4, +-1, +-3/2, +-2, +-3} (the planted +-3
+    # kept): each MXFP4 group's codes are exact -- all eight E2M1 magnitudes
+    # occur, the zero-exponent 0.5 among them -- and so are the E4M3 codes;
+    # with integer queries every score is exact in any precision, so the
+    # selections must match the oracle's.
+    wl = workloads.make_tok("tok_tiny_2k", seed=16, device=DEV, integer=True, batch=3,
+                            seq_len=None, ragged_range=(64, 4096))
+    vals = torch.tensor([0.0, 0.25, 0.5, 0.75, 1.0, 1.5, 2.0, 3.0], device=DEV)
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(16)
+    mag = vals[torch.randint(0, 8, wl.sel_tok.shape, generator=gen, device=DEV)]
+    sign = torch.where(torch.rand(wl.sel_tok.shape, generator=gen, device=DEV) < 0.5, -1.0, 1.0)
+    keep = wl.sel_tok.float().abs() == 3
+    wl.sel_tok = torch.where(keep, wl.sel_tok.float(), mag * sign).to(torch.bfloat16)
+    wl.top_p = safe_top_p_tok(wl, fmt=fmt)
+    gpu = run_gpu_tok(wl, fmt=fmt)
+    assert gpu["status"] == 0
+    ora = run_oracle_tok(wl, fmt=fmt)
+    _same(gpu, ora, wl)
+    check_tok_outputs(gpu, ora, wl)
