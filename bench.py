@@ -391,7 +391,7 @@ def run_spot(args, world, rank, local):
         "graph": {"ms_per_step": round(ms_graph, 5),
                   "value": round(shard_summary(B, world, ms_graph, layers_model), 3),
                   "note": "the same steps replayed from captured CUDA graphs"},
-        "gpu_launches": K * 2,          # selection (scoring fused), sparse decode per step
+        "gpu_launches": K * 3,          # block scoring, selection, sparse decode per step
         "clocks": clk.summary(),
     }
     return res, layers

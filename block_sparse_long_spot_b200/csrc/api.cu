@@ -112,28 +112,26 @@ bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Lay
     L.status = off;
     off += kStatusBytes;
     L.unit_done = off;
+    off += static_cast<size_t>(U) * sizeof(uint32_t);
+    L.sel_done = off;
     off = round_up(off + static_cast<size_t>(U) * sizeof(uint32_t), 256);
     L.partials = off;
     off = round_up(off + static_cast<size_t>(grid + U) * G * kPartialFloatsPerHead * sizeof(float),
                    256);
+    L.scores = off;
+    off = round_up(off + static_cast<size_t>(U) * max_blocks * sizeof(float), 256);
     L.total = off;
-    L.tok_scores = 0;
     *out = L;
     return true;
 }
 
-// Token selector: the decode layout of (batch x num_kv_heads) units plus the
-// block scores [batch][max_blocks] fp32.
+// Token selector: the decode layout of (batch x num_kv_heads) units; its
+// block scores [batch][max_blocks] use the front of the scores region.
 bool tok_workspace_layout(const spot_tok_layer_desc_t* d, int batch, int max_blocks,
                           Layout* out) {
     spot_layer_desc_t bd = {d->num_q_heads, d->num_kv_heads, kHeadDim, kBlock, kSelDim,
                             SPOT_SEL_BF16, d->num_pages};
-    Layout L;
-    if (!workspace_layout(&bd, batch, max_blocks, &L)) return false;
-    L.tok_scores = L.total;
-    L.total = round_up(L.total + static_cast<size_t>(batch) * max_blocks * sizeof(float), 256);
-    *out = L;
-    return true;
+    return workspace_layout(&bd, batch, max_blocks, out);
 }
 
 }  // namespace spot
@@ -173,7 +171,9 @@ spot_status_t do_select(const spot_layer_desc_t* d, const spot_select_params_t* 
     sl.topk_blocks = pr->topk_blocks;
     sl.quantize_queries = pr->quantize_queries;
     sl.blocks_per_page = 1;
-    sl.scores_in = nullptr;
+    sl.scores_out = reinterpret_cast<float*>(base + L.scores);
+    sl.scores_in = sl.scores_out;
+    sl.sel_done = reinterpret_cast<uint32_t*>(base + L.sel_done);
     sl.sel_idx = sel_idx;
     sl.sel_cnt = sel_cnt;
     sl.status = reinterpret_cast<uint32_t*>(base + L.status);
@@ -472,7 +472,7 @@ spot_status_t do_tok_select(const spot_tok_layer_desc_t* d, const spot_select_pa
             : make_bytes_map(&sm, sel_data, rows * rb / 128, (kTokBlock * kIdxHeads * rb) / 128);
     if (!ok_map) return SPOT_ERR_CUDA;
     uint8_t* base = static_cast<uint8_t*>(ws);
-    float* scores = reinterpret_cast<float*>(base + L.tok_scores);
+    float* scores = reinterpret_cast<float*>(base + L.scores);
     uint32_t* status = reinterpret_cast<uint32_t*>(base + L.status);
     TokScoreParams tp;
     tp.q_idx = q_idx;

@@ -1,8 +1,11 @@
 // select.cu -- selector scoring and block selection (SpotAttention §2.1,
-// §2.3 Eq. 6-8), one fused kernel with one CTA per (sequence, KV head).
+// §2.3 Eq. 6-8): a scoring kernel spread over the whole GPU, then the
+// selection kernel (one CTA per (sequence, KV head)) launched behind it with
+// programmatic dependent launch.
 //
 // Scoring: s[j] = (1/tau) sum_{h in group} w[b,h] ReLU(q_sel[b,h] . k[page(b,j),g])
-//   for every complete block j.  Each warp scores tiles of 16 blocks with
+//   for every complete block j.  A CTA of 4 warps takes 256 blocks of one
+//   unit; each warp scores tiles of 16 blocks with
 //   bf16 mma.sync (keys as the M operand, the group's selector queries as
 //   N = 8), four tiles at a time so their gathered loads are in flight
 //   together.  INT4 / MXFP4 / INT8 / FP8 E4M3 keys are widened to bf16 in
@@ -12,8 +15,8 @@
 //   group's selector queries are first quantised with the key format's rule
 //   (quant.cuh) and their scales join the keys' after the mma.  The head
 //   dimension is consumed in a permuted order, identical for the keys and the
-//   queries, that lets every lane load 16 contiguous bytes.  Scores stay in
-//   shared memory.
+//   queries, that lets every lane load 16 contiguous bytes.  The scores go
+//   to the workspace ([unit][block] fp32, read back from L2).
 //
 // Selection: residual softmax numerators exp(s - max) are computed in fp64
 //   and held as 2^-40 fixed-point integers (exact, order-independent sums).
@@ -27,10 +30,13 @@
 //   block index first).  The K_min floor and static top-K use the same search
 //   on counts.  A block scan compacts the kept blocks in ascending order.
 //
-// The token-level selector reuses the selection with its block scores
-// computed by tok_select.cu (one CTA per sequence, blocks of 16 tokens).
+// The token-level selector and sparse prefill reuse the selection with their
+// block scores computed by tok_select.cu (one unit per sequence, blocks of 16
+// tokens) and prefill.cu (one unit per (query tile, KV head)).
 #include <cuda_fp8.h>
 #include <math.h>
+
+#include <mutex>
 
 #include "quant.cuh"
 #include "spot_device.cuh"
@@ -585,47 +591,46 @@ size_t select_smem_bytes(int max_blocks) {
 namespace {
 
 
-template <int FMT>
-__global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectParams p) {
-    extern __shared__ __align__(16) uint8_t smem[];
+// Shared-memory carve-up of the selection (select_smem_bytes(max_blocks)
+// bytes): 8-byte arrays first, then 4-, 2- and 1-byte ones, so every array
+// stays aligned whatever max_blocks is.
+__device__ __forceinline__ SelSmem carve_select_smem(uint8_t* smem, int max_blocks) {
     SelSmem sm;
-    {
-        uint8_t* q = smem;
-        // 8-byte arrays first, then 4-, 2- and 1-byte ones: every array stays
-        // aligned whatever max_blocks is
-        sm.mass = reinterpret_cast<unsigned long long*>(q);
-        q += sizeof(unsigned long long) * p.max_blocks;
-        sm.cval = reinterpret_cast<unsigned long long*>(q);
-        q += sizeof(unsigned long long) * NT;
-        sm.red = reinterpret_cast<unsigned long long*>(q);
-        q += sizeof(unsigned long long) * 3 * NW;
-        sm.score = reinterpret_cast<float*>(q);
-        q += sizeof(float) * p.max_blocks;
-        sm.keys = reinterpret_cast<uint32_t*>(q);
-        q += sizeof(uint32_t) * p.max_blocks;
-        sm.hmass = reinterpret_cast<uint32_t*>(q);
-        q += sizeof(uint32_t) * kNB;
-        sm.hcnt = reinterpret_cast<uint32_t*>(q);
-        q += sizeof(uint32_t) * kNB;
-        sm.ckey = reinterpret_cast<uint32_t*>(q);
-        q += sizeof(uint32_t) * NT;
-        sm.cidx = reinterpret_cast<int*>(q);
-        q += sizeof(int) * NT;
-        sm.misc = reinterpret_cast<int*>(q);
-        q += sizeof(int) * 8;
-        sm.scan = reinterpret_cast<int*>(q);
-        q += sizeof(int) * (NW + 1);
-        sm.fscan = reinterpret_cast<float*>(q);
-        q += sizeof(float) * (NW + 1);
-        sm.vb = reinterpret_cast<uint16_t*>(q);
-        q += sizeof(uint16_t) * p.max_blocks;
-        sm.keep = q;
-    }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // precomputed scores: the lengths and p may come from a preceding kernel too
-    if constexpr (FMT == kSelectFromScores) pdl_wait();
+    uint8_t* q = smem;
+    sm.mass = reinterpret_cast<unsigned long long*>(q);
+    q += sizeof(unsigned long long) * max_blocks;
+    sm.cval = reinterpret_cast<unsigned long long*>(q);
+    q += sizeof(unsigned long long) * NT;
+    sm.red = reinterpret_cast<unsigned long long*>(q);
+    q += sizeof(unsigned long long) * 3 * NW;
+    sm.score = reinterpret_cast<float*>(q);
+    q += sizeof(float) * max_blocks;
+    sm.keys = reinterpret_cast<uint32_t*>(q);
+    q += sizeof(uint32_t) * max_blocks;
+    sm.hmass = reinterpret_cast<uint32_t*>(q);
+    q += sizeof(uint32_t) * kNB;
+    sm.hcnt = reinterpret_cast<uint32_t*>(q);
+    q += sizeof(uint32_t) * kNB;
+    sm.ckey = reinterpret_cast<uint32_t*>(q);
+    q += sizeof(uint32_t) * NT;
+    sm.cidx = reinterpret_cast<int*>(q);
+    q += sizeof(int) * NT;
+    sm.misc = reinterpret_cast<int*>(q);
+    q += sizeof(int) * 8;
+    sm.scan = reinterpret_cast<int*>(q);
+    q += sizeof(int) * (NW + 1);
+    sm.fscan = reinterpret_cast<float*>(q);
+    q += sizeof(float) * (NW + 1);
+    sm.vb = reinterpret_cast<uint16_t*>(q);
+    q += sizeof(uint16_t) * max_blocks;
+    sm.keep = q;
+    return sm;
+}
 
-    const int u = blockIdx.x;
+// Selection of unit u (all threads of the CTA) on its block scores: in
+// shared memory already (`in_smem`), else read from p.scores_in.
+__device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, bool in_smem) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = u / p.num_kv_heads;
     const int L = max(p.seq_lens[b], 0);
     const int bsz = kBlock / p.blocks_per_page;        // tokens per selection block
@@ -651,7 +656,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     pdl_trigger();                                    // the decode kernel may start its prologue
 
     // ---- selector scores of the complete blocks (§2.1), into shared memory
-    if constexpr (FMT == kSelectFromScores) {
+    if (!in_smem) {
         const float* src = p.scores_in + static_cast<int64_t>(u) * p.max_blocks;
         constexpr int kBatch = 8;                     // loads in flight per thread
         for (int j0 = threadIdx.x; j0 < n_full; j0 += NT * kBatch) {
@@ -664,23 +669,6 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
 #pragma unroll
             for (int k = 0; k < kBatch; ++k)
                 if (j0 + k * NT < n_full) sm.score[j0 + k * NT] = v[k];
-        }
-    } else {
-        const int g = u - b * p.num_kv_heads;
-        uint32_t qw[8];
-        float qsc[2][2], wh0, wh1;
-        load_queries<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
-        const int tiles = (n_full + 15) / 16;
-        const int step = NW * kTileBatch;
-        int pa[kTileBatch], pb[kTileBatch];
-        if (warp < tiles) load_pages(p, b, warp, NW, n_full, lane, pa, pb);
-        for (int t0 = warp; t0 < tiles; t0 += step) {
-            // the next batch's page ids load while this batch's keys do
-            int na[kTileBatch], nb2[kTileBatch];
-            if (t0 + step < tiles) load_pages(p, b, t0 + step, NW, n_full, lane, na, nb2);
-            score_tiles<FMT>(p, g, qw, qsc, wh0, wh1, t0, NW, n_full, sm.score, lane, pa, pb);
-#pragma unroll
-            for (int k = 0; k < kTileBatch; ++k) { pa[k] = na[k]; pb[k] = nb2[k]; }
         }
     }
     __syncthreads();
@@ -886,40 +874,123 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     if (threadIdx.x == 0) p.sel_cnt[u] = cnt;
 }
 
+// Selection on scores computed by a preceding kernel (token-level selector,
+// sparse prefill): one CTA per unit.
+__global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const SelSmem sm = carve_select_smem(smem, p.max_blocks);
+    pdl_wait();                  // the scores (and the lengths and p) may come from it
+    select_unit(p, blockIdx.x, sm, false);
+}
+
+// Scoring (§2.1, Eq. 2) and selection in one launch.  The C CTAs of a unit
+// share its 16-block tiles: CTA c takes rounds c, c + C, ... of 64 tiles
+// (one batch of kTileBatch tiles per warp per round, the next round's page
+// ids loading while this round's keys do).  With C = 1 the scores stay in
+// shared memory and the CTA selects at once; otherwise they go to
+// p.scores_out and the unit's last CTA to finish -- a per-unit arrival
+// counter in the workspace, reset to zero by that CTA -- selects from them.
+template <int FMT>
+__global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const SelectParams p,
+                                                                         int C) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const SelSmem sm = carve_select_smem(smem, p.max_blocks);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int u = blockIdx.x / C, c = blockIdx.x - u * C;
+    const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+    const int L = max(p.seq_lens[b], 0);
+    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
+    const int n_full = min(L / (kBlock / p.blocks_per_page), cap);   // overflow: flagged
+    const int tiles = (n_full + 15) / 16;                            // by the selection
+    float* out = C == 1 ? sm.score : p.scores_out + static_cast<int64_t>(u) * p.max_blocks;
+    constexpr int kRound = NW * kTileBatch;
+    const int step = C * kRound;
+    const int first = c * kRound + warp;
+    if (first < tiles) {                                             // warp-uniform
+        uint32_t qw[8];
+        float qsc[2][2], wh0, wh1;
+        load_queries<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
+        int pa[kTileBatch], pb[kTileBatch];
+        load_pages(p, b, first, NW, n_full, lane, pa, pb);
+        for (int t0 = first; t0 < tiles; t0 += step) {
+            int na[kTileBatch], nb2[kTileBatch];
+            if (t0 + step < tiles) load_pages(p, b, t0 + step, NW, n_full, lane, na, nb2);
+            score_tiles<FMT>(p, g, qw, qsc, wh0, wh1, t0, NW, n_full, out, lane, pa, pb);
+#pragma unroll
+            for (int k = 0; k < kTileBatch; ++k) { pa[k] = na[k]; pb[k] = nb2[k]; }
+        }
+    }
+    if (C > 1) {
+        __syncthreads();                              // this CTA's score stores are issued
+        if (threadIdx.x == 0) {
+            __threadfence();                          // ... and visible before it arrives
+            const unsigned old = atomicAdd(&p.sel_done[u], 1u);
+            const int last = old == static_cast<unsigned>(C - 1);
+            if (last) p.sel_done[u] = 0u;
+            sm.misc[7] = last;
+        }
+        __syncthreads();
+        if (!sm.misc[7]) return;
+        __threadfence();                              // the other CTAs' scores
+    }
+    select_unit(p, u, sm, C == 1);
+}
+
+}  // namespace
+
+namespace {
+
+std::mutex g_sms_mutex;
+int g_sms[64] = {};
+
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lock(g_sms_mutex);
+    if (g_sms[dev] == 0 &&
+        cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        g_sms[dev] = 0;
+    return g_sms[dev];
+}
+
+template <int FMT>
+cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(score_select_kernel<FMT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    // CTAs per unit: enough to cover the longest sequence in one round of
+    // 64 tiles each, as far as one wave of one CTA per SM allows
+    const int U = p.batch * p.num_kv_heads;
+    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
+    const int rounds = max(1, ((cap + 15) / 16 + NW * kTileBatch - 1) / (NW * kTileBatch));
+    const int C = max(1, min(rounds, sm_count() / max(U, 1)));
+    score_select_kernel<FMT><<<U * C, kSelectThreads, smem, s>>>(p, C);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s) {
     const size_t smem = select_smem_bytes(p.max_blocks);
-    const dim3 grid(p.batch * p.num_kv_heads), block(kSelectThreads);
-    cudaError_t e;
-    if (fmt == kSelectFromScores) {
-        e = cudaFuncSetAttribute(select_kernel<kSelectFromScores>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess)
-            e = launch_pdl(select_kernel<kSelectFromScores>, grid, block, smem, s, p);
-    } else if (fmt == SPOT_SEL_BF16) {
-        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_BF16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess) select_kernel<SPOT_SEL_BF16><<<grid, block, smem, s>>>(p);
-    } else if (fmt == SPOT_SEL_INT4_G32_F16) {
-        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_INT4_G32_F16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess) select_kernel<SPOT_SEL_INT4_G32_F16><<<grid, block, smem, s>>>(p);
-    } else if (fmt == SPOT_SEL_MXFP4_G32_E8M0) {
-        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_MXFP4_G32_E8M0>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess) select_kernel<SPOT_SEL_MXFP4_G32_E8M0><<<grid, block, smem, s>>>(p);
-    } else if (fmt == SPOT_SEL_FP8_E4M3) {
-        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_FP8_E4M3>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess) select_kernel<SPOT_SEL_FP8_E4M3><<<grid, block, smem, s>>>(p);
-    } else {
-        e = cudaFuncSetAttribute(select_kernel<SPOT_SEL_INT8_F16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess) select_kernel<SPOT_SEL_INT8_F16><<<grid, block, smem, s>>>(p);
+    if (p.batch * p.num_kv_heads <= 0) return cudaErrorInvalidValue;
+    switch (fmt) {
+        case kSelectFromScores: {
+            const cudaError_t e = cudaFuncSetAttribute(
+                select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            if (e != cudaSuccess) return e;
+            const dim3 grid(p.batch * p.num_kv_heads), block(kSelectThreads);
+            const cudaError_t l = launch_pdl(select_kernel, grid, block, smem, s, p);
+            return l != cudaSuccess ? l : cudaGetLastError();
+        }
+        case SPOT_SEL_BF16: return launch_score_select<SPOT_SEL_BF16>(p, smem, s);
+        case SPOT_SEL_INT4_G32_F16: return launch_score_select<SPOT_SEL_INT4_G32_F16>(p, smem, s);
+        case SPOT_SEL_MXFP4_G32_E8M0:
+            return launch_score_select<SPOT_SEL_MXFP4_G32_E8M0>(p, smem, s);
+        case SPOT_SEL_FP8_E4M3: return launch_score_select<SPOT_SEL_FP8_E4M3>(p, smem, s);
+        case SPOT_SEL_INT8_F16: return launch_score_select<SPOT_SEL_INT8_F16>(p, smem, s);
+        default: return cudaErrorInvalidValue;
     }
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
 }
 
 }  // namespace spot

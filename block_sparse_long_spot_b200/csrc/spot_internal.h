@@ -43,15 +43,16 @@ constexpr int kTokBlocksPerPage = kBlock / kTokBlock;     // 4
 constexpr int kSelectFromScores = -1;  // launch_select "format": scores precomputed
 
 struct Layout {
-    size_t status, unit_done, partials, total;
-    size_t tok_scores;                  // token selector: block scores [B][max_blocks]
+    size_t status, unit_done, sel_done, partials, total;
+    size_t scores;                      // block scores [units][max_blocks] fp32 (the token
+                                        // selector uses [B][max_blocks] of it)
     int grid;                           // persistent CTAs of the decode kernel
 };
 
 // Workspace layout for a shape on the current device.
 bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Layout* out);
 
-// Parameters of the fused scoring + selection kernel.
+// Parameters of the block scoring kernel and of the selection kernel.
 struct SelectParams {
     const uint16_t* q_sel;
     const float* w;
@@ -66,7 +67,10 @@ struct SelectParams {
     int32_t mode, sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
     int32_t quantize_queries;           // quantise q_sel with the key format's rule
     int32_t blocks_per_page;            // selection blocks per page-table entry (1 or 4)
-    const float* scores_in;             // kSelectFromScores: block scores [units][max_blocks]
+    const float* scores_in;             // selection: block scores [units][max_blocks]
+    float* scores_out;                  // block scoring: the same array, written
+    uint32_t* sel_done;                 // [units] arrival counters of the scoring CTAs,
+                                        // zero between calls
     int32_t* sel_idx;
     int32_t* sel_cnt;
     uint32_t* status;

@@ -121,10 +121,12 @@ typedef struct {
 } spot_select_params_t;
 
 /* Bytes of scratch the select / sparse-decode / decode-step calls need for
- * this shape on the CURRENT device (it depends on the SM count).  The first
- * 256 bytes hold the device status word: zero them once before first use
- * (e.g. allocate the workspace zero-filled).  Returns 0 for a shape this
- * build does not support. */
+ * this shape on the CURRENT device (it depends on the SM count).  Zero the
+ * whole workspace once before its first use (e.g. allocate it zero-filled):
+ * its first 256 bytes hold the device status word, and it holds per-unit
+ * arrival counters of the scoring and decode kernels that must start at
+ * zero; every call leaves those counters at zero again.  Returns 0 for a
+ * shape this build does not support. */
 size_t spot_workspace_size(const spot_layer_desc_t* desc, int32_t batch, int32_t max_blocks);
 
 /* Append (write, quantising if the format asks) one selector key per
@@ -274,7 +276,7 @@ typedef struct {
 } spot_tok_layer_desc_t;
 
 /* Scratch bytes for the token selector's calls (same rules as
- * spot_workspace_size: zero the first 256 bytes once).  0 if unsupported. */
+ * spot_workspace_size: zero it once before first use).  0 if unsupported. */
 size_t spot_tok_workspace_size(const spot_tok_layer_desc_t* desc, int32_t batch,
                                int32_t max_blocks);
 

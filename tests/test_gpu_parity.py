@@ -239,6 +239,47 @@ def _assert_same_selection_or_near(gpu, ora, wl):
     assert diff <= 1
 
 
+def test_scoring_split_over_ctas_bit_exact_and_repeatable():
+    # Contexts of 300K - 512K tokens (up to 8192 blocks per (sequence, KV
+    # head)) over only 16 units: each unit's scoring is spread over several
+    # CTAs and the unit's last CTA to finish selects.  Integer selector inputs
+    # make every score exact, so every selection must equal the oracle's, and
+    # a second call on the same workspace must repeat it (the arrival
+    # counters are back at zero).
+    wl = workloads.make("ragged_hybrid", seed=13, device=DEV, integer=True, batch=2,
+                        sel_fmt="bf16", ragged_range=(300000, 524288))
+    data, scales = oracle_selector_pool(wl, "bf16")
+    a = dict(q_sel=workloads.bits(wl.q_sel), w=None, sel_data=data, sel_scales=scales,
+             page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy())
+    wl.top_p = safe_top_p(wl, "bf16", args=a)
+    scores = oracle_scores(wl, "bf16", args=a)
+    sp = wl.spec
+    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
+                            kmin_blocks=sp.kmin_blocks)
+    lens, top_p = a["seq_lens"], wl.top_p.cpu().numpy()
+    want = {}
+    for b in range(wl.batch):
+        nb = (int(lens[b]) + 63) // 64
+        for g in range(wl.num_kv_heads):
+            sel, _ = oracle.select_from_scores(scores[b, g, :nb], nb=nb, n_full=int(lens[b]) // 64,
+                                               params=pr, p=float(top_p[b]))
+            want[b, g] = sel.tolist()
+    desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, "bf16")
+    prm = spot.select_params("topp", sp.sink_blocks, sp.recency_blocks, sp.kmin_blocks)
+    ws = spot.new_workspace(desc, wl.batch, wl.max_blocks, DEV)
+    for call in range(2):
+        sel_idx = torch.full((wl.batch, wl.num_kv_heads, wl.max_blocks), -1, dtype=torch.int32,
+                             device=DEV)
+        sel_cnt = torch.full((wl.batch, wl.num_kv_heads), -1, dtype=torch.int32, device=DEV)
+        spot.select(desc, prm, wl.q_sel, None, wl.sel_keys, None, wl.page_table, wl.seq_lens,
+                    wl.top_p, sel_idx, sel_cnt, ws)
+        torch.cuda.synchronize()
+        assert spot.read_device_status(ws) == 0
+        got = {"sel_idx": sel_idx.cpu().numpy(), "sel_cnt": sel_cnt.cpu().numpy()}
+        for (b, g), sel in want.items():
+            assert unit_selection(got, b, g) == sel, (call, b, g)
+
+
 # ------------------------------------------------------------ edge cases
 
 def test_ragged_partial_blocks_and_empty_sequences():
