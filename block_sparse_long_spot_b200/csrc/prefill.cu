@@ -18,17 +18,19 @@
 //                         buffer; the epilogue forms each query's weighted
 //                         ReLU head sum and keeps the maximum over queries
 //   select_kernel         the decode selection on those scores (select.cu)
-//   prefill_attn_kernel   per (tile, KV head, 128 query-head rows): flash
-//                         attention over the selected blocks, K / V tiles by
-//                         TMA into a 4-stage ring, 8 mma.sync consumer warps
-//                         of 16 rows each, causal mask on the tile's own
-//                         block, online softmax in the log2 domain.
+//   prefill_attn_kernel   per (tile, KV head, 256 query-head rows): flash
+//                         attention over the selected blocks on the tcgen05
+//                         tensor cores (S and O accumulate in tensor memory),
+//                         K / V tiles by TMA into a 4-stage ring, causal mask
+//                         on the tile's own block, online softmax in the
+//                         log2 domain by two 128-row warpgroups.
 #include <math.h>
 
 #include <mutex>
 
 #include "spot_device.cuh"
 #include "spot_internal.h"
+#include "tc.cuh"
 
 namespace spot {
 namespace {
@@ -247,14 +249,41 @@ prefill_score_kernel(const PrefillParams p) {
 }
 
 // ------------------------------------------------------------------ attention
-
-constexpr int kAttnWarps = 8;                     // consumer warps, 16 rows each
-constexpr int kAttnThreads = (kAttnWarps + 1) * 32;
+//
+// One CTA per (tile, KV head, 256 (head, query) rows): two row groups of 128
+// rows share every K / V tile.  Warp roles:
+//   warps 0-3 / 4-7  softmax warpgroups of row groups 0 / 1 (thread = row;
+//                    warp w reads tensor-memory lanes 32 (w % 4) .. + 31)
+//   warp 8           TMA producer: K / V tiles of the selected blocks into a
+//                    4-stage ring (two 64 x 64 boxes each, 128-byte swizzle)
+//   warp 9           tcgen05 issuer (one thread) and tensor-memory owner
+// Per K / V tile i the issuer computes S_r = Q_r K^T (M = 128, N = 64,
+// K = 128) into tensor memory for both row groups and, once row group r's
+// softmax has written P_r (bf16, K-major with the 128-byte swizzle) to
+// shared memory, O_r += P_r V (M = 128, N = 128, K = 64, V read MN-major
+// straight from its TMA tile).  The two groups are staggered by half a tile
+// so one group's softmax overlaps the other's MMAs.  The softmax keeps each
+// row's reference maximum m and only moves it (rescaling O in tensor memory)
+// when a tile's maximum exceeds it by more than 8 in the log2 domain, so P
+// stays below 2^8 and O / l is unchanged.
 constexpr int kAttnStages = 4;
-constexpr int kAttnRows = kAttnWarps * 16;        // (query, head) rows per CTA
+constexpr int kAttnRows = 256;                    // (head, query) rows per CTA
+constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kAttnThreads = 10 * 32;
 constexpr int kHalfTile = kBlock * 64 * 2;        // 8 KiB: 64 rows x 64 bf16
+constexpr int kQHalf = 128 * 64 * 2;              // 16 KiB: 128 rows x 64 bf16
+constexpr int kPBytes = 128 * kBlock * 2;         // 16 KiB: 128 rows x 64 keys bf16
+constexpr uint32_t kTmemCols = 512;               // O_0, O_1 (128 each), S_0, S_1 (64 each)
+constexpr uint32_t kColO = 0, kColS = 256;
+constexpr int kAttnBars = 2 * kAttnStages + 8;
 
-__global__ void __launch_bounds__(kAttnThreads)
+size_t attn_smem_bytes() {
+    return 1024 + 4 * static_cast<size_t>(kQHalf) +
+           static_cast<size_t>(kAttnStages) * kStageBytes + 2 * kPBytes +
+           kAttnBars * sizeof(uint64_t) + 16;
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
 prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
                     const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -262,10 +291,19 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* base = smem_raw + pad;
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + kAttnStages * kStageBytes);
+    const uint32_t sbase = raw + pad;
+    // Q_r half h at (2 r + h) kQHalf; stages; P_r; barriers
+    constexpr uint32_t kOffKV = 4 * kQHalf;
+    constexpr uint32_t kOffP = kOffKV + kAttnStages * kStageBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + kOffP + 2 * kPBytes);
     uint64_t* empty = full + kAttnStages;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kAttnStages);
-    const uint32_t stage_base = smem_u32(base);
+    uint64_t* bar_q = empty + kAttnStages;        // queries staged (8 softmax warps)
+    uint64_t* bar_s = bar_q + 1;                  // [2] S_r computed
+    uint64_t* bar_p = bar_s + 2;                  // [2] P_r written (4 warps)
+    uint64_t* bar_o = bar_p + 2;                  // [2] O_r += P_r V completed
+    uint64_t* bar_fin = bar_o + 2;                // every issued MMA completed
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(full + kAttnBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     // heavy tiles (late in a sequence, many blocks) first
     const int lin = gridDim.x - 1 - blockIdx.x;
@@ -275,236 +313,292 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
     if (threadIdx.x == 0) {
         for (int s = 0; s < kAttnStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kAttnWarps);
+            mbar_init(&empty[s], 1);
         }
+        mbar_init(bar_q, 8);
+        for (int r = 0; r < 2; ++r) {
+            mbar_init(&bar_s[r], 1);
+            mbar_init(&bar_p[r], 4);
+            mbar_init(&bar_o[r], 1);
+        }
+        mbar_init(bar_fin, 1);
         fence_mbar_init();
         *abort_flag = 0;
     }
-    if (warp == kAttnWarps && lane == 0) {
+    if (warp == kWarpTma && lane == 0) {
         prefetch_tensormap(&k_map);
         prefetch_tensormap(&v_map);
     }
+    if (warp == kWarpMma) tmem_alloc(tmem_holder, kTmemCols);
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
     pdl_wait();                                   // the selection
     pdl_trigger();
     const int4 info = p.tile_info[t];
+    const bool live = info.x >= 0;
     const int b = info.x;
-    if (b < 0) return;
-    const int G = p.group;
-    const int L_eff = info.z + 1;
-    const int nb = min((L_eff + kBlock - 1) / kBlock, p.max_blocks);
-    int cnt = p.sel_cnt[unit];
-    if (cnt < 0 || cnt > nb) {
-        if (threadIdx.x == 0 && rg == 0) flag_status(p.status, kStatusBounds);
-        cnt = min(max(cnt, 0), nb);
+    int cnt = 0;
+    if (live) {
+        const int nb = min((info.z + 1 + kBlock - 1) / kBlock, p.max_blocks);
+        cnt = p.sel_cnt[unit];
+        if (cnt < 0 || cnt > nb) {
+            if (threadIdx.x == 0 && rg == 0) flag_status(p.status, kStatusBounds);
+            cnt = min(max(cnt, 0), nb);
+        }
     }
     const int32_t* sel = p.sel_idx + static_cast<int64_t>(unit) * p.max_blocks;
 
-    if (warp == kAttnWarps) {
-        // ================================================= producer warp
-        if (lane != 0) return;
-        const uint64_t policy = l2_policy_evict_first();
-        int issued = 0;
-        bool alive = true;
+    if (warp == kWarpTma) {
+        // ================================================= producer
+        if (lane == 0 && live) {
+            const uint64_t policy = l2_policy_evict_first();
+            int issued = 0;
+            bool alive = true;
+            for (int i = 0; i < cnt; ++i) {
+                const int s = i % kAttnStages, round = i / kAttnStages;
+                if (*abort_flag ||
+                    (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1))) {
+                    flag_status(p.status, kStatusTimeout);
+                    *abort_flag = 1;
+                    alive = false;
+                    break;
+                }
+                const int j = sel[i];
+                int page = -1;
+                if (j >= 0 && j < p.max_blocks && j < p.pt_stride)
+                    page = p.page_table[static_cast<int64_t>(b) * p.pt_stride + j];
+                if (page < 0 || page >= p.num_pages) {
+                    flag_status(p.status, kStatusBounds);
+                    page = 0;
+                }
+                const int r = (page * p.num_kv_heads + g) * kBlock;
+                mbar_arrive_expect_tx(&full[s], kStageBytes);
+                uint8_t* dst = base + kOffKV + s * kStageBytes;
+                tma_load_2d(dst, &k_map, &full[s], 0, r, policy);
+                tma_load_2d(dst + kHalfTile, &k_map, &full[s], 64, r, policy);
+                tma_load_2d(dst + 2 * kHalfTile, &v_map, &full[s], 0, r, policy);
+                tma_load_2d(dst + 3 * kHalfTile, &v_map, &full[s], 64, r, policy);
+                ++issued;
+            }
+            if (!alive) {
+                for (int k = max(0, issued - kAttnStages); k < issued; ++k)
+                    (void)mbar_wait_bounded(&full[k % kAttnStages], (k / kAttnStages) & 1);
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // ================================================= tcgen05 issuer
+        if (lane == 0 && live && cnt > 0) {
+            constexpr uint32_t idS = umma_idesc_bf16(128, kBlock, false);
+            constexpr uint32_t idO = umma_idesc_bf16(128, kHeadDim, true);
+            // S_r = Q_r K^T: A = Q_r (K-major), B = K tile (K-major), 8 steps of 16 dims
+            auto issue_s = [&](int r, int s) {
+                const uint32_t qa = sbase + 2 * r * kQHalf;
+                const uint32_t kb = sbase + kOffKV + s * kStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t o = (kk & 3) * 32;
+                    const uint64_t a = umma_desc_sw128(qa + (kk >> 2) * kQHalf + o, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(kb + (kk >> 2) * kHalfTile + o, 16, 1024);
+                    umma_bf16(tmem + kColS + 64 * r, a, bd, idS, kk > 0);
+                }
+            };
+            // O_r += P_r V: A = P_r (K-major), B = V tile (MN-major: dims contiguous,
+            // dims 64-127 one half tile on), 4 steps of 16 keys
+            auto issue_pv = [&](int r, int s, bool acc) {
+                const uint32_t pa = sbase + kOffP + r * kPBytes;
+                const uint32_t vb = sbase + kOffKV + s * kStageBytes + 2 * kHalfTile;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t a = umma_desc_sw128(pa + kk * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(vb + kk * 16 * 128, kHalfTile, 1024);
+                    umma_bf16(tmem + kColO + 128 * r, a, bd, idO, acc || kk > 0);
+                }
+            };
+            bool ok = mbar_wait_bounded(bar_q, 0);
+            tc_fence_after();
+            for (int i = 0; ok && i <= cnt; ++i) {
+                const int s = i % kAttnStages;
+                if (i < cnt) {
+                    ok = !*abort_flag && mbar_wait_bounded(&full[s], (i / kAttnStages) & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(0, s);
+                    umma_commit(&bar_s[0]);
+                }
+                if (i >= 1) {
+                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[1], (i - 1) & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int sp = (i - 1) % kAttnStages;
+                    issue_pv(1, sp, i - 1 > 0);
+                    umma_commit(&bar_o[1]);
+                    umma_commit(&empty[sp]);
+                }
+                if (i < cnt) {
+                    issue_s(1, s);
+                    umma_commit(&bar_s[1]);
+                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[0], i & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(0, s, i > 0);
+                    umma_commit(&bar_o[0]);
+                }
+            }
+            if (!ok) {
+                flag_status(p.status, kStatusTimeout);
+                *abort_flag = 1;
+            }
+            // every MMA issued completes before the tensor memory is released
+            umma_commit(bar_fin);
+            (void)mbar_wait_bounded(bar_fin, 0);
+        }
+    } else {
+        // ================================================= softmax warpgroups
+        const int r = warp >> 2;                  // row group
+        const int wq = warp & 3;                  // tensor-memory lane quarter
+        const int row = wq * 32 + lane;           // row within the group
+        const uint32_t lanes = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem + lanes + kColS + 64 * r;
+        const uint32_t tO = tmem + lanes + kColO + 128 * r;
+        const int G = p.group;
+        const int rho = rg * kAttnRows + r * 128 + row;
+        const int hh = rho / 64, qi = rho % 64;
+        const int nq = live ? info.z - info.y + 1 : 0;
+        const bool row_ok = hh < G && qi < nq;
+        const int pos = info.y + qi;
+        const int m_tile = live ? info.y / kBlock : 0;
+        const int64_t orow = row_ok ? (static_cast<int64_t>(info.w) + qi) * p.num_q_heads +
+                                          g * G + hh
+                                    : 0;
+        // ---- this row's query -> Q_r (K-major, 128-byte swizzle); zeros past the tile
+        {
+            const uint4* src = reinterpret_cast<const uint4*>(p.q + orow * kHeadDim);
+            uint4 v[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) v[c] = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<uint4*>(base + (2 * r + (c >> 3)) * kQHalf + row * 128 +
+                                          (((c & 7) ^ (row & 7)) << 4)) = v[c];
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_q);
+        }
+        uint8_t* prow = base + kOffP + r * kPBytes + row * 128;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
         for (int i = 0; i < cnt; ++i) {
-            const int s = i % kAttnStages, round = i / kAttnStages;
-            if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
-                flag_status(p.status, kStatusTimeout);
-                *abort_flag = 1;
-                alive = false;
-                break;
-            }
+            ok = !*abort_flag && mbar_wait_bounded(&bar_s[r], i & 1);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            float sa[32], sb[32];
+            tmem_ld32(tS, sa);
+            tmem_ld32(tS + 32, sb);
+            tmem_wait_ld();
             const int j = sel[i];
-            int page = -1;
-            if (j >= 0 && j < nb && j < p.pt_stride)
-                page = p.page_table[static_cast<int64_t>(b) * p.pt_stride + j];
-            if (page < 0 || page >= p.num_pages) {
-                flag_status(p.status, kStatusBounds);
-                page = 0;
+            const bool diag = j >= m_tile;        // the tile's own block: causal mask
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float x = sa[c] * p.scale_log2;
+                if (diag && j * kBlock + c > pos) x = -INFINITY;
+                sa[c] = x;
+                mx = fmaxf(mx, x);
+                float y = sb[c] * p.scale_log2;
+                if (diag && j * kBlock + 32 + c > pos) y = -INFINITY;
+                sb[c] = y;
+                mx = fmaxf(mx, y);
             }
-            const int r = (page * p.num_kv_heads + g) * kBlock;
-            mbar_arrive_expect_tx(&full[s], kStageBytes);
-            uint8_t* dst = base + s * kStageBytes;
-            tma_load_2d(dst, &k_map, &full[s], 0, r, policy);
-            tma_load_2d(dst + kHalfTile, &k_map, &full[s], 64, r, policy);
-            tma_load_2d(dst + 2 * kHalfTile, &v_map, &full[s], 0, r, policy);
-            tma_load_2d(dst + 3 * kHalfTile, &v_map, &full[s], 64, r, policy);
-            ++issued;
-        }
-        if (!alive) {
-            for (int k = max(0, issued - kAttnStages); k < issued; ++k)
-                (void)mbar_wait_bounded(&full[k % kAttnStages], (k / kAttnStages) & 1);
-        }
-        return;
-    }
-
-    // ===================================================== consumer warps
-    const int c4 = lane & 3, r8 = lane >> 2;
-    const int rho0 = rg * kAttnRows + warp * 16;  // first (head, query) row of this warp
-    const int hh = rho0 / 64;                     // head within the group (16 rows never straddle)
-    const int qb0 = rho0 % 64;                    // first query index within the tile
-    const int nq = info.z - info.y + 1;
-    const bool head_ok = hh < G;
-    const int m_tile = info.y / kBlock;           // the tile's own block (causal mask)
-    // query positions of this lane's two rows
-    const int qa = qb0 + r8, qc = qa + 8;
-    const int pos_a = info.y + qa, pos_c = info.y + qc;
-
-    // Q fragments (A operand, rows = queries, k = head dims)
-    uint32_t qf[8][4];
-    {
-        const int64_t ra = static_cast<int64_t>(info.w) + qa, rc = static_cast<int64_t>(info.w) + qc;
-        const bool va = head_ok && qa < nq, vc = head_ok && qc < nq;
-        const uint32_t* pa = reinterpret_cast<const uint32_t*>(
-            p.q + ((va ? ra : 0) * p.num_q_heads + g * G + (head_ok ? hh : 0)) * kHeadDim);
-        const uint32_t* pc = reinterpret_cast<const uint32_t*>(
-            p.q + ((vc ? rc : 0) * p.num_q_heads + g * G + (head_ok ? hh : 0)) * kHeadDim);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            qf[ks][0] = va ? __ldg(pa + 8 * ks + c4) : 0u;
-            qf[ks][1] = vc ? __ldg(pc + 8 * ks + c4) : 0u;
-            qf[ks][2] = va ? __ldg(pa + 8 * ks + 4 + c4) : 0u;
-            qf[ks][3] = vc ? __ldg(pc + 8 * ks + 4 + c4) : 0u;
-        }
-    }
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float oacc[16][4];
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
-
-    for (int i = 0; i < cnt; ++i) {
-        const int s = i % kAttnStages;
-        int ok = *abort_flag == 0;
-        if (ok) ok = mbar_wait_bounded(&full[s], (i / kAttnStages) & 1);
-        if (!__all_sync(0xffffffffu, ok)) {
-            if (lane == 0) {
-                flag_status(p.status, kStatusTimeout);
-                *abort_flag = 1;
+            // P_r and O_r are free once O_r += P_r V of the previous tile completed
+            if (i > 0) {
+                ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (i - 1) & 1);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
             }
-            break;
-        }
-        const int j = sel[i];
-        const uint32_t kb = stage_base + s * kStageBytes;
-        const uint32_t vb = kb + 2 * kHalfTile;
-        // ---- S = Q K^T: 16 rows x 64 keys (8 n-tiles)
-        float sc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t hb = kb + (ks >> 2) * kHalfTile;
-            const int chunk = ((ks & 3) << 1) + ((lane >> 3) & 1);
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(swz128(hb, key, chunk), b0, b1, b2, b3);
-                mma_bf16_16816(sc[2 * np], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
-                mma_bf16_16816(sc[2 * np + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b2, b3);
+            const float m_new = fmaxf(m_ref, mx);
+            const bool grow = m_new > m_ref + 8.f;
+            float alpha = 1.f;
+            if (grow) {
+                alpha = exp2f(m_ref - m_new);     // 0 while m_ref = -inf
+                l *= alpha;
+                m_ref = m_new;
             }
-        }
-        // ---- causal mask on the tile's own block (key position <= query position)
-        if (j >= m_tile) {
+            if (i > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
+                    float o[32];
+                    tmem_ld32(tO + c0, o);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int kp = j * kBlock + nt * 8 + 2 * c4;
-                if (kp > pos_a) sc[nt][0] = -INFINITY;
-                if (kp + 1 > pos_a) sc[nt][1] = -INFINITY;
-                if (kp > pos_c) sc[nt][2] = -INFINITY;
-                if (kp + 1 > pos_c) sc[nt][3] = -INFINITY;
+                    for (int c = 0; c < 32; ++c) o[c] *= alpha;
+                    tmem_st32(tO + c0, o);
+                }
+                tmem_wait_st();
             }
-        }
-        // ---- online softmax (rows r8 and r8 + 8)
-        float x0 = -INFINITY, x1 = -INFINITY;
+            const float ref = m_ref == -INFINITY ? 0.f : m_ref;
+            float sum = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            x0 = fmaxf(x0, fmaxf(sc[nt][0], sc[nt][1]));
-            x1 = fmaxf(x1, fmaxf(sc[nt][2], sc[nt][3]));
-        }
-        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
-        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
-        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 1));
-        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2));
-        const float n0 = fmaxf(m0, x0 * p.scale_log2), n1 = fmaxf(m1, x1 * p.scale_log2);
-        const float ref0 = (n0 == -INFINITY) ? 0.f : n0, ref1 = (n1 == -INFINITY) ? 0.f : n1;
-        const float al0 = exp2f(m0 - ref0), al1 = exp2f(m1 - ref1);
-        m0 = n0;
-        m1 = n1;
-        float s0 = 0.f, s1 = 0.f;
-        uint32_t pa[8][2];
+            for (int ch = 0; ch < 8; ++ch) {
+                float e[8];
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const float p0 = exp2f(fmaf(sc[nt][0], p.scale_log2, -ref0));
-            const float p1 = exp2f(fmaf(sc[nt][1], p.scale_log2, -ref0));
-            const float p2 = exp2f(fmaf(sc[nt][2], p.scale_log2, -ref1));
-            const float p3 = exp2f(fmaf(sc[nt][3], p.scale_log2, -ref1));
-            s0 += p0 + p1;
-            s1 += p2 + p3;
-            pa[nt][0] = pack_bf16(p0, p1);
-            pa[nt][1] = pack_bf16(p2, p3);
-        }
-        l0 = l0 * al0 + s0;
-        l1 = l1 * al1 + s1;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            oacc[nt][0] *= al0;
-            oacc[nt][1] *= al0;
-            oacc[nt][2] *= al1;
-            oacc[nt][3] *= al1;
-        }
-        // ---- O += P V: 4 k-steps of 16 keys x 16 n-tiles of 8 dims
-#pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            const uint32_t a0 = pa[2 * kt][0], a1 = pa[2 * kt][1];
-            const uint32_t a2 = pa[2 * kt + 1][0], a3 = pa[2 * kt + 1][1];
-            const int key = kt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                const uint32_t hb = vb + (np >> 2) * kHalfTile;
-                const int chunk = ((np & 3) << 1) + (lane >> 4);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_trans(swz128(hb, key, chunk), b0, b1, b2, b3);
-                mma_bf16_16816(oacc[2 * np], a0, a1, a2, a3, b0, b1);
-                mma_bf16_16816(oacc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+                for (int k = 0; k < 8; ++k) {
+                    const int c = ch * 8 + k;
+                    e[k] = exp2f((c < 32 ? sa[c & 31] : sb[c & 31]) - ref);
+                    sum += e[k];
+                }
+                *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
+                    make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]),
+                               pack_bf16(e[4], e[5]), pack_bf16(e[6], e[7]));
             }
+            l += sum;
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_p[r]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-    }
-
-    // ---- epilogue: out = O / l, lse (natural log)
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if (!head_ok) return;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int q = half ? qc : qa;
-        if (q >= nq) continue;
-        const float l = half ? l1 : l0, m = half ? m1 : m0;
+        if (ok && cnt > 0) {
+            ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (cnt - 1) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+        }
+        if (!ok && lane == 0) {
+            flag_status(p.status, kStatusTimeout);
+            *abort_flag = 1;
+        }
+        // ---- epilogue: out = O / l, lse (natural log)
+        const bool write = row_ok && ok;
         const bool empty_row = !(l > 0.f);
         const float inv = empty_row ? 0.f : 1.f / l;
-        const int64_t h = (static_cast<int64_t>(info.w) + q) * p.num_q_heads + g * G + hh;
-        float* o = p.out + h * kHeadDim;
+        float* o_out = p.out + orow * kHeadDim;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
+            float o[32];
+            if (ok && cnt > 0) {
+                tmem_ld32(tO + c0, o);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int d = nt * 8 + 2 * c4;
-            *reinterpret_cast<float2*>(o + d) =
-                make_float2(oacc[nt][2 * half] * inv, oacc[nt][2 * half + 1] * inv);
+                for (int c = 0; c < 32; ++c) o[c] = 0.f;
+            }
+            if (write) {
+#pragma unroll
+                for (int c = 0; c < 32; c += 4)
+                    *reinterpret_cast<float4*>(o_out + c0 + c) =
+                        make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+            }
         }
-        if (p.lse && c4 == 0)
-            p.lse[h] = empty_row ? -INFINITY : (m + log2f(l)) * 0.6931471805599453f;
+        if (write && p.lse)
+            p.lse[orow] = empty_row ? -INFINITY : (m_ref + log2f(l)) * 0.6931471805599453f;
     }
-}
-
-size_t attn_smem_bytes() {
-    return 1024 + static_cast<size_t>(kAttnStages) * kStageBytes +
-           2 * kAttnStages * sizeof(uint64_t) + 16;
+    // ---- the tensor memory goes back once every warp is done with it
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
 }
 
 std::mutex g_prefill_mutex;
