@@ -305,11 +305,14 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(full + kAttnBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
-    // heavy tiles (late in a sequence, many blocks) first
-    const int lin = gridDim.x - 1 - blockIdx.x;
+    // KV head slowest, so the CTAs running together share one head's K / V
+    // in L2; within a head, heavy tiles (late in a sequence, many blocks) first
     const int groups = p.row_groups;
-    const int unit = lin / groups, rg = lin - unit * groups;
-    const int t = unit / p.num_kv_heads, g = unit - t * p.num_kv_heads;
+    const int per_head = p.max_tiles * groups;
+    const int g = blockIdx.x / per_head;
+    const int lin = per_head - 1 - (blockIdx.x - g * per_head);
+    const int t = lin / groups, rg = lin - t * groups;
+    const int unit = t * p.num_kv_heads + g;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kAttnStages; ++s) {
             mbar_init(&full[s], 1);
@@ -353,7 +356,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
     if (warp == kWarpTma) {
         // ================================================= producer
         if (lane == 0 && live) {
-            const uint64_t policy = l2_policy_evict_first();
+            const uint64_t policy = l2_policy_evict_last();     // re-read by later tiles
             int issued = 0;
             bool alive = true;
             for (int i = 0; i < cnt; ++i) {
@@ -487,30 +490,33 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
             if (lane == 0) mbar_arrive(bar_q);
         }
         uint8_t* prow = base + kOffP + r * kPBytes + row * 128;
+        const float sl2 = p.scale_log2;           // > 0: the maximum commutes with it
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
+        int j_next = cnt > 0 ? sel[0] : 0;
         for (int i = 0; i < cnt; ++i) {
+            const int j = j_next;
+            if (i + 1 < cnt) j_next = sel[i + 1];
             ok = !*abort_flag && mbar_wait_bounded(&bar_s[r], i & 1);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            float sa[32], sb[32];
-            tmem_ld32(tS, sa);
-            tmem_ld32(tS + 32, sb);
+            float sv[64];
+            tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(sv));
+            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
             tmem_wait_ld();
-            const int j = sel[i];
-            const bool diag = j >= m_tile;        // the tile's own block: causal mask
-            float mx = -INFINITY;
+            if (j >= m_tile) {                    // the tile's own block: causal mask
+                const int lim = pos - j * kBlock; // keys c > lim lie after this query
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                float x = sa[c] * p.scale_log2;
-                if (diag && j * kBlock + c > pos) x = -INFINITY;
-                sa[c] = x;
-                mx = fmaxf(mx, x);
-                float y = sb[c] * p.scale_log2;
-                if (diag && j * kBlock + 32 + c > pos) y = -INFINITY;
-                sb[c] = y;
-                mx = fmaxf(mx, y);
+                for (int c = 0; c < 64; ++c)
+                    if (c > lim) sv[c] = -INFINITY;
             }
+            float pm[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) pm[k] = sv[k];
+#pragma unroll
+            for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], sv[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sl2;
             // P_r and O_r are free once O_r += P_r V of the previous tile completed
             if (i > 0) {
                 ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (i - 1) & 1);
@@ -537,22 +543,19 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
                 }
                 tmem_wait_st();
             }
-            const float ref = m_ref == -INFINITY ? 0.f : m_ref;
-            float sum = 0.f;
+            const float nref = m_ref == -INFINITY ? 0.f : -m_ref;
+            float ps[8];
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
                 float e[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int c = ch * 8 + k;
-                    e[k] = exp2f((c < 32 ? sa[c & 31] : sb[c & 31]) - ref);
-                    sum += e[k];
-                }
+                for (int k = 0; k < 8; ++k) e[k] = fast_exp2(fmaf(sv[ch * 8 + k], sl2, nref));
+                ps[ch] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
                 *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
                     make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]),
                                pack_bf16(e[4], e[5]), pack_bf16(e[6], e[7]));
             }
-            l += sum;
+            l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
