@@ -255,35 +255,37 @@ prefill_score_kernel(const PrefillParams p) {
 //   warps 0-3 / 4-7  softmax warpgroups of row groups 0 / 1 (thread = row;
 //                    warp w reads tensor-memory lanes 32 (w % 4) .. + 31)
 //   warp 8           TMA producer: K / V tiles of the selected blocks into a
-//                    4-stage ring (two 64 x 64 boxes each, 128-byte swizzle)
+//                    5-stage ring (two 64 x 64 boxes each, 128-byte swizzle)
 //   warp 9           tcgen05 issuer (one thread) and tensor-memory owner
-// Per K / V tile i the issuer computes S_r = Q_r K^T (M = 128, N = 64,
-// K = 128) into tensor memory for both row groups and, once row group r's
-// softmax has written P_r (bf16, K-major with the 128-byte swizzle) to
-// shared memory, O_r += P_r V (M = 128, N = 128, K = 64, V read MN-major
-// straight from its TMA tile).  The two groups are staggered by half a tile
-// so one group's softmax overlaps the other's MMAs.  The softmax keeps each
-// row's reference maximum m and only moves it (rescaling O in tensor memory)
-// when a tile's maximum exceeds it by more than 8 in the log2 domain, so P
-// stays below 2^8 and O / l is unchanged.
-constexpr int kAttnStages = 4;
+// A step takes two selected blocks (128 keys; the last step of an odd count
+// one).  Per step the issuer computes S_r = Q_r K^T (M = 128, K = 128, one
+// N = 64 MMA group per block) into tensor memory for both row groups; row
+// group r's softmax turns S_r into P_r (bf16), written over S_r's first 64
+// columns, and the issuer then runs O_r += P_r V with P_r read from tensor
+// memory (M = 128, N = 128, K = 16 per MMA, V read MN-major straight from
+// its TMA tiles).  The row groups are staggered by half a step so one
+// group's softmax overlaps the other's MMAs.  The softmax keeps each row's
+// reference maximum m and only moves it (rescaling O in tensor memory) when
+// a step's maximum exceeds it by more than 8 in the log2 domain, so P stays
+// below 2^8 and O / l is unchanged.
+constexpr int kAttnStages = 5;
 constexpr int kAttnRows = 256;                    // (head, query) rows per CTA
 constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr int kAttnThreads = 10 * 32;
 constexpr int kHalfTile = kBlock * 64 * 2;        // 8 KiB: 64 rows x 64 bf16
 constexpr int kQHalf = 128 * 64 * 2;              // 16 KiB: 128 rows x 64 bf16
-constexpr int kPBytes = 128 * kBlock * 2;         // 16 KiB: 128 rows x 64 keys bf16
-constexpr uint32_t kTmemCols = 512;               // O_0, O_1 (128 each), S_0, S_1 (64 each)
-constexpr uint32_t kColO = 0, kColS = 256;
+constexpr uint32_t kTmemCols = 512;               // O_0, O_1, S_0, S_1: 128 columns each
+constexpr uint32_t kColO = 0, kColS = 256;        // O_r at 128 r, S_r / P_r at 256 + 128 r
 constexpr int kAttnBars = 2 * kAttnStages + 8;
 
 size_t attn_smem_bytes() {
     return 1024 + 4 * static_cast<size_t>(kQHalf) +
-           static_cast<size_t>(kAttnStages) * kStageBytes + 2 * kPBytes +
-           kAttnBars * sizeof(uint64_t) + 16;
+           static_cast<size_t>(kAttnStages) * kStageBytes + kAttnBars * sizeof(uint64_t) + 16;
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1)
+// 10 warps: two of the four SM sub-partitions hold three of them, so a
+// thread may use at most 16384 / 96 registers
+__global__ void __maxnreg__(168)
 prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
                     const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -292,10 +294,9 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* base = smem_raw + pad;
     const uint32_t sbase = raw + pad;
-    // Q_r half h at (2 r + h) kQHalf; stages; P_r; barriers
+    // Q_r half h at (2 r + h) kQHalf; stages; barriers
     constexpr uint32_t kOffKV = 4 * kQHalf;
-    constexpr uint32_t kOffP = kOffKV + kAttnStages * kStageBytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + kOffP + 2 * kPBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + kOffKV + kAttnStages * kStageBytes);
     uint64_t* empty = full + kAttnStages;
     uint64_t* bar_q = empty + kAttnStages;        // queries staged (8 softmax warps)
     uint64_t* bar_s = bar_q + 1;                  // [2] S_r computed
@@ -351,6 +352,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
             cnt = min(max(cnt, 0), nb);
         }
     }
+    const int steps = (cnt + 1) / 2;
     const int32_t* sel = p.sel_idx + static_cast<int64_t>(unit) * p.max_blocks;
 
     if (warp == kWarpTma) {
@@ -395,57 +397,69 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
         if (lane == 0 && live && cnt > 0) {
             constexpr uint32_t idS = umma_idesc_bf16(128, kBlock, false);
             constexpr uint32_t idO = umma_idesc_bf16(128, kHeadDim, true);
-            // S_r = Q_r K^T: A = Q_r (K-major), B = K tile (K-major), 8 steps of 16 dims
-            auto issue_s = [&](int r, int s) {
+            // block i's S columns for row group r: A = Q_r (K-major), B = the
+            // block's K tile (K-major), 8 steps of 16 dims
+            auto issue_s = [&](int r, int i) {
                 const uint32_t qa = sbase + 2 * r * kQHalf;
-                const uint32_t kb = sbase + kOffKV + s * kStageBytes;
+                const uint32_t kb = sbase + kOffKV + (i % kAttnStages) * kStageBytes;
+                const uint32_t d = tmem + kColS + 128 * r + 64 * (i & 1);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t o = (kk & 3) * 32;
                     const uint64_t a = umma_desc_sw128(qa + (kk >> 2) * kQHalf + o, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(kb + (kk >> 2) * kHalfTile + o, 16, 1024);
-                    umma_bf16(tmem + kColS + 64 * r, a, bd, idS, kk > 0);
+                    umma_bf16(d, a, bd, idS, kk > 0);
                 }
             };
-            // O_r += P_r V: A = P_r (K-major), B = V tile (MN-major: dims contiguous,
-            // dims 64-127 one half tile on), 4 steps of 16 keys
-            auto issue_pv = [&](int r, int s, bool acc) {
-                const uint32_t pa = sbase + kOffP + r * kPBytes;
-                const uint32_t vb = sbase + kOffKV + s * kStageBytes + 2 * kHalfTile;
+            // O_r += P_r V over the step's blocks: A = P_r in tensor memory (16 keys
+            // = 8 columns per MMA), B = V tile (MN-major: dims contiguous, dims
+            // 64-127 one half tile on), 4 MMAs of 16 keys per block
+            auto issue_pv = [&](int r, int k, bool acc) {
+                const uint32_t pa = tmem + kColS + 128 * r;
+                const int nblk = min(2, cnt - 2 * k);
+                for (int h = 0; h < nblk; ++h) {
+                    const int i = 2 * k + h;
+                    const uint32_t vb = sbase + kOffKV + (i % kAttnStages) * kStageBytes +
+                                        2 * kHalfTile;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a = umma_desc_sw128(pa + kk * 32, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(vb + kk * 16 * 128, kHalfTile, 1024);
-                    umma_bf16(tmem + kColO + 128 * r, a, bd, idO, acc || kk > 0);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bd = umma_desc_sw128(vb + kk * 16 * 128, kHalfTile, 1024);
+                        umma_bf16_ts(tmem + kColO + 128 * r, pa + 32 * h + 8 * kk, bd, idO,
+                                     acc || h > 0 || kk > 0);
+                    }
                 }
+            };
+            auto wait_full = [&](int i) {
+                return !*abort_flag &&
+                       mbar_wait_bounded(&full[i % kAttnStages], (i / kAttnStages) & 1);
             };
             bool ok = mbar_wait_bounded(bar_q, 0);
             tc_fence_after();
-            for (int i = 0; ok && i <= cnt; ++i) {
-                const int s = i % kAttnStages;
-                if (i < cnt) {
-                    ok = !*abort_flag && mbar_wait_bounded(&full[s], (i / kAttnStages) & 1);
+            for (int k = 0; ok && k <= steps; ++k) {
+                const int i0 = 2 * k, nblk = k < steps ? min(2, cnt - i0) : 0;
+                if (k < steps) {
+                    for (int h = 0; ok && h < nblk; ++h) ok = wait_full(i0 + h);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_s(0, s);
+                    for (int h = 0; h < nblk; ++h) issue_s(0, i0 + h);
                     umma_commit(&bar_s[0]);
                 }
-                if (i >= 1) {
-                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[1], (i - 1) & 1);
+                if (k >= 1) {
+                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[1], (k - 1) & 1);
                     if (!ok) break;
                     tc_fence_after();
-                    const int sp = (i - 1) % kAttnStages;
-                    issue_pv(1, sp, i - 1 > 0);
+                    issue_pv(1, k - 1, k - 1 > 0);
                     umma_commit(&bar_o[1]);
-                    umma_commit(&empty[sp]);
+                    for (int i = 2 * (k - 1); i < min(cnt, 2 * k); ++i)
+                        umma_commit(&empty[i % kAttnStages]);
                 }
-                if (i < cnt) {
-                    issue_s(1, s);
+                if (k < steps) {
+                    for (int h = 0; h < nblk; ++h) issue_s(1, i0 + h);
                     umma_commit(&bar_s[1]);
-                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[0], i & 1);
+                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[0], k & 1);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(0, s, i > 0);
+                    issue_pv(0, k, k > 0);
                     umma_commit(&bar_o[0]);
                 }
             }
@@ -463,7 +477,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
         const int wq = warp & 3;                  // tensor-memory lane quarter
         const int row = wq * 32 + lane;           // row within the group
         const uint32_t lanes = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t tS = tmem + lanes + kColS + 64 * r;
+        const uint32_t tS = tmem + lanes + kColS + 128 * r;
         const uint32_t tO = tmem + lanes + kColO + 128 * r;
         const int G = p.group;
         const int rho = rg * kAttnRows + r * 128 + row;
@@ -489,37 +503,50 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_q);
         }
-        uint8_t* prow = base + kOffP + r * kPBytes + row * 128;
         const float sl2 = p.scale_log2;           // > 0: the maximum commutes with it
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        int j_next = cnt > 0 ? sel[0] : 0;
-        for (int i = 0; i < cnt; ++i) {
-            const int j = j_next;
-            if (i + 1 < cnt) j_next = sel[i + 1];
-            ok = !*abort_flag && mbar_wait_bounded(&bar_s[r], i & 1);
+        for (int k = 0; k < steps; ++k) {
+            const int ja = sel[2 * k];
+            const bool two = 2 * k + 1 < cnt;
+            const int jb = two ? sel[2 * k + 1] : 0;
+            ok = !*abort_flag && mbar_wait_bounded(&bar_s[r], k & 1);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            float sv[64];
-            tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(sv));
-            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+            float sv[128];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float t32[32];
+                tmem_ld32(tS + 32 * q, t32);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sv[32 * q + c] = t32[c];
+            }
             tmem_wait_ld();
-            if (j >= m_tile) {                    // the tile's own block: causal mask
-                const int lim = pos - j * kBlock; // keys c > lim lie after this query
+            if (ja >= m_tile) {                   // the tile's own block: causal mask
+                const int lim = pos - ja * kBlock;
 #pragma unroll
                 for (int c = 0; c < 64; ++c)
                     if (c > lim) sv[c] = -INFINITY;
             }
-            float pm[8];
+            if (!two || jb >= m_tile) {           // no second block, or the diagonal
+                const int lim = two ? pos - jb * kBlock : -1;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) pm[k] = sv[k];
+                for (int c = 0; c < 64; ++c)
+                    if (c > lim) sv[64 + c] = -INFINITY;
+            }
+            float pm[16];
 #pragma unroll
-            for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], sv[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sl2;
-            // P_r and O_r are free once O_r += P_r V of the previous tile completed
-            if (i > 0) {
-                ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (i - 1) & 1);
+            for (int c = 0; c < 16; ++c) pm[c] = sv[c];
+#pragma unroll
+            for (int c = 16; c < 128; ++c) pm[c & 15] = fmaxf(pm[c & 15], sv[c]);
+#pragma unroll
+            for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; ++c) pm[c] = fmaxf(pm[c], pm[c + w]);
+            const float mx = pm[0] * sl2;
+            // O_r and the P_r columns are free once the previous O_r += P_r V completed
+            if (k > 0) {
+                ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (k - 1) & 1);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
             }
@@ -531,38 +558,39 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
                 l *= alpha;
                 m_ref = m_new;
             }
-            if (i > 0 && __any_sync(0xffffffffu, grow)) {
+            if (k > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
-                    float o[32];
-                    tmem_ld32(tO + c0, o);
+                for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
+                    float o[16];
+                    tmem_ld16(tO + c0, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] *= alpha;
-                    tmem_st32(tO + c0, o);
+                    for (int c = 0; c < 16; ++c) o[c] *= alpha;
+                    tmem_st16(tO + c0, o);
                 }
-                tmem_wait_st();
             }
             const float nref = m_ref == -INFINITY ? 0.f : -m_ref;
-            float ps[8];
+            float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                float e[8];
+            for (int q = 0; q < 2; ++q) {
+                uint32_t pk[32];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = fast_exp2(fmaf(sv[ch * 8 + k], sl2, nref));
-                ps[ch] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-                *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
-                    make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]),
-                               pack_bf16(e[4], e[5]), pack_bf16(e[6], e[7]));
+                for (int c = 0; c < 32; ++c) {
+                    const float e0 = fast_exp2(fmaf(sv[64 * q + 2 * c], sl2, nref));
+                    const float e1 = fast_exp2(fmaf(sv[64 * q + 2 * c + 1], sl2, nref));
+                    ps[4 * q + (c & 3)] += e0 + e1;
+                    pk[c] = pack_bf16(e0, e1);
+                }
+                tmem_st32u(tS + 32 * q, pk);
             }
             l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-            fence_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_p[r]);
         }
-        if (ok && cnt > 0) {
-            ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (cnt - 1) & 1);
+        if (ok && steps > 0) {
+            ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (steps - 1) & 1);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
         }
@@ -578,7 +606,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
 #pragma unroll 1
         for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
             float o[32];
-            if (ok && cnt > 0) {
+            if (ok && steps > 0) {
                 tmem_ld32(tO + c0, o);
                 tmem_wait_ld();
             } else {
