@@ -397,18 +397,23 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
         if (lane == 0 && live && cnt > 0) {
             constexpr uint32_t idS = umma_idesc_bf16(128, kBlock, false);
             constexpr uint32_t idO = umma_idesc_bf16(128, kHeadDim, true);
+            // Descriptors are built once per operand base; a step inside the
+            // operand adds (bytes >> 4) to the start-address field (no carry:
+            // shared addresses stay below 256 KiB).
+            const uint64_t dq[2] = {umma_desc_sw128(sbase, 16, 1024),
+                                    umma_desc_sw128(sbase + 2 * kQHalf, 16, 1024)};
+            const uint64_t dk0 = umma_desc_sw128(sbase + kOffKV, 16, 1024);
+            const uint64_t dv0 = umma_desc_sw128(sbase + kOffKV + 2 * kHalfTile, kHalfTile, 1024);
             // block i's S columns for row group r: A = Q_r (K-major), B = the
             // block's K tile (K-major), 8 steps of 16 dims
             auto issue_s = [&](int r, int i) {
-                const uint32_t qa = sbase + 2 * r * kQHalf;
-                const uint32_t kb = sbase + kOffKV + (i % kAttnStages) * kStageBytes;
+                const uint64_t bk = dk0 + (((i % kAttnStages) * kStageBytes) >> 4);
                 const uint32_t d = tmem + kColS + 128 * r + 64 * (i & 1);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t o = (kk & 3) * 32;
-                    const uint64_t a = umma_desc_sw128(qa + (kk >> 2) * kQHalf + o, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(kb + (kk >> 2) * kHalfTile + o, 16, 1024);
-                    umma_bf16(d, a, bd, idS, kk > 0);
+                    const uint32_t o = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+                    const uint32_t ob = ((kk >> 2) * kHalfTile + (kk & 3) * 32) >> 4;
+                    umma_bf16(d, dq[r] + o, bk + ob, idS, kk > 0);
                 }
             };
             // O_r += P_r V over the step's blocks: A = P_r in tensor memory (16 keys
@@ -416,17 +421,14 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
             // 64-127 one half tile on), 4 MMAs of 16 keys per block
             auto issue_pv = [&](int r, int k, bool acc) {
                 const uint32_t pa = tmem + kColS + 128 * r;
+                const uint32_t dO = tmem + kColO + 128 * r;
                 const int nblk = min(2, cnt - 2 * k);
                 for (int h = 0; h < nblk; ++h) {
-                    const int i = 2 * k + h;
-                    const uint32_t vb = sbase + kOffKV + (i % kAttnStages) * kStageBytes +
-                                        2 * kHalfTile;
+                    const uint64_t bv = dv0 + ((((2 * k + h) % kAttnStages) * kStageBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd = umma_desc_sw128(vb + kk * 16 * 128, kHalfTile, 1024);
-                        umma_bf16_ts(tmem + kColO + 128 * r, pa + 32 * h + 8 * kk, bd, idO,
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16_ts(dO, pa + 32 * h + 8 * kk, bv + ((kk * 16 * 128) >> 4), idO,
                                      acc || h > 0 || kk > 0);
-                    }
                 }
             };
             auto wait_full = [&](int i) {
