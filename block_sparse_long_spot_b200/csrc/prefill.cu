@@ -255,11 +255,15 @@ prefill_score_kernel(const PrefillParams p) {
 //   warps 0-3 / 4-7  softmax warpgroups of row groups 0 / 1 (thread = row;
 //                    warp w reads tensor-memory lanes 32 (w % 4) .. + 31)
 //   warp 8           TMA producer: K / V tiles of the selected blocks into a
-//                    5-stage ring (two 64 x 64 boxes each, 128-byte swizzle)
+//                    4-stage ring (two 64 x 64 boxes each, 128-byte swizzle);
+//                    the stages are laid out by quarter (K dims 0-63 of every
+//                    stage, then K dims 64-127, V dims 0-63, V dims 64-127),
+//                    so the two blocks of a step (stages 2 p, 2 p + 1) form one
+//                    128-row operand
 //   warp 9           tcgen05 issuer (one thread) and tensor-memory owner
 // A step takes two selected blocks (128 keys; the last step of an odd count
-// one).  Per step the issuer computes S_r = Q_r K^T (M = 128, K = 128, one
-// N = 64 MMA group per block) into tensor memory for both row groups; row
+// one).  Per step the issuer computes S_r = Q_r K^T (M = 128, N = 128,
+// K = 16 per MMA) into tensor memory for both row groups; row
 // group r's softmax turns S_r into P_r (bf16), written over S_r's first 64
 // columns, and the issuer then runs O_r += P_r V with P_r read from tensor
 // memory (M = 128, N = 128, K = 16 per MMA, V read MN-major straight from
@@ -268,7 +272,7 @@ prefill_score_kernel(const PrefillParams p) {
 // reference maximum m and only moves it (rescaling O in tensor memory) when
 // a step's maximum exceeds it by more than 8 in the log2 domain, so P stays
 // below 2^8 and O / l is unchanged.
-constexpr int kAttnStages = 5;
+constexpr int kAttnStages = 4;                    // two steps of two blocks
 constexpr int kAttnRows = 256;                    // (head, query) rows per CTA
 constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr int kAttnThreads = 10 * 32;
@@ -277,6 +281,7 @@ constexpr int kQHalf = 128 * 64 * 2;              // 16 KiB: 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;               // O_0, O_1, S_0, S_1: 128 columns each
 constexpr uint32_t kColO = 0, kColS = 256;        // O_r at 128 r, S_r / P_r at 256 + 128 r
 constexpr int kAttnBars = 2 * kAttnStages + 8;
+constexpr int kRegion = kAttnStages * kHalfTile;  // one quarter (K / V, dims half) of every stage
 
 size_t attn_smem_bytes() {
     return 1024 + 4 * static_cast<size_t>(kQHalf) +
@@ -380,11 +385,11 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
                 }
                 const int r = (page * p.num_kv_heads + g) * kBlock;
                 mbar_arrive_expect_tx(&full[s], kStageBytes);
-                uint8_t* dst = base + kOffKV + s * kStageBytes;
+                uint8_t* dst = base + kOffKV + s * kHalfTile;
                 tma_load_2d(dst, &k_map, &full[s], 0, r, policy);
-                tma_load_2d(dst + kHalfTile, &k_map, &full[s], 64, r, policy);
-                tma_load_2d(dst + 2 * kHalfTile, &v_map, &full[s], 0, r, policy);
-                tma_load_2d(dst + 3 * kHalfTile, &v_map, &full[s], 64, r, policy);
+                tma_load_2d(dst + kRegion, &k_map, &full[s], 64, r, policy);
+                tma_load_2d(dst + 2 * kRegion, &v_map, &full[s], 0, r, policy);
+                tma_load_2d(dst + 3 * kRegion, &v_map, &full[s], 64, r, policy);
                 ++issued;
             }
             if (!alive) {
@@ -395,70 +400,71 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
     } else if (warp == kWarpMma) {
         // ================================================= tcgen05 issuer
         if (lane == 0 && live && cnt > 0) {
-            constexpr uint32_t idS = umma_idesc_bf16(128, kBlock, false);
             constexpr uint32_t idO = umma_idesc_bf16(128, kHeadDim, true);
             // Descriptors are built once per operand base; a step inside the
             // operand adds (bytes >> 4) to the start-address field (no carry:
             // shared addresses stay below 256 KiB).
+            constexpr uint32_t idS2 = umma_idesc_bf16(128, 2 * kBlock, false);
             const uint64_t dq[2] = {umma_desc_sw128(sbase, 16, 1024),
                                     umma_desc_sw128(sbase + 2 * kQHalf, 16, 1024)};
-            const uint64_t dk0 = umma_desc_sw128(sbase + kOffKV, 16, 1024);
-            const uint64_t dv0 = umma_desc_sw128(sbase + kOffKV + 2 * kHalfTile, kHalfTile, 1024);
-            // block i's S columns for row group r: A = Q_r (K-major), B = the
-            // block's K tile (K-major), 8 steps of 16 dims
-            auto issue_s = [&](int r, int i) {
-                const uint64_t bk = dk0 + (((i % kAttnStages) * kStageBytes) >> 4);
-                const uint32_t d = tmem + kColS + 128 * r + 64 * (i & 1);
+            const uint64_t dk = umma_desc_sw128(sbase + kOffKV, 16, 1024);
+            const uint64_t dv = umma_desc_sw128(sbase + kOffKV + 2 * kRegion, kRegion, 1024);
+            // S_r of step k: A = Q_r (K-major), B = the step's 128 K rows (K-major,
+            // blocks 2 k and 2 k + 1 in stages 2 p, 2 p + 1), 8 steps of 16 dims
+            auto issue_s = [&](int r, int k) {
+                const uint64_t bk = dk + (((k & 1) * 2 * kHalfTile) >> 4);
+                const uint32_t d = tmem + kColS + 128 * r;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t o = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-                    const uint32_t ob = ((kk >> 2) * kHalfTile + (kk & 3) * 32) >> 4;
-                    umma_bf16(d, dq[r] + o, bk + ob, idS, kk > 0);
+                    const uint32_t oa = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+                    const uint32_t ob = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
+                    umma_bf16(d, dq[r] + oa, bk + ob, idS2, kk > 0);
                 }
             };
-            // O_r += P_r V over the step's blocks: A = P_r in tensor memory (16 keys
-            // = 8 columns per MMA), B = V tile (MN-major: dims contiguous, dims
-            // 64-127 one half tile on), 4 MMAs of 16 keys per block
+            // O_r += P_r V: A = P_r in tensor memory (16 keys = 8 columns per
+            // MMA), B = the step's V rows (MN-major: dims contiguous, dims 64-127
+            // one quarter on), 4 MMAs per block
             auto issue_pv = [&](int r, int k, bool acc) {
-                const uint32_t pa = tmem + kColS + 128 * r;
-                const uint32_t dO = tmem + kColO + 128 * r;
-                const int nblk = min(2, cnt - 2 * k);
-                for (int h = 0; h < nblk; ++h) {
-                    const uint64_t bv = dv0 + ((((2 * k + h) % kAttnStages) * kStageBytes) >> 4);
+                const uint64_t bv = dv + (((k & 1) * 2 * kHalfTile) >> 4);
+                const uint32_t pa = tmem + kColS + 128 * r, d = tmem + kColO + 128 * r;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16_ts(dO, pa + 32 * h + 8 * kk, bv + ((kk * 16 * 128) >> 4), idO,
-                                     acc || h > 0 || kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16_ts(d, pa + 8 * kk, bv + ((kk * 16 * 128) >> 4), idO, acc || kk > 0);
+                if (2 * k + 1 < cnt) {
+#pragma unroll
+                    for (int kk = 4; kk < 8; ++kk)
+                        umma_bf16_ts(d, pa + 8 * kk, bv + ((kk * 16 * 128) >> 4), idO, true);
                 }
             };
-            auto wait_full = [&](int i) {
-                return !*abort_flag &&
-                       mbar_wait_bounded(&full[i % kAttnStages], (i / kAttnStages) & 1);
+            auto wait_step = [&](int k) {
+                const int i0 = 2 * k;
+                bool w = mbar_wait_bounded(&full[i0 & 3], (i0 >> 2) & 1);
+                if (w && i0 + 1 < cnt) w = mbar_wait_bounded(&full[(i0 + 1) & 3], ((i0 + 1) >> 2) & 1);
+                return w;
             };
             bool ok = mbar_wait_bounded(bar_q, 0);
             tc_fence_after();
             for (int k = 0; ok && k <= steps; ++k) {
-                const int i0 = 2 * k, nblk = k < steps ? min(2, cnt - i0) : 0;
                 if (k < steps) {
-                    for (int h = 0; ok && h < nblk; ++h) ok = wait_full(i0 + h);
+                    ok = wait_step(k);
                     if (!ok) break;
                     tc_fence_after();
-                    for (int h = 0; h < nblk; ++h) issue_s(0, i0 + h);
+                    issue_s(0, k);
                     umma_commit(&bar_s[0]);
                 }
                 if (k >= 1) {
-                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[1], (k - 1) & 1);
+                    ok = mbar_wait_bounded(&bar_p[1], (k - 1) & 1);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(1, k - 1, k - 1 > 0);
                     umma_commit(&bar_o[1]);
-                    for (int i = 2 * (k - 1); i < min(cnt, 2 * k); ++i)
-                        umma_commit(&empty[i % kAttnStages]);
+                    umma_commit(&empty[(2 * k - 2) & 3]);
+                    if (2 * k - 1 < cnt) umma_commit(&empty[(2 * k - 1) & 3]);
                 }
                 if (k < steps) {
-                    for (int h = 0; h < nblk; ++h) issue_s(1, i0 + h);
+                    issue_s(1, k);
                     umma_commit(&bar_s[1]);
-                    ok = !*abort_flag && mbar_wait_bounded(&bar_p[0], k & 1);
+                    ok = mbar_wait_bounded(&bar_p[0], k & 1);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(0, k, k > 0);
