@@ -43,8 +43,14 @@ HBM_FALLBACK_GBS = 6650.0
 # the same workload (profiles/sparse_decode_kernel_qwen3_32b_128k.md), valid
 # only for the kernel source it was taken on (sha256 prefix of the .cu file).
 NCU_TRAFFIC = {
-    "qwen3_32b_128k": {"bytes": 728982528 + 3904768, "kernel_sha256": "82c100300b60004f"},
-    "qwen3_8b_128k_tok": {"bytes": 246840064 + 4134144, "kernel_sha256": "82c100300b60004f"},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
+    # kernel (profiles/), valid while its source files are unchanged
+    "qwen3_32b_128k": {"bytes": 728982528 + 3904768, "files": ["sparse_decode.cu"],
+                       "sha256": "82c100300b60004f"},
+    "qwen3_8b_128k_tok": {"bytes": 246840064 + 4134144, "files": ["sparse_decode.cu"],
+                          "sha256": "82c100300b60004f"},
+    "qwen3_8b_prefill_32k": {"bytes": 411750912 + 500070656, "files": ["prefill.cu", "tc.cuh"],
+                             "sha256": "f0bbd2a8ac8dd39b"},
 }
 
 
@@ -53,10 +59,11 @@ def measured_traffic(workload: str):
     rec = NCU_TRAFFIC.get(workload)
     if rec is None:
         return None
-    src = os.path.join(ROOT, "block_sparse_long_spot_b200", "csrc", "sparse_decode.cu")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    return rec["bytes"] if sha == rec["kernel_sha256"] else None
+    h = hashlib.sha256()
+    for name in rec["files"]:
+        with open(os.path.join(ROOT, "block_sparse_long_spot_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return rec["bytes"] if h.hexdigest()[:16] == rec["sha256"] else None
 
 
 def peaks():
@@ -796,7 +803,9 @@ def run_spot_prefill(args, world, rank, local):
                    "parallelism": f"dp{world} (sequences)"},
         "roofline": {"bound": "tensor", "kernel": "sparse prefill (all four kernels)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_kind,
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.workload),
+                     "traffic_kernel": "prefill_attn_kernel (dram read + write of one launch)",
+                     "peak_source": peak_kind,
                      "algorithmic_flops_per_step": int(f_attn + f_score),
                      "attention_flops": int(f_attn), "scoring_flops": int(f_score)},
         "e2e": {"value": round(tokens * world / (ms_e2e / 1e3 * sp_layers(args)), 1),
