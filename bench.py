@@ -199,6 +199,64 @@ def step_bytes(wl, sel_cnt: np.ndarray, fmt: str):
             "selector": sel_cache}
 
 
+class CopyPipeline:
+    """End-to-end stepping with the host copies overlapped: each step's
+    inputs go from pinned host memory to one of two device buffers on an
+    upload stream, the step computes on `stream` from that buffer into one of
+    two output buffers, and the output goes back to pinned host memory on a
+    download stream while the next step computes (uploads and downloads on
+    separate streams, so neither queues behind the other's wait).  Events
+    order every buffer reuse; time() brackets K steps from the first upload
+    to the last download on the device."""
+
+    def __init__(self, dev, host_inputs, out_like, stream):
+        self.stream = stream
+        self.up = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        self.host_inputs = host_inputs                    # per layer: tuple of pinned tensors
+        self.dev_in = [[torch.empty_like(t, device=dev) for t in host_inputs[0]] for _ in range(2)]
+        self.dev_out = [torch.empty_like(out_like) for _ in range(2)]
+        self.host_out = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory()
+                         for _ in range(2)]
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_done = [torch.cuda.Event() for _ in range(2)]
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]
+        self.h2d = sum(t.numel() * t.element_size() for t in host_inputs[0])
+        self.d2h = out_like.numel() * out_like.element_size()
+
+    def step(self, i, compute):
+        k = i & 1
+        self.up.wait_event(self.ev_done[k])           # step i - 2 is done with dev_in[k]
+        with torch.cuda.stream(self.up):
+            for d, h in zip(self.dev_in[k], self.host_inputs[i % len(self.host_inputs)]):
+                d.copy_(h, non_blocking=True)
+            self.ev_in[k].record(self.up)
+        self.stream.wait_event(self.ev_in[k])
+        self.stream.wait_event(self.ev_out[k])        # dev_out[k] of step i - 2 downloaded
+        compute(i, *self.dev_in[k], self.dev_out[k])
+        self.ev_done[k].record(self.stream)
+        self.down.wait_event(self.ev_done[k])
+        with torch.cuda.stream(self.down):
+            self.host_out[k].copy_(self.dev_out[k], non_blocking=True)
+            self.ev_out[k].record(self.down)
+
+    def time(self, K, warmup, compute):
+        for i in range(warmup):
+            self.step(i, compute)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        self.up.wait_event(e0)
+        self.down.wait_event(e0)
+        for i in range(K):
+            self.step(i, compute)
+        self.stream.wait_event(self.ev_out[(K - 1) & 1])
+        self.stream.wait_event(self.ev_out[K & 1])
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
+
 def run_spot(args, world, rank, local):
     import block_sparse_long_spot_b200 as spot
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
@@ -308,33 +366,19 @@ def run_spot(args, world, rank, local):
     del graphs
 
     # ---- end to end through the public call with host buffers
-    pin_q = [layers[l][0].q.cpu().pin_memory() for l in range(len(layers))]
-    pin_qs = [layers[l][0].q_sel.cpu().pin_memory() for l in range(len(layers))]
-    host_out = torch.empty(B, Hq, 128, dtype=torch.float32).pin_memory()
-    q_dev = torch.empty_like(layers[0][0].q)
-    qs_dev = torch.empty_like(layers[0][0].q_sel)
+    pipe = CopyPipeline(dev, [(layers[l][0].q.cpu().pin_memory(),
+                               layers[l][0].q_sel.cpu().pin_memory()) for l in range(len(layers))],
+                        out, stream)
 
-    def e2e_step(i):
+    def e2e_compute(i, q_dev, qs_dev, out_dev):
         wl, desc, data, scales = layers[i % len(layers)]
-        q_dev.copy_(pin_q[i % len(layers)], non_blocking=True)
-        qs_dev.copy_(pin_qs[i % len(layers)], non_blocking=True)
         spot.decode_step(desc, prm, qs_dev, wl.w, data, scales, q_dev, wl.k_pool, wl.v_pool,
                          wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt,
-                         out, lse, ws, stream)
-        host_out.copy_(out, non_blocking=True)
+                         out_dev, lse, ws, stream)
 
-    for i in range(args.warmup):
-        e2e_step(i)
-    torch.cuda.synchronize()
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(K):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(pipe.time(K, args.warmup, e2e_compute), world)
     barrier(world)
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K, world)
     status = spot.read_device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status} after timing")
@@ -393,12 +437,13 @@ def run_spot(args, world, rank, local):
         },
         "e2e": {"value": round(value_e2e, 3), "unit": "tokens/s",
                 "ms_per_step": round(ms_e2e, 5),
-                "h2d_bytes_per_step": int(layers[0][0].q.numel() * 2 + layers[0][0].q_sel.numel() * 2),
-                "d2h_bytes_per_step": int(out.numel() * 4)},
+                "h2d_bytes_per_step": pipe.h2d, "d2h_bytes_per_step": pipe.d2h,
+                "copies": "double-buffered; uploads and downloads on a second stream overlap "
+                          "the neighbouring steps' compute"},
         "graph": {"ms_per_step": round(ms_graph, 5),
                   "value": round(shard_summary(B, world, ms_graph, layers_model), 3),
                   "note": "the same steps replayed from captured CUDA graphs"},
-        "gpu_launches": K * 3,          # block scoring, selection, sparse decode per step
+        "gpu_launches": K * 2,          # scoring + selection (one launch), sparse decode per step
         "clocks": clk.summary(),
     }
     return res, layers
@@ -532,33 +577,19 @@ def run_spot_tok(args, world, rank, local):
     sel_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     dec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
 
-    pin_q = [wl.q.cpu().pin_memory() for wl, _ in layers]
-    pin_qi = [wl.q_idx.cpu().pin_memory() for wl, _ in layers]
-    host_out = torch.empty(B, Hq, 128, dtype=torch.float32).pin_memory()
-    q_dev, qi_dev = torch.empty_like(wl0.q), torch.empty_like(wl0.q_idx)
+    pipe = CopyPipeline(dev, [(wl.q.cpu().pin_memory(), wl.q_idx.cpu().pin_memory())
+                              for wl, _ in layers], out, stream)
 
-    def e2e_step(i):
+    def e2e_compute(i, q_dev, qi_dev, out_dev):
         wl, desc = layers[i % len(layers)]
         sd, ss = pools[i % len(layers)]
-        q_dev.copy_(pin_q[i % len(layers)], non_blocking=True)
-        qi_dev.copy_(pin_qi[i % len(layers)], non_blocking=True)
         spot.tok_decode_step(desc, prm, qi_dev, wl.w_idx, sd, ss, q_dev, wl.k_pool,
                              wl.v_pool, wl.page_table, wl.seq_lens, wl.top_p, wl.sm_scale,
-                             sel_idx, sel_cnt, out, lse, wss[i % len(layers)], stream)
-        host_out.copy_(out, non_blocking=True)
+                             sel_idx, sel_cnt, out_dev, lse, wss[i % len(layers)], stream)
 
-    for i in range(args.warmup):
-        e2e_step(i)
-    torch.cuda.synchronize()
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(K):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(pipe.time(K, args.warmup, e2e_compute), world)
     barrier(world)
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K, world)
     for ws in wss:
         status = spot.read_device_status(ws)
         if status != 0:
@@ -622,8 +653,9 @@ def run_spot_tok(args, world, rank, local):
             "algorithmic_bytes_per_step": int(b_step)},
         "e2e": {"value": round(value_e2e, 3), "unit": "tokens/s",
                 "ms_per_step": round(ms_e2e, 5),
-                "h2d_bytes_per_step": int(wl0.q.numel() * 2 + wl0.q_idx.numel() * 2),
-                "d2h_bytes_per_step": int(out.numel() * 4)},
+                "h2d_bytes_per_step": pipe.h2d, "d2h_bytes_per_step": pipe.d2h,
+                "copies": "double-buffered; uploads and downloads on a second stream overlap "
+                          "the neighbouring steps' compute"},
         "gpu_launches": K * 3,          # token scoring, selection, sparse decode per step
         "clocks": clk.summary(),
     }, layers
@@ -716,12 +748,12 @@ def run_spot_prefill(args, world, rank, local):
     lse = torch.empty(rows, Hq, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(i, q=None, q_sel=None):
+    def step(i, q=None, q_sel=None, o=None):
         w = layers[i % len(layers)]
         spot.prefill(descs[i % len(layers)], prm, w.q_sel if q_sel is None else q_sel, w.w,
                      w.sel_keys, w.q if q is None else q, w.k_pool, w.v_pool, w.page_table,
-                     w.seq_lens, w.q_lens, w.top_p, w.sm_scale, sel_idx, sel_cnt, out, lse,
-                     wss[i % len(layers)], stream)
+                     w.seq_lens, w.q_lens, w.top_p, w.sm_scale, sel_idx, sel_cnt,
+                     out if o is None else o, lse, wss[i % len(layers)], stream)
 
     flops = []
     sel0 = None
@@ -752,26 +784,9 @@ def run_spot_prefill(args, world, rank, local):
     barrier(world)
     ms_step = max_over_ranks(t0.elapsed_time(t1) / K, world)
     # end to end: the step's queries (q, q_sel) copied from pinned host memory
-    pin = [(w.q.cpu().pin_memory(), w.q_sel.cpu().pin_memory()) for w in layers]
-    host_out = torch.empty(rows, Hq, 128, dtype=torch.float32).pin_memory()
-    q_dev, qs_dev = torch.empty_like(wl0.q), torch.empty_like(wl0.q_sel)
-
-    def e2e_step(i):
-        hq, hqs = pin[i % len(layers)]
-        q_dev.copy_(hq, non_blocking=True)
-        qs_dev.copy_(hqs, non_blocking=True)
-        step(i, q_dev, qs_dev)
-        host_out.copy_(out, non_blocking=True)
-
-    e2e_step(0)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(K):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / K, world)
+    pipe = CopyPipeline(dev, [(w.q.cpu().pin_memory(), w.q_sel.cpu().pin_memory())
+                              for w in layers], out, stream)
+    ms_e2e = max_over_ranks(pipe.time(K, 1, lambda i, q, qs, o: step(i, q, qs, o)), world)
     for ws in wss:
         if spot.read_device_status(ws) != 0:
             raise RuntimeError("device status after timing")
@@ -810,8 +825,9 @@ def run_spot_prefill(args, world, rank, local):
                      "attention_flops": int(f_attn), "scoring_flops": int(f_score)},
         "e2e": {"value": round(tokens * world / (ms_e2e / 1e3 * sp_layers(args)), 1),
                 "unit": "tokens/s", "ms_per_step": round(ms_e2e, 4),
-                "h2d_bytes_per_step": int(wl0.q.numel() * 2 + wl0.q_sel.numel() * 2),
-                "d2h_bytes_per_step": int(out.numel() * 4)},
+                "h2d_bytes_per_step": pipe.h2d, "d2h_bytes_per_step": pipe.d2h,
+                "copies": "double-buffered; uploads and downloads on a second stream overlap "
+                          "the neighbouring steps' compute"},
         "gpu_launches": K * 4,          # plan, tile scores, selection, attention per step
         "clocks": clk.summary(),
     }, (layers, sel0[0], sel0[1])
