@@ -856,12 +856,36 @@ static int tok_key_row(const orc_tok_shape_t* sh, const void* data, const void* 
     return -1;
 }
 
+/* The index-head queries of sequence b as fp64 [H_idx][d_idx].  With
+ * quantize_queries (SpotAttention §5.3 and App. G Tab. 9 quantise the
+ * selector's queries together with its key cache) each head's query row
+ * goes through the same quantiser as a key row of the format and is read
+ * back exactly; otherwise the bf16 values are widened. */
+static int tok_queries(const orc_tok_shape_t* sh, const orc_params_t* pr, int b,
+                       const uint16_t* q_idx, double* qv) {
+    int Hi = sh->idx_heads, di = sh->idx_dim;
+    const uint16_t* q0 = q_idx + (int64_t)b * Hi * di;
+    if (!pr->quantize_queries || sh->sel_fmt == ORC_FMT_BF16) {
+        for (int64_t i = 0; i < (int64_t)Hi * di; ++i) qv[i] = bf16_to_f64(q0[i]);
+        return 0;
+    }
+    uint8_t* codes = (uint8_t*)malloc((size_t)Hi * di);
+    uint16_t* scales = (uint16_t*)malloc((size_t)Hi * (di / 32 + 1) * sizeof(uint16_t));
+    int rc = (codes && scales) ? 0 : -2;
+    if (rc == 0) rc = oracle_quantize_selector(sh->sel_fmt, Hi, di, q0, codes, scales);
+    if (rc == 0) rc = oracle_dequant_selector(sh->sel_fmt, Hi, di, codes, scales, qv);
+    free(codes);
+    free(scales);
+    return rc;
+}
+
 /* Score of every complete selection block of sequence b (§2.1 and §2.3):
  * the token score s[t] = (1/tau) sum_h w_h ReLU(q^I_h . k^I_{h,t}) with one
  * key per index head and token, and the block score is the maximum of its
  * tokens' scores.  Token t's keys sit in sel_tok[page][t % ps][h][d_idx]
- * with page = page_table[b][t / ps].  w (NULL -> 1/H_idx) is [B][H_idx].
- * Writes n_full = floor(seq_len / sel_block) scores into out. */
+ * with page = page_table[b][t / ps].  w (NULL -> 1/H_idx) is [B][H_idx];
+ * the queries are those of tok_queries.  Writes n_full =
+ * floor(seq_len / sel_block) scores into out. */
 static int tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, int b,
                            const uint16_t* q_idx, const float* w, const void* sel_tok,
                            const void* sel_scales, const int32_t* page_table, int32_t seq_len,
@@ -869,21 +893,27 @@ static int tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, in
     int Hi = sh->idx_heads, di = sh->idx_dim, sb = sh->sel_block, ps = sh->page_size;
     int64_t n_full = seq_len / sb;
     double* k = (double*)malloc((size_t)di * sizeof(double));
-    if (!k) return -2;
+    double* qv = (double*)malloc((size_t)Hi * di * sizeof(double));
+    if (!k || !qv || tok_queries(sh, pr, b, q_idx, qv) != 0) {
+        free(k);
+        free(qv);
+        return -2;
+    }
     for (int64_t j = 0; j < n_full; ++j) {
         double best = -INFINITY;
         for (int64_t t = j * sb; t < (j + 1) * sb; ++t) {
             int32_t page = page_table[(int64_t)b * sh->max_pages + t / ps];
             double s = 0.0;
             for (int h = 0; h < Hi; ++h) {
-                const uint16_t* q = q_idx + ((int64_t)b * Hi + h) * di;
+                const double* q = qv + (int64_t)h * di;
                 if (tok_key_row(sh, sel_tok, sel_scales,
                                 ((int64_t)page * ps + t % ps) * Hi + h, k)) {
                     free(k);
+                    free(qv);
                     return -1;
                 }
                 double dot = 0.0;
-                for (int d = 0; d < di; ++d) dot += bf16_to_f64(q[d]) * k[d];
+                for (int d = 0; d < di; ++d) dot += q[d] * k[d];
                 double wh = w ? (double)w[(int64_t)b * Hi + h] : 1.0 / Hi;
                 s += wh * (dot > 0.0 ? dot : 0.0);
             }
@@ -893,6 +923,7 @@ static int tok_unit_scores(const orc_tok_shape_t* sh, const orc_params_t* pr, in
         out[j] = best;
     }
     free(k);
+    free(qv);
     return 0;
 }
 

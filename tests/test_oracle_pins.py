@@ -810,3 +810,62 @@ def test_tok_quantised_keys_follow_the_key_quantiser(fmt):
             tok.append(float((w[0] * np.maximum(dots, 0.0)).sum()))
         assert abs(got[0, j] - max(tok)) <= 1e-12 * max(1.0, abs(max(tok))), j
     assert np.isnan(got[0, L // 16:]).all()
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "fp8", "int8"])
+def test_tok_quantised_queries_follow_the_key_quantiser(fmt):
+    # With quantize_queries each index head's 128-element query row goes
+    # through the key format's quantiser (pinned above) and is read back
+    # exactly; the scores are the plain token scores of the read-back query
+    # and key rows.
+    rng = np.random.default_rng(31)
+    P, Hi, L = 2, 2, 100
+    keys = _bf16_bits(rng.normal(size=(P, 64, Hi, 128)))
+    data, scales = oracle.quantize_selector(fmt, keys)
+    q = _bf16_bits(rng.normal(size=(1, Hi, 128)) * 0.3)
+    w = np.array([[0.6, 0.5]], np.float32)
+    pt = np.array([[1, 0]], np.int32)
+    sh = oracle.make_tok_shape(1, 4, 2, P, 2, idx_heads=Hi, sel_fmt=fmt)
+    got = oracle.tok_block_scores(sh, oracle.make_params(quantize_queries=True), q, w, data, pt,
+                                  np.array([L], np.int32), sel_scales=scales)
+    kd = oracle.dequant_selector(fmt, data.reshape(-1, data.shape[-1]),
+                                 None if scales is None else scales.reshape(-1, scales.shape[-1]),
+                                 128).reshape(P, 64, Hi, 128)
+    qc, qs = oracle.quantize_selector(fmt, q[0])
+    qd = oracle.dequant_selector(fmt, qc, qs, 128)
+    plain = oracle.tok_block_scores(sh, oracle.make_params(), q, w, data, pt,
+                                    np.array([L], np.int32), sel_scales=scales)
+    differs = False
+    for j in range(L // 16):
+        tok = []
+        for t in range(16 * j, 16 * j + 16):
+            dots = np.einsum("hd,hd->h", qd, kd[pt[0, t // 64], t % 64])
+            tok.append(float((w[0] * np.maximum(dots, 0.0)).sum()))
+        assert abs(got[0, j] - max(tok)) <= 1e-12 * max(1.0, abs(max(tok))), j
+        differs |= got[0, j] != plain[0, j]
+    assert differs                      # the queries really were quantised
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "fp8"])
+def test_tok_quantised_queries_lossless_on_small_integers(fmt):
+    # Queries in {-3..3} are stored exactly by MXFP4 (power-of-two group
+    # scales) and E4M3, so quantising them changes no score; bf16 keys ignore
+    # the switch altogether.
+    rng = np.random.default_rng(32)
+    P, Hi, L = 2, 4, 128
+    keys = _bf16_bits(rng.integers(-3, 4, size=(P, 64, Hi, 128)).astype(np.float64))
+    data, scales = oracle.quantize_selector(fmt, keys)
+    q = _bf16_bits(rng.integers(-3, 4, size=(1, Hi, 128)).astype(np.float64))
+    pt = np.array([[0, 1]], np.int32)
+    sh = oracle.make_tok_shape(1, 4, 2, P, 2, idx_heads=Hi, sel_fmt=fmt)
+    a = oracle.tok_block_scores(sh, oracle.make_params(quantize_queries=True), q, None, data, pt,
+                                np.array([L], np.int32), sel_scales=scales)
+    b = oracle.tok_block_scores(sh, oracle.make_params(), q, None, data, pt,
+                                np.array([L], np.int32), sel_scales=scales)
+    assert np.array_equal(a, b)
+    shb = oracle.make_tok_shape(1, 4, 2, P, 2, idx_heads=Hi)
+    c = oracle.tok_block_scores(shb, oracle.make_params(quantize_queries=True), q, None, keys, pt,
+                                np.array([L], np.int32))
+    d = oracle.tok_block_scores(shb, oracle.make_params(), q, None, keys, pt,
+                                np.array([L], np.int32))
+    assert np.array_equal(c, d)
