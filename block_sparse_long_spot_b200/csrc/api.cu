@@ -441,7 +441,6 @@ spot_status_t check_tok_select_args(const spot_tok_layer_desc_t* d,
                                     int32_t* sel_idx, int32_t* sel_cnt) {
     spot_status_t st = check_params(pr);
     if (st != SPOT_OK) return st;
-    if (pr->quantize_queries) return SPOT_ERR_UNSUPPORTED;
     if (!q_idx || !sel_data || !page_table || !seq_lens || !sel_idx || !sel_cnt)
         return SPOT_ERR_INVALID_ARG;
     if (needs_scales(d->sel_fmt) && (!sel_scales || !aligned(sel_scales, 16)))
@@ -488,6 +487,7 @@ spot_status_t do_tok_select(const spot_tok_layer_desc_t* d, const spot_select_pa
     tp.num_ctas = tok_score_grid(d->sel_fmt, batch);
     tp.fmt = d->sel_fmt;
     tp.sel_scales = sel_scales;
+    tp.quantize_queries = pr->quantize_queries;
     tp.status = status;
     if (tp.num_ctas <= 0) return SPOT_ERR_CUDA;
     if (launch_tok_score(tp, sm, s) != cudaSuccess) return SPOT_ERR_CUDA;

@@ -119,6 +119,7 @@ struct TokScoreParams {
     int32_t num_ctas;
     int32_t fmt;                        // spot_sel_fmt_t of the per-token key rows
     const void* sel_scales;             // their scales (INT4 / MXFP4 / INT8), else null
+    int32_t quantize_queries;           // quantise q_idx with the key format's rule
     uint32_t* status;
 };
 

@@ -81,7 +81,8 @@ __device__ __forceinline__ int range_begin(int64_t N, int64_t P, int64_t i) {
 //          the scale group c.
 template <int FMT>
 __device__ __forceinline__ void tile_dots(uint32_t kb, const uint8_t* sc_smem, int mt, int lane,
-                                          const uint32_t (&qf)[8][2], float (&acc)[4]) {
+                                          const uint32_t (&qf)[8][2], const float (&qs)[4][2],
+                                          float (&acc)[4]) {
     acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
     const int r8 = lane >> 2;
     const int rowA = mt * 16 + r8, rowB = rowA + 8;       // this lane's two rows
@@ -110,12 +111,18 @@ __device__ __forceinline__ void tile_dots(uint32_t kb, const uint8_t* sc_smem, i
             mma_f16_16816(acc, lo[0], lo[1], hi[0], hi[1], qf[2 * cp][0], qf[2 * cp][1]);
             mma_f16_16816(acc, lo[2], lo[3], hi[2], hi[3], qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
         }
+        float sa = qs[0][0], sb = qs[0][1];            // query scales of columns 2 c4, + 1
         if constexpr (FMT == SPOT_SEL_INT8_F16) {
             const __half* s = reinterpret_cast<const __half*>(sc_smem);
-            const float sa = __half2float(s[rowA]), sb = __half2float(s[rowB]);
+            const float ka = __half2float(s[rowA]), kb2 = __half2float(s[rowB]);
+            acc[0] *= ka * sa;
+            acc[1] *= ka * sb;
+            acc[2] *= kb2 * sa;
+            acc[3] *= kb2 * sb;
+        } else {
             acc[0] *= sa;
-            acc[1] *= sa;
-            acc[2] *= sb;
+            acc[1] *= sb;
+            acc[2] *= sa;
             acc[3] *= sb;
         }
     } else {
@@ -155,10 +162,10 @@ __device__ __forceinline__ void tile_dots(uint32_t kb, const uint8_t* sc_smem, i
                 sa = e8m0_value(sc_smem[rowA * 4 + c]);
                 sb = e8m0_value(sc_smem[rowB * 4 + c]);
             }
-            acc[0] = fmaf(g[c][0], sa, acc[0]);
-            acc[1] = fmaf(g[c][1], sa, acc[1]);
-            acc[2] = fmaf(g[c][2], sb, acc[2]);
-            acc[3] = fmaf(g[c][3], sb, acc[3]);
+            acc[0] = fmaf(g[c][0], sa * qs[c][0], acc[0]);
+            acc[1] = fmaf(g[c][1], sa * qs[c][1], acc[1]);
+            acc[2] = fmaf(g[c][2], sb * qs[c][0], acc[2]);
+            acc[3] = fmaf(g[c][3], sb * qs[c][1], acc[3]);
         }
     }
 }
@@ -183,10 +190,17 @@ __device__ __forceinline__ int query_dim(int ks, int j, int e, int c4) {
 // |q| lands in [2^14, 2^15) -- no overflow, and only elements below 2^-29 of
 // that maximum round -- returning 2^-s for the head of this lane's column
 // (index head (lane >> 2) & 3), times 2^14 for MXFP4 (whose widened keys
-// carry 2^-14).
+// carry 2^-14).  With `quantize` (quantised keys only) each head's query is
+// first quantised with the key format's rule (quant.cuh; INT4 / MXFP4 per
+// group of 32 dims, INT8 per head): the fragments hold the codes' values,
+// exact in f16, and qs[c][col] receives the query scale of group c (INT8 /
+// FP8: qs[0]) for this lane's accumulator columns 2 c4 and 2 c4 + 1.
 template <int FMT>
 __device__ __forceinline__ float load_tok_queries(const uint16_t* q_idx, int b, int lane,
-                                                  uint32_t (&qf)[8][2]) {
+                                                  bool quantize, uint32_t (&qf)[8][2],
+                                                  float (&qs)[4][2]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) qs[c][0] = qs[c][1] = 1.f;
     const int c4 = lane & 3, r8 = lane >> 2;
     const bool real = r8 < kIdxHeads;
     const uint16_t* qrow = q_idx + (static_cast<int64_t>(b) * kIdxHeads + (real ? r8 : 0)) * kIdxDim;
@@ -212,6 +226,66 @@ __device__ __forceinline__ float load_tok_queries(const uint16_t* q_idx, int b, 
                     v[ks][j][e] = __uint_as_float(static_cast<uint32_t>(bits) << 16);
                     am = fmaxf(am, fabsf(v[ks][j][e]));
                 }
+        if (quantize) {
+            // per-group (4-bit: ks = 2 c, 2 c + 1 hold dims 32 c ..) or per-head scales
+            float gs[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float ga = 0.f;
+                if constexpr (FMT == SPOT_SEL_INT4_G32_F16 || FMT == SPOT_SEL_MXFP4_G32_E8M0) {
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) ga = fmaxf(ga, fabsf(v[2 * c + t][j][e]));
+                } else {
+                    ga = am;
+                }
+                ga = fmaxf(ga, __shfl_xor_sync(0xffffffffu, ga, 1));
+                ga = fmaxf(ga, __shfl_xor_sync(0xffffffffu, ga, 2));
+                gs[c] = ga;                           // group (or head) maximum
+            }
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int c = ks >> 1;
+                float sc = 1.f;
+                int X = 0;
+                if constexpr (FMT == SPOT_SEL_INT4_G32_F16) sc = f16_bits_value(f16_scale_bits(gs[c], 7.0));
+                else if constexpr (FMT == SPOT_SEL_INT8_F16) sc = f16_bits_value(f16_scale_bits(gs[0], 127.0));
+                else if constexpr (FMT == SPOT_SEL_MXFP4_G32_E8M0) X = mx_exponent(gs[c]);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float cv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float x = v[ks][j][e];
+                        if constexpr (FMT == SPOT_SEL_INT4_G32_F16)
+                            cv[e] = static_cast<float>(int_code(x, sc, -8, 7));
+                        else if constexpr (FMT == SPOT_SEL_INT8_F16)
+                            cv[e] = static_cast<float>(int_code(x, sc, -128, 127));
+                        else if constexpr (FMT == SPOT_SEL_MXFP4_G32_E8M0)
+                            cv[e] = e2m1_value(mx_code(x, X));
+                        else
+                            cv[e] = fp8_value(fp8_code(x));
+                    }
+                    const __half2 h = __floats2half2_rn(cv[0], cv[1]);
+                    qf[ks][j] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+            }
+            // this lane's columns 2 c4, 2 c4 + 1 are index heads held by quads 2 c4, 2 c4 + 1
+            const int c4 = lane & 3;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float s = 1.f;
+                if constexpr (FMT == SPOT_SEL_INT4_G32_F16) s = f16_bits_value(f16_scale_bits(gs[c], 7.0));
+                else if constexpr (FMT == SPOT_SEL_INT8_F16) s = f16_bits_value(f16_scale_bits(gs[0], 127.0));
+                else if constexpr (FMT == SPOT_SEL_MXFP4_G32_E8M0) s = ldexpf(1.f, mx_exponent(gs[c]));
+                qs[c][0] = __shfl_sync(0xffffffffu, s, 4 * (2 * c4));
+                qs[c][1] = __shfl_sync(0xffffffffu, s, (4 * (2 * c4 + 1)) & 31);
+            }
+            return FMT == SPOT_SEL_MXFP4_G32_E8M0 ? 16384.f : 1.f;
+        }
         am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));   // the quad holds one head
         am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
         const int sh = am > 0.f ? min(120, max(-113, 14 - ilogbf(am))) : 0;
@@ -363,13 +437,14 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
     const bool odd = head & 1;
     int cur_b = -1;
     uint32_t qf[8][2];
+    float qs[4][2];
     float wh = 0.f, unscale = 1.f;
     for (int it = warp; it < n_it; it += NCS) {
         const int pos = beg + it;
         const int b = find_seq(seq_off, B, pos);
         const int j = pos - seq_off[b];
         if (b != cur_b) {
-            unscale = load_tok_queries<FMT>(p.q_idx, b, lane, qf);
+            unscale = load_tok_queries<FMT>(p.q_idx, b, lane, p.quantize_queries != 0, qf, qs);
             wh = p.w ? p.w[static_cast<int64_t>(b) * kIdxHeads + head] : 1.f / kIdxHeads;
             cur_b = b;
         }
@@ -391,7 +466,7 @@ tok_score_kernel(const __grid_constant__ CUtensorMap sel_map, const TokScorePara
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
             float acc[4];
-            tile_dots<FMT>(kb, scl, mt, lane, qf, acc);
+            tile_dots<FMT>(kb, scl, mt, lane, qf, qs, acc);
             float top = (odd ? acc[1] : acc[0]) * unscale;
             float bot = (odd ? acc[3] : acc[2]) * unscale;
             top = owner ? wh * fmaxf(top, 0.f) : 0.f;

@@ -259,8 +259,11 @@ spot_status_t spot_sparse_decode_noalloc(const spot_layer_desc_t* desc, const ui
  *                    ascending, first sel_cnt entries valid
  *   sel_cnt    int32 [batch]
  * The selection parameters count blocks of sel_block tokens (the paper's
- * sink 128 / recency 256 / K_min 512 tokens are 8 / 16 / 32 blocks);
- * quantize_queries must be 0.  nb(b) = ceil(seq_lens[b] / sel_block); an
+ * sink 128 / recency 256 / K_min 512 tokens are 8 / 16 / 32 blocks).  With
+ * quantize_queries each index head's 128-element query is quantised with
+ * the key format's rule (group-32 INT4 / MXFP4, one fp16 scale per head for
+ * INT8, E4M3) and its exact values enter the score; no effect for bf16 keys.
+ * nb(b) = ceil(seq_lens[b] / sel_block); an
  * incomplete last block has no score and is always kept.
  * ------------------------------------------------------------------------ */
 typedef struct {

@@ -264,14 +264,14 @@ def gpu_tok_pool(wl, fmt, desc):
 
 
 def run_gpu_tok(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None, temperature=1.0,
-                max_blocks=None, pool=None, fmt="bf16"):
+                max_blocks=None, pool=None, fmt="bf16", quantize_queries=False):
     dev = wl.q.device
     B, Hq, Hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
     mb = wl.max_blocks if max_blocks is None else max_blocks
     kmin, sink, rec = _tok_sel(wl.spec, kmin, sink, rec)
     desc = spot.tok_layer_desc(Hq, Hkv, wl.num_pages, sel_fmt=fmt)
     data, scales = gpu_tok_pool(wl, fmt, desc) if pool is None else pool
-    prm = spot.select_params(mode, sink, rec, kmin, topk, temperature)
+    prm = spot.select_params(mode, sink, rec, kmin, topk, temperature, quantize_queries)
     ws = spot.new_tok_workspace(desc, B, mb, dev)
     sel_idx = torch.full((B, mb), -1, dtype=torch.int32, device=dev)
     sel_cnt = torch.full((B,), -1, dtype=torch.int32, device=dev)
@@ -301,12 +301,12 @@ def tok_oracle_args(wl, fmt="bf16"):
 
 
 def tok_oracle_shape_params(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None,
-                            temperature=1.0, max_blocks=None, fmt="bf16"):
+                            temperature=1.0, max_blocks=None, fmt="bf16", quantize_queries=False):
     kmin, sink, rec = _tok_sel(wl.spec, kmin, sink, rec)
     sh = oracle.make_tok_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.num_pages,
                                wl.max_pages, max_blocks=wl.max_blocks if max_blocks is None
                                else max_blocks, sel_fmt=fmt)
-    pr = oracle.make_params(mode, sink, rec, kmin, topk, temperature)
+    pr = oracle.make_params(mode, sink, rec, kmin, topk, temperature, quantize_queries)
     return sh, pr
 
 

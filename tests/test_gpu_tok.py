@@ -255,3 +255,43 @@ def test_tok_every_e2m1_magnitude_bit_exact(fmt):
     ora = run_oracle_tok(wl, fmt=fmt)
     _same(gpu, ora, wl)
     check_tok_outputs(gpu, ora, wl)
+
+
+# ------------------------------------------------ quantised index-head queries
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "fp8"])
+def test_tok_quantised_queries_integer_inputs_bit_exact(fmt):
+    # queries and keys in {-3..3}: MXFP4 and E4M3 store them losslessly, so the
+    # scores are exact on both sides and the selections must match
+    wl = workloads.make_tok("tok_tiny_2k", seed=17, device=DEV, integer=True, batch=3,
+                            seq_len=None, ragged_range=(64, 4096))
+    wl.top_p = safe_top_p_tok(wl, fmt=fmt, quantize_queries=True)
+    gpu = run_gpu_tok(wl, fmt=fmt, quantize_queries=True)
+    assert gpu["status"] == 0
+    ora = run_oracle_tok(wl, fmt=fmt, quantize_queries=True)
+    _same(gpu, ora, wl)
+    check_tok_outputs(gpu, ora, wl)
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_tok_quantised_queries_tiny(fmt):
+    wl = workloads.make_tok("tok_tiny_2k", seed=18, device=DEV)
+    gpu = run_gpu_tok(wl, fmt=fmt, quantize_queries=True)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl, fmt)
+    ora = run_oracle_tok(wl, args=args, fmt=fmt, quantize_queries=True)
+    scores = oracle_tok_scores(wl, args=args, fmt=fmt, quantize_queries=True)
+    assert check_tok_selection_near_cut(gpu, ora, scores, wl) <= 1
+    _, n = check_tok_outputs(gpu, ora, wl)
+    assert n >= wl.batch - 1
+
+
+def test_tok_quantised_queries_full_size_int4():
+    wl = workloads.make_tok("qwen3_8b_128k_tok", seed=3, device=DEV)
+    gpu = run_gpu_tok(wl, fmt="int4", quantize_queries=True)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl, "int4")
+    ora = run_oracle_tok(wl, args=args, fmt="int4", quantize_queries=True)
+    scores = oracle_tok_scores(wl, args=args, fmt="int4", quantize_queries=True)
+    assert check_tok_selection_near_cut(gpu, ora, scores, wl) <= 1
+    check_tok_outputs(gpu, ora, wl)
