@@ -542,16 +542,19 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap k_map,
                 for (int c = 0; c < 64; ++c)
                     if (c > lim) sv[64 + c] = -INFINITY;
             }
-            float pm[16];
+            float pm[16];                         // three-input maxima: 16 lanes of 8
 #pragma unroll
-            for (int c = 0; c < 16; ++c) pm[c] = sv[c];
+            for (int c = 0; c < 16; ++c) pm[c] = fmax3(sv[c], sv[c + 16], sv[c + 32]);
 #pragma unroll
-            for (int c = 16; c < 128; ++c) pm[c & 15] = fmaxf(pm[c & 15], sv[c]);
+            for (int c = 0; c < 16; ++c) pm[c] = fmax3(pm[c], sv[c + 48], sv[c + 64]);
 #pragma unroll
-            for (int w = 8; w > 0; w >>= 1)
+            for (int c = 0; c < 16; ++c) pm[c] = fmax3(pm[c], sv[c + 80], sv[c + 96]);
 #pragma unroll
-                for (int c = 0; c < w; ++c) pm[c] = fmaxf(pm[c], pm[c + w]);
-            const float mx = pm[0] * sl2;
+            for (int c = 0; c < 16; ++c) pm[c] = fmaxf(pm[c], sv[c + 112]);
+#pragma unroll
+            for (int c = 0; c < 5; ++c) pm[c] = fmax3(pm[3 * c], pm[3 * c + 1], pm[3 * c + 2]);
+            const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[15]),
+                                   -INFINITY) * sl2;
             // O_r and the P_r columns are free once the previous O_r += P_r V completed
             if (k > 0) {
                 ok = !*abort_flag && mbar_wait_bounded(&bar_o[r], (k - 1) & 1);
