@@ -49,8 +49,8 @@ NCU_TRAFFIC = {
                        "sha256": "82c100300b60004f"},
     "qwen3_8b_128k_tok": {"bytes": 246840064 + 4134144, "files": ["sparse_decode.cu"],
                           "sha256": "82c100300b60004f"},
-    "qwen3_8b_prefill_32k": {"bytes": 411750912 + 500070656, "files": ["prefill.cu", "tc.cuh"],
-                             "sha256": "f0bbd2a8ac8dd39b"},
+    "qwen3_8b_prefill_32k": {"bytes": 411734016 + 499205376, "files": ["prefill.cu", "tc.cuh"],
+                             "sha256": "362fd0bc4a92eeba"},
 }
 
 
