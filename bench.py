@@ -751,7 +751,7 @@ def run_spot_prefill(args, world, rank, local):
     def step(i, q=None, q_sel=None, o=None):
         w = layers[i % len(layers)]
         spot.prefill(descs[i % len(layers)], prm, w.q_sel if q_sel is None else q_sel, w.w,
-                     w.sel_keys, w.q if q is None else q, w.k_pool, w.v_pool, w.page_table,
+                     w.sel_keys, None, w.q if q is None else q, w.k_pool, w.v_pool, w.page_table,
                      w.seq_lens, w.q_lens, w.top_p, w.sm_scale, sel_idx, sel_cnt,
                      out if o is None else o, lse, wss[i % len(layers)], stream)
 

@@ -108,8 +108,8 @@ def lib():
         L.spot_prefill_num_tiles.restype = ctypes.c_int64
         L.spot_prefill_workspace_size.argtypes = [P, i32, i32, i32]
         L.spot_prefill_workspace_size.restype = sz
-        L.spot_prefill.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, P, P, i32, i32, f32, P, P,
-                                   i32, P, P, P, sz, P]
+        L.spot_prefill.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, P, P, P, i32, i32, f32, P,
+                                   P, i32, P, P, P, sz, P]
         L.spot_prefill.restype = ctypes.c_int
         L.spot_read_device_status.argtypes = [P, P]
         L.spot_check_wait_timeout.argtypes = [P, P]
@@ -364,17 +364,19 @@ def new_prefill_workspace(desc: LayerDesc, batch: int, max_tiles: int, max_block
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def prefill(desc: LayerDesc, params: SelectParams, q_sel, w, sel_data, q, k_pool, v_pool,
-            page_table, seq_lens, q_lens, top_p, softmax_scale, sel_idx, sel_cnt, out, lse,
-            workspace, stream=None):
+def prefill(desc: LayerDesc, params: SelectParams, q_sel, w, sel_data, sel_scales, q, k_pool,
+            v_pool, page_table, seq_lens, q_lens, top_p, softmax_scale, sel_idx, sel_cnt, out,
+            lse, workspace, stream=None):
     """Sparse prefill of packed chunk queries: per (tile, KV head) selection
     into sel_idx int32 [max_tiles, Hkv, max_blocks] / sel_cnt [max_tiles, Hkv],
-    causal attention into out fp32 [rows, Hq, D] (+ lse [rows, Hq])."""
+    causal attention into out fp32 [rows, Hq, D] (+ lse [rows, Hq]).  The
+    selector pool (sel_data, sel_scales) is in the descriptor's format."""
     B = int(seq_lens.shape[0])
     max_tiles, max_blocks = int(sel_idx.shape[0]), int(sel_idx.shape[-1])
     code = lib().spot_prefill(
         ctypes.byref(desc), ctypes.byref(params), _ptr(q_sel, torch.bfloat16, "q_sel"),
-        _ptr(w, torch.float32, "w"), _ptr(sel_data, torch.bfloat16, "sel_data"),
+        _ptr(w, torch.float32, "w"), _ptr(sel_data, name="sel_data"),
+        _ptr(sel_scales, name="sel_scales"),
         _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
         _ptr(v_pool, torch.bfloat16, "v_pool"), _ptr(page_table, torch.int32, "page_table"),
         int(page_table.shape[-1]), _ptr(seq_lens, torch.int32, "seq_lens"),

@@ -717,7 +717,6 @@ spot_status_t check_prefill_shape(const spot_layer_desc_t* d, int batch, int max
                                   int max_blocks) {
     spot_status_t st = check_desc(d);
     if (st != SPOT_OK) return st;
-    if (d->sel_fmt != SPOT_SEL_BF16) return SPOT_ERR_UNSUPPORTED;
     if (batch < 0 || max_tiles < 0 || max_blocks <= 0) return SPOT_ERR_INVALID_ARG;
     if (max_blocks > kMaxBlocks || batch > kMaxUnits) return SPOT_ERR_UNSUPPORTED;
     // selection grid and unit indices
@@ -753,6 +752,7 @@ size_t spot_prefill_workspace_size(const spot_layer_desc_t* desc, int32_t batch,
 
 spot_status_t spot_prefill(const spot_layer_desc_t* desc, const spot_select_params_t* params,
                            const uint16_t* q_sel, const float* w, const void* sel_data,
+                           const void* sel_scales,
                            const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
                            const int32_t* page_table, int32_t pt_stride,
                            const int32_t* seq_lens, const int32_t* q_lens, const float* top_p,
@@ -764,12 +764,13 @@ spot_status_t spot_prefill(const spot_layer_desc_t* desc, const spot_select_para
     if (batch == 0 || max_tiles == 0) return SPOT_OK;
     st = check_params(params);
     if (st != SPOT_OK) return st;
-    if (params->quantize_queries) return SPOT_ERR_UNSUPPORTED;
     if (!q_sel || !sel_data || !q || !k_pool || !v_pool || !page_table || !seq_lens || !q_lens ||
         !sel_idx || !sel_cnt || !out)
         return SPOT_ERR_INVALID_ARG;
     if (params->mode == SPOT_MODE_TOPP && !top_p) return SPOT_ERR_INVALID_ARG;
     if (pt_stride <= 0 || !isfinite(softmax_scale)) return SPOT_ERR_INVALID_ARG;
+    if (needs_scales(desc->sel_fmt) && (!sel_scales || !aligned(sel_scales, 16)))
+        return SPOT_ERR_INVALID_ARG;
     if (!aligned(q_sel, 16) || !aligned(sel_data, 16) || !aligned(q, 16) ||
         !aligned(k_pool, 256) || !aligned(v_pool, 256) || !aligned(page_table, 4) ||
         !aligned(seq_lens, 4) || !aligned(q_lens, 4) || !aligned(sel_idx, 4) ||
@@ -802,6 +803,9 @@ spot_status_t spot_prefill(const spot_layer_desc_t* desc, const spot_select_para
     p.group = desc->num_q_heads / desc->num_kv_heads;
     p.max_blocks = max_blocks;
     p.sel_data = sel_data;
+    p.sel_scales = needs_scales(desc->sel_fmt) ? sel_scales : nullptr;
+    p.fmt = desc->sel_fmt;
+    p.quantize_queries = desc->sel_fmt == SPOT_SEL_BF16 ? 0 : params->quantize_queries;
     p.q_sel = q_sel;
     p.w = w;
     p.inv_temp = 1.0f / params->temperature;

@@ -28,6 +28,7 @@
 
 #include <mutex>
 
+#include "quant.cuh"
 #include "spot_device.cuh"
 #include "spot_internal.h"
 #include "tc.cuh"
@@ -245,6 +246,215 @@ prefill_score_kernel(const PrefillParams p) {
             if (j < n_full) out[j] = m * p.inv_temp;
         }
         __syncthreads();                          // keys[kt & 1] and pmax are reused
+    }
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Quantised selector keys (INT4 / MXFP4 / FP8 / INT8): the tile's keys are
+// staged as code rows (64 bytes of 8-bit codes or 32 of 4-bit codes) plus
+// the 4-byte word holding each key's scales, by cp.async into a double
+// buffer; each lane widens its own code bytes to bf16 in registers (exact;
+// 8-bit: dims [16 c4, 16 c4 + 16), 4-bit: dims [8 c4, 8 c4 + 8) of each
+// 32-dim group, the order selector_query_words gives the queries) and the
+// key and query scales go to the accumulators, as in the decode selection.
+template <int FMT>
+__global__ void __launch_bounds__(kScoreThreads)
+prefill_score_q_kernel(const PrefillParams p) {
+    constexpr bool k8 = FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16;
+    constexpr int CB = k8 ? kSelDim : kSelDim / 2;                 // code bytes per key
+    constexpr int SB = FMT == SPOT_SEL_INT4_G32_F16 ? 4 : (FMT == SPOT_SEL_FP8_E4M3 ? 0 : 2);
+    __shared__ __align__(16) uint8_t codes[2][64 * CB];
+    __shared__ uint32_t scw[2][64];               // the word holding a key's scales
+    __shared__ uint8_t sco[2][64];                // their byte offset in that word
+    __shared__ float pmax[kScoreWarps][64];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c4 = lane & 3, r8 = lane >> 2;
+    const int unit = blockIdx.x;                  // tile * Hkv + g
+    const int t = unit / p.num_kv_heads, g = unit - t * p.num_kv_heads;
+    pdl_wait();                                   // the tile table
+    pdl_trigger();
+    const int4 info = p.tile_info[t];
+    const int b = info.x;
+    if (b < 0) return;
+    const int n_full = min((info.z + 1) / kBlock, min(p.max_blocks, p.pt_stride));
+    if (n_full <= 0) return;
+    const int nq = info.z - info.y + 1;
+    const int G = p.group;
+
+    // query fragments of this warp's 8 queries (n-tile nt: query 8 warp + nt,
+    // column r8: head r8), in the key tiles' dim order; weights and query
+    // scales of this lane's accumulator columns (heads 2 c4, 2 c4 + 1)
+    uint32_t qw[8][8];
+    float w0[8], w1[8], qs0[8][2], qs1[8][2];
+    bool qvalid[8];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        const int q = warp * 8 + nt;
+        qvalid[nt] = q < nq;
+        const int64_t row = info.w + q;
+        const bool real = qvalid[nt] && r8 < G;
+        const uint16_t* qr = p.q_sel + ((real ? row : 0) * p.num_q_heads + g * G +
+                                        (real ? r8 : 0)) * kSelDim;
+        float qs[2];
+        selector_query_words<FMT>(qr, c4, real, p.quantize_queries != 0, qw[nt], qs);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const float a = __shfl_sync(0xffffffffu, qs[hf], 8 * c4);
+            const float c = __shfl_sync(0xffffffffu, qs[hf], 8 * c4 + 4);
+            if (hf == 0) { qs0[nt][0] = a; qs0[nt][1] = c; }
+            else { qs1[nt][0] = a; qs1[nt][1] = c; }
+        }
+        const int64_t wr = row * p.num_q_heads + g * G;
+        w0[nt] = (qvalid[nt] && 2 * c4 < G) ? (p.w ? p.w[wr + 2 * c4] : 1.f / G) : 0.f;
+        w1[nt] = (qvalid[nt] && 2 * c4 + 1 < G) ? (p.w ? p.w[wr + 2 * c4 + 1] : 1.f / G) : 0.f;
+        if (k8) {                                 // one positive scale per head: into the weight
+            w0[nt] *= qs0[nt][0];
+            w1[nt] *= qs0[nt][1];
+        }
+    }
+
+    auto stage = [&](int j0, int buf) {
+        const int key = threadIdx.x >> 2, part = threadIdx.x & 3;
+        const int j = j0 + key;
+        if (j >= n_full) return;
+        int page = p.page_table[static_cast<int64_t>(b) * p.pt_stride + j];
+        if (page < 0 || page >= p.num_pages) {
+            if (part == 0) flag_status(p.status, kStatusBounds);
+            page = 0;
+        }
+        const int64_t krow = static_cast<int64_t>(page) * p.num_kv_heads + g;
+        if (part * 16 < CB)
+            cp_async16(smem_u32(codes[buf] + key * CB + part * 16),
+                       static_cast<const uint8_t*>(p.sel_data) + krow * CB + part * 16);
+        if (SB > 0 && part == 0) {
+            const int64_t off = krow * SB;
+            const int64_t word = off & ~static_cast<int64_t>(3);
+            const uint8_t* sc = static_cast<const uint8_t*>(p.sel_scales);
+            if (word + 4 <= static_cast<int64_t>(p.num_pages) * p.num_kv_heads * SB) {
+                cp_async4(smem_u32(&scw[buf][key]), sc + word);
+                sco[buf][key] = static_cast<uint8_t>(off & 3);
+            } else {                              // the pool's last 2-byte scale, odd row count
+                scw[buf][key] = *reinterpret_cast<const uint16_t*>(sc + off);
+                sco[buf][key] = 0;
+            }
+        }
+    };
+    // scale of group grp (0 / 1) of staged key k
+    auto key_scale = [&](int buf, int k, int grp) -> float {
+        const uint32_t wd = scw[buf][k];
+        if (FMT == SPOT_SEL_INT4_G32_F16) {
+            return __half2float(__ushort_as_half(static_cast<unsigned short>(wd >> (16 * grp))));
+        } else if (FMT == SPOT_SEL_MXFP4_G32_E8M0) {
+            return e8m0_value((wd >> (8 * (sco[buf][k] + grp))) & 0xFFu);
+        } else if (FMT == SPOT_SEL_INT8_F16) {
+            return __half2float(__ushort_as_half(static_cast<unsigned short>(wd >> (8 * sco[buf][k]))));
+        }
+        return 1.f;
+    };
+
+    const int n_tiles = (n_full + 63) / 64;
+    stage(0, 0);
+    cp_async_commit();
+    float* out = p.scores + static_cast<int64_t>(unit) * p.max_blocks;
+    for (int kt = 0; kt < n_tiles; ++kt) {
+        const int buf = kt & 1;
+        if (kt + 1 < n_tiles) stage((kt + 1) * 64, buf ^ 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+            const int ka = mt * 16 + r8, kb = ka + 8;   // this lane's two keys
+            float acc[8][4];
+            if constexpr (k8) {
+                const uint4 xa = *reinterpret_cast<const uint4*>(codes[buf] + ka * CB + 16 * c4);
+                const uint4 xb = *reinterpret_cast<const uint4*>(codes[buf] + kb * CB + 16 * c4);
+                const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w};
+                const uint32_t wb[4] = {xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 4; ++s2) {
+                    const uint32_t a0 = pair8_to_bf16x2<FMT>(wa[s2]), a1 = pair8_to_bf16x2<FMT>(wb[s2]);
+                    const uint32_t a2 = pair8_to_bf16x2<FMT>(wa[s2] >> 16);
+                    const uint32_t a3 = pair8_to_bf16x2<FMT>(wb[s2] >> 16);
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt)
+                        mma_bf16_16816(acc[nt], a0, a1, a2, a3, qw[nt][2 * s2], qw[nt][2 * s2 + 1]);
+                }
+                const float sa = key_scale(buf, ka, 0), sb = key_scale(buf, kb, 0);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    acc[nt][0] *= sa;
+                    acc[nt][1] *= sa;
+                    acc[nt][2] *= sb;
+                    acc[nt][3] *= sb;
+                }
+            } else {
+                const uint32_t* ca = reinterpret_cast<const uint32_t*>(codes[buf] + ka * CB);
+                const uint32_t* cb = reinterpret_cast<const uint32_t*>(codes[buf] + kb * CB);
+                const uint32_t ga[2] = {ca[c4], ca[4 + c4]}, gb[2] = {cb[c4], cb[4 + c4]};
+                const float sa[2] = {key_scale(buf, ka, 0), key_scale(buf, ka, 1)};
+                const float sb[2] = {key_scale(buf, kb, 0), key_scale(buf, kb, 1)};
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+                for (int grp = 0; grp < 2; ++grp) {
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt) {
+                        float gacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int s2 = 0; s2 < 2; ++s2)
+                            mma_bf16_16816(gacc, byte_to_bf16x2<FMT>((ga[grp] >> (16 * s2)) & 0xFFu),
+                                           byte_to_bf16x2<FMT>((gb[grp] >> (16 * s2)) & 0xFFu),
+                                           byte_to_bf16x2<FMT>((ga[grp] >> (16 * s2 + 8)) & 0xFFu),
+                                           byte_to_bf16x2<FMT>((gb[grp] >> (16 * s2 + 8)) & 0xFFu),
+                                           qw[nt][4 * grp + 2 * s2], qw[nt][4 * grp + 2 * s2 + 1]);
+                        const float q0 = grp ? qs1[nt][0] : qs0[nt][0];
+                        const float q1 = grp ? qs1[nt][1] : qs0[nt][1];
+                        acc[nt][0] = fmaf(gacc[0], sa[grp] * q0, acc[nt][0]);
+                        acc[nt][1] = fmaf(gacc[1], sa[grp] * q1, acc[nt][1]);
+                        acc[nt][2] = fmaf(gacc[2], sb[grp] * q0, acc[nt][2]);
+                        acc[nt][3] = fmaf(gacc[3], sb[grp] * q1, acc[nt][3]);
+                    }
+                }
+            }
+            // keys 16 mt + r8 and + 8; per query: weighted ReLU head sum
+            float best0 = -INFINITY, best1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                float s0 = w0[nt] * fmaxf(acc[nt][0], 0.f) + w1[nt] * fmaxf(acc[nt][1], 0.f);
+                float s1 = w0[nt] * fmaxf(acc[nt][2], 0.f) + w1[nt] * fmaxf(acc[nt][3], 0.f);
+                s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+                s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+                if (qvalid[nt]) {
+                    best0 = fmaxf(best0, s0);
+                    best1 = fmaxf(best1, s1);
+                }
+            }
+            if (c4 == 0) {
+                pmax[warp][mt * 16 + r8] = best0;
+                pmax[warp][mt * 16 + r8 + 8] = best1;
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < 64) {
+            const int j = kt * 64 + threadIdx.x;
+            float m = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kScoreWarps; ++w) m = fmaxf(m, pmax[w][threadIdx.x]);
+            if (j < n_full) out[j] = m * p.inv_temp;
+        }
+        __syncthreads();                          // codes[buf] and pmax are reused
     }
 }
 
@@ -658,7 +868,28 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& k_map,
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int units = p.max_tiles * p.num_kv_heads;
-    e = launch_pdl(prefill_score_kernel, dim3(units), dim3(kScoreThreads), 0, s, p);
+    switch (p.fmt) {
+        case SPOT_SEL_BF16:
+            e = launch_pdl(prefill_score_kernel, dim3(units), dim3(kScoreThreads), 0, s, p);
+            break;
+        case SPOT_SEL_INT4_G32_F16:
+            e = launch_pdl(prefill_score_q_kernel<SPOT_SEL_INT4_G32_F16>, dim3(units),
+                           dim3(kScoreThreads), 0, s, p);
+            break;
+        case SPOT_SEL_MXFP4_G32_E8M0:
+            e = launch_pdl(prefill_score_q_kernel<SPOT_SEL_MXFP4_G32_E8M0>, dim3(units),
+                           dim3(kScoreThreads), 0, s, p);
+            break;
+        case SPOT_SEL_FP8_E4M3:
+            e = launch_pdl(prefill_score_q_kernel<SPOT_SEL_FP8_E4M3>, dim3(units),
+                           dim3(kScoreThreads), 0, s, p);
+            break;
+        case SPOT_SEL_INT8_F16:
+            e = launch_pdl(prefill_score_q_kernel<SPOT_SEL_INT8_F16>, dim3(units),
+                           dim3(kScoreThreads), 0, s, p);
+            break;
+        default: return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
     // selection on the tile scores: one unit per (tile, KV head)
     SelectParams sl = {};

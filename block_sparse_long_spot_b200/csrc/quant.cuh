@@ -82,6 +82,101 @@ __device__ __forceinline__ float fp8_value(uint32_t code) {
     return __half2float(__half(h));
 }
 
+// ---- block-key selector scoring (shared by the decode selection and the
+// sparse-prefill tile scores): per-key scale groups and the selector-query
+// layout the tensor-core tiles consume
+
+// Scale of group grp (dims 32 grp .. + 31) of 64-element key row `row`.
+template <int FMT>
+__device__ __forceinline__ float group_scale(const void* scales, int64_t row, int grp) {
+    if (FMT == SPOT_SEL_INT4_G32_F16) {
+        const __half h = reinterpret_cast<const __half*>(scales)[row * 2 + grp];
+        return __half2float(h);
+    } else {
+        const uint32_t e = reinterpret_cast<const uint8_t*>(scales)[row * 2 + grp];
+        if (e == 255u) return __int_as_float(0x7fc00000);          // NaN
+        if (e == 0u) return __int_as_float(0x00400000);            // 2^-127
+        return __int_as_float(static_cast<int>(e << 23));          // 2^(e-127)
+    }
+}
+
+// Quantises this lane's 16 query elements f (two halves of 8, see
+// load_queries) with the key format's rule and replaces them by their codes'
+// values (exact in bf16).  qs[h]: the scale of half h, the query head's
+// group scale for the 4-bit formats (half 0 lies in dims 0-31, half 1 in
+// dims 32-63) and its per-head scale for INT8; 1 for FP8.  The four lanes of
+// a quad (same r8) hold one query head between them.
+template <int FMT>
+__device__ __forceinline__ void quantize_query(float (&f)[16], float (&qs)[2]) {
+    if (FMT == SPOT_SEL_FP8_E4M3) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) f[i] = fp8_value(fp8_code(f[i]));
+        qs[0] = qs[1] = 1.f;
+        return;
+    }
+    float am[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) am[i >> 3] = fmaxf(am[i >> 3], fabsf(f[i]));
+    if (FMT == SPOT_SEL_INT8_F16) am[0] = am[1] = fmaxf(am[0], am[1]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        am[h] = fmaxf(am[h], __shfl_xor_sync(0xffffffffu, am[h], 1));
+        am[h] = fmaxf(am[h], __shfl_xor_sync(0xffffffffu, am[h], 2));
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (FMT == SPOT_SEL_MXFP4_G32_E8M0) {
+            const int X = mx_exponent(am[h]);
+#pragma unroll
+            for (int i = 8 * h; i < 8 * h + 8; ++i) f[i] = e2m1_value(mx_code(f[i], X));
+            qs[h] = ldexpf(1.f, X);
+        } else {
+            const bool i8 = FMT == SPOT_SEL_INT8_F16;
+            const float sc = f16_bits_value(f16_scale_bits(am[h], i8 ? 127.0 : 7.0));
+#pragma unroll
+            for (int i = 8 * h; i < 8 * h + 8; ++i)
+                f[i] = static_cast<float>(int_code(f[i], sc, i8 ? -128 : -8, i8 ? 127 : 7));
+            qs[h] = sc;
+        }
+    }
+}
+
+// The lane's 16 elements of one selector query row (64 dims) in the order
+// the block-key tiles consume the head dimension, as 8 bf16 pairs: bf16 /
+// 8-bit keys: dims [16 c4, 16 c4 + 16); 4-bit keys: dims [8 c4, 8 c4 + 8)
+// and [32 + 8 c4, 32 + 8 c4 + 8).  With `quantize` (quantised formats) the
+// elements become their codes' values and qs[half] the half's scale
+// (quantize_query), else qs = 1.  Every lane of the warp takes part (the
+// four lanes of a quad hold one row).
+template <int FMT>
+__device__ __forceinline__ void selector_query_words(const uint16_t* qrow, int c4, bool real,
+                                                     bool quantize, uint32_t (&qw)[8],
+                                                     float (&qs)[2]) {
+    const uint4* q4 = reinterpret_cast<const uint4*>(qrow);
+    uint4 x0, x1;
+    if (FMT == SPOT_SEL_BF16 || FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
+        x0 = real ? __ldg(q4 + 2 * c4) : make_uint4(0, 0, 0, 0);
+        x1 = real ? __ldg(q4 + 2 * c4 + 1) : make_uint4(0, 0, 0, 0);
+    } else {
+        x0 = real ? __ldg(q4 + c4) : make_uint4(0, 0, 0, 0);
+        x1 = real ? __ldg(q4 + 4 + c4) : make_uint4(0, 0, 0, 0);
+    }
+    qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
+    qw[4] = x1.x; qw[5] = x1.y; qw[6] = x1.z; qw[7] = x1.w;
+    qs[0] = qs[1] = 1.f;
+    if (FMT != SPOT_SEL_BF16 && quantize) {
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[2 * i] = __uint_as_float(qw[i] << 16);
+            f[2 * i + 1] = __uint_as_float(qw[i] & 0xFFFF0000u);
+        }
+        quantize_query<FMT>(f, qs);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qw[i] = pack_bf16(f[2 * i], f[2 * i + 1]);
+    }
+}
+
 // ---- code -> bf16 widening for the tensor-core scoring paths (every INT4,
 // E2M1, INT8 and E4M3 value is exact in bf16; scales are applied after the
 // mma)

@@ -51,20 +51,6 @@ constexpr int kTileBatch = 4;           // 16-block tiles a warp scores with loa
 
 // --------------------------------------------------------------- scoring
 
-template <int FMT>
-__device__ __forceinline__ float group_scale(const void* scales, int64_t row, int grp) {
-    if (FMT == SPOT_SEL_INT4_G32_F16) {
-        const __half h = reinterpret_cast<const __half*>(scales)[row * 2 + grp];
-        return __half2float(h);
-    } else {
-        const uint32_t e = reinterpret_cast<const uint8_t*>(scales)[row * 2 + grp];
-        if (e == 255u) return __int_as_float(0x7fc00000);          // NaN
-        if (e == 0u) return __int_as_float(0x00400000);            // 2^-127
-        return __int_as_float(static_cast<int>(e << 23));          // 2^(e-127)
-    }
-}
-
-
 // Scores of tiles t0, t0 + stride, ... (kTileBatch of them) of 16 blocks
 // each, for KV head g, into scores[j] (j < n_full), given the blocks' page
 // ids (load_pages).  qw: the group's selector queries as mma B fragments
@@ -209,47 +195,6 @@ __device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
     }
 }
 
-// Quantises this lane's 16 query elements f (two halves of 8, see
-// load_queries) with the key format's rule and replaces them by their codes'
-// values (exact in bf16).  qs[h]: the scale of half h, the query head's
-// group scale for the 4-bit formats (half 0 lies in dims 0-31, half 1 in
-// dims 32-63) and its per-head scale for INT8; 1 for FP8.  The four lanes of
-// a quad (same r8) hold one query head between them.
-template <int FMT>
-__device__ __forceinline__ void quantize_query(float (&f)[16], float (&qs)[2]) {
-    if (FMT == SPOT_SEL_FP8_E4M3) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) f[i] = fp8_value(fp8_code(f[i]));
-        qs[0] = qs[1] = 1.f;
-        return;
-    }
-    float am[2] = {0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) am[i >> 3] = fmaxf(am[i >> 3], fabsf(f[i]));
-    if (FMT == SPOT_SEL_INT8_F16) am[0] = am[1] = fmaxf(am[0], am[1]);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        am[h] = fmaxf(am[h], __shfl_xor_sync(0xffffffffu, am[h], 1));
-        am[h] = fmaxf(am[h], __shfl_xor_sync(0xffffffffu, am[h], 2));
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        if (FMT == SPOT_SEL_MXFP4_G32_E8M0) {
-            const int X = mx_exponent(am[h]);
-#pragma unroll
-            for (int i = 8 * h; i < 8 * h + 8; ++i) f[i] = e2m1_value(mx_code(f[i], X));
-            qs[h] = ldexpf(1.f, X);
-        } else {
-            const bool i8 = FMT == SPOT_SEL_INT8_F16;
-            const float sc = f16_bits_value(f16_scale_bits(am[h], i8 ? 127.0 : 7.0));
-#pragma unroll
-            for (int i = 8 * h; i < 8 * h + 8; ++i)
-                f[i] = static_cast<float>(int_code(f[i], sc, i8 ? -128 : -8, i8 ? 127 : 7));
-            qs[h] = sc;
-        }
-    }
-}
-
 // Selector queries of head group g as mma B fragments (lane: head r8), the
 // weights of heads 2 c4, 2 c4 + 1, and the query scales of those two heads
 // qsc[half][column] (all 1 unless the queries are quantised).
@@ -261,39 +206,15 @@ __device__ __forceinline__ void load_queries(const SelectParams& p, int b, int g
     const int G = p.group;
     const bool real = r8 < G;
     const int h = g * G + (real ? r8 : 0);
-    const uint4* qrow = reinterpret_cast<const uint4*>(
-        p.q_sel + (static_cast<int64_t>(b) * p.num_q_heads + h) * kSelDim);
-    // bf16 / 8-bit keys: lane c4 owns dims [16 c4, 16 c4 + 16);
-    // 4-bit keys: dims [8 c4, 8 c4 + 8) and [32 + 8 c4, 32 + 8 c4 + 8).
-    uint4 x0, x1;
-    if (FMT == SPOT_SEL_BF16 || FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
-        x0 = real ? __ldg(qrow + 2 * c4) : make_uint4(0, 0, 0, 0);
-        x1 = real ? __ldg(qrow + 2 * c4 + 1) : make_uint4(0, 0, 0, 0);
-    } else {
-        x0 = real ? __ldg(qrow + c4) : make_uint4(0, 0, 0, 0);
-        x1 = real ? __ldg(qrow + 4 + c4) : make_uint4(0, 0, 0, 0);
-    }
-    qw[0] = x0.x; qw[1] = x0.y; qw[2] = x0.z; qw[3] = x0.w;
-    qw[4] = x1.x; qw[5] = x1.y; qw[6] = x1.z; qw[7] = x1.w;
-    qsc[0][0] = qsc[0][1] = qsc[1][0] = qsc[1][1] = 1.f;
-    if (FMT != SPOT_SEL_BF16 && p.quantize_queries) {
-        float f[16];
+    const uint16_t* qrow = p.q_sel + (static_cast<int64_t>(b) * p.num_q_heads + h) * kSelDim;
+    float qs[2];
+    selector_query_words<FMT>(qrow, c4, real, FMT != SPOT_SEL_BF16 && p.quantize_queries, qw, qs);
+    // column 0 / 1 of this lane's accumulators = heads 2 c4 / 2 c4 + 1,
+    // whose scales sit in lanes 4 * (2 c4) and 4 * (2 c4 + 1)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            f[2 * i] = __uint_as_float(qw[i] << 16);
-            f[2 * i + 1] = __uint_as_float(qw[i] & 0xFFFF0000u);
-        }
-        float qs[2];
-        quantize_query<FMT>(f, qs);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qw[i] = pack_bf16(f[2 * i], f[2 * i + 1]);
-        // column 0 / 1 of this lane's accumulators = heads 2 c4 / 2 c4 + 1,
-        // whose scales sit in lanes 4 * (2 c4) and 4 * (2 c4 + 1)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            qsc[hf][0] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4);
-            qsc[hf][1] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4 + 4);
-        }
+    for (int hf = 0; hf < 2; ++hf) {
+        qsc[hf][0] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4);
+        qsc[hf][1] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4 + 4);
     }
     const int64_t wrow = static_cast<int64_t>(b) * p.num_q_heads + g * G;
     wh0 = (2 * c4 < G) ? (p.w ? p.w[wrow + 2 * c4] : 1.f / G) : 0.f;

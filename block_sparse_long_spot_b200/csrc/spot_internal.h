@@ -148,7 +148,10 @@ struct PrefillParams {
     float* tile_p;                      // [max_tiles]
     const int32_t* page_table;
     int32_t pt_stride, num_pages, num_q_heads, num_kv_heads, group, max_blocks;
-    const void* sel_data;               // bf16 selector keys [num_pages][Hkv][64]
+    const void* sel_data;               // selector keys [num_pages][Hkv] rows in `fmt`
+    const void* sel_scales;             // their scales (INT4 / MXFP4 / INT8), else null
+    int32_t fmt;                        // spot_sel_fmt_t of the selector keys
+    int32_t quantize_queries;           // quantise q_sel with the key format's rule
     const uint16_t* q_sel;              // [rows][Hq][64]
     const float* w;                     // [rows][Hq] or null
     float inv_temp;

@@ -339,7 +339,10 @@ spot_status_t spot_tok_decode_step(const spot_tok_layer_desc_t* desc,
  * tile's last position would keep (same parameters, Eq. 6-8), scored by the
  * maximum over the tile's queries of (1/tau) sum_h w_h ReLU(q_sel_h . k);
  * every query attends to the keys of its tile's selection at positions up
- * to its own.  bf16 selector keys; quantize_queries must be 0.
+ * to its own.  The selector keys may be in any spot_sel_fmt_t (sel_scales as
+ * for spot_select: NULL for bf16 / FP8, 16-byte aligned otherwise), and with
+ * quantize_queries each query head's selector query is quantised with the
+ * key format's rule, as in spot_select.
  *
  * Layouts:
  *   q_sel   bf16 [rows][num_q_heads][sel_dim]     w fp32 [rows][num_q_heads] or NULL
@@ -363,6 +366,7 @@ size_t spot_prefill_workspace_size(const spot_layer_desc_t* desc, int32_t batch,
 
 spot_status_t spot_prefill(const spot_layer_desc_t* desc, const spot_select_params_t* params,
                            const uint16_t* q_sel, const float* w, const void* sel_data,
+                           const void* sel_scales,
                            const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
                            const int32_t* page_table, int32_t pt_stride,
                            const int32_t* seq_lens, const int32_t* q_lens, const float* top_p,

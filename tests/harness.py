@@ -35,9 +35,11 @@ def gpu_selector_pool(wl, fmt, device):
     ptn = pt.cpu().numpy()
     for b in range(wl.batch):
         nb = int(lens[b]) // 64               # complete blocks carry keys
-        seq_ids += [b] * nb
-        blk_ids += list(range(nb))
-        pages += ptn[b, :nb].tolist()
+        for j in range(nb):
+            if 0 <= ptn[b, j] < wl.num_pages:   # a test may corrupt an entry on purpose
+                seq_ids.append(b)
+                blk_ids.append(j)
+                pages.append(int(ptn[b, j]))
     if seq_ids:
         keys = wl.sel_keys[torch.as_tensor(pages, device=device).long()].contiguous()
         desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, fmt)
@@ -392,21 +394,24 @@ def _pf_sel(spec, kmin, sink, rec):
 
 
 def run_gpu_prefill(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None, temperature=1.0,
-                    max_tiles=None):
+                    max_tiles=None, fmt="bf16", quantize_queries=False):
     dev = wl.q.device
     Hq, Hkv, mb = wl.num_q_heads, wl.num_kv_heads, wl.max_blocks
     kmin, sink, rec = _pf_sel(wl.spec, kmin, sink, rec)
     nt = spot.prefill_num_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
     mt = max(nt, 1) if max_tiles is None else max_tiles
-    desc = spot.layer_desc(Hq, Hkv, wl.num_pages, "bf16")
-    prm = spot.select_params(mode, sink, rec, kmin, topk, temperature)
+    desc = spot.layer_desc(Hq, Hkv, wl.num_pages, fmt)
+    prm = spot.select_params(mode, sink, rec, kmin, topk, temperature, quantize_queries)
+    # bf16 keys as they are (a test may corrupt the page table on purpose, so
+    # nothing here gathers through it); other formats through the append
+    data, scales = (wl.sel_keys, None) if fmt == "bf16" else gpu_selector_pool(wl, fmt, dev)
     ws = spot.new_prefill_workspace(desc, wl.batch, mt, mb, dev)
     rows = int(wl.q.shape[0])
     sel_idx = torch.full((mt, Hkv, mb), -1, dtype=torch.int32, device=dev)
     sel_cnt = torch.full((mt, Hkv), -1, dtype=torch.int32, device=dev)
     out = torch.full((max(rows, 1), Hq, 128), float("nan"), dtype=torch.float32, device=dev)
     lse = torch.full((max(rows, 1), Hq), float("nan"), dtype=torch.float32, device=dev)
-    spot.prefill(desc, prm, wl.q_sel, wl.w, wl.sel_keys, wl.q, wl.k_pool, wl.v_pool,
+    spot.prefill(desc, prm, wl.q_sel, wl.w, data, scales, wl.q, wl.k_pool, wl.v_pool,
                  wl.page_table, wl.seq_lens, wl.q_lens, wl.top_p, wl.sm_scale, sel_idx, sel_cnt,
                  out, lse, ws)
     torch.cuda.synchronize()
@@ -416,9 +421,10 @@ def run_gpu_prefill(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None, tem
             "status": status, "num_tiles": nt}
 
 
-def prefill_oracle_args(wl):
+def prefill_oracle_args(wl, fmt="bf16"):
+    data, scales = oracle_selector_pool(wl, fmt)
     return dict(q_sel=workloads.bits(wl.q_sel), w=host_bytes(wl.w),
-                sel_data=workloads.bits(wl.sel_keys), sel_scales=None, q=workloads.bits(wl.q),
+                sel_data=data, sel_scales=scales, q=workloads.bits(wl.q),
                 k_pool=workloads.bits(wl.k_pool), v_pool=workloads.bits(wl.v_pool),
                 page_table=wl.page_table.cpu().numpy(), seq_lens=wl.seq_lens.cpu().numpy(),
                 q_lens=wl.q_lens.cpu().numpy(), top_p=wl.top_p.cpu().numpy(),
@@ -426,22 +432,23 @@ def prefill_oracle_args(wl):
 
 
 def prefill_shape_params(wl, mode="topp", kmin=None, topk=0, sink=None, rec=None,
-                         temperature=1.0):
+                         temperature=1.0, fmt="bf16", quantize_queries=False):
     kmin, sink, rec = _pf_sel(wl.spec, kmin, sink, rec)
-    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, "bf16",
+    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, fmt,
                            wl.num_pages, wl.max_blocks)
-    return sh, oracle.make_params(mode, sink, rec, kmin, topk, temperature)
+    return sh, oracle.make_params(mode, sink, rec, kmin, topk, temperature, quantize_queries)
 
 
 def run_oracle_prefill(wl, tiles=None, args=None, **kw):
     sh, pr = prefill_shape_params(wl, **kw)
-    return oracle.prefill_step(sh, pr, tiles=tiles, **(args or prefill_oracle_args(wl)))
+    return oracle.prefill_step(sh, pr, tiles=tiles,
+                               **(args or prefill_oracle_args(wl, kw.get("fmt", "bf16"))))
 
 
 def oracle_prefill_scores(wl, tiles=None, args=None, **kw):
     sh, pr = prefill_shape_params(wl, **kw)
-    a = args or prefill_oracle_args(wl)
-    return oracle.prefill_scores(sh, pr, a["q_sel"], a["w"], a["sel_data"], None,
+    a = args or prefill_oracle_args(wl, kw.get("fmt", "bf16"))
+    return oracle.prefill_scores(sh, pr, a["q_sel"], a["w"], a["sel_data"], a["sel_scales"],
                                  a["page_table"], a["seq_lens"], a["q_lens"], tiles=tiles)
 
 

@@ -120,3 +120,34 @@ def test_prefill_bad_page_id_and_small_max_tiles_are_reported():
     wl = workloads.make_prefill("prefill_tiny", seed=6, device=DEV)
     gpu = run_gpu_prefill(wl, max_tiles=2)
     assert gpu["status"] == 5
+
+
+# ------------------------------------------------ quantised selector keys / queries
+
+@pytest.mark.parametrize("fmt,qq", [("mxfp4", False), ("fp8", False), ("mxfp4", True),
+                                    ("fp8", True)])
+def test_prefill_quantised_keys_integer_inputs_select_bit_exact(fmt, qq):
+    # selector queries and keys in {-3..3}: MXFP4 and E4M3 store them
+    # losslessly, so every tile score is exact on both sides
+    wl = workloads.make_prefill("prefill_tiny", seed=7, device=DEV, integer=True,
+                                seq_lens=[1000, 300], q_lens=[300, 300])
+    wl.top_p = safe_top_p_prefill(wl, fmt=fmt, quantize_queries=qq)
+    gpu = run_gpu_prefill(wl, fmt=fmt, quantize_queries=qq)
+    assert gpu["status"] == 0
+    ora = run_oracle_prefill(wl, fmt=fmt, quantize_queries=qq)
+    _same(gpu, ora, wl)
+    check_prefill_outputs(gpu, ora, wl)
+
+
+@pytest.mark.parametrize("fmt,qq", [("int4", False), ("mxfp4", False), ("fp8", False),
+                                    ("int8", False), ("int4", True), ("int8", True)])
+def test_prefill_quantised_keys_tiny(fmt, qq):
+    wl = workloads.make_prefill("prefill_tiny", seed=8, device=DEV)
+    gpu = run_gpu_prefill(wl, fmt=fmt, quantize_queries=qq)
+    assert gpu["status"] == 0
+    args = prefill_oracle_args(wl, fmt)
+    ora = run_oracle_prefill(wl, args=args, fmt=fmt, quantize_queries=qq)
+    scores = oracle_prefill_scores(wl, args=args, fmt=fmt, quantize_queries=qq)
+    assert check_prefill_selection_near_cut(gpu, ora, scores, wl) <= 1
+    _, n = check_prefill_outputs(gpu, ora, wl)
+    assert n >= gpu["num_tiles"] * wl.num_kv_heads - 1
