@@ -726,6 +726,27 @@ def prefill_flops(wl, sel_idx: np.ndarray, sel_cnt: np.ndarray):
     return attn, score
 
 
+def block_pool(spot, wl, desc, fmt):
+    """A layer's per-block selector pool in `fmt`: the workload's bf16 keys as
+    they are, or written through the library's quantising append (every
+    complete block of every sequence)."""
+    if fmt == "bf16":
+        return wl.sel_keys, None
+    dev = wl.q.device
+    data, scales = spot.selector_pool(fmt, wl.num_pages, wl.num_kv_heads, device=dev)
+    lens = wl.seq_lens.cpu().numpy()
+    pt = wl.page_table.cpu().numpy()
+    seq = np.concatenate([np.full(int(L) // 64, b) for b, L in enumerate(lens)]).astype(np.int32)
+    blk = np.concatenate([np.arange(int(L) // 64) for L in lens]).astype(np.int32)
+    if seq.size:
+        keys = wl.sel_keys[torch.as_tensor(pt[seq, blk].astype(np.int64), device=dev)].contiguous()
+        spot.append_selector_keys(desc, data, scales, wl.page_table,
+                                  torch.as_tensor(seq, device=dev), torch.as_tensor(blk, device=dev),
+                                  keys)
+    torch.cuda.synchronize()
+    return data, scales
+
+
 def run_spot_prefill(args, world, rank, local):
     """One sparse-prefill layer (plan, tile scoring, selection, attention)
     per step over the whole chunk."""
@@ -738,7 +759,9 @@ def run_spot_prefill(args, world, rank, local):
     sp = wl0.spec
     Hq, Hkv, mb = wl0.num_q_heads, wl0.num_kv_heads, wl0.max_blocks
     nt = spot.prefill_num_tiles(wl0.seq_lens.cpu().numpy(), wl0.q_lens.cpu().numpy())
-    descs = [spot.layer_desc(Hq, Hkv, w.num_pages, "bf16") for w in layers]
+    fmt = args.sel_fmt
+    descs = [spot.layer_desc(Hq, Hkv, w.num_pages, fmt) for w in layers]
+    pools = [block_pool(spot, w, d, fmt) for w, d in zip(layers, descs)]
     prm = spot.select_params("topp", sp.sink_blocks, sp.recency_blocks, sp.kmin_blocks)
     wss = [spot.new_prefill_workspace(d, wl0.batch, nt, mb, dev) for d in descs]
     rows = int(wl0.q.shape[0])
@@ -750,8 +773,9 @@ def run_spot_prefill(args, world, rank, local):
 
     def step(i, q=None, q_sel=None, o=None):
         w = layers[i % len(layers)]
+        sd, ss = pools[i % len(layers)]
         spot.prefill(descs[i % len(layers)], prm, w.q_sel if q_sel is None else q_sel, w.w,
-                     w.sel_keys, None, w.q if q is None else q, w.k_pool, w.v_pool, w.page_table,
+                     sd, ss, w.q if q is None else q, w.k_pool, w.v_pool, w.page_table,
                      w.seq_lens, w.q_lens, w.top_p, w.sm_scale, sel_idx, sel_cnt,
                      out if o is None else o, lse, wss[i % len(layers)], stream)
 
@@ -810,6 +834,7 @@ def run_spot_prefill(args, world, rank, local):
         "config": {"workload": args.workload, "batch_per_gpu": wl0.batch, "q_heads": Hq,
                    "kv_heads": Hkv, "head_dim": 128, "context": int(wl0.seq_lens.max().item()),
                    "chunk": int(wl0.q_lens.max().item()), "tiles": nt, "block": 64,
+                   "sel_fmt": fmt,
                    "top_p": sp.top_p, "sink_blocks": sp.sink_blocks,
                    "recency_blocks": sp.recency_blocks, "kmin_blocks": sp.kmin_blocks,
                    "layers_in_model": sp_layers(args), "layer_caches_rotated": nl,
@@ -833,7 +858,7 @@ def run_spot_prefill(args, world, rank, local):
     }, (layers, sel0[0], sel0[1])
 
 
-def cpu_baseline_prefill(wl, sel_idx, sel_cnt, layers_model):
+def cpu_baseline_prefill(wl, sel_idx, sel_cnt, layers_model, fmt="bf16"):
     """The fp64 oracle's sparse prefill on the host cores for two tiles (the
     last and a middle one, all KV heads), scaled to the layer by the share of
     the layer's attention FLOPs those tiles hold, then to the model."""
@@ -841,13 +866,15 @@ def cpu_baseline_prefill(wl, sel_idx, sel_cnt, layers_model):
     info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
     nt = len(info)
     tiles = [nt - 1, nt // 2]
-    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, "bf16",
+    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, fmt,
                            wl.num_pages, wl.max_blocks)
     sp = wl.spec
     pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
                             kmin_blocks=sp.kmin_blocks)
-    args = dict(q_sel=workloads.bits(wl.q_sel), w=None, sel_data=workloads.bits(wl.sel_keys),
-                sel_scales=None, q=workloads.bits(wl.q), k_pool=workloads.bits(wl.k_pool),
+    bits = workloads.bits(wl.sel_keys)
+    sd, ss = (bits, None) if fmt == "bf16" else oracle.quantize_selector(fmt, bits)
+    args = dict(q_sel=workloads.bits(wl.q_sel), w=None, sel_data=sd,
+                sel_scales=ss, q=workloads.bits(wl.q), k_pool=workloads.bits(wl.k_pool),
                 v_pool=workloads.bits(wl.v_pool), page_table=wl.page_table.cpu().numpy(),
                 seq_lens=wl.seq_lens.cpu().numpy(), q_lens=wl.q_lens.cpu().numpy(),
                 top_p=wl.top_p.cpu().numpy(), sm_scale=wl.sm_scale)
@@ -1043,7 +1070,7 @@ def main():
             if world == 1 and not args.no_cpu_baseline:
                 if pf:
                     res["cpu_baseline"] = cpu_baseline_prefill(layers[0][0], layers[1], layers[2],
-                                                               sp_layers(args))
+                                                               sp_layers(args), args.sel_fmt)
                 else:
                     res["cpu_baseline"] = (cpu_baseline_tok(layers[0][0], args.sel_fmt) if tok else
                                            cpu_baseline(layers[0][0], args.sel_fmt))

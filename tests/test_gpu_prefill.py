@@ -151,3 +151,21 @@ def test_prefill_quantised_keys_tiny(fmt, qq):
     assert check_prefill_selection_near_cut(gpu, ora, scores, wl) <= 1
     _, n = check_prefill_outputs(gpu, ora, wl)
     assert n >= gpu["num_tiles"] * wl.num_kv_heads - 1
+
+
+def test_prefill_full_size_int4_keys_sampled_tiles():
+    """The 32K-token prefill with INT4 selector keys (written by the library's
+    quantising append) in the benchmark's launch configuration: selection and
+    outputs of sampled tiles against the oracle on the same codes."""
+    wl = workloads.make_prefill("qwen3_8b_prefill_32k", seed=4, device=DEV)
+    gpu = run_gpu_prefill(wl, fmt="int4")
+    assert gpu["status"] == 0
+    nt = gpu["num_tiles"]
+    tiles = [1, nt // 3, nt - 1]
+    args = prefill_oracle_args(wl, "int4")
+    ora = run_oracle_prefill(wl, tiles=tiles, args=args, fmt="int4")
+    scores = oracle_prefill_scores(wl, tiles=tiles, args=args, fmt="int4")
+    n_diff = check_prefill_selection_near_cut(gpu, ora, scores, wl, tiles=tiles)
+    assert n_diff <= 1
+    _, n = check_prefill_outputs(gpu, ora, wl, tiles=tiles)
+    assert n >= len(tiles) * wl.num_kv_heads - n_diff
