@@ -1035,6 +1035,59 @@ def run_reference_tok(args, world, rank):
     }
 
 
+def run_reference_prefill(args, world, rank):
+    """Reference arm for the sparse-prefill workloads: the fp64 oracle's
+    prefill on the host cores, one tile (all KV heads) per step at tiles
+    spread evenly over the chunk (at most 8 timed tiles, so the run stays
+    bounded); the layer time is the mean tile time x the layer's tiles."""
+    if rank != 0:
+        return None
+    import oracle
+    wl = workloads.make_prefill(args.workload, seed=0, device="cpu")
+    fmt = args.sel_fmt
+    sp = wl.spec
+    lens, ql = wl.seq_lens.numpy(), wl.q_lens.numpy()
+    nt = len(oracle.prefill_tiles(lens, ql))
+    sh = oracle.make_shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, 128, 64, 64, fmt,
+                           wl.num_pages, wl.max_blocks)
+    pr = oracle.make_params(sink_blocks=sp.sink_blocks, recency_blocks=sp.recency_blocks,
+                            kmin_blocks=sp.kmin_blocks)
+    bits = workloads.bits(wl.sel_keys)
+    sd, ss = (bits, None) if fmt == "bf16" else oracle.quantize_selector(fmt, bits)
+    a = dict(q_sel=workloads.bits(wl.q_sel), w=None, sel_data=sd, sel_scales=ss,
+             q=workloads.bits(wl.q), k_pool=workloads.bits(wl.k_pool),
+             v_pool=workloads.bits(wl.v_pool), page_table=wl.page_table.numpy(), seq_lens=lens,
+             q_lens=ql, top_p=wl.top_p.numpy(), sm_scale=wl.sm_scale)
+    n = min(args.steps, 8)
+    strata = [int((k + 0.5) * nt / n) for k in range(n)]
+    for _ in range(args.warmup):                  # warm-up on the chunk's first (cheapest) tile
+        oracle.prefill_step(sh, pr, tiles=[0], **a)
+    times = []
+    for t in strata:
+        t0 = time.perf_counter()
+        oracle.prefill_step(sh, pr, tiles=[t], **a)
+        times.append(time.perf_counter() - t0)
+    layer_s = float(np.mean(times)) * nt
+    tokens = int(ql.sum())
+    layers_model = sp_layers(args)
+    value = tokens / (layer_s * layers_model)
+    sample = (f"{n} tiles spread over the chunk's {nt} (all KV heads), one per step; "
+              f"mean tile time x {nt} tiles x{layers_model} layers")
+    return {
+        "impl": "reference",
+        "metric": "prefill tokens/s at L=32K (whole model = per-layer time x layers)",
+        "value": round(value, 6), "unit": "tokens/s", "n_gpus": world, "steps": n,
+        "warmup": args.warmup, "ms_per_step": round(layer_s * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 with planted hot blocks)",
+        "config": {"workload": args.workload, "sel_fmt": fmt, "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s",
+                         "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1056,7 +1109,8 @@ def main():
         if args.impl == "reference":
             if world > 1:
                 torch.distributed.barrier()
-            res = (run_reference_tok if tok else run_reference)(args, world, rank)
+            res = (run_reference_tok if tok else
+                   run_reference_prefill if pf else run_reference)(args, world, rank)
             if res is not None:
                 print(json.dumps(res), flush=True)
             return
