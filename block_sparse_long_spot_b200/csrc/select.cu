@@ -47,7 +47,7 @@ namespace {
 
 constexpr int kSelectThreads = 512;
 constexpr int kFixShift = 40;
-constexpr int kTileBatch = 4;           // 16-block tiles a warp scores with loads in flight
+constexpr int kTileBatch = 2;           // 16-block tiles a warp scores with loads in flight
 
 // --------------------------------------------------------------- scoring
 
@@ -549,11 +549,13 @@ __device__ __forceinline__ SelSmem carve_select_smem(uint8_t* smem, int max_bloc
 }
 
 // Selection of unit u (all threads of the CTA) on its block scores: in
-// shared memory already (`in_smem`), else read from p.scores_in.
-__device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, bool in_smem) {
+// shared memory already (`in_smem`), else read from p.scores_in.  L is the
+// sequence's length (>= 0) and pb its top-p (p.top_p[b], 1 without one),
+// both read by the caller ahead of its other work.
+__device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, bool in_smem, int L,
+                            float pb) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = u / p.num_kv_heads;
-    const int L = max(p.seq_lens[b], 0);
     const int bsz = kBlock / p.blocks_per_page;        // tokens per selection block
     int nb = (L + bsz - 1) / bsz;
     int n_full = L / bsz;
@@ -661,14 +663,13 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
         if (p.mode == SPOT_MODE_TOPK) {
             n_take = min(max(p.topk_blocks, 0), n);
         } else {
-            const float pb = p.top_p ? p.top_p[b] : 1.f;
             n_take = pb >= 1.f ? n : (pb <= 0.f ? 0 : -1);
         }
     }
     bool done = false;
     if (n_take < 0) {
         unsigned long long T = static_cast<unsigned long long>(
-            ceil(static_cast<double>(p.top_p[b]) * static_cast<double>(Z)));
+            ceil(static_cast<double>(pb) * static_cast<double>(Z)));
         T = T < 1ull ? 1ull : (T > Z ? Z : T);
         int before;
         if (threadIdx.x == 0) sm.misc[3] = 0;
@@ -801,11 +802,14 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     extern __shared__ __align__(16) uint8_t smem[];
     const SelSmem sm = carve_select_smem(smem, p.max_blocks);
     pdl_wait();                  // the scores (and the lengths and p) may come from it
-    select_unit(p, blockIdx.x, sm, false);
+    const int b = blockIdx.x / p.num_kv_heads;
+    const int L = max(p.seq_lens[b], 0);
+    const float pb = p.top_p ? p.top_p[b] : 1.f;
+    select_unit(p, blockIdx.x, sm, false, L, pb);
 }
 
 // Scoring (§2.1, Eq. 2) and selection in one launch.  The C CTAs of a unit
-// share its 16-block tiles: CTA c takes rounds c, c + C, ... of 64 tiles
+// share its 16-block tiles: CTA c takes rounds c, c + C, ... of NW * kTileBatch tiles
 // (one batch of kTileBatch tiles per warp per round, the next round's page
 // ids loading while this round's keys do).  With C = 1 the scores stay in
 // shared memory and the CTA selects at once; otherwise they go to
@@ -820,6 +824,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
     const int u = blockIdx.x / C, c = blockIdx.x - u * C;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
     const int L = max(p.seq_lens[b], 0);
+    const float pb = p.top_p ? p.top_p[b] : 1.f;                     // for the selection
     const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
     const int n_full = min(L / (kBlock / p.blocks_per_page), cap);   // overflow: flagged
     const int tiles = (n_full + 15) / 16;                            // by the selection
@@ -854,7 +859,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
         if (!sm.misc[7]) return;
         __threadfence();                              // the other CTAs' scores
     }
-    select_unit(p, u, sm, C == 1);
+    select_unit(p, u, sm, C == 1, L, pb);
 }
 
 }  // namespace
@@ -881,7 +886,7 @@ cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     // CTAs per unit: enough to cover the longest sequence in one round of
-    // 64 tiles each, as far as one wave of one CTA per SM allows
+    // NW * kTileBatch tiles each, as far as one wave of one CTA per SM allows
     const int U = p.batch * p.num_kv_heads;
     const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
     const int rounds = max(1, ((cap + 15) / 16 + NW * kTileBatch - 1) / (NW * kTileBatch));
