@@ -113,8 +113,7 @@ bool workspace_layout(const spot_layer_desc_t* d, int batch, int max_blocks, Lay
     off += kStatusBytes;
     L.unit_done = off;
     off += static_cast<size_t>(U) * sizeof(uint32_t);
-    L.sel_done = off;
-    off = round_up(off + static_cast<size_t>(U) * sizeof(uint32_t), 256);
+    off = round_up(off, 256);
     L.partials = off;
     off = round_up(off + static_cast<size_t>(grid + U) * G * kPartialFloatsPerHead * sizeof(float),
                    256);
@@ -171,9 +170,6 @@ spot_status_t do_select(const spot_layer_desc_t* d, const spot_select_params_t* 
     sl.topk_blocks = pr->topk_blocks;
     sl.quantize_queries = pr->quantize_queries;
     sl.blocks_per_page = 1;
-    sl.scores_out = reinterpret_cast<float*>(base + L.scores);
-    sl.scores_in = sl.scores_out;
-    sl.sel_done = reinterpret_cast<uint32_t*>(base + L.sel_done);
     sl.sel_idx = sel_idx;
     sl.sel_cnt = sel_cnt;
     sl.status = reinterpret_cast<uint32_t*>(base + L.status);

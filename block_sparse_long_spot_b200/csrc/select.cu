@@ -1,22 +1,23 @@
 // select.cu -- selector scoring and block selection (SpotAttention §2.1,
-// §2.3 Eq. 6-8): a scoring kernel spread over the whole GPU, then the
-// selection kernel (one CTA per (sequence, KV head)) launched behind it with
+// §2.3 Eq. 6-8) in one launch, for the per-block selector; the same
+// selection also runs alone on scores computed by another kernel (token
+// selector, sparse prefill).  The decode kernel is launched behind it with
 // programmatic dependent launch.
 //
 // Scoring: s[j] = (1/tau) sum_{h in group} w[b,h] ReLU(q_sel[b,h] . k[page(b,j),g])
-//   for every complete block j.  A CTA of 4 warps takes 256 blocks of one
-//   unit; each warp scores tiles of 16 blocks with
-//   bf16 mma.sync (keys as the M operand, the group's selector queries as
-//   N = 8), four tiles at a time so their gathered loads are in flight
-//   together.  INT4 / MXFP4 / INT8 / FP8 E4M3 keys are widened to bf16 in
-//   registers (all these code sets are exact in bf16) and the scales (per 32
-//   for INT4 / MXFP4, per key for INT8) are applied to the accumulators
-//   afterwards, so dequantisation is exact.  With quantize_queries the
-//   group's selector queries are first quantised with the key format's rule
-//   (quant.cuh) and their scales join the keys' after the mma.  The head
-//   dimension is consumed in a permuted order, identical for the keys and the
-//   queries, that lets every lane load 16 contiguous bytes.  The scores go
-//   to the workspace ([unit][block] fp32, read back from L2).
+//   for every complete block j.  The C CTAs of 16 warps of a unit (one
+//   thread-block cluster) split its blocks; each warp scores tiles of 16
+//   blocks with bf16 mma.sync (keys as the M operand, the group's selector
+//   queries as N = 8), kTileBatch tiles at a time so their gathered loads are
+//   in flight together.  INT4 / MXFP4 / INT8 / FP8 E4M3 keys are widened to
+//   bf16 in registers (all these code sets are exact in bf16) and the scales
+//   (per 32 for INT4 / MXFP4, per key for INT8) are applied to the
+//   accumulators afterwards, so dequantisation is exact.  With
+//   quantize_queries the group's selector queries are first quantised with
+//   the key format's rule (quant.cuh) and their scales join the keys' after
+//   the mma.  The head dimension is consumed in a permuted order, identical
+//   for the keys and the queries, that lets every lane load 16 contiguous
+//   bytes.  The scores go into the shared memory of the cluster's first CTA.
 //
 // Selection: residual softmax numerators exp(s - max) are computed in fp64
 //   and held as 2^-40 fixed-point integers (exact, order-independent sums).
@@ -33,6 +34,7 @@
 // The token-level selector and sparse prefill reuse the selection with their
 // block scores computed by tok_select.cu (one unit per sequence, blocks of 16
 // tokens) and prefill.cu (one unit per (query tile, KV head)).
+#include <cooperative_groups.h>
 #include <cuda_fp8.h>
 #include <math.h>
 
@@ -47,6 +49,7 @@ namespace {
 
 constexpr int kSelectThreads = 512;
 constexpr int kFixShift = 40;
+constexpr int kMaxCluster = 8;          // scoring CTAs of one unit (a portable cluster)
 constexpr int kTileBatch = 2;           // 16-block tiles a warp scores with loads in flight
 
 // --------------------------------------------------------------- scoring
@@ -278,74 +281,85 @@ __device__ __forceinline__ void block_sum3(const SelSmem& sm, unsigned long long
     __syncthreads();
 }
 
-// Exclusive prefix over the block of a float (two barriers); *total = sum.
-__device__ __forceinline__ float block_exclusive_scan_f(const SelSmem& sm, float v, float* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    if (lane == 31) sm.fscan[warp] = incl;
-    __syncthreads();
-    float base = 0.f, tot = 0.f;
-    for (int w = 0; w < NW; ++w) {
-        if (w < warp) base += sm.fscan[w];
-        tot += sm.fscan[w];
-    }
-    *total = tot;
-    __syncthreads();
-    return base + incl - v;
-}
-
 // Bucket of the cut, found on the bucket histograms: the first bucket (from
-// the top) where the cumulative value reaches `target`.  by_mass uses the
-// approximate fp32 masses (the caller corrects the result exactly), else the
-// exact counts.  Returns the bucket; *before receives the exact count of
-// elements in the buckets above it (count mode only).
-__device__ int cut_bucket(const SelSmem& sm, double target, bool by_mass, int* before,
+// the top) where the cumulative value reaches `target` (>= 1).  by_mass uses
+// the approximate 2^-18 fixed-point masses (the caller corrects the result
+// exactly; their total stays below 2^31), else the exact counts.  Returns the
+// bucket; *before receives the exact count of the elements in the buckets
+// above it.  Two barriers: the warps' totals, then a lane scan in the one
+// warp whose buckets hold the crossing point.
+__device__ int cut_bucket(const SelSmem& sm, uint32_t target, bool by_mass, int* before,
                           int nbk) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int PER = nbk / NT;
-    float loc = 0.f;
+    uint32_t loc = 0;
     int cnt = 0, last = -1;
     for (int k = 0; k < PER; ++k) {
         const int bkt = threadIdx.x * PER + k;
-        loc += static_cast<float>(by_mass ? sm.hmass[bkt] : sm.hcnt[bkt]);
-        cnt += sm.hcnt[bkt];
-        if (sm.hcnt[bkt]) last = bkt;
+        const uint32_t c = sm.hcnt[bkt];
+        loc += by_mass ? sm.hmass[bkt] : c;
+        cnt += static_cast<int>(c);
+        if (c) last = bkt;
     }
-    if (threadIdx.x == 0) { sm.misc[0] = -1; sm.misc[1] = -1; }
-    int ctot;
-    const int cbase = block_exclusive_scan<NT>(cnt, sm.scan, &ctot);
-    float ftot;
-    const float fbase = block_exclusive_scan_f(sm, loc, &ftot);
-    // the thread whose buckets hold the crossing point records it
-    float run = fbase;
-    int crun = cbase;
-    for (int k = 0; k < PER; ++k) {
-        const int bkt = threadIdx.x * PER + k;
-        const float v = static_cast<float>(by_mass ? sm.hmass[bkt] : sm.hcnt[bkt]);
-        const bool hit = by_mass ? (run < target && run + v >= target)
-                                 : (crun < target && crun + static_cast<int>(sm.hcnt[bkt]) >= target);
-        if (hit && sm.hcnt[bkt]) {
-            sm.misc[0] = bkt;
-            sm.misc[2] = crun;
+    const uint32_t wv = warp_sum(loc);
+    const int wc = warp_sum(cnt);
+    int wl = last;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wl = max(wl, __shfl_xor_sync(0xffffffffu, wl, o));
+    int* wtot = reinterpret_cast<int*>(sm.red);        // [NW] values, counts, last buckets
+    if (lane == 0) {
+        wtot[warp] = static_cast<int>(wv);
+        wtot[NW + warp] = wc;
+        wtot[2 * NW + warp] = wl;
+    }
+    __syncthreads();
+    // every thread finds the warp whose buckets reach the target
+    uint32_t run = 0;
+    int crun = 0, cw = -1, ctot = 0, lastb = -1;
+    for (int w = 0; w < NW; ++w) {
+        const uint32_t v = static_cast<uint32_t>(wtot[w]);
+        const int c = wtot[NW + w];
+        if (cw < 0) {
+            if (run + v >= target) cw = w;
+            else { run += v; crun += c; }
         }
-        run += v;
-        crun += sm.hcnt[bkt];
+        ctot += c;
+        lastb = max(lastb, wtot[2 * NW + w]);
     }
-    if (last >= 0) atomicMax(&sm.misc[1], last);
-    __syncthreads();
-    int b = sm.misc[0];
-    int bef = sm.misc[2];
-    if (b < 0) {            // fp32 rounding kept the total below the target
-        b = sm.misc[1];
-        bef = ctot - static_cast<int>(sm.hcnt[b]);
+    if (warp == cw) {                                 // warp-uniform
+        uint32_t incl = loc;
+        int cincl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+            const int y = __shfl_up_sync(0xffffffffu, cincl, o);
+            if (lane >= o) { incl += x; cincl += y; }
+        }
+        uint32_t r = run + incl - loc;
+        int cr = crun + cincl - cnt;
+        if (r < target && r + loc >= target) {        // one lane
+            for (int k = 0; k < PER; ++k) {
+                const int bkt = threadIdx.x * PER + k;
+                const uint32_t c = sm.hcnt[bkt];
+                const uint32_t v = by_mass ? sm.hmass[bkt] : c;
+                if (c && r + v >= target) {
+                    sm.misc[0] = bkt;
+                    sm.misc[2] = cr;
+                    break;
+                }
+                r += v;
+                cr += static_cast<int>(c);
+            }
+        }
     }
-    *before = bef;
     __syncthreads();
-    return b;
+    if (cw >= 0) {
+        *before = sm.misc[2];
+        return sm.misc[0];
+    }
+    // the rounded masses stayed below the target: the lowest non-empty bucket
+    *before = ctot - static_cast<int>(sm.hcnt[lastb]);
+    return lastb;
 }
 
 struct Cut {
@@ -555,7 +569,6 @@ __device__ __forceinline__ SelSmem carve_select_smem(uint8_t* smem, int max_bloc
 __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, bool in_smem, int L,
                             float pb) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int b = u / p.num_kv_heads;
     const int bsz = kBlock / p.blocks_per_page;        // tokens per selection block
     int nb = (L + bsz - 1) / bsz;
     int n_full = L / bsz;
@@ -673,8 +686,8 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
         T = T < 1ull ? 1ull : (T > Z ? Z : T);
         int before;
         if (threadIdx.x == 0) sm.misc[3] = 0;
-        int bk = cut_bucket(sm, ldexp(static_cast<double>(T), kApproxShift - kFixShift), true,
-                            &before, nbk);
+        const double tq = ceil(ldexp(static_cast<double>(T), kApproxShift - kFixShift));
+        int bk = cut_bucket(sm, tq < 1.0 ? 1u : static_cast<uint32_t>(tq), true, &before, nbk);
         // Exact check of the bucket on the fixed-point masses.  The first
         // pass also writes the keep flags and gathers the bucket's candidates
         // (sm.misc[3] was zeroed before cut_bucket's barriers); if the
@@ -740,7 +753,7 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
             __syncthreads();
         } else {
             int before;
-            const int bk = cut_bucket(sm, static_cast<double>(n_take), false, &before, nbk);
+            const int bk = cut_bucket(sm, static_cast<uint32_t>(n_take), false, &before, nbk);
             if (threadIdx.x == 0) sm.misc[3] = 0;
             for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
             __syncthreads();
@@ -809,12 +822,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
 }
 
 // Scoring (§2.1, Eq. 2) and selection in one launch.  The C CTAs of a unit
-// share its 16-block tiles: CTA c takes rounds c, c + C, ... of NW * kTileBatch tiles
-// (one batch of kTileBatch tiles per warp per round, the next round's page
-// ids loading while this round's keys do).  With C = 1 the scores stay in
-// shared memory and the CTA selects at once; otherwise they go to
-// p.scores_out and the unit's last CTA to finish -- a per-unit arrival
-// counter in the workspace, reset to zero by that CTA -- selects from them.
+// (one thread-block cluster when C > 1) share its 16-block tiles: CTA c
+// takes rounds c, c + C, ... of NW * kTileBatch tiles (one batch of
+// kTileBatch tiles per warp per round, the next round's page ids loading
+// while this round's keys do).  Every CTA stores its scores straight into
+// the shared memory of the cluster's first CTA, which selects once the
+// cluster barrier (release / acquire at cluster scope) has passed.
 template <int FMT>
 __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const SelectParams p,
                                                                          int C) {
@@ -828,7 +841,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
     const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
     const int n_full = min(L / (kBlock / p.blocks_per_page), cap);   // overflow: flagged
     const int tiles = (n_full + 15) / 16;                            // by the selection
-    float* out = C == 1 ? sm.score : p.scores_out + static_cast<int64_t>(u) * p.max_blocks;
+    float* out = sm.score;                                           // the leader's
+    if (C > 1) out = cooperative_groups::this_cluster().map_shared_rank(sm.score, 0);
     constexpr int kRound = NW * kTileBatch;
     const int step = C * kRound;
     const int first = c * kRound + warp;
@@ -847,19 +861,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
         }
     }
     if (C > 1) {
-        __syncthreads();                              // this CTA's score stores are issued
-        if (threadIdx.x == 0) {
-            __threadfence();                          // ... and visible before it arrives
-            const unsigned old = atomicAdd(&p.sel_done[u], 1u);
-            const int last = old == static_cast<unsigned>(C - 1);
-            if (last) p.sel_done[u] = 0u;
-            sm.misc[7] = last;
-        }
-        __syncthreads();
-        if (!sm.misc[7]) return;
-        __threadfence();                              // the other CTAs' scores
+        cooperative_groups::this_cluster().sync();    // all of the unit's scores are in
+        if (c != 0) return;
     }
-    select_unit(p, u, sm, C == 1, L, pb);
+    select_unit(p, u, sm, true, L, pb);
 }
 
 }  // namespace
@@ -890,9 +895,21 @@ cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t
     const int U = p.batch * p.num_kv_heads;
     const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
     const int rounds = max(1, ((cap + 15) / 16 + NW * kTileBatch - 1) / (NW * kTileBatch));
-    const int C = max(1, min(rounds, sm_count() / max(U, 1)));
-    score_select_kernel<FMT><<<U * C, kSelectThreads, smem, s>>>(p, C);
-    return cudaGetLastError();
+    const int C = max(1, min(min(rounds, kMaxCluster), sm_count() / max(U, 1)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(U * C);
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, score_select_kernel<FMT>, p, C);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

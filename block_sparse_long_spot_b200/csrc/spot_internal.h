@@ -43,7 +43,7 @@ constexpr int kTokBlocksPerPage = kBlock / kTokBlock;     // 4
 constexpr int kSelectFromScores = -1;  // launch_select "format": scores precomputed
 
 struct Layout {
-    size_t status, unit_done, sel_done, partials, total;
+    size_t status, unit_done, partials, total;
     size_t scores;                      // block scores [units][max_blocks] fp32 (the token
                                         // selector uses [B][max_blocks] of it)
     int grid;                           // persistent CTAs of the decode kernel
@@ -67,10 +67,8 @@ struct SelectParams {
     int32_t mode, sink_blocks, recency_blocks, kmin_blocks, topk_blocks;
     int32_t quantize_queries;           // quantise q_sel with the key format's rule
     int32_t blocks_per_page;            // selection blocks per page-table entry (1 or 4)
-    const float* scores_in;             // selection: block scores [units][max_blocks]
-    float* scores_out;                  // block scoring: the same array, written
-    uint32_t* sel_done;                 // [units] arrival counters of the scoring CTAs,
-                                        // zero between calls
+    const float* scores_in;             // selection on precomputed block scores
+                                        // [units][max_blocks]
     int32_t* sel_idx;
     int32_t* sel_cnt;
     uint32_t* status;

@@ -124,8 +124,8 @@ typedef struct {
  * this shape on the CURRENT device (it depends on the SM count).  Zero the
  * whole workspace once before its first use (e.g. allocate it zero-filled):
  * its first 256 bytes hold the device status word, and it holds per-unit
- * arrival counters of the scoring and decode kernels that must start at
- * zero; every call that completes leaves those counters at zero again.  After
+ * arrival counters of the decode kernel that must start at zero; every call
+ * that completes leaves those counters at zero again.  After
  * a call whose status reads SPOT_ERR_DEVICE_TIMEOUT, zero the whole workspace
  * before its next use.  Returns 0 for a shape this build does not support. */
 size_t spot_workspace_size(const spot_layer_desc_t* desc, int32_t batch, int32_t max_blocks);
