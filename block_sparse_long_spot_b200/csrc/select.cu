@@ -77,7 +77,8 @@ __device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
                                             const uint32_t (&qw)[8], const float (&qsc)[2][2],
                                             float wh0, float wh1, int t0, int stride, int n_full, float* scores,
                                             int lane, const int (&pga)[kTileBatch],
-                                            const int (&pgb)[kTileBatch]) {
+                                            const int (&pgb)[kTileBatch], int r0, int r1,
+                                            float& wmax, float& wmin) {
     const int c4 = lane & 3, r8 = lane >> 2;
     int64_t rowa[kTileBatch], rowb[kTileBatch];
 #pragma unroll
@@ -192,8 +193,11 @@ __device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
         sb += __shfl_xor_sync(0xffffffffu, sb, 2);
         const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
         if (c4 == 0) {
-            if (ja < n_full) scores[ja] = sa * p.inv_temp;
-            if (jb < n_full) scores[jb] = sb * p.inv_temp;
+            const float va = sa * p.inv_temp, vb = sb * p.inv_temp;
+            if (ja < n_full) scores[ja] = va;
+            if (jb < n_full) scores[jb] = vb;
+            if (ja >= r0 && ja < r1) { wmax = fmaxf(wmax, va); wmin = fminf(wmin, va); }
+            if (jb >= r0 && jb < r1) { wmax = fmaxf(wmax, vb); wmin = fminf(wmin, vb); }
         }
     }
 }
@@ -257,6 +261,7 @@ struct SelSmem {
     int* misc;                    // [8]
     int* scan;                    // [NW + 1]
     float* fscan;                 // [NW + 1]
+    float* part;                  // [2][kMaxCluster * NW] scoring warps' residual max, min
 };
 
 // Sums of three values over the block (two barriers).
@@ -520,7 +525,7 @@ size_t select_smem_bytes(int max_blocks) {
            kNB * (sizeof(uint32_t) + sizeof(uint32_t)) +
            NT * (sizeof(uint32_t) + sizeof(int) + sizeof(unsigned long long)) +
            3 * NW * sizeof(unsigned long long) + 8 * sizeof(int) +
-           2 * (NW + 1) * sizeof(int) + 128;
+           2 * (NW + 1) * sizeof(int) + 2 * kMaxCluster * NW * sizeof(float) + 128;
 }
 
 namespace {
@@ -556,33 +561,56 @@ __device__ __forceinline__ SelSmem carve_select_smem(uint8_t* smem, int max_bloc
     q += sizeof(int) * (NW + 1);
     sm.fscan = reinterpret_cast<float*>(q);
     q += sizeof(float) * (NW + 1);
+    sm.part = reinterpret_cast<float*>(q);
+    q += sizeof(float) * 2 * kMaxCluster * NW;
     sm.vb = reinterpret_cast<uint16_t*>(q);
     q += sizeof(uint16_t) * max_blocks;
     sm.keep = q;
     return sm;
 }
 
+// Blocks of a sequence of L tokens: nb in all and n_full complete ones
+// (both at most the table's capacity; `over` when it had to clip), and the
+// residual blocks [r0, r1) left by the sink and recency reservations (the
+// incomplete last block is always a recency block, so r1 <= n_full).
+struct BlockSpan {
+    int nb, n_full, r0, r1;
+    bool over;
+};
+__device__ __forceinline__ BlockSpan block_span(const SelectParams& p, int L) {
+    BlockSpan sp;
+    const int bsz = kBlock / p.blocks_per_page;        // tokens per selection block
+    sp.nb = (L + bsz - 1) / bsz;
+    sp.n_full = L / bsz;
+    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
+    sp.over = sp.nb > cap;
+    if (sp.over) {
+        sp.nb = cap;
+        sp.n_full = min(sp.n_full, cap);
+    }
+    const int sink = min(max(p.sink_blocks, 0), sp.nb);
+    int rec = max(p.recency_blocks, 0);
+    rec = max(rec, sp.nb - sp.n_full);
+    rec = min(rec, sp.nb);
+    sp.r0 = sink;
+    sp.r1 = max(sink, sp.nb - rec);
+    return sp;
+}
+
 // Selection of unit u (all threads of the CTA) on its block scores: in
 // shared memory already (`in_smem`), else read from p.scores_in.  L is the
 // sequence's length (>= 0) and pb its top-p (p.top_p[b], 1 without one),
-// both read by the caller ahead of its other work.
+// both read by the caller ahead of its other work.  With nparts > 0 the
+// maximum and minimum of the residual scores are folded from nparts
+// partial values in sm.part (written by the scoring warps) instead of from
+// the scores.
 __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, bool in_smem, int L,
-                            float pb) {
+                            float pb, int nparts) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int bsz = kBlock / p.blocks_per_page;        // tokens per selection block
-    int nb = (L + bsz - 1) / bsz;
-    int n_full = L / bsz;
-    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
-    if (nb > cap) {
-        if (threadIdx.x == 0) flag_status(p.status, kStatusBounds);
-        nb = cap;
-        n_full = min(n_full, cap);
-    }
-    const int sink = min(max(p.sink_blocks, 0), nb);
-    int rec = max(p.recency_blocks, 0);
-    rec = max(rec, nb - n_full);
-    rec = min(rec, nb);
-    const int r0 = sink, r1 = max(sink, nb - rec);    // residual blocks [r0, r1)
+    const BlockSpan sp = block_span(p, L);
+    if (sp.over && threadIdx.x == 0) flag_status(p.status, kStatusBounds);
+    const int nb = sp.nb, n_full = sp.n_full;
+    const int r0 = sp.r0, r1 = sp.r1;                 // residual blocks [r0, r1)
     const int n = r1 - r0;
     const int n_reserved = nb - n;
     const float* s = sm.score;
@@ -609,29 +637,41 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     }
     __syncthreads();
 
-    // ---- residual scores -> keys, maximum and minimum
-    float mloc = -INFINITY, nloc = INFINITY;
-    for (int i = threadIdx.x; i < n; i += NT) {
-        const float v = s[r0 + i];
-        sm.keys[i] = score_key(v);
-        mloc = fmaxf(mloc, v);
-        nloc = fminf(nloc, v);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
-        nloc = fminf(nloc, __shfl_xor_sync(0xffffffffu, nloc, o));
-    }
-    float* wmin = reinterpret_cast<float*>(sm.scan);  // next written after two barriers
-    if (lane == 0) {
-        sm.fscan[warp] = mloc;
-        wmin[warp] = nloc;
-    }
-    __syncthreads();
+    // ---- maximum and minimum of the residual scores (and their keys)
     float smax_f = -INFINITY, smin_f = INFINITY;
-    for (int w = 0; w < NW; ++w) {
-        smax_f = fmaxf(smax_f, sm.fscan[w]);
-        smin_f = fminf(smin_f, wmin[w]);
+    if (nparts > 0) {                                 // every warp folds the partials
+        for (int i = lane; i < nparts; i += 32) {
+            smax_f = fmaxf(smax_f, sm.part[i]);
+            smin_f = fminf(smin_f, sm.part[kMaxCluster * NW + i]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            smax_f = fmaxf(smax_f, __shfl_xor_sync(0xffffffffu, smax_f, o));
+            smin_f = fminf(smin_f, __shfl_xor_sync(0xffffffffu, smin_f, o));
+        }
+    } else {
+        float mloc = -INFINITY, nloc = INFINITY;
+        for (int i = threadIdx.x; i < n; i += NT) {
+            const float v = s[r0 + i];
+            sm.keys[i] = score_key(v);
+            mloc = fmaxf(mloc, v);
+            nloc = fminf(nloc, v);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+            nloc = fminf(nloc, __shfl_xor_sync(0xffffffffu, nloc, o));
+        }
+        float* wmin = reinterpret_cast<float*>(sm.scan);  // next written after two barriers
+        if (lane == 0) {
+            sm.fscan[warp] = mloc;
+            wmin[warp] = nloc;
+        }
+        __syncthreads();
+        for (int w = 0; w < NW; ++w) {
+            smax_f = fmaxf(smax_f, sm.fscan[w]);
+            smin_f = fminf(smin_f, wmin[w]);
+        }
     }
     const double smax = static_cast<double>(smax_f);
     // buckets per unit of score: the residual range spans all nbk buckets,
@@ -660,6 +700,7 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
             if (i >= n) break;
             const unsigned long long f = __double2ull_rn(ldexp(e[k], kFixShift));
             sm.mass[i] = f;
+            if (nparts > 0) sm.keys[i] = score_key(v[k]);
             const int bkt = static_cast<int>(fminf((smax_f - v[k]) * bscale, nbk - 1.f));
             sm.vb[i] = static_cast<uint16_t>(bkt);
             atomicAdd(&sm.hcnt[bkt], 1u);
@@ -818,7 +859,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
     const int b = blockIdx.x / p.num_kv_heads;
     const int L = max(p.seq_lens[b], 0);
     const float pb = p.top_p ? p.top_p[b] : 1.f;
-    select_unit(p, blockIdx.x, sm, false, L, pb);
+    select_unit(p, blockIdx.x, sm, false, L, pb, 0);
 }
 
 // Scoring (§2.1, Eq. 2) and selection in one launch.  The C CTAs of a unit
@@ -837,12 +878,17 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
     const int u = blockIdx.x / C, c = blockIdx.x - u * C;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
     const int L = max(p.seq_lens[b], 0);
-    const float pb = p.top_p ? p.top_p[b] : 1.f;                     // for the selection
-    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
-    const int n_full = min(L / (kBlock / p.blocks_per_page), cap);   // overflow: flagged
-    const int tiles = (n_full + 15) / 16;                            // by the selection
+    const float ptop = p.top_p ? p.top_p[b] : 1.f;                   // for the selection
+    const BlockSpan sp = block_span(p, L);                           // overflow: flagged
+    const int n_full = sp.n_full;                                    // by the selection
+    const int tiles = (n_full + 15) / 16;
     float* out = sm.score;                                           // the leader's
-    if (C > 1) out = cooperative_groups::this_cluster().map_shared_rank(sm.score, 0);
+    float* part = sm.part;
+    if (C > 1) {
+        out = cooperative_groups::this_cluster().map_shared_rank(sm.score, 0);
+        part = cooperative_groups::this_cluster().map_shared_rank(sm.part, 0);
+    }
+    float wmax = -INFINITY, wmin = INFINITY;                         // residual scores
     constexpr int kRound = NW * kTileBatch;
     const int step = C * kRound;
     const int first = c * kRound + warp;
@@ -855,16 +901,26 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
         for (int t0 = first; t0 < tiles; t0 += step) {
             int na[kTileBatch], nb2[kTileBatch];
             if (t0 + step < tiles) load_pages(p, b, t0 + step, NW, n_full, lane, na, nb2);
-            score_tiles<FMT>(p, g, qw, qsc, wh0, wh1, t0, NW, n_full, out, lane, pa, pb);
+            score_tiles<FMT>(p, g, qw, qsc, wh0, wh1, t0, NW, n_full, out, lane, pa, pb, sp.r0,
+                             sp.r1, wmax, wmin);
 #pragma unroll
             for (int k = 0; k < kTileBatch; ++k) { pa[k] = na[k]; pb[k] = nb2[k]; }
         }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+        wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
+    }
+    if (lane == 0) {
+        part[c * NW + warp] = wmax;
+        part[kMaxCluster * NW + c * NW + warp] = wmin;
     }
     if (C > 1) {
         cooperative_groups::this_cluster().sync();    // all of the unit's scores are in
         if (c != 0) return;
     }
-    select_unit(p, u, sm, true, L, pb);
+    select_unit(p, u, sm, true, L, ptop, C * NW);
 }
 
 }  // namespace
