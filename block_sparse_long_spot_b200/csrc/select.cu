@@ -415,16 +415,17 @@ __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long lon
         }
         if (threadIdx.x < 32) {                       // one warp ranks the few candidates
             const int lane = threadIdx.x;
-            int rank = 0, j = -1;
-            if (lane < c) {
-                const uint32_t k = sm.ckey[lane];
-                j = sm.cidx[lane];
-                for (int d = 0; d < c; ++d) {
-                    const uint32_t kd = sm.ckey[d];
-                    rank += (kd > k) || (kd == k && sm.cidx[d] < j);
-                }
-                sm.cval[rank] = by_mass ? sm.mass[j] : 1ull;
+            const uint32_t k = lane < c ? sm.ckey[lane] : 0u;
+            const int j = lane < c ? sm.cidx[lane] : -1;
+            const unsigned long long mj = (lane < c && by_mass) ? sm.mass[j] : 1ull;
+            int rank = 0;
+#pragma unroll
+            for (int d = 0; d < 32; ++d) {            // candidate d sits in lane d
+                const uint32_t kd = __shfl_sync(0xffffffffu, k, d);
+                const int jd = __shfl_sync(0xffffffffu, j, d);
+                rank += (d < c) && ((kd > k) || (kd == k && jd < j));
             }
+            if (lane < c) sm.cval[rank] = mj;         // the values in rank order
             __syncwarp();
             const unsigned long long v = lane < c ? sm.cval[lane] : 0ull;
             unsigned long long incl = v;
@@ -812,6 +813,32 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     const int per_w = ((nb + NW - 1) / NW + 31) & ~31;
     const int wlo = min(nb, warp * per_w), whi = min(nb, wlo + per_w);
     const unsigned lt = (1u << lane) - 1u;
+    int* list = reinterpret_cast<int*>(sm.keys);
+    int32_t* out = p.sel_idx + static_cast<int64_t>(u) * p.max_blocks;
+    if (take == 0) {
+        // no ties to count in block order: one pass, each warp packing its
+        // kept ids at the front of its own id range of the list and, after
+        // one barrier for the warps' counts, writing them out at its offset
+        int wk = 0;
+        for (int j0 = wlo; j0 < whi; j0 += 32) {
+            const int j = j0 + lane;
+            const int f = j >= whi ? 0 : ((j < r0 || j >= r1) ? 1 : sm.keep[j - r0]);
+            const unsigned kbal = __ballot_sync(0xffffffffu, f == 1);
+            if (f == 1) list[wlo + wk + __popc(kbal & lt)] = j;
+            wk += __popc(kbal);
+        }
+        if (lane == 0) sm.scan[warp] = wk;
+        __syncthreads();
+        int kb = 0, ktot = 0;
+        for (int w = 0; w < NW; ++w) {
+            const int a = sm.scan[w];
+            if (w < warp) kb += a;
+            ktot += a;
+        }
+        for (int t = lane; t < wk; t += 32) out[kb + t] = list[wlo + t];
+        if (threadIdx.x == 0) p.sel_cnt[u] = ktot;
+        return;
+    }
     int wk = 0, wt = 0;
     for (int j0 = wlo; j0 < whi; j0 += 32) {
         const int j = j0 + lane;
@@ -831,7 +858,6 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
         ktot += a;
         ttot += t;
     }
-    int* list = reinterpret_cast<int*>(sm.keys);
     int pos = kb + min(tb, static_cast<int>(take)), tr = tb;
     for (int j0 = wlo; j0 < whi; j0 += 32) {
         const int j = j0 + lane;
@@ -845,7 +871,6 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     }
     const int cnt = ktot + min(ttot, static_cast<int>(take));
     __syncthreads();
-    int32_t* out = p.sel_idx + static_cast<int64_t>(u) * p.max_blocks;
     for (int i = threadIdx.x; i < cnt; i += NT) out[i] = list[i];
     if (threadIdx.x == 0) p.sel_cnt[u] = cnt;
 }
