@@ -22,13 +22,14 @@
 // Selection: residual softmax numerators exp(s - max) are computed in fp64
 //   and held as 2^-40 fixed-point integers (exact, order-independent sums).
 //   The nucleus cut is a bucketed threshold search: the residual blocks are
-//   histogrammed into 1024 or 2048 buckets of the score's distance from the maximum,
-//   scaled so the residual range spans them all (monotone in the score;
-//   exact counts, 2^-18 fixed-point masses), the
-//   bucket where the cumulative mass from the top reaches p * Z is found by a
-//   block scan and confirmed on the exact fixed-point masses, and the few
-//   blocks inside that bucket are ranked exactly (score descending, lower
-//   block index first).  The K_min floor and static top-K use the same search
+//   histogrammed into 1024 or 2048 buckets of the score's distance from the
+//   maximum, scaled so the residual range spans them all (monotone in the
+//   score), with exact counts and exact fixed-point masses (the low words
+//   add up with returning 32-bit shared atomics, and the add that wraps one
+//   carries into the high word); the bucket where the cumulative mass from
+//   the top reaches p * Z is found from the warps' totals and one lane
+//   scan, and the few blocks inside that bucket are ranked exactly (score
+//   descending, lower block index first).  The K_min floor and static top-K use the same search
 //   on counts.  A block scan compacts the kept blocks in ascending order.
 //
 // The token-level selector and sparse prefill reuse the selection with their
@@ -241,8 +242,6 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 constexpr int kNB = 2048;              // most value buckets of the first pass (1024 up to
                                         // 2048 residual blocks, then 2048), spread over the
                                         // residual scores' range
-constexpr int kApproxShift = 18;        // bucket masses for the search: 2^-18 fixed point
-                                        // (<= 8192 elements of mass <= 1 fit in 32 bits)
 constexpr int NT = kSelectThreads;
 constexpr int NW = NT / 32;
 
@@ -252,7 +251,8 @@ struct SelSmem {
     unsigned long long* mass;     // [max_blocks] fixed-point exp(s - max)
     uint16_t* vb;                 // [max_blocks] value bucket (0 = the top scores)
     uint8_t* keep;                // [max_blocks] 1 keep, 2 tie at the cut, 0 drop
-    uint32_t* hmass;              // [kNB] approximate mass per bucket, 2^-18 fixed point
+    uint32_t* hlo;                // [kNB] exact mass per bucket (2^-40 fixed point):
+    uint32_t* hhi;                //       low word (wrapping) and high word (+ carries)
     uint32_t* hcnt;               // [kNB] exact count per bucket
     uint32_t* ckey;               // [NT] candidates of the cut bucket: key
     int* cidx;                    //      element index
@@ -286,70 +286,86 @@ __device__ __forceinline__ void block_sum3(const SelSmem& sm, unsigned long long
     __syncthreads();
 }
 
-// Bucket of the cut, found on the bucket histograms: the first bucket (from
-// the top) where the cumulative value reaches `target` (>= 1).  by_mass uses
-// the approximate 2^-18 fixed-point masses (the caller corrects the result
-// exactly; their total stays below 2^31), else the exact counts.  Returns the
-// bucket; *before receives the exact count of the elements in the buckets
-// above it.  Two barriers: the warps' totals, then a lane scan in the one
-// warp whose buckets hold the crossing point.
-__device__ int cut_bucket(const SelSmem& sm, uint32_t target, bool by_mass, int* before,
-                          int nbk) {
+// Exact mass of bucket b, 2^-40 fixed point.
+__device__ __forceinline__ unsigned long long bucket_mass(const SelSmem& sm, int b) {
+    return (static_cast<unsigned long long>(sm.hhi[b]) << 32) | sm.hlo[b];
+}
+
+// Bucket of the cut on the exact bucket histograms (complete, behind a
+// barrier, before the call): the first bucket from the top where the
+// cumulative mass (by_mass) or count reaches the target.  by_mass: the
+// target is T = ceil(pb * Z), Z the residual blocks' total mass, clamped to
+// [1, Z], and *target receives it; else *target holds the count to reach
+// (>= 1).  Returns the bucket; *before receives the count and *above the
+// mass (count) of the elements in the buckets above it.  Two barriers: the
+// warps' totals, then a lane scan in the one warp whose buckets hold the
+// crossing point.
+__device__ int cut_bucket(const SelSmem& sm, bool by_mass, float pb, unsigned long long* target,
+                          int* before, unsigned long long* above, int nbk) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int PER = nbk / NT;
-    uint32_t loc = 0;
+    unsigned long long loc = 0;
     int cnt = 0, last = -1;
     for (int k = 0; k < PER; ++k) {
         const int bkt = threadIdx.x * PER + k;
         const uint32_t c = sm.hcnt[bkt];
-        loc += by_mass ? sm.hmass[bkt] : c;
+        loc += by_mass ? bucket_mass(sm, bkt) : c;
         cnt += static_cast<int>(c);
         if (c) last = bkt;
     }
-    const uint32_t wv = warp_sum(loc);
+    const unsigned long long wv = warp_sum(loc);
     const int wc = warp_sum(cnt);
     int wl = last;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wl = max(wl, __shfl_xor_sync(0xffffffffu, wl, o));
-    int* wtot = reinterpret_cast<int*>(sm.red);        // [NW] values, counts, last buckets
+    int* wint = reinterpret_cast<int*>(sm.red + NW);  // [NW] counts, [NW] last buckets
     if (lane == 0) {
-        wtot[warp] = static_cast<int>(wv);
-        wtot[NW + warp] = wc;
-        wtot[2 * NW + warp] = wl;
+        sm.red[warp] = wv;
+        wint[warp] = wc;
+        wint[NW + warp] = wl;
     }
     __syncthreads();
+    unsigned long long tot = 0;
+    for (int w = 0; w < NW; ++w) tot += sm.red[w];
+    unsigned long long tgt = *target;
+    if (by_mass) {
+        tgt = static_cast<unsigned long long>(ceil(static_cast<double>(pb) * static_cast<double>(tot)));
+        tgt = tgt < 1ull ? 1ull : (tgt > tot ? tot : tgt);
+        *target = tgt;
+    }
     // every thread finds the warp whose buckets reach the target
-    uint32_t run = 0;
+    unsigned long long run = 0;
     int crun = 0, cw = -1, ctot = 0, lastb = -1;
     for (int w = 0; w < NW; ++w) {
-        const uint32_t v = static_cast<uint32_t>(wtot[w]);
-        const int c = wtot[NW + w];
+        const unsigned long long v = sm.red[w];
+        const int c = wint[w];
         if (cw < 0) {
-            if (run + v >= target) cw = w;
+            if (run + v >= tgt) cw = w;
             else { run += v; crun += c; }
         }
         ctot += c;
-        lastb = max(lastb, wtot[2 * NW + w]);
+        lastb = max(lastb, wint[NW + w]);
     }
     if (warp == cw) {                                 // warp-uniform
-        uint32_t incl = loc;
+        unsigned long long incl = loc;
         int cincl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+            const unsigned long long x = __shfl_up_sync(0xffffffffu, incl, o);
             const int y = __shfl_up_sync(0xffffffffu, cincl, o);
             if (lane >= o) { incl += x; cincl += y; }
         }
-        uint32_t r = run + incl - loc;
+        unsigned long long r = run + incl - loc;
         int cr = crun + cincl - cnt;
-        if (r < target && r + loc >= target) {        // one lane
+        if (r < tgt && r + loc >= tgt) {              // one lane
             for (int k = 0; k < PER; ++k) {
                 const int bkt = threadIdx.x * PER + k;
                 const uint32_t c = sm.hcnt[bkt];
-                const uint32_t v = by_mass ? sm.hmass[bkt] : c;
-                if (c && r + v >= target) {
+                const unsigned long long v = by_mass ? bucket_mass(sm, bkt) : c;
+                if (c && r + v >= tgt) {
                     sm.misc[0] = bkt;
                     sm.misc[2] = cr;
+                    sm.red[3 * NW - 1] = r;
                     break;
                 }
                 r += v;
@@ -360,10 +376,12 @@ __device__ int cut_bucket(const SelSmem& sm, uint32_t target, bool by_mass, int*
     __syncthreads();
     if (cw >= 0) {
         *before = sm.misc[2];
+        *above = sm.red[3 * NW - 1];
         return sm.misc[0];
     }
-    // the rounded masses stayed below the target: the lowest non-empty bucket
+    // (not reached: the target never exceeds the total) the lowest non-empty bucket
     *before = ctot - static_cast<int>(sm.hcnt[lastb]);
+    *above = tot - (by_mass ? bucket_mass(sm, lastb) : sm.hcnt[lastb]);
     return lastb;
 }
 
@@ -523,7 +541,7 @@ size_t select_smem_bytes(int max_blocks) {
     return static_cast<size_t>(max_blocks) *
                (sizeof(float) + sizeof(uint32_t) + sizeof(unsigned long long) +
                 sizeof(uint16_t) + 1) +
-           kNB * (sizeof(uint32_t) + sizeof(uint32_t)) +
+           kNB * 3 * sizeof(uint32_t) +
            NT * (sizeof(uint32_t) + sizeof(int) + sizeof(unsigned long long)) +
            3 * NW * sizeof(unsigned long long) + 8 * sizeof(int) +
            2 * (NW + 1) * sizeof(int) + 2 * kMaxCluster * NW * sizeof(float) + 128;
@@ -548,7 +566,9 @@ __device__ __forceinline__ SelSmem carve_select_smem(uint8_t* smem, int max_bloc
     q += sizeof(float) * max_blocks;
     sm.keys = reinterpret_cast<uint32_t*>(q);
     q += sizeof(uint32_t) * max_blocks;
-    sm.hmass = reinterpret_cast<uint32_t*>(q);
+    sm.hlo = reinterpret_cast<uint32_t*>(q);
+    q += sizeof(uint32_t) * kNB;
+    sm.hhi = reinterpret_cast<uint32_t*>(q);
     q += sizeof(uint32_t) * kNB;
     sm.hcnt = reinterpret_cast<uint32_t*>(q);
     q += sizeof(uint32_t) * kNB;
@@ -616,7 +636,7 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     const int n_reserved = nb - n;
     const float* s = sm.score;
     const int nbk = n > 2048 ? 2048 : 1024;          // value buckets
-    for (int i = threadIdx.x; i < nbk; i += NT) { sm.hmass[i] = 0u; sm.hcnt[i] = 0u; }
+    for (int i = threadIdx.x; i < nbk; i += NT) { sm.hlo[i] = 0u; sm.hhi[i] = 0u; sm.hcnt[i] = 0u; }
     if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
     pdl_trigger();                                    // the decode kernel may start its prologue
 
@@ -681,9 +701,8 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     const float range = fminf(smax_f - smin_f, 40.f);
     const float bscale = range > 1e-30f ? static_cast<float>(nbk - 1) / range : 1.f;
 
-    // ---- exact fixed-point numerators exp(s - max), their total Z, value
-    // buckets (monotone in the score) with exact counts and fp32 masses
-    unsigned long long zloc = 0;
+    // ---- exact fixed-point numerators exp(s - max), value
+    // buckets (monotone in the score) with exact counts and masses
     constexpr int kUnroll = 4;                        // independent exps in flight
     for (int i0 = threadIdx.x; i0 < n; i0 += kUnroll * NT) {
         float v[kUnroll];
@@ -705,12 +724,14 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
             const int bkt = static_cast<int>(fminf((smax_f - v[k]) * bscale, nbk - 1.f));
             sm.vb[i] = static_cast<uint16_t>(bkt);
             atomicAdd(&sm.hcnt[bkt], 1u);
-            atomicAdd(&sm.hmass[bkt], static_cast<uint32_t>(ldexp(e[k], kApproxShift) + 0.5));
-            zloc += f;
+            // exact bucket mass: the add that wraps the low word carries
+            const uint32_t lo = static_cast<uint32_t>(f), hi = static_cast<uint32_t>(f >> 32);
+            const uint32_t old = atomicAdd(&sm.hlo[bkt], lo);
+            const uint32_t up = hi + (old + lo < old ? 1u : 0u);
+            if (up) atomicAdd(&sm.hhi[bkt], up);
         }
     }
-    unsigned long long Z = zloc, d1 = 0, d2 = 0;
-    block_sum3(sm, Z, d1, d2);
+    __syncthreads();                                  // the histograms are complete
 
     // ---- how many residual blocks to keep, and which
     int n_take = 0;        // -1: decided by the mass cut below
@@ -723,61 +744,24 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     }
     bool done = false;
     if (n_take < 0) {
-        unsigned long long T = static_cast<unsigned long long>(
-            ceil(static_cast<double>(pb) * static_cast<double>(Z)));
-        T = T < 1ull ? 1ull : (T > Z ? Z : T);
+        // the nucleus cut on the exact masses: T = ceil(p Z); the blocks of
+        // the buckets above the crossing one are kept, and its own blocks
+        // are ranked exactly.  The keep-flag pass also gathers a small
+        // bucket's candidates (sm.misc[3] is zeroed before cut_bucket's
+        // barriers).
+        unsigned long long T = 0, A;
         int before;
         if (threadIdx.x == 0) sm.misc[3] = 0;
-        const double tq = ceil(ldexp(static_cast<double>(T), kApproxShift - kFixShift));
-        int bk = cut_bucket(sm, tq < 1.0 ? 1u : static_cast<uint32_t>(tq), true, &before, nbk);
-        // Exact check of the bucket on the fixed-point masses.  The first
-        // pass also writes the keep flags and gathers the bucket's candidates
-        // (sm.misc[3] was zeroed before cut_bucket's barriers); if the
-        // approximate bucket was off, step to the neighbouring non-empty
-        // bucket and redo the flags and the gather.
-        unsigned long long A, Bm, Ac;
+        const int bk = cut_bucket(sm, true, pb, &T, &before, &A, nbk);
         const bool small = sm.hcnt[bk] <= 32u;
-        {
-            A = 0; Bm = 0; Ac = 0;
-            for (int i0 = threadIdx.x - lane; i0 < n; i0 += NT) {   // warp-uniform
-                const int i = i0 + lane;
-                const int v = i < n ? sm.vb[i] : -1;
-                if (i < n) sm.keep[i] = v < bk ? 1 : 0;
-                if (i < n && v < bk) {
-                    A += sm.mass[i];
-                    ++Ac;
-                } else if (v == bk) {
-                    Bm += sm.mass[i];
-                }
-                if (small) push_candidate(sm, v == bk, i);
-            }
-            block_sum3(sm, A, Bm, Ac);
+        for (int i0 = threadIdx.x - lane; i0 < n; i0 += NT) {   // warp-uniform
+            const int i = i0 + lane;
+            const int v = i < n ? sm.vb[i] : -1;
+            if (i < n) sm.keep[i] = v < bk ? 1 : 0;
+            if (small) push_candidate(sm, v == bk, i);
         }
-        bool gathered = small;
-        for (int guard = 0; guard < nbk; ++guard) {
-            int step = 0;
-            if (A >= T) step = -1;
-            else if (A + Bm < T) step = 1;
-            if (step == 0) break;
-            int nbk_ = bk + step;
-            while (nbk_ >= 0 && nbk_ < nbk && sm.hcnt[nbk_] == 0) nbk_ += step;
-            if (nbk_ < 0 || nbk_ >= nbk) break;
-            bk = nbk_;
-            gathered = false;
-            A = 0; Bm = 0; Ac = 0;
-            for (int i = threadIdx.x; i < n; i += NT) {
-                const int v = sm.vb[i];
-                if (v < bk) { A += sm.mass[i]; ++Ac; }
-                else if (v == bk) Bm += sm.mass[i];
-            }
-            block_sum3(sm, A, Bm, Ac);
-        }
-        if (!gathered) {
-            if (threadIdx.x == 0) sm.misc[3] = 0;
-            for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
-            __syncthreads();
-        }
-        n_take = static_cast<int>(Ac) + resolve_bucket(sm, n, bk, A, T, true, gathered);
+        __syncthreads();
+        n_take = before + resolve_bucket(sm, n, bk, A, T, true, small);
         done = true;
         const int floor_res = p.kmin_blocks - n_reserved;      // |S| >= K_min
         if (n_take < floor_res) {
@@ -795,7 +779,8 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
             __syncthreads();
         } else {
             int before;
-            const int bk = cut_bucket(sm, static_cast<uint32_t>(n_take), false, &before, nbk);
+            unsigned long long tq = static_cast<unsigned long long>(n_take), above;
+            const int bk = cut_bucket(sm, false, 1.f, &tq, &before, &above, nbk);
             if (threadIdx.x == 0) sm.misc[3] = 0;
             for (int i = threadIdx.x; i < n; i += NT) sm.keep[i] = sm.vb[i] < bk ? 1 : 0;
             __syncthreads();
