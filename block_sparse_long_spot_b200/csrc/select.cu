@@ -463,12 +463,15 @@ __device__ int resolve_bucket(const SelSmem& sm, int n, int b, unsigned long lon
     }
     if (threadIdx.x == 0) sm.misc[4] = c - 1;
     if (c <= NT) {
-        gather_bucket(sm, n, b);
-        __syncthreads();
+        if (!gathered) {
+            gather_bucket(sm, n, b);
+            __syncthreads();
+        }
         int rank = 0;
         if (threadIdx.x < c) {
             const uint32_t k = sm.ckey[threadIdx.x];
             const int j = sm.cidx[threadIdx.x];
+#pragma unroll 8
             for (int d = 0; d < c; ++d) {
                 const uint32_t kd = sm.ckey[d];
                 rank += (kd > k) || (kd == k && sm.cidx[d] < j);
@@ -643,7 +646,7 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     // ---- selector scores of the complete blocks (§2.1), into shared memory
     if (!in_smem) {
         const float* src = p.scores_in + static_cast<int64_t>(u) * p.max_blocks;
-        constexpr int kBatch = 8;                     // loads in flight per thread
+        constexpr int kBatch = 16;                    // loads in flight per thread
         for (int j0 = threadIdx.x; j0 < n_full; j0 += NT * kBatch) {
             float v[kBatch];
 #pragma unroll
@@ -746,22 +749,22 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     if (n_take < 0) {
         // the nucleus cut on the exact masses: T = ceil(p Z); the blocks of
         // the buckets above the crossing one are kept, and its own blocks
-        // are ranked exactly.  The keep-flag pass also gathers a small
-        // bucket's candidates (sm.misc[3] is zeroed before cut_bucket's
-        // barriers).
+        // are ranked exactly.  The keep-flag pass also gathers the bucket's
+        // candidates when they fit the candidate list (sm.misc[3] is zeroed
+        // before cut_bucket's barriers).
         unsigned long long T = 0, A;
         int before;
         if (threadIdx.x == 0) sm.misc[3] = 0;
         const int bk = cut_bucket(sm, true, pb, &T, &before, &A, nbk);
-        const bool small = sm.hcnt[bk] <= 32u;
+        const bool gath = sm.hcnt[bk] <= static_cast<uint32_t>(NT);
         for (int i0 = threadIdx.x - lane; i0 < n; i0 += NT) {   // warp-uniform
             const int i = i0 + lane;
             const int v = i < n ? sm.vb[i] : -1;
             if (i < n) sm.keep[i] = v < bk ? 1 : 0;
-            if (small) push_candidate(sm, v == bk, i);
+            if (gath) push_candidate(sm, v == bk, i);
         }
         __syncthreads();
-        n_take = before + resolve_bucket(sm, n, bk, A, T, true, small);
+        n_take = before + resolve_bucket(sm, n, bk, A, T, true, gath);
         done = true;
         const int floor_res = p.kmin_blocks - n_reserved;      // |S| >= K_min
         if (n_take < floor_res) {
