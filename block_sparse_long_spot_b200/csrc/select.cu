@@ -976,7 +976,7 @@ cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = C > 1 ? 1 : 0;                     // C = 1: a plain launch
     e = cudaLaunchKernelEx(&cfg, score_select_kernel<FMT>, p, C);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
