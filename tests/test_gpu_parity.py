@@ -239,14 +239,15 @@ def _assert_same_selection_or_near(gpu, ora, wl):
     assert diff <= 1
 
 
-def test_scoring_split_over_ctas_bit_exact_and_repeatable():
+@pytest.mark.parametrize("batch", [2, 8])
+def test_scoring_split_over_ctas_bit_exact_and_repeatable(batch):
     # Contexts of 300K - 512K tokens (up to 8192 blocks per (sequence, KV
-    # head)) over only 16 units: each unit's scoring is spread over several
-    # CTAs and the unit's last CTA to finish selects.  Integer selector inputs
-    # make every score exact, so every selection must equal the oracle's, and
-    # a second call on the same workspace must repeat it (the arrival
-    # counters are back at zero).
-    wl = workloads.make("ragged_hybrid", seed=13, device=DEV, integer=True, batch=2,
+    # head)) over only 16 or 64 units: each unit's scoring is spread over a
+    # cluster of 8 or 2 CTAs, which store their scores into the first CTA's
+    # shared memory, and that CTA selects.  Integer selector inputs make
+    # every score exact, so every selection must equal the oracle's, and a
+    # second call on the same workspace must repeat it.
+    wl = workloads.make("ragged_hybrid", seed=13, device=DEV, integer=True, batch=batch,
                         sel_fmt="bf16", ragged_range=(300000, 524288))
     data, scales = oracle_selector_pool(wl, "bf16")
     a = dict(q_sel=workloads.bits(wl.q_sel), w=None, sel_data=data, sel_scales=scales,
