@@ -385,12 +385,6 @@ __device__ int cut_bucket(const SelSmem& sm, bool by_mass, float pb, unsigned lo
     return lastb;
 }
 
-struct Cut {
-    int bucket;            // elements in buckets above it are kept, below it dropped
-    int kept_above;        // elements kept from the buckets above
-    int kept_in_bucket;    // elements kept from the bucket itself
-};
-
 // Appends element i (when `hit`) to the candidate list (sm.ckey / sm.cidx,
 // length sm.misc[3]) with one shared atomic per warp.  Every lane of the
 // warp must call it.
