@@ -934,12 +934,16 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
 
 namespace {
 
-std::mutex g_sms_mutex;
-int g_sms[64] = {};
+constexpr int kMemoDevices = 64;
+std::mutex g_sms_mutex;                  // guards both tables below
+int g_sms[kMemoDevices] = {};
+// Dynamic shared memory already allowed per device and kernel: slot 0 the
+// selection on precomputed scores, slot 1 + FMT the fused kernel of FMT.
+size_t g_smem_set[kMemoDevices][6] = {};
 
 int sm_count() {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMemoDevices) return 0;
     std::lock_guard<std::mutex> lock(g_sms_mutex);
     if (g_sms[dev] == 0 &&
         cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -947,11 +951,25 @@ int sm_count() {
     return g_sms[dev];
 }
 
+// Allows `kernel` smem bytes of dynamic shared memory on the current device
+// (one driver call per device, kernel and larger size).
+template <typename Kernel>
+cudaError_t allow_smem(Kernel kernel, int slot, size_t smem) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMemoDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_sms_mutex);
+    if (g_smem_set[dev][slot] >= smem) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e == cudaSuccess) g_smem_set[dev][slot] = smem;
+    return e;
+}
+
 template <int FMT>
 cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(score_select_kernel<FMT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = allow_smem(score_select_kernel<FMT>, 1 + FMT, smem);
     if (e != cudaSuccess) return e;
     // CTAs per unit: enough to cover the longest sequence in one round of
     // NW * kTileBatch tiles each, as far as one wave of one CTA per SM allows
@@ -982,8 +1000,7 @@ cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s) {
     if (p.batch * p.num_kv_heads <= 0) return cudaErrorInvalidValue;
     switch (fmt) {
         case kSelectFromScores: {
-            const cudaError_t e = cudaFuncSetAttribute(
-                select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            const cudaError_t e = allow_smem(select_kernel, 0, smem);
             if (e != cudaSuccess) return e;
             const dim3 grid(p.batch * p.num_kv_heads), block(kSelectThreads);
             const cudaError_t l = launch_pdl(select_kernel, grid, block, smem, s, p);
