@@ -252,7 +252,8 @@ struct SelSmem {
     uint16_t* vb;                 // [max_blocks] value bucket (0 = the top scores)
     uint8_t* keep;                // [max_blocks] 1 keep, 2 tie at the cut, 0 drop
     uint32_t* hlo;                // [kNB] exact mass per bucket (2^-40 fixed point):
-    uint32_t* hhi;                //       low word (wrapping) and high word (+ carries)
+    uint32_t* hhi;                //       low word (wrapping) and high word (+ carries);
+                                  //       <= kMaxBlocks masses <= 2^40 keep it < 2^22
     uint32_t* hcnt;               // [kNB] exact count per bucket
     uint32_t* ckey;               // [NT] candidates of the cut bucket: key
     int* cidx;                    //      element index
