@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
         return;
     }
     if (p.fmt == SPOT_SEL_INT8_F16) {
-        float km = fmaxf(fabsf(x0), fabsf(x1));
+        float km = fmaxf(poison_abs(x0), poison_abs(x1));
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o));
         const uint16_t sbits = f16_scale_bits(km, 127.0);
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
         if (lane == 0) reinterpret_cast<uint16_t*>(p.sel_scales)[row] = sbits;
         return;
     }
-    float amax = fmaxf(fabsf(x0), fabsf(x1));
+    float amax = fmaxf(poison_abs(x0), poison_abs(x1));
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const int grp = lane >> 4;

@@ -9,6 +9,13 @@
 //   FP8:   E4M3 round-to-nearest-even, saturating at +-448, zero stored as +0;
 //   INT8:  scale = binary16 RNE of amax/127 per key, code =
 //          clamp(rne(x / scale), -128, 127).
+// Non-finite inputs (OCP MX v1.0's rule for a block holding NaN or infinity,
+// carried over to every scaled format): a scale group with any NaN or +-inf
+// element gets the NaN scale (E8M0 0xFF; binary16 0x7E00 for INT4 / INT8)
+// and all-zero codes, so the whole group reads back as NaN; an FP8 element
+// that is NaN or +-inf is stored as the E4M3 NaN 0x7F.  The group maxima
+// below are taken with poison_abs, which maps NaN to +inf, so a group holds a
+// non-finite element exactly when its maximum is +inf.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -23,8 +30,16 @@
 
 namespace spot {
 
-// binary16 bits of amax / div, round to nearest even, saturating at 65504.
+// |x| for a group maximum: NaN counts as +inf, so that fmaxf (which drops
+// NaN operands) still marks the group as holding a non-finite element.
+__device__ __forceinline__ float poison_abs(float x) {
+    return x != x ? INFINITY : fabsf(x);
+}
+
+// binary16 bits of amax / div, round to nearest even, saturating at 65504;
+// the NaN scale 0x7E00 when amax is not finite (the group holds NaN / inf).
 __device__ __forceinline__ uint16_t f16_scale_bits(float amax, double div) {
+    if (!(amax <= 3.402823466e38f)) return static_cast<uint16_t>(0x7E00u);
     const double t = static_cast<double>(amax) / div;
     return (t >= 65504.0) ? static_cast<uint16_t>(0x7BFFu) : __half_as_ushort(__double2half(t));
 }
@@ -40,9 +55,16 @@ __device__ __forceinline__ int int_code(float x, float scale, int lo, int hi) {
     return static_cast<int>(fmin(static_cast<double>(hi), fmax(static_cast<double>(lo), q)));
 }
 
-// MXFP4 shared exponent X of a group with maximum magnitude amax.
+// MXFP4 shared exponent X of a group with maximum magnitude amax; 128 (E8M0
+// 0xFF, the NaN scale) when amax is not finite.
 __device__ __forceinline__ int mx_exponent(float amax) {
+    if (!(amax <= 3.402823466e38f)) return 128;
     return amax > 0.f ? min(127, max(-127, ilogbf(amax) - 2)) : -127;
+}
+
+// Value of the MXFP4 scale 2^X (NaN for X = 128).
+__device__ __forceinline__ float mx_scale(int X) {
+    return X > 127 ? __int_as_float(0x7fc00000) : ldexpf(1.f, X);
 }
 
 // |v| -> E2M1 magnitude code, nearest, ties to the even code, saturating.
@@ -58,8 +80,10 @@ __device__ __forceinline__ uint32_t e2m1_code(float a) {
     return c;
 }
 
-// MXFP4 element code (bit 3 = sign) of x in a group with exponent X.
+// MXFP4 element code (bit 3 = sign) of x in a group with exponent X (0 in a
+// NaN-scaled group).
 __device__ __forceinline__ uint32_t mx_code(float x, int X) {
+    if (X > 127) return 0u;
     return e2m1_code(fabsf(ldexpf(x, -X))) | (x < 0.f ? 8u : 0u);
 }
 
@@ -72,8 +96,9 @@ __device__ __forceinline__ float e2m1_value(uint32_t code) {
     return (code & 8u) ? -v : v;
 }
 
-// FP8 E4M3 code of x (zero stored as +0).
+// FP8 E4M3 code of x (zero stored as +0, NaN and +-inf as the NaN 0x7F).
 __device__ __forceinline__ uint32_t fp8_code(float x) {
+    if (!(fabsf(x) <= 3.402823466e38f)) return 0x7Fu;
     return x == 0.f ? 0u : static_cast<uint32_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
 }
 
@@ -116,7 +141,7 @@ __device__ __forceinline__ void quantize_query(float (&f)[16], float (&qs)[2]) {
     }
     float am[2] = {0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < 16; ++i) am[i >> 3] = fmaxf(am[i >> 3], fabsf(f[i]));
+    for (int i = 0; i < 16; ++i) am[i >> 3] = fmaxf(am[i >> 3], poison_abs(f[i]));
     if (FMT == SPOT_SEL_INT8_F16) am[0] = am[1] = fmaxf(am[0], am[1]);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -129,7 +154,7 @@ __device__ __forceinline__ void quantize_query(float (&f)[16], float (&qs)[2]) {
             const int X = mx_exponent(am[h]);
 #pragma unroll
             for (int i = 8 * h; i < 8 * h + 8; ++i) f[i] = e2m1_value(mx_code(f[i], X));
-            qs[h] = ldexpf(1.f, X);
+            qs[h] = mx_scale(X);
         } else {
             const bool i8 = FMT == SPOT_SEL_INT8_F16;
             const float sc = f16_bits_value(f16_scale_bits(am[h], i8 ? 127.0 : 7.0));

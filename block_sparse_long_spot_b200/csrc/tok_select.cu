@@ -224,7 +224,7 @@ __device__ __forceinline__ float load_tok_queries(const uint16_t* q_idx, int b, 
                 for (int e = 0; e < 2; ++e) {
                     const uint16_t bits = real ? __ldg(qrow + query_dim<FMT>(ks, j, e, c4)) : 0;
                     v[ks][j][e] = __uint_as_float(static_cast<uint32_t>(bits) << 16);
-                    am = fmaxf(am, fabsf(v[ks][j][e]));
+                    am = fmaxf(am, poison_abs(v[ks][j][e]));
                 }
         if (quantize) {
             // per-group (4-bit: ks = 2 c, 2 c + 1 hold dims 32 c ..) or per-head scales
@@ -238,7 +238,7 @@ __device__ __forceinline__ float load_tok_queries(const uint16_t* q_idx, int b, 
 #pragma unroll
                         for (int j = 0; j < 2; ++j)
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) ga = fmaxf(ga, fabsf(v[2 * c + t][j][e]));
+                            for (int e = 0; e < 2; ++e) ga = fmaxf(ga, poison_abs(v[2 * c + t][j][e]));
                 } else {
                     ga = am;
                 }
@@ -280,7 +280,7 @@ __device__ __forceinline__ float load_tok_queries(const uint16_t* q_idx, int b, 
                 float s = 1.f;
                 if constexpr (FMT == SPOT_SEL_INT4_G32_F16) s = f16_bits_value(f16_scale_bits(gs[c], 7.0));
                 else if constexpr (FMT == SPOT_SEL_INT8_F16) s = f16_bits_value(f16_scale_bits(gs[0], 127.0));
-                else if constexpr (FMT == SPOT_SEL_MXFP4_G32_E8M0) s = ldexpf(1.f, mx_exponent(gs[c]));
+                else if constexpr (FMT == SPOT_SEL_MXFP4_G32_E8M0) s = mx_scale(mx_exponent(gs[c]));
                 qs[c][0] = __shfl_sync(0xffffffffu, s, 4 * (2 * c4));
                 qs[c][1] = __shfl_sync(0xffffffffu, s, (4 * (2 * c4 + 1)) & 31);
             }
@@ -533,7 +533,7 @@ __global__ void __launch_bounds__(128) tok_append_kernel(const TokAppendParams p
     }
     float am = 0.f;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) am = fmaxf(am, fabsf(f[k]));
+    for (int k = 0; k < 16; ++k) am = fmaxf(am, poison_abs(f[k]));
     uint8_t* codes = static_cast<uint8_t*>(p.sel_data);
     if (p.fmt == SPOT_SEL_FP8_E4M3 || p.fmt == SPOT_SEL_INT8_F16) {
         uint32_t out[4] = {0u, 0u, 0u, 0u};

@@ -11,7 +11,7 @@
  * Long-Context Transformers" (arXiv HTML).  Each function names the section
  * or equation it follows.  Everything is computed in fp64 with plain loops,
  * in the order the definitions state; the only library primitives are exp(),
- * log(), frexp()/ldexp() and qsort().
+ * log(), frexp()/ldexp(), isfinite() and qsort().
  *
  * Readings taken where the paper is silent:
  *  - one selector key per (block, KV head); the index heads of a KV head are
@@ -37,7 +37,14 @@
  *    byte per element and no scale (8 bits = 0.5x bf16, App. G Tab. 9),
  *    round to nearest even, saturating at +-448;
  *  - INT8 keys: symmetric, one binary16 scale per key = fp16_rne(amax/127)
- *    (saturating at 65504), code = clamp(rne(x/scale), -128, 127).
+ *    (saturating at 65504), code = clamp(rne(x/scale), -128, 127);
+ *  - non-finite inputs: OCP MX v1.0 gives a block that holds a NaN or an
+ *    infinity the NaN shared scale.  The same rule is taken for every scaled
+ *    format: a scale group (32 elements for INT4 / MXFP4, the whole key for
+ *    INT8) holding NaN or +-inf stores the NaN scale (E8M0 0xFF, binary16
+ *    0x7E00) and all-zero codes, so it reads back as NaN; FP8 stores a NaN or
+ *    +-inf element as the E4M3 NaN 0x7F.  The selector score's ReLU maps an
+ *    undefined (NaN) dot product to 0.
  *
  * Parity status: every function here is pinned by tests/test_oracle_pins.py
  * (hand-worked examples, brute force, closed forms, library special cases).
@@ -130,8 +137,9 @@ static double e4m3_to_f64(uint8_t code) {
 }
 
 /* fp64 -> E4M3, round to nearest even, magnitudes beyond 448 saturate to
- * 448 (the largest finite E4M3). */
+ * 448 (the largest finite E4M3); NaN and +-inf become the NaN 0x7F. */
 static uint8_t f64_to_e4m3_sat(double x) {
+    if (!isfinite(x)) return 0x7F;
     uint8_t sign = (x < 0.0) ? 0x80 : 0x00;
     double a = fabs(x);
     if (a >= 448.0) return sign | 0x7E;
@@ -191,6 +199,10 @@ int oracle_dequant_selector(int fmt, int64_t rows, int ds, const void* data,
     return 0;
 }
 
+/* binary16 quiet NaN: the scale of an INT4 group or INT8 key that holds a
+ * NaN or an infinity. */
+#define F16_NAN_BITS ((uint16_t)0x7E00)
+
 /* Round |a| to the E2M1 grid, nearest, ties to the even code, saturating
  * at 6.  Returns the 3-bit magnitude code. */
 static unsigned e2m1_rne_code(double a) {
@@ -226,9 +238,16 @@ int oracle_quantize_selector(int fmt, int64_t rows, int ds, const uint16_t* keys
         }
         if (fmt == ORC_FMT_INT8) {
             double amax = 0.0;
+            int finite = 1;
             for (int i = 0; i < ds; ++i) {
                 double x = fabs(bf16_to_f64(row[i]));
-                if (x > amax) amax = x;
+                if (!isfinite(x)) finite = 0;
+                else if (x > amax) amax = x;
+            }
+            if (!finite) {                         /* NaN scale, zero codes */
+                ((uint16_t*)scales)[r] = F16_NAN_BITS;
+                memset((int8_t*)data + r * ds, 0, (size_t)ds);
+                continue;
             }
             uint16_t sbits = f64_to_f16_sat(amax / 127.0);
             ((uint16_t*)scales)[r] = sbits;
@@ -249,9 +268,20 @@ int oracle_quantize_selector(int fmt, int64_t rows, int ds, const uint16_t* keys
         memset(out, 0, (size_t)ds / 2);
         for (int g = 0; g < ds / 32; ++g) {
             double amax = 0.0;
+            int finite = 1;
             for (int i = 0; i < 32; ++i) {
                 double x = fabs(bf16_to_f64(row[g * 32 + i]));
-                if (x > amax) amax = x;
+                if (!isfinite(x)) finite = 0;
+                else if (x > amax) amax = x;
+            }
+            if (!finite) {                         /* NaN scale; the codes stay 0 */
+                if (fmt == ORC_FMT_INT4)
+                    ((uint16_t*)scales)[r * (ds / 32) + g] = F16_NAN_BITS;
+                else if (fmt == ORC_FMT_MXFP4)
+                    ((uint8_t*)scales)[r * (ds / 32) + g] = 0xFF;
+                else
+                    return -1;
+                continue;
             }
             if (fmt == ORC_FMT_INT4) {
                 uint16_t sbits = f64_to_f16_sat(amax / 7.0);

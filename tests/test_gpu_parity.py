@@ -88,16 +88,21 @@ def test_integer_inputs_quantised_queries_select_bit_exact(fmt):
 
 
 @pytest.mark.parametrize("fmt", ["int4", "mxfp4", "fp8", "int8"])
-def test_quantised_queries_tiny(fmt):
-    wl = workloads.make("tiny_4k", seed=3, device=DEV, sel_fmt=fmt)
+def test_quantised_queries_small(fmt):
+    # 4 sequences x 8 KV heads = 32 units of real-valued scores: units may
+    # differ only by blocks next to the cut (the near-cut rule checks each),
+    # and every unit whose selection agrees has its outputs compared.
+    wl = workloads.make("qwen3_4b_32k", seed=3, device=DEV, sel_fmt=fmt, seq_len=4096, batch=4)
     gpu = run_gpu(wl, fmt, quantize_queries=True)
     assert gpu["status"] == 0
     scores = oracle_scores(wl, fmt, quantize_queries=True)
     assert not np.allclose(scores, oracle_scores(wl, fmt), equal_nan=True)
     ora = run_oracle(wl, fmt, quantize_queries=True)
-    assert check_selection_near_cut(gpu, ora, scores, wl) <= 1
+    units = wl.batch * wl.num_kv_heads
+    n_diff = check_selection_near_cut(gpu, ora, scores, wl)
+    assert n_diff <= 2
     _, _, n = check_outputs(gpu, ora, wl)
-    assert n >= wl.batch * wl.num_kv_heads - 1
+    assert n == units - n_diff
 
 
 def test_integer_inputs_topk_and_kmin_modes():
@@ -127,13 +132,27 @@ def test_append_matches_oracle_quantiser(fmt):
 
 
 def test_append_extreme_values_match_oracle():
-    # Zeros, tiny subnormal-range, huge and mixed-sign groups.
-    rows = 64
-    x = torch.randn(rows, 1, 64) * torch.logspace(-40, 38, rows)[:, None, None]
+    # Zeros, subnormal-range, huge and mixed-sign groups from a seeded draw,
+    # plus rows that hold +-inf and NaN explicitly: both quantisers follow
+    # the same rule for them (a NaN scale and zero codes for the group, the
+    # E4M3 NaN for an FP8 element), so the pools must be bit-identical.
+    rows = 72
+    gen = torch.Generator().manual_seed(20)
+    x = torch.randn(rows, 1, 64, generator=gen) * torch.logspace(-40, 37, rows)[:, None, None]
     x[0] = 0.0
     x[1, 0, :32] = 0.0
     x[2, 0, 5] = 3.0e38
     x[3] = -x[3].abs()
+    x[64, 0, 7] = float("inf")                       # group 0 only
+    x[65, 0, 40] = float("-inf")                     # group 1 only
+    x[66, 0, 0] = float("nan")
+    x[67, 0, 33] = float("nan")
+    x[67, 0, 2] = float("inf")                       # both groups
+    x[68] = 3.3895313892515355e38                    # the bf16 maximum everywhere
+    x[68, 0, 1::2] *= -1
+    x[69] = 2.0 ** -130                              # bf16 subnormals only
+    x[70, 0, :] = torch.linspace(-1e-38, 1e-38, 64)
+    x[71, 0, ::3] = float("nan")
     keys = x.to(torch.bfloat16).to(DEV)
     pt = torch.arange(rows, dtype=torch.int32, device=DEV).view(1, rows)
     for fmt in ("int4", "mxfp4", "fp8", "int8"):
@@ -149,6 +168,32 @@ def test_append_extreme_values_match_oracle():
             sc = sc.view(torch.int16).numpy().view(np.uint16) if fmt in ("int4", "int8") \
                 else sc.numpy()
             assert np.array_equal(sc, o_scales), fmt
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "fp8", "int8"])
+@pytest.mark.parametrize("qq", [False, True])
+def test_nonfinite_selector_inputs_select_like_oracle(fmt, qq):
+    # Selector keys holding +-inf / NaN are stored with a NaN scale (or the
+    # E4M3 NaN), and a query head holding NaN gives NaN dot products: the
+    # score's ReLU turns each undefined dot product into 0 on both sides, so
+    # with integer-valued inputs the selections must still be identical.
+    wl = workloads.make("qwen3_4b_32k", seed=21, device=DEV, integer=True, seq_len=4096, batch=2)
+    pt = wl.page_table.cpu().numpy()
+    poison = [(0, 3, 0, 5, float("inf")), (0, 10, 1, 40, float("-inf")),
+              (1, 7, 2, 0, float("nan")), (1, 20, 3, 33, float("nan")),
+              (1, 21, 3, 2, float("inf"))]
+    for b, j, g, d, v in poison:
+        wl.sel_keys[int(pt[b, j]), g, d] = v
+    wl.q_sel[1, 5, 17] = float("nan")                # one index head of KV head 1
+    wl.top_p = safe_top_p(wl, fmt, quantize_queries=qq)
+    scores = oracle_scores(wl, fmt, quantize_queries=qq)
+    for b, j, g, _, _ in poison:
+        assert scores[b, g, j] == 0.0
+    gpu = run_gpu(wl, fmt, quantize_queries=qq)
+    assert gpu["status"] == 0
+    ora = run_oracle(wl, fmt, quantize_queries=qq)
+    _assert_same_selection(gpu, ora, wl)
+    check_outputs(gpu, ora, wl)
 
 
 def test_sparse_decode_on_oracle_selection():

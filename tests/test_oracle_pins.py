@@ -206,6 +206,50 @@ def test_encode_known_codes():
     assert scales[0].tolist() == [i4["scale_bits"], i4["scale_bits"]]
 
 
+def _codes_of(fmt, data):
+    """Element codes of one 64-element key row (signed for int4 / int8)."""
+    if fmt in ("int4", "mxfp4"):
+        c = [int(data[i // 2] >> (4 * (i % 2))) & 0xF for i in range(64)]
+        return [x - 16 if (fmt == "int4" and x >= 8) else x for x in c]
+    if fmt == "int8":
+        return data.view(np.int8).astype(int).tolist()
+    return data.astype(int).tolist()
+
+
+def test_nonfinite_and_extreme_groups():
+    # Hand-worked rows (tests/golden/selector_codes.json): a group holding NaN
+    # or an infinity gets the NaN scale and zero codes (OCP MX's rule, read
+    # for every scaled format), FP8 stores such an element as its NaN, and the
+    # bf16 maximum / subnormal range land where the format definitions say.
+    for case in _golden("selector_codes.json")["nonfinite_and_extremes"]["cases"]:
+        fmt = case["fmt"]
+        bits = np.zeros(64, np.uint16)
+        for i, b in case["set"]:
+            bits[i] = b
+        data, scales = oracle.quantize_selector(fmt, bits[None])
+        want = [0] * 64
+        for i, c in case["codes"]:
+            want[i] = c
+        assert _codes_of(fmt, data[0]) == want, case["note"]
+        if case["scales"] is None:
+            assert scales is None
+        else:
+            assert scales[0].tolist() == case["scales"], case["note"]
+        # a poisoned group reads back as NaN, every other element as finite
+        back = oracle.dequant_selector(fmt, data, scales, 64)[0]
+        nonfinite = np.zeros(64, bool)
+        for i, b in case["set"]:
+            if (b & 0x7F80) == 0x7F80:
+                nonfinite[i] = True
+        if fmt == "fp8":
+            poisoned = nonfinite
+        elif fmt == "int8":
+            poisoned = np.full(64, nonfinite.any())
+        else:
+            poisoned = np.repeat(nonfinite.reshape(2, 32).any(1), 32)
+        assert np.isnan(back[poisoned]).all() and np.isfinite(back[~poisoned]).all(), case["note"]
+
+
 def test_int4_scale_is_binary16_rne():
     # The scale is amax/7 rounded to the nearest binary16 (numpy's IEEE
     # conversion is the independent reference), saturating at 65504.
