@@ -164,9 +164,28 @@ def layer_seed(rank: int, layer: int) -> int:
     return 1000 * rank + layer
 
 
+def rank_sequences(batch_total: int, world: int, rank: int) -> list:
+    """Sequences of a global batch that rank `rank` decodes: a contiguous
+    share, the first batch_total % world ranks one more (data parallel over
+    sequences; no sequence is split, so no rank needs another's data)."""
+    base, extra = divmod(batch_total, world)
+    lo = rank * base + min(rank, extra)
+    return list(range(lo, lo + base + (1 if rank < extra else 0)))
+
+
 def shard_summary(batch_per_rank: int, world: int, ms_step_max: float, layers_model: int):
     """Whole-job decode throughput: tokens of all ranks over the slowest rank."""
     return batch_per_rank * world / (ms_step_max / 1e3 * layers_model)
+
+
+def bench_metric(workload: str) -> str:
+    """The metric line of a decode workload (the headline names L = 128K)."""
+    if workload == "ragged_hybrid":
+        return ("decode tokens/s, ragged L ~ U[8K, 128K] (whole model = per-layer step x "
+                "sparse layers)")
+    if workload == "qwen3_4b_32k":
+        return "decode tokens/s at L=32K (whole model = per-layer step x sparse layers)"
+    return "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)"
 
 
 def unit_counts(wl):
@@ -395,7 +414,7 @@ def run_spot(args, world, rank, local):
     value_e2e = shard_summary(B, world, ms_e2e, layers_model)
     achieved = b_sparse / (dec_ms / 1e3) / 1e9
     res = {
-        "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
+        "metric": bench_metric(args.workload),
         "value": round(value, 3),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -608,7 +627,7 @@ def run_spot_tok(args, world, rank, local):
     kb, kms = (b_sparse, dec_ms) if dom_sparse else (b_select, sel_ms)
     achieved = kb / (kms / 1e3) / 1e9
     return {
-        "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
+        "metric": bench_metric(args.workload),
         "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "us_per_layer": round(ms_step * 1e3, 2), "higher_is_better": True, "scaling": "weak",
@@ -942,60 +961,131 @@ def time_oracle(prep, units=None):
     return time.perf_counter() - t
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class OracleSampler:
+    """Bounded samples of one layer for the fp64 oracle: a sample is the
+    decode step (scoring, selection, attention) of `per` consecutive
+    (sequence, KV head) units of the layer, walking round the layer's units
+    from sample to sample.  Host copies are made outside the timed calls and
+    kept for the last sequences touched."""
+
+    def __init__(self, wl, fmt, per):
+        self.wl, self.fmt = wl, fmt
+        self.U = wl.batch * wl.num_kv_heads
+        self.per = max(1, min(per, self.U))
+        self.next = 0
+        self.cache = {}
+
+    def _prep(self, seqs):
+        key = tuple(seqs)
+        if key not in self.cache:
+            self.cache.clear()                    # one sample's sequences on the host at a time
+            self.cache[key] = prepare_oracle(self.wl, self.fmt, seqs)
+        return self.cache[key]
+
+    def take(self):
+        """Runs the next sample; returns (seconds, units run)."""
+        Hkv = self.wl.num_kv_heads
+        units = [(self.next + k) % self.U for k in range(self.per)]
+        self.next = (self.next + self.per) % self.U
+        seqs = sorted({u // Hkv for u in units})
+        local = [seqs.index(u // Hkv) * Hkv + u % Hkv for u in units]
+        return time_oracle(self._prep(seqs), units=local), len(units)
+
+
 def cpu_baseline(wl, fmt, min_s=10.0, max_s=30.0):
-    """The fp64 oracle on the host cores, one sequence of the layer at a time
-    (all its KV heads in parallel), repeated over the sequences until about
-    10 s of work; scaled to the whole layer and the model's layers."""
+    """The fp64 oracle on the host: samples of as many (sequence, KV head)
+    units as there are cores, run in parallel over the units on every core
+    until about min_s of work, then single units on one core; the rate in
+    units per second becomes decode tokens/s of the model (one token of a
+    sequence = its Hkv units in every sparse layer)."""
     import oracle
-    total, n = 0.0, 0
-    while total < min_s and n < 64:
-        prep = prepare_oracle(wl, fmt, [n % wl.batch])
-        total += time_oracle(prep)
-        n += 1
+    cores = host_cores()
+    units_per_token = wl.num_kv_heads * wl.spec.layers_sparse
+    smp = OracleSampler(wl, fmt, cores)
+    oracle.set_num_threads(cores)
+    total, done = 0.0, 0
+    while total < min_s and done < 64 * smp.U:
+        sec, n = smp.take()
+        total += sec
+        done += n
         if total > max_s:
             break
-    per_seq = total / n
-    value = wl.batch / (per_seq * wl.batch * wl.spec.layers_sparse)
-    return {"value": round(value, 6), "unit": "tokens/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"fp64 oracle decode step of one sequence (all {wl.num_kv_heads} KV heads) "
-                      f"of the layer, {n} runs over the batch, {total:.1f} s; "
-                      f"x{wl.batch} sequences x{wl.spec.layers_sparse} layers"}
+    rate_all = done / total
+    one = OracleSampler(wl, fmt, 1)
+    oracle.set_num_threads(1)
+    t1, d1 = 0.0, 0
+    while t1 < min_s / 2 and d1 < smp.U:
+        sec, n = one.take()
+        t1 += sec
+        d1 += n
+    rate_one = d1 / t1
+    oracle.set_num_threads(cores)
+    return {"value": round(rate_all / units_per_token, 6), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle", "cpu": cpu_model(),
+            "single_thread": {"value": round(rate_one / units_per_token, 6), "cores": 1,
+                              "sample": f"{d1} units one at a time, {t1:.1f} s"},
+            "sample": f"fp64 oracle decode step (scoring, selection, attention) over {done} "
+                      f"(sequence, KV head) units of the layer in samples of {smp.per} units "
+                      f"run in parallel on {cores} threads, {total:.1f} s; tokens/s = "
+                      f"units/s / ({wl.num_kv_heads} KV heads x {wl.spec.layers_sparse} sparse "
+                      f"layers)"}
 
 
 def run_reference(args, world, rank):
     """The fp64 CPU oracle as the reference arm, on the same workload: each
-    step times one (sequence, KV head) unit of the layer on the host cores
-    and scales by the layer's units and the model's layers."""
+    step is one bounded sample of the layer -- the decode step of as many
+    (sequence, KV head) units as the host has cores, in parallel on all of
+    them -- walking round the layer's units; tokens/s = units per second /
+    (KV heads x sparse layers), ms_per_step the measured time of one sample."""
     if rank != 0:
         return None
     import oracle
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wl = workloads.make(args.workload, seed=0, device=dev, sel_fmt=args.sel_fmt)
-    B, Hkv = wl.batch, wl.num_kv_heads
-    preps = {}
-    times = []
+    cores = host_cores()
+    oracle.set_num_threads(cores)
+    smp = OracleSampler(wl, args.sel_fmt, cores)
+    secs, units = [], 0
     for i in range(args.warmup + args.steps):
-        b, g = (i // Hkv) % B, i % Hkv
-        if b not in preps:
-            preps[b] = prepare_oracle(wl, args.sel_fmt, [b])
-        sec = time_oracle(preps[b], units=[g])
+        sec, n = smp.take()
         if i >= args.warmup:
-            times.append(sec)
-    per_layer = float(np.mean(times)) * B * Hkv
-    value = B / (per_layer * wl.spec.layers_sparse)
-    sample = (f"one (sequence, KV head) unit of the layer per step, rotating over all "
-              f"{B * Hkv}; x{B * Hkv} units x{wl.spec.layers_sparse} layers")
+            secs.append(sec)
+            units += n
+    total = float(sum(secs))
+    units_per_token = wl.num_kv_heads * wl.spec.layers_sparse
+    value = units / total / units_per_token
+    sample = (f"each step: the fp64 oracle decode step of {smp.per} consecutive (sequence, KV head) "
+              f"units of the {smp.U}-unit layer, in parallel on {cores} threads, walking round "
+              f"the layer; tokens/s = units/s / ({wl.num_kv_heads} KV heads x "
+              f"{wl.spec.layers_sparse} sparse layers)")
     return {
         "impl": "reference",
-        "metric": "decode tokens/s at L=128K (whole model = per-layer step x sparse layers)",
+        "metric": bench_metric(args.workload),
         "value": round(value, 6), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(per_layer * 1e3, 3),
+        "warmup": args.warmup, "ms_per_step": round(total / len(secs) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 with planted hot blocks)",
         "config": {"workload": args.workload, "sel_fmt": args.sel_fmt, "sample": sample},
-        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s",
-                         "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle", "cpu": cpu_model(), "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -90,6 +90,8 @@ def _load():
         lib.oracle_prefill_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, dbl, P, i32,
                                             P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -104,6 +106,11 @@ def _c(a, dtype):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Threads for later oracle calls; returns the count in effect."""
+    return int(_load().oracle_set_num_threads(int(n)))
 
 
 def make_shape(batch, num_q_heads, num_kv_heads, head_dim, block_size, sel_dim, sel_fmt,

@@ -1044,3 +1044,16 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* Sets the number of OpenMP threads later calls use (n >= 1); returns the
+ * count in effect.  Lets one process time the oracle on every host core and
+ * on one. */
+int oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
