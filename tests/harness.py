@@ -472,18 +472,48 @@ def check_prefill_selection_near_cut(gpu, ora, scores, wl, tiles=None, kmin=None
     return n_diff
 
 
+P_ROUND = 2.0 ** -9          # relative rounding of a softmax weight stored as bf16
+
+
+def prefill_weighted_abs_v(wl, ora, t, g):
+    """sum_i w_i |v_i| per (query row, head, dim) of tile t, KV head g, with
+    w the exact (fp64) causal softmax weights over the tile's selected
+    tokens: the scale of the error that rounding the weights to bf16 before
+    P.V can cause (reading r21 of the design notes)."""
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    b, lo, hi, r0 = info[t]
+    G = wl.num_q_heads // wl.num_kv_heads
+    sel = ora["sel_idx"][t, g, :ora["sel_cnt"][t, g]]
+    pt = wl.page_table[b].cpu().numpy()
+    pos = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in sel]) if len(sel) else \
+        np.zeros(0, np.int64)
+    pos = pos[pos <= hi]
+    pages = torch.as_tensor(pt[pos // 64].astype(np.int64))
+    rows_in = torch.as_tensor(pos % 64)
+    k = wl.k_pool[pages.to(wl.k_pool.device), g, rows_in.to(wl.k_pool.device)].double().cpu()
+    v = wl.v_pool[pages.to(wl.v_pool.device), g, rows_in.to(wl.v_pool.device)].double().cpu()
+    q = wl.q[r0:r0 + hi - lo + 1, g * G:(g + 1) * G].double().cpu()      # [rows, G, D]
+    logits = torch.einsum("rhd,kd->rhk", q, k) * wl.sm_scale
+    qpos = torch.arange(lo, hi + 1)[:, None, None]
+    logits = logits.masked_fill(torch.as_tensor(pos)[None, None, :] > qpos, float("-inf"))
+    w = torch.softmax(logits, dim=-1).nan_to_num(0.0)
+    return torch.einsum("rhk,kd->rhd", w, v.abs()).numpy()
+
+
 def check_prefill_outputs(gpu, ora, wl, tiles=None):
     """Element-wise check of the query rows of every (tile, KV head) whose
     selections agree; returns (max abs err, units compared).
 
-    Tolerance: the kernel rounds the softmax weights p to bf16 (relative
-    2^-9) before the P.V product, an output error of at most
-    2^-9 * sum_i p_i |v_i| / l <= 2^-9 * max |v|.  Decode rows average
-    hundreds of tokens and stay far inside ATOL; a prefill row near its
-    chunk's start may see a handful, so the bound itself is added."""
+    Tolerance (reading r21): the attention kernel rounds the softmax weights
+    to bf16 (relative 2^-9) before the P.V product and divides by the sum of
+    the unrounded weights, so an output element can move by up to
+    2^-9 * sum_i w_i |v_i| beyond the fp32 error the decode rule covers.  A
+    decode row averages hundreds of tokens, where this stays far inside the
+    2e-3 term; a prefill row near the start of a sequence may attend a
+    handful, so that bound, computed per element from the exact weights, is
+    added to the shared 2e-3 + 1e-2 |ref| rule."""
     info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
     G = wl.num_q_heads // wl.num_kv_heads
-    atol = ATOL + 2.0 ** -9 * float(wl.v_pool.abs().max().item())
     worst, n = 0.0, 0
     for t in (range(len(info)) if tiles is None else tiles):
         _, lo, hi, r0 = info[t]
@@ -494,7 +524,8 @@ def check_prefill_outputs(gpu, ora, wl, tiles=None):
             hs = slice(g * G, (g + 1) * G)
             o_g, o_r = gpu["out"][rows, hs], ora["out"][rows, hs]
             err = np.abs(o_g - o_r)
-            assert not (err > atol + RTOL * np.abs(o_r)).any(), (t, g, float(err.max()))
+            bound = ATOL + RTOL * np.abs(o_r) + P_ROUND * prefill_weighted_abs_v(wl, ora, t, g)
+            assert not (err > bound).any(), (t, g, float(err.max()))
             l_g, l_r = gpu["lse"][rows, hs], ora["lse"][rows, hs]
             fin = np.isfinite(l_r)
             assert np.array_equal(fin, np.isfinite(l_g)), (t, g)

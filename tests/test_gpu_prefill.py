@@ -9,8 +9,9 @@ import torch
 import block_sparse_long_spot_b200 as spot
 import oracle
 import workloads
-from harness import (check_prefill_outputs, check_prefill_selection_near_cut,
-                     oracle_prefill_scores, prefill_oracle_args, run_gpu_prefill,
+from harness import (ATOL, RTOL, P_ROUND, check_prefill_outputs,
+                     check_prefill_selection_near_cut, oracle_prefill_scores,
+                     prefill_weighted_abs_v, prefill_oracle_args, run_gpu_prefill,
                      run_oracle_prefill, safe_top_p_prefill, tile_selection)
 
 pytestmark = pytest.mark.gpu
@@ -45,6 +46,39 @@ def test_prefill_tiny():
     assert check_prefill_selection_near_cut(gpu, ora, scores, wl) <= 1
     _, n = check_prefill_outputs(gpu, ora, wl)
     assert n >= gpu["num_tiles"] * wl.num_kv_heads - 1
+
+
+def test_prefill_worst_rows_within_the_bf16_weight_bound():
+    # Whole sequences prefilled from position 0: the first rows attend 1, 2,
+    # ... keys, where rounding the softmax weights to bf16 weighs most.
+    # Every element must lie within 2e-3 + 1e-2 |ref| + 2^-9 sum_i w_i |v_i|
+    # (reading r21), and rows attending at least 256 keys within the plain
+    # decode rule 2e-3 + 1e-2 |ref|.
+    wl = workloads.make_prefill("prefill_tiny", seed=7, device=DEV, integer=True,
+                                seq_lens=[640, 130, 64], q_lens=[640, 130, 64])
+    wl.top_p = safe_top_p_prefill(wl)
+    gpu = run_gpu_prefill(wl)
+    assert gpu["status"] == 0
+    ora = run_oracle_prefill(wl)
+    _same(gpu, ora, wl)
+    info = oracle.prefill_tiles(wl.seq_lens.cpu().numpy(), wl.q_lens.cpu().numpy())
+    G = wl.num_q_heads // wl.num_kv_heads
+    worst_extra = 0.0
+    for t, (b, lo, hi, r0) in enumerate(info):
+        rows = slice(r0, r0 + hi - lo + 1)
+        for g in range(wl.num_kv_heads):
+            hs = slice(g * G, (g + 1) * G)
+            o_g, o_r = gpu["out"][rows, hs], ora["out"][rows, hs]
+            err = np.abs(o_g - o_r)
+            plain = ATOL + RTOL * np.abs(o_r)
+            assert (err <= plain + P_ROUND * prefill_weighted_abs_v(wl, ora, t, g)).all(), (t, g)
+            sel = ora["sel_idx"][t, g, :ora["sel_cnt"][t, g]]
+            keys = np.array([sum(min(64, max(0, pos - 64 * j + 1)) for j in sel)
+                             for pos in range(lo, hi + 1)])
+            many = keys >= 256
+            assert (err[many] <= plain[many]).all(), (t, g)
+            worst_extra = max(worst_extra, float((err - plain).max()))
+    print(f"largest excess over the decode rule: {worst_extra:.2e}")
 
 
 @pytest.mark.parametrize("lens,qlens", [
