@@ -39,12 +39,11 @@ import workloads  # noqa: E402
 
 HBM_FALLBACK_GBS = 6650.0
 
-# DRAM bytes (read + write) of one sparse-decode launch from an ncu capture of
-# the same workload (profiles/sparse_decode_kernel_qwen3_32b_128k.md), valid
-# only for the kernel source it was taken on (sha256 prefix of the .cu file).
+# DRAM bytes (read + write) of one launch of each workload's dominant kernel
+# (dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of the
+# same workload), valid only while the kernel's source files are unchanged
+# (sha256 prefix over them); otherwise the roofline's traffic is null.
 NCU_TRAFFIC = {
-    # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
-    # kernel (profiles/), valid while its source files are unchanged
     "qwen3_32b_128k": {"bytes": 728982528 + 3904768, "files": ["sparse_decode.cu"],
                        "sha256": "82c100300b60004f"},
     "qwen3_8b_128k_tok": {"bytes": 246840064 + 4134144, "files": ["sparse_decode.cu"],

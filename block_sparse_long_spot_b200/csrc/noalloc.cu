@@ -12,6 +12,8 @@
 // holds that array until the process exits.
 #include <math.h>
 
+#include <cuda.h>
+
 #include <mutex>
 
 #include "spot_internal.h"
@@ -24,20 +26,55 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch, resolved once per device with that
-// device current (in host code the symbol name is only a host-side handle).
+// Device address of g_noalloc_scratch, resolved with the device current (in
+// host code the symbol name is only a host-side handle) and remembered per
+// device together with the context it belongs to: after a cudaDeviceReset
+// the runtime makes a new primary context, the module is loaded again and
+// the array may sit elsewhere, so a changed context triggers a new lookup.
 std::mutex g_addr_mutex;
-void* g_addr[kMaxDevices] = {};
+struct ScratchSlot {
+    CUcontext ctx;
+    void* addr;
+};
+ScratchSlot g_slot[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry-point lookup (the
+// library does not link the driver library directly).
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    });
+    return fn;
+}
 
 cudaError_t scratch_address(int dev, void** out) {
+    const CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return cudaErrorNotSupported;
     std::lock_guard<std::mutex> lock(g_addr_mutex);
-    if (!g_addr[dev]) {
-        void* p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_addr[dev] = p;
+    CUcontext ctx = nullptr;
+    if (g_slot[dev].addr && get(&ctx) == CUDA_SUCCESS && ctx == g_slot[dev].ctx) {
+        *out = g_slot[dev].addr;
+        return cudaSuccess;
     }
-    *out = g_addr[dev];
+    // first call on this device, or its context changed: look the array up
+    // (this also makes the runtime's primary context current) and remember
+    // the context it was found in
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+    g_slot[dev].ctx = ctx;
+    g_slot[dev].addr = p;
+    *out = p;
     return cudaSuccess;
 }
 

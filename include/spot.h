@@ -209,12 +209,19 @@ spot_status_t spot_decode_step(const spot_layer_desc_t* desc, const spot_select_
  * the tensors of one call but no allocator, and so cannot provide the
  * workspace spot_sparse_decode takes.
  * Same arguments and results as spot_sparse_decode without the workspace.
- * The scratch (status word, per-unit offsets, split partials) is a static
- * device array of 8 MiB inside the library; every GPU that loads the library
- * holds it until the process exits.  The call allocates nothing.
+ * The scratch (status word, per-unit arrival counters, split partials) is a
+ * static device array of 8 MiB inside the library; every GPU that loads the
+ * library holds it until the process exits.  The call allocates nothing.
  *   - The first call on a device looks up that array's device address with
- *     the device current (cudaGetSymbolAddress) and remembers it; make that
- *     first call before any stream capture.
+ *     the device current (cudaGetSymbolAddress) and remembers it with the
+ *     device's current context; make that first call before any stream
+ *     capture.  A call that finds a different context (after a
+ *     cudaDeviceReset) looks the address up again, so it too must come
+ *     before any capture.
+ *   - Every call first zeroes the status word and the per-unit arrival
+ *     counters on `stream` (an asynchronous memset into the static array),
+ *     so an earlier call that timed out leaves no state behind; the split
+ *     partials are written before they are read.
  *   - A shape whose scratch exceeds 8 MiB returns SPOT_ERR_WORKSPACE (about
  *     (grid + U) * G * 528 bytes with U = batch * num_kv_heads and grid =
  *     the SM count; e.g. 256 units of G = 4 need 0.9 MB).
