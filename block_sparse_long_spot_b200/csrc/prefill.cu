@@ -118,17 +118,6 @@ constexpr int kScoreWarps = 8;
 constexpr int kScoreThreads = kScoreWarps * 32;
 constexpr int kKeyStride = 72;                 // bf16 per staged key row (64 + 8 pad)
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // Stage keys [j0, j0 + 64) of KV head g of sequence b (rows past n_full are
 // left as they are; their scores are not written).
 __device__ __forceinline__ void stage_keys(const PrefillParams& p, int b, int g, int j0,

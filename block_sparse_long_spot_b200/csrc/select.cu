@@ -49,157 +49,306 @@ namespace spot {
 namespace {
 
 constexpr int kSelectThreads = 512;
-constexpr int kFixShift = 40;
+constexpr int kFixShift = 40;           // masses are held as multiples of 2^-kFixShift
 constexpr int kMaxCluster = 8;          // scoring CTAs of one unit (a portable cluster)
-constexpr int kTileBatch = 2;           // 16-block tiles a warp scores with loads in flight
+constexpr int NT = kSelectThreads;
+constexpr int NW = NT / 32;
 
 // --------------------------------------------------------------- scoring
 
-// Scores of tiles t0, t0 + stride, ... (kTileBatch of them) of 16 blocks
-// each, for KV head g, into scores[j] (j < n_full), given the blocks' page
-// ids (load_pages).  qw: the group's selector queries as mma B fragments
-// (lane: head r8); wh0 / wh1: weights of heads 2 c4, 2 c4 + 1 (0 for
-// padding heads).
-// Page ids of the blocks of tiles t0, t0 + stride, ... (rows r8 and r8 + 8).
-__device__ __forceinline__ void load_pages(const SelectParams& p, int b, int t0, int stride,
-                                           int n_full, int lane, int (&pa)[kTileBatch],
-                                           int (&pb)[kTileBatch]) {
-    const int r8 = lane >> 2;
+// Selector rows are first gathered into shared memory with cp.async (every
+// row of a pass in flight at once: one round trip for the page ids, one for
+// the rows), then scored from there.  Row layout in shared memory per
+// format: bf16 rows of 128 bytes at a 144-byte stride (no bank conflicts in
+// the fragment loads); 8-bit code rows of 64 bytes; 4-bit code rows of 32
+// bytes whose two 16-byte halves swap places when bit 2 of the row index is
+// set (rows r and r + 4 then use different banks).  Scales go to a separate
+// array of one 32-bit word per row.
+template <int FMT>
+__host__ __device__ constexpr int row_bytes() {
+    return FMT == SPOT_SEL_BF16 ? 128
+           : (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) ? 64 : 32;
+}
+template <int FMT>
+__host__ __device__ constexpr int row_stride() {
+    return FMT == SPOT_SEL_BF16 ? 144 : row_bytes<FMT>();
+}
+template <int FMT>
+__host__ __device__ constexpr bool has_scales() {
+    return FMT == SPOT_SEL_INT4_G32_F16 || FMT == SPOT_SEL_MXFP4_G32_E8M0 ||
+           FMT == SPOT_SEL_INT8_F16;
+}
+constexpr int kMaxRowsPerThread = 8;    // rows one thread stages per pass
+
+// Byte offset of 16-byte piece h of staged row r.
+template <int FMT>
+__device__ __forceinline__ int piece_off(int r, int h) {
+    if (row_bytes<FMT>() == 32) return r * 32 + ((h ^ ((r >> 2) & 1)) << 4);
+    return r * row_stride<FMT>() + (h << 4);
+}
+
+// Cluster barrier halves (every thread of every CTA of the cluster arrives
+// once per phase): an arrival that orders nothing, and the wait for the
+// phase, so CTAs learn that all of the cluster has started.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
+
+// Issues the gathering of the selector rows of blocks j0 .. j0 + n - 1 of
+// sequence b, KV head g (page ids pg from stage_pages) into shared memory: row r goes to staging row r and
+// is copied by thread r % NT, in row group r / NT (one cp.async commit group
+// per row group, kMaxRowsPerThread groups always, empty ones included).  An
+// out-of-range page id is recorded and page 0 read instead.  The rows' scale
+// words are loaded into sc[] (stored by stage_wait).
+// Page ids of the rows this thread stages (loaded ahead, so that their
+// latency overlaps other loads).
+__device__ __forceinline__ void stage_pages(const SelectParams& p, int b, int j0, int n,
+                                            int (&pg)[kMaxRowsPerThread]) {
 #pragma unroll
-    for (int k = 0; k < kTileBatch; ++k) {
-        const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
-        pa[k] = (ja < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + ja] : 0;
-        pb[k] = (jb < n_full) ? p.page_table[static_cast<int64_t>(b) * p.pt_stride + jb] : 0;
+    for (int k = 0; k < kMaxRowsPerThread; ++k) {
+        const int r = threadIdx.x + k * NT;
+        pg[k] = r < n ? __ldg(p.page_table + static_cast<int64_t>(b) * p.pt_stride + j0 + r) : 0;
     }
 }
 
 template <int FMT>
-__device__ __forceinline__ void score_tiles(const SelectParams& p, int g,
-                                            const uint32_t (&qw)[8], const float (&qsc)[2][2],
-                                            float wh0, float wh1, int t0, int stride, int n_full, float* scores,
-                                            int lane, const int (&pga)[kTileBatch],
-                                            const int (&pgb)[kTileBatch], int r0, int r1,
-                                            float& wmax, float& wmin) {
+__device__ __forceinline__ void stage_issue(const SelectParams& p, int g, int n,
+                                            const int (&pg)[kMaxRowsPerThread], uint8_t* stg,
+                                            uint32_t (&sc)[kMaxRowsPerThread]) {
+    const uint32_t st = smem_u32(stg);
+#pragma unroll
+    for (int k = 0; k < kMaxRowsPerThread; ++k) {
+        const int r = threadIdx.x + k * NT;
+        sc[k] = 0u;
+        if (r < n) {
+            int pa = pg[k];
+            if (pa < 0 || pa >= p.num_pages) {
+                flag_status(p.status, kStatusBounds);
+                pa = 0;
+            }
+            const int64_t row = static_cast<int64_t>(pa) * p.num_kv_heads + g;
+            const uint8_t* src = static_cast<const uint8_t*>(p.sel_data) + row * row_bytes<FMT>();
+#pragma unroll
+            for (int h = 0; h < row_bytes<FMT>() / 16; ++h)
+                cp_async16(st + piece_off<FMT>(r, h), src + 16 * h);
+            if (FMT == SPOT_SEL_INT4_G32_F16)
+                sc[k] = __ldg(reinterpret_cast<const uint32_t*>(p.sel_scales) + row);
+            else if (FMT == SPOT_SEL_MXFP4_G32_E8M0 || FMT == SPOT_SEL_INT8_F16)
+                sc[k] = __ldg(reinterpret_cast<const uint16_t*>(p.sel_scales) + row);
+        }
+        cp_async_commit();
+    }
+}
+
+// Waits until row group k (rows k NT .. k NT + NT - 1) has landed for every
+// thread, its scale words stored; returns behind a barrier.
+template <int FMT>
+__device__ __forceinline__ void stage_wait(int k, int n, const uint32_t (&sc)[kMaxRowsPerThread],
+                                           uint32_t* stg_sc) {
+    switch (kMaxRowsPerThread - 1 - k) {           // groups after k may still be in flight
+        case 7: cp_async_wait<7>(); break;
+        case 6: cp_async_wait<6>(); break;
+        case 5: cp_async_wait<5>(); break;
+        case 4: cp_async_wait<4>(); break;
+        case 3: cp_async_wait<3>(); break;
+        case 2: cp_async_wait<2>(); break;
+        case 1: cp_async_wait<1>(); break;
+        default: cp_async_wait<0>(); break;
+    }
+    static_assert(kMaxRowsPerThread == 8, "stage_wait covers eight groups");
+    if (has_scales<FMT>()) {
+        const int r = threadIdx.x + k * NT;
+#pragma unroll
+        for (int kk = 0; kk < kMaxRowsPerThread; ++kk)
+            if (kk == k && r < n) stg_sc[r] = sc[kk];
+    }
+    __syncthreads();
+}
+
+// Selector queries of head group g for the quantised-key scorer, as f16 mma
+// B fragments (lane: head r8) in the pairing that the exact code widening
+// of quant.cuh produces: 4-bit keys give a lane the element pairs (j, j + 4)
+// of its 8 dims per group, so qf[4 grp + 2 s] = dims (8 c4 + 2 s, + 4) and
+// qf[4 grp + 2 s + 1] = dims (8 c4 + 2 s + 1, + 5) of group grp (plus 32
+// grp); 8-bit keys give pairs (2 i, 2 i + 1) of dims [16 c4, 16 c4 + 16).
+// Queries that are not quantised are scaled by 2^sh per head so that the
+// largest |q| lies in [2^14, 2^15) (every bf16 query value then converts to
+// f16 exactly unless it is below 2^-29 of its head's largest); quantised
+// queries are their codes, exact in f16.  qsc[half][col] receives the
+// scale that undoes either (2^-sh, or the query's group / head scale) for
+// the heads of columns 2 c4, 2 c4 + 1.
+template <int FMT>
+__device__ __forceinline__ void load_queries_f16(const SelectParams& p, int b, int g, int lane,
+                                                 uint32_t (&qf)[8], float (&qsc)[2][2],
+                                                 float& wh0, float& wh1) {
+    constexpr bool four = FMT == SPOT_SEL_INT4_G32_F16 || FMT == SPOT_SEL_MXFP4_G32_E8M0;
     const int c4 = lane & 3, r8 = lane >> 2;
-    int64_t rowa[kTileBatch], rowb[kTileBatch];
-#pragma unroll
-    for (int k = 0; k < kTileBatch; ++k) {
-        int pa = pga[k], pb = pgb[k];
-        if (pa < 0 || pa >= p.num_pages) { flag_status(p.status, kStatusBounds); pa = 0; }
-        if (pb < 0 || pb >= p.num_pages) { flag_status(p.status, kStatusBounds); pb = 0; }
-        rowa[k] = static_cast<int64_t>(pa) * p.num_kv_heads + g;
-        rowb[k] = static_cast<int64_t>(pb) * p.num_kv_heads + g;
+    const int G = p.group;
+    const bool real = r8 < G;
+    const int h = g * G + (real ? r8 : 0);
+    const uint4* q4 = reinterpret_cast<const uint4*>(p.q_sel + (static_cast<int64_t>(b) * p.num_q_heads + h) * kSelDim);
+    uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
+    if (real) {
+        x0 = __ldg(q4 + (four ? c4 : 2 * c4));
+        x1 = __ldg(q4 + (four ? 4 + c4 : 2 * c4 + 1));
     }
-    float acc[kTileBatch][4];
-    if (FMT == SPOT_SEL_BF16) {
-        uint4 a0[kTileBatch], a1[kTileBatch], b0[kTileBatch], b1[kTileBatch];
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    float f[16];
 #pragma unroll
-        for (int k = 0; k < kTileBatch; ++k) {
-            const uint4* ka = reinterpret_cast<const uint4*>(p.sel_data) + rowa[k] * 8 + 2 * c4;
-            const uint4* kb = reinterpret_cast<const uint4*>(p.sel_data) + rowb[k] * 8 + 2 * c4;
-            a0[k] = __ldg(ka);
-            a1[k] = __ldg(ka + 1);
-            b0[k] = __ldg(kb);
-            b1[k] = __ldg(kb + 1);
-        }
-#pragma unroll
-        for (int k = 0; k < kTileBatch; ++k) {
-            const uint32_t wa[8] = {a0[k].x, a0[k].y, a0[k].z, a0[k].w,
-                                    a1[k].x, a1[k].y, a1[k].z, a1[k].w};
-            const uint32_t wb[8] = {b0[k].x, b0[k].y, b0[k].z, b0[k].w,
-                                    b1[k].x, b1[k].y, b1[k].z, b1[k].w};
-            acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16_16816(acc[k], wa[2 * s], wb[2 * s], wa[2 * s + 1], wb[2 * s + 1],
-                               qw[2 * s], qw[2 * s + 1]);
-        }
-    } else if (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
-        // 64-byte rows: lane c4 owns bytes (= dims) [16 c4, 16 c4 + 16)
-        uint4 ra[kTileBatch], rb[kTileBatch];
-        float sca[kTileBatch], scb[kTileBatch];
-#pragma unroll
-        for (int k = 0; k < kTileBatch; ++k) {
-            ra[k] = __ldg(reinterpret_cast<const uint4*>(p.sel_data) + rowa[k] * 4 + c4);
-            rb[k] = __ldg(reinterpret_cast<const uint4*>(p.sel_data) + rowb[k] * 4 + c4);
-            if (FMT == SPOT_SEL_INT8_F16) {
-                sca[k] = __half2float(reinterpret_cast<const __half*>(p.sel_scales)[rowa[k]]);
-                scb[k] = __half2float(reinterpret_cast<const __half*>(p.sel_scales)[rowb[k]]);
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < kTileBatch; ++k) {
-            const uint32_t wa[4] = {ra[k].x, ra[k].y, ra[k].z, ra[k].w};
-            const uint32_t wb[4] = {rb[k].x, rb[k].y, rb[k].z, rb[k].w};
-            acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16_16816(acc[k], pair8_to_bf16x2<FMT>(wa[s]), pair8_to_bf16x2<FMT>(wb[s]),
-                               pair8_to_bf16x2<FMT>(wa[s] >> 16), pair8_to_bf16x2<FMT>(wb[s] >> 16),
-                               qw[2 * s], qw[2 * s + 1]);
-            if (FMT == SPOT_SEL_INT8_F16) {
-                acc[k][0] = acc[k][0] * sca[k] * qsc[0][0];
-                acc[k][1] = acc[k][1] * sca[k] * qsc[0][1];
-                acc[k][2] = acc[k][2] * scb[k] * qsc[0][0];
-                acc[k][3] = acc[k][3] * scb[k] * qsc[0][1];
-            }
-        }
+    for (int i = 0; i < 8; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+    float qs[2];
+    if (p.quantize_queries) {
+        quantize_query<FMT>(f, qs);
     } else {
-        uint32_t ga0[kTileBatch], ga1[kTileBatch], gb0[kTileBatch], gb1[kTileBatch];
-        float sa0[kTileBatch], sa1[kTileBatch], sb0[kTileBatch], sb1[kTileBatch];
+        float am = 0.f;
 #pragma unroll
-        for (int k = 0; k < kTileBatch; ++k) {
-            const uint32_t* da = reinterpret_cast<const uint32_t*>(p.sel_data) + rowa[k] * 8;
-            const uint32_t* db = reinterpret_cast<const uint32_t*>(p.sel_data) + rowb[k] * 8;
-            ga0[k] = __ldg(da + c4);
-            ga1[k] = __ldg(da + 4 + c4);
-            gb0[k] = __ldg(db + c4);
-            gb1[k] = __ldg(db + 4 + c4);
-            sa0[k] = group_scale<FMT>(p.sel_scales, rowa[k], 0);
-            sa1[k] = group_scale<FMT>(p.sel_scales, rowa[k], 1);
-            sb0[k] = group_scale<FMT>(p.sel_scales, rowb[k], 0);
-            sb1[k] = group_scale<FMT>(p.sel_scales, rowb[k], 1);
-        }
+        for (int i = 0; i < 16; ++i) am = fmaxf(am, poison_abs(f[i]));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));     // the quad holds one head
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+        const int sh = am > 0.f ? min(120, max(-113, 14 - ilogbf(am))) : 0;
+        const float up = __int_as_float((sh + 127) << 23);          // 2^sh, exact
 #pragma unroll
-        for (int k = 0; k < kTileBatch; ++k) {
-            // group 0 -> acc0 (k-steps 0, 1), group 1 -> acc1 (k-steps 2, 3)
-            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                mma_bf16_16816(acc0, byte_to_bf16x2<FMT>((ga0[k] >> (16 * s)) & 0xFFu),
-                               byte_to_bf16x2<FMT>((gb0[k] >> (16 * s)) & 0xFFu),
-                               byte_to_bf16x2<FMT>((ga0[k] >> (16 * s + 8)) & 0xFFu),
-                               byte_to_bf16x2<FMT>((gb0[k] >> (16 * s + 8)) & 0xFFu),
-                               qw[2 * s], qw[2 * s + 1]);
-                mma_bf16_16816(acc1, byte_to_bf16x2<FMT>((ga1[k] >> (16 * s)) & 0xFFu),
-                               byte_to_bf16x2<FMT>((gb1[k] >> (16 * s)) & 0xFFu),
-                               byte_to_bf16x2<FMT>((ga1[k] >> (16 * s + 8)) & 0xFFu),
-                               byte_to_bf16x2<FMT>((gb1[k] >> (16 * s + 8)) & 0xFFu),
-                               qw[4 + 2 * s], qw[4 + 2 * s + 1]);
-            }
-            acc[k][0] = acc0[0] * sa0[k] * qsc[0][0] + acc1[0] * sa1[k] * qsc[1][0];
-            acc[k][1] = acc0[1] * sa0[k] * qsc[0][1] + acc1[1] * sa1[k] * qsc[1][1];
-            acc[k][2] = acc0[2] * sb0[k] * qsc[0][0] + acc1[2] * sb1[k] * qsc[1][0];
-            acc[k][3] = acc0[3] * sb0[k] * qsc[0][1] + acc1[3] * sb1[k] * qsc[1][1];
-        }
+        for (int i = 0; i < 16; ++i) f[i] *= up;
+        qs[0] = qs[1] = __int_as_float((127 - sh) << 23);           // 2^-sh
     }
-    // epilogue: weighted ReLU sum over the group's heads (columns 2 c4, 2 c4 + 1)
 #pragma unroll
-    for (int k = 0; k < kTileBatch; ++k) {
-        float sa = wh0 * fmaxf(acc[k][0], 0.f) + wh1 * fmaxf(acc[k][1], 0.f);
-        float sb = wh0 * fmaxf(acc[k][2], 0.f) + wh1 * fmaxf(acc[k][3], 0.f);
-        sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-        sa += __shfl_xor_sync(0xffffffffu, sa, 2);
-        sb += __shfl_xor_sync(0xffffffffu, sb, 1);
-        sb += __shfl_xor_sync(0xffffffffu, sb, 2);
-        const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
-        if (c4 == 0) {
-            const float va = sa * p.inv_temp, vb = sb * p.inv_temp;
-            if (ja < n_full) scores[ja] = va;
-            if (jb < n_full) scores[jb] = vb;
-            if (ja >= r0 && ja < r1) { wmax = fmaxf(wmax, va); wmin = fminf(wmin, va); }
-            if (jb >= r0 && jb < r1) { wmax = fmaxf(wmax, vb); wmin = fminf(wmin, vb); }
+    for (int i = 0; i < 8; ++i) {
+        int e0 = 2 * i, e1 = 2 * i + 1;
+        if (four) {                                   // i = 4 grp + 2 s + t
+            const int grp = i >> 2, s2 = (i >> 1) & 1, t = i & 1;
+            e0 = 8 * grp + 2 * s2 + t;
+            e1 = e0 + 4;
         }
+        const __half2 hv = __floats2half2_rn(f[e0], f[e1]);
+        qf[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        qsc[hf][0] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4);
+        qsc[hf][1] = __shfl_sync(0xffffffffu, qs[hf], 8 * c4 + 4);
+    }
+    const int64_t wrow = static_cast<int64_t>(b) * p.num_q_heads + g * G;
+    wh0 = (2 * c4 < G) ? (p.w ? p.w[wrow + 2 * c4] : 1.f / G) : 0.f;
+    wh1 = (2 * c4 + 1 < G) ? (p.w ? p.w[wrow + 2 * c4 + 1] : 1.f / G) : 0.f;
+}
+
+// Scale of group grp (dims 32 grp .. + 31) from a staged scale word.
+template <int FMT>
+__device__ __forceinline__ float staged_scale(uint32_t w, int grp) {
+    if (FMT == SPOT_SEL_INT4_G32_F16)
+        return __half2float(__ushort_as_half(static_cast<uint16_t>(w >> (16 * grp))));
+    if (FMT == SPOT_SEL_INT8_F16) return __half2float(__ushort_as_half(static_cast<uint16_t>(w)));
+    return e8m0_value((w >> (8 * grp)) & 0xFFu);
+}
+
+// Query-key dot products of the 16 staged rows 16 t .. 16 t + 15 for the
+// group's heads: keys as the mma M operand, the selector queries as N = 8
+// (qw: B fragments, lane: head r8; qsc: query scales).  acc: rows r8 and
+// r8 + 8 of this lane, columns (heads) 2 c4 and 2 c4 + 1.  Branch-free, so
+// that a warp's two tiles in flight interleave.
+template <int FMT>
+__device__ __forceinline__ void tile_dots(const uint8_t* stg, const uint32_t* stg_sc, int t,
+                                          const uint32_t (&qw)[8], const float (&qsc)[2][2],
+                                          int lane, float (&acc)[4]) {
+    const int c4 = lane & 3, r8 = lane >> 2;
+    const int ra = 16 * t + r8, rb = ra + 8;
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+    if (FMT == SPOT_SEL_BF16) {
+        const uint4 a0 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(ra, 2 * c4));
+        const uint4 a1 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(ra, 2 * c4 + 1));
+        const uint4 b0 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(rb, 2 * c4));
+        const uint4 b1 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(rb, 2 * c4 + 1));
+        const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_bf16_16816(acc, wa[2 * s], wb[2 * s], wa[2 * s + 1], wb[2 * s + 1], qw[2 * s],
+                           qw[2 * s + 1]);
+    } else if (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
+        // 64-byte rows: lane c4 owns bytes (= dims) [16 c4, 16 c4 + 16), widened
+        // exactly to f16 four codes at a time (pairs (0, 1) and (2, 3))
+        const uint4 ra4 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(ra, c4));
+        const uint4 rb4 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(rb, c4));
+        const uint32_t wa[4] = {ra4.x, ra4.y, ra4.z, ra4.w};
+        const uint32_t wb[4] = {rb4.x, rb4.y, rb4.z, rb4.w};
+#pragma unroll
+        for (int s2 = 0; s2 < 4; ++s2) {
+            uint32_t alo, ahi, blo, bhi;
+            if (FMT == SPOT_SEL_INT8_F16) {
+                int8x4_to_f16x2(wa[s2], alo, ahi);
+                int8x4_to_f16x2(wb[s2], blo, bhi);
+            } else {
+                e4m3x4_to_f16x2(wa[s2], alo, ahi);
+                e4m3x4_to_f16x2(wb[s2], blo, bhi);
+            }
+            mma_f16_16816(acc, alo, blo, ahi, bhi, qw[2 * s2], qw[2 * s2 + 1]);
+        }
+        const float sca = FMT == SPOT_SEL_INT8_F16 ? staged_scale<FMT>(stg_sc[ra], 0) : 1.f;
+        const float scb = FMT == SPOT_SEL_INT8_F16 ? staged_scale<FMT>(stg_sc[rb], 0) : 1.f;
+        acc[0] = acc[0] * sca * qsc[0][0];
+        acc[1] = acc[1] * sca * qsc[0][1];
+        acc[2] = acc[2] * scb * qsc[0][0];
+        acc[3] = acc[3] * scb * qsc[0][1];
+    } else {
+        // 32-byte rows: lane c4 owns bytes [4 c4, 4 c4 + 4) of each 16-byte
+        // half (half 0 = group 0 = dims 0-31, half 1 = group 1), widened
+        // exactly to f16 (pairs (j, j + 4); E2M1 as value x 2^-14, undone in
+        // the scale)
+        const uint32_t swa = stg_sc[ra], swb = stg_sc[rb];
+        float accg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
+            const uint32_t wa = *reinterpret_cast<const uint32_t*>(stg + piece_off<FMT>(ra, grp) + 4 * c4);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(stg + piece_off<FMT>(rb, grp) + 4 * c4);
+            uint32_t oa[4], ob[4];
+            if (FMT == SPOT_SEL_INT4_G32_F16) {
+                int4x8_to_f16x2(wa, oa);
+                int4x8_to_f16x2(wb, ob);
+            } else {
+                e2m1x8_to_f16x2_scaled(wa, oa);
+                e2m1x8_to_f16x2_scaled(wb, ob);
+            }
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2)
+                mma_f16_16816(accg[grp], oa[2 * s2], ob[2 * s2], oa[2 * s2 + 1], ob[2 * s2 + 1],
+                              qw[4 * grp + 2 * s2], qw[4 * grp + 2 * s2 + 1]);
+        }
+        constexpr float kw = FMT == SPOT_SEL_MXFP4_G32_E8M0 ? 16384.f : 1.f;
+        const float sa0 = staged_scale<FMT>(swa, 0) * kw, sa1 = staged_scale<FMT>(swa, 1) * kw;
+        const float sb0 = staged_scale<FMT>(swb, 0) * kw, sb1 = staged_scale<FMT>(swb, 1) * kw;
+        acc[0] = accg[0][0] * sa0 * qsc[0][0] + accg[1][0] * sa1 * qsc[1][0];
+        acc[1] = accg[0][1] * sa0 * qsc[0][1] + accg[1][1] * sa1 * qsc[1][1];
+        acc[2] = accg[0][2] * sb0 * qsc[0][0] + accg[1][2] * sb1 * qsc[1][0];
+        acc[3] = accg[0][3] * sb0 * qsc[0][1] + accg[1][3] * sb1 * qsc[1][1];
+    }
+}
+
+// Scores of tile t from its dot products: weighted ReLU sum over the group's
+// heads (wh0 / wh1: weights of heads 2 c4, 2 c4 + 1, 0 for padding heads),
+// written for the rows below n (blocks j0 + row); tracks the maximum /
+// minimum of the residual scores [r0, r1).
+__device__ __forceinline__ void tile_scores(const SelectParams& p, const float (&acc)[4], int t,
+                                            int j0, int n, float wh0, float wh1, float* scores,
+                                            int lane, int r0, int r1, float& wmax, float& wmin) {
+    const int c4 = lane & 3, r8 = lane >> 2;
+    const int ra = 16 * t + r8, rb = ra + 8;
+    float sa = wh0 * fmaxf(acc[0], 0.f) + wh1 * fmaxf(acc[1], 0.f);
+    float sb = wh0 * fmaxf(acc[2], 0.f) + wh1 * fmaxf(acc[3], 0.f);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+    sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+    sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+    if (c4 == 0) {
+        const int ja = j0 + ra, jb = j0 + rb;
+        const float va = sa * p.inv_temp, vb = sb * p.inv_temp;
+        if (ra < n) scores[ja] = va;
+        if (rb < n) scores[jb] = vb;
+        if (ra < n && ja >= r0 && ja < r1) { wmax = fmaxf(wmax, va); wmin = fminf(wmin, va); }
+        if (rb < n && jb >= r0 && jb < r1) { wmax = fmaxf(wmax, vb); wmin = fminf(wmin, vb); }
     }
 }
 
@@ -242,8 +391,6 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 constexpr int kNB = 2048;              // most value buckets of the first pass (1024 up to
                                         // 2048 residual blocks, then 2048), spread over the
                                         // residual scores' range
-constexpr int NT = kSelectThreads;
-constexpr int NW = NT / 32;
 
 struct SelSmem {
     float* score;                 // [max_blocks] selector scores of the complete blocks
@@ -692,31 +839,32 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
             smin_f = fminf(smin_f, wmin[w]);
         }
     }
-    const double smax = static_cast<double>(smax_f);
     // buckets per unit of score: the residual range spans all nbk buckets,
     // up to 40 below the maximum (exp(-40) is below the fixed point's 2^-40;
     // anything lower shares the last bucket)
     const float range = fminf(smax_f - smin_f, 40.f);
     const float bscale = range > 1e-30f ? static_cast<float>(nbk - 1) / range : 1.f;
 
-    // ---- exact fixed-point numerators exp(s - max), value
-    // buckets (monotone in the score) with exact counts and masses
+    // ---- fixed-point numerators exp(s - max) (fp32 exp2 of the difference
+    // times log2 e, within about 2e-6 relative of exp for the differences
+    // whose mass matters; each held exactly as 2^-40 fixed point so that
+    // every sum below is exact and order-independent), value buckets
+    // (monotone in the score) with exact counts and masses
     constexpr int kUnroll = 4;                        // independent exps in flight
     for (int i0 = threadIdx.x; i0 < n; i0 += kUnroll * NT) {
-        float v[kUnroll];
-        double e[kUnroll];
+        float v[kUnroll], e[kUnroll];
 #pragma unroll
         for (int k = 0; k < kUnroll; ++k) {
             const int i = i0 + k * NT;
             v[k] = i < n ? s[r0 + i] : smax_f;
         }
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k) e[k] = exp(static_cast<double>(v[k]) - smax);
+        for (int k = 0; k < kUnroll; ++k) e[k] = exp2f((v[k] - smax_f) * 1.4426950408889634f);
 #pragma unroll
         for (int k = 0; k < kUnroll; ++k) {
             const int i = i0 + k * NT;
             if (i >= n) break;
-            const unsigned long long f = __double2ull_rn(ldexp(e[k], kFixShift));
+            const unsigned long long f = __float2ull_rn(e[k] * static_cast<float>(1ull << kFixShift));
             sm.mass[i] = f;
             if (nparts > 0) sm.keys[i] = score_key(v[k]);
             const int bkt = static_cast<int>(fminf((smax_f - v[k]) * bscale, nbk - 1.f));
@@ -871,17 +1019,20 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
 }
 
 // Scoring (§2.1, Eq. 2) and selection in one launch.  The C CTAs of a unit
-// (one thread-block cluster when C > 1) share its 16-block tiles: CTA c
-// takes rounds c, c + C, ... of NW * kTileBatch tiles (one batch of
-// kTileBatch tiles per warp per round, the next round's page ids loading
-// while this round's keys do).  Every CTA stores its scores straight into
-// the shared memory of the cluster's first CTA, which selects once the
-// cluster barrier (release / acquire at cluster scope) has passed.
+// (one thread-block cluster when C > 1) split its 16-block tiles into C
+// contiguous shares; each CTA gathers its share's selector rows into its
+// own shared memory (in passes of at most `pass_rows` rows) and scores them
+// there, each warp taking every NW-th tile.  Every CTA stores its scores
+// straight into the shared memory of the cluster's first CTA, which selects
+// once the cluster barrier (release / acquire at cluster scope) has passed.
 template <int FMT>
 __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const SelectParams p,
-                                                                         int C) {
+                                                                         int C, int stage_off,
+                                                                         int pass_rows) {
     extern __shared__ __align__(16) uint8_t smem[];
     const SelSmem sm = carve_select_smem(smem, p.max_blocks);
+    uint8_t* stg = smem + stage_off;                                 // staged rows
+    uint32_t* stg_sc = reinterpret_cast<uint32_t*>(stg + pass_rows * row_stride<FMT>());
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int u = blockIdx.x / C, c = blockIdx.x - u * C;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
@@ -890,30 +1041,52 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
     const BlockSpan sp = block_span(p, L);                           // overflow: flagged
     const int n_full = sp.n_full;                                    // by the selection
     const int tiles = (n_full + 15) / 16;
+    const int t_lo = static_cast<int>(static_cast<int64_t>(tiles) * c / C);
+    const int t_hi = static_cast<int>(static_cast<int64_t>(tiles) * (c + 1) / C);
+    const int j_lo = 16 * t_lo, j_hi = min(n_full, 16 * t_hi);     // this CTA's blocks
     float* out = sm.score;                                           // the leader's
     float* part = sm.part;
     if (C > 1) {
+        cluster_arrive_relaxed();                                    // matched by the wait below
         out = cooperative_groups::this_cluster().map_shared_rank(sm.score, 0);
         part = cooperative_groups::this_cluster().map_shared_rank(sm.part, 0);
     }
     float wmax = -INFINITY, wmin = INFINITY;                         // residual scores
-    constexpr int kRound = NW * kTileBatch;
-    const int step = C * kRound;
-    const int first = c * kRound + warp;
-    if (first < tiles) {                                             // warp-uniform
+    if (j_hi > j_lo) {
+        int pg[kMaxRowsPerThread];
+        stage_pages(p, b, j_lo, min(pass_rows, j_hi - j_lo), pg);   // in flight with the queries
         uint32_t qw[8];
         float qsc[2][2], wh0, wh1;
-        load_queries<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
-        int pa[kTileBatch], pb[kTileBatch];
-        load_pages(p, b, first, NW, n_full, lane, pa, pb);
-        for (int t0 = first; t0 < tiles; t0 += step) {
-            int na[kTileBatch], nb2[kTileBatch];
-            if (t0 + step < tiles) load_pages(p, b, t0 + step, NW, n_full, lane, na, nb2);
-            score_tiles<FMT>(p, g, qw, qsc, wh0, wh1, t0, NW, n_full, out, lane, pa, pb, sp.r0,
-                             sp.r1, wmax, wmin);
-#pragma unroll
-            for (int k = 0; k < kTileBatch; ++k) { pa[k] = na[k]; pb[k] = nb2[k]; }
+        if (FMT == SPOT_SEL_BF16) load_queries<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
+        else load_queries_f16<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
+        for (int j0 = j_lo; j0 < j_hi; j0 += pass_rows) {
+            const int n = min(pass_rows, j_hi - j0);
+            if (j0 != j_lo) stage_pages(p, b, j0, n, pg);
+            uint32_t sc[kMaxRowsPerThread];
+            stage_issue<FMT>(p, g, n, pg, stg, sc);
+            if (C > 1 && j0 == j_lo) {
+                // every CTA of the cluster has started before the first remote
+                // store into the leader's shared memory
+                cluster_wait();
+            }
+            // row group k (NT rows, 2 tiles per warp) is scored while the
+            // groups after it are still landing
+            for (int k = 0; k * NT < n; ++k) {
+                stage_wait<FMT>(k, n, sc, stg_sc);
+                const int t0 = k * (NT / 16) + warp, t1 = t0 + NW;
+                const bool two = 16 * t1 < n;
+                float a0[4], a1[4];
+                if (16 * t0 < n) tile_dots<FMT>(stg, stg_sc, t0, qw, qsc, lane, a0);
+                if (two) tile_dots<FMT>(stg, stg_sc, t1, qw, qsc, lane, a1);
+                if (16 * t0 < n)
+                    tile_scores(p, a0, t0, j0, n, wh0, wh1, out, lane, sp.r0, sp.r1, wmax, wmin);
+                if (two)
+                    tile_scores(p, a1, t1, j0, n, wh0, wh1, out, lane, sp.r0, sp.r1, wmax, wmin);
+            }
+            __syncthreads();                                         // staging is free again
         }
+    } else if (C > 1) {
+        cluster_wait();
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -968,16 +1141,35 @@ cudaError_t allow_smem(Kernel kernel, int slot, size_t smem) {
     return e;
 }
 
+// Largest dynamic shared memory a CTA may use on the current device.
+int smem_optin() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    return v;
+}
+
 template <int FMT>
-cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t s) {
-    cudaError_t e = allow_smem(score_select_kernel<FMT>, 1 + FMT, smem);
-    if (e != cudaSuccess) return e;
-    // CTAs per unit: enough to cover the longest sequence in one round of
-    // NW * kTileBatch tiles each, as far as one wave of one CTA per SM allows
+cudaError_t launch_score_select(const SelectParams& p, size_t smem_sel, cudaStream_t s) {
+    // CTAs per unit: one per 32 tiles of the longest sequence, as far as one
+    // wave of one CTA per SM allows (at most a portable cluster of 8)
     const int U = p.batch * p.num_kv_heads;
     const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
-    const int rounds = max(1, ((cap + 15) / 16 + NW * kTileBatch - 1) / (NW * kTileBatch));
-    const int C = max(1, min(min(rounds, kMaxCluster), sm_count() / max(U, 1)));
+    const int tiles = (cap + 15) / 16;
+    const int C = max(1, min(min((tiles + 31) / 32, kMaxCluster), sm_count() / max(U, 1)));
+    // staging for one CTA's share of rows (whole 16-row tiles), in passes of
+    // what fits next to the selection's shared memory
+    const int share = 16 * ((tiles + C - 1) / C);
+    const size_t off = (smem_sel + 15) / 16 * 16;
+    const size_t per_row = row_stride<FMT>() + sizeof(uint32_t);
+    const size_t limit = static_cast<size_t>(smem_optin());
+    if (limit < off + 16 * per_row) return cudaErrorInvalidValue;
+    int pass_rows = static_cast<int>(min((limit - off) / per_row, static_cast<size_t>(NT * kMaxRowsPerThread)));
+    pass_rows = min(pass_rows / 16 * 16, share);
+    const size_t smem = off + static_cast<size_t>(pass_rows) * per_row;
+    cudaError_t e = allow_smem(score_select_kernel<FMT>, 1 + FMT, smem);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(U * C);
     cfg.blockDim = dim3(kSelectThreads);
@@ -990,7 +1182,7 @@ cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = C > 1 ? 1 : 0;                     // C = 1: a plain launch
-    e = cudaLaunchKernelEx(&cfg, score_select_kernel<FMT>, p, C);
+    e = cudaLaunchKernelEx(&cfg, score_select_kernel<FMT>, p, C, static_cast<int>(off), pass_rows);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -87,15 +87,18 @@ __device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
 // Merge the partials of unit u (blocks [lo, hi) of the flattened list) and
 // write out / lse of its G heads, with all NC consumer warps (tid < NC*32).
 // The partials are one per CTA whose range touched the unit; other CTAs of
-// this launch wrote them, so they are read through L2 (ld.global.cg).  First
-// the (m, l) of every slot and head go to shared memory (ml, at least
-// nslots * G * 2 floats: every load in flight at once), then each thread
-// takes (head, 4 dims) items and combines the slots' accumulators with their
-// log-sum-exp weights, kMergeBatch slots' loads in flight per step.
-constexpr int kMergeBatch = 8;           // slot loads in flight per thread and step
+// this launch wrote them, so they are read through L2 (ld.global.cg).  This
+// runs while the rest of the grid still streams from HBM, when every L2
+// round trip is slow, so it takes one round trip per kMergeBatch slots: a
+// thread owns up to kMergeItems (head, 4 dims) items and issues the loads of
+// (m, l, acc) of all of them for a whole batch of slots before using any,
+// folding batches with a running maximum (the usual log-sum-exp merge).
+// Slots are folded in CTA order, so the result does not depend on timing.
+constexpr int kMergeBatch = 8;           // slots per batch
+constexpr int kMergeItems = (kMaxGroup * (kHeadDim / 4) + NC * 32 - 1) / (NC * 32);
 
 __device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t N, int64_t P,
-                           float* ml, int tid) {
+                           int tid) {
     constexpr int T = NC * 32;
     const int G = p.group;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
@@ -103,57 +106,73 @@ __device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t
     const int nslots = i1 - i0 + 1;
     const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
     const bool some_idle = N < P;          // only then can a CTA own no blocks
-    for (int t = tid; t < nslots * G; t += T) {
-        const int k = t / G, n = t - k * G;
-        const int i = i0 + k;
-        float m = -INFINITY, l = 0.f;
-        if (!(some_idle && range_begin(N, P, i) == range_begin(N, P, i + 1))) {
-            const float* sl = p.partials + static_cast<int64_t>(i + u) * stride;
-            m = __ldcg(sl + G * kHeadDim + n);
-            l = __ldcg(sl + G * (kHeadDim + 1) + n);
-        }
-        ml[2 * t] = m;
-        ml[2 * t + 1] = l;
+    float M[kMergeItems], L[kMergeItems];
+    float4 a[kMergeItems];
+#pragma unroll
+    for (int r = 0; r < kMergeItems; ++r) {
+        M[r] = -INFINITY;
+        L[r] = 0.f;
+        a[r] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    consumer_barrier();
-    for (int item = tid; item < G * (kHeadDim / 4); item += T) {
-        const int n = item / (kHeadDim / 4), d4 = item - n * (kHeadDim / 4);
-        float M = -INFINITY;
-        for (int k = 0; k < nslots; ++k) M = fmaxf(M, ml[2 * (k * G + n)]);
-        float L = 0.f;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (M != -INFINITY) {
-            for (int k0 = 0; k0 < nslots; k0 += kMergeBatch) {
-                float wk[kMergeBatch];
-                float4 v[kMergeBatch];
+    for (int k0 = 0; k0 < nslots; k0 += kMergeBatch) {
+        float mk[kMergeItems][kMergeBatch], lk[kMergeItems][kMergeBatch];
+        float4 v[kMergeItems][kMergeBatch];
 #pragma unroll
-                for (int k = 0; k < kMergeBatch; ++k) {
-                    const float m = k0 + k < nslots ? ml[2 * ((k0 + k) * G + n)] : -INFINITY;
-                    wk[k] = (m == -INFINITY) ? 0.f : exp2f(m - M);
-                    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (wk[k] != 0.f)
-                        v[k] = __ldcg(reinterpret_cast<const float4*>(
-                                          p.partials + static_cast<int64_t>(i0 + k0 + k + u) *
-                                                           stride + n * kHeadDim) + d4);
-                }
+        for (int r = 0; r < kMergeItems; ++r) {
+            const int item = tid + r * T;
+            const int n = item / (kHeadDim / 4), d4 = item - n * (kHeadDim / 4);
 #pragma unroll
-                for (int k = 0; k < kMergeBatch; ++k) {
-                    if (wk[k] != 0.f) L = fmaf(wk[k], ml[2 * ((k0 + k) * G + n) + 1], L);
-                    a.x = fmaf(wk[k], v[k].x, a.x);
-                    a.y = fmaf(wk[k], v[k].y, a.y);
-                    a.z = fmaf(wk[k], v[k].z, a.z);
-                    a.w = fmaf(wk[k], v[k].w, a.w);
-                }
+            for (int k = 0; k < kMergeBatch; ++k) {
+                const int i = i0 + k0 + k;
+                mk[r][k] = -INFINITY;
+                lk[r][k] = 0.f;
+                v[r][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (n >= G || k0 + k >= nslots) continue;
+                if (some_idle && range_begin(N, P, i) == range_begin(N, P, i + 1)) continue;
+                const float* sl = p.partials + static_cast<int64_t>(i + u) * stride;
+                mk[r][k] = __ldcg(sl + G * kHeadDim + n);
+                lk[r][k] = __ldcg(sl + G * (kHeadDim + 1) + n);
+                v[r][k] = __ldcg(reinterpret_cast<const float4*>(sl + n * kHeadDim) + d4);
             }
         }
-        const bool empty = !(L > 0.f);    // only if every tile was rejected as out of range
-        const float inv = empty ? 0.f : 1.f / L;
+#pragma unroll
+        for (int r = 0; r < kMergeItems; ++r) {
+            float Mb = M[r];
+#pragma unroll
+            for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, mk[r][k]);
+            if (Mb == -INFINITY) continue;
+            const float sc = (M[r] == -INFINITY) ? 0.f : exp2f(M[r] - Mb);
+            L[r] *= sc;
+            a[r].x *= sc;
+            a[r].y *= sc;
+            a[r].z *= sc;
+            a[r].w *= sc;
+#pragma unroll
+            for (int k = 0; k < kMergeBatch; ++k) {
+                if (mk[r][k] == -INFINITY) continue;   // empty or never written
+                const float wk = exp2f(mk[r][k] - Mb);
+                L[r] = fmaf(wk, lk[r][k], L[r]);
+                a[r].x = fmaf(wk, v[r][k].x, a[r].x);
+                a[r].y = fmaf(wk, v[r][k].y, a[r].y);
+                a[r].z = fmaf(wk, v[r][k].z, a[r].z);
+                a[r].w = fmaf(wk, v[r][k].w, a[r].w);
+            }
+            M[r] = Mb;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kMergeItems; ++r) {
+        const int item = tid + r * T;
+        const int n = item / (kHeadDim / 4), d4 = item - n * (kHeadDim / 4);
+        if (n >= G) continue;
+        const bool empty = !(L[r] > 0.f);  // only if every tile was rejected as out of range
+        const float inv = empty ? 0.f : 1.f / L[r];
         const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
         reinterpret_cast<float4*>(p.out + h * kHeadDim)[d4] =
-            make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
-        if (p.lse && d4 == 0) p.lse[h] = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+            make_float4(a[r].x * inv, a[r].y * inv, a[r].z * inv, a[r].w * inv);
+        if (p.lse && d4 == 0)
+            p.lse[h] = empty ? -INFINITY : (M[r] + log2f(L[r])) * 0.6931471805599453f;
     }
-    consumer_barrier();                   // ml (shared scratch) is free again
 }
 
 // Valid tokens of the four 16-row slices of a 64-row tile, one byte each.
@@ -571,8 +590,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
         consumer_barrier();
         if (flags[1]) {
             __threadfence();
-            // red_acc is free again: the CTA's partial has been written
-            merge_unit(p, u, unit_off[u], unit_off[u + 1], N, P, red_acc, threadIdx.x);
+            merge_unit(p, u, unit_off[u], unit_off[u + 1], N, P, threadIdx.x);
         }
         pos = seg_end;
     }
@@ -631,9 +649,7 @@ int decode_grid(int units) {
                                                       kThreads, smem) != cudaSuccess)
         return 0;
     m.units = units;
-    // the merge keeps (m, l) of up to `grid` slots x 8 heads in red_acc
-    constexpr int kMaxGrid = NC * kMaxGroup * kPartialFloatsPerHead / (2 * kMaxGroup);
-    m.grid = min(sms * max(per_sm, 1), kMaxGrid);
+    m.grid = sms * max(per_sm, 1);
     return m.grid;
 }
 
