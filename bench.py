@@ -44,12 +44,12 @@ HBM_FALLBACK_GBS = 6650.0
 # same workload), valid only while the kernel's source files are unchanged
 # (sha256 prefix over them); otherwise the roofline's traffic is null.
 NCU_TRAFFIC = {
-    "qwen3_32b_128k": {"bytes": 728982528 + 3904768, "files": ["sparse_decode.cu"],
-                       "sha256": "82c100300b60004f"},
+    "qwen3_32b_128k": {"bytes": 729075456 + 3837184, "files": ["sparse_decode.cu"],
+                       "sha256": "00f3a2b731258513"},
     "qwen3_8b_128k_tok": {"bytes": 246840064 + 4134144, "files": ["sparse_decode.cu"],
                           "sha256": "82c100300b60004f"},
-    "qwen3_8b_prefill_32k": {"bytes": 411734016 + 499205376, "files": ["prefill.cu", "tc.cuh"],
-                             "sha256": "362fd0bc4a92eeba"},
+    "qwen3_8b_prefill_32k": {"bytes": 411903488 + 499184128, "files": ["prefill.cu", "tc.cuh"],
+                             "sha256": "716d0750e6195d2d"},
 }
 
 
@@ -284,7 +284,7 @@ def run_spot(args, world, rank, local):
     for l in range(args.layers):
         # layers of one model share sequence lengths and page tables
         wl = workloads.make(args.workload, seed=layer_seed(rank, l), device=dev, sel_fmt=fmt,
-                            structure_from=layers[0][0] if layers else None)
+                            batch=args.batch, structure_from=layers[0][0] if layers else None)
         desc = spot.layer_desc(wl.num_q_heads, wl.num_kv_heads, wl.num_pages, fmt)
         if fmt == "bf16":
             data, scales = wl.sel_keys, None
@@ -1058,7 +1058,7 @@ def run_reference(args, world, rank):
         return None
     import oracle
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    wl = workloads.make(args.workload, seed=0, device=dev, sel_fmt=args.sel_fmt)
+    wl = workloads.make(args.workload, seed=0, device=dev, sel_fmt=args.sel_fmt, batch=args.batch)
     cores = host_cores()
     oracle.set_num_threads(cores)
     smp = OracleSampler(wl, args.sel_fmt, cores)
@@ -1187,6 +1187,9 @@ def main():
     ap.add_argument("--sel-fmt", default=None)
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per GPU (default: the workload's own); a smaller batch "
+                         "keeps an ncu capture within a few GB of device memory")
     args = ap.parse_args()
     tok = args.workload in workloads.TOK_SPECS
     pf = args.workload in workloads.PREFILL_SPECS

@@ -56,35 +56,15 @@ constexpr int NW = NT / 32;
 
 // --------------------------------------------------------------- scoring
 
-// Selector rows are first gathered into shared memory with cp.async (every
-// row of a pass in flight at once: one round trip for the page ids, one for
-// the rows), then scored from there.  Row layout in shared memory per
-// format: bf16 rows of 128 bytes at a 144-byte stride (no bank conflicts in
-// the fragment loads); 8-bit code rows of 64 bytes; 4-bit code rows of 32
-// bytes whose two 16-byte halves swap places when bit 2 of the row index is
-// set (rows r and r + 4 then use different banks).  Scales go to a separate
-// array of one 32-bit word per row.
+// Scoring loads the selector rows straight into registers, a warp's tiles
+// kTileBatch at a time (their gathered loads in flight together, the next
+// round's page ids loading meanwhile), and keeps the kernel's shared memory
+// to the selection's own: a CTA of the sparse-decode kernel that follows
+// (programmatic dependent launch) then fits on the same SM and starts its
+// prologue before this kernel's CTAs have left.
 template <int FMT>
-__host__ __device__ constexpr int row_bytes() {
-    return FMT == SPOT_SEL_BF16 ? 128
-           : (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) ? 64 : 32;
-}
-template <int FMT>
-__host__ __device__ constexpr int row_stride() {
-    return FMT == SPOT_SEL_BF16 ? 144 : row_bytes<FMT>();
-}
-template <int FMT>
-__host__ __device__ constexpr bool has_scales() {
-    return FMT == SPOT_SEL_INT4_G32_F16 || FMT == SPOT_SEL_MXFP4_G32_E8M0 ||
-           FMT == SPOT_SEL_INT8_F16;
-}
-constexpr int kMaxRowsPerThread = 8;    // rows one thread stages per pass
-
-// Byte offset of 16-byte piece h of staged row r.
-template <int FMT>
-__device__ __forceinline__ int piece_off(int r, int h) {
-    if (row_bytes<FMT>() == 32) return r * 32 + ((h ^ ((r >> 2) & 1)) << 4);
-    return r * row_stride<FMT>() + (h << 4);
+__host__ __device__ constexpr int tile_batch() {
+    return FMT == SPOT_SEL_BF16 ? 2 : 4;          // bf16 fragments hold 4x the registers
 }
 
 // Cluster barrier halves (every thread of every CTA of the cluster arrives
@@ -95,75 +75,63 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
 
-// Issues the gathering of the selector rows of blocks j0 .. j0 + n - 1 of
-// sequence b, KV head g (page ids pg from stage_pages) into shared memory: row r goes to staging row r and
-// is copied by thread r % NT, in row group r / NT (one cp.async commit group
-// per row group, kMaxRowsPerThread groups always, empty ones included).  An
-// out-of-range page id is recorded and page 0 read instead.  The rows' scale
-// words are loaded into sc[] (stored by stage_wait).
-// Page ids of the rows this thread stages (loaded ahead, so that their
-// latency overlaps other loads).
-__device__ __forceinline__ void stage_pages(const SelectParams& p, int b, int j0, int n,
-                                            int (&pg)[kMaxRowsPerThread]) {
-#pragma unroll
-    for (int k = 0; k < kMaxRowsPerThread; ++k) {
-        const int r = threadIdx.x + k * NT;
-        pg[k] = r < n ? __ldg(p.page_table + static_cast<int64_t>(b) * p.pt_stride + j0 + r) : 0;
-    }
-}
+// One lane's key fragments of a 16-block tile (rows r8 and r8 + 8): bf16:
+// dims [16 c4, 16 c4 + 16) of each row (a0 / a1 row a, b0 / b1 row b);
+// 8-bit: bytes [16 c4, 16 c4 + 16) of each row; 4-bit: bytes [4 c4, 4 c4 +
+// 4) of each 16-byte half (half 0 = group 0 = dims 0-31, half 1 = group 1)
+// of each row; plus the rows' scale words (INT4: both fp16 group scales,
+// MXFP4: both E8M0 bytes, INT8: the fp16 row scale).
+struct KeyFrag {
+    uint4 a0, a1, b0, b1;
+    uint32_t sa, sb;
+};
 
 template <int FMT>
-__device__ __forceinline__ void stage_issue(const SelectParams& p, int g, int n,
-                                            const int (&pg)[kMaxRowsPerThread], uint8_t* stg,
-                                            uint32_t (&sc)[kMaxRowsPerThread]) {
-    const uint32_t st = smem_u32(stg);
-#pragma unroll
-    for (int k = 0; k < kMaxRowsPerThread; ++k) {
-        const int r = threadIdx.x + k * NT;
-        sc[k] = 0u;
-        if (r < n) {
-            int pa = pg[k];
-            if (pa < 0 || pa >= p.num_pages) {
-                flag_status(p.status, kStatusBounds);
-                pa = 0;
-            }
-            const int64_t row = static_cast<int64_t>(pa) * p.num_kv_heads + g;
-            const uint8_t* src = static_cast<const uint8_t*>(p.sel_data) + row * row_bytes<FMT>();
-#pragma unroll
-            for (int h = 0; h < row_bytes<FMT>() / 16; ++h)
-                cp_async16(st + piece_off<FMT>(r, h), src + 16 * h);
-            if (FMT == SPOT_SEL_INT4_G32_F16)
-                sc[k] = __ldg(reinterpret_cast<const uint32_t*>(p.sel_scales) + row);
-            else if (FMT == SPOT_SEL_MXFP4_G32_E8M0 || FMT == SPOT_SEL_INT8_F16)
-                sc[k] = __ldg(reinterpret_cast<const uint16_t*>(p.sel_scales) + row);
+__device__ __forceinline__ void load_frag(const SelectParams& p, int64_t rowa, int64_t rowb,
+                                          int c4, KeyFrag& f) {
+    if (FMT == SPOT_SEL_BF16) {
+        const uint4* ka = reinterpret_cast<const uint4*>(p.sel_data) + rowa * 8 + 2 * c4;
+        const uint4* kb = reinterpret_cast<const uint4*>(p.sel_data) + rowb * 8 + 2 * c4;
+        f.a0 = __ldg(ka);
+        f.a1 = __ldg(ka + 1);
+        f.b0 = __ldg(kb);
+        f.b1 = __ldg(kb + 1);
+    } else if (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
+        f.a0 = __ldg(reinterpret_cast<const uint4*>(p.sel_data) + rowa * 4 + c4);
+        f.b0 = __ldg(reinterpret_cast<const uint4*>(p.sel_data) + rowb * 4 + c4);
+        if (FMT == SPOT_SEL_INT8_F16) {
+            f.sa = __ldg(reinterpret_cast<const uint16_t*>(p.sel_scales) + rowa);
+            f.sb = __ldg(reinterpret_cast<const uint16_t*>(p.sel_scales) + rowb);
         }
-        cp_async_commit();
+    } else {
+        const uint32_t* da = reinterpret_cast<const uint32_t*>(p.sel_data) + rowa * 8;
+        const uint32_t* db = reinterpret_cast<const uint32_t*>(p.sel_data) + rowb * 8;
+        f.a0.x = __ldg(da + c4);
+        f.a0.y = __ldg(da + 4 + c4);
+        f.b0.x = __ldg(db + c4);
+        f.b0.y = __ldg(db + 4 + c4);
+        if (FMT == SPOT_SEL_INT4_G32_F16) {
+            f.sa = __ldg(reinterpret_cast<const uint32_t*>(p.sel_scales) + rowa);
+            f.sb = __ldg(reinterpret_cast<const uint32_t*>(p.sel_scales) + rowb);
+        } else {
+            f.sa = __ldg(reinterpret_cast<const uint16_t*>(p.sel_scales) + rowa);
+            f.sb = __ldg(reinterpret_cast<const uint16_t*>(p.sel_scales) + rowb);
+        }
     }
 }
 
-// Waits until row group k (rows k NT .. k NT + NT - 1) has landed for every
-// thread, its scale words stored; returns behind a barrier.
+// Page ids of the blocks of tiles t0, t0 + stride, ... (rows r8 and r8 + 8).
 template <int FMT>
-__device__ __forceinline__ void stage_wait(int k, int n, const uint32_t (&sc)[kMaxRowsPerThread],
-                                           uint32_t* stg_sc) {
-    switch (kMaxRowsPerThread - 1 - k) {           // groups after k may still be in flight
-        case 7: cp_async_wait<7>(); break;
-        case 6: cp_async_wait<6>(); break;
-        case 5: cp_async_wait<5>(); break;
-        case 4: cp_async_wait<4>(); break;
-        case 3: cp_async_wait<3>(); break;
-        case 2: cp_async_wait<2>(); break;
-        case 1: cp_async_wait<1>(); break;
-        default: cp_async_wait<0>(); break;
-    }
-    static_assert(kMaxRowsPerThread == 8, "stage_wait covers eight groups");
-    if (has_scales<FMT>()) {
-        const int r = threadIdx.x + k * NT;
+__device__ __forceinline__ void load_pages(const SelectParams& p, int b, int t0, int stride,
+                                           int n_full, int lane, int (&pa)[tile_batch<FMT>()],
+                                           int (&pb)[tile_batch<FMT>()]) {
+    const int r8 = lane >> 2;
 #pragma unroll
-        for (int kk = 0; kk < kMaxRowsPerThread; ++kk)
-            if (kk == k && r < n) stg_sc[r] = sc[kk];
+    for (int k = 0; k < tile_batch<FMT>(); ++k) {
+        const int ja = (t0 + k * stride) * 16 + r8, jb = ja + 8;
+        pa[k] = (ja < n_full) ? __ldg(p.page_table + static_cast<int64_t>(b) * p.pt_stride + ja) : 0;
+        pb[k] = (jb < n_full) ? __ldg(p.page_table + static_cast<int64_t>(b) * p.pt_stride + jb) : 0;
     }
-    __syncthreads();
 }
 
 // Selector queries of head group g for the quantised-key scorer, as f16 mma
@@ -236,45 +204,34 @@ __device__ __forceinline__ void load_queries_f16(const SelectParams& p, int b, i
     wh1 = (2 * c4 + 1 < G) ? (p.w ? p.w[wrow + 2 * c4 + 1] : 1.f / G) : 0.f;
 }
 
-// Scale of group grp (dims 32 grp .. + 31) from a staged scale word.
+// Scale of group grp (dims 32 grp .. + 31) from a row's scale word.
 template <int FMT>
-__device__ __forceinline__ float staged_scale(uint32_t w, int grp) {
+__device__ __forceinline__ float frag_scale(uint32_t w, int grp) {
     if (FMT == SPOT_SEL_INT4_G32_F16)
         return __half2float(__ushort_as_half(static_cast<uint16_t>(w >> (16 * grp))));
     if (FMT == SPOT_SEL_INT8_F16) return __half2float(__ushort_as_half(static_cast<uint16_t>(w)));
     return e8m0_value((w >> (8 * grp)) & 0xFFu);
 }
 
-// Query-key dot products of the 16 staged rows 16 t .. 16 t + 15 for the
-// group's heads: keys as the mma M operand, the selector queries as N = 8
-// (qw: B fragments, lane: head r8; qsc: query scales).  acc: rows r8 and
-// r8 + 8 of this lane, columns (heads) 2 c4 and 2 c4 + 1.  Branch-free, so
-// that a warp's two tiles in flight interleave.
+// Query-key dot products of one tile from its fragments, for the group's
+// heads: keys as the mma M operand, the selector queries as N = 8 (qw: B
+// fragments, lane: head r8; qsc: query scales).  acc: rows r8 and r8 + 8 of
+// this lane, columns (heads) 2 c4 and 2 c4 + 1.
 template <int FMT>
-__device__ __forceinline__ void tile_dots(const uint8_t* stg, const uint32_t* stg_sc, int t,
-                                          const uint32_t (&qw)[8], const float (&qsc)[2][2],
-                                          int lane, float (&acc)[4]) {
-    const int c4 = lane & 3, r8 = lane >> 2;
-    const int ra = 16 * t + r8, rb = ra + 8;
+__device__ __forceinline__ void frag_dots(const KeyFrag& f, const uint32_t (&qw)[8],
+                                          const float (&qsc)[2][2], float (&acc)[4]) {
     acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
     if (FMT == SPOT_SEL_BF16) {
-        const uint4 a0 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(ra, 2 * c4));
-        const uint4 a1 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(ra, 2 * c4 + 1));
-        const uint4 b0 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(rb, 2 * c4));
-        const uint4 b1 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(rb, 2 * c4 + 1));
-        const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const uint32_t wa[8] = {f.a0.x, f.a0.y, f.a0.z, f.a0.w, f.a1.x, f.a1.y, f.a1.z, f.a1.w};
+        const uint32_t wb[8] = {f.b0.x, f.b0.y, f.b0.z, f.b0.w, f.b1.x, f.b1.y, f.b1.z, f.b1.w};
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            mma_bf16_16816(acc, wa[2 * s], wb[2 * s], wa[2 * s + 1], wb[2 * s + 1], qw[2 * s],
-                           qw[2 * s + 1]);
+        for (int s2 = 0; s2 < 4; ++s2)
+            mma_bf16_16816(acc, wa[2 * s2], wb[2 * s2], wa[2 * s2 + 1], wb[2 * s2 + 1], qw[2 * s2],
+                           qw[2 * s2 + 1]);
     } else if (FMT == SPOT_SEL_FP8_E4M3 || FMT == SPOT_SEL_INT8_F16) {
-        // 64-byte rows: lane c4 owns bytes (= dims) [16 c4, 16 c4 + 16), widened
-        // exactly to f16 four codes at a time (pairs (0, 1) and (2, 3))
-        const uint4 ra4 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(ra, c4));
-        const uint4 rb4 = *reinterpret_cast<const uint4*>(stg + piece_off<FMT>(rb, c4));
-        const uint32_t wa[4] = {ra4.x, ra4.y, ra4.z, ra4.w};
-        const uint32_t wb[4] = {rb4.x, rb4.y, rb4.z, rb4.w};
+        // codes widened exactly to f16 four at a time (pairs (0, 1) and (2, 3))
+        const uint32_t wa[4] = {f.a0.x, f.a0.y, f.a0.z, f.a0.w};
+        const uint32_t wb[4] = {f.b0.x, f.b0.y, f.b0.z, f.b0.w};
 #pragma unroll
         for (int s2 = 0; s2 < 4; ++s2) {
             uint32_t alo, ahi, blo, bhi;
@@ -287,30 +244,26 @@ __device__ __forceinline__ void tile_dots(const uint8_t* stg, const uint32_t* st
             }
             mma_f16_16816(acc, alo, blo, ahi, bhi, qw[2 * s2], qw[2 * s2 + 1]);
         }
-        const float sca = FMT == SPOT_SEL_INT8_F16 ? staged_scale<FMT>(stg_sc[ra], 0) : 1.f;
-        const float scb = FMT == SPOT_SEL_INT8_F16 ? staged_scale<FMT>(stg_sc[rb], 0) : 1.f;
+        const float sca = FMT == SPOT_SEL_INT8_F16 ? frag_scale<FMT>(f.sa, 0) : 1.f;
+        const float scb = FMT == SPOT_SEL_INT8_F16 ? frag_scale<FMT>(f.sb, 0) : 1.f;
         acc[0] = acc[0] * sca * qsc[0][0];
         acc[1] = acc[1] * sca * qsc[0][1];
         acc[2] = acc[2] * scb * qsc[0][0];
         acc[3] = acc[3] * scb * qsc[0][1];
     } else {
-        // 32-byte rows: lane c4 owns bytes [4 c4, 4 c4 + 4) of each 16-byte
-        // half (half 0 = group 0 = dims 0-31, half 1 = group 1), widened
-        // exactly to f16 (pairs (j, j + 4); E2M1 as value x 2^-14, undone in
-        // the scale)
-        const uint32_t swa = stg_sc[ra], swb = stg_sc[rb];
+        // codes widened exactly to f16 (pairs (j, j + 4); E2M1 as value x
+        // 2^-14, undone in the scale)
         float accg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const uint32_t wa[2] = {f.a0.x, f.a0.y}, wb[2] = {f.b0.x, f.b0.y};
 #pragma unroll
         for (int grp = 0; grp < 2; ++grp) {
-            const uint32_t wa = *reinterpret_cast<const uint32_t*>(stg + piece_off<FMT>(ra, grp) + 4 * c4);
-            const uint32_t wb = *reinterpret_cast<const uint32_t*>(stg + piece_off<FMT>(rb, grp) + 4 * c4);
             uint32_t oa[4], ob[4];
             if (FMT == SPOT_SEL_INT4_G32_F16) {
-                int4x8_to_f16x2(wa, oa);
-                int4x8_to_f16x2(wb, ob);
+                int4x8_to_f16x2(wa[grp], oa);
+                int4x8_to_f16x2(wb[grp], ob);
             } else {
-                e2m1x8_to_f16x2_scaled(wa, oa);
-                e2m1x8_to_f16x2_scaled(wb, ob);
+                e2m1x8_to_f16x2_scaled(wa[grp], oa);
+                e2m1x8_to_f16x2_scaled(wb[grp], ob);
             }
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2)
@@ -318,8 +271,8 @@ __device__ __forceinline__ void tile_dots(const uint8_t* stg, const uint32_t* st
                               qw[4 * grp + 2 * s2], qw[4 * grp + 2 * s2 + 1]);
         }
         constexpr float kw = FMT == SPOT_SEL_MXFP4_G32_E8M0 ? 16384.f : 1.f;
-        const float sa0 = staged_scale<FMT>(swa, 0) * kw, sa1 = staged_scale<FMT>(swa, 1) * kw;
-        const float sb0 = staged_scale<FMT>(swb, 0) * kw, sb1 = staged_scale<FMT>(swb, 1) * kw;
+        const float sa0 = frag_scale<FMT>(f.sa, 0) * kw, sa1 = frag_scale<FMT>(f.sa, 1) * kw;
+        const float sb0 = frag_scale<FMT>(f.sb, 0) * kw, sb1 = frag_scale<FMT>(f.sb, 1) * kw;
         acc[0] = accg[0][0] * sa0 * qsc[0][0] + accg[1][0] * sa1 * qsc[1][0];
         acc[1] = accg[0][1] * sa0 * qsc[0][1] + accg[1][1] * sa1 * qsc[1][1];
         acc[2] = accg[0][2] * sb0 * qsc[0][0] + accg[1][2] * sb1 * qsc[1][0];
@@ -327,15 +280,14 @@ __device__ __forceinline__ void tile_dots(const uint8_t* stg, const uint32_t* st
     }
 }
 
-// Scores of tile t from its dot products: weighted ReLU sum over the group's
-// heads (wh0 / wh1: weights of heads 2 c4, 2 c4 + 1, 0 for padding heads),
-// written for the rows below n (blocks j0 + row); tracks the maximum /
-// minimum of the residual scores [r0, r1).
+// Scores of tile t (blocks 16 t .. 16 t + 15) from its dot products:
+// weighted ReLU sum over the group's heads (wh0 / wh1: weights of heads
+// 2 c4, 2 c4 + 1, 0 for padding heads), written for the blocks below n_full;
+// tracks the maximum / minimum of the residual scores [r0, r1).
 __device__ __forceinline__ void tile_scores(const SelectParams& p, const float (&acc)[4], int t,
-                                            int j0, int n, float wh0, float wh1, float* scores,
+                                            int n_full, float wh0, float wh1, float* scores,
                                             int lane, int r0, int r1, float& wmax, float& wmin) {
     const int c4 = lane & 3, r8 = lane >> 2;
-    const int ra = 16 * t + r8, rb = ra + 8;
     float sa = wh0 * fmaxf(acc[0], 0.f) + wh1 * fmaxf(acc[1], 0.f);
     float sb = wh0 * fmaxf(acc[2], 0.f) + wh1 * fmaxf(acc[3], 0.f);
     sa += __shfl_xor_sync(0xffffffffu, sa, 1);
@@ -343,12 +295,12 @@ __device__ __forceinline__ void tile_scores(const SelectParams& p, const float (
     sb += __shfl_xor_sync(0xffffffffu, sb, 1);
     sb += __shfl_xor_sync(0xffffffffu, sb, 2);
     if (c4 == 0) {
-        const int ja = j0 + ra, jb = j0 + rb;
+        const int ja = 16 * t + r8, jb = ja + 8;
         const float va = sa * p.inv_temp, vb = sb * p.inv_temp;
-        if (ra < n) scores[ja] = va;
-        if (rb < n) scores[jb] = vb;
-        if (ra < n && ja >= r0 && ja < r1) { wmax = fmaxf(wmax, va); wmin = fminf(wmin, va); }
-        if (rb < n && jb >= r0 && jb < r1) { wmax = fmaxf(wmax, vb); wmin = fminf(wmin, vb); }
+        if (ja < n_full) scores[ja] = va;
+        if (jb < n_full) scores[jb] = vb;
+        if (ja >= r0 && ja < r1) { wmax = fmaxf(wmax, va); wmin = fminf(wmin, va); }
+        if (jb >= r0 && jb < r1) { wmax = fmaxf(wmax, vb); wmin = fminf(wmin, vb); }
     }
 }
 
@@ -445,92 +397,108 @@ __device__ __forceinline__ unsigned long long bucket_mass(const SelSmem& sm, int
 // target is T = ceil(pb * Z), Z the residual blocks' total mass, clamped to
 // [1, Z], and *target receives it; else *target holds the count to reach
 // (>= 1).  Returns the bucket; *before receives the count and *above the
-// mass (count) of the elements in the buckets above it.  Two barriers: the
-// warps' totals, then a lane scan in the one warp whose buckets hold the
-// crossing point.
+// mass (count) of the elements in the buckets above it.  One barrier: the
+// warps publish the totals of their bucket slices; then every warp finds the
+// crossing slice with a lane scan over those totals and, redundantly but
+// identically, the crossing bucket inside it from the histograms.
+// Bucket slice of warp w, lane l: buckets (32 w + l) * PER .. + PER - 1.
+__device__ __forceinline__ void lane_buckets(const SelSmem& sm, bool by_mass, int lb, int per,
+                                             unsigned long long& v, int& c) {
+    v = 0;
+    c = 0;
+    for (int k = 0; k < per; ++k) {
+        const uint32_t n = sm.hcnt[lb + k];
+        v += by_mass ? bucket_mass(sm, lb + k) : n;
+        c += static_cast<int>(n);
+    }
+}
+
 __device__ int cut_bucket(const SelSmem& sm, bool by_mass, float pb, unsigned long long* target,
                           int* before, unsigned long long* above, int nbk) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int PER = nbk / NT;
-    unsigned long long loc = 0;
-    int cnt = 0, last = -1;
-    for (int k = 0; k < PER; ++k) {
-        const int bkt = threadIdx.x * PER + k;
-        const uint32_t c = sm.hcnt[bkt];
-        loc += by_mass ? bucket_mass(sm, bkt) : c;
-        cnt += static_cast<int>(c);
-        if (c) last = bkt;
-    }
+    unsigned long long loc;
+    int cnt;
+    lane_buckets(sm, by_mass, threadIdx.x * PER, PER, loc, cnt);
     const unsigned long long wv = warp_sum(loc);
     const int wc = warp_sum(cnt);
-    int wl = last;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wl = max(wl, __shfl_xor_sync(0xffffffffu, wl, o));
-    int* wint = reinterpret_cast<int*>(sm.red + NW);  // [NW] counts, [NW] last buckets
+    int* wint = reinterpret_cast<int*>(sm.red + NW);  // [NW] counts
     if (lane == 0) {
         sm.red[warp] = wv;
         wint[warp] = wc;
-        wint[NW + warp] = wl;
     }
     __syncthreads();
-    unsigned long long tot = 0;
-    for (int w = 0; w < NW; ++w) tot += sm.red[w];
+    // every warp: the slices' totals, one per lane, and their inclusive scan
+    static_assert(NW <= 32, "one lane per warp slice");
+    const unsigned long long sv = lane < NW ? sm.red[lane] : 0ull;
+    const int scn = lane < NW ? wint[lane] : 0;
+    unsigned long long incl = sv;
+    int cincl = scn;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long x = __shfl_up_sync(0xffffffffu, incl, o);
+        const int y = __shfl_up_sync(0xffffffffu, cincl, o);
+        if (lane >= o) { incl += x; cincl += y; }
+    }
+    const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
+    const int ctot = __shfl_sync(0xffffffffu, cincl, 31);
     unsigned long long tgt = *target;
     if (by_mass) {
         tgt = static_cast<unsigned long long>(ceil(static_cast<double>(pb) * static_cast<double>(tot)));
         tgt = tgt < 1ull ? 1ull : (tgt > tot ? tot : tgt);
         *target = tgt;
     }
-    // every thread finds the warp whose buckets reach the target
-    unsigned long long run = 0;
-    int crun = 0, cw = -1, ctot = 0, lastb = -1;
-    for (int w = 0; w < NW; ++w) {
-        const unsigned long long v = sm.red[w];
-        const int c = wint[w];
-        if (cw < 0) {
-            if (run + v >= tgt) cw = w;
-            else { run += v; crun += c; }
-        }
-        ctot += c;
-        lastb = max(lastb, wint[NW + w]);
-    }
-    if (warp == cw) {                                 // warp-uniform
-        unsigned long long incl = loc;
-        int cincl = cnt;
+    const unsigned cross = __ballot_sync(0xffffffffu, lane < NW && incl >= tgt);
+    if (cross == 0u) {
+        // (not reached: the target never exceeds the total) the lowest
+        // non-empty bucket, found from the top by every warp alike
+        int lastb = 0;
+        for (int bk = lane; bk < nbk; bk += 32)
+            if (sm.hcnt[bk] != 0u) lastb = bk;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long x = __shfl_up_sync(0xffffffffu, incl, o);
-            const int y = __shfl_up_sync(0xffffffffu, cincl, o);
-            if (lane >= o) { incl += x; cincl += y; }
-        }
-        unsigned long long r = run + incl - loc;
-        int cr = crun + cincl - cnt;
-        if (r < tgt && r + loc >= tgt) {              // one lane
-            for (int k = 0; k < PER; ++k) {
-                const int bkt = threadIdx.x * PER + k;
-                const uint32_t c = sm.hcnt[bkt];
-                const unsigned long long v = by_mass ? bucket_mass(sm, bkt) : c;
-                if (c && r + v >= tgt) {
-                    sm.misc[0] = bkt;
-                    sm.misc[2] = cr;
-                    sm.red[3 * NW - 1] = r;
-                    break;
-                }
-                r += v;
-                cr += static_cast<int>(c);
-            }
-        }
+        for (int o = 16; o > 0; o >>= 1) lastb = max(lastb, __shfl_xor_sync(0xffffffffu, lastb, o));
+        *before = ctot - static_cast<int>(sm.hcnt[lastb]);
+        *above = tot - (by_mass ? bucket_mass(sm, lastb) : sm.hcnt[lastb]);
+        return lastb;
     }
-    __syncthreads();
-    if (cw >= 0) {
-        *before = sm.misc[2];
-        *above = sm.red[3 * NW - 1];
-        return sm.misc[0];
+    const int cw = __ffs(cross) - 1;                  // the crossing slice (warp)
+    const unsigned long long run = __shfl_sync(0xffffffffu, incl - sv, cw);
+    const int crun = __shfl_sync(0xffffffffu, cincl - scn, cw);
+    // its lanes' sums (re-read from the histograms), scanned; the lane whose
+    // buckets reach the target walks them
+    unsigned long long v;
+    int c;
+    lane_buckets(sm, by_mass, (cw * 32 + lane) * PER, PER, v, c);
+    unsigned long long li = v;
+    int lci = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long x = __shfl_up_sync(0xffffffffu, li, o);
+        const int y = __shfl_up_sync(0xffffffffu, lci, o);
+        if (lane >= o) { li += x; lci += y; }
     }
-    // (not reached: the target never exceeds the total) the lowest non-empty bucket
-    *before = ctot - static_cast<int>(sm.hcnt[lastb]);
-    *above = tot - (by_mass ? bucket_mass(sm, lastb) : sm.hcnt[lastb]);
-    return lastb;
+    const unsigned hit = __ballot_sync(0xffffffffu, run + li >= tgt);
+    const int cl = __ffs(hit) - 1;                    // non-empty: the slice reaches tgt
+    int bk_out = 0, cr_out = 0;
+    unsigned long long r_out = 0;
+    if (lane == cl) {
+        unsigned long long r = run + li - v;
+        int cr = crun + lci - c;
+        const int lb = (cw * 32 + lane) * PER;
+        bk_out = lb + PER - 1;
+        for (int k = 0; k < PER; ++k) {
+            const uint32_t n = sm.hcnt[lb + k];
+            const unsigned long long m = by_mass ? bucket_mass(sm, lb + k) : n;
+            if (n && r + m >= tgt) { bk_out = lb + k; break; }
+            r += m;
+            cr += static_cast<int>(n);
+        }
+        r_out = r;
+        cr_out = cr;
+    }
+    *before = __shfl_sync(0xffffffffu, cr_out, cl);
+    *above = __shfl_sync(0xffffffffu, r_out, cl);
+    return __shfl_sync(0xffffffffu, bk_out, cl);
 }
 
 // Appends element i (when `hit`) to the candidate list (sm.ckey / sm.cidx,
@@ -735,6 +703,18 @@ __device__ __forceinline__ SelSmem carve_select_smem(uint8_t* smem, int max_bloc
     return sm;
 }
 
+// Zeroes the bucket histograms and the tie count of the selection; called at
+// kernel entry, so that it overlaps the scoring (select_unit's first barrier
+// orders it before the histograms are filled).
+__device__ __forceinline__ void clear_select(const SelSmem& sm) {
+    for (int i = threadIdx.x; i < kNB; i += NT) {
+        sm.hlo[i] = 0u;
+        sm.hhi[i] = 0u;
+        sm.hcnt[i] = 0u;
+    }
+    if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
+}
+
 // Blocks of a sequence of L tokens: nb in all and n_full complete ones
 // (both at most the table's capacity; `over` when it had to clip), and the
 // residual blocks [r0, r1) left by the sink and recency reservations (the
@@ -780,9 +760,7 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     const int n = r1 - r0;
     const int n_reserved = nb - n;
     const float* s = sm.score;
-    const int nbk = n > 2048 ? 2048 : 1024;          // value buckets
-    for (int i = threadIdx.x; i < nbk; i += NT) { sm.hlo[i] = 0u; sm.hhi[i] = 0u; sm.hcnt[i] = 0u; }
-    if (threadIdx.x == 0) sm.misc[5] = 0;             // ties taken at a key cut
+    const int nbk = n > 2048 ? 2048 : 1024;          // value buckets (zeroed by clear_select)
     pdl_trigger();                                    // the decode kernel may start its prologue
 
     // ---- selector scores of the complete blocks (§2.1), into shared memory
@@ -1011,6 +989,7 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
 __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
     const SelSmem sm = carve_select_smem(smem, p.max_blocks);
+    clear_select(sm);
     pdl_wait();                  // the scores (and the lengths and p) may come from it
     const int b = blockIdx.x / p.num_kv_heads;
     const int L = max(p.seq_lens[b], 0);
@@ -1019,21 +998,20 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(const SelectP
 }
 
 // Scoring (§2.1, Eq. 2) and selection in one launch.  The C CTAs of a unit
-// (one thread-block cluster when C > 1) split its 16-block tiles into C
-// contiguous shares; each CTA gathers its share's selector rows into its
-// own shared memory (in passes of at most `pass_rows` rows) and scores them
-// there, each warp taking every NW-th tile.  Every CTA stores its scores
-// straight into the shared memory of the cluster's first CTA, which selects
-// once the cluster barrier (release / acquire at cluster scope) has passed.
+// (one thread-block cluster when C > 1) share its 16-block tiles: CTA c
+// takes rounds c, c + C, ... of NW * kTileBatch tiles (one batch of
+// kTileBatch tiles per warp per round, the next round's page ids loading
+// while this round's keys do).  Every CTA stores its scores straight into
+// the shared memory of the cluster's first CTA, which selects once the
+// cluster barrier (release / acquire at cluster scope) has passed.
 template <int FMT>
 __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const SelectParams p,
-                                                                         int C, int stage_off,
-                                                                         int pass_rows) {
+                                                                         int C) {
+    constexpr int TB = tile_batch<FMT>();
     extern __shared__ __align__(16) uint8_t smem[];
     const SelSmem sm = carve_select_smem(smem, p.max_blocks);
-    uint8_t* stg = smem + stage_off;                                 // staged rows
-    uint32_t* stg_sc = reinterpret_cast<uint32_t*>(stg + pass_rows * row_stride<FMT>());
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    clear_select(sm);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c4 = lane & 3;
     const int u = blockIdx.x / C, c = blockIdx.x - u * C;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
     const int L = max(p.seq_lens[b], 0);
@@ -1041,9 +1019,6 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
     const BlockSpan sp = block_span(p, L);                           // overflow: flagged
     const int n_full = sp.n_full;                                    // by the selection
     const int tiles = (n_full + 15) / 16;
-    const int t_lo = static_cast<int>(static_cast<int64_t>(tiles) * c / C);
-    const int t_hi = static_cast<int>(static_cast<int64_t>(tiles) * (c + 1) / C);
-    const int j_lo = 16 * t_lo, j_hi = min(n_full, 16 * t_hi);     // this CTA's blocks
     float* out = sm.score;                                           // the leader's
     float* part = sm.part;
     if (C > 1) {
@@ -1051,43 +1026,44 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
         out = cooperative_groups::this_cluster().map_shared_rank(sm.score, 0);
         part = cooperative_groups::this_cluster().map_shared_rank(sm.part, 0);
     }
+    bool waited = C == 1;             // every CTA of the cluster known to have started
     float wmax = -INFINITY, wmin = INFINITY;                         // residual scores
-    if (j_hi > j_lo) {
-        int pg[kMaxRowsPerThread];
-        stage_pages(p, b, j_lo, min(pass_rows, j_hi - j_lo), pg);   // in flight with the queries
+    constexpr int kRound = NW * TB;
+    const int step = C * kRound;
+    const int first = c * kRound + warp;
+    if (first < tiles) {                                             // warp-uniform
+        int pa[TB], pb[TB];
+        load_pages<FMT>(p, b, first, NW, n_full, lane, pa, pb);      // in flight with the queries
         uint32_t qw[8];
         float qsc[2][2], wh0, wh1;
         if (FMT == SPOT_SEL_BF16) load_queries<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
         else load_queries_f16<FMT>(p, b, g, lane, qw, qsc, wh0, wh1);
-        for (int j0 = j_lo; j0 < j_hi; j0 += pass_rows) {
-            const int n = min(pass_rows, j_hi - j0);
-            if (j0 != j_lo) stage_pages(p, b, j0, n, pg);
-            uint32_t sc[kMaxRowsPerThread];
-            stage_issue<FMT>(p, g, n, pg, stg, sc);
-            if (C > 1 && j0 == j_lo) {
-                // every CTA of the cluster has started before the first remote
-                // store into the leader's shared memory
+        for (int t0 = first; t0 < tiles; t0 += step) {
+            KeyFrag fr[TB];
+#pragma unroll
+            for (int k = 0; k < TB; ++k) {
+                int ra = pa[k], rb = pb[k];
+                if (ra < 0 || ra >= p.num_pages) { flag_status(p.status, kStatusBounds); ra = 0; }
+                if (rb < 0 || rb >= p.num_pages) { flag_status(p.status, kStatusBounds); rb = 0; }
+                load_frag<FMT>(p, static_cast<int64_t>(ra) * p.num_kv_heads + g,
+                               static_cast<int64_t>(rb) * p.num_kv_heads + g, c4, fr[k]);
+            }
+            if (t0 + step < tiles) load_pages<FMT>(p, b, t0 + step, NW, n_full, lane, pa, pb);
+            float acc[TB][4];
+#pragma unroll
+            for (int k = 0; k < TB; ++k) frag_dots<FMT>(fr[k], qw, qsc, acc[k]);
+            if (!waited) {
+                // before the first remote store into the leader's shared memory
                 cluster_wait();
+                waited = true;
             }
-            // row group k (NT rows, 2 tiles per warp) is scored while the
-            // groups after it are still landing
-            for (int k = 0; k * NT < n; ++k) {
-                stage_wait<FMT>(k, n, sc, stg_sc);
-                const int t0 = k * (NT / 16) + warp, t1 = t0 + NW;
-                const bool two = 16 * t1 < n;
-                float a0[4], a1[4];
-                if (16 * t0 < n) tile_dots<FMT>(stg, stg_sc, t0, qw, qsc, lane, a0);
-                if (two) tile_dots<FMT>(stg, stg_sc, t1, qw, qsc, lane, a1);
-                if (16 * t0 < n)
-                    tile_scores(p, a0, t0, j0, n, wh0, wh1, out, lane, sp.r0, sp.r1, wmax, wmin);
-                if (two)
-                    tile_scores(p, a1, t1, j0, n, wh0, wh1, out, lane, sp.r0, sp.r1, wmax, wmin);
-            }
-            __syncthreads();                                         // staging is free again
+#pragma unroll
+            for (int k = 0; k < TB; ++k)
+                tile_scores(p, acc[k], t0 + k * NW, n_full, wh0, wh1, out, lane, sp.r0, sp.r1,
+                            wmax, wmin);
         }
-    } else if (C > 1) {
-        cluster_wait();
     }
+    if (!waited) cluster_wait();
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
@@ -1141,35 +1117,17 @@ cudaError_t allow_smem(Kernel kernel, int slot, size_t smem) {
     return e;
 }
 
-// Largest dynamic shared memory a CTA may use on the current device.
-int smem_optin() {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-        return 0;
-    return v;
-}
-
 template <int FMT>
-cudaError_t launch_score_select(const SelectParams& p, size_t smem_sel, cudaStream_t s) {
-    // CTAs per unit: one per 32 tiles of the longest sequence, as far as one
-    // wave of one CTA per SM allows (at most a portable cluster of 8)
-    const int U = p.batch * p.num_kv_heads;
-    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
-    const int tiles = (cap + 15) / 16;
-    const int C = max(1, min(min((tiles + 31) / 32, kMaxCluster), sm_count() / max(U, 1)));
-    // staging for one CTA's share of rows (whole 16-row tiles), in passes of
-    // what fits next to the selection's shared memory
-    const int share = 16 * ((tiles + C - 1) / C);
-    const size_t off = (smem_sel + 15) / 16 * 16;
-    const size_t per_row = row_stride<FMT>() + sizeof(uint32_t);
-    const size_t limit = static_cast<size_t>(smem_optin());
-    if (limit < off + 16 * per_row) return cudaErrorInvalidValue;
-    int pass_rows = static_cast<int>(min((limit - off) / per_row, static_cast<size_t>(NT * kMaxRowsPerThread)));
-    pass_rows = min(pass_rows / 16 * 16, share);
-    const size_t smem = off + static_cast<size_t>(pass_rows) * per_row;
+cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t s) {
     cudaError_t e = allow_smem(score_select_kernel<FMT>, 1 + FMT, smem);
     if (e != cudaSuccess) return e;
+    // CTAs per unit: enough to cover the longest sequence in one round of
+    // NW * kTileBatch tiles each, as far as one wave of one CTA per SM allows
+    const int U = p.batch * p.num_kv_heads;
+    const int cap = min(p.max_blocks, p.pt_stride * p.blocks_per_page);
+    constexpr int kRound = NW * tile_batch<FMT>();
+    const int rounds = max(1, ((cap + 15) / 16 + kRound - 1) / kRound);
+    const int C = max(1, min(min(rounds, kMaxCluster), sm_count() / max(U, 1)));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(U * C);
     cfg.blockDim = dim3(kSelectThreads);
@@ -1182,7 +1140,7 @@ cudaError_t launch_score_select(const SelectParams& p, size_t smem_sel, cudaStre
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = C > 1 ? 1 : 0;                     // C = 1: a plain launch
-    e = cudaLaunchKernelEx(&cfg, score_select_kernel<FMT>, p, C, static_cast<int>(off), pass_rows);
+    e = cudaLaunchKernelEx(&cfg, score_select_kernel<FMT>, p, C);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
