@@ -763,10 +763,14 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
     const int nbk = n > 2048 ? 2048 : 1024;          // value buckets (zeroed by clear_select)
     pdl_trigger();                                    // the decode kernel may start its prologue
 
-    // ---- selector scores of the complete blocks (§2.1), into shared memory
+    // ---- selector scores of the complete blocks (§2.1), into shared memory;
+    // scores read from global memory also give the residual keys and each
+    // warp's maximum / minimum on the way
+    float* wmin = reinterpret_cast<float*>(sm.scan);  // next written after two barriers
     if (!in_smem) {
         const float* src = p.scores_in + static_cast<int64_t>(u) * p.max_blocks;
         constexpr int kBatch = 16;                    // loads in flight per thread
+        float mloc = -INFINITY, nloc = INFINITY;
         for (int j0 = threadIdx.x; j0 < n_full; j0 += NT * kBatch) {
             float v[kBatch];
 #pragma unroll
@@ -775,15 +779,37 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
                 v[k] = j < n_full ? __ldcg(src + j) : 0.f;
             }
 #pragma unroll
-            for (int k = 0; k < kBatch; ++k)
-                if (j0 + k * NT < n_full) sm.score[j0 + k * NT] = v[k];
+            for (int k = 0; k < kBatch; ++k) {
+                const int j = j0 + k * NT;
+                if (j >= n_full) continue;
+                sm.score[j] = v[k];
+                if (j >= r0 && j < r1) {
+                    sm.keys[j - r0] = score_key(v[k]);
+                    mloc = fmaxf(mloc, v[k]);
+                    nloc = fminf(nloc, v[k]);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+            nloc = fminf(nloc, __shfl_xor_sync(0xffffffffu, nloc, o));
+        }
+        if (lane == 0) {
+            sm.fscan[warp] = mloc;
+            wmin[warp] = nloc;
         }
     }
     __syncthreads();
 
     // ---- maximum and minimum of the residual scores (and their keys)
     float smax_f = -INFINITY, smin_f = INFINITY;
-    if (nparts > 0) {                                 // every warp folds the partials
+    if (!in_smem) {                                   // the warps' values, written above
+        for (int w = 0; w < NW; ++w) {
+            smax_f = fmaxf(smax_f, sm.fscan[w]);
+            smin_f = fminf(smin_f, wmin[w]);
+        }
+    } else if (nparts > 0) {                          // every warp folds the partials
         for (int i = lane; i < nparts; i += 32) {
             smax_f = fmaxf(smax_f, sm.part[i]);
             smin_f = fminf(smin_f, sm.part[kMaxCluster * NW + i]);
@@ -806,7 +832,6 @@ __device__ void select_unit(const SelectParams& p, int u, const SelSmem& sm, boo
             mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
             nloc = fminf(nloc, __shfl_xor_sync(0xffffffffu, nloc, o));
         }
-        float* wmin = reinterpret_cast<float*>(sm.scan);  // next written after two barriers
         if (lane == 0) {
             sm.fscan[warp] = mloc;
             wmin[warp] = nloc;
@@ -1011,6 +1036,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) score_select_kernel(const S
     extern __shared__ __align__(16) uint8_t smem[];
     const SelSmem sm = carve_select_smem(smem, p.max_blocks);
     clear_select(sm);
+    // Launched with programmatic stream serialisation: every input may come
+    // from the kernel before this one on the stream, so nothing is read (and
+    // nothing written) until that grid has completed; a predecessor that lets
+    // its dependents launch early hides this launch's latency.
+    pdl_wait();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c4 = lane & 3;
     const int u = blockIdx.x / C, c = blockIdx.x - u * C;
     const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
@@ -1133,13 +1163,15 @@ cudaError_t launch_score_select(const SelectParams& p, size_t smem, cudaStream_t
     cfg.blockDim = dim3(kSelectThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = C > 1 ? 1 : 0;                     // C = 1: a plain launch
+    cfg.numAttrs = C > 1 ? 2 : 1;                     // C = 1: no cluster
     e = cudaLaunchKernelEx(&cfg, score_select_kernel<FMT>, p, C);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
