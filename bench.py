@@ -41,22 +41,29 @@ HBM_FALLBACK_GBS = 6650.0
 
 # DRAM bytes (read + write) of one launch of each workload's dominant kernel
 # (dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of the
-# same workload), valid only while the kernel's source files are unchanged
-# (sha256 prefix over them); otherwise the roofline's traffic is null.
+# same workload; where the layer caches rotated per step select different
+# amounts, the mean over one launch per cache), valid only while the kernel's
+# source files are unchanged (sha256 prefix over them); otherwise the
+# roofline's traffic is null.
 NCU_TRAFFIC = {
-    "qwen3_32b_128k": {"bytes": 729075456 + 3837184, "files": ["sparse_decode.cu"],
-                       "sha256": "00f3a2b731258513"},
-    "qwen3_8b_128k_tok": {"bytes": 246840064 + 4134144, "files": ["sparse_decode.cu"],
-                          "sha256": "82c100300b60004f"},
-    "qwen3_8b_prefill_32k": {"bytes": 411903488 + 499184128, "files": ["prefill.cu", "tc.cuh"],
+    "qwen3_32b_128k": {"bytes": 735295168 + 1231040, "sel_fmt": "bf16",
+                       "files": ["sparse_decode.cu"],
+                       "sha256": "8561a6cf16c24959"},
+    "qwen3_8b_128k_tok": {"bytes": 307643200 + 1214400, "sel_fmt": "bf16",
+                          "files": ["sparse_decode.cu"],
+                          "sha256": "8561a6cf16c24959"},
+    "qwen3_8b_prefill_32k": {"bytes": 411903488 + 499184128, "sel_fmt": "bf16",
+                             "files": ["prefill.cu", "tc.cuh"],
                              "sha256": "716d0750e6195d2d"},
 }
 
 
-def measured_traffic(workload: str):
+def measured_traffic(args):
+    """The recorded per-launch DRAM bytes, only for the exact capture: same
+    workload, selector format and batch, and the kernel source unchanged."""
     import hashlib
-    rec = NCU_TRAFFIC.get(workload)
-    if rec is None:
+    rec = NCU_TRAFFIC.get(args.workload)
+    if rec is None or args.batch is not None or args.sel_fmt != rec["sel_fmt"]:
         return None
     h = hashlib.sha256()
     for name in rec["files"]:
@@ -443,7 +450,7 @@ def run_spot(args, world, rank, local):
         "roofline": {
             "bound": "hbm", "kernel": "sparse decode (attention + combine)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.workload),
+            "frac": round(achieved / peak, 4), "traffic": measured_traffic(args),
             "peak_source": peak_kind,
             "algorithmic_bytes_per_launch": int(b_sparse), "ms_per_launch": round(dec_ms, 5),
         },
@@ -653,7 +660,7 @@ def run_spot_tok(args, world, rank, local):
                       "token selector (scoring + selection)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": measured_traffic(args.workload) if dom_sparse else None,
+            "traffic": measured_traffic(args) if dom_sparse else None,
             "peak_source": peak_kind,
             "algorithmic_bytes_per_launch": int(kb), "ms_per_launch": round(kms, 5),
         },
@@ -861,7 +868,7 @@ def run_spot_prefill(args, world, rank, local):
                    "parallelism": f"dp{world} (sequences)"},
         "roofline": {"bound": "tensor", "kernel": "sparse prefill (all four kernels)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.workload),
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(args),
                      "traffic_kernel": "prefill_attn_kernel (dram read + write of one launch)",
                      "peak_source": peak_kind,
                      "algorithmic_flops_per_step": int(f_attn + f_score),

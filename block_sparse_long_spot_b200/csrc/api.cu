@@ -88,6 +88,19 @@ bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_row
     return r == CUDA_SUCCESS;
 }
 
+bool make_split_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), 2};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2, 128};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_bytes_map(CUtensorMap* map, const void* base, int64_t lines, int box_lines) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -183,8 +196,9 @@ spot_status_t do_decode(const spot_layer_desc_t* d, const uint16_t* q, const uin
                         int32_t max_blocks, int32_t batch, float softmax_scale, float* out,
                         float* lse, void* ws, const Layout& L, cudaStream_t s) {
     CUtensorMap km, vm;
-    if (!make_pool_map(&km, k_pool, d->num_pages, d->num_kv_heads) ||
-        !make_pool_map(&vm, v_pool, d->num_pages, d->num_kv_heads))
+    const int64_t rows = static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock;
+    if (!make_split_rows_map(&km, k_pool, rows, kBlock) ||
+        !make_split_rows_map(&vm, v_pool, rows, kBlock))
         return SPOT_ERR_CUDA;
     uint8_t* base = static_cast<uint8_t*>(ws);
     DecodeParams p;
@@ -523,7 +537,8 @@ spot_status_t do_tok_decode(const spot_tok_layer_desc_t* d, const uint16_t* q,
                             const Layout& L, cudaStream_t s) {
     CUtensorMap km, vm;
     const int64_t rows = static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock;
-    if (!make_rows_map(&km, k_pool, rows, kTokBlock) || !make_rows_map(&vm, v_pool, rows, kTokBlock))
+    if (!make_split_rows_map(&km, k_pool, rows, kTokBlock) ||
+        !make_split_rows_map(&vm, v_pool, rows, kTokBlock))
         return SPOT_ERR_CUDA;
     uint8_t* base = static_cast<uint8_t*>(ws);
     DecodeParams p;

@@ -128,8 +128,9 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
     if (scratch_address(dev, &scratch) != cudaSuccess) return SPOT_ERR_CUDA;
 
     CUtensorMap km, vm;
-    if (!make_pool_map(&km, k_pool, d->num_pages, d->num_kv_heads) ||
-        !make_pool_map(&vm, v_pool, d->num_pages, d->num_kv_heads))
+    const int64_t rows = static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock;
+    if (!make_split_rows_map(&km, k_pool, rows, kBlock) ||
+        !make_split_rows_map(&vm, v_pool, rows, kBlock))
         return SPOT_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* base = static_cast<uint8_t*>(scratch);

@@ -14,7 +14,8 @@
 // counter is reset to zero by that CTA, so it is zero again for the next call.
 //
 // Inside a CTA one producer warp issues TMA tile loads of the gathered pages
-// (two 64 x 64 bf16 boxes each for K and V, 128-byte swizzled) into a ring
+// (one 3-D box each for K and V: both 128-byte halves of the block's 64 rows,
+// 128-byte swizzled; fewer, larger boxes keep more bytes in flight) into a ring
 // of stages guarded by mbarriers; NC consumer warps each take every NC-th
 // tile and keep their own online-softmax state for the G <= 8 query heads of
 // the unit's KV head:
@@ -26,10 +27,10 @@
 //
 // The same kernel serves the token-level selector (S16): there one
 // selection per sequence, in blocks of 16 tokens, is shared by every KV head
-// of the sequence, and a stage gathers four selected 16-token blocks (four
-// 16-row boxes each for K and V, into the four 16-row slices of the tile), so
-// the consumers' 64-token tile computation is unchanged; each slice carries
-// its own count of valid tokens.
+// of the sequence, and a stage gathers four selected 16-token blocks (one
+// 16-row box of both halves per block for K and for V), so the consumers'
+// 64-token tile computation is unchanged but for the slice-major addressing;
+// each slice carries its own count of valid tokens.
 #include <math.h>
 #include <stdio.h>
 
@@ -50,8 +51,19 @@ static_assert(STAGES % NC == 0, "stage count must be a multiple of the consumer 
 constexpr int kThreads = (NC + 1) * 32;
 constexpr int kHalfTile = kBlock * 64 * 2;   // 8 KiB: 64 rows x 64 bf16
 
+// Shared-memory layout of the K (and, 16 KiB on, the V) part of a stage.
+// Whole blocks: [half][64 rows][128 B], the hi half kHalfTile after the lo.
+// 16-token slices (S16): [slice][half][16 rows][128 B], 4 KiB per slice.
+// kHalfStride<S16> is the offset of the hi half; row r of the tile (slice
+// r / 16) sits at 128-byte row r + kSliceSkip<S16> * (r / 16) of its half,
+// which keeps each half's rows 1024-byte-atom aligned for the swizzle.
+template <bool S16>
+constexpr int kHalfStride = S16 ? kHalfTile / 4 : kHalfTile;
+template <bool S16>
+constexpr int kSliceSkip = S16 ? 16 : 0;
+
 struct Smem {
-    // stage s: [K lo | K hi | V lo | V hi], 8 KiB each, 1024-byte aligned
+    // stage s: K then V, 16 KiB each (layout above), 1024-byte aligned
     uint32_t stage_base;
     uint64_t* full;
     uint64_t* empty;
@@ -362,12 +374,10 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                         uint8_t* dst = base + s * kStageBytes;
 #pragma unroll
                         for (int e = 0; e < (S16 ? 4 : 1); ++e) {
-                            // S16: slice e = rows [16 e, 16 e + 16) of each half
-                            uint8_t* d = dst + e * (kHalfTile / 4);
-                            tma_load_2d(d, &k_map, &full[s], 0, r[e], policy);
-                            tma_load_2d(d + kHalfTile, &k_map, &full[s], 64, r[e], policy);
-                            tma_load_2d(d + 2 * kHalfTile, &v_map, &full[s], 0, r[e], policy);
-                            tma_load_2d(d + 3 * kHalfTile, &v_map, &full[s], 64, r[e], policy);
+                            // S16: slice e = tile rows [16 e, 16 e + 16)
+                            uint8_t* d = dst + e * (2 * kHalfStride<S16>);
+                            tma_load_3d(d, &k_map, &full[s], 0, r[e], 0, policy);
+                            tma_load_3d(d + 2 * kHalfTile, &v_map, &full[s], 0, r[e], 0, policy);
                         }
                     }
                 }
@@ -442,11 +452,12 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                 for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t hb = kb + (ks >> 2) * kHalfTile;
+                const uint32_t hb = kb + (ks >> 2) * kHalfStride<S16>;
                 const int chunk = ((ks & 3) << 1) + (lane >> 4);
 #pragma unroll
                 for (int mt = 0; mt < 4; ++mt) {
-                    const int row = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    const int row = mt * (16 + kSliceSkip<S16>) + (lane & 7) +
+                                    (((lane >> 3) & 1) << 3);
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4(swz128(hb, row, chunk), a0, a1, a2, a3);
                     mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
@@ -506,11 +517,11 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
             // ---- O^T += V^T P^T: 8 m-tiles of 16 dims x 4 k-tiles of 16 tokens
 #pragma unroll
             for (int md = 0; md < 8; ++md) {
-                const uint32_t hb = vb + (md >> 2) * kHalfTile;
+                const uint32_t hb = vb + (md >> 2) * kHalfStride<S16>;
                 const int chunk = ((md & 3) << 1) + ((lane >> 3) & 1);
 #pragma unroll
                 for (int kt = 0; kt < 4; ++kt) {
-                    const int row = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
+                    const int row = kt * (16 + kSliceSkip<S16>) + (lane & 7) + ((lane >> 4) << 3);
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4_trans(swz128(hb, row, chunk), a0, a1, a2, a3);
                     mma_bf16_16816(acc[md], a0, a1, a2, a3, pb[kt][0], pb[kt][1]);

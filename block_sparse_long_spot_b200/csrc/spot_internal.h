@@ -209,6 +209,12 @@ bool make_pool_map(CUtensorMap* map, const void* pool, int num_pages, int num_kv
 // Tensor map over `rows` rows of 128 bf16 (256 B), box 64 columns x
 // box_rows rows, 128-byte swizzle.
 bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
+// Tensor map over `rows` rows of 128 bf16 (256 B) viewed as [2 halves][rows]
+// [64 bf16] (the half is the outermost coordinate, 128 B apart): one box of
+// 64 columns x box_rows rows x 2 halves brings both 128-byte halves of
+// box_rows consecutive rows in one copy, laid out [half][row][128 B] with
+// 128-byte swizzle.
+bool make_split_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 // Tensor map over `lines` lines of 128 bytes, box 128 bytes x box_lines,
 // 128-byte swizzle.
 bool make_bytes_map(CUtensorMap* map, const void* base, int64_t lines, int box_lines);
