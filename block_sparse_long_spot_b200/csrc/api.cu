@@ -101,6 +101,16 @@ bool make_split_rows_map(CUtensorMap* map, const void* base, int64_t rows, int b
     return r == CUDA_SUCCESS;
 }
 
+bool make_decode_maps(DecodeMaps* m, const void* k_pool, const void* v_pool, int64_t rows,
+                      bool slices) {
+    *m = DecodeMaps{};
+    for (int h = slices ? 1 : 4; h <= 4; ++h)
+        if (!make_split_rows_map(&m->k[h - 1], k_pool, rows, 16 * h) ||
+            !make_split_rows_map(&m->v[h - 1], v_pool, rows, 16 * h))
+            return false;
+    return true;
+}
+
 bool make_bytes_map(CUtensorMap* map, const void* base, int64_t lines, int box_lines) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -195,11 +205,9 @@ spot_status_t do_decode(const spot_layer_desc_t* d, const uint16_t* q, const uin
                         const int32_t* seq_lens, const int32_t* sel_idx, const int32_t* sel_cnt,
                         int32_t max_blocks, int32_t batch, float softmax_scale, float* out,
                         float* lse, void* ws, const Layout& L, cudaStream_t s) {
-    CUtensorMap km, vm;
+    DecodeMaps maps;
     const int64_t rows = static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock;
-    if (!make_split_rows_map(&km, k_pool, rows, kBlock) ||
-        !make_split_rows_map(&vm, v_pool, rows, kBlock))
-        return SPOT_ERR_CUDA;
+    if (!make_decode_maps(&maps, k_pool, v_pool, rows, false)) return SPOT_ERR_CUDA;
     uint8_t* base = static_cast<uint8_t*>(ws);
     DecodeParams p;
     p.q = q;
@@ -221,7 +229,7 @@ spot_status_t do_decode(const spot_layer_desc_t* d, const uint16_t* q, const uin
     p.out = out;
     p.lse = lse;
     p.status = reinterpret_cast<uint32_t*>(base + L.status);
-    if (launch_sparse_decode(p, km, vm, false, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    if (launch_sparse_decode(p, maps, false, s) != cudaSuccess) return SPOT_ERR_CUDA;
     return SPOT_OK;
 }
 
@@ -535,11 +543,9 @@ spot_status_t do_tok_decode(const spot_tok_layer_desc_t* d, const uint16_t* q,
                             const int32_t* sel_cnt, int32_t max_blocks, int32_t batch,
                             float softmax_scale, float* out, float* lse, void* ws,
                             const Layout& L, cudaStream_t s) {
-    CUtensorMap km, vm;
+    DecodeMaps maps;
     const int64_t rows = static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock;
-    if (!make_split_rows_map(&km, k_pool, rows, kTokBlock) ||
-        !make_split_rows_map(&vm, v_pool, rows, kTokBlock))
-        return SPOT_ERR_CUDA;
+    if (!make_decode_maps(&maps, k_pool, v_pool, rows, true)) return SPOT_ERR_CUDA;
     uint8_t* base = static_cast<uint8_t*>(ws);
     DecodeParams p;
     p.q = q;
@@ -561,7 +567,7 @@ spot_status_t do_tok_decode(const spot_tok_layer_desc_t* d, const uint16_t* q,
     p.out = out;
     p.lse = lse;
     p.status = reinterpret_cast<uint32_t*>(base + L.status);
-    if (launch_sparse_decode(p, km, vm, true, s) != cudaSuccess) return SPOT_ERR_CUDA;
+    if (launch_sparse_decode(p, maps, true, s) != cudaSuccess) return SPOT_ERR_CUDA;
     return SPOT_OK;
 }
 

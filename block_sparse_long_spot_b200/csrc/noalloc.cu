@@ -127,11 +127,9 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
     void* scratch = nullptr;
     if (scratch_address(dev, &scratch) != cudaSuccess) return SPOT_ERR_CUDA;
 
-    CUtensorMap km, vm;
+    DecodeMaps maps;
     const int64_t rows = static_cast<int64_t>(d->num_pages) * d->num_kv_heads * kBlock;
-    if (!make_split_rows_map(&km, k_pool, rows, kBlock) ||
-        !make_split_rows_map(&vm, v_pool, rows, kBlock))
-        return SPOT_ERR_CUDA;
+    if (!make_decode_maps(&maps, k_pool, v_pool, rows, false)) return SPOT_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* base = static_cast<uint8_t*>(scratch);
     // The status word and the per-unit arrival counters must start at zero;
@@ -158,5 +156,5 @@ extern "C" spot_status_t spot_sparse_decode_noalloc(
     p.out = out;
     p.lse = lse;
     p.status = reinterpret_cast<uint32_t*>(base);
-    return launch_sparse_decode(p, km, vm, false, s) == cudaSuccess ? SPOT_OK : SPOT_ERR_CUDA;
+    return launch_sparse_decode(p, maps, false, s) == cudaSuccess ? SPOT_OK : SPOT_ERR_CUDA;
 }

@@ -27,10 +27,12 @@
 //
 // The same kernel serves the token-level selector (S16): there one
 // selection per sequence, in blocks of 16 tokens, is shared by every KV head
-// of the sequence, and a stage gathers four selected 16-token blocks (one
-// 16-row box of both halves per block for K and for V), so the consumers'
-// 64-token tile computation is unchanged but for the slice-major addressing;
-// each slice carries its own count of valid tokens.
+// of the sequence, and a stage gathers four selected 16-token blocks, so the
+// consumers' 64-token tile computation is unchanged but for the addressing.
+// Slices that are the next 16 rows of the same 64-row page block as the
+// slice before them form a run, and each run comes in one box of both halves
+// (16, 32, 48 or 64 rows: one tensor map per height) for K and for V; each
+// slice carries its own count of valid tokens.
 #include <math.h>
 #include <stdio.h>
 
@@ -53,14 +55,22 @@ constexpr int kHalfTile = kBlock * 64 * 2;   // 8 KiB: 64 rows x 64 bf16
 
 // Shared-memory layout of the K (and, 16 KiB on, the V) part of a stage.
 // Whole blocks: [half][64 rows][128 B], the hi half kHalfTile after the lo.
-// 16-token slices (S16): [slice][half][16 rows][128 B], 4 KiB per slice.
-// kHalfStride<S16> is the offset of the hi half; row r of the tile (slice
-// r / 16) sits at 128-byte row r + kSliceSkip<S16> * (r / 16) of its half,
-// which keeps each half's rows 1024-byte-atom aligned for the swizzle.
-template <bool S16>
-constexpr int kHalfStride = S16 ? kHalfTile / 4 : kHalfTile;
-template <bool S16>
-constexpr int kSliceSkip = S16 ? 16 : 0;
+// 16-token slices: [run][half][16 x run length rows][128 B]; a run of h
+// slices starting at slice r0 takes 4 KiB x h from 4 KiB x r0, its hi half
+// 2 KiB x h after its lo half.  Every half starts on a 2 KiB boundary, so the
+// 128-byte swizzle (row index mod 8 within a 1 KiB atom) is the same as in a
+// single box.
+constexpr int kSliceHalf = kHalfTile / 4;    // 2 KiB: 16 rows x 64 bf16
+
+// Bit k of a stage's run mask is set when slice k starts a run (bit 0 always).
+// First slice and length (in slices) of the run holding slice k.
+__device__ __forceinline__ int run_first(uint32_t starts, int k) {
+    return 31 - __clz(starts & ((2u << k) - 1u));
+}
+__device__ __forceinline__ int run_length(uint32_t starts, int first) {
+    const uint32_t rest = starts >> (first + 1);
+    return rest ? __ffs(rest) : 4 - first;
+}
 
 struct Smem {
     // stage s: K then V, 16 KiB each (layout above), 1024-byte aligned
@@ -198,8 +208,7 @@ __device__ __forceinline__ uint32_t pack_valid64(int nvalid) {
 
 template <bool S16>
 __global__ void __launch_bounds__(kThreads)
-sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
-                     const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
+sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -216,7 +225,8 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
     uint64_t* full = reinterpret_cast<uint64_t*>(tail);
     uint64_t* empty = full + STAGES;
     int* valid = reinterpret_cast<int*>(empty + STAGES);
-    int* scan = valid + STAGES;
+    int* runs = valid + STAGES;                        // [STAGES] run masks (16-token slices)
+    int* scan = runs + STAGES;
     volatile int* flags = scan + (kThreads / 32 + 1);   // [0] abort, [1] unit complete
     int* unit_off = scan + (kThreads / 32 + 1) + 2;
     const uint32_t stage_base = smem_u32(base);
@@ -230,9 +240,10 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
         flags[0] = 0;
         flags[1] = 0;
     }
-    if (warp == NC && lane == 0) {
-        prefetch_tensormap(&k_map);
-        prefetch_tensormap(&v_map);
+    if (warp == NC && lane < (S16 ? 4 : 1)) {
+        const int h = S16 ? lane : 3;
+        prefetch_tensormap(&maps.k[h]);
+        prefetch_tensormap(&maps.v[h]);
     }
     pdl_wait();                                       // selection of the previous kernel
     pdl_trigger();
@@ -294,7 +305,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
         for (int base_it = 0; base_it < n_it && alive; base_it += 32) {
             const int it = base_it + lane;
             int row[S16 ? 4 : 1] = {};
-            uint32_t vpack = 0;
+            uint32_t vpack = 0, starts = 1;
             if (it < n_it) {
                 const int pos = beg + it;
                 const int u = find_unit(unit_off, U, pos);
@@ -334,6 +345,10 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         if (row[k] < 0) row[k] = fallback;
+#pragma unroll
+                    for (int k = 1; k < 4; ++k)
+                        if (row[k] != row[k - 1] + kTokBlock || (row[k] & (kBlock - 1)) == 0)
+                            starts |= 1u << k;
                 } else {
                     const int j = p.sel_idx[static_cast<int64_t>(u) * p.max_blocks + i];
                     const int nb = (L + kBlock - 1) / kBlock;
@@ -358,6 +373,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
 #pragma unroll
                 for (int e = 0; e < (S16 ? 4 : 1); ++e) r[e] = __shfl_sync(0xffffffffu, row[e], k);
                 const uint32_t v = __shfl_sync(0xffffffffu, vpack, k);
+                const uint32_t st = S16 ? __shfl_sync(0xffffffffu, starts, k) : 1u;
                 const int itk = base_it + k;
                 const int s = itk % STAGES;
                 const int round = itk / STAGES;
@@ -370,14 +386,24 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                         ok = 0;
                     } else {
                         valid[s] = static_cast<int>(v);
+                        runs[s] = static_cast<int>(st);
                         mbar_arrive_expect_tx(&full[s], kStageBytes);
                         uint8_t* dst = base + s * kStageBytes;
+                        if (S16) {
 #pragma unroll
-                        for (int e = 0; e < (S16 ? 4 : 1); ++e) {
-                            // S16: slice e = tile rows [16 e, 16 e + 16)
-                            uint8_t* d = dst + e * (2 * kHalfStride<S16>);
-                            tma_load_3d(d, &k_map, &full[s], 0, r[e], 0, policy);
-                            tma_load_3d(d + 2 * kHalfTile, &v_map, &full[s], 0, r[e], 0, policy);
+                            for (int e = 0; e < 4; ++e) {
+                                if (!((st >> e) & 1u)) continue;
+                                // the run of slices e .. e + h - 1: tile rows
+                                // [16 e, 16 (e + h)), one box of 16 h rows
+                                const int h = run_length(st, e);
+                                uint8_t* d = dst + e * (2 * kSliceHalf);
+                                tma_load_3d(d, &maps.k[h - 1], &full[s], 0, r[e], 0, policy);
+                                tma_load_3d(d + 2 * kHalfTile, &maps.v[h - 1], &full[s], 0, r[e], 0,
+                                            policy);
+                            }
+                        } else {
+                            tma_load_3d(dst, &maps.k[3], &full[s], 0, r[0], 0, policy);
+                            tma_load_3d(dst + 2 * kHalfTile, &maps.v[3], &full[s], 0, r[0], 0, policy);
                         }
                     }
                 }
@@ -443,6 +469,21 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
             const uint32_t vpack = static_cast<uint32_t>(valid[s]);
             const uint32_t kb = stage_base + s * kStageBytes;
             const uint32_t vb = kb + 2 * kHalfTile;
+            // per 16-row slice m of the tile: offset of its first row in its
+            // lo half (slo) and of its hi half from its lo half (shs)
+            uint32_t slo[4], shs[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                if (S16) {
+                    const uint32_t st = static_cast<uint32_t>(runs[s]);
+                    const int f = run_first(st, m);
+                    slo[m] = static_cast<uint32_t>((f + m) * kSliceHalf);
+                    shs[m] = static_cast<uint32_t>(run_length(st, f) * kSliceHalf);
+                } else {
+                    slo[m] = static_cast<uint32_t>(m * kSliceHalf);
+                    shs[m] = kHalfTile;
+                }
+            }
 
             // ---- S^T = K Q^T: 4 m-tiles of 16 tokens
             float sc[4][4];
@@ -452,12 +493,11 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                 for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t hb = kb + (ks >> 2) * kHalfStride<S16>;
                 const int chunk = ((ks & 3) << 1) + (lane >> 4);
+                const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
                 for (int mt = 0; mt < 4; ++mt) {
-                    const int row = mt * (16 + kSliceSkip<S16>) + (lane & 7) +
-                                    (((lane >> 3) & 1) << 3);
+                    const uint32_t hb = kb + slo[mt] + (ks >> 2) * shs[mt];
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4(swz128(hb, row, chunk), a0, a1, a2, a3);
                     mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
@@ -517,11 +557,11 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
             // ---- O^T += V^T P^T: 8 m-tiles of 16 dims x 4 k-tiles of 16 tokens
 #pragma unroll
             for (int md = 0; md < 8; ++md) {
-                const uint32_t hb = vb + (md >> 2) * kHalfStride<S16>;
                 const int chunk = ((md & 3) << 1) + ((lane >> 3) & 1);
+                const int row = (lane & 7) + ((lane >> 4) << 3);
 #pragma unroll
                 for (int kt = 0; kt < 4; ++kt) {
-                    const int row = kt * (16 + kSliceSkip<S16>) + (lane & 7) + ((lane >> 4) << 3);
+                    const uint32_t hb = vb + slo[kt] + (md >> 2) * shs[kt];
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4_trans(swz128(hb, row, chunk), a0, a1, a2, a3);
                     mma_bf16_16816(acc[md], a0, a1, a2, a3, pb[kt][0], pb[kt][1]);
@@ -612,7 +652,7 @@ sparse_decode_kernel(const __grid_constant__ CUtensorMap k_map,
 size_t decode_smem_bytes(int units) {
     return 1024 /* alignment slack */ + static_cast<size_t>(STAGES) * kStageBytes +
            NC * kMaxGroup * (kPartialFloatsPerHead + 2) * sizeof(float) +
-           2 * STAGES * sizeof(uint64_t) + STAGES * sizeof(int) +
+           2 * STAGES * sizeof(uint64_t) + 2 * STAGES * sizeof(int) +
            (kThreads / 32 + 1 + 2) * sizeof(int) + static_cast<size_t>(units + 1) * sizeof(int);
 }
 
@@ -664,8 +704,8 @@ int decode_grid(int units) {
     return m.grid;
 }
 
-cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
-                                 const CUtensorMap& v_map, bool shared16, cudaStream_t s) {
+cudaError_t launch_sparse_decode(const DecodeParams& p, const DecodeMaps& maps, bool shared16,
+                                 cudaStream_t s) {
     const int U = p.batch * p.num_kv_heads;
     const size_t smem = decode_smem_bytes(U);
     int dev = 0;
@@ -679,9 +719,9 @@ cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map
     if (e != cudaSuccess) return e;
     if (shared16)
         return launch_pdl(sparse_decode_kernel<true>, dim3(p.num_ctas), dim3(kThreads), smem, s,
-                          k_map, v_map, p);
+                          maps, p);
     return launch_pdl(sparse_decode_kernel<false>, dim3(p.num_ctas), dim3(kThreads), smem, s,
-                      k_map, v_map, p);
+                      maps, p);
 }
 
 }  // namespace spot

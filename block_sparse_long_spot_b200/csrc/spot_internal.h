@@ -74,6 +74,13 @@ struct SelectParams {
     uint32_t* status;
 };
 
+// Tensor maps of the sparse-decode kernel (see make_decode_maps), passed by
+// value as one grid-constant kernel parameter.
+struct DecodeMaps {
+    CUtensorMap k[4];
+    CUtensorMap v[4];
+};
+
 struct DecodeParams {
     const uint16_t* q;
     const int32_t* page_table;
@@ -186,8 +193,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 cudaError_t launch_select(const SelectParams& p, int fmt, cudaStream_t s);
 // shared16: the token selector's layout (one selection per sequence shared
 // by its KV heads, blocks of kTokBlock tokens; maps with 16-row boxes).
-cudaError_t launch_sparse_decode(const DecodeParams& p, const CUtensorMap& k_map,
-                                 const CUtensorMap& v_map, bool shared16, cudaStream_t s);
+cudaError_t launch_sparse_decode(const DecodeParams& p, const DecodeMaps& maps, bool shared16,
+                                 cudaStream_t s);
 cudaError_t launch_tok_score(const TokScoreParams& p, const CUtensorMap& sel_map, cudaStream_t s);
 cudaError_t launch_tok_append(const TokAppendParams& p, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& k_map,
@@ -215,6 +222,12 @@ bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_row
 // box_rows consecutive rows in one copy, laid out [half][row][128 B] with
 // 128-byte swizzle.
 bool make_split_rows_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
+// The sparse-decode kernel's maps over the K and V pools (`rows` rows of 128
+// bf16 each): k[h - 1] / v[h - 1] are split-row maps with boxes of 16 h
+// rows.  Whole 64-token blocks use k[3] / v[3] only (the others are left
+// zero); 16-token slices (slices = true) use all four heights.
+bool make_decode_maps(DecodeMaps* m, const void* k_pool, const void* v_pool, int64_t rows,
+                      bool slices);
 // Tensor map over `lines` lines of 128 bytes, box 128 bytes x box_lines,
 // 128-byte swizzle.
 bool make_bytes_map(CUtensorMap* map, const void* base, int64_t lines, int box_lines);
