@@ -276,14 +276,13 @@ sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams
     }
     if (threadIdx.x == 0) unit_off[U] = total;
     __syncthreads();
-    if (blockIdx.x == 0) {
-        // (sequence, KV head) units with nothing selected: out = 0, lse = -inf
-        for (int t = threadIdx.x; t < U * G * (kHeadDim / 4); t += kThreads) {
-            const int u = t / (G * (kHeadDim / 4));
-            if (unit_off[u + 1] != unit_off[u]) continue;
-            const int r = t - u * G * (kHeadDim / 4);
-            const int n = r / (kHeadDim / 4), d4 = r - n * (kHeadDim / 4);
-            const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+    // (sequence, KV head) units with nothing selected: out = 0, lse = -inf.
+    // Unit u is checked by CTA u mod P only, so no CTA's start is held up.
+    for (int u = blockIdx.x; u < U; u += p.num_ctas) {
+        if (unit_off[u + 1] != unit_off[u]) continue;
+        const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+        for (int t = threadIdx.x; t < G * (kHeadDim / 4); t += kThreads) {
+            const int n = t / (kHeadDim / 4), d4 = t - n * (kHeadDim / 4);
             const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
             reinterpret_cast<float4*>(p.out + h * kHeadDim)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (p.lse && d4 == 0) p.lse[h] = -INFINITY;
@@ -423,26 +422,25 @@ sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams
     // ===================================================== consumer warps
     const int c4 = lane & 3;         // column pair: heads 2*c4, 2*c4+1
     const int r8 = lane >> 2;        // row within an 8-row group
+    // Q^T fragments of unit u (B operand, k = head dim, n = head): lane holds
+    // head r8, dims 16 ks + 2 c4 + {0,1} (b0) and + 8 (b1).
+    auto load_q = [&](int u, uint32_t (&qf)[8][2]) {
+        const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+        const bool real = r8 < G;
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+            p.q + (static_cast<int64_t>(b) * p.num_q_heads + g * G + (real ? r8 : 0)) * kHeadDim);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            qf[ks][0] = real ? __ldg(qrow + ks * 8 + c4) : 0u;
+            qf[ks][1] = real ? __ldg(qrow + ks * 8 + 4 + c4) : 0u;
+        }
+    };
     int pos = beg;
+    uint32_t qf[8][2];
+    load_q(find_unit(unit_off, U, pos), qf);
     while (pos < end) {
         const int u = find_unit(unit_off, U, pos);
         const int seg_end = min(end, unit_off[u + 1]);
-        const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
-
-        // Q^T fragments (B operand, k = head dim, n = head): lane holds
-        // head r8, dims 16 ks + 2 c4 + {0,1} (b0) and + 8 (b1).
-        uint32_t qf[8][2];
-        {
-            const bool real = r8 < G;
-            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-                p.q + (static_cast<int64_t>(b) * p.num_q_heads + g * G + (real ? r8 : 0)) *
-                          kHeadDim);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                qf[ks][0] = real ? __ldg(qrow + ks * 8 + c4) : 0u;
-                qf[ks][1] = real ? __ldg(qrow + ks * 8 + 4 + c4) : 0u;
-            }
-        }
         float m0 = -INFINITY, m1 = -INFINITY;     // running max (log2 domain)
         float l0 = 0.f, l1 = 0.f;                 // this lane's share of the sum
         float acc[8][4];
@@ -571,6 +569,11 @@ sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams
             if (lane == 0) mbar_arrive(&empty[s]);
         }
 
+        // the next unit's Q, in flight while this unit's partial is written
+        uint32_t qn[8][2];
+        const bool more = seg_end < end;
+        if (more) load_q(find_unit(unit_off, U, seg_end), qn);
+
         // ---- merge the NC warps' states for unit u inside the CTA, then
         // write the CTA's partial (one slot per CTA and unit)
 #pragma unroll
@@ -628,20 +631,25 @@ sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams
                 }
             }
         }
-        __threadfence();                 // the partial is visible GPU-wide ...
-        consumer_barrier();
-        if (warp == 0 && lane == 0) {    // ... before this CTA's arrival is counted
+        consumer_barrier();              // every store of the partial precedes ...
+        if (warp == 0 && lane == 0) {    // ... this CTA's arrival, a release at GPU
+            // scope; the last arrival's acquire makes the other partials visible
+            // to the whole CTA after the barrier below
             const unsigned seg_len = static_cast<unsigned>(seg_end - pos);
             const unsigned cnt_u = static_cast<unsigned>(unit_off[u + 1] - unit_off[u]);
-            const unsigned old = atomicAdd(&p.unit_done[u], seg_len);
+            const unsigned old = atomic_add_acq_rel_gpu(&p.unit_done[u], seg_len);
             const int last = (old + seg_len == cnt_u);
             if (last) p.unit_done[u] = 0u;          // every arrival is in: ready for the next call
             flags[1] = last;
         }
         consumer_barrier();
-        if (flags[1]) {
-            __threadfence();
-            merge_unit(p, u, unit_off[u], unit_off[u + 1], N, P, threadIdx.x);
+        if (flags[1]) merge_unit(p, u, unit_off[u], unit_off[u + 1], N, P, threadIdx.x);
+        if (more) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                qf[ks][0] = qn[ks][0];
+                qf[ks][1] = qn[ks][1];
+            }
         }
         pos = seg_end;
     }

@@ -87,6 +87,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// Atomic add at GPU scope with acquire-release semantics: the caller's
+// writes (and those it observed, e.g. through a CTA barrier) are visible to
+// whoever acquires this location after it, and it sees everything released
+// to this location before it.
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* a, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(a), "r"(v)
+                 : "memory");
+    return old;
+}
+
 // ---------------------------------------------------------------- TMA
 
 // 2-D tiled bulk tensor load global -> shared memory of this CTA, completion
