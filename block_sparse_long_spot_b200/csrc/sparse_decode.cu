@@ -106,6 +106,19 @@ __device__ __forceinline__ int owner_cta(int64_t N, int64_t P, int64_t pos) {
     return static_cast<int>(((pos + 1) * P - 1) / N);
 }
 
+// out / lse of head n of unit u from its merged state: the unnormalised sum
+// a (dims 4 d4 .. 4 d4 + 3), the log2-domain maximum M and the sum L.
+__device__ __forceinline__ void store_head(const DecodeParams& p, int u, int n, int d4, float4 a,
+                                           float M, float L) {
+    const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
+    const bool empty = !(L > 0.f);  // only if every tile was rejected as out of range
+    const float inv = empty ? 0.f : 1.f / L;
+    const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * p.group + n;
+    reinterpret_cast<float4*>(p.out + h * kHeadDim)[d4] =
+        make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+    if (p.lse && d4 == 0) p.lse[h] = empty ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+}
+
 // Merge the partials of unit u (blocks [lo, hi) of the flattened list) and
 // write out / lse of its G heads, with all NC consumer warps (tid < NC*32).
 // The partials are one per CTA whose range touched the unit; other CTAs of
@@ -123,7 +136,6 @@ __device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t
                            int tid) {
     constexpr int T = NC * 32;
     const int G = p.group;
-    const int b = u / p.num_kv_heads, g = u - b * p.num_kv_heads;
     const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
     const int nslots = i1 - i0 + 1;
     const int64_t stride = static_cast<int64_t>(G) * kPartialFloatsPerHead;
@@ -186,14 +198,7 @@ __device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t
     for (int r = 0; r < kMergeItems; ++r) {
         const int item = tid + r * T;
         const int n = item / (kHeadDim / 4), d4 = item - n * (kHeadDim / 4);
-        if (n >= G) continue;
-        const bool empty = !(L[r] > 0.f);  // only if every tile was rejected as out of range
-        const float inv = empty ? 0.f : 1.f / L[r];
-        const int64_t h = static_cast<int64_t>(b) * p.num_q_heads + g * G + n;
-        reinterpret_cast<float4*>(p.out + h * kHeadDim)[d4] =
-            make_float4(a[r].x * inv, a[r].y * inv, a[r].z * inv, a[r].w * inv);
-        if (p.lse && d4 == 0)
-            p.lse[h] = empty ? -INFINITY : (M[r] + log2f(L[r])) * 0.6931471805599453f;
+        if (n < G) store_head(p, u, n, d4, a[r], M[r], L[r]);
     }
 }
 
@@ -603,6 +608,10 @@ sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams
             }
         }
         consumer_barrier();
+        // A segment that is the whole unit is the unit's only contribution:
+        // its merged state is the result (the arithmetic of a one-partial
+        // merge), with no partial, arrival or merge.
+        const bool whole = pos == unit_off[u] && seg_end == unit_off[u + 1];
         {
             float* slot = p.partials + static_cast<int64_t>(blockIdx.x + u) *
                                            (static_cast<int64_t>(G) * kPartialFloatsPerHead);
@@ -624,6 +633,10 @@ sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams
                     a.z = fmaf(f, v.z, a.z);
                     a.w = fmaf(f, v.w, a.w);
                 }
+                if (whole) {
+                    store_head(p, u, n, lane, a, M, L);
+                    continue;
+                }
                 reinterpret_cast<float4*>(slot + n * kHeadDim)[lane] = a;
                 if (lane == 0) {
                     slot[G * kHeadDim + n] = M;
@@ -632,18 +645,20 @@ sparse_decode_kernel(const __grid_constant__ DecodeMaps maps, const DecodeParams
             }
         }
         consumer_barrier();              // every store of the partial precedes ...
-        if (warp == 0 && lane == 0) {    // ... this CTA's arrival, a release at GPU
-            // scope; the last arrival's acquire makes the other partials visible
-            // to the whole CTA after the barrier below
-            const unsigned seg_len = static_cast<unsigned>(seg_end - pos);
-            const unsigned cnt_u = static_cast<unsigned>(unit_off[u + 1] - unit_off[u]);
-            const unsigned old = atomic_add_acq_rel_gpu(&p.unit_done[u], seg_len);
-            const int last = (old + seg_len == cnt_u);
-            if (last) p.unit_done[u] = 0u;          // every arrival is in: ready for the next call
-            flags[1] = last;
+        if (!whole) {
+            if (warp == 0 && lane == 0) {    // ... this CTA's arrival, a release at GPU
+                // scope; the last arrival's acquire makes the other partials
+                // visible to the whole CTA after the barrier below
+                const unsigned seg_len = static_cast<unsigned>(seg_end - pos);
+                const unsigned cnt_u = static_cast<unsigned>(unit_off[u + 1] - unit_off[u]);
+                const unsigned old = atomic_add_acq_rel_gpu(&p.unit_done[u], seg_len);
+                const int last = (old + seg_len == cnt_u);
+                if (last) p.unit_done[u] = 0u;      // every arrival is in: ready for the next call
+                flags[1] = last;
+            }
+            consumer_barrier();
+            if (flags[1]) merge_unit(p, u, unit_off[u], unit_off[u + 1], N, P, threadIdx.x);
         }
-        consumer_barrier();
-        if (flags[1]) merge_unit(p, u, unit_off[u], unit_off[u + 1], N, P, threadIdx.x);
         if (more) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
