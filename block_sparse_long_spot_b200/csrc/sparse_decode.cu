@@ -129,12 +129,14 @@ __device__ __forceinline__ void store_head(const DecodeParams& p, int u, int n, 
 // (m, l, acc) of all of them for a whole batch of slots before using any,
 // folding batches with a running maximum (the usual log-sum-exp merge).
 // Slots are folded in CTA order, so the result does not depend on timing.
-constexpr int kMergeBatch = 8;           // slots per batch
-constexpr int kMergeItems = (kMaxGroup * (kHeadDim / 4) + NC * 32 - 1) / (NC * 32);
-
-__device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t N, int64_t P,
-                           int tid) {
+// ITEMS x BATCH loads of each kind are in flight per thread: G <= 4 heads
+// need one item per thread, which leaves room for batches of 16 slots.
+template <int ITEMS, int BATCH>
+__device__ void merge_unit_t(const DecodeParams& p, int u, int lo, int hi, int64_t N, int64_t P,
+                             int tid) {
     constexpr int T = NC * 32;
+    constexpr int kMergeItems = ITEMS;
+    constexpr int kMergeBatch = BATCH;
     const int G = p.group;
     const int i0 = owner_cta(N, P, lo), i1 = owner_cta(N, P, hi - 1);
     const int nslots = i1 - i0 + 1;
@@ -200,6 +202,17 @@ __device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t
         const int n = item / (kHeadDim / 4), d4 = item - n * (kHeadDim / 4);
         if (n < G) store_head(p, u, n, d4, a[r], M[r], L[r]);
     }
+}
+
+constexpr int kMergeLoads = 16;          // slots x items of loads in flight per thread
+static_assert(kMaxGroup * (kHeadDim / 4) <= 2 * NC * 32, "two items per thread cover G <= 8");
+
+__device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t N, int64_t P,
+                           int tid) {
+    if (p.group * (kHeadDim / 4) <= NC * 32)
+        merge_unit_t<1, kMergeLoads>(p, u, lo, hi, N, P, tid);
+    else
+        merge_unit_t<2, kMergeLoads / 2>(p, u, lo, hi, N, P, tid);
 }
 
 // Valid tokens of the four 16-row slices of a 64-row tile, one byte each.
