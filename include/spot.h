@@ -24,7 +24,7 @@
  *     status word inside the workspace and read with
  *     spot_read_device_status().  Kernels never trap: a bad index is
  *     recorded and the access is skipped.
- *   - Shapes this build supports: head_dim 128, block_size 64 (one KV page
+ *   - Shapes the library supports: head_dim 128, block_size 64 (one KV page
  *     per block), sel_dim 64, 1 <= num_q_heads / num_kv_heads <= 8,
  *     batch * num_kv_heads <= 4096, max_blocks <= 8192 (512K tokens).  Other shapes
  *     return SPOT_ERR_UNSUPPORTED.
@@ -73,7 +73,7 @@ extern "C" {
 typedef enum {
     SPOT_OK = 0,
     SPOT_ERR_INVALID_ARG = 1,     /* null / misaligned pointer, bad size or parameter */
-    SPOT_ERR_UNSUPPORTED = 2,     /* shape outside what this build implements */
+    SPOT_ERR_UNSUPPORTED = 2,     /* shape outside what the library implements */
     SPOT_ERR_WORKSPACE = 3,       /* workspace smaller than spot_workspace_size() */
     SPOT_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
     SPOT_ERR_DEVICE_BOUNDS = 5,   /* a kernel met an out-of-range page id / block index */
@@ -127,7 +127,7 @@ typedef struct {
  * arrival counters of the decode kernel that must start at zero; every call
  * that completes leaves those counters at zero again.  After
  * a call whose status reads SPOT_ERR_DEVICE_TIMEOUT, zero the whole workspace
- * before its next use.  Returns 0 for a shape this build does not support. */
+ * before its next use.  Returns 0 for a shape the library does not support. */
 size_t spot_workspace_size(const spot_layer_desc_t* desc, int32_t batch, int32_t max_blocks);
 
 /* Append (write, quantising if the format asks) one selector key per
