@@ -130,7 +130,7 @@ __device__ __forceinline__ void store_head(const DecodeParams& p, int u, int n, 
 // folding batches with a running maximum (the usual log-sum-exp merge).
 // Slots are folded in CTA order, so the result does not depend on timing.
 // ITEMS x BATCH loads of each kind are in flight per thread: G <= 4 heads
-// need one item per thread, which leaves room for batches of 16 slots.
+// need one item per thread, which leaves registers for larger batches.
 template <int ITEMS, int BATCH>
 __device__ void merge_unit_t(const DecodeParams& p, int u, int lo, int hi, int64_t N, int64_t P,
                              int tid) {
@@ -204,15 +204,16 @@ __device__ void merge_unit_t(const DecodeParams& p, int u, int lo, int hi, int64
     }
 }
 
-constexpr int kMergeLoads = 16;          // slots x items of loads in flight per thread
 static_assert(kMaxGroup * (kHeadDim / 4) <= 2 * NC * 32, "two items per thread cover G <= 8");
 
+// Up to 24 slots per round trip with one item per thread (G <= 4: the token
+// selector's units have about 19 partials each), 8 with two.
 __device__ void merge_unit(const DecodeParams& p, int u, int lo, int hi, int64_t N, int64_t P,
                            int tid) {
     if (p.group * (kHeadDim / 4) <= NC * 32)
-        merge_unit_t<1, kMergeLoads>(p, u, lo, hi, N, P, tid);
+        merge_unit_t<1, 24>(p, u, lo, hi, N, P, tid);
     else
-        merge_unit_t<2, kMergeLoads / 2>(p, u, lo, hi, N, P, tid);
+        merge_unit_t<2, 8>(p, u, lo, hi, N, P, tid);
 }
 
 // Valid tokens of the four 16-row slices of a 64-row tile, one byte each.
