@@ -46,12 +46,12 @@ HBM_FALLBACK_GBS = 6650.0
 # source files are unchanged (sha256 prefix over them); otherwise the
 # roofline's traffic is null.
 NCU_TRAFFIC = {
-    "qwen3_32b_128k": {"bytes": 735314304 + 1009536, "sel_fmt": "bf16",
+    "qwen3_32b_128k": {"bytes": 735307072 + 1026368, "sel_fmt": "bf16",
                        "files": ["sparse_decode.cu"],
-                       "sha256": "37ca48560f47874f"},
-    "qwen3_8b_128k_tok": {"bytes": 307646592 + 933952, "sel_fmt": "bf16",
+                       "sha256": "b0c2289e0c531333"},
+    "qwen3_8b_128k_tok": {"bytes": 307664896 + 965504, "sel_fmt": "bf16",
                           "files": ["sparse_decode.cu"],
-                          "sha256": "37ca48560f47874f"},
+                          "sha256": "b0c2289e0c531333"},
     "qwen3_8b_prefill_32k": {"bytes": 411903488 + 499184128, "sel_fmt": "bf16",
                              "files": ["prefill.cu", "tc.cuh"],
                              "sha256": "716d0750e6195d2d"},
