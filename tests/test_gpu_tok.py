@@ -94,6 +94,30 @@ def test_tok_ragged_partial_blocks_and_empty_sequences():
     assert np.all(np.isneginf(gpu["lse"][0]))
 
 
+@pytest.mark.parametrize("dense", [True, False])
+def test_tok_runs_of_slices_stop_at_page_blocks(dense):
+    """One KV head and a contiguous page table put consecutive pages next to
+    each other in the pool, so the 16-token slices of a run could run on into
+    the next page: the attention must still match the oracle, with every
+    block reserved (runs of four slices) and with the nucleus selection."""
+    wl = workloads.make_tok("tok_tiny_2k", seed=9, device=DEV, batch=2, num_q_heads=8,
+                            num_kv_heads=1, page_order="contiguous")
+    kw = dict(sink=300, rec=0) if dense else {}
+    gpu = run_gpu_tok(wl, **kw)
+    assert gpu["status"] == 0
+    args = tok_oracle_args(wl)
+    ora = run_oracle_tok(wl, args=args, **kw)
+    if dense:
+        _same(gpu, ora, wl)
+        n_diff = 0
+    else:
+        scores = oracle_tok_scores(wl, args=args)
+        n_diff = check_tok_selection_near_cut(gpu, ora, scores, wl)
+        assert n_diff <= 1
+    _, n = check_tok_outputs(gpu, ora, wl)
+    assert n >= wl.batch - n_diff
+
+
 @pytest.mark.parametrize("batch,seq_len", [(1, 131072), (2, None)])
 def test_tok_full_size(batch, seq_len):
     """Qwen3-8B layer at 128K (and two ragged sequences): the selection of
