@@ -48,10 +48,10 @@ HBM_FALLBACK_GBS = 6650.0
 NCU_TRAFFIC = {
     "qwen3_32b_128k": {"bytes": 735307072 + 1026368, "sel_fmt": "bf16",
                        "files": ["sparse_decode.cu"],
-                       "sha256": "b0c2289e0c531333"},
+                       "sha256": "e463ade2fe28a806"},
     "qwen3_8b_128k_tok": {"bytes": 307664896 + 965504, "sel_fmt": "bf16",
                           "files": ["sparse_decode.cu"],
-                          "sha256": "b0c2289e0c531333"},
+                          "sha256": "e463ade2fe28a806"},
     "qwen3_8b_prefill_32k": {"bytes": 411903488 + 499184128, "sel_fmt": "bf16",
                              "files": ["prefill.cu", "tc.cuh"],
                              "sha256": "716d0750e6195d2d"},

@@ -12,10 +12,12 @@
 // arrival counter in the workspace reaches the unit's block count) merges the
 // unit's partials with their log-sum-exp weights and writes the output; the
 // counter is reset to zero by that CTA, so it is zero again for the next call.
+// A CTA whose range holds a whole unit writes that unit's output itself, with
+// no partial and no arrival.
 //
 // Inside a CTA one producer warp issues TMA tile loads of the gathered pages
 // (one 3-D box each for K and V: both 128-byte halves of the block's 64 rows,
-// 128-byte swizzled; fewer, larger boxes keep more bytes in flight) into a ring
+// 128-byte swizzled; fewer, larger copies per stage stream faster) into a ring
 // of stages guarded by mbarriers; NC consumer warps each take every NC-th
 // tile and keep their own online-softmax state for the G <= 8 query heads of
 // the unit's KV head:
